@@ -1,0 +1,248 @@
+/*
+ * oracle.c -- slow, plain fp64 CPU restatement of the fused row-normalisation ops.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may include, link or call
+ * this file.  Only the tests, the smoke check and the benchmark's CPU-baseline leg
+ * use it.  It shares no code, header, table or constant with the CUDA library
+ * (rope_add_rms_b200/csrc); the only thing both sides share is the seeded input
+ * generator, which holds none of the arithmetic below.
+ *
+ * Sources (docs.rs nuvec-core 0.5.0, "Enum FastOp", Variants section; docs.rs
+ * nuvec-nn 0.4.0 src/layers.rs, RmsNorm / LayerNorm / Rope; miniVLLM docs "Layers",
+ * LayerNorm section):
+ *   RmsNorm     (x, w): x / sqrt(mean(x^2) + eps) * w over the last axis,
+ *               w is 1-D or the scalar 1.
+ *   AddRmsNorm  (x, r, w): h = x + r, then RmsNorm of h; the updated residual h is
+ *               returned next to the normalised row (miniVLLM LayerNorm.forward,
+ *               steps 1-3: x_new = x + residual, normalise x_new, return both).
+ *   LayerNorm   (x, w, b): (x - mean) / sqrt(var + eps) * w + b over the last axis,
+ *               w and b are 1-D or the scalars 1 and 0.
+ *   Rope        rotary embedding of the first dims features (dims even), as the two
+ *               halves or as interleaved pairs ("traditional"); base and a position
+ *               scale; forward = false is the inverse rotation.
+ *   NormRope    each [b, h, l] row RMS-normalised (when eps is given) and then
+ *               rotated as Rope at position offset + l.
+ *
+ * Readings taken where the pages leave a step open (each one is listed with its
+ * reason in the design notes):
+ *   - eps, base and scale are fp32 values (FastOp stores them as f32::to_bits);
+ *     they enter here widened exactly to fp64.
+ *   - AddRmsNorm normalises the h that is returned, i.e. h after rounding to the
+ *     I/O type; h itself is the fp32 sum x + r rounded once to the I/O type.
+ *   - var is the population variance (divide by D).
+ *   - Rope frequencies: theta_i = base^(-2 i / dims), angle (offset + l) * scale *
+ *     theta_i, rotation [[cos, -sin], [sin, cos]] on the pair (p, q); halves pair
+ *     (i, i + dims/2), traditional pairs (2i, 2i + 1); features j >= dims pass
+ *     through unrotated.
+ *   - In NormRope the row is normalised (times w) over all D features first and
+ *     then rotated; normalize = 0 is plain Rope (no w).
+ *
+ * Arithmetic: every input element is widened exactly to double; sums are plain
+ * left-to-right loops in double; sqrt, pow, sin and cos are the host libm's double
+ * routines.  Build with -O2 -ffp-contract=off and without fast-math.
+ * All row functions work on a row range [r0, r1) so that a caller can spread
+ * rows over threads; they allocate a scratch row with malloc and return 0, or -1
+ * when that allocation fails.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* element types of the oracle's own: 0 = IEEE binary32, 1 = bfloat16 (raw bits) */
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+
+/* ---- widening and rounding -------------------------------------------------- */
+
+static float f32_from_bits(uint32_t u) {
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static uint32_t bits_from_f32(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return u;
+}
+
+/* A bfloat16 is the upper half of a binary32: widening is exact. */
+static double widen(const void* base, int dt, int64_t i) {
+    if (dt == ORACLE_F32) return (double)((const float*)base)[i];
+    uint16_t b = ((const uint16_t*)base)[i];
+    return (double)f32_from_bits((uint32_t)b << 16);
+}
+
+/*
+ * Round a double to the nearest bfloat16, ties to even, in ONE rounding (no detour
+ * through binary32).  bfloat16 has 8 significant bits, exponents -126..127 and
+ * subnormals spaced 2^-133.  The value is scaled by the quantum of its binade so
+ * that the rounding is rint() of a double in [128, 256), which is exact.
+ */
+uint16_t oracle_bf16_from_f64(double v) {
+    if (isnan(v)) return signbit(v) ? 0xFFC0u : 0x7FC0u;
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    if (isinf(a)) return sign | 0x7F80u;
+    if (a == 0.0) return sign;
+    int e;
+    (void)frexp(a, &e);            /* a = f * 2^e, f in [0.5, 1) */
+    int qexp = (e < -125 ? -125 : e) - 8;
+    double n = rint(ldexp(a, -qexp));   /* default rounding mode: nearest, ties even */
+    double r = ldexp(n, qexp);          /* exact: n has at most 9 bits */
+    if (r > 3.3895313892515355e38) return sign | 0x7F80u;   /* beyond max finite */
+    /* r is a bfloat16 value, hence exactly a binary32 whose low 16 bits are zero */
+    return sign | (uint16_t)(bits_from_f32((float)r) >> 16);
+}
+
+void oracle_round_bf16(const double* v, uint16_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_from_f64(v[i]);
+}
+
+static void store_io(void* base, int dt, int64_t i, float v) {
+    if (dt == ORACLE_F32)
+        ((float*)base)[i] = v;
+    else
+        ((uint16_t*)base)[i] = oracle_bf16_from_f64((double)v);
+}
+
+/* ---- one-row definitions ------------------------------------------------------ */
+
+/* RmsNorm of one row held in double: y_j = x_j / sqrt(mean(x^2) + eps) * w_j. */
+static void rms_row(const double* x, const void* w, int dt, int64_t D, double eps, double* y) {
+    double sumsq = 0.0;
+    for (int64_t j = 0; j < D; ++j) sumsq += x[j] * x[j];
+    double denom = sqrt(sumsq / (double)D + eps);
+    for (int64_t j = 0; j < D; ++j) {
+        double wj = w ? widen(w, dt, j) : 1.0;
+        y[j] = x[j] / denom * wj;
+    }
+}
+
+/* LayerNorm of one row: y_j = (x_j - mean) / sqrt(var + eps) * w_j + b_j. */
+static void layer_row(const double* x, const void* w, const void* b, int dt, int64_t D,
+                      double eps, double* y) {
+    double sum = 0.0;
+    for (int64_t j = 0; j < D; ++j) sum += x[j];
+    double mean = sum / (double)D;
+    double sqdev = 0.0;
+    for (int64_t j = 0; j < D; ++j) sqdev += (x[j] - mean) * (x[j] - mean);
+    double var = sqdev / (double)D;
+    double denom = sqrt(var + eps);
+    for (int64_t j = 0; j < D; ++j) {
+        double wj = w ? widen(w, dt, j) : 1.0;
+        double bj = b ? widen(b, dt, j) : 0.0;
+        y[j] = (x[j] - mean) / denom * wj + bj;
+    }
+}
+
+/*
+ * Rope of one row at position pos: pair i (0 <= i < dims/2) turns by
+ * phi_i = pos * scale * base^(-2 i / dims); forward = 0 turns by -phi_i.
+ * Features from dims on are copied unchanged.
+ */
+static void rope_row(const double* x, int64_t D, int64_t dims, int traditional, double base,
+                     double scale, double pos, int forward, double* y) {
+    int64_t half = dims / 2;
+    for (int64_t j = 0; j < D; ++j) y[j] = x[j];
+    for (int64_t i = 0; i < half; ++i) {
+        double theta = pow(base, -2.0 * (double)i / (double)dims);
+        double phi = pos * scale * theta;
+        if (!forward) phi = -phi;
+        int64_t p = traditional ? 2 * i : i;
+        int64_t q = traditional ? 2 * i + 1 : i + half;
+        double c = cos(phi), s = sin(phi);
+        y[p] = x[p] * c - x[q] * s;
+        y[q] = x[p] * s + x[q] * c;
+    }
+}
+
+static void load_row(const void* src, int dt, int64_t row, int64_t D, double* dst) {
+    for (int64_t j = 0; j < D; ++j) dst[j] = widen(src, dt, row * D + j);
+}
+
+/* ---- exported ops: rows [r0, r1) of [rows, D] row-major arrays -------------- */
+
+int oracle_rms_norm(const void* x, const void* w, double* y, int64_t r0, int64_t r1, int64_t D,
+                    float eps, int dt) {
+    double* row = (double*)malloc((size_t)D * sizeof(double));
+    if (!row) return -1;
+    for (int64_t k = r0; k < r1; ++k) {
+        load_row(x, dt, k, D, row);
+        rms_row(row, w, dt, D, (double)eps, y + k * D);
+    }
+    free(row);
+    return 0;
+}
+
+/* h = x + r added in binary32 and rounded once to the I/O type; y = RmsNorm(h). */
+int oracle_add_rms_norm(const void* x, const void* r, const void* w, double* y, void* h,
+                        int64_t r0, int64_t r1, int64_t D, float eps, int dt) {
+    double* row = (double*)malloc((size_t)D * sizeof(double));
+    if (!row) return -1;
+    for (int64_t k = r0; k < r1; ++k) {
+        for (int64_t j = 0; j < D; ++j) {
+            int64_t i = k * D + j;
+            float sum = (float)widen(x, dt, i) + (float)widen(r, dt, i);
+            store_io(h, dt, i, sum);
+            row[j] = widen(h, dt, i);    /* the rounded h, as returned */
+        }
+        rms_row(row, w, dt, D, (double)eps, y + k * D);
+    }
+    free(row);
+    return 0;
+}
+
+int oracle_layer_norm(const void* x, const void* w, const void* b, double* y, int64_t r0,
+                      int64_t r1, int64_t D, float eps, int dt) {
+    double* row = (double*)malloc((size_t)D * sizeof(double));
+    if (!row) return -1;
+    for (int64_t k = r0; k < r1; ++k) {
+        load_row(x, dt, k, D, row);
+        layer_row(row, w, b, dt, D, (double)eps, y + k * D);
+    }
+    free(row);
+    return 0;
+}
+
+/* Rope on rows already in double (rows of [.., L, D], row k at l = k mod L). */
+int oracle_rope_f64(const double* x, double* y, int64_t r0, int64_t r1, int64_t L, int64_t D,
+                    int64_t dims, int traditional, float base, float scale, int64_t offset,
+                    int forward) {
+    for (int64_t k = r0; k < r1; ++k) {
+        double pos = (double)offset + (double)(k % L);
+        rope_row(x + k * D, D, dims, traditional, (double)base, (double)scale, pos, forward,
+                 y + k * D);
+    }
+    return 0;
+}
+
+/*
+ * NormRope on rows of x [B, H, L, D] flattened to [rows, D]: row k sits at
+ * l = k mod L and position offset + l.  normalize != 0: RmsNorm(x, w, eps) over all
+ * D features, then Rope.  normalize == 0: Rope of x alone (w unused).
+ */
+int oracle_norm_rope(const void* x, const void* w, double* y, int64_t r0, int64_t r1, int64_t L,
+                     int64_t D, int64_t dims, int traditional, float base, float scale,
+                     int64_t offset, int normalize, float eps, int dt) {
+    double* row = (double*)malloc((size_t)D * sizeof(double));
+    double* nrm = (double*)malloc((size_t)D * sizeof(double));
+    if (!row || !nrm) {
+        free(row);
+        free(nrm);
+        return -1;
+    }
+    for (int64_t k = r0; k < r1; ++k) {
+        load_row(x, dt, k, D, row);
+        if (normalize)
+            rms_row(row, w, dt, D, (double)eps, nrm);
+        else
+            memcpy(nrm, row, (size_t)D * sizeof(double));
+        double pos = (double)offset + (double)(k % L);
+        rope_row(nrm, D, dims, traditional, (double)base, (double)scale, pos, 1, y + k * D);
+    }
+    free(row);
+    free(nrm);
+    return 0;
+}

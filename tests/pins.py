@@ -1,0 +1,387 @@
+"""Pins of the CPU oracle: checks against what the pages and the mathematics fix.
+
+Each ``check_*`` takes an ``oracle.Oracle`` and raises AssertionError when the oracle
+disagrees with a closed form, an invariant, an independent library routine, a brute
+force enumeration or a hand-worked case.  ``tests/test_oracle_pins.py`` runs them on
+the real oracle; ``tests/test_oracle_mutants.py`` runs them on copies of the oracle
+with a planted mistake and requires every mistake to be caught.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def bf16_bits(values) -> np.ndarray:
+    """bfloat16 bit patterns of values (rounded by torch, to nearest even)."""
+    t = torch.as_tensor(np.asarray(values, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def widen_bf16(bits) -> np.ndarray:
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(
+        np.float64)
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _randn_bf16(shape, seed, scale=1.0):
+    return bf16_bits(_rng(seed).standard_normal(shape) * scale)
+
+
+def _close(a, b, rtol, atol=0.0, what=""):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    err = np.abs(a - b)
+    lim = atol + rtol * np.abs(b)
+    bad = err > lim
+    assert not bad.any(), f"{what}: {int(bad.sum())} mismatches, worst {float(err.max()):.3e}"
+
+
+# ---- rounding -----------------------------------------------------------------------
+
+def check_round_bf16_vs_torch(o):
+    """binary32 -> bfloat16 must equal torch's conversion (round to nearest even)."""
+    rng = _rng(1)
+    v = np.concatenate([
+        rng.standard_normal(20000),
+        rng.standard_normal(5000) * 1e30, rng.standard_normal(5000) * 1e-30,
+        rng.standard_normal(5000) * 1e-39,            # binary32 subnormals
+        [0.0, -0.0, 1.0, -1.0, 3.3895313892515355e38, 3.4e38, -3.4e38, np.inf, -np.inf],
+    ]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = o.round_bf16(v.astype(np.float64))
+    bad = got != ref
+    assert not bad.any(), f"round_bf16 differs from torch at {v[bad][:5]}"
+    assert (o.round_bf16(np.array([np.nan])) & 0x7FFF)[0] > 0x7F80, "NaN must stay NaN"
+
+
+def _all_finite_bf16():
+    bits = np.arange(0, 0x7F80, dtype=np.uint32)           # +0 .. max finite
+    vals = (bits << 16).view(np.float32).astype(np.float64)
+    return vals, bits.astype(np.uint16)
+
+
+def check_round_bf16_bruteforce(o):
+    """float64 -> bfloat16 in one rounding: nearest of all bfloat16 values, ties even."""
+    vals, bits = _all_finite_bf16()
+    rng = _rng(2)
+    k = rng.integers(1, len(vals) - 1, 20000)
+    lo, hi = vals[k - 1], vals[k]
+    mid = lo + (hi - lo) / 2                                # exact ties
+    off = (hi - lo) * rng.uniform(-0.49, 0.49, k.shape)      # off the tie
+    near = mid + off
+    tiny_above = np.nextafter(mid, np.inf)
+    tiny_below = np.nextafter(mid, -np.inf)
+    for v in (mid, near, tiny_above, tiny_below):
+        got = o.round_bf16(v)
+        j = np.searchsorted(vals, v)                        # vals[j-1] < v <= vals[j]
+        a, b = vals[j - 1], vals[j]
+        da, db = v - a, b - v
+        want = np.where(da < db, bits[j - 1], np.where(db < da, bits[j],
+                        np.where(bits[j - 1] % 2 == 0, bits[j - 1], bits[j])))
+        assert (got == want).all(), "round_bf16 is not nearest-even"
+        assert (o.round_bf16(-v) == (want | 0x8000)).all(), "round_bf16 sign handling"
+
+
+# ---- add_rms_norm: h ------------------------------------------------------------------
+
+def check_h_exact(o):
+    """h = binary32(x) + binary32(r), rounded once to the I/O type (bit exact)."""
+    x = _randn_bf16((37, 96), 3)
+    r = _randn_bf16((37, 96), 4, scale=3.0)
+    _, h = o.add_rms_norm(x, r, None, 1e-5)
+    s = (widen_bf16(x).astype(np.float32) + widen_bf16(r).astype(np.float32))
+    want = torch.from_numpy(s).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert (h == want).all(), "bf16 h is not RNE(x + r)"
+    xf = _rng(5).standard_normal((9, 33)).astype(np.float32)
+    rf = _rng(6).standard_normal((9, 33)).astype(np.float32)
+    _, hf = o.add_rms_norm(xf, rf, None, 1e-5)
+    assert (hf == xf + rf).all(), "f32 h is not x + r"
+
+
+def check_add_rms_is_rms_of_h(o):
+    """AddRmsNorm is RmsNorm of the returned (rounded) h."""
+    x = _randn_bf16((21, 64), 7)
+    r = _randn_bf16((21, 64), 8)
+    w = bf16_bits(_rng(9).uniform(0.5, 1.5, 64))
+    y, h = o.add_rms_norm(x, r, w, 1e-5)
+    _close(y, o.rms_norm(h, w, 1e-5), 1e-15, what="add_rms_norm vs rms_norm(h)")
+
+
+# ---- rms_norm -------------------------------------------------------------------------
+
+def check_rms_constant_rows(o):
+    """A constant row c gives c*w/sqrt(c^2 + eps); a +-1 row gives +-w/sqrt(1 + eps)."""
+    D = 48
+    w = bf16_bits(_rng(10).uniform(0.5, 1.5, D))
+    wv = widen_bf16(w)
+    cs = widen_bf16(bf16_bits([0.75, -3.0, 1e-3, 250.0]))
+    x = bf16_bits(np.repeat(cs[:, None], D, axis=1))
+    eps = np.float32(1e-5)
+    y = o.rms_norm(x, w, float(eps))
+    want = cs[:, None] * wv[None, :] / np.sqrt(cs[:, None] ** 2 + float(eps))
+    _close(y, want, 1e-14, what="constant rows")
+    sgn = np.where(_rng(11).random((5, D)) < 0.5, -1.0, 1.0)
+    y2 = o.rms_norm(bf16_bits(sgn), w, float(eps))
+    _close(y2, sgn * wv / math.sqrt(1 + float(eps)), 1e-14, what="+-1 rows")
+
+
+def check_rms_mean_square_invariant(o):
+    """With w = 1 the output has mean square ms / (ms + eps)."""
+    x = _randn_bf16((40, 128), 12, scale=0.05)
+    eps = float(np.float32(1e-3))
+    y = o.rms_norm(x, None, eps)
+    ms = (widen_bf16(x) ** 2).mean(axis=1)
+    _close((y ** 2).mean(axis=1), ms / (ms + eps), 1e-12, what="mean square")
+
+
+def check_rms_scaling(o):
+    """rms(c x, eps) == rms(x, eps / c^2) for c a power of two (exact rescaling)."""
+    x = _randn_bf16((16, 80), 13)
+    w = bf16_bits(_rng(14).uniform(0.5, 1.5, 80))
+    for c in (8.0, 2.0 ** -5):
+        xs = bf16_bits(widen_bf16(x) * c)
+        eps = float(np.float32(1e-4))
+        _close(o.rms_norm(xs, w, eps), o.rms_norm(x, w, float(np.float32(eps / c ** 2))),
+               1e-14, what=f"scaling c={c}")
+        _close(o.rms_norm(xs, w, 0.0), o.rms_norm(x, w, 0.0), 1e-14, what="scale invariance")
+
+
+def check_rms_vs_torch(o):
+    """Agreement with torch.nn.functional.rms_norm in float64 on the CPU."""
+    for dt in ("bf16", "f32"):
+        raw = _rng(15).standard_normal((33, 200)) * 2
+        wr = _rng(16).uniform(0.5, 1.5, 200)
+        if dt == "bf16":
+            x, w = bf16_bits(raw), bf16_bits(wr)
+            xv, wv = widen_bf16(x), widen_bf16(w)
+        else:
+            x, w = raw.astype(np.float32), wr.astype(np.float32)
+            xv, wv = x.astype(np.float64), w.astype(np.float64)
+        eps = float(np.float32(1e-6))
+        ref = F.rms_norm(torch.from_numpy(xv), (200,), torch.from_numpy(wv), eps).numpy()
+        _close(o.rms_norm(x, w, eps), ref, 1e-12, what=f"rms_norm vs torch ({dt})")
+
+
+# ---- layer_norm -----------------------------------------------------------------------
+
+def check_layer_norm_moments(o):
+    """With w = 1, b = 0: zero mean and variance var / (var + eps)."""
+    x = bf16_bits(_rng(17).standard_normal((30, 256)) * 2 + 0.5)
+    eps = float(np.float32(1e-2))
+    y = o.layer_norm(x, None, None, eps)
+    xv = widen_bf16(x)
+    var = xv.var(axis=1)
+    assert (np.abs(y.mean(axis=1)) <= 1e-12 * np.abs(y).max(axis=1)).all(), "mean(y) != 0"
+    _close(y.var(axis=1), var / (var + eps), 1e-10, what="var(y)")
+
+
+def check_layer_norm_translation(o):
+    """LayerNorm ignores a constant shift of the row (shift exact in binary32)."""
+    x = _rng(18).integers(-100, 100, (12, 64)).astype(np.float32)
+    w = _rng(19).uniform(0.5, 1.5, 64).astype(np.float32)
+    b = _rng(20).uniform(-1, 1, 64).astype(np.float32)
+    eps = float(np.float32(1e-5))
+    _close(o.layer_norm(x + np.float32(1024), w, b, eps), o.layer_norm(x, w, b, eps), 1e-13,
+           atol=1e-13, what="translation")
+
+
+def check_layer_norm_zero_weight(o):
+    """w = 0 gives y = b exactly."""
+    x = _randn_bf16((6, 40), 21)
+    b = bf16_bits(_rng(22).standard_normal(40) * 0.1)
+    y = o.layer_norm(x, bf16_bits(np.zeros(40)), b, 1e-5)
+    assert (y == widen_bf16(b)[None, :]).all(), "w = 0 must give b"
+
+
+def check_layer_norm_vs_torch(o):
+    """Agreement with torch.nn.functional.layer_norm in float64 on the CPU."""
+    x = bf16_bits(_rng(23).standard_normal((25, 300)) * 2 + 0.5)
+    w = bf16_bits(_rng(24).uniform(0.5, 1.5, 300))
+    b = bf16_bits(_rng(25).standard_normal(300) * 0.1)
+    eps = float(np.float32(1e-5))
+    ref = F.layer_norm(torch.from_numpy(widen_bf16(x)), (300,), torch.from_numpy(widen_bf16(w)),
+                       torch.from_numpy(widen_bf16(b)), eps).numpy()
+    _close(o.layer_norm(x, w, b, eps), ref, 1e-12, atol=1e-13, what="layer_norm vs torch")
+
+
+# ---- rope -------------------------------------------------------------------------------
+
+def _pairs(D, dims, trad):
+    half = dims // 2
+    return [(2 * i, 2 * i + 1) if trad else (i, i + half) for i in range(half)]
+
+
+def check_rope_norm_and_passthrough(o):
+    """Each pair keeps its norm; features past dims are unchanged."""
+    x = _rng(26).standard_normal((3 * 7, 40))
+    for trad in (0, 1):
+        y = o.rope_f64(x, 7, 24, trad, 10000.0, 1.0, 11)
+        for p, q in _pairs(40, 24, trad):
+            _close(y[:, p] ** 2 + y[:, q] ** 2, x[:, p] ** 2 + x[:, q] ** 2, 1e-12,
+                   what="pair norm")
+        assert (y[:, 24:] == x[:, 24:]).all(), "features past dims must pass through"
+
+
+def check_rope_inverse(o):
+    """forward = false undoes forward = true."""
+    x = _rng(27).standard_normal((2 * 9, 32))
+    for trad in (0, 1):
+        y = o.rope_f64(x, 9, 32, trad, 500.0, 0.75, 4096, forward=True)
+        _close(o.rope_f64(y, 9, 32, trad, 500.0, 0.75, 4096, forward=False), x, 1e-11,
+               atol=1e-12, what="inverse")
+
+
+def check_rope_position_zero(o):
+    """Position 0 is the identity."""
+    x = _rng(28).standard_normal((5, 16))
+    for trad in (0, 1):
+        assert (o.rope_f64(x, 1, 16, trad, 10000.0, 1.0, 0) == x).all(), "pos 0 must be identity"
+
+
+def check_rope_shift(o):
+    """(offset = o, l) is the same position as (offset = 0, l + o)."""
+    x = _rng(29).standard_normal((8, 16))
+    a = o.rope_f64(x, 8, 16, 0, 10000.0, 1.0, 5)
+    padded = np.concatenate([np.zeros((5, 16)), x])
+    b = o.rope_f64(padded, 13, 16, 0, 10000.0, 1.0, 0)[5:]
+    _close(a, b, 1e-15, what="offset shift")
+    # row k of a [B, H, L, D] batch is at l = k mod L
+    stacked = np.concatenate([x, x])
+    c = o.rope_f64(stacked, 8, 16, 0, 10000.0, 1.0, 5)
+    _close(c[8:], a, 1e-15, what="l = k mod L")
+
+
+def check_rope_pair_angles(o):
+    """Pair i turns by pos * scale * base^(-2i/dims): theta_0 = 1, counter-clockwise."""
+    base, scale, pos = 100.0, 0.25, 3
+    for (dims, D), trad in [((16, 16), 0), ((16, 16), 1), ((8, 20), 0), ((8, 20), 1)]:
+        rows = []
+        for p, q in _pairs(D, dims, trad):
+            e = np.zeros(D)
+            e[p] = 1.0
+            rows.append(e)
+        y = o.rope_f64(np.array(rows), 1, dims, trad, base, scale, pos)
+        for i, (p, q) in enumerate(_pairs(D, dims, trad)):
+            ang = pos * scale * base ** (-2.0 * i / dims)
+            _close([y[i, p], y[i, q]], [math.cos(ang), math.sin(ang)], 1e-14, atol=1e-15,
+                   what=f"angle of pair {i}")
+    # pair 0 turns by exactly pos * scale whatever the base
+    e = np.zeros((1, 4))
+    e[0, 0] = 1.0
+    y = o.rope_f64(e, 1, 4, 0, 1234.5, 0.5, 7)
+    _close(y[0, [0, 2]], [math.cos(3.5), math.sin(3.5)], 1e-15, atol=1e-16, what="theta_0 = 1")
+
+
+def check_rope_traditional_is_permuted_halves(o):
+    """Traditional pairs equal halves pairs conjugated by the de-interleave permutation."""
+    D, dims = 20, 12
+    x = _rng(30).standard_normal((6, D))
+    perm = np.concatenate([np.arange(0, dims, 2), np.arange(1, dims, 2), np.arange(dims, D)])
+    yt = o.rope_f64(x, 3, dims, 1, 10000.0, 1.0, 2)
+    yh = o.rope_f64(x[:, perm], 3, dims, 0, 10000.0, 1.0, 2)
+    back = np.empty_like(yh)
+    back[:, perm] = yh
+    _close(yt, back, 1e-15, what="traditional vs halves")
+
+
+def check_rope_complex(o):
+    """Rotation written as complex multiplication (n_p + i n_q) * exp(i phi)."""
+    D, dims, L = 32, 32, 5
+    x = _rng(31).standard_normal((2 * L, D))
+    half = dims // 2
+    y = o.rope_f64(x, L, dims, 0, 10000.0, 1.0, 100)
+    pos = 100 + (np.arange(2 * L) % L)
+    phi = pos[:, None] * (10000.0 ** (-np.arange(half) * 2.0 / dims))[None, :]
+    z = (x[:, :half] + 1j * x[:, half:dims]) * np.exp(1j * phi)
+    _close(y[:, :half], z.real, 1e-12, atol=1e-12, what="complex real")
+    _close(y[:, half:dims], z.imag, 1e-12, atol=1e-12, what="complex imag")
+
+
+def check_norm_rope_composition(o):
+    """NormRope = Rope(RmsNorm(x, w)); normalize = 0 is Rope alone."""
+    Bsz, H, L, D, dims = 2, 3, 5, 48, 32
+    x = _randn_bf16((Bsz * H * L, D), 32)
+    w = bf16_bits(_rng(33).uniform(0.5, 1.5, D))
+    eps = float(np.float32(1e-6))
+    for trad in (0, 1):
+        y = o.norm_rope(x, w, L, dims, trad, 10000.0, 1.0, 4096, 1, eps)
+        want = o.rope_f64(o.rms_norm(x, w, eps), L, dims, trad, 10000.0, 1.0, 4096)
+        _close(y, want, 1e-15, what="norm_rope composition")
+        y0 = o.norm_rope(x, w, L, dims, trad, 10000.0, 1.0, 7, 0, eps)
+        _close(y0, o.rope_f64(widen_bf16(x), L, dims, trad, 10000.0, 1.0, 7), 1e-15,
+               what="normalize = 0")
+
+
+# ---- hand-worked cases -----------------------------------------------------------------
+
+_MATH = {k: getattr(math, k) for k in ("sqrt", "cos", "sin", "pi")}
+
+
+def _io_array(vals, dt):
+    if vals is None:
+        return None
+    a = np.asarray(vals, np.float64)
+    if dt == "bf16":
+        b = bf16_bits(a)
+        assert (widen_bf16(b) == a).all(), "hand case input not exact in bf16"
+        return b
+    f = a.astype(np.float32)
+    assert (f.astype(np.float64) == a).all(), "hand case input not exact in f32"
+    return f
+
+
+def check_hand_cases(o):
+    """Cases worked by hand from the definitions (tests/golden/hand_cases.json)."""
+    with open(os.path.join(GOLDEN, "hand_cases.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        dt = c["dtype"]
+        x = _io_array(c["x"], dt)
+        w = _io_array(c.get("w"), dt)
+        eps = c["eps"]
+        want = np.array([[eval(e, {"__builtins__": {}}, _MATH) for e in row]
+                         for row in c["expected"]])
+        if c["op"] == "rms_norm":
+            y = o.rms_norm(x, w, eps)
+        elif c["op"] == "add_rms_norm":
+            y, h = o.add_rms_norm(x, _io_array(c["r"], dt), w, eps)
+            hv = widen_bf16(h) if dt == "bf16" else h.astype(np.float64)
+            assert (hv == np.asarray(c["expected_h"])).all(), f"{c['name']}: h"
+        elif c["op"] == "layer_norm":
+            y = o.layer_norm(x, w, _io_array(c.get("b"), dt), eps)
+        elif c["op"] == "norm_rope":
+            y = o.norm_rope(x, w, c["L"], c["dims"], c["traditional"], c["base"], c["scale"],
+                            c["offset"], c["normalize"], eps)
+        else:
+            raise AssertionError(f"unknown op {c['op']}")
+        _close(y, want, 1e-14, atol=1e-15, what=c["name"])
+
+
+def check_minivllm_example(o):
+    """The residual example of the miniVLLM Layers page (shapes only on the page)."""
+    with open(os.path.join(GOLDEN, "minivllm_example.json")) as f:
+        ex = json.load(f)
+    shape = ex["shape"]
+    rows, D = int(np.prod(shape[:-1])), shape[-1]
+    x = _rng(34).standard_normal((rows, D)).astype(np.float32)
+    r = _rng(35).standard_normal((rows, D)).astype(np.float32)
+    w = np.ones(D, np.float32)
+    eps = float(np.float32(ex["eps"]))
+    y, h = o.add_rms_norm(x, r, w, eps)
+    assert (h == x + r).all(), "updated residual must be x + residual"
+    ms = (h.astype(np.float64) ** 2).mean(axis=1)
+    _close((y ** 2).mean(axis=1), ms / (ms + eps), 1e-12, what="example mean square")
+
+
+ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

@@ -1,0 +1,80 @@
+"""Planted mistakes in copies of the oracle must each fail at least one pin (CPU only).
+
+Each mutant is a text substitution in a temporary copy of oracle/oracle.c -- a dropped
+term, a wrong sign, index or order, a wrong rounding -- compiled on its own.  The real
+oracle source is never modified.
+"""
+import os
+
+import pytest
+
+import oracle
+import pins
+
+MUTANTS = {
+    "rms_drops_eps": ("sqrt(sumsq / (double)D + eps)", "sqrt(sumsq / (double)D)"),
+    "rms_sum_not_mean": ("sqrt(sumsq / (double)D + eps)", "sqrt(sumsq + eps)"),
+    "rms_weight_reversed": ("double wj = w ? widen(w, dt, j) : 1.0;\n        y[j] = x[j] / denom",
+                            "double wj = w ? widen(w, dt, D - 1 - j) : 1.0;\n        y[j] = x[j] / denom"),
+    "rms_null_weight_is_zero": ("double wj = w ? widen(w, dt, j) : 1.0;\n        y[j] = x[j] / denom",
+                                "double wj = w ? widen(w, dt, j) : 0.0;\n        y[j] = x[j] / denom"),
+    "rms_multiplies_by_denom": ("y[j] = x[j] / denom * wj;", "y[j] = x[j] * denom * wj;"),
+    "add_normalises_unrounded_h": ("row[j] = widen(h, dt, i);", "row[j] = (double)sum;"),
+    "add_drops_residual": ("float sum = (float)widen(x, dt, i) + (float)widen(r, dt, i);",
+                           "float sum = (float)widen(x, dt, i);"),
+    "layer_unbiased_variance": ("double var = sqdev / (double)D;",
+                                "double var = sqdev / (double)(D - 1);"),
+    "layer_drops_mean_in_output": ("y[j] = (x[j] - mean) / denom * wj + bj;",
+                                   "y[j] = x[j] / denom * wj + bj;"),
+    "layer_drops_bias": ("y[j] = (x[j] - mean) / denom * wj + bj;",
+                         "y[j] = (x[j] - mean) / denom * wj;"),
+    "layer_drops_eps": ("double denom = sqrt(var + eps);", "double denom = sqrt(var);"),
+    "layer_bias_before_scale": ("y[j] = (x[j] - mean) / denom * wj + bj;",
+                                "y[j] = ((x[j] - mean) / denom + bj) * wj;"),
+    "rope_wrong_sign": ("y[p] = x[p] * c - x[q] * s;", "y[p] = x[p] * c + x[q] * s;"),
+    "rope_clockwise": ("y[q] = x[p] * s + x[q] * c;", "y[q] = -x[p] * s + x[q] * c;"),
+    "rope_theta_factor": ("pow(base, -2.0 * (double)i / (double)dims)",
+                          "pow(base, -1.0 * (double)i / (double)dims)"),
+    "rope_theta_over_D": ("pow(base, -2.0 * (double)i / (double)dims)",
+                          "pow(base, -2.0 * (double)i / (double)D)"),
+    "rope_halves_over_D": ("int64_t q = traditional ? 2 * i + 1 : i + half;",
+                           "int64_t q = traditional ? 2 * i + 1 : i + D / 2;"),
+    "rope_traditional_swapped": ("int64_t p = traditional ? 2 * i : i;",
+                                 "int64_t p = traditional ? 2 * i + 1 : i;\n        if (traditional) { int64_t t_ = 2 * i; (void)t_; }"),
+    "rope_ignores_scale": ("double phi = pos * scale * theta;", "double phi = pos * theta;"),
+    "rope_inverse_not_negated": ("if (!forward) phi = -phi;", "(void)forward;"),
+    "rope_ignores_offset": ("double pos = (double)offset + (double)(k % L);\n        rope_row(x + k * D",
+                            "double pos = (double)(k % L);\n        rope_row(x + k * D"),
+    "norm_rope_ignores_offset": ("double pos = (double)offset + (double)(k % L);\n        rope_row(nrm",
+                                 "double pos = (double)(k % L);\n        rope_row(nrm"),
+    "norm_rope_position_k_div_L": ("double pos = (double)offset + (double)(k % L);\n        rope_row(nrm",
+                                   "double pos = (double)offset + (double)(k / L);\n        rope_row(nrm"),
+    "norm_rope_skips_normalise": ("if (normalize)\n            rms_row(row, w, dt, D, (double)eps, nrm);",
+                                  "if (0)\n            rms_row(row, w, dt, D, (double)eps, nrm);"),
+    "round_truncates": ("double n = rint(ldexp(a, -qexp));", "double n = trunc(ldexp(a, -qexp));"),
+    "round_ties_away": ("double n = rint(ldexp(a, -qexp));", "double n = round(ldexp(a, -qexp));"),
+    "round_subnormal_quantum": ("int qexp = (e < -125 ? -125 : e) - 8;", "int qexp = e - 8;"),
+}
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(oracle.SOURCE) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, source, tmp_path):
+    old, new = MUTANTS[name]
+    assert source.count(old) == 1, f"mutation site for {name} not found exactly once"
+    src = tmp_path / "oracle_mutant.c"
+    src.write_text(source.replace(old, new))
+    lib = oracle.compile_oracle(str(src), str(tmp_path / "liboracle_mutant.so"))
+    mutant = oracle.Oracle(lib)
+    failed = []
+    for check in pins.ALL_CHECKS:
+        try:
+            check(mutant)
+        except AssertionError:
+            failed.append(check.__name__)
+    assert failed, f"planted mistake {name!r} passed every pin"
