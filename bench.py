@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Throughput of the fused row-normalisation path on B200 (one JSON line on stdout).
+
+Default workload (one step = one add_rms_norm call through the C ABI):
+    add_rms_norm, bfloat16 I/O, x and r [8192, 4096] ~ N(0, 1), w [4096] ~ U(0.5, 1.5),
+    eps = 1e-5; outputs y and h = x + r.
+Metric: achieved HBM GB/s of algorithmic bytes (4 N s + D s per call, s = 2) and rows/s,
+against B200's HBM peak.  L2 is flushed (a write of 2x the L2 size) before every step;
+each step is timed alone with CUDA events on the launching stream.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --sweep        # add_rms_norm over D x rows x dtype, one line per point
+
+Multi-GPU (torchrun, one process per GPU): rows are independent, so every rank runs its
+own batch of the same shape (weak scaling); there is no data-path collective.  The
+reported time is the maximum over ranks of the summed per-step device times.
+
+``--impl reference`` times the CPU oracle (the only reference that exists for this
+path: the pages publish no implementation or numbers) on a bounded sample of the same
+workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "add_rms_norm achieved HBM GB/s and rows/s vs 8 TB/s peak (1×B200)"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+WORKLOAD = {"rows": 8192, "D": 4096, "dtype": "bf16", "eps": 1e-5}
+KERNEL_SOURCES = ["rope_add_rms_b200/csrc/rms.cuh", "rope_add_rms_b200/csrc/common.cuh",
+                  "rope_add_rms_b200/csrc/layer.cuh", "rope_add_rms_b200/csrc/rope.cuh",
+                  "rope_add_rms_b200/csrc/nvnorm_api.cu"]
+
+
+# ---- environment --------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """dram bytes per launch recorded from an ncu capture, if the kernels are unchanged."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = d.get(kernel_key)
+    if not ent or ent.get("source_hash") != source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples of one GPU while a region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [r[0] for r in rows]
+        reasons = sorted({self.NAMES[i] for r in rows for i, v in enumerate(r[2])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---- workloads ----------------------------------------------------------------------
+
+def algorithmic_bytes(op, rows, D, s):
+    if op == "add_rms_norm":
+        return 4 * rows * D * s + D * s
+    if op == "rms_norm":
+        return 2 * rows * D * s + D * s
+    if op == "layer_norm":
+        return 2 * rows * D * s + 2 * D * s
+    if op == "norm_rope":
+        return 2 * rows * D * s + D * s
+    raise ValueError(op)
+
+
+class Case:
+    """Device-resident inputs/outputs of one workload and a callable that runs it once."""
+
+    def __init__(self, op, shape, dtype, seed, **kw):
+        from rope_add_rms_b200 import synth
+        import rope_add_rms_b200 as nv
+        self.op, self.dtype, self.kw = op, dtype, kw
+        tdt = synth.DTYPES[dtype]
+        self.s = torch.empty((), dtype=tdt).element_size()
+        if op == "norm_rope":
+            B, H, L, D = shape
+            inp = synth.norm_rope_inputs(B, H, L, D, dtype, seed)
+            self.rows, self.D, self.L = B * H * L, D, L
+        else:
+            rows, D = shape
+            self.rows, self.D = rows, D
+            if op == "add_rms_norm":
+                inp = synth.add_rms_inputs(rows, D, dtype, seed)
+            elif op == "rms_norm":
+                inp = synth.rms_inputs(rows, D, dtype, seed)
+            else:
+                inp = synth.layer_norm_inputs(rows, D, dtype, seed)
+        self.host = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+        self.dev = {k: (v.cuda() if v is not None else None) for k, v in self.host.items()}
+        x = self.dev["x"]
+        self.y = torch.empty_like(x)
+        self.h = torch.empty_like(x) if op == "add_rms_norm" else None
+        self.bytes = algorithmic_bytes(op, self.rows, self.D, self.s)
+        self.nv = nv
+        if op == "add_rms_norm":
+            self.host_out = [torch.empty_like(self.host["x"]).pin_memory() for _ in range(2)]
+        else:
+            self.host_out = [torch.empty_like(self.host["x"]).pin_memory()]
+
+    def run(self, stream=None):
+        d, nv = self.dev, self.nv
+        if self.op == "add_rms_norm":
+            nv.nv_add_rms_norm(d["x"], d["r"], d["w"], self.y, self.h, self.kw["eps"], stream)
+        elif self.op == "rms_norm":
+            nv.nv_rms_norm(d["x"], d["w"], self.y, self.kw["eps"], stream)
+        elif self.op == "layer_norm":
+            nv.nv_layer_norm(d["x"], d["w"], d["b"], self.y, self.kw["eps"], stream)
+        else:
+            k = self.kw
+            nv.nv_norm_rope(d["x"], d["w"], self.y, self.L, k["dims"], k["traditional"], k["base"],
+                            k["scale"], k["offset"], 1, k["eps"], stream)
+
+    def run_e2e(self, stream):
+        """Host -> device copy of the step's inputs, the call, device -> host of its outputs."""
+        self.dev["x"].copy_(self.host["x"], non_blocking=True)
+        if self.op == "add_rms_norm":
+            self.dev["r"].copy_(self.host["r"], non_blocking=True)
+        self.run(stream)
+        self.host_out[0].copy_(self.y, non_blocking=True)
+        if self.h is not None:
+            self.host_out[1].copy_(self.h, non_blocking=True)
+
+    def e2e_bytes(self):
+        n_in = 2 if self.op == "add_rms_norm" else 1
+        n_out = 2 if self.op == "add_rms_norm" else 1
+        per = self.rows * self.D * self.s
+        return n_in * per, n_out * per
+
+
+def l2_flush_buffer():
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    return torch.empty(2 * max(l2, 64 << 20), dtype=torch.uint8, device="cuda")
+
+
+def time_steps(case, steps, warmup, flush, e2e=False):
+    """Per-step device times (ms) of `steps` runs, each after an L2 flush."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush.zero_()
+        (case.run_e2e if e2e else case.run)(stream)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        (case.run_e2e if e2e else case.run)(stream)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+# ---- arms -----------------------------------------------------------------------------
+
+def cpu_baseline(seconds=10.0, sample_rows=2048):
+    """The CPU oracle on a bounded sample of the default workload (rank 0, N = 1)."""
+    import oracle
+    from rope_add_rms_b200 import synth
+    rows, D = sample_rows, WORKLOAD["D"]
+    inp = synth.add_rms_inputs(rows, D, "bf16", 0)
+    x, r, w = (synth.to_numpy(inp[k]) for k in ("x", "r", "w"))
+    o = oracle.get()
+    threads = oracle.default_threads()
+    o.add_rms_norm(x, r, w, WORKLOAD["eps"], threads=threads)     # warm
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        o.add_rms_norm(x, r, w, WORKLOAD["eps"], threads=threads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or reps >= 1000:
+            break
+    gbs = algorithmic_bytes("add_rms_norm", rows, D, 2) * reps / el / 1e9
+    return {"value": round(gbs, 3), "unit": "GB/s", "cores": o.last_threads, "kind": "oracle",
+            "sample": f"{reps} x add_rms_norm bf16 [{rows}, {D}] (of the [8192, 4096] workload), "
+                      f"{el:.1f} s wall, fp64 C oracle, rows split over threads",
+            "rows_per_s": round(rows * reps / el, 1)}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    from rope_add_rms_b200 import synth
+    rows, D = 512, WORKLOAD["D"]
+    inp = synth.add_rms_inputs(rows, D, "bf16", 0)
+    x, r, w = (synth.to_numpy(inp[k]) for k in ("x", "r", "w"))
+    o = oracle.get()
+    threads = oracle.default_threads()
+    for _ in range(args.warmup):
+        o.add_rms_norm(x, r, w, WORKLOAD["eps"], threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        o.add_rms_norm(x, r, w, WORKLOAD["eps"], threads=threads)
+    el = time.perf_counter() - t0
+    nbytes = algorithmic_bytes("add_rms_norm", rows, D, 2)
+    gbs = nbytes * args.steps / el / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "add_rms_norm bf16 [8192,4096] eps 1e-5 (CPU oracle on a "
+                               "512-row sample per step)", "rows": rows, "D": D},
+        "rows_per_s": round(rows * args.steps / el, 1),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": o.last_threads,
+                         "kind": "oracle",
+                         "sample": f"{args.steps} steps x add_rms_norm bf16 [{rows}, {D}]"},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def other_configs(flush, steps):
+    """Fractions of the roofline for the other workloads (reported, not the headline)."""
+    peak, _ = measured_peak()
+    out = {}
+    cases = {
+        "layer_norm bf16 [16384,8192] x~N(0.5,2^2) eps 1e-5":
+            Case("layer_norm", (16384, 8192), "bf16", 0, eps=1e-5),
+        "norm_rope bf16 [8,32,2048,128] halves offset 0 eps 1e-6":
+            Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6, dims=128, traditional=0,
+                 base=10000.0, scale=1.0, offset=0),
+        "norm_rope bf16 [8,32,2048,128] traditional offset 4096 eps 1e-6":
+            Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6, dims=128, traditional=1,
+                 base=10000.0, scale=1.0, offset=4096),
+        "rms_norm f32 [64,512] eps 1e-6":
+            Case("rms_norm", (64, 512), "f32", 0, eps=1e-6),
+    }
+    for name, c in cases.items():
+        ts = time_steps(c, steps, 3, flush)
+        med = statistics.median(ts)
+        gbs = c.bytes / (med * 1e-3) / 1e9
+        out[name] = {"median_us": round(med * 1e3, 2), "GB/s": round(gbs, 1),
+                     "frac_of_measured_hbm": round(gbs / peak, 4),
+                     "rows_per_s": round(c.rows / (med * 1e-3), 1)}
+        del c
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args):
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    import rope_add_rms_b200 as nv
+    nv.library()
+
+    case = Case("add_rms_norm", (WORKLOAD["rows"], WORKLOAD["D"]), WORKLOAD["dtype"], seed=rank,
+                eps=WORKLOAD["eps"])
+    flush = l2_flush_buffer()
+
+    def barrier():
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    # warm-up, then the timed steps with clocks sampled during them
+    barrier()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ts = time_steps(case, args.steps, args.warmup, flush)
+    barrier()
+    total_ms = sum(ts)
+    e2e_steps = max(3, min(args.steps, 20))
+    te = time_steps(case, e2e_steps, 3, flush, e2e=True)
+    barrier()
+    e2e_ms = sum(te)
+    if pg:
+        t = torch.tensor([total_ms, e2e_ms], device="cuda", dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms, e2e_ms = t.tolist()
+
+    extras = None
+    if rank == 0 and not args.no_extras and world == 1:
+        extras = other_configs(flush, max(5, min(args.steps, 50)))
+    baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        baseline = cpu_baseline(args.cpu_seconds)
+
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        step_bytes = case.bytes
+        value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+        per_launch_ms = statistics.mean(ts)
+        achieved = step_bytes / (per_launch_ms * 1e-3) / 1e9
+        bi, bo = case.e2e_bytes()
+        e2e_value = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
+        plan = nv.nv_describe_plan("add_rms_norm", WORKLOAD["rows"], WORKLOAD["D"],
+                                   torch.bfloat16)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "add_rms_norm bf16 x,r [8192,4096] ~N(0,1), w [4096] "
+                                   "~U(0.5,1.5), eps 1e-5 (outputs y, h); per GPU",
+                       "rows": WORKLOAD["rows"], "D": WORKLOAD["D"], "global_batch_rows":
+                           WORKLOAD["rows"] * world,
+                       "l2": "flushed before every step (write of 2x L2)",
+                       "parallelism": f"row shards x{world}, no collective",
+                       "plan": plan},
+            "rows_per_s": round(world * WORKLOAD["rows"] * args.steps / (total_ms * 1e-3), 1),
+            "step_us": {"median": round(statistics.median(ts) * 1e3, 3),
+                        "p10": round(float(np.percentile(ts, 10)) * 1e3, 3),
+                        "p90": round(float(np.percentile(ts, 90)) * 1e3, 3)},
+            "frac_of_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": ncu_traffic("add_rms_norm_bf16_8192x4096"),
+                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_kind == "measured" else "fallback 6650 GB/s",
+                         "kernel": f"rms_rows_kernel<bf16, VPT={plan['vec_per_thread']}, ADD>",
+                         "bytes_per_launch": step_bytes},
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": bi,
+                    "d2h_bytes_per_step": bo,
+                    "ms_per_step": round(e2e_ms / e2e_steps, 4), "steps": e2e_steps,
+                    "how": "pinned host x, r -> device, nv_add_rms_norm, y, h -> pinned host; "
+                           "all on one stream inside the events"},
+            "gpu_launches": args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": baseline,
+            "other_configs": extras,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def run_sweep(args):
+    """add_rms_norm over D x rows x dtype (eps 1e-6): one JSON line per point."""
+    torch.cuda.set_device(dist_env()[2])
+    flush = l2_flush_buffer()
+    peak, _ = measured_peak()
+    for dtype in ("bf16", "f32"):
+        for D in (2048, 4096, 5120, 8192, 16384):
+            for rows in (1, 16, 256, 4096, 65536):
+                c = Case("add_rms_norm", (rows, D), dtype, 0, eps=1e-6)
+                ts = time_steps(c, args.steps, args.warmup, flush)
+                med = statistics.median(ts)
+                gbs = c.bytes / (med * 1e-3) / 1e9
+                print(json.dumps({"op": "add_rms_norm", "dtype": dtype, "rows": rows, "D": D,
+                                  "median_us": round(med * 1e3, 2), "GB/s": round(gbs, 1),
+                                  "frac": round(gbs / peak, 4),
+                                  "rows_per_s": round(rows / (med * 1e-3), 1),
+                                  "bound": "hbm" if rows >= 4096 else "latency"}), flush=True)
+                del c
+                torch.cuda.empty_cache()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=None)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

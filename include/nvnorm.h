@@ -1,0 +1,176 @@
+/*
+ * nvnorm.h -- C ABI of the B200 (sm_100a) fused row-normalisation library, libnvnorm.so.
+ *
+ * Every op works row by row over the last axis of a contiguous row-major array
+ * [rows, D] (rows = the product of the leading axes), with one element type for
+ * all tensors of a call.  Arithmetic is float32 inside the kernels, with wider
+ * arithmetic where a bfloat16 result would otherwise lose its last bit (layer_norm
+ * statistics, the rope rotation); the results are rounded once, to nearest even.
+ *
+ * Ownership and memory
+ *   - The caller owns every buffer.  The library allocates no memory, keeps no
+ *     per-call state and has no handle.  All pointers are device (or managed)
+ *     memory of the CURRENT device; each one is checked on the host against its
+ *     allocation's extent before anything is launched.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream); a
+ *     return of NV_OK means the kernel was launched, not that it finished.
+ *   - An output may be the very same buffer as an input (y == x, h == x, h == r):
+ *     each row is read completely before it is written.  Any other overlap between
+ *     an output and another buffer, and y == h, are rejected.
+ *
+ * Errors
+ *   - Every argument is validated on the host before any launch; a failure
+ *     returns NV_ERR_INVALID_ARG (or NV_ERR_UNSUPPORTED) and launches nothing.
+ *   - rows == 0 is valid and launches nothing.
+ *   - A launch failure reported by the CUDA runtime returns NV_ERR_CUDA.
+ *   - nv_last_error() gives a message for the last non-OK status of the calling
+ *     thread.  No C++ exception crosses this interface.
+ *   - Invalid input values (Inf, NaN) are not errors: they propagate through the
+ *     row that holds them, per IEEE arithmetic, and reach no other row.
+ *
+ * Scalars: eps, base and scale are float32 values, as the op definitions store them
+ * (docs.rs nuvec-core 0.5.0, Enum FastOp: every field is f32::to_bits).
+ */
+#ifndef NVNORM_H
+#define NVNORM_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NV_API __attribute__((visibility("default")))
+#else
+#define NV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (the same handle as cudaStream_t / CUstream). */
+typedef struct CUstream_st* nv_stream_t;
+
+typedef enum {
+    NV_F32 = 0,  /* IEEE binary32 */
+    NV_BF16 = 1, /* bfloat16 */
+    NV_F16 = 2   /* IEEE binary16: reserved, returns NV_ERR_UNSUPPORTED */
+} nv_dtype;
+
+typedef enum {
+    NV_OK = 0,
+    NV_ERR_INVALID_ARG = 1,
+    NV_ERR_UNSUPPORTED = 2,
+    NV_ERR_CUDA = 3
+} nv_status;
+
+/*
+ * rms_norm -- docs.rs nuvec-core 0.5.0, Enum FastOp, variant RmsNorm:
+ *   y = x / sqrt(mean(x^2) + eps) * w over the last axis; w is 1-D or the scalar 1
+ *   (nuvec-nn src/layers.rs, RmsNorm::forward; miniVLLM Layers page, LayerNorm with
+ *   residual = None).
+ * x [rows, D] in; w [D] in, or NULL for w = 1; y [rows, D] out (may be x).
+ * rows >= 0, D >= 1, eps finite and >= 0.
+ */
+NV_API nv_status nv_rms_norm(const void* x, const void* w, void* y, int64_t rows, int64_t D, float eps,
+                      nv_dtype dt, nv_stream_t stream);
+
+/*
+ * add_rms_norm -- docs.rs nuvec-core 0.5.0, Enum FastOp, variant AddRmsNorm:
+ *   h = x + r and RmsNorm of h; miniVLLM Layers page, LayerNorm.forward with a
+ *   residual (x_new = x + residual, normalise x_new, return (normalised, x_new)).
+ * h is the float32 sum x + r rounded once to the I/O type, and y normalises exactly
+ * that rounded h, so add_rms_norm(x, r) == rms_norm(h) bit for bit.
+ * x, r [rows, D] in; w [D] in or NULL (w = 1); y [rows, D] out; h [rows, D] out.
+ * h may be x or r; y may be x or r; y != h.
+ */
+NV_API nv_status nv_add_rms_norm(const void* x, const void* r, const void* w, void* y, void* h,
+                          int64_t rows, int64_t D, float eps, nv_dtype dt, nv_stream_t stream);
+
+/*
+ * layer_norm -- docs.rs nuvec-core 0.5.0, Enum FastOp, variant LayerNorm:
+ *   y = (x - mean) / sqrt(var + eps) * w + b over the last axis, w and b 1-D or the
+ *   scalars 1 and 0 (nuvec-nn src/layers.rs, LayerNorm: affine / without_bias).
+ * var is the population variance (sum of squared deviations / D).
+ * x [rows, D] in; w [D] or NULL (w = 1); b [D] or NULL (b = 0); y [rows, D] out.
+ */
+NV_API nv_status nv_layer_norm(const void* x, const void* w, const void* b, void* y, int64_t rows,
+                        int64_t D, float eps, nv_dtype dt, nv_stream_t stream);
+
+/*
+ * norm_rope -- docs.rs nuvec-core 0.5.0, Enum FastOp, variants NormRope and Rope
+ * (non-cache form): each [b, h, l] row of x [B, H, L, D] is RMS-normalised with eps
+ * and w, then its first dims features are rotated at position offset + l:
+ *   theta_i = base^(-2 i / dims), phi_i = (offset + l) * scale * theta_i,
+ *   (y_p, y_q) = (n_p cos phi_i - n_q sin phi_i, n_p sin phi_i + n_q cos phi_i)
+ * for the pairs (p, q) = (i, i + dims/2) (traditional = 0: the two halves) or
+ * (2i, 2i + 1) (traditional != 0: interleaved pairs).  Features j >= dims keep the
+ * normalised value.  normalize == 0 is plain Rope: no normalisation, w and eps unused.
+ * x [rows, D] in with rows = B*H*L (row k at l = k mod L); w [D] or NULL (w = 1);
+ * y [rows, D] out (may be x).
+ * L >= 1, rows % L == 0, dims even with 0 < dims <= D, base > 0 and finite, scale
+ * finite, offset >= 0, eps finite and >= 0 (checked only when normalize != 0).
+ */
+NV_API nv_status nv_norm_rope(const void* x, const void* w, void* y, int64_t rows, int64_t L, int64_t D,
+                       int32_t dims, int32_t traditional, float base, float scale, int64_t offset,
+                       int32_t normalize, float eps, nv_dtype dt, nv_stream_t stream);
+
+/* Name of a status code (static storage). */
+NV_API const char* nv_status_string(nv_status status);
+
+/* Message for the calling thread's last non-OK status ("" if none yet). */
+NV_API const char* nv_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+NV_API int32_t nv_version(void);
+
+/*
+ * Kernel-variant control, for tests and benchmarks.  The plain entry points above
+ * pick a variant from (op, dtype, D, rows, alignment); the *_ex forms take a plan
+ * that forces one.  A plan that the shape cannot use returns NV_ERR_UNSUPPORTED.
+ *   path            NV_PATH_AUTO, or one of the kernel families below
+ *   vec_per_thread  16-byte vectors per thread and row (register paths; 0 = auto)
+ *   threads_per_row threads that share one row (multiple of 32, <= 1024; 0 = auto)
+ *   rows_per_cta    rows one CTA works on at a time (0 = auto)
+ *   ctas_per_sm     persistent grid size per SM (0 = auto)
+ */
+typedef enum {
+    NV_PATH_AUTO = 0,
+    NV_PATH_ROWS = 1,    /* row held in registers, 16-byte vector loads */
+    NV_PATH_GENERIC = 2, /* any D and alignment: scalar loop, two passes over the row */
+    NV_PATH_STAGED = 3   /* persistent, rows staged in shared memory by bulk async copies */
+} nv_path;
+
+typedef struct {
+    int32_t path;
+    int32_t vec_per_thread;
+    int32_t threads_per_row;
+    int32_t rows_per_cta;
+    int32_t ctas_per_sm;
+} nv_plan;
+
+NV_API nv_status nv_rms_norm_ex(const void* x, const void* w, void* y, int64_t rows, int64_t D,
+                         float eps, nv_dtype dt, nv_stream_t stream, const nv_plan* plan);
+NV_API nv_status nv_add_rms_norm_ex(const void* x, const void* r, const void* w, void* y, void* h,
+                             int64_t rows, int64_t D, float eps, nv_dtype dt, nv_stream_t stream,
+                             const nv_plan* plan);
+NV_API nv_status nv_layer_norm_ex(const void* x, const void* w, const void* b, void* y, int64_t rows,
+                           int64_t D, float eps, nv_dtype dt, nv_stream_t stream,
+                           const nv_plan* plan);
+NV_API nv_status nv_norm_rope_ex(const void* x, const void* w, void* y, int64_t rows, int64_t L,
+                          int64_t D, int32_t dims, int32_t traditional, float base, float scale,
+                          int64_t offset, int32_t normalize, float eps, nv_dtype dt,
+                          nv_stream_t stream, const nv_plan* plan);
+
+/*
+ * The plan that the plain entry point would use for these arguments (for reports).
+ * op: 0 rms_norm, 1 add_rms_norm, 2 layer_norm, 3 norm_rope.  Returns NV_OK and
+ * fills *plan, or an error status as the op itself would for invalid sizes.  For
+ * norm_rope, D is the row length and dims/traditional are not considered; pointer
+ * alignment is assumed to be 16 bytes.
+ */
+NV_API nv_status nv_describe_plan(int32_t op, int64_t rows, int64_t D, nv_dtype dt, nv_plan* plan);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVNORM_H */

@@ -1,0 +1,220 @@
+"""rope_add_rms_b200 -- Python binding of libnvnorm.so, the B200 fused row-normalisation library.
+
+This module only marshals arguments: every step of every op runs in the CUDA kernels of
+``libnvnorm.so`` (built from ``csrc/`` for sm_100a).  There is no fallback: if the library
+is missing or a call fails, an exception is raised.  PyTorch supplies device memory and
+the current stream.
+
+The ``nv_*`` functions mirror the C entry points of ``include/nvnorm.h`` and write into
+caller-provided output tensors.  ``rms_norm``, ``add_rms_norm``, ``layer_norm`` and
+``norm_rope`` allocate their outputs and return them.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "NvError", "Plan", "library", "library_path",
+    "nv_rms_norm", "nv_add_rms_norm", "nv_layer_norm", "nv_norm_rope", "nv_describe_plan",
+    "rms_norm", "add_rms_norm", "layer_norm", "norm_rope",
+    "PATH_AUTO", "PATH_ROWS", "PATH_GENERIC", "PATH_STAGED",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libnvnorm.so")
+
+NV_F32, NV_BF16, NV_F16 = 0, 1, 2
+NV_OK, NV_ERR_INVALID_ARG, NV_ERR_UNSUPPORTED, NV_ERR_CUDA = 0, 1, 2, 3
+PATH_AUTO, PATH_ROWS, PATH_GENERIC, PATH_STAGED = 0, 1, 2, 3
+
+_DT = {torch.float32: NV_F32, torch.bfloat16: NV_BF16, torch.float16: NV_F16}
+
+
+class NvError(RuntimeError):
+    """A non-OK status from libnvnorm.so, with the library's message."""
+
+    def __init__(self, fn: str, status: int, message: str):
+        self.status = status
+        self.message = message
+        super().__init__(f"{fn}: {_status_name(status)}: {message}")
+
+
+class Plan(ctypes.Structure):
+    """nv_plan: kernel-variant selection (0 fields mean automatic)."""
+    _fields_ = [("path", ctypes.c_int32), ("vec_per_thread", ctypes.c_int32),
+                ("threads_per_row", ctypes.c_int32), ("rows_per_cta", ctypes.c_int32),
+                ("ctas_per_sm", ctypes.c_int32)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """Load libnvnorm.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise ImportError(f"{library_path} is missing: build it with "
+                          "`python -m rope_add_rms_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(library_path)
+    vp, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+    pp = ctypes.POINTER(Plan)
+    sigs = {
+        "nv_rms_norm": [vp, vp, vp, i64, i64, f32, i32, vp],
+        "nv_add_rms_norm": [vp, vp, vp, vp, vp, i64, i64, f32, i32, vp],
+        "nv_layer_norm": [vp, vp, vp, vp, i64, i64, f32, i32, vp],
+        "nv_norm_rope": [vp, vp, vp, i64, i64, i64, i32, i32, f32, f32, i64, i32, f32, i32, vp],
+        "nv_rms_norm_ex": [vp, vp, vp, i64, i64, f32, i32, vp, pp],
+        "nv_add_rms_norm_ex": [vp, vp, vp, vp, vp, i64, i64, f32, i32, vp, pp],
+        "nv_layer_norm_ex": [vp, vp, vp, vp, i64, i64, f32, i32, vp, pp],
+        "nv_norm_rope_ex": [vp, vp, vp, i64, i64, i64, i32, i32, f32, f32, i64, i32, f32, i32,
+                            vp, pp],
+        "nv_describe_plan": [i32, i64, i64, i32, pp],
+    }
+    for name, args in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.nv_status_string.argtypes = [ctypes.c_int]
+    lib.nv_status_string.restype = ctypes.c_char_p
+    lib.nv_last_error.argtypes = []
+    lib.nv_last_error.restype = ctypes.c_char_p
+    lib.nv_version.argtypes = []
+    lib.nv_version.restype = ctypes.c_int32
+    _lib = lib
+    return lib
+
+
+def _status_name(status: int) -> str:
+    return library().nv_status_string(status).decode()
+
+
+def _check(fn: str, status: int):
+    if status != NV_OK:
+        raise NvError(fn, status, library().nv_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype(*ts):
+    dts = {t.dtype for t in ts if t is not None}
+    if len(dts) != 1:
+        raise TypeError(f"all tensors must share one dtype, got {sorted(map(str, dts))}")
+    dt = dts.pop()
+    if dt not in _DT:
+        raise TypeError(f"unsupported dtype {dt}")
+    return _DT[dt]
+
+
+def _rows_D(x):
+    if not x.is_contiguous():
+        raise ValueError("tensors must be contiguous (row-major, last axis contiguous)")
+    D = x.shape[-1] if x.dim() else 1
+    return (x.numel() // D if D else 0), D
+
+
+def _plan(plan):
+    if plan is None:
+        return None
+    if isinstance(plan, dict):
+        plan = Plan(**plan)
+    return ctypes.byref(plan)
+
+
+# ---- C-ABI mirrors (outputs provided by the caller) ------------------------------------
+
+def nv_rms_norm(x, w, y, eps, stream=None, plan=None):
+    rows, D = _rows_D(x)
+    lib = library()
+    args = (_ptr(x), _ptr(w), _ptr(y), rows, D, eps, _dtype(x, w, y), _stream(stream))
+    st = lib.nv_rms_norm(*args) if plan is None else lib.nv_rms_norm_ex(*args, _plan(plan))
+    _check("nv_rms_norm", st)
+
+
+def nv_add_rms_norm(x, r, w, y, h, eps, stream=None, plan=None):
+    rows, D = _rows_D(x)
+    lib = library()
+    args = (_ptr(x), _ptr(r), _ptr(w), _ptr(y), _ptr(h), rows, D, eps, _dtype(x, r, w, y, h),
+            _stream(stream))
+    st = lib.nv_add_rms_norm(*args) if plan is None else lib.nv_add_rms_norm_ex(*args, _plan(plan))
+    _check("nv_add_rms_norm", st)
+
+
+def nv_layer_norm(x, w, b, y, eps, stream=None, plan=None):
+    rows, D = _rows_D(x)
+    lib = library()
+    args = (_ptr(x), _ptr(w), _ptr(b), _ptr(y), rows, D, eps, _dtype(x, w, b, y), _stream(stream))
+    st = lib.nv_layer_norm(*args) if plan is None else lib.nv_layer_norm_ex(*args, _plan(plan))
+    _check("nv_layer_norm", st)
+
+
+def nv_norm_rope(x, w, y, L, dims, traditional, base, scale, offset, normalize, eps,
+                 stream=None, plan=None):
+    rows, D = _rows_D(x)
+    lib = library()
+    args = (_ptr(x), _ptr(w), _ptr(y), rows, L, D, dims, int(bool(traditional)), base, scale,
+            offset, int(bool(normalize)), eps, _dtype(x, w, y), _stream(stream))
+    st = lib.nv_norm_rope(*args) if plan is None else lib.nv_norm_rope_ex(*args, _plan(plan))
+    _check("nv_norm_rope", st)
+
+
+def nv_describe_plan(op: str, rows: int, D: int, dtype) -> dict:
+    """The kernel variant the library picks for op on [rows, D] (16-byte aligned data)."""
+    ops = {"rms_norm": 0, "add_rms_norm": 1, "layer_norm": 2, "norm_rope": 3}
+    p = Plan()
+    _check("nv_describe_plan", library().nv_describe_plan(ops[op], rows, D, _DT[dtype],
+                                                           ctypes.byref(p)))
+    return p.as_dict()
+
+
+# ---- allocating wrappers ---------------------------------------------------------------
+
+def rms_norm(x, w=None, eps=1e-5, stream=None):
+    """y = x / sqrt(mean(x^2) + eps) * w over the last axis."""
+    y = torch.empty_like(x)
+    nv_rms_norm(x, w, y, eps, stream)
+    return y
+
+
+def add_rms_norm(x, r, w=None, eps=1e-5, stream=None):
+    """(y, h): h = x + r (rounded to x's dtype), y = rms_norm(h, w, eps)."""
+    y = torch.empty_like(x)
+    h = torch.empty_like(x)
+    nv_add_rms_norm(x, r, w, y, h, eps, stream)
+    return y, h
+
+
+def layer_norm(x, w=None, b=None, eps=1e-5, stream=None):
+    """y = (x - mean) / sqrt(var + eps) * w + b over the last axis."""
+    y = torch.empty_like(x)
+    nv_layer_norm(x, w, b, y, eps, stream)
+    return y
+
+
+def norm_rope(x, w=None, dims=None, traditional=False, base=10000.0, scale=1.0, offset=0,
+              eps=1e-6, stream=None):
+    """RMS-normalise each row of x [..., L, D] (eps None: skip), then rotate its first dims
+    features at positions offset + l (l the index on the second-to-last axis)."""
+    if x.dim() < 2:
+        raise ValueError("x must be [..., L, D]")
+    L, D = x.shape[-2], x.shape[-1]
+    y = torch.empty_like(x)
+    normalize = eps is not None
+    nv_norm_rope(x, w, y, L, D if dims is None else dims, traditional, base, scale, offset,
+                 normalize, eps if normalize else 0.0, stream)
+    return y

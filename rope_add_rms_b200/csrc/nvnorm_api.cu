@@ -1,0 +1,590 @@
+// nvnorm_api.cu -- the C ABI of libnvnorm.so: argument validation, kernel-variant
+// selection and launch.  Declarations and the contract of every entry point are in
+// include/nvnorm.h.
+#include <cuda.h>  // CUresult / CUdeviceptr for the driver range query (no libcuda link)
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "nvnorm.h"
+
+#include "common.cuh"
+#include "layer.cuh"
+#include "rms.cuh"
+#include "rope.cuh"
+
+namespace {
+
+using namespace nvn;
+
+constexpr int kVersion = 100;  // 0.1.0
+
+// ---- error reporting ------------------------------------------------------------------
+thread_local char g_msg[512] = "";
+
+nv_status fail(nv_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+nv_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(NV_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// ---- device facts, cached per device ---------------------------------------------------
+struct DevInfo {
+    int sms = 0;
+    bool ready = false;
+};
+constexpr int kMaxDevices = 64;
+DevInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+nv_status current_device(int* dev, DevInfo* info) {
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (*dev < 0 || *dev >= kMaxDevices) return fail(NV_ERR_UNSUPPORTED, "device %d", *dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevInfo& d = g_dev[*dev];
+    if (!d.ready) {
+        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, *dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        d.ready = true;
+    }
+    *info = d;
+    return NV_OK;
+}
+
+// ---- pointer checks ----------------------------------------------------------------------
+// cuMemGetAddressRange, fetched through the runtime so the library needs no libcuda link.
+using RangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
+RangeFn range_fn() {
+    static RangeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<RangeFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+struct Buf {
+    const void* p;
+    size_t bytes;
+    const char* name;
+    bool output;
+    bool row_input;  // an output may be the very same buffer as a row input
+};
+
+// The buffer must be device (or managed) memory of the current device and lie inside
+// one allocation.
+nv_status check_pointer(const Buf& b, int dev) {
+    cudaPointerAttributes at;
+    cudaError_t e = cudaPointerGetAttributes(&at, b.p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(NV_ERR_INVALID_ARG, "%s (%p) is not a CUDA pointer: %s", b.name, b.p,
+                    cudaGetErrorString(e));
+    }
+    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
+        return fail(NV_ERR_INVALID_ARG, "%s (%p) is not device memory", b.name, b.p);
+    if (at.type == cudaMemoryTypeDevice && at.device != dev)
+        return fail(NV_ERR_INVALID_ARG, "%s (%p) belongs to device %d, current device is %d",
+                    b.name, b.p, at.device, dev);
+    RangeFn fn = range_fn();
+    if (fn) {
+        CUdeviceptr base = 0;
+        size_t size = 0;
+        if (fn(&base, &size, (CUdeviceptr)(uintptr_t)b.p) != CUDA_SUCCESS)
+            return fail(NV_ERR_INVALID_ARG, "%s (%p): allocation not found", b.name, b.p);
+        const uintptr_t lo = (uintptr_t)b.p;
+        if (lo + b.bytes > (uintptr_t)base + size)
+            return fail(NV_ERR_INVALID_ARG,
+                        "%s (%p): %zu bytes run past the end of its allocation "
+                        "(%zu bytes at %p)",
+                        b.name, b.p, b.bytes, size, (void*)(uintptr_t)base);
+    }
+    return NV_OK;
+}
+
+nv_status check_buffers(const Buf* bufs, int n, int dev) {
+    for (int i = 0; i < n; ++i) {
+        if (!bufs[i].p) continue;
+        nv_status st = check_pointer(bufs[i], dev);
+        if (st != NV_OK) return st;
+    }
+    // an output may not overlap anything, except that it may be exactly a row input
+    for (int i = 0; i < n; ++i) {
+        if (!bufs[i].p || !bufs[i].output) continue;
+        const uintptr_t a0 = (uintptr_t)bufs[i].p, a1 = a0 + bufs[i].bytes;
+        for (int j = 0; j < n; ++j) {
+            if (j == i || !bufs[j].p) continue;
+            const uintptr_t b0 = (uintptr_t)bufs[j].p, b1 = b0 + bufs[j].bytes;
+            if (a0 >= b1 || b0 >= a1) continue;
+            if (a0 == b0 && bufs[i].bytes == bufs[j].bytes && bufs[j].row_input) continue;
+            return fail(NV_ERR_INVALID_ARG, "output %s overlaps %s", bufs[i].name, bufs[j].name);
+        }
+    }
+    return NV_OK;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+size_t elem_size(nv_dtype dt) { return dt == NV_F32 ? 4 : 2; }
+
+nv_status check_common(int64_t rows, int64_t D, float eps, nv_dtype dt, bool check_eps = true) {
+    if (dt == NV_F16) return fail(NV_ERR_UNSUPPORTED, "dtype NV_F16 is not supported");
+    if (dt != NV_F32 && dt != NV_BF16) return fail(NV_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    if (rows < 0) return fail(NV_ERR_INVALID_ARG, "rows = %lld < 0", (long long)rows);
+    if (D < 1) return fail(NV_ERR_INVALID_ARG, "D = %lld < 1", (long long)D);
+    if (D > (int64_t)1 << 30) return fail(NV_ERR_UNSUPPORTED, "D = %lld > 2^30", (long long)D);
+    if (check_eps && (!std::isfinite(eps) || eps < 0.f))
+        return fail(NV_ERR_INVALID_ARG, "eps = %g must be finite and >= 0", (double)eps);
+    const size_t s = elem_size(dt);
+    if ((uint64_t)rows > (uint64_t)INT64_MAX / ((uint64_t)D * s))
+        return fail(NV_ERR_INVALID_ARG, "rows * D overflows");
+    return NV_OK;
+}
+
+// ---- plans --------------------------------------------------------------------------------
+enum Op { OP_RMS = 0, OP_ADD = 1, OP_LAYER = 2, OP_ROPE = 3 };
+
+int pow2_ceil(int v) {
+    int p = 1;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+// Largest vectors-per-thread the register kernels are instantiated for, and the
+// largest CTA each instance is built for.
+int max_vpt(Op op) { return op == OP_LAYER ? 4 : 8; }
+int max_threads(Op op, int vpt) {
+    return op == OP_LAYER ? layer_max_threads(vpt) : rms_max_threads(vpt);
+}
+
+// Register-path shape: VPT vectors per thread, G threads per row.
+bool rows_shape(Op op, int nvec, int vpt_req, int g_req, int* vpt, int* G) {
+    int v = vpt_req;
+    if (v == 0) {
+        // smallest VPT whose row group fits in 256 threads, else in 1024
+        v = 0;
+        for (int c = 1; c <= max_vpt(op); c *= 2)
+            if ((nvec + c - 1) / c <= 256) { v = c; break; }
+        if (v == 0)
+            for (int c = 1; c <= max_vpt(op); c *= 2)
+                if ((nvec + c - 1) / c <= max_threads(op, c)) { v = c; break; }
+        if (v == 0) return false;
+    }
+    if (v != 1 && v != 2 && v != 4 && v != 8) return false;
+    if (v > max_vpt(op)) return false;
+    int g = g_req;
+    if (g == 0) g = ((nvec + v - 1) / v + 31) / 32 * 32;
+    if (g % 32 != 0 || g < 32 || g > max_threads(op, v)) return false;
+    if ((int64_t)g * v < nvec) return false;
+    *vpt = v;
+    *G = g;
+    return true;
+}
+
+nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, const nv_plan* req,
+                    nv_plan* out) {
+    nv_plan p{};
+    if (req) p = *req;
+    const int vecw = 16 / (int)elem_size(dt);
+    const bool vec_ok = aligned && D % vecw == 0 && D / vecw <= 8192;
+    const int nvec = vec_ok ? (int)(D / vecw) : 0;
+    if (p.path == NV_PATH_AUTO) p.path = vec_ok ? NV_PATH_ROWS : NV_PATH_GENERIC;
+    if (p.path == NV_PATH_ROWS) {
+        if (!vec_ok) return fail(NV_ERR_UNSUPPORTED, "register path needs D %% %d == 0 and "
+                                 "16-byte aligned pointers", vecw);
+        int vpt = 0, G = 0;
+        if (!rows_shape(op, nvec, p.vec_per_thread, p.threads_per_row, &vpt, &G))
+            return fail(NV_ERR_UNSUPPORTED, "no register-path shape for D = %lld (vpt %d, G %d)",
+                        (long long)D, p.vec_per_thread, p.threads_per_row);
+        p.vec_per_thread = vpt;
+        p.threads_per_row = G;
+        if (p.rows_per_cta == 0) p.rows_per_cta = std::max(1, std::min(256, max_threads(op, vpt)) / G);
+        if (p.rows_per_cta * G > max_threads(op, vpt) || p.rows_per_cta < 1)
+            return fail(NV_ERR_UNSUPPORTED, "rows_per_cta %d x G %d", p.rows_per_cta, G);
+    } else if (p.path == NV_PATH_GENERIC) {
+        p.vec_per_thread = 0;
+        p.threads_per_row = 256;
+        p.rows_per_cta = 1;
+    } else {
+        return fail(NV_ERR_UNSUPPORTED, "path %d is not available for this op", p.path);
+    }
+    if (p.ctas_per_sm < 0) return fail(NV_ERR_INVALID_ARG, "ctas_per_sm < 0");
+    (void)rows;
+    *out = p;
+    return NV_OK;
+}
+
+// ---- launching -----------------------------------------------------------------------------
+template <typename K>
+int occupancy(K kernel, int block, size_t smem) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, block, smem) != cudaSuccess) {
+        cudaGetLastError();
+        n = 1;
+    }
+    return std::max(n, 1);
+}
+
+int64_t grid_for(int64_t units, int sms, int per_sm) {
+    return std::max<int64_t>(1, std::min<int64_t>(units, (int64_t)sms * per_sm));
+}
+
+template <typename K>
+nv_status launch(K kernel, int64_t units, int block, size_t smem, int ctas_per_sm,
+                 const DevInfo& di, cudaStream_t s, const RowArgs& a) {
+    const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : occupancy(kernel, block, smem);
+    const int64_t grid = grid_for(units, di.sms, per_sm);
+    kernel<<<(unsigned)grid, block, smem, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return NV_OK;
+}
+
+template <typename T, bool ADD>
+nv_status run_rms(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs a) {
+    if (p.path == NV_PATH_GENERIC)
+        return launch(rms_generic_kernel<T, ADD>, a.rows, 256, 0, p.ctas_per_sm, di, s, a);
+    a.G = p.threads_per_row;
+    a.rows_per_cta = p.rows_per_cta;
+    const int block = a.G * a.rows_per_cta;
+    const int64_t units = (a.rows + a.rows_per_cta - 1) / a.rows_per_cta;
+    switch (p.vec_per_thread) {
+        case 1: return launch(rms_rows_kernel<T, 1, ADD>, units, block, 0, p.ctas_per_sm, di, s, a);
+        case 2: return launch(rms_rows_kernel<T, 2, ADD>, units, block, 0, p.ctas_per_sm, di, s, a);
+        case 4: return launch(rms_rows_kernel<T, 4, ADD>, units, block, 0, p.ctas_per_sm, di, s, a);
+        case 8: return launch(rms_rows_kernel<T, 8, ADD>, units, block, 0, p.ctas_per_sm, di, s, a);
+    }
+    return fail(NV_ERR_UNSUPPORTED, "vec_per_thread %d", p.vec_per_thread);
+}
+
+template <typename T>
+nv_status run_layer(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs a) {
+    if (p.path == NV_PATH_GENERIC)
+        return launch(layer_generic_kernel<T>, a.rows, 256, 0, p.ctas_per_sm, di, s, a);
+    a.G = p.threads_per_row;
+    a.rows_per_cta = p.rows_per_cta;
+    const int block = a.G * a.rows_per_cta;
+    const int64_t units = (a.rows + a.rows_per_cta - 1) / a.rows_per_cta;
+    switch (p.vec_per_thread) {
+        case 1: return launch(layer_rows_kernel<T, 1>, units, block, 0, p.ctas_per_sm, di, s, a);
+        case 2: return launch(layer_rows_kernel<T, 2>, units, block, 0, p.ctas_per_sm, di, s, a);
+        case 4: return launch(layer_rows_kernel<T, 4>, units, block, 0, p.ctas_per_sm, di, s, a);
+    }
+    return fail(NV_ERR_UNSUPPORTED, "vec_per_thread %d", p.vec_per_thread);
+}
+
+nv_status row_op(Op op, const void* x, const void* r, const void* w, const void* b, void* y,
+                 void* h, int64_t rows, int64_t D, float eps, nv_dtype dt, nv_stream_t stream,
+                 const nv_plan* req) {
+    nv_status st = check_common(rows, D, eps, dt);
+    if (st != NV_OK) return st;
+    if (rows == 0) return NV_OK;
+    const size_t s = elem_size(dt);
+    const size_t nbytes = (size_t)rows * (size_t)D * s;
+    const size_t pbytes = (size_t)D * s;
+    if (!x) return fail(NV_ERR_INVALID_ARG, "x is NULL");
+    if (!y) return fail(NV_ERR_INVALID_ARG, "y is NULL");
+    if (op == OP_ADD && !r) return fail(NV_ERR_INVALID_ARG, "r is NULL");
+    if (op == OP_ADD && !h) return fail(NV_ERR_INVALID_ARG, "h is NULL");
+    if (op == OP_ADD && y == h) return fail(NV_ERR_INVALID_ARG, "y and h are the same buffer");
+
+    int dev = 0;
+    DevInfo di;
+    st = current_device(&dev, &di);
+    if (st != NV_OK) return st;
+    const Buf bufs[] = {
+        {x, nbytes, "x", false, true},
+        {op == OP_ADD ? r : nullptr, nbytes, "r", false, true},
+        {w, pbytes, "w", false, false},
+        {op == OP_LAYER ? b : nullptr, pbytes, "b", false, false},
+        {y, nbytes, "y", true, false},
+        {op == OP_ADD ? h : nullptr, nbytes, "h", true, false},
+    };
+    st = check_buffers(bufs, 6, dev);
+    if (st != NV_OK) return st;
+
+    bool al = aligned16(x) && aligned16(y) && (!w || aligned16(w));
+    if (op == OP_ADD) al = al && aligned16(r) && aligned16(h);
+    if (op == OP_LAYER) al = al && (!b || aligned16(b));
+    nv_plan p;
+    st = make_plan(op, rows, D, dt, al, req, &p);
+    if (st != NV_OK) return st;
+
+    RowArgs a{};
+    a.x = x;
+    a.r = r;
+    a.w = w;
+    a.b = b;
+    a.y = y;
+    a.h = h;
+    a.rows = rows;
+    a.D = (int)D;
+    a.nvec = (int)(D * (int64_t)s / 16);
+    a.eps = eps;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf = dt == NV_BF16;
+    switch (op) {
+        case OP_RMS:
+            return bf ? run_rms<__nv_bfloat16, false>(p, di, cs, a) : run_rms<float, false>(p, di, cs, a);
+        case OP_ADD:
+            return bf ? run_rms<__nv_bfloat16, true>(p, di, cs, a) : run_rms<float, true>(p, di, cs, a);
+        case OP_LAYER:
+            return bf ? run_layer<__nv_bfloat16>(p, di, cs, a) : run_layer<float>(p, di, cs, a);
+        default:
+            return fail(NV_ERR_INVALID_ARG, "op %d", (int)op);
+    }
+}
+
+// ---- norm_rope -------------------------------------------------------------------------------
+struct RopePlan {
+    bool rows;
+    int lpr;
+    int bt;
+    int64_t n_chunks;
+};
+
+template <typename T, bool TRAD>
+nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a) {
+    const size_t smem = (size_t)a.half * sizeof(float4);
+    auto kern = rope_rows_kernel<T, TRAD>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    }
+    const int64_t grid = a.L * a.n_chunks;
+    kern<<<(unsigned)grid, 256, smem, s>>>(a);
+    (void)di;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return NV_OK;
+}
+
+template <typename T>
+nv_status launch_rope_generic(const DevInfo& di, int ctas_per_sm, cudaStream_t s,
+                              const RopeArgs& a) {
+    auto kern = rope_generic_kernel<T>;
+    const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : occupancy(kern, 128, 0);
+    const int64_t grid = grid_for(a.BH * a.L, di.sms, per_sm);
+    kern<<<(unsigned)grid, 128, 0, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return NV_OK;
+}
+
+nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_dtype dt,
+                    bool aligned, int sms, const nv_plan* req, nv_plan* out, RopePlan* rp) {
+    nv_plan p{};
+    if (req) p = *req;
+    const int vecw = 16 / (int)elem_size(dt);
+    const int64_t nvec = D / vecw;
+    const bool vec_ok = aligned && D % vecw == 0 && nvec <= 32 &&
+                        (trad || (dims / 2) % vecw == 0);
+    if (p.path == NV_PATH_AUTO) p.path = vec_ok ? NV_PATH_ROWS : NV_PATH_GENERIC;
+    rp->rows = p.path == NV_PATH_ROWS;
+    if (p.path == NV_PATH_ROWS) {
+        if (!vec_ok)
+            return fail(NV_ERR_UNSUPPORTED, "norm_rope register path needs D %% %d == 0, "
+                        "D <= %d, 16-byte alignment and (halves) dims/2 %% %d == 0",
+                        vecw, 32 * vecw, vecw);
+        const int lpr = pow2_ceil((int)std::max<int64_t>(nvec, 1));
+        const int slots = 256 / lpr;
+        const int64_t BH = rows / L;
+        int64_t bt = p.rows_per_cta;
+        if (bt <= 0) {
+            const int64_t target = (rows + 8LL * sms - 1) / (8LL * sms);
+            bt = std::max<int64_t>(slots * 4, std::min<int64_t>(target, 256));
+            bt = std::min<int64_t>(bt, std::max<int64_t>(BH, 1));
+        }
+        rp->lpr = lpr;
+        rp->bt = (int)bt;
+        rp->n_chunks = (BH + bt - 1) / bt;
+        if (L * rp->n_chunks >= ((int64_t)1 << 31))
+            return fail(NV_ERR_UNSUPPORTED, "norm_rope grid too large");
+        p.vec_per_thread = 1;
+        p.threads_per_row = lpr;
+        p.rows_per_cta = (int)bt;
+    } else if (p.path == NV_PATH_GENERIC) {
+        p.vec_per_thread = 0;
+        p.threads_per_row = 128;
+        p.rows_per_cta = 1;
+    } else {
+        return fail(NV_ERR_UNSUPPORTED, "path %d is not available for norm_rope", p.path);
+    }
+    *out = p;
+    return NV_OK;
+}
+
+nv_status rope_op(const void* x, const void* w, void* y, int64_t rows, int64_t L, int64_t D,
+                  int32_t dims, int32_t traditional, float base, float scale, int64_t offset,
+                  int32_t normalize, float eps, nv_dtype dt, nv_stream_t stream,
+                  const nv_plan* req) {
+    nv_status st = check_common(rows, D, eps, dt, normalize != 0);
+    if (st != NV_OK) return st;
+    if (L < 1) return fail(NV_ERR_INVALID_ARG, "L = %lld < 1", (long long)L);
+    if (rows % L != 0)
+        return fail(NV_ERR_INVALID_ARG, "rows = %lld is not a multiple of L = %lld",
+                    (long long)rows, (long long)L);
+    if (dims <= 0 || dims % 2 != 0 || dims > D)
+        return fail(NV_ERR_INVALID_ARG, "dims = %d must be even with 0 < dims <= D = %lld", dims,
+                    (long long)D);
+    if (!(base > 0.f) || !std::isfinite(base))
+        return fail(NV_ERR_INVALID_ARG, "base = %g must be finite and > 0", (double)base);
+    if (!std::isfinite(scale)) return fail(NV_ERR_INVALID_ARG, "scale must be finite");
+    if (offset < 0) return fail(NV_ERR_INVALID_ARG, "offset = %lld < 0", (long long)offset);
+    if (offset > ((int64_t)1 << 52) - L)
+        return fail(NV_ERR_INVALID_ARG, "offset + L must stay below 2^52");
+    if (rows == 0) return NV_OK;
+    if (!x) return fail(NV_ERR_INVALID_ARG, "x is NULL");
+    if (!y) return fail(NV_ERR_INVALID_ARG, "y is NULL");
+
+    int dev = 0;
+    DevInfo di;
+    st = current_device(&dev, &di);
+    if (st != NV_OK) return st;
+    const size_t s = elem_size(dt);
+    const size_t nbytes = (size_t)rows * (size_t)D * s;
+    const Buf bufs[] = {
+        {x, nbytes, "x", false, true},
+        {normalize ? w : nullptr, (size_t)D * s, "w", false, false},
+        {y, nbytes, "y", true, false},
+    };
+    st = check_buffers(bufs, 3, dev);
+    if (st != NV_OK) return st;
+
+    const bool al = aligned16(x) && aligned16(y) && (!w || !normalize || aligned16(w));
+    nv_plan p;
+    RopePlan rp{};
+    st = rope_plan(rows, L, D, dims, traditional != 0, dt, al, di.sms, req, &p, &rp);
+    if (st != NV_OK) return st;
+
+    RopeArgs a{};
+    a.x = x;
+    a.w = normalize ? w : nullptr;
+    a.y = y;
+    a.BH = rows / L;
+    a.L = L;
+    a.offset = offset;
+    a.n_chunks = rp.n_chunks;
+    a.D = (int)D;
+    a.nvec = (int)(D * (int64_t)s / 16);
+    a.dims = dims;
+    a.half = dims / 2;
+    a.lpr = rp.lpr;
+    a.bt = rp.bt;
+    a.base = base;
+    a.scale = scale;
+    a.eps = eps;
+    a.normalize = normalize != 0;
+    a.traditional = traditional != 0;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf = dt == NV_BF16;
+    if (rp.rows) {
+        if (traditional)
+            return bf ? launch_rope_rows<__nv_bfloat16, true>(di, cs, a)
+                      : launch_rope_rows<float, true>(di, cs, a);
+        return bf ? launch_rope_rows<__nv_bfloat16, false>(di, cs, a)
+                  : launch_rope_rows<float, false>(di, cs, a);
+    }
+    return bf ? launch_rope_generic<__nv_bfloat16>(di, p.ctas_per_sm, cs, a)
+              : launch_rope_generic<float>(di, p.ctas_per_sm, cs, a);
+}
+
+}  // namespace
+
+// ---- exported C ABI -------------------------------------------------------------------------
+extern "C" {
+
+nv_status nv_rms_norm_ex(const void* x, const void* w, void* y, int64_t rows, int64_t D,
+                         float eps, nv_dtype dt, nv_stream_t stream, const nv_plan* plan) {
+    return row_op(OP_RMS, x, nullptr, w, nullptr, y, nullptr, rows, D, eps, dt, stream, plan);
+}
+
+nv_status nv_rms_norm(const void* x, const void* w, void* y, int64_t rows, int64_t D, float eps,
+                      nv_dtype dt, nv_stream_t stream) {
+    return nv_rms_norm_ex(x, w, y, rows, D, eps, dt, stream, nullptr);
+}
+
+nv_status nv_add_rms_norm_ex(const void* x, const void* r, const void* w, void* y, void* h,
+                             int64_t rows, int64_t D, float eps, nv_dtype dt, nv_stream_t stream,
+                             const nv_plan* plan) {
+    return row_op(OP_ADD, x, r, w, nullptr, y, h, rows, D, eps, dt, stream, plan);
+}
+
+nv_status nv_add_rms_norm(const void* x, const void* r, const void* w, void* y, void* h,
+                          int64_t rows, int64_t D, float eps, nv_dtype dt, nv_stream_t stream) {
+    return nv_add_rms_norm_ex(x, r, w, y, h, rows, D, eps, dt, stream, nullptr);
+}
+
+nv_status nv_layer_norm_ex(const void* x, const void* w, const void* b, void* y, int64_t rows,
+                           int64_t D, float eps, nv_dtype dt, nv_stream_t stream,
+                           const nv_plan* plan) {
+    return row_op(OP_LAYER, x, nullptr, w, b, y, nullptr, rows, D, eps, dt, stream, plan);
+}
+
+nv_status nv_layer_norm(const void* x, const void* w, const void* b, void* y, int64_t rows,
+                        int64_t D, float eps, nv_dtype dt, nv_stream_t stream) {
+    return nv_layer_norm_ex(x, w, b, y, rows, D, eps, dt, stream, nullptr);
+}
+
+nv_status nv_norm_rope_ex(const void* x, const void* w, void* y, int64_t rows, int64_t L,
+                          int64_t D, int32_t dims, int32_t traditional, float base, float scale,
+                          int64_t offset, int32_t normalize, float eps, nv_dtype dt,
+                          nv_stream_t stream, const nv_plan* plan) {
+    return rope_op(x, w, y, rows, L, D, dims, traditional, base, scale, offset, normalize, eps,
+                   dt, stream, plan);
+}
+
+nv_status nv_norm_rope(const void* x, const void* w, void* y, int64_t rows, int64_t L, int64_t D,
+                       int32_t dims, int32_t traditional, float base, float scale, int64_t offset,
+                       int32_t normalize, float eps, nv_dtype dt, nv_stream_t stream) {
+    return nv_norm_rope_ex(x, w, y, rows, L, D, dims, traditional, base, scale, offset, normalize,
+                           eps, dt, stream, nullptr);
+}
+
+nv_status nv_describe_plan(int32_t op, int64_t rows, int64_t D, nv_dtype dt, nv_plan* plan) {
+    if (!plan) return fail(NV_ERR_INVALID_ARG, "plan is NULL");
+    nv_status st = check_common(rows, D, 0.f, dt);
+    if (st != NV_OK) return st;
+    if (op < 0 || op > 3) return fail(NV_ERR_INVALID_ARG, "op %d", op);
+    if (op == OP_ROPE) {
+        RopePlan rp{};
+        // position count unknown here: describe one position holding every row
+        return rope_plan(rows, 1, D, (int)(D - D % 2), false, dt, true, 148, nullptr, plan, &rp);
+    }
+    return make_plan((Op)op, rows, D, dt, true, nullptr, plan);
+}
+
+const char* nv_status_string(nv_status status) {
+    switch (status) {
+        case NV_OK: return "NV_OK";
+        case NV_ERR_INVALID_ARG: return "NV_ERR_INVALID_ARG";
+        case NV_ERR_UNSUPPORTED: return "NV_ERR_UNSUPPORTED";
+        case NV_ERR_CUDA: return "NV_ERR_CUDA";
+    }
+    return "NV_STATUS_UNKNOWN";
+}
+
+const char* nv_last_error(void) { return g_msg; }
+
+int32_t nv_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,256 @@
+// rope.cuh -- norm_rope kernels (RMS normalisation followed by the rotary embedding).
+//
+// Definitions: docs.rs nuvec-core 0.5.0, Enum FastOp, variants NormRope and Rope;
+// docs.rs nuvec-nn 0.4.0 src/layers.rs, Rope (halves by default, base 10000, scale
+// applied to positions).  Row k of x [B, H, L, D] sits at l = k mod L and is rotated
+// at position offset + l: pair i turns by phi_i = (offset + l) * scale * theta_i with
+// theta_i = base^(-2 i / dims); pairs are (i, i + dims/2) or, traditional, (2i, 2i + 1).
+//
+// Precision.  A pair output y_p = inv * (a_p cos - a_q sin), a = x * w, can cancel.
+// A float32 angle (ulp(6000 rad) ~ 4.9e-4) or a float32 cos/sin (error 2^-24 |a|)
+// misses the bfloat16 result by more than one ulp whenever |y_p| is much smaller
+// than |a|.  So:
+//   - each CTA builds the cos/sin of its positions in double precision (pow, sincos)
+//     and keeps each as a float pair hi + lo (the split is exact to ~2^-48);
+//   - a = x * w is exact in float32 for bfloat16 inputs (8 x 8 significant bits);
+//   - the pair combination is evaluated with error-free products (fma), so the
+//     float32 result is accurate to ~2^-23 relative plus ~2^-46 |a| absolute;
+//   - the common factor inv = rsqrt(mean(x^2) + eps) multiplies last (a relative
+//     error, harmless).
+#pragma once
+
+#include "common.cuh"
+
+namespace nvn {
+
+struct RopeArgs {
+    const void* x;
+    const void* w;
+    void* y;
+    int64_t BH;         // rows / L
+    int64_t L;
+    int64_t offset;
+    int64_t n_chunks;   // bh chunks per position
+    int D;
+    int nvec;           // 16-byte vectors per row
+    int dims;
+    int half;           // dims / 2
+    int lpr;            // lanes per row (power of two <= 32), register path
+    int bt;             // bh rows per CTA, register path
+    float base;
+    float scale;
+    float eps;
+    int normalize;
+    int traditional;
+};
+
+// z = a_o * c + a_t * s for c = c_hi + c_lo, s = s_hi + s_lo (hi/lo float splits).
+// t1 + e1 is a_t * s_hi exactly; the remaining products are ~2^-24 |a| and their own
+// rounding is ~2^-48 |a|.
+__device__ __forceinline__ float rotate_pair(float a_o, float a_t, float c_hi, float c_lo,
+                                             float s_hi, float s_lo) {
+    const float t1 = __fmul_rn(a_t, s_hi);
+    const float e1 = __fmaf_rn(a_t, s_hi, -t1);
+    const float z1 = __fmaf_rn(a_o, c_hi, t1);
+    const float c2 = __fmaf_rn(a_t, s_lo, e1);
+    const float c3 = __fmaf_rn(a_o, c_lo, c2);
+    return __fadd_rn(z1, c3);
+}
+
+// cos and sin of (pos * scale * base^(-2 i / dims)) in double, split into float hi/lo.
+__device__ __forceinline__ float4 angle_entry(double pos, double scale, double base, int i,
+                                              int dims) {
+    const double theta = pow(base, -2.0 * (double)i / (double)dims);
+    const double phi = pos * scale * theta;
+    double s, c;
+    sincos(phi, &s, &c);
+    const float ch = __double2float_rn(c);
+    const float sh = __double2float_rn(s);
+    return make_float4(ch, __double2float_rn(c - (double)ch), sh, __double2float_rn(s - (double)sh));
+}
+
+// ---- register path ------------------------------------------------------------------
+// One CTA = one position l and a chunk of bt rows (b, h) at that position, so the
+// angle table of l is built once (dims/2 double sincos) and reused by all of them.
+// A group of lpr lanes holds one row, one 16-byte vector per lane; each slot of the
+// CTA takes rows slot, slot + slots, ...; kUnroll rows are loaded before any math.
+// Halves pairing needs (dims/2) % VEC == 0: a lane's vector is then wholly the p side,
+// wholly the q side or wholly past dims, and its partner vector sits hv = half/VEC
+// lanes away (one shuffle per word).  Traditional pairs live inside one vector.
+template <typename T, bool TRAD>
+__global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
+    using E = Elem<T>;
+    constexpr int VEC = E::kVec;
+    constexpr int kUnroll = 4;
+    extern __shared__ float4 tab[];  // [half]: (cos_hi, cos_lo, sin_hi, sin_lo)
+
+    const int64_t chunk = blockIdx.x % a.n_chunks;
+    const int64_t l = blockIdx.x / a.n_chunks;
+    const int lpr = a.lpr;
+    const int lane = threadIdx.x & (lpr - 1);  // vector index within the row
+    const int slot = threadIdx.x / lpr;
+    const int slots = blockDim.x / lpr;
+    const int v = lane;
+    const bool has_vec = v < a.nvec;
+    const int hv = a.half / VEC;  // halves: partner distance in vectors
+
+    // partner vector (halves) and the sign of sin for this lane's elements
+    int pv = v;
+    if (!TRAD) pv = (v < hv) ? v + hv : (v < 2 * hv ? v - hv : v);
+
+    // per-column weights of this lane's elements and of their partners
+    const bool norm = a.normalize != 0;
+    V16 w_own = (norm && a.w && has_vec) ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16)
+                                         : ones_vec<T>();
+    V16 w_par = w_own;
+    if (!TRAD && pv != v && norm && a.w && pv < a.nvec)
+        w_par = ld_param(static_cast<const char*>(a.w) + (size_t)pv * 16);
+
+    // first rows' loads go out before the table is built
+    const int64_t bh0 = chunk * (int64_t)a.bt;
+    const int64_t bh_end = min(bh0 + (int64_t)a.bt, a.BH);
+    const size_t row_bytes = (size_t)a.D * sizeof(T);
+    const size_t lstride = (size_t)a.L * row_bytes;  // between consecutive bh at fixed l
+    const char* xbase = static_cast<const char*>(a.x) + (size_t)l * row_bytes + (size_t)v * 16;
+    char* ybase = static_cast<char*>(a.y) + (size_t)l * row_bytes + (size_t)v * 16;
+
+    // Every thread runs the same trip count (rows past bh_end are predicated off):
+    // the shuffles below involve the whole warp, which may hold several rows.
+    V16 xv[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t b = bh0 + slot + (int64_t)u * slots;
+        if (has_vec && b < bh_end) xv[u] = ld_stream(xbase + (size_t)b * lstride);
+    }
+
+    const double pos = (double)(a.offset + l);
+    for (int i = threadIdx.x; i < a.half; i += blockDim.x)
+        tab[i] = angle_entry(pos, (double)a.scale, (double)a.base, i, a.dims);
+    __syncthreads();
+
+    // this lane's table entries, sin already carrying the sign of its side
+    float c_hi[VEC], c_lo[VEC], s_hi[VEC], s_lo[VEC];
+    bool rot[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        const int j = v * VEC + e;
+        rot[e] = has_vec && j < a.dims;
+        int i = 0;
+        float sg = 1.f;
+        if (TRAD) {
+            i = j >> 1;
+            sg = (j & 1) ? 1.f : -1.f;
+        } else {
+            i = (j < a.half) ? j : j - a.half;
+            sg = (j < a.half) ? -1.f : 1.f;
+        }
+        const float4 t4 = rot[e] ? tab[i] : make_float4(1.f, 0.f, 0.f, 0.f);
+        c_hi[e] = t4.x;
+        c_lo[e] = t4.y;
+        s_hi[e] = sg * t4.z;
+        s_lo[e] = sg * t4.w;
+    }
+
+    const float Df = (float)a.D;
+    for (int64_t base = bh0; base < bh_end; base += (int64_t)kUnroll * slots) {
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t b = base + slot + (int64_t)u * slots;
+            const bool live = has_vec && b < bh_end;
+            V16 xo = live ? xv[u] : zeros_vec<T>();
+            // the next round's load for this unroll slot goes out now
+            const int64_t bn = b + (int64_t)kUnroll * slots;
+            if (has_vec && bn < bh_end) xv[u] = ld_stream(xbase + (size_t)bn * lstride);
+
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                const float f = E::get(xo, e);
+                ss = fmaf(f, f, ss);
+            }
+            ss = group_sum(ss, lpr);
+            const float inv = norm ? rsqrtf(__fdiv_rn(ss, Df) + a.eps) : 1.f;
+
+            V16 xp = xo;  // partner words
+            if (!TRAD) {
+                const int src = pv & (lpr - 1);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) xp.u[q] = __shfl_sync(0xFFFFFFFFu, xo.u[q], src, lpr);
+            }
+            if (live) {
+                V16 o;
+#pragma unroll
+                for (int e = 0; e < VEC; e += 2) {
+                    float yy[2];
+#pragma unroll
+                    for (int d = 0; d < 2; ++d) {
+                        const int ee = e + d;
+                        const float a_o = __fmul_rn(E::get(xo, ee), E::get(w_own, ee));
+                        float z = a_o;
+                        if (rot[ee]) {
+                            const int te = TRAD ? (ee ^ 1) : ee;
+                            const float a_t = TRAD ? __fmul_rn(E::get(xo, te), E::get(w_own, te))
+                                                   : __fmul_rn(E::get(xp, te), E::get(w_par, te));
+                            z = rotate_pair(a_o, a_t, c_hi[ee], c_lo[ee], s_hi[ee], s_lo[ee]);
+                        }
+                        yy[d] = __fmul_rn(z, inv);
+                    }
+                    E::put2(o, e, yy[0], yy[1]);
+                }
+                st_stream(ybase + (size_t)b * lstride, o);
+            }
+        }
+    }
+}
+
+// ---- generic path ---------------------------------------------------------------------
+// Any D, dims and alignment: one CTA per row.  Pass 1: sum of squares.  Pass 2: each
+// thread takes whole pairs (reads both members, then writes both, so y may be x) with
+// its angle computed in double, then the features past dims.
+template <typename T>
+__global__ void __launch_bounds__(128) rope_generic_kernel(const RopeArgs a) {
+    using E = Elem<T>;
+    __shared__ float red[2][32];
+    const int nw = blockDim.x >> 5;
+    const bool norm = a.normalize != 0;
+    const int64_t rows = a.BH * a.L;
+    int it = 0;
+    for (int64_t row = blockIdx.x; row < rows; row += gridDim.x, ++it) {
+        const int64_t r0 = row * (int64_t)a.D;
+        float inv = 1.f;
+        if (norm) {
+            float ss = 0.f;
+            for (int j = threadIdx.x; j < a.D; j += blockDim.x) {
+                const float f = E::load1(a.x, r0 + j);
+                ss = fmaf(f, f, ss);
+            }
+            ss = warp_sum(ss);
+            float* buf = red[it & 1];
+            if ((threadIdx.x & 31) == 0) buf[threadIdx.x >> 5] = ss;
+            __syncthreads();
+            ss = 0.f;
+            for (int i = 0; i < nw; ++i) ss += buf[i];
+            inv = rsqrtf(__fdiv_rn(ss, (float)a.D) + a.eps);
+        }
+        const double pos = (double)(a.offset + row % a.L);
+        for (int i = threadIdx.x; i < a.half; i += blockDim.x) {
+            const int p = a.traditional ? 2 * i : i;
+            const int q = a.traditional ? 2 * i + 1 : i + a.half;
+            const float wp = (norm && a.w) ? E::load1(a.w, p) : 1.f;
+            const float wq = (norm && a.w) ? E::load1(a.w, q) : 1.f;
+            const float ap = __fmul_rn(E::load1(a.x, r0 + p), wp);
+            const float aq = __fmul_rn(E::load1(a.x, r0 + q), wq);
+            const float4 t = angle_entry(pos, (double)a.scale, (double)a.base, i, a.dims);
+            const float yp = rotate_pair(ap, aq, t.x, t.y, -t.z, -t.w);
+            const float yq = rotate_pair(aq, ap, t.x, t.y, t.z, t.w);
+            E::store1(a.y, r0 + p, __fmul_rn(yp, inv));
+            E::store1(a.y, r0 + q, __fmul_rn(yq, inv));
+        }
+        for (int j = a.dims + threadIdx.x; j < a.D; j += blockDim.x) {
+            const float wj = (norm && a.w) ? E::load1(a.w, j) : 1.f;
+            E::store1(a.y, r0 + j, __fmul_rn(__fmul_rn(E::load1(a.x, r0 + j), wj), inv));
+        }
+    }
+}
+
+}  // namespace nvn

@@ -1,0 +1,146 @@
+"""The C ABI on a machine without a GPU: symbols, status strings, host-side validation.
+
+Every call here fails (or returns NV_OK for rows == 0) before the library touches the
+CUDA runtime, so nothing is launched.
+"""
+import ctypes
+import math
+import os
+import re
+import subprocess
+
+import pytest
+
+import rope_add_rms_b200 as nv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvnorm.h")
+
+OK, INVALID, UNSUPPORTED = nv.NV_OK, nv.NV_ERR_INVALID_ARG, nv.NV_ERR_UNSUPPORTED
+BF16, F32, F16 = nv.NV_BF16, nv.NV_F32, nv.NV_F16
+FAKE = ctypes.c_void_p(0x10000)     # never dereferenced: validation stops first
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*NV_API\s+(?:const\s+)?\w+\*?\s+(nv_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for fn in ("nv_rms_norm", "nv_add_rms_norm", "nv_layer_norm", "nv_norm_rope",
+               "nv_status_string", "nv_last_error"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", nv.library_path], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    lib = nv.library()
+    for f in declared_functions():
+        getattr(lib, f)
+    # nothing else leaks out of the library (hidden visibility)
+    ours = {s for s in exported if s.startswith("nv_")}
+    assert ours == set(declared_functions())
+
+
+def test_status_strings_and_version():
+    lib = nv.library()
+    assert lib.nv_status_string(0) == b"NV_OK"
+    assert lib.nv_status_string(1) == b"NV_ERR_INVALID_ARG"
+    assert lib.nv_status_string(2) == b"NV_ERR_UNSUPPORTED"
+    assert lib.nv_status_string(3) == b"NV_ERR_CUDA"
+    assert lib.nv_status_string(99) == b"NV_STATUS_UNKNOWN"
+    assert lib.nv_version() >= 100
+
+
+def rms(x=FAKE, w=None, y=FAKE, rows=4, D=8, eps=1e-5, dt=BF16):
+    return nv.library().nv_rms_norm(x, w, y, rows, D, eps, dt, None)
+
+
+def add(x=FAKE, r=FAKE, w=None, y=FAKE, h=ctypes.c_void_p(0x20000), rows=4, D=8, eps=1e-5,
+        dt=BF16):
+    return nv.library().nv_add_rms_norm(x, r, w, y, h, rows, D, eps, dt, None)
+
+
+def layer(x=FAKE, w=None, b=None, y=FAKE, rows=4, D=8, eps=1e-5, dt=BF16):
+    return nv.library().nv_layer_norm(x, w, b, y, rows, D, eps, dt, None)
+
+
+def rope(x=FAKE, w=None, y=FAKE, rows=8, L=4, D=8, dims=8, trad=0, base=10000.0, scale=1.0,
+         offset=0, normalize=1, eps=1e-6, dt=BF16):
+    return nv.library().nv_norm_rope(x, w, y, rows, L, D, dims, trad, base, scale, offset,
+                                     normalize, eps, dt, None)
+
+
+def last_error():
+    return nv.library().nv_last_error().decode()
+
+
+@pytest.mark.parametrize("call, status, words", [
+    (lambda: rms(dt=7), INVALID, "dtype"),
+    (lambda: rms(dt=F16), UNSUPPORTED, "F16"),
+    (lambda: rms(rows=-1), INVALID, "rows"),
+    (lambda: rms(D=0), INVALID, "D"),
+    (lambda: rms(eps=-1e-5), INVALID, "eps"),
+    (lambda: rms(eps=math.nan), INVALID, "eps"),
+    (lambda: rms(eps=math.inf), INVALID, "eps"),
+    (lambda: rms(x=None), INVALID, "x is NULL"),
+    (lambda: rms(y=None), INVALID, "y is NULL"),
+    (lambda: rms(rows=2 ** 62, D=2 ** 20), INVALID, "overflows"),
+    (lambda: add(r=None), INVALID, "r is NULL"),
+    (lambda: add(h=None), INVALID, "h is NULL"),
+    (lambda: add(h=FAKE), INVALID, "same buffer"),
+    (lambda: layer(D=-3), INVALID, "D"),
+    (lambda: layer(eps=-0.5, dt=F32), INVALID, "eps"),
+    (lambda: rope(L=0), INVALID, "L"),
+    (lambda: rope(rows=9, L=4), INVALID, "multiple of L"),
+    (lambda: rope(dims=7), INVALID, "dims"),
+    (lambda: rope(dims=0), INVALID, "dims"),
+    (lambda: rope(dims=10, D=8), INVALID, "dims"),
+    (lambda: rope(base=0.0), INVALID, "base"),
+    (lambda: rope(base=-2.0), INVALID, "base"),
+    (lambda: rope(base=math.inf), INVALID, "base"),
+    (lambda: rope(scale=math.nan), INVALID, "scale"),
+    (lambda: rope(offset=-1), INVALID, "offset"),
+    (lambda: rope(eps=-1.0), INVALID, "eps"),
+    (lambda: rope(x=None), INVALID, "x is NULL"),
+])
+def test_invalid_arguments_are_rejected_on_the_host(call, status, words):
+    assert call() == status
+    assert words in last_error()
+
+
+def test_zero_rows_is_a_no_op():
+    assert rms(x=None, y=None, rows=0) == OK
+    assert add(x=None, r=None, y=None, h=None, rows=0) == OK
+    assert layer(x=None, y=None, rows=0) == OK
+    assert rope(x=None, y=None, rows=0) == OK
+
+
+def test_plain_rope_ignores_eps():
+    # normalize == 0: eps is unused, so a negative eps is not an error (stops at x NULL)
+    assert rope(normalize=0, eps=-1.0, x=None) == INVALID
+    assert "x is NULL" in last_error()
+
+
+@pytest.mark.parametrize("op, D, dtype, want", [
+    ("add_rms_norm", 4096, "bf16", dict(path=1, vec_per_thread=2, threads_per_row=256)),
+    ("add_rms_norm", 5120, "bf16", dict(path=1, vec_per_thread=4, threads_per_row=160)),
+    ("add_rms_norm", 16384, "f32", dict(path=1, vec_per_thread=8, threads_per_row=512)),
+    ("add_rms_norm", 7, "bf16", dict(path=2)),
+    ("add_rms_norm", 2 ** 17, "bf16", dict(path=2)),
+    ("rms_norm", 512, "f32", dict(path=1, vec_per_thread=1, threads_per_row=128)),
+    ("layer_norm", 8192, "bf16", dict(path=1, vec_per_thread=4, threads_per_row=256)),
+    ("norm_rope", 128, "bf16", dict(path=1, vec_per_thread=1, threads_per_row=16)),
+    ("norm_rope", 1000, "bf16", dict(path=2)),
+])
+def test_plan_selection(op, D, dtype, want):
+    import torch
+    p = nv.nv_describe_plan(op, 8192, D, {"bf16": torch.bfloat16, "f32": torch.float32}[dtype])
+    for k, v in want.items():
+        assert p[k] == v, (op, D, dtype, p)

@@ -1,0 +1,308 @@
+"""GPU parity: every op and kernel variant of libnvnorm.so against the CPU oracle.
+
+Inputs come from rope_add_rms_b200.synth (seeded, rounded to the I/O type on the host);
+the same bytes go to the device and to the oracle.  Tolerances are those of
+tests/checks.py: h bit-exact, bfloat16 y within one bfloat16 step of the oracle
+rounded to bfloat16, float32 y within 1e-5 (1 + |ref|).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rope_add_rms_b200 as nv
+from rope_add_rms_b200 import synth
+from checks import Guarded, check_exact, check_out, to_host_bits
+
+pytestmark = pytest.mark.gpu
+
+DT = {"bf16": torch.bfloat16, "f32": torch.float32}
+
+
+def dev(t):
+    return None if t is None else t.cuda()
+
+
+def host(t):
+    return None if t is None else synth.to_numpy(t)
+
+
+def run_add(inp, eps, plan=None, guard=True):
+    x, r, w = dev(inp["x"]), dev(inp["r"]), dev(inp["w"])
+    if guard:
+        gy, gh = Guarded(x.shape, x.dtype), Guarded(x.shape, x.dtype)
+        y, h = gy.t, gh.t
+    else:
+        y, h = torch.empty_like(x), torch.empty_like(x)
+    nv.nv_add_rms_norm(x, r, w, y, h, eps, plan=plan)
+    torch.cuda.synchronize()
+    if guard:
+        assert gy.bands_intact() and gh.bands_intact(), "kernel wrote outside y or h"
+    return y, h
+
+
+# ---- add_rms_norm / rms_norm ---------------------------------------------------------------
+
+ADD_SHAPES = [(147, 4096), (149, 5120), (33, 2048), (7, 16384), (1, 8192), (300, 1000),
+              (64, 512), (3, 8), (256, 64), (5, 20000), (2, 32768)]
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,D", ADD_SHAPES)
+def test_add_rms_norm(rows, D, dt):
+    inp = synth.add_rms_inputs(rows, D, dt, seed=rows + D)
+    eps = 1e-6
+    y, h = run_add(inp, eps)
+    ref, href = oracle.add_rms_norm(host(inp["x"]), host(inp["r"]), host(inp["w"]), eps)
+    check_exact(h, href, "h")
+    check_out(y, ref)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,D", [(17, 7), (3, 127), (2, 129), (9, 1), (5, 33), (4, 1001)])
+def test_add_rms_norm_ragged_D_takes_generic_path(rows, D, dt):
+    inp = synth.add_rms_inputs(rows, D, dt, seed=D)
+    y, h = run_add(inp, 1e-5)
+    ref, href = oracle.add_rms_norm(host(inp["x"]), host(inp["r"]), host(inp["w"]), 1e-5)
+    check_exact(h, href, "h")
+    check_out(y, ref)
+
+
+VARIANTS = [dict(path=nv.PATH_GENERIC)] + [
+    dict(path=nv.PATH_ROWS, vec_per_thread=v) for v in (1, 2, 4, 8)] + [
+    dict(path=nv.PATH_ROWS, vec_per_thread=2, rows_per_cta=4, threads_per_row=256),
+    dict(path=nv.PATH_ROWS, vec_per_thread=1, threads_per_row=1024),
+    dict(path=nv.PATH_ROWS, vec_per_thread=2, ctas_per_sm=1),
+    dict(path=nv.PATH_ROWS, vec_per_thread=8, threads_per_row=64, rows_per_cta=8),
+]
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("plan", VARIANTS, ids=lambda p: "-".join(f"{k}{v}" for k, v in p.items()))
+def test_add_rms_norm_every_variant(plan, dt):
+    rows, D = 301, 4096
+    inp = synth.add_rms_inputs(rows, D, dt, seed=11)
+    y, h = run_add(inp, 1e-5, plan=nv.Plan(**plan))
+    ref, href = oracle.add_rms_norm(host(inp["x"]), host(inp["r"]), host(inp["w"]), 1e-5)
+    check_exact(h, href, "h")
+    check_out(y, ref)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,D,weight", [(64, 512, True), (129, 4096, False), (10, 7, True),
+                                           (31, 16384, True)])
+def test_rms_norm(rows, D, weight, dt):
+    inp = synth.rms_inputs(rows, D, dt, seed=3, weight=weight)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    g = Guarded(x.shape, x.dtype)
+    nv.nv_rms_norm(x, w, g.t, 1e-6)
+    torch.cuda.synchronize()
+    assert g.bands_intact()
+    check_out(g.t, oracle.rms_norm(host(inp["x"]), host(inp["w"]), 1e-6))
+
+
+def test_rms_norm_small_config_fp32():
+    """rms_norm fp32 x [64, 512] ~ N(0,1), w ~ U(0.5,1.5), eps 1e-6, seed 0 (full compare)."""
+    inp = synth.rms_inputs(64, 512, "f32", seed=0)
+    y = nv.rms_norm(dev(inp["x"]), dev(inp["w"]), eps=1e-6)
+    torch.cuda.synchronize()
+    check_out(y, oracle.rms_norm(host(inp["x"]), host(inp["w"]), 1e-6))
+
+
+def test_add_rms_norm_equals_rms_norm_of_h():
+    inp = synth.add_rms_inputs(97, 4096, "bf16", seed=5)
+    y, h = run_add(inp, 1e-5)
+    y2 = nv.rms_norm(h, dev(inp["w"]), eps=1e-5)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("alias", ["h=x", "h=r", "y=x", "y=r", "y=x,h=r"])
+def test_add_rms_norm_in_place(alias):
+    rows, D = 77, 4096
+    inp = synth.add_rms_inputs(rows, D, "bf16", seed=6)
+    ref, href = oracle.add_rms_norm(host(inp["x"]), host(inp["r"]), host(inp["w"]), 1e-5)
+    x, r, w = dev(inp["x"]), dev(inp["r"]), dev(inp["w"])
+    y, h = torch.empty_like(x), torch.empty_like(x)
+    for a in alias.split(","):
+        out, src = a.split("=")
+        t = x if src == "x" else r
+        if out == "y":
+            y = t
+        else:
+            h = t
+    nv.nv_add_rms_norm(x, r, w, y, h, 1e-5)
+    torch.cuda.synchronize()
+    check_exact(h, href, "h")
+    check_out(y, ref)
+
+
+def test_misaligned_pointers_take_generic_path():
+    rows, D = 19, 4096
+    inp = synth.add_rms_inputs(rows, D, "bf16", seed=8)
+    n = rows * D
+    big = torch.empty(4 * n + 16, dtype=torch.bfloat16, device="cuda")
+    x, r, y, h = (big[1 + k * n: 1 + (k + 1) * n].view(rows, D) for k in range(4))  # 2-byte offset
+    x.copy_(inp["x"])
+    r.copy_(inp["r"])
+    w = dev(inp["w"])
+    nv.nv_add_rms_norm(x, r, w, y, h, 1e-5)
+    torch.cuda.synchronize()
+    ref, href = oracle.add_rms_norm(host(inp["x"]), host(inp["r"]), host(inp["w"]), 1e-5)
+    check_exact(h, href, "h")
+    check_out(y, ref)
+    with pytest.raises(nv.NvError, match="UNSUPPORTED"):
+        nv.nv_add_rms_norm(x, r, w, y, h, 1e-5, plan=nv.Plan(path=nv.PATH_ROWS))
+
+
+def test_zero_and_special_rows():
+    D = 4096
+    x = torch.zeros(4, D, dtype=torch.bfloat16)
+    x[1] = 3.0
+    x[2, 5] = float("nan")
+    x[3, 7] = float("inf")
+    r = torch.zeros_like(x)
+    w = torch.ones(D, dtype=torch.bfloat16)
+    y, h = nv.add_rms_norm(x.cuda(), r.cuda(), w.cuda(), eps=1e-5)
+    torch.cuda.synchronize()
+    yh = y.float().cpu()
+    assert (yh[0] == 0).all(), "a zero row normalises to zero when eps > 0"
+    ref = oracle.add_rms_norm(host(x), host(r), host(w), 1e-5)[0]
+    check_out(y[:2], ref[:2])
+    assert torch.isnan(yh[2]).all() and torch.isnan(yh[3]).any(), "NaN/Inf stay in their row"
+
+
+def test_zero_rows_launches_nothing():
+    x = torch.empty(0, 4096, dtype=torch.bfloat16, device="cuda")
+    y, h = nv.add_rms_norm(x, x.clone())
+    assert y.shape == (0, 4096) and h.shape == (0, 4096)
+
+
+def test_host_memory_undersized_and_overlapping_buffers_are_rejected():
+    import ctypes
+    x = torch.randn(8, 256, dtype=torch.bfloat16, device="cuda")
+    w = torch.ones(256, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty_like(x)
+    with pytest.raises(nv.NvError, match="not device memory"):
+        nv.nv_rms_norm(x.cpu().pin_memory(), w, y, 1e-5)
+    # 2^20 rows of 256 cannot fit the (at most a few MB) allocation holding x
+    st = nv.library().nv_rms_norm(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(w.data_ptr()),
+                                  ctypes.c_void_p(y.data_ptr()), 1 << 20, 256, 1e-5, nv.NV_BF16,
+                                  None)
+    assert st == nv.NV_ERR_INVALID_ARG
+    assert "past the end" in nv.library().nv_last_error().decode()
+    with pytest.raises(nv.NvError, match="overlaps"):
+        nv.nv_rms_norm(x, x[0], x, 1e-5)      # y == x is fine; w inside the output is not
+    with pytest.raises(nv.NvError, match="same buffer"):
+        nv.nv_add_rms_norm(x, x.clone(), w, y, y, 1e-5)
+    big = torch.zeros(3 * 2048, dtype=torch.bfloat16, device="cuda")
+    xs, ys = big[:2048].view(8, 256), big[128:128 + 2048].view(8, 256)
+    with pytest.raises(nv.NvError, match="overlaps"):
+        nv.nv_rms_norm(xs, w, ys, 1e-5)      # partial overlap of input and output
+
+
+# ---- layer_norm --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,D,wb", [(147, 8192, (1, 1)), (149, 5120, (1, 0)), (33, 4096, (0, 0)),
+                                        (5, 16384, (1, 1)), (64, 512, (1, 1)), (9, 1001, (1, 1)),
+                                        (3, 1, (1, 1)), (300, 256, (0, 1))])
+def test_layer_norm(rows, D, wb, dt):
+    inp = synth.layer_norm_inputs(rows, D, dt, seed=D + rows, weight=bool(wb[0]), bias=bool(wb[1]))
+    x, w, b = dev(inp["x"]), dev(inp["w"]), dev(inp["b"])
+    g = Guarded(x.shape, x.dtype)
+    nv.nv_layer_norm(x, w, b, g.t, 1e-5)
+    torch.cuda.synchronize()
+    assert g.bands_intact()
+    check_out(g.t, oracle.layer_norm(host(inp["x"]), host(inp["w"]), host(inp["b"]), 1e-5))
+
+
+@pytest.mark.parametrize("plan", [dict(path=nv.PATH_GENERIC)] +
+                         [dict(path=nv.PATH_ROWS, vec_per_thread=v) for v in (1, 2, 4)])
+def test_layer_norm_every_variant(plan):
+    inp = synth.layer_norm_inputs(211, 4096, "bf16", seed=2)
+    x = dev(inp["x"])
+    y = torch.empty_like(x)
+    nv.nv_layer_norm(x, dev(inp["w"]), dev(inp["b"]), y, 1e-5, plan=nv.Plan(**plan))
+    torch.cuda.synchronize()
+    check_out(y, oracle.layer_norm(host(inp["x"]), host(inp["w"]), host(inp["b"]), 1e-5))
+
+
+def test_layer_norm_in_place_and_large_mean():
+    x = synth.normal((64, 4096), 300.0, 0.5, 0, 0, "bf16")   # |mean| >> std
+    ref = oracle.layer_norm(host(x), None, None, 1e-5)
+    xd = x.cuda()
+    nv.nv_layer_norm(xd, None, None, xd, 1e-5)
+    torch.cuda.synchronize()
+    check_out(xd, ref)
+
+
+# ---- norm_rope ---------------------------------------------------------------------------
+
+ROPE_CASES = [
+    # B, H, L, D, dims, traditional, offset, normalize, weight
+    (2, 4, 64, 128, 128, 0, 0, 1, True),
+    (2, 4, 64, 128, 128, 1, 4096, 1, True),
+    (1, 3, 50, 128, 64, 0, 7, 1, True),
+    (1, 3, 50, 128, 32, 1, 7, 1, True),
+    (2, 2, 33, 64, 64, 0, 100000, 1, True),
+    (1, 2, 40, 256, 256, 0, 5, 1, False),
+    (1, 2, 40, 256, 128, 1, 5, 0, True),
+    (3, 1, 17, 128, 128, 0, 0, 0, False),
+    (1, 5, 9, 100, 50, 0, 3, 1, True),       # half = 25: generic path
+    (1, 2, 12, 1000, 96, 1, 2, 1, True),     # D > 256: generic path
+    (1, 1, 6, 6, 4, 0, 1, 1, True),
+    (1, 600, 1, 128, 128, 0, 4095, 1, True),  # decode-like: one position, many rows
+]
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("case", ROPE_CASES, ids=lambda c: "x".join(map(str, c)))
+def test_norm_rope(case, dt):
+    B, H, L, D, dims, trad, offset, normalize, weight = case
+    inp = synth.norm_rope_inputs(B, H, L, D, dt, seed=L + D, weight=weight)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    g = Guarded(x.shape, x.dtype)
+    eps = 1e-6
+    nv.nv_norm_rope(x, w, g.t, L, dims, trad, 10000.0, 1.0, offset, normalize, eps)
+    torch.cuda.synchronize()
+    assert g.bands_intact()
+    ref = oracle.norm_rope(host(inp["x"]), host(inp["w"]), L, dims, trad, 10000.0, 1.0, offset,
+                           normalize, eps)
+    check_out(g.t, ref)
+
+
+@pytest.mark.parametrize("trad", [0, 1])
+def test_norm_rope_base_and_scale(trad):
+    B, H, L, D = 1, 4, 32, 128
+    inp = synth.norm_rope_inputs(B, H, L, D, "bf16", seed=9)
+    x = dev(inp["x"])
+    y = torch.empty_like(x)
+    nv.nv_norm_rope(x, dev(inp["w"]), y, L, 128, trad, 500000.0, 0.125, 8192, 1, 1e-5)
+    torch.cuda.synchronize()
+    ref = oracle.norm_rope(host(inp["x"]), host(inp["w"]), L, 128, trad, 500000.0, 0.125, 8192, 1,
+                           1e-5)
+    check_out(y, ref)
+
+
+def test_norm_rope_generic_path_matches_register_path():
+    inp = synth.norm_rope_inputs(2, 4, 64, 128, "bf16", seed=1)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    ys = []
+    for path in (nv.PATH_ROWS, nv.PATH_GENERIC):
+        y = torch.empty_like(x)
+        nv.nv_norm_rope(x, w, y, 64, 128, 0, 10000.0, 1.0, 4096, 1, 1e-6, plan=nv.Plan(path=path))
+        ys.append(y)
+    torch.cuda.synchronize()
+    ref = oracle.norm_rope(host(inp["x"]), host(inp["w"]), 64, 128, 0, 10000.0, 1.0, 4096, 1, 1e-6)
+    for y in ys:
+        check_out(y, ref)
+
+
+def test_norm_rope_in_place():
+    inp = synth.norm_rope_inputs(2, 4, 16, 128, "bf16", seed=4)
+    ref = oracle.norm_rope(host(inp["x"]), host(inp["w"]), 16, 128, 1, 10000.0, 1.0, 4096, 1, 1e-6)
+    x = dev(inp["x"])
+    nv.nv_norm_rope(x, dev(inp["w"]), x, 16, 128, 1, 10000.0, 1.0, 4096, 1, 1e-6)
+    torch.cuda.synchronize()
+    check_out(x, ref)
