@@ -206,7 +206,12 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
     const int vecw = 16 / (int)elem_size(dt);
     const bool vec_ok = aligned && D % vecw == 0 && D / vecw <= 8192;
     const int nvec = vec_ok ? (int)(D / vecw) : 0;
-    if (p.path == NV_PATH_AUTO) p.path = vec_ok ? NV_PATH_ROWS : NV_PATH_GENERIC;
+    if (p.path == NV_PATH_AUTO) {
+        int v = 0, g = 0;
+        p.path = vec_ok && rows_shape(op, nvec, p.vec_per_thread, p.threads_per_row, &v, &g)
+                     ? NV_PATH_ROWS
+                     : NV_PATH_GENERIC;
+    }
     if (p.path == NV_PATH_ROWS) {
         if (!vec_ok) return fail(NV_ERR_UNSUPPORTED, "register path needs D %% %d == 0 and "
                                  "16-byte aligned pointers", vecw);
