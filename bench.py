@@ -5,8 +5,10 @@ Default workload (one step = one add_rms_norm call through the C ABI):
     add_rms_norm, bfloat16 I/O, x and r [8192, 4096] ~ N(0, 1), w [4096] ~ U(0.5, 1.5),
     eps = 1e-5; outputs y and h = x + r.
 Metric: achieved HBM GB/s of algorithmic bytes (4 N s + D s per call, s = 2) and rows/s,
-against B200's HBM peak.  L2 is flushed (a write of 2x the L2 size) before every step;
-each step is timed alone with CUDA events on the launching stream.
+against B200's HBM peak.  Each step is timed with CUDA events on the launching stream.
+Steps rotate over device buffer sets that together exceed L2 several times and run back
+to back, so no step reads data a previous step left in L2 and every step pays the
+write-back of its predecessor's output (workloads smaller than L2 flush it instead).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --sweep        # add_rms_norm over D x rows x dtype, one line per point
@@ -159,7 +161,13 @@ def algorithmic_bytes(op, rows, D, s):
 
 
 class Case:
-    """Device-resident inputs/outputs of one workload and a callable that runs it once."""
+    """Device-resident inputs/outputs of one workload and a callable that runs it once.
+
+    Large workloads keep `nsets` copies of their device buffers and step i uses copy
+    i % nsets, so consecutive steps touch disjoint memory larger than L2 and run back to
+    back (each step then also pays the write-back of the previous step's dirty lines,
+    as in a steady stream).  Workloads too small for that are timed after an L2 flush.
+    """
 
     def __init__(self, op, shape, dtype, seed, **kw):
         from rope_add_rms_b200 import synth
@@ -181,45 +189,63 @@ class Case:
             else:
                 inp = synth.layer_norm_inputs(rows, D, dtype, seed)
         self.host = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
-        self.dev = {k: (v.cuda() if v is not None else None) for k, v in self.host.items()}
-        x = self.dev["x"]
-        self.y = torch.empty_like(x)
-        self.h = torch.empty_like(x) if op == "add_rms_norm" else None
         self.bytes = algorithmic_bytes(op, self.rows, self.D, self.s)
+        l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+        n_row_tensors = 4 if op == "add_rms_norm" else 2
+        set_bytes = n_row_tensors * self.rows * self.D * self.s
+        if set_bytes >= l2:
+            self.nsets = max(2, min(8, -(-3 * l2 // set_bytes)))
+        else:
+            self.nsets = 1
+        self.sets = []
+        for _ in range(self.nsets):
+            d = {k: (v.cuda() if v is not None else None) for k, v in self.host.items()}
+            d["y"] = torch.empty_like(d["x"])
+            d["h"] = torch.empty_like(d["x"]) if op == "add_rms_norm" else None
+            self.sets.append(d)
         self.nv = nv
-        if op == "add_rms_norm":
-            self.host_out = [torch.empty_like(self.host["x"]).pin_memory() for _ in range(2)]
-        else:
-            self.host_out = [torch.empty_like(self.host["x"]).pin_memory()]
+        n_out = 2 if op == "add_rms_norm" else 1
+        self.host_out = [torch.empty_like(self.host["x"]).pin_memory() for _ in range(n_out)]
+        self.plan = None
 
-    def run(self, stream=None):
-        d, nv = self.dev, self.nv
+    @property
+    def rotating(self):
+        return self.nsets > 1
+
+    def l2_note(self):
+        if self.rotating:
+            mb = self.nsets * (4 if self.op == "add_rms_norm" else 2) * self.rows * self.D * self.s
+            return (f"inputs larger than L2: {self.nsets} buffer sets ({mb / 1e6:.0f} MB) "
+                    "rotated, steps back to back, no flush")
+        return "L2 flushed before every step (write of 2x L2)"
+
+    def run(self, stream=None, i=0):
+        d, nv, k = self.sets[i % self.nsets], self.nv, self.kw
         if self.op == "add_rms_norm":
-            nv.nv_add_rms_norm(d["x"], d["r"], d["w"], self.y, self.h, self.kw["eps"], stream)
+            nv.nv_add_rms_norm(d["x"], d["r"], d["w"], d["y"], d["h"], k["eps"], stream, self.plan)
         elif self.op == "rms_norm":
-            nv.nv_rms_norm(d["x"], d["w"], self.y, self.kw["eps"], stream)
+            nv.nv_rms_norm(d["x"], d["w"], d["y"], k["eps"], stream, self.plan)
         elif self.op == "layer_norm":
-            nv.nv_layer_norm(d["x"], d["w"], d["b"], self.y, self.kw["eps"], stream)
+            nv.nv_layer_norm(d["x"], d["w"], d["b"], d["y"], k["eps"], stream, self.plan)
         else:
-            k = self.kw
-            nv.nv_norm_rope(d["x"], d["w"], self.y, self.L, k["dims"], k["traditional"], k["base"],
-                            k["scale"], k["offset"], 1, k["eps"], stream)
+            nv.nv_norm_rope(d["x"], d["w"], d["y"], self.L, k["dims"], k["traditional"], k["base"],
+                            k["scale"], k["offset"], 1, k["eps"], stream, self.plan)
 
-    def run_e2e(self, stream):
+    def run_e2e(self, stream=None, i=0):
         """Host -> device copy of the step's inputs, the call, device -> host of its outputs."""
-        self.dev["x"].copy_(self.host["x"], non_blocking=True)
+        d = self.sets[0]
+        d["x"].copy_(self.host["x"], non_blocking=True)
         if self.op == "add_rms_norm":
-            self.dev["r"].copy_(self.host["r"], non_blocking=True)
-        self.run(stream)
-        self.host_out[0].copy_(self.y, non_blocking=True)
-        if self.h is not None:
-            self.host_out[1].copy_(self.h, non_blocking=True)
+            d["r"].copy_(self.host["r"], non_blocking=True)
+        self.run(stream, 0)
+        self.host_out[0].copy_(d["y"], non_blocking=True)
+        if self.op == "add_rms_norm":
+            self.host_out[1].copy_(d["h"], non_blocking=True)
 
     def e2e_bytes(self):
-        n_in = 2 if self.op == "add_rms_norm" else 1
-        n_out = 2 if self.op == "add_rms_norm" else 1
+        n = 2 if self.op == "add_rms_norm" else 1
         per = self.rows * self.D * self.s
-        return n_in * per, n_out * per
+        return n * per, n * per
 
 
 def l2_flush_buffer():
@@ -227,19 +253,40 @@ def l2_flush_buffer():
     return torch.empty(2 * max(l2, 64 << 20), dtype=torch.uint8, device="cuda")
 
 
-def time_steps(case, steps, warmup, flush, e2e=False):
-    """Per-step device times (ms) of `steps` runs, each after an L2 flush."""
+def time_span(case, steps, warmup):
+    """K back-to-back steps over rotating buffer sets, bracketed by one pair of CUDA
+    events on the launching stream; returns the span in ms."""
     stream = torch.cuda.current_stream()
-    for _ in range(warmup):
-        flush.zero_()
-        (case.run_e2e if e2e else case.run)(stream)
+    for i in range(warmup):
+        case.run(stream, i)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        case.run(stream, i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
+
+
+def time_steps(case, steps, warmup, flush, e2e=False):
+    """Per-step device times (ms): CUDA events around each call on the launching stream."""
+    stream = torch.cuda.current_stream()
+    fn = case.run_e2e if e2e else case.run
+    use_flush = e2e or not case.rotating
+    for i in range(warmup):
+        if use_flush:
+            flush.zero_()
+        fn(stream, i)
     torch.cuda.synchronize()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     for i in range(steps):
-        flush.zero_()
+        if use_flush:
+            flush.zero_()
         starts[i].record(stream)
-        (case.run_e2e if e2e else case.run)(stream)
+        fn(stream, i)
         ends[i].record(stream)
     torch.cuda.synchronize()
     return [s.elapsed_time(e) for s, e in zip(starts, ends)]
@@ -326,8 +373,10 @@ def other_configs(flush, steps):
             Case("rms_norm", (64, 512), "f32", 0, eps=1e-6),
     }
     for name, c in cases.items():
-        ts = time_steps(c, steps, 3, flush)
-        med = statistics.median(ts)
+        if c.rotating:
+            med = time_span(c, steps, 3) / steps
+        else:
+            med = statistics.median(time_steps(c, steps, 3, flush))
         gbs = c.bytes / (med * 1e-3) / 1e9
         out[name] = {"median_us": round(med * 1e3, 2), "GB/s": round(gbs, 1),
                      "frac_of_measured_hbm": round(gbs / peak, 4),
@@ -359,12 +408,14 @@ def run_ours(args):
             pg.barrier()
         torch.cuda.synchronize()
 
-    # warm-up, then the timed steps with clocks sampled during them
+    # warm-up, then the timed steps (back to back, one event pair) with clocks sampled
     barrier()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        ts = time_steps(case, args.steps, args.warmup, flush)
+        total_ms = time_span(case, args.steps, args.warmup)
     barrier()
-    total_ms = sum(ts)
+    # per-step distribution, each step bracketed by its own events (informational)
+    ts = time_steps(case, min(args.steps, 100), 3, flush)
+    barrier()
     e2e_steps = max(3, min(args.steps, 20))
     te = time_steps(case, e2e_steps, 3, flush, e2e=True)
     barrier()
@@ -385,7 +436,7 @@ def run_ours(args):
         peak, peak_kind = measured_peak()
         step_bytes = case.bytes
         value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
-        per_launch_ms = statistics.mean(ts)
+        per_launch_ms = total_ms / args.steps      # average launch duration, back to back
         achieved = step_bytes / (per_launch_ms * 1e-3) / 1e9
         bi, bo = case.e2e_bytes()
         e2e_value = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
@@ -400,13 +451,16 @@ def run_ours(args):
                                    "~U(0.5,1.5), eps 1e-5 (outputs y, h); per GPU",
                        "rows": WORKLOAD["rows"], "D": WORKLOAD["D"], "global_batch_rows":
                            WORKLOAD["rows"] * world,
-                       "l2": "flushed before every step (write of 2x L2)",
+                       "l2": case.l2_note(),
                        "parallelism": f"row shards x{world}, no collective",
                        "plan": plan},
             "rows_per_s": round(world * WORKLOAD["rows"] * args.steps / (total_ms * 1e-3), 1),
             "step_us": {"median": round(statistics.median(ts) * 1e3, 3),
                         "p10": round(float(np.percentile(ts, 10)) * 1e3, 3),
-                        "p90": round(float(np.percentile(ts, 90)) * 1e3, 3)},
+                        "p90": round(float(np.percentile(ts, 90)) * 1e3, 3),
+                        "how": "each step alone between its own events (not the headline)"},
+            "timing": "K steps back to back over rotating buffer sets, one CUDA event pair "
+                      "on the launching stream; max over ranks",
             "frac_of_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
@@ -441,8 +495,10 @@ def run_sweep(args):
         for D in (2048, 4096, 5120, 8192, 16384):
             for rows in (1, 16, 256, 4096, 65536):
                 c = Case("add_rms_norm", (rows, D), dtype, 0, eps=1e-6)
-                ts = time_steps(c, args.steps, args.warmup, flush)
-                med = statistics.median(ts)
+                if c.rotating:
+                    med = time_span(c, args.steps, args.warmup) / args.steps
+                else:
+                    med = statistics.median(time_steps(c, args.steps, args.warmup, flush))
                 gbs = c.bytes / (med * 1e-3) / 1e9
                 print(json.dumps({"op": "add_rms_norm", "dtype": dtype, "rows": rows, "D": D,
                                   "median_us": round(med * 1e3, 2), "GB/s": round(gbs, 1),

@@ -123,6 +123,15 @@ NV_API const char* nv_last_error(void);
 NV_API int32_t nv_version(void);
 
 /*
+ * Device-side bounded waits that ran out, on the current device, since the library
+ * was loaded (or last reset).  Only the staged kernels wait on the copy engine; each
+ * wait gives up after about one second, counts a fault here, lets its copies in
+ * flight land and leaves the rest of its rows unwritten.  Synchronises the device.
+ * count: out, non-NULL.  reset != 0 sets the counter back to zero after reading it.
+ */
+NV_API nv_status nv_fault_count(uint32_t* count, int32_t reset);
+
+/*
  * Kernel-variant control, for tests and benchmarks.  The plain entry points above
  * pick a variant from (op, dtype, D, rows, alignment); the *_ex forms take a plan
  * that forces one.  A plan that the shape cannot use returns NV_ERR_UNSUPPORTED.
@@ -131,13 +140,22 @@ NV_API int32_t nv_version(void);
  *   threads_per_row threads that share one row (multiple of 32, <= 1024; 0 = auto)
  *   rows_per_cta    rows one CTA works on at a time (0 = auto)
  *   ctas_per_sm     persistent grid size per SM (0 = auto)
+ *   launch          NV_LAUNCH_DEFAULT: programmatic dependent launch -- the kernel may
+ *                   be scheduled while the preceding kernel of the stream finishes, and
+ *                   it waits for that kernel (griddepcontrol.wait) before reading or
+ *                   writing any global memory, so results are the same as with a plain
+ *                   launch; NV_LAUNCH_PLAIN: ordinary stream-ordered launch.
  */
 typedef enum {
     NV_PATH_AUTO = 0,
     NV_PATH_ROWS = 1,    /* row held in registers, 16-byte vector loads */
     NV_PATH_GENERIC = 2, /* any D and alignment: scalar loop, two passes over the row */
-    NV_PATH_STAGED = 3   /* persistent, rows staged in shared memory by bulk async copies */
+    NV_PATH_STAGED = 3   /* persistent, rows staged in shared memory by bulk async copies;
+                            rms_norm and add_rms_norm only.  rows_per_cta = rows in flight
+                            per CTA (shared-memory stages), ctas_per_sm = CTAs per SM */
 } nv_path;
+
+typedef enum { NV_LAUNCH_DEFAULT = 0, NV_LAUNCH_PLAIN = 1 } nv_launch;
 
 typedef struct {
     int32_t path;
@@ -145,6 +163,7 @@ typedef struct {
     int32_t threads_per_row;
     int32_t rows_per_cta;
     int32_t ctas_per_sm;
+    int32_t launch;
 } nv_plan;
 
 NV_API nv_status nv_rms_norm_ex(const void* x, const void* w, void* y, int64_t rows, int64_t D,

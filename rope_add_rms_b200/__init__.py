@@ -19,8 +19,9 @@ import torch
 __all__ = [
     "NvError", "Plan", "library", "library_path",
     "nv_rms_norm", "nv_add_rms_norm", "nv_layer_norm", "nv_norm_rope", "nv_describe_plan",
+    "nv_fault_count",
     "rms_norm", "add_rms_norm", "layer_norm", "norm_rope",
-    "PATH_AUTO", "PATH_ROWS", "PATH_GENERIC", "PATH_STAGED",
+    "PATH_AUTO", "PATH_ROWS", "PATH_GENERIC", "PATH_STAGED", "LAUNCH_DEFAULT", "LAUNCH_PLAIN",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,6 +30,7 @@ library_path = os.path.join(_HERE, "libnvnorm.so")
 NV_F32, NV_BF16, NV_F16 = 0, 1, 2
 NV_OK, NV_ERR_INVALID_ARG, NV_ERR_UNSUPPORTED, NV_ERR_CUDA = 0, 1, 2, 3
 PATH_AUTO, PATH_ROWS, PATH_GENERIC, PATH_STAGED = 0, 1, 2, 3
+LAUNCH_DEFAULT, LAUNCH_PLAIN = 0, 1
 
 _DT = {torch.float32: NV_F32, torch.bfloat16: NV_BF16, torch.float16: NV_F16}
 
@@ -46,7 +48,7 @@ class Plan(ctypes.Structure):
     """nv_plan: kernel-variant selection (0 fields mean automatic)."""
     _fields_ = [("path", ctypes.c_int32), ("vec_per_thread", ctypes.c_int32),
                 ("threads_per_row", ctypes.c_int32), ("rows_per_cta", ctypes.c_int32),
-                ("ctas_per_sm", ctypes.c_int32)]
+                ("ctas_per_sm", ctypes.c_int32), ("launch", ctypes.c_int32)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_}
@@ -88,6 +90,8 @@ def library() -> ctypes.CDLL:
     lib.nv_last_error.restype = ctypes.c_char_p
     lib.nv_version.argtypes = []
     lib.nv_version.restype = ctypes.c_int32
+    lib.nv_fault_count.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]
+    lib.nv_fault_count.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -180,6 +184,13 @@ def nv_describe_plan(op: str, rows: int, D: int, dtype) -> dict:
     _check("nv_describe_plan", library().nv_describe_plan(ops[op], rows, D, _DT[dtype],
                                                            ctypes.byref(p)))
     return p.as_dict()
+
+
+def nv_fault_count(reset: bool = False) -> int:
+    """Bounded device waits that ran out on the current device (synchronises it)."""
+    c = ctypes.c_uint32(0)
+    _check("nv_fault_count", library().nv_fault_count(ctypes.byref(c), int(bool(reset))))
+    return c.value
 
 
 # ---- allocating wrappers ---------------------------------------------------------------

@@ -94,6 +94,17 @@ __device__ __forceinline__ V16 zeros_vec() {
     return V16{{0u, 0u, 0u, 0u}};
 }
 
+// ---- programmatic dependent launch ---------------------------------------------------
+// Every kernel starts with pdl_wait() before it touches global memory: when it was
+// launched with programmatic stream serialization after a kernel that lets dependents
+// start early, this blocks until that kernel has completed and its memory is visible;
+// otherwise it returns at once.  pdl_release() lets the next such kernel in the stream
+// be scheduled while this one still runs (that kernel waits in its own pdl_wait()).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- reductions ---------------------------------------------------------------------
 // Butterfly sum over aligned groups of `width` lanes (width a power of two <= 32).
 template <typename F>

@@ -61,6 +61,8 @@ __device__ __forceinline__ double row_sum_f64(double v, double* buf, int slot, i
 // ---- register path ------------------------------------------------------------------
 template <typename T, int VPT>
 __global__ void __launch_bounds__(layer_max_threads(VPT)) layer_rows_kernel(const RowArgs a) {
+    pdl_wait();
+    pdl_release();
     using E = Elem<T>;
     constexpr int VEC = E::kVec;
     const int G = a.G;
@@ -144,6 +146,8 @@ __global__ void __launch_bounds__(layer_max_threads(VPT)) layer_rows_kernel(cons
 // it writes index j in the last one.
 template <typename T>
 __global__ void __launch_bounds__(256) layer_generic_kernel(const RowArgs a) {
+    pdl_wait();
+    pdl_release();
     using E = Elem<T>;
     __shared__ double red[4][32];
     const int wpr = blockDim.x >> 5;

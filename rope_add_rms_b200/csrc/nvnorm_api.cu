@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "nvnorm.h"
 
@@ -17,6 +18,7 @@
 #include "layer.cuh"
 #include "rms.cuh"
 #include "rope.cuh"
+#include "staged.cuh"
 
 namespace {
 
@@ -42,6 +44,8 @@ nv_status cuda_fail(cudaError_t e, const char* what) {
 // ---- device facts, cached per device ---------------------------------------------------
 struct DevInfo {
     int sms = 0;
+    int smem_optin = 0;   // largest dynamic + static shared memory one CTA may use
+    int smem_per_sm = 0;
     bool ready = false;
 };
 constexpr int kMaxDevices = 64;
@@ -56,6 +60,11 @@ nv_status current_device(int* dev, DevInfo* info) {
     DevInfo& d = g_dev[*dev];
     if (!d.ready) {
         e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, *dev);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, *dev);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&d.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor,
+                                       *dev);
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
         d.ready = true;
     }
@@ -199,8 +208,15 @@ bool rows_shape(Op op, int nvec, int vpt_req, int g_req, int* vpt, int* G) {
     return true;
 }
 
+// Staged path: shared memory of one CTA for `stages` rows in flight.
+size_t staged_smem(Op op, int64_t D, nv_dtype dt, int stages) {
+    const size_t stage = (size_t)(op == OP_ADD ? 2 : 1) * (size_t)D * elem_size(dt);
+    return (size_t)stages * (stage + 8);
+}
+constexpr int kStaticSmemReserve = 2048;  // static shared memory + per-CTA system use
+
 nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, const nv_plan* req,
-                    nv_plan* out) {
+                    nv_plan* out, const DevInfo* di = nullptr) {
     nv_plan p{};
     if (req) p = *req;
     const int vecw = 16 / (int)elem_size(dt);
@@ -228,6 +244,26 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
         p.vec_per_thread = 0;
         p.threads_per_row = 256;
         p.rows_per_cta = 1;
+    } else if (p.path == NV_PATH_STAGED) {
+        if (op == OP_LAYER)
+            return fail(NV_ERR_UNSUPPORTED, "the staged path covers rms_norm and add_rms_norm");
+        if (!vec_ok) return fail(NV_ERR_UNSUPPORTED, "staged path needs D %% %d == 0 and "
+                                 "16-byte aligned pointers", vecw);
+        int vpt = 0, G = 0;
+        if (!rows_shape(op, nvec, p.vec_per_thread, p.threads_per_row, &vpt, &G) || G > 512)
+            return fail(NV_ERR_UNSUPPORTED, "no staged shape for D = %lld (vpt %d, G %d)",
+                        (long long)D, p.vec_per_thread, p.threads_per_row);
+        p.vec_per_thread = vpt;
+        p.threads_per_row = G;
+        const int optin = di ? di->smem_optin : 232448;
+        const int per_sm = di ? di->smem_per_sm : 233472;
+        if (p.ctas_per_sm == 0) p.ctas_per_sm = 1;
+        const int budget = std::min(optin, per_sm / p.ctas_per_sm) - kStaticSmemReserve;
+        const size_t one = staged_smem(op, D, dt, 1);
+        if (p.rows_per_cta == 0) p.rows_per_cta = (int)std::min<size_t>(8, budget / one);
+        if (p.rows_per_cta < 2 || staged_smem(op, D, dt, p.rows_per_cta) > (size_t)budget)
+            return fail(NV_ERR_UNSUPPORTED, "staged path: %d stages of %zu bytes do not fit "
+                        "%d bytes of shared memory", p.rows_per_cta, one, budget);
     } else {
         return fail(NV_ERR_UNSUPPORTED, "path %d is not available for this op", p.path);
     }
@@ -252,21 +288,63 @@ int64_t grid_for(int64_t units, int sms, int per_sm) {
     return std::max<int64_t>(1, std::min<int64_t>(units, (int64_t)sms * per_sm));
 }
 
+// Launch with programmatic stream serialization allowed (unless the plan asks for a
+// plain launch): the kernel may be scheduled while the preceding kernel of the stream
+// finishes, and waits for it in pdl_wait() before touching global memory.
+thread_local bool g_pdl = true;
+
+template <typename... KArgs, typename... Args>
+nv_status launch_kernel(void (*kernel)(KArgs...), int64_t grid, int block, size_t smem,
+                        cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = g_pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return NV_OK;
+}
+
 template <typename K>
 nv_status launch(K kernel, int64_t units, int block, size_t smem, int ctas_per_sm,
                  const DevInfo& di, cudaStream_t s, const RowArgs& a) {
     const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : occupancy(kernel, block, smem);
     const int64_t grid = grid_for(units, di.sms, per_sm);
-    kernel<<<(unsigned)grid, block, smem, s>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
-    return NV_OK;
+    return launch_kernel(kernel, grid, block, smem, s, a);
+}
+
+template <typename K>
+nv_status launch_staged(K kernel, const nv_plan& p, size_t smem, const DevInfo& di,
+                        cudaStream_t s, const RowArgs& a) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    const int64_t grid = grid_for(a.rows, di.sms, p.ctas_per_sm);
+    return launch_kernel(kernel, grid, p.threads_per_row, smem, s, a, p.rows_per_cta);
 }
 
 template <typename T, bool ADD>
 nv_status run_rms(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs a) {
     if (p.path == NV_PATH_GENERIC)
         return launch(rms_generic_kernel<T, ADD>, a.rows, 256, 0, p.ctas_per_sm, di, s, a);
+    if (p.path == NV_PATH_STAGED) {
+        const size_t smem = staged_smem(ADD ? OP_ADD : OP_RMS, a.D,
+                                        sizeof(T) == 4 ? NV_F32 : NV_BF16, p.rows_per_cta);
+        switch (p.vec_per_thread) {
+            case 1: return launch_staged(rms_staged_kernel<T, 1, ADD>, p, smem, di, s, a);
+            case 2: return launch_staged(rms_staged_kernel<T, 2, ADD>, p, smem, di, s, a);
+            case 4: return launch_staged(rms_staged_kernel<T, 4, ADD>, p, smem, di, s, a);
+            case 8: return launch_staged(rms_staged_kernel<T, 8, ADD>, p, smem, di, s, a);
+        }
+        return fail(NV_ERR_UNSUPPORTED, "vec_per_thread %d", p.vec_per_thread);
+    }
     a.G = p.threads_per_row;
     a.rows_per_cta = p.rows_per_cta;
     const int block = a.G * a.rows_per_cta;
@@ -330,8 +408,9 @@ nv_status row_op(Op op, const void* x, const void* r, const void* w, const void*
     if (op == OP_ADD) al = al && aligned16(r) && aligned16(h);
     if (op == OP_LAYER) al = al && (!b || aligned16(b));
     nv_plan p;
-    st = make_plan(op, rows, D, dt, al, req, &p);
+    st = make_plan(op, rows, D, dt, al, req, &p, &di);
     if (st != NV_OK) return st;
+    g_pdl = p.launch != NV_LAUNCH_PLAIN;
 
     RowArgs a{};
     a.x = x;
@@ -375,12 +454,8 @@ nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a)
                                              (int)smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     }
-    const int64_t grid = a.L * a.n_chunks;
-    kern<<<(unsigned)grid, 256, smem, s>>>(a);
     (void)di;
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
-    return NV_OK;
+    return launch_kernel(kern, a.L * a.n_chunks, 256, smem, s, a);
 }
 
 template <typename T>
@@ -388,11 +463,7 @@ nv_status launch_rope_generic(const DevInfo& di, int ctas_per_sm, cudaStream_t s
                               const RopeArgs& a) {
     auto kern = rope_generic_kernel<T>;
     const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : occupancy(kern, 128, 0);
-    const int64_t grid = grid_for(a.BH * a.L, di.sms, per_sm);
-    kern<<<(unsigned)grid, 128, 0, s>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
-    return NV_OK;
+    return launch_kernel(kern, grid_for(a.BH * a.L, di.sms, per_sm), 128, 0, s, a);
 }
 
 nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_dtype dt,
@@ -480,6 +551,7 @@ nv_status rope_op(const void* x, const void* w, void* y, int64_t rows, int64_t L
     RopePlan rp{};
     st = rope_plan(rows, L, D, dims, traditional != 0, dt, al, di.sms, req, &p, &rp);
     if (st != NV_OK) return st;
+    g_pdl = p.launch != NV_LAUNCH_PLAIN;
 
     RopeArgs a{};
     a.x = x;
@@ -589,6 +661,18 @@ const char* nv_status_string(nv_status status) {
 }
 
 const char* nv_last_error(void) { return g_msg; }
+
+nv_status nv_fault_count(uint32_t* count, int32_t reset) {
+    if (!count) return fail(NV_ERR_INVALID_ARG, "count is NULL");
+    cudaError_t e = cudaMemcpyFromSymbol(count, nvn::nvn_fault_count, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol");
+    if (reset) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyToSymbol(nvn::nvn_fault_count, &zero, sizeof(uint32_t));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
+    }
+    return NV_OK;
+}
 
 int32_t nv_version(void) { return kVersion; }
 

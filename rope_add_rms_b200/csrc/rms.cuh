@@ -42,6 +42,8 @@ __host__ __device__ constexpr bool weights_in_regs(int vpt) { return vpt <= 2; }
 
 template <typename T, int VPT, bool ADD>
 __global__ void __launch_bounds__(rms_max_threads(VPT)) rms_rows_kernel(const RowArgs a) {
+    pdl_wait();
+    pdl_release();
     using E = Elem<T>;
     constexpr int VEC = E::kVec;
     const int G = a.G;
@@ -143,6 +145,8 @@ __global__ void __launch_bounds__(rms_max_threads(VPT)) rms_rows_kernel(const Ro
 // -- the same thread touches the same index in both passes -- and writes y.
 template <typename T, bool ADD>
 __global__ void __launch_bounds__(256) rms_generic_kernel(const RowArgs a) {
+    pdl_wait();
+    pdl_release();
     using E = Elem<T>;
     __shared__ float red[2][32];
     const int nw = blockDim.x >> 5;

@@ -98,13 +98,7 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
     int pv = v;
     if (!TRAD) pv = (v < hv) ? v + hv : (v < 2 * hv ? v - hv : v);
 
-    // per-column weights of this lane's elements and of their partners
     const bool norm = a.normalize != 0;
-    V16 w_own = (norm && a.w && has_vec) ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16)
-                                         : ones_vec<T>();
-    V16 w_par = w_own;
-    if (!TRAD && pv != v && norm && a.w && pv < a.nvec)
-        w_par = ld_param(static_cast<const char*>(a.w) + (size_t)pv * 16);
 
     // first rows' loads go out before the table is built
     const int64_t bh0 = chunk * (int64_t)a.bt;
@@ -114,6 +108,14 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
     const char* xbase = static_cast<const char*>(a.x) + (size_t)l * row_bytes + (size_t)v * 16;
     char* ybase = static_cast<char*>(a.y) + (size_t)l * row_bytes + (size_t)v * 16;
 
+    // The angle table touches no global memory, so it is built before waiting on a
+    // preceding kernel (programmatic dependent launch).
+    const double pos = (double)(a.offset + l);
+    for (int i = threadIdx.x; i < a.half; i += blockDim.x)
+        tab[i] = angle_entry(pos, (double)a.scale, (double)a.base, i, a.dims);
+    pdl_wait();
+    pdl_release();
+
     // Every thread runs the same trip count (rows past bh_end are predicated off):
     // the shuffles below involve the whole warp, which may hold several rows.
     V16 xv[kUnroll];
@@ -122,10 +124,12 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
         const int64_t b = bh0 + slot + (int64_t)u * slots;
         if (has_vec && b < bh_end) xv[u] = ld_stream(xbase + (size_t)b * lstride);
     }
-
-    const double pos = (double)(a.offset + l);
-    for (int i = threadIdx.x; i < a.half; i += blockDim.x)
-        tab[i] = angle_entry(pos, (double)a.scale, (double)a.base, i, a.dims);
+    // per-column weights of this lane's elements and of their partners
+    V16 w_own = (norm && a.w && has_vec) ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16)
+                                         : ones_vec<T>();
+    V16 w_par = w_own;
+    if (!TRAD && pv != v && norm && a.w && pv < a.nvec)
+        w_par = ld_param(static_cast<const char*>(a.w) + (size_t)pv * 16);
     __syncthreads();
 
     // this lane's table entries, sin already carrying the sign of its side
@@ -209,6 +213,8 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
 // its angle computed in double, then the features past dims.
 template <typename T>
 __global__ void __launch_bounds__(128) rope_generic_kernel(const RopeArgs a) {
+    pdl_wait();
+    pdl_release();
     using E = Elem<T>;
     __shared__ float red[2][32];
     const int nw = blockDim.x >> 5;

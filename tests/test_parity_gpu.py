@@ -207,6 +207,52 @@ def test_host_memory_undersized_and_overlapping_buffers_are_rejected():
         nv.nv_rms_norm(xs, w, ys, 1e-5)      # partial overlap of input and output
 
 
+# ---- staged (bulk-copy) path ----------------------------------------------------------------
+
+STAGED = [dict(path=nv.PATH_STAGED),
+          dict(path=nv.PATH_STAGED, rows_per_cta=2, ctas_per_sm=1),
+          dict(path=nv.PATH_STAGED, rows_per_cta=4, ctas_per_sm=2, vec_per_thread=4),
+          dict(path=nv.PATH_STAGED, rows_per_cta=3, ctas_per_sm=3, vec_per_thread=1),
+          dict(path=nv.PATH_STAGED, rows_per_cta=5, ctas_per_sm=1, vec_per_thread=8)]
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("plan", STAGED, ids=lambda p: "-".join(f"{k}{v}" for k, v in p.items()))
+@pytest.mark.parametrize("rows,D", [(301, 4096), (1, 4096), (1000, 2048), (37, 5120), (5, 8192)])
+def test_add_rms_norm_staged(rows, D, plan, dt):
+    inp = synth.add_rms_inputs(rows, D, dt, seed=rows * 7 + D)
+    try:
+        y, h = run_add(inp, 1e-6, plan=nv.Plan(**plan))
+    except nv.NvError as e:          # the shape does not fit this forced plan
+        assert e.status == nv.NV_ERR_UNSUPPORTED
+        pytest.skip(str(e))
+    assert nv.nv_fault_count() == 0
+    ref, href = oracle.add_rms_norm(host(inp["x"]), host(inp["r"]), host(inp["w"]), 1e-6)
+    check_exact(h, href, "h")
+    check_out(y, ref)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("weight", [True, False])
+def test_rms_norm_staged(dt, weight):
+    inp = synth.rms_inputs(513, 4096, dt, seed=1, weight=weight)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    y = torch.empty_like(x)
+    nv.nv_rms_norm(x, w, y, 1e-6, plan=nv.Plan(path=nv.PATH_STAGED))
+    assert nv.nv_fault_count() == 0
+    check_out(y, oracle.rms_norm(host(inp["x"]), host(inp["w"]), 1e-6))
+
+
+def test_staged_in_place():
+    inp = synth.add_rms_inputs(300, 4096, "bf16", seed=2)
+    ref, href = oracle.add_rms_norm(host(inp["x"]), host(inp["r"]), host(inp["w"]), 1e-5)
+    x, r, w = dev(inp["x"]), dev(inp["r"]), dev(inp["w"])
+    nv.nv_add_rms_norm(x, r, w, x, r, 1e-5, plan=nv.Plan(path=nv.PATH_STAGED))   # y=x, h=r
+    assert nv.nv_fault_count() == 0
+    check_exact(r, href, "h")
+    check_out(x, ref)
+
+
 # ---- layer_norm --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
@@ -312,3 +358,70 @@ def test_norm_rope_in_place():
     nv.nv_norm_rope(x, dev(inp["w"]), x, 16, 128, 1, 10000.0, 1.0, 4096, 1, 1e-6)
     torch.cuda.synchronize()
     check_out(x, ref)
+
+
+# ---- programmatic dependent launch ---------------------------------------------------------
+
+@pytest.mark.parametrize("launch", [nv.LAUNCH_DEFAULT, nv.LAUNCH_PLAIN])
+@pytest.mark.parametrize("path", [nv.PATH_ROWS, nv.PATH_STAGED, nv.PATH_GENERIC])
+def test_dependent_chain(path, launch):
+    """Each call reads the previous call's outputs, launched back to back; every step
+    must match the oracle applied to that step's own (device-produced) inputs."""
+    rows, D, steps = 1024, 4096, 6
+    inp = synth.add_rms_inputs(rows, D, "bf16", seed=21)
+    x, r, w = dev(inp["x"]), dev(inp["r"]), dev(inp["w"])
+    plan = nv.Plan(path=path, launch=launch)
+    hist = [(x, r)]
+    for _ in range(steps):
+        y, h = torch.empty_like(x), torch.empty_like(x)
+        nv.nv_add_rms_norm(x, r, w, y, h, 1e-5, plan=plan)
+        x, r = y, h
+        hist.append((x, r))
+    torch.cuda.synchronize()
+    assert nv.nv_fault_count() == 0
+    for i in range(steps):
+        (xi, ri), (yo, ho) = hist[i], hist[i + 1]
+        ref, href = oracle.add_rms_norm(to_host_bits(xi), to_host_bits(ri), host(inp["w"]), 1e-5)
+        check_exact(ho, href, f"h of step {i}")
+        check_out(yo, ref, f"y of step {i}")
+
+
+def test_dependent_chain_across_ops_in_place():
+    """add_rms_norm -> layer_norm -> norm_rope -> rms_norm, each in place on the previous
+    output, all launched back to back with programmatic dependent launch."""
+    B, H, L, D = 2, 8, 64, 128
+    rows = B * H * L
+    inp = synth.add_rms_inputs(rows, D, "bf16", seed=22)
+    x, r, w = dev(inp["x"]), dev(inp["r"]), dev(inp["w"])
+    x0, r0 = to_host_bits(x), to_host_bits(r)
+    y = torch.empty_like(x)
+    nv.nv_add_rms_norm(x, r, w, y, r, 1e-5)               # h in place over r
+    nv.nv_layer_norm(y, w, None, y, 1e-5)                  # in place
+    nv.nv_norm_rope(y, w, y, L, D, 0, 10000.0, 1.0, 4096, 1, 1e-6)   # in place
+    nv.nv_rms_norm(y, None, y, 1e-6)                       # in place
+    torch.cuda.synchronize()
+    # replay on the oracle, feeding each stage the bf16 values the GPU stage produced:
+    # re-run the chain stage by stage on the device without overlap to get them
+    a = dev(inp["x"]).clone()
+    rr = dev(inp["r"]).clone()
+    stages = []
+    plain = nv.Plan(launch=nv.LAUNCH_PLAIN)
+    s1 = torch.empty_like(a)
+    nv.nv_add_rms_norm(a, rr, w, s1, rr, 1e-5, plan=plain); torch.cuda.synchronize()
+    stages.append(s1.clone())
+    nv.nv_layer_norm(s1, w, None, s1, 1e-5, plan=plain); torch.cuda.synchronize()
+    stages.append(s1.clone())
+    nv.nv_norm_rope(s1, w, s1, L, D, 0, 10000.0, 1.0, 4096, 1, 1e-6, plan=plain)
+    torch.cuda.synchronize()
+    stages.append(s1.clone())
+    nv.nv_rms_norm(s1, None, s1, 1e-6, plan=plain); torch.cuda.synchronize()
+    stages.append(s1.clone())
+    assert torch.equal(y.view(torch.int16), stages[-1].view(torch.int16)), \
+        "back-to-back launches changed the result"
+    wh = host(inp["w"])
+    ref1, _ = oracle.add_rms_norm(x0, r0, wh, 1e-5)
+    check_out(stages[0], ref1, "add_rms_norm")
+    check_out(stages[1], oracle.layer_norm(to_host_bits(stages[0]), wh, None, 1e-5), "layer_norm")
+    check_out(stages[2], oracle.norm_rope(to_host_bits(stages[1]), wh, L, D, 0, 10000.0, 1.0, 4096,
+                                          1, 1e-6), "norm_rope")
+    check_out(stages[3], oracle.rms_norm(to_host_bits(stages[2]), None, 1e-6), "rms_norm")
