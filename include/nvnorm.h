@@ -136,10 +136,14 @@ NV_API nv_status nv_fault_count(uint32_t* count, int32_t reset);
  * pick a variant from (op, dtype, D, rows, alignment); the *_ex forms take a plan
  * that forces one.  A plan that the shape cannot use returns NV_ERR_UNSUPPORTED.
  *   path            NV_PATH_AUTO, or one of the kernel families below
- *   vec_per_thread  16-byte vectors per thread and row (register paths; 0 = auto)
+ *   vec_per_thread  16-byte vectors per thread and row (register paths; 0 = auto; for
+ *                   norm_rope 1 = one vector per lane, 2 = both halves of the rotation
+ *                   per lane, which needs halves pairing and dims == D)
  *   threads_per_row threads that share one row (multiple of 32, <= 1024; 0 = auto)
  *   rows_per_cta    rows one CTA works on at a time (0 = auto)
- *   ctas_per_sm     persistent grid size per SM (0 = auto)
+ *   ctas_per_sm     0: one CTA per row group (register and generic paths) or one CTA
+ *                   per SM (staged path); > 0: a persistent grid of that many CTAs per
+ *                   SM walking the rows
  *   launch          NV_LAUNCH_DEFAULT: programmatic dependent launch -- the kernel may
  *                   be scheduled while the preceding kernel of the stream finishes, and
  *                   it waits for that kernel (griddepcontrol.wait) before reading or

@@ -35,7 +35,11 @@ struct Elem<float> {
         static_cast<float*>(p)[i] = v;
     }
     __device__ __forceinline__ static float round(float v) { return v; }
-    __device__ __forceinline__ static float one_bits_word() { return 1.0f; }
+    // elements e, e + 1 (e even) as a float pair, and back
+    __device__ __forceinline__ static float2 get2(const V16& v, int e) {
+        return make_float2(__uint_as_float(v.u[e]), __uint_as_float(v.u[e + 1]));
+    }
+    __device__ __forceinline__ static void put2(V16& v, int e, float2 p) { put2(v, e, p.x, p.y); }
 };
 
 template <>
@@ -61,7 +65,18 @@ struct Elem<__nv_bfloat16> {
     __device__ __forceinline__ static float round(float v) {
         return __bfloat162float(__float2bfloat16_rn(v));
     }
+    __device__ __forceinline__ static float2 get2(const V16& v, int e) {
+        const uint32_t w = v.u[e >> 1];
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    }
+    __device__ __forceinline__ static void put2(V16& v, int e, float2 p) { put2(v, e, p.x, p.y); }
 };
+
+// ---- packed float32 pairs (Blackwell FFMA2 / FADD2 / FMUL2; IEEE per lane) ------------
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
 
 // ---- 16-byte global memory access -------------------------------------------------
 // Streaming loads (read once: evict-first) and stores for the row data; plain cached

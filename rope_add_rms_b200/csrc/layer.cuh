@@ -58,7 +58,60 @@ __device__ __forceinline__ double row_sum_f64(double v, double* buf, int slot, i
     return v;
 }
 
+// Float32 output of one element and whether it passes the error test above.
+struct LnOut {
+    float mu_hi, mu_lo, rf, kmu;
+    bool two_sub;
+    __device__ __forceinline__ float y(float x, float w, float b, bool& ok) const {
+        const float A = __fmul_rn(rf, w);
+        const float d = two_sub ? __fsub_rn(__fsub_rn(x, mu_hi), mu_lo) : __fsub_rn(x, mu_hi);
+        const float v = __fmaf_rn(d, A, b);
+        ok = fabsf(v) > __fmaf_rn(kmu, fabsf(A), 0x1p-11f * fabsf(b));
+        return v;
+    }
+};
+
+// Recompute the elements of one output vector that fail the error test, in double
+// precision: y = (x - mean) * (rstd * w) + b, then round (via float32) to the I/O type.
+template <typename T>
+__device__ __noinline__ V16 fix_near_cancellation(V16 o, const LnOut f, V16 xv, V16 wv, V16 bv,
+                                                  double mean, double rstd) {
+    using E = Elem<T>;
+#pragma unroll 1
+    for (int e = 0; e < E::kVec; ++e) {
+        bool ok;
+        f.y(E::get(xv, e), E::get(wv, e), E::get(bv, e), ok);
+        if (ok) continue;
+        const double y = fma((double)E::get(xv, e) - mean, rstd * (double)E::get(wv, e),
+                             (double)E::get(bv, e));
+        const int e0 = e & ~1;
+        const float keep = E::get(o, e0 ^ (e & 1) ^ 1);  // the other element of the pair
+        const float yf = __double2float_rn(y);
+        if (e & 1)
+            E::put2(o, e0, keep, yf);
+        else
+            E::put2(o, e0, yf, keep);
+    }
+    return o;
+}
+
 // ---- register path ------------------------------------------------------------------
+// Conversions between float32 and double run at a quarter of the double-add rate on
+// B200, so each element is widened once: the statistics are the double sums S1 = sum x
+// and S2 = sum x^2 (exact for bfloat16 rows of ordinary range), var = S2/D - mean^2.
+// When mean^2 > 2^20 var the one-pass form could lose bits, and the row (every thread
+// of the CTA holds the same row, so the branch is CTA-uniform) redoes the centred sum
+// sum (x - mean)^2 in double.
+//
+// The output is formed in float32 with A = rstd * w and y = fma(d, A, b), where d is
+// x - mean_hi (one subtraction) or, for rows whose mean is large against their
+// spread, (x - mean_hi) - mean_lo with mean = mean_hi + mean_lo.  d and A each carry
+// at most ~2^-23 relative error, plus the absolute error of the mean kept, m = |mean_lo|
+// (one subtraction) or 2^-48 |mean| (two); so the error of y is below
+// 2^-22 |d A| + m |A| + 2^-24 |y|, and since |d A| <= |y| + |b| it stays under half a
+// bfloat16 step (2^-9 |y|) whenever |y| > 2^-11 |b| + 2^10 m |A| (a factor-2 margin on
+// each term).  Only a near cancellation of d A against b fails that test -- a few
+// elements in ten thousand -- and those elements are recomputed in double.
 template <typename T, int VPT>
 __global__ void __launch_bounds__(layer_max_threads(VPT)) layer_rows_kernel(const RowArgs a) {
     pdl_wait();
@@ -69,21 +122,22 @@ __global__ void __launch_bounds__(layer_max_threads(VPT)) layer_rows_kernel(cons
     const int slot = threadIdx.x / G;
     const int t = threadIdx.x - slot * G;
     const int wpr = G >> 5;
-    // four buffers: (mean, variance) x iteration parity
-    __shared__ double red[4][32];
+    // [parity][S1, S2][warp]; a row spanning several warps is alone in its CTA
+    __shared__ double red[2][2][32];
 
-    V16 wv[VPT], bv[VPT];
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-        const int v = t + k * G;
-        const bool in = v < a.nvec;
-        wv[k] = (a.w != nullptr && in) ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16)
-                                       : ones_vec<T>();
-        bv[k] = (a.b != nullptr && in) ? ld_param(static_cast<const char*>(a.b) + (size_t)v * 16)
-                                       : zeros_vec<T>();
-    }
-    const double Dd = (double)a.D;
+    const double invD = 1.0 / (double)a.D;
     const double eps = (double)a.eps;
+    constexpr bool kPRegs = weights_in_regs(VPT);
+    V16 wv[VPT], bv[VPT];
+    if constexpr (kPRegs) {
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            const int v = t + k * G;
+            const bool in = v < a.nvec;
+            wv[k] = (a.w && in) ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16) : ones_vec<T>();
+            bv[k] = (a.b && in) ? ld_param(static_cast<const char*>(a.b) + (size_t)v * 16) : zeros_vec<T>();
+        }
+    }
 
     int it = 0;
     for (int64_t base = (int64_t)blockIdx.x * a.rows_per_cta; base < a.rows;
@@ -96,44 +150,98 @@ __global__ void __launch_bounds__(layer_max_threads(VPT)) layer_rows_kernel(cons
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
             const int v = t + k * G;
-            if (active && v < a.nvec)
-                xv[k] = ld_stream(static_cast<const char*>(a.x) + roff + (size_t)v * 16);
+            xv[k] = (active && v < a.nvec)
+                        ? ld_stream(static_cast<const char*>(a.x) + roff + (size_t)v * 16)
+                        : zeros_vec<T>();
         }
 
-        double s1 = 0.0;
+        // two independent accumulator chains per sum
+        double s1 = 0.0, s2 = 0.0, s1b = 0.0, s2b = 0.0;
 #pragma unroll
         for (int k = 0; k < VPT; ++k)
-            if (active && t + k * G < a.nvec)
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) s1 += (double)E::get(xv[k], e);
-        const double mean = row_sum_f64(s1, red[(it & 1) * 2], slot, wpr) / Dd;
-
-        double s2 = 0.0;
+            for (int e = 0; e < VEC; e += 2) {
+                const double x0 = (double)E::get(xv[k], e);
+                const double x1 = (double)E::get(xv[k], e + 1);
+                s1 += x0;
+                s1b += x1;
+                s2 = fma(x0, x0, s2);
+                s2b = fma(x1, x1, s2b);
+            }
+        s1 += s1b;
+        s2 += s2b;
+        s1 = warp_sum(s1);
+        s2 = warp_sum(s2);
+        if (wpr > 1) {
+            double* b1 = red[it & 1][0];
+            double* b2 = red[it & 1][1];
+            if ((threadIdx.x & 31) == 0) {
+                b1[threadIdx.x >> 5] = s1;
+                b2[threadIdx.x >> 5] = s2;
+            }
+            __syncthreads();
+            s1 = 0.0;
+            s2 = 0.0;
+            for (int i = 0; i < wpr; ++i) {
+                s1 += b1[i];
+                s2 += b2[i];
+            }
+        }
+        const double mean = s1 * invD;
+        double var = s2 * invD - mean * mean;
+        if (!(var > ldexp(mean * mean, -20))) {
+            // centred second pass (uniform over the row's threads)
+            double c2 = 0.0;
 #pragma unroll
-        for (int k = 0; k < VPT; ++k)
-            if (active && t + k * G < a.nvec)
+            for (int k = 0; k < VPT; ++k)
+                if (t + k * G < a.nvec)
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    const double d = (double)E::get(xv[k], e) - mean;
-                    s2 = fma(d, d, s2);
-                }
-        const double var = row_sum_f64(s2, red[(it & 1) * 2 + 1], slot, wpr) / Dd;
-        const double rstd = 1.0 / sqrt(var + eps);
+                    for (int e = 0; e < VEC; ++e) {
+                        const double dd = (double)E::get(xv[k], e) - mean;
+                        c2 = fma(dd, dd, c2);
+                    }
+            c2 = warp_sum(c2);
+            if (wpr > 1) {
+                __syncthreads();  // every thread has read red[it & 1] above
+                double* b1 = red[it & 1][0];
+                if ((threadIdx.x & 31) == 0) b1[threadIdx.x >> 5] = c2;
+                __syncthreads();
+                c2 = 0.0;
+                for (int i = 0; i < wpr; ++i) c2 += b1[i];
+            }
+            var = c2 * invD;
+        }
+        const double rstd = rsqrt(var + eps);
+        const float mu_hi = __double2float_rn(mean);
+        const float mu_lo = __double2float_rn(mean - (double)mu_hi);
+        LnOut f;
+        f.mu_hi = mu_hi;
+        f.mu_lo = mu_lo;
+        f.rf = __double2float_rn(rstd);
+        // one subtraction unless the dropped mean_lo would flag more than ~2^-16 of the row
+        f.two_sub = 0x1p10f * fabsf(mu_lo) * f.rf > 0x1p-16f;
+        f.kmu = f.two_sub ? 0x1p-37f * fabsf(mu_hi) : 0x1p10f * fabsf(mu_lo);
 
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
             const int v = t + k * G;
             if (active && v < a.nvec) {
+                if constexpr (!kPRegs) {
+                    wv[k] = a.w ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16) : ones_vec<T>();
+                    bv[k] = a.b ? ld_param(static_cast<const char*>(a.b) + (size_t)v * 16) : zeros_vec<T>();
+                }
                 V16 o;
+                bool all_ok = true;
 #pragma unroll
                 for (int e = 0; e < VEC; e += 2) {
-                    const double d0 = (double)E::get(xv[k], e) - mean;
-                    const double d1 = (double)E::get(xv[k], e + 1) - mean;
-                    const double y0 = fma(d0, rstd * (double)E::get(wv[k], e), (double)E::get(bv[k], e));
-                    const double y1 =
-                        fma(d1, rstd * (double)E::get(wv[k], e + 1), (double)E::get(bv[k], e + 1));
-                    put2_f64<T>(o, e, y0, y1);
+                    bool ok0, ok1;
+                    const float y0 = f.y(E::get(xv[k], e), E::get(wv[k], e), E::get(bv[k], e), ok0);
+                    const float y1 =
+                        f.y(E::get(xv[k], e + 1), E::get(wv[k], e + 1), E::get(bv[k], e + 1), ok1);
+                    all_ok = all_ok && ok0 && ok1;
+                    E::put2(o, e, y0, y1);
                 }
+                if (!all_ok) o = fix_near_cancellation<T>(o, f, xv[k], wv[k], bv[k], mean, rstd);
                 st_stream(static_cast<char*>(a.y) + roff + (size_t)v * 16, o);
             }
         }

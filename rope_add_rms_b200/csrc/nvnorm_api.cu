@@ -179,22 +179,26 @@ int pow2_ceil(int v) {
 
 // Largest vectors-per-thread the register kernels are instantiated for, and the
 // largest CTA each instance is built for.
-int max_vpt(Op op) { return op == OP_LAYER ? 4 : 8; }
+int max_vpt(Op) { return 8; }
 int max_threads(Op op, int vpt) {
     return op == OP_LAYER ? layer_max_threads(vpt) : rms_max_threads(vpt);
 }
 
 // Register-path shape: VPT vectors per thread, G threads per row.
+// Automatic choice (measured on B200 over D = 1024..16384, bf16 and fp32): four
+// 16-byte vectors per thread and tensor -- enough loads in flight per thread while
+// keeping several CTAs per SM -- unless the row would then need more threads than
+// the kernel is built for; short rows use fewer vectors so a warp is not mostly idle.
 bool rows_shape(Op op, int nvec, int vpt_req, int g_req, int* vpt, int* G) {
     int v = vpt_req;
     if (v == 0) {
-        // smallest VPT whose row group fits in 256 threads, else in 1024
         v = 0;
-        for (int c = 1; c <= max_vpt(op); c *= 2)
-            if ((nvec + c - 1) / c <= 256) { v = c; break; }
-        if (v == 0)
-            for (int c = 1; c <= max_vpt(op); c *= 2)
+        if (nvec <= 32 * 4) {
+            v = std::max(1, pow2_ceil((nvec + 31) / 32));
+        } else {
+            for (int c = 4; c <= max_vpt(op); c *= 2)
                 if ((nvec + c - 1) / c <= max_threads(op, c)) { v = c; break; }
+        }
         if (v == 0) return false;
     }
     if (v != 1 && v != 2 && v != 4 && v != 8) return false;
@@ -237,9 +241,14 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
                         (long long)D, p.vec_per_thread, p.threads_per_row);
         p.vec_per_thread = vpt;
         p.threads_per_row = G;
-        if (p.rows_per_cta == 0) p.rows_per_cta = std::max(1, std::min(256, max_threads(op, vpt)) / G);
+        // CTAs of at least 128 threads; a layer_norm row spanning several warps is alone
+        if (p.rows_per_cta == 0)
+            p.rows_per_cta = (op == OP_LAYER && G > 32) ? 1 : std::max(1, 128 / G);
         if (p.rows_per_cta * G > max_threads(op, vpt) || p.rows_per_cta < 1)
             return fail(NV_ERR_UNSUPPORTED, "rows_per_cta %d x G %d", p.rows_per_cta, G);
+        if (op == OP_LAYER && G > 32 && p.rows_per_cta != 1)
+            return fail(NV_ERR_UNSUPPORTED, "layer_norm: a row spanning several warps is alone "
+                        "in its CTA (rows_per_cta must be 1)");
     } else if (p.path == NV_PATH_GENERIC) {
         p.vec_per_thread = 0;
         p.threads_per_row = 256;
@@ -312,11 +321,14 @@ nv_status launch_kernel(void (*kernel)(KArgs...), int64_t grid, int block, size_
     return NV_OK;
 }
 
+// ctas_per_sm == 0: one CTA per unit of work (the hardware scheduler balances the
+// tail); > 0: a persistent grid of that many CTAs per SM looping over the units.
 template <typename K>
 nv_status launch(K kernel, int64_t units, int block, size_t smem, int ctas_per_sm,
                  const DevInfo& di, cudaStream_t s, const RowArgs& a) {
-    const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : occupancy(kernel, block, smem);
-    const int64_t grid = grid_for(units, di.sms, per_sm);
+    const int64_t grid =
+        ctas_per_sm > 0 ? grid_for(units, di.sms, ctas_per_sm) : std::min<int64_t>(units, INT32_MAX);
+    (void)smem;
     return launch_kernel(kernel, grid, block, smem, s, a);
 }
 
@@ -370,6 +382,7 @@ nv_status run_layer(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs
         case 1: return launch(layer_rows_kernel<T, 1>, units, block, 0, p.ctas_per_sm, di, s, a);
         case 2: return launch(layer_rows_kernel<T, 2>, units, block, 0, p.ctas_per_sm, di, s, a);
         case 4: return launch(layer_rows_kernel<T, 4>, units, block, 0, p.ctas_per_sm, di, s, a);
+        case 8: return launch(layer_rows_kernel<T, 8>, units, block, 0, p.ctas_per_sm, di, s, a);
     }
     return fail(NV_ERR_UNSUPPORTED, "vec_per_thread %d", p.vec_per_thread);
 }
@@ -440,15 +453,16 @@ nv_status row_op(Op op, const void* x, const void* r, const void* w, const void*
 // ---- norm_rope -------------------------------------------------------------------------------
 struct RopePlan {
     bool rows;
+    bool pairs;  // both halves of the rotation in one lane (dims == D)
     int lpr;
     int bt;
     int64_t n_chunks;
 };
 
 template <typename T, bool TRAD>
-nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a) {
+nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a, bool pairs) {
     const size_t smem = (size_t)a.half * sizeof(float4);
-    auto kern = rope_rows_kernel<T, TRAD>;
+    auto kern = (pairs && !TRAD) ? rope_pairs_kernel<T> : rope_rows_kernel<T, TRAD>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -474,20 +488,25 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
     const int64_t nvec = D / vecw;
     const bool vec_ok = aligned && D % vecw == 0 && nvec <= 32 &&
                         (trad || (dims / 2) % vecw == 0);
-    if (p.path == NV_PATH_AUTO) p.path = vec_ok ? NV_PATH_ROWS : NV_PATH_GENERIC;
+    // both halves per lane: every feature rotated, an even number of vectors
+    const bool pairs_ok = !trad && aligned && D % vecw == 0 && dims == D && nvec % 2 == 0 &&
+                          nvec / 2 <= 32;
+    if (p.path == NV_PATH_AUTO) p.path = (vec_ok || pairs_ok) ? NV_PATH_ROWS : NV_PATH_GENERIC;
     rp->rows = p.path == NV_PATH_ROWS;
+    rp->pairs = rp->rows && pairs_ok && p.vec_per_thread != 1;
     if (p.path == NV_PATH_ROWS) {
-        if (!vec_ok)
+        if (!vec_ok && !rp->pairs)
             return fail(NV_ERR_UNSUPPORTED, "norm_rope register path needs D %% %d == 0, "
                         "D <= %d, 16-byte alignment and (halves) dims/2 %% %d == 0",
                         vecw, 32 * vecw, vecw);
-        const int lpr = pow2_ceil((int)std::max<int64_t>(nvec, 1));
+        const int lanes_needed = rp->pairs ? (int)(nvec / 2) : (int)nvec;
+        const int lpr = pow2_ceil(std::max(lanes_needed, 1));
         const int slots = 256 / lpr;
         const int64_t BH = rows / L;
         int64_t bt = p.rows_per_cta;
         if (bt <= 0) {
             const int64_t target = (rows + 8LL * sms - 1) / (8LL * sms);
-            bt = std::max<int64_t>(slots * 4, std::min<int64_t>(target, 256));
+            bt = std::max<int64_t>(slots * (rp->pairs ? 2 : 4), std::min<int64_t>(target, 256));
             bt = std::min<int64_t>(bt, std::max<int64_t>(BH, 1));
         }
         rp->lpr = lpr;
@@ -495,7 +514,7 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
         rp->n_chunks = (BH + bt - 1) / bt;
         if (L * rp->n_chunks >= ((int64_t)1 << 31))
             return fail(NV_ERR_UNSUPPORTED, "norm_rope grid too large");
-        p.vec_per_thread = 1;
+        p.vec_per_thread = rp->pairs ? 2 : 1;
         p.threads_per_row = lpr;
         p.rows_per_cta = (int)bt;
     } else if (p.path == NV_PATH_GENERIC) {
@@ -576,10 +595,10 @@ nv_status rope_op(const void* x, const void* w, void* y, int64_t rows, int64_t L
     const bool bf = dt == NV_BF16;
     if (rp.rows) {
         if (traditional)
-            return bf ? launch_rope_rows<__nv_bfloat16, true>(di, cs, a)
-                      : launch_rope_rows<float, true>(di, cs, a);
-        return bf ? launch_rope_rows<__nv_bfloat16, false>(di, cs, a)
-                  : launch_rope_rows<float, false>(di, cs, a);
+            return bf ? launch_rope_rows<__nv_bfloat16, true>(di, cs, a, rp.pairs)
+                      : launch_rope_rows<float, true>(di, cs, a, rp.pairs);
+        return bf ? launch_rope_rows<__nv_bfloat16, false>(di, cs, a, rp.pairs)
+                  : launch_rope_rows<float, false>(di, cs, a, rp.pairs);
     }
     return bf ? launch_rope_generic<__nv_bfloat16>(di, p.ctas_per_sm, cs, a)
               : launch_rope_generic<float>(di, p.ctas_per_sm, cs, a);

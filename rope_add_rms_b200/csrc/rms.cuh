@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(rms_max_threads(VPT)) rms_rows_kernel(const Ro
                         : ones_vec<T>();
         }
     }
-    const float Df = (float)a.D;
+    const float invD = 1.0f / (float)a.D;
 
     int it = 0;
     for (int64_t base = (int64_t)blockIdx.x * a.rows_per_cta; base < a.rows;
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(rms_max_threads(VPT)) rms_rows_kernel(const Ro
             const int w0 = slot * wpr;
             for (int i = 0; i < wpr; ++i) ss += buf[w0 + i];
         }
-        const float inv = rsqrtf(__fdiv_rn(ss, Df) + a.eps);
+        const float inv = rsqrtf(__fmaf_rn(ss, invD, a.eps));
 
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(256) rms_generic_kernel(const RowArgs a) {
         __syncthreads();
         ss = 0.f;
         for (int i = 0; i < nw; ++i) ss += buf[i];
-        const float inv = rsqrtf(__fdiv_rn(ss, (float)a.D) + a.eps);
+        const float inv = rsqrtf(__fmaf_rn(ss, 1.0f / (float)a.D, a.eps));
         for (int j = threadIdx.x; j < a.D; j += blockDim.x) {
             const float hv = ADD ? E::load1(a.h, r0 + j) : E::load1(a.x, r0 + j);
             const float wj = a.w ? E::load1(a.w, j) : 1.f;

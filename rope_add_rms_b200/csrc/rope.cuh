@@ -69,6 +69,29 @@ __device__ __forceinline__ float4 angle_entry(double pos, double scale, double b
     return make_float4(ch, __double2float_rn(c - (double)ch), sh, __double2float_rn(s - (double)sh));
 }
 
+// The same on an element pair, in packed float32 arithmetic.
+__device__ __forceinline__ float2 rotate_pair2(float2 a_o, float2 a_t, float2 c_hi, float2 c_lo,
+                                               float2 s_hi, float2 s_lo) {
+    const float2 t1 = mul2(a_t, s_hi);
+    const float2 e1 = fma2(a_t, s_hi, neg2(t1));
+    const float2 z1 = fma2(a_o, c_hi, t1);
+    const float2 c2 = fma2(a_t, s_lo, e1);
+    const float2 c3 = fma2(a_o, c_lo, c2);
+    return add2(z1, c3);
+}
+
+// z = a_o * c - a_t * s on an element pair (the p side of halves pairing with the
+// unsigned table), with the same error-free splitting.
+__device__ __forceinline__ float2 rotate_sub2(float2 a_o, float2 a_t, float2 c_hi, float2 c_lo,
+                                              float2 s_hi, float2 s_lo) {
+    const float2 t1 = mul2(a_t, s_hi);
+    const float2 e1 = fma2(a_t, s_hi, neg2(t1));  // a_t s_hi - t1, exact
+    const float2 z1 = fma2(a_o, c_hi, neg2(t1));
+    const float2 c2 = fma2(a_t, s_lo, e1);
+    const float2 c3 = fma2(a_o, c_lo, neg2(c2));
+    return add2(z1, c3);
+}
+
 // ---- register path ------------------------------------------------------------------
 // One CTA = one position l and a chunk of bt rows (b, h) at that position, so the
 // angle table of l is built once (dims/2 double sincos) and reused by all of them.
@@ -124,21 +147,30 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
         const int64_t b = bh0 + slot + (int64_t)u * slots;
         if (has_vec && b < bh_end) xv[u] = ld_stream(xbase + (size_t)b * lstride);
     }
-    // per-column weights of this lane's elements and of their partners
-    V16 w_own = (norm && a.w && has_vec) ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16)
-                                         : ones_vec<T>();
-    V16 w_par = w_own;
+    // per-column weights of this lane's elements and of their partners, as floats
+    const V16 w_own_v = (norm && a.w && has_vec)
+                            ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16)
+                            : ones_vec<T>();
+    V16 w_par_v = w_own_v;
     if (!TRAD && pv != v && norm && a.w && pv < a.nvec)
-        w_par = ld_param(static_cast<const char*>(a.w) + (size_t)pv * 16);
+        w_par_v = ld_param(static_cast<const char*>(a.w) + (size_t)pv * 16);
+    float2 w_own[VEC / 2], w_par[VEC / 2];
+#pragma unroll
+    for (int e = 0; e < VEC; e += 2) {
+        w_own[e / 2] = E::get2(w_own_v, e);
+        w_par[e / 2] = E::get2(w_par_v, e);
+    }
     __syncthreads();
 
-    // this lane's table entries, sin already carrying the sign of its side
-    float c_hi[VEC], c_lo[VEC], s_hi[VEC], s_lo[VEC];
-    bool rot[VEC];
+    // this lane's table entries, sin already carrying the sign of its side; elements
+    // past dims get the identity (cos 1, sin 0) and the scalar path below
+    float2 c_hi[VEC / 2], c_lo[VEC / 2], s_hi[VEC / 2], s_lo[VEC / 2];
+    bool all_rot = has_vec;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
         const int j = v * VEC + e;
-        rot[e] = has_vec && j < a.dims;
+        const bool r = has_vec && j < a.dims;
+        all_rot = all_rot && r;
         int i = 0;
         float sg = 1.f;
         if (TRAD) {
@@ -148,14 +180,19 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
             i = (j < a.half) ? j : j - a.half;
             sg = (j < a.half) ? -1.f : 1.f;
         }
-        const float4 t4 = rot[e] ? tab[i] : make_float4(1.f, 0.f, 0.f, 0.f);
-        c_hi[e] = t4.x;
-        c_lo[e] = t4.y;
-        s_hi[e] = sg * t4.z;
-        s_lo[e] = sg * t4.w;
+        float4 t4 = make_float4(1.f, 0.f, 0.f, 0.f);
+        if (r) t4 = tab[i];
+        float* ch = reinterpret_cast<float*>(&c_hi[e / 2]);
+        float* cl = reinterpret_cast<float*>(&c_lo[e / 2]);
+        float* sh = reinterpret_cast<float*>(&s_hi[e / 2]);
+        float* sl = reinterpret_cast<float*>(&s_lo[e / 2]);
+        ch[e & 1] = t4.x;
+        cl[e & 1] = t4.y;
+        sh[e & 1] = sg * t4.z;
+        sl[e & 1] = sg * t4.w;
     }
 
-    const float Df = (float)a.D;
+    const float invD = 1.0f / (float)a.D;
     for (int64_t base = bh0; base < bh_end; base += (int64_t)kUnroll * slots) {
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
@@ -166,14 +203,16 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
             const int64_t bn = b + (int64_t)kUnroll * slots;
             if (has_vec && bn < bh_end) xv[u] = ld_stream(xbase + (size_t)bn * lstride);
 
-            float ss = 0.f;
+            float2 x2[VEC / 2];
+            float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-                const float f = E::get(xo, e);
-                ss = fmaf(f, f, ss);
+            for (int e = 0; e < VEC; e += 2) {
+                x2[e / 2] = E::get2(xo, e);
+                ss2 = fma2(x2[e / 2], x2[e / 2], ss2);
             }
-            ss = group_sum(ss, lpr);
-            const float inv = norm ? rsqrtf(__fdiv_rn(ss, Df) + a.eps) : 1.f;
+            const float ss = group_sum(__fadd_rn(ss2.x, ss2.y), lpr);
+            const float inv = norm ? rsqrtf(__fmaf_rn(ss, invD, a.eps)) : 1.f;
+            const float2 inv2 = make_float2(inv, inv);
 
             V16 xp = xo;  // partner words
             if (!TRAD) {
@@ -182,26 +221,163 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
                 for (int q = 0; q < 4; ++q) xp.u[q] = __shfl_sync(0xFFFFFFFFu, xo.u[q], src, lpr);
             }
             if (live) {
-                V16 o;
+                // a = x * w, exact in float32 for bfloat16 data; each product formed once
+                float2 ao[VEC / 2], at[VEC / 2];
 #pragma unroll
                 for (int e = 0; e < VEC; e += 2) {
-                    float yy[2];
+                    ao[e / 2] = mul2(x2[e / 2], w_own[e / 2]);
+                    if (TRAD)
+                        at[e / 2] = make_float2(ao[e / 2].y, ao[e / 2].x);
+                    else
+                        at[e / 2] = mul2(E::get2(xp, e), w_par[e / 2]);
+                }
+                V16 o;
+                if (all_rot) {
 #pragma unroll
-                    for (int d = 0; d < 2; ++d) {
-                        const int ee = e + d;
-                        const float a_o = __fmul_rn(E::get(xo, ee), E::get(w_own, ee));
-                        float z = a_o;
-                        if (rot[ee]) {
-                            const int te = TRAD ? (ee ^ 1) : ee;
-                            const float a_t = TRAD ? __fmul_rn(E::get(xo, te), E::get(w_own, te))
-                                                   : __fmul_rn(E::get(xp, te), E::get(w_par, te));
-                            z = rotate_pair(a_o, a_t, c_hi[ee], c_lo[ee], s_hi[ee], s_lo[ee]);
-                        }
-                        yy[d] = __fmul_rn(z, inv);
+                    for (int e = 0; e < VEC; e += 2) {
+                        const int q = e / 2;
+                        const float2 z =
+                            rotate_pair2(ao[q], at[q], c_hi[q], c_lo[q], s_hi[q], s_lo[q]);
+                        E::put2(o, e, mul2(z, inv2));
                     }
-                    E::put2(o, e, yy[0], yy[1]);
+                } else {
+                    // a vector holding features past dims: those keep a = x * w
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) {
+                        const int q = e / 2;
+                        const float* aof = reinterpret_cast<const float*>(&ao[q]);
+                        const float* atf = reinterpret_cast<const float*>(&at[q]);
+                        const float* ch = reinterpret_cast<const float*>(&c_hi[q]);
+                        const float* cl = reinterpret_cast<const float*>(&c_lo[q]);
+                        const float* sh = reinterpret_cast<const float*>(&s_hi[q]);
+                        const float* sl = reinterpret_cast<const float*>(&s_lo[q]);
+                        const int h = e & 1;
+                        const int j = v * VEC + e;
+                        float z = aof[h];
+                        if (j < a.dims) z = rotate_pair(aof[h], atf[h], ch[h], cl[h], sh[h], sl[h]);
+                        const float y = __fmul_rn(z, inv);
+                        if (h)
+                            E::put2(o, e - 1, E::get(o, e - 1), y);
+                        else
+                            E::put2(o, e, y, 0.f);
+                    }
                 }
                 st_stream(ybase + (size_t)b * lstride, o);
+            }
+        }
+    }
+}
+
+// ---- register path, both halves per lane (halves pairing, dims == D) -----------------------
+// Each lane holds vectors v and v + nvec/2 of a row (16-byte vectors, nvec even).  With
+// halves pairing and dims == D these are exactly the p and q members of the pairs
+// i = v*VEC .. v*VEC + VEC - 1, so the partner of every element is in the lane's own
+// registers (no shuffles) and one table entry serves both of its elements.
+template <typename T>
+__global__ void __launch_bounds__(256) rope_pairs_kernel(const RopeArgs a) {
+    using E = Elem<T>;
+    constexpr int VEC = E::kVec;
+    constexpr int kUnroll = 2;
+    extern __shared__ float4 tab[];  // [half]: (cos_hi, cos_lo, sin_hi, sin_lo)
+
+    const int64_t chunk = blockIdx.x % a.n_chunks;
+    const int64_t l = blockIdx.x / a.n_chunks;
+    const int lpr = a.lpr;
+    const int lane = threadIdx.x & (lpr - 1);
+    const int slot = threadIdx.x / lpr;
+    const int slots = blockDim.x / lpr;
+    const int hvec = a.nvec / 2;
+    const int v0 = lane, v1 = lane + hvec;
+    const bool has_vec = lane < hvec;
+
+    const double pos = (double)(a.offset + l);
+    for (int i = threadIdx.x; i < a.half; i += blockDim.x)
+        tab[i] = angle_entry(pos, (double)a.scale, (double)a.base, i, a.dims);
+    pdl_wait();
+    pdl_release();
+
+    const int64_t bh0 = chunk * (int64_t)a.bt;
+    const int64_t bh_end = min(bh0 + (int64_t)a.bt, a.BH);
+    const size_t row_bytes = (size_t)a.D * sizeof(T);
+    const size_t lstride = (size_t)a.L * row_bytes;
+    const char* xbase = static_cast<const char*>(a.x) + (size_t)l * row_bytes;
+    char* ybase = static_cast<char*>(a.y) + (size_t)l * row_bytes;
+
+    V16 xv[kUnroll][2];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int64_t b = bh0 + slot + (int64_t)u * slots;
+        if (has_vec && b < bh_end) {
+            xv[u][0] = ld_stream(xbase + (size_t)b * lstride + (size_t)v0 * 16);
+            xv[u][1] = ld_stream(xbase + (size_t)b * lstride + (size_t)v1 * 16);
+        }
+    }
+
+    const bool norm = a.normalize != 0;
+    float2 w0[VEC / 2], w1[VEC / 2];
+    {
+        const V16 wa = (norm && a.w && has_vec)
+                           ? ld_param(static_cast<const char*>(a.w) + (size_t)v0 * 16) : ones_vec<T>();
+        const V16 wb = (norm && a.w && has_vec)
+                           ? ld_param(static_cast<const char*>(a.w) + (size_t)v1 * 16) : ones_vec<T>();
+#pragma unroll
+        for (int e = 0; e < VEC; e += 2) {
+            w0[e / 2] = E::get2(wa, e);
+            w1[e / 2] = E::get2(wb, e);
+        }
+    }
+    __syncthreads();
+
+    float2 c_hi[VEC / 2], c_lo[VEC / 2], s_hi[VEC / 2], s_lo[VEC / 2];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        float4 t4 = make_float4(1.f, 0.f, 0.f, 0.f);
+        if (has_vec) t4 = tab[v0 * VEC + e];
+        reinterpret_cast<float*>(&c_hi[e / 2])[e & 1] = t4.x;
+        reinterpret_cast<float*>(&c_lo[e / 2])[e & 1] = t4.y;
+        reinterpret_cast<float*>(&s_hi[e / 2])[e & 1] = t4.z;
+        reinterpret_cast<float*>(&s_lo[e / 2])[e & 1] = t4.w;
+    }
+
+    const float invD = 1.0f / (float)a.D;
+    for (int64_t base = bh0; base < bh_end; base += (int64_t)kUnroll * slots) {
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t b = base + slot + (int64_t)u * slots;
+            const bool live = has_vec && b < bh_end;
+            V16 xa = live ? xv[u][0] : zeros_vec<T>();
+            V16 xb = live ? xv[u][1] : zeros_vec<T>();
+            const int64_t bn = b + (int64_t)kUnroll * slots;
+            if (has_vec && bn < bh_end) {
+                xv[u][0] = ld_stream(xbase + (size_t)bn * lstride + (size_t)v0 * 16);
+                xv[u][1] = ld_stream(xbase + (size_t)bn * lstride + (size_t)v1 * 16);
+            }
+            float2 x0[VEC / 2], x1[VEC / 2];
+            float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int e = 0; e < VEC; e += 2) {
+                x0[e / 2] = E::get2(xa, e);
+                x1[e / 2] = E::get2(xb, e);
+                ss2 = fma2(x0[e / 2], x0[e / 2], ss2);
+                ss2 = fma2(x1[e / 2], x1[e / 2], ss2);
+            }
+            const float ss = group_sum(__fadd_rn(ss2.x, ss2.y), lpr);
+            const float inv = norm ? rsqrtf(__fmaf_rn(ss, invD, a.eps)) : 1.f;
+            const float2 inv2 = make_float2(inv, inv);
+            if (live) {
+                V16 o0, o1;
+#pragma unroll
+                for (int e = 0; e < VEC; e += 2) {
+                    const int q = e / 2;
+                    const float2 a0 = mul2(x0[q], w0[q]);  // exact for bfloat16 data
+                    const float2 a1 = mul2(x1[q], w1[q]);
+                    const float2 z0 = rotate_sub2(a0, a1, c_hi[q], c_lo[q], s_hi[q], s_lo[q]);
+                    const float2 z1 = rotate_pair2(a1, a0, c_hi[q], c_lo[q], s_hi[q], s_lo[q]);
+                    E::put2(o0, e, mul2(z0, inv2));
+                    E::put2(o1, e, mul2(z1, inv2));
+                }
+                st_stream(ybase + (size_t)b * lstride + (size_t)v0 * 16, o0);
+                st_stream(ybase + (size_t)b * lstride + (size_t)v1 * 16, o1);
             }
         }
     }
@@ -236,7 +412,7 @@ __global__ void __launch_bounds__(128) rope_generic_kernel(const RopeArgs a) {
             __syncthreads();
             ss = 0.f;
             for (int i = 0; i < nw; ++i) ss += buf[i];
-            inv = rsqrtf(__fdiv_rn(ss, (float)a.D) + a.eps);
+            inv = rsqrtf(__fmaf_rn(ss, 1.0f / (float)a.D, a.eps));
         }
         const double pos = (double)(a.offset + row % a.L);
         for (int i = threadIdx.x; i < a.half; i += blockDim.x) {

@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(512) rms_staged_kernel(const RowArgs a, const 
                          : ones_vec<T>();
         }
     }
-    const float Df = (float)a.D;
+    const float invD = 1.0f / (float)a.D;
 
     int64_t k = 0;
     for (; k < nmine; ++k) {
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(512) rms_staged_kernel(const RowArgs a, const 
         }
         ss = 0.f;
         for (int i = 0; i < wpr; ++i) ss += buf[i];
-        const float inv = rsqrtf(__fdiv_rn(ss, Df) + a.eps);
+        const float inv = rsqrtf(__fmaf_rn(ss, invD, a.eps));
 #pragma unroll
         for (int kk = 0; kk < VPT; ++kk) {
             const int v = t + kk * G;

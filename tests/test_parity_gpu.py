@@ -270,7 +270,8 @@ def test_layer_norm(rows, D, wb, dt):
 
 
 @pytest.mark.parametrize("plan", [dict(path=nv.PATH_GENERIC)] +
-                         [dict(path=nv.PATH_ROWS, vec_per_thread=v) for v in (1, 2, 4)])
+                         [dict(path=nv.PATH_ROWS, vec_per_thread=v) for v in (1, 2, 4, 8)] +
+                         [dict(path=nv.PATH_ROWS, vec_per_thread=4, ctas_per_sm=2)])
 def test_layer_norm_every_variant(plan):
     inp = synth.layer_norm_inputs(211, 4096, "bf16", seed=2)
     x = dev(inp["x"])
@@ -278,6 +279,19 @@ def test_layer_norm_every_variant(plan):
     nv.nv_layer_norm(x, dev(inp["w"]), dev(inp["b"]), y, 1e-5, plan=nv.Plan(**plan))
     torch.cuda.synchronize()
     check_out(y, oracle.layer_norm(host(inp["x"]), host(inp["w"]), host(inp["b"]), 1e-5))
+
+
+@pytest.mark.parametrize("dt,mean,std", [("f32", 1e4, 1.0), ("f32", -3e5, 0.01), ("bf16", 3000.0, 40.0),
+                                          ("bf16", 3000.0, 0.25), ("f32", 0.0, 1e-30)])
+def test_layer_norm_mean_far_from_zero(dt, mean, std):
+    """|mean| >> std takes the centred second pass of the statistics."""
+    for D in (4096, 64):
+        x = synth.normal((33, D), mean, std, 1, 0, dt)
+        w = synth.uniform((D,), 0.5, 1.5, 1, 2, dt)
+        b = synth.normal((D,), 0.0, 0.1, 1, 3, dt)
+        y = nv.layer_norm(x.cuda(), w.cuda(), b.cuda(), eps=1e-5)
+        torch.cuda.synchronize()
+        check_out(y, oracle.layer_norm(host(x), host(w), host(b), 1e-5))
 
 
 def test_layer_norm_in_place_and_large_mean():
@@ -337,18 +351,27 @@ def test_norm_rope_base_and_scale(trad):
     check_out(y, ref)
 
 
-def test_norm_rope_generic_path_matches_register_path():
-    inp = synth.norm_rope_inputs(2, 4, 64, 128, "bf16", seed=1)
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("D", [128, 64, 256])
+def test_norm_rope_every_variant(D, dt):
+    """Generic path, one vector per lane, both halves per lane (halves, dims == D)."""
+    inp = synth.norm_rope_inputs(2, 4, 64, D, dt, seed=1)
     x, w = dev(inp["x"]), dev(inp["w"])
-    ys = []
-    for path in (nv.PATH_ROWS, nv.PATH_GENERIC):
-        y = torch.empty_like(x)
-        nv.nv_norm_rope(x, w, y, 64, 128, 0, 10000.0, 1.0, 4096, 1, 1e-6, plan=nv.Plan(path=path))
-        ys.append(y)
-    torch.cuda.synchronize()
-    ref = oracle.norm_rope(host(inp["x"]), host(inp["w"]), 64, 128, 0, 10000.0, 1.0, 4096, 1, 1e-6)
-    for y in ys:
-        check_out(y, ref)
+    plans = [dict(path=nv.PATH_GENERIC), dict(path=nv.PATH_ROWS, vec_per_thread=1),
+             dict(path=nv.PATH_ROWS, vec_per_thread=2), dict(path=nv.PATH_ROWS, rows_per_cta=3)]
+    for trad in (0, 1):
+        ref = oracle.norm_rope(host(inp["x"]), host(inp["w"]), 64, D, trad, 10000.0, 1.0, 4096,
+                               1, 1e-6)
+        for p in plans:
+            y = torch.empty_like(x)
+            try:
+                nv.nv_norm_rope(x, w, y, 64, D, trad, 10000.0, 1.0, 4096, 1, 1e-6,
+                                plan=nv.Plan(**p))
+            except nv.NvError as e:
+                assert e.status == nv.NV_ERR_UNSUPPORTED
+                continue
+            torch.cuda.synchronize()
+            check_out(y, ref, f"{p} trad={trad}")
 
 
 def test_norm_rope_in_place():
