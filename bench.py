@@ -17,9 +17,9 @@ Multi-GPU (torchrun, one process per GPU): rows are independent, so every rank r
 own batch of the same shape (weak scaling); there is no data-path collective.  The
 reported time is the maximum over ranks of the summed per-step device times.
 
-``--impl reference`` times the CPU oracle (the only reference that exists for this
-path: the pages publish no implementation or numbers) on a bounded sample of the same
-workload, on rank 0 only.
+``--impl reference`` times the CPU oracle on a bounded sample of the same workload, on
+rank 0 only: the published description of these ops comes with no implementation and no
+measurements, so the oracle is the only reference there is.
 """
 from __future__ import annotations
 
@@ -44,9 +44,8 @@ METRIC = "add_rms_norm achieved HBM GB/s and rows/s vs 8 TB/s peak (1×B200)"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 WORKLOAD = {"rows": 8192, "D": 4096, "dtype": "bf16", "eps": 1e-5}
-KERNEL_SOURCES = ["rope_add_rms_b200/csrc/rms.cuh", "rope_add_rms_b200/csrc/common.cuh",
-                  "rope_add_rms_b200/csrc/layer.cuh", "rope_add_rms_b200/csrc/rope.cuh",
-                  "rope_add_rms_b200/csrc/nvnorm_api.cu"]
+# sources of the timed kernel: recorded ncu traffic is void once these change
+KERNEL_SOURCES = ["rope_add_rms_b200/csrc/rms.cuh", "rope_add_rms_b200/csrc/common.cuh"]
 
 
 # ---- environment --------------------------------------------------------------------
@@ -74,8 +73,9 @@ def source_hash():
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key):
-    """dram bytes per launch recorded from an ncu capture, if the kernels are unchanged."""
+def ncu_traffic(kernel_key, plan):
+    """dram bytes per launch recorded from an ncu capture, if neither the kernel's
+    sources nor its launch plan have changed since."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -83,7 +83,7 @@ def ncu_traffic(kernel_key):
     except (OSError, ValueError):
         return None
     ent = d.get(kernel_key)
-    if not ent or ent.get("source_hash") != source_hash():
+    if not ent or ent.get("source_hash") != source_hash() or ent.get("plan") != plan:
         return None
     return ent.get("bytes_per_launch")
 
@@ -144,6 +144,28 @@ class ClockSampler:
                           if v.lower() == "active"})
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(r[1] for r in rows),
                 "reasons": reasons, "samples": len(rows)}
+
+
+# ---- ranks ------------------------------------------------------------------------------
+
+def shard_seed(rank: int) -> int:
+    """Each rank runs its own batch of rows (weak scaling): rank r's inputs use seed r."""
+    return rank
+
+
+def max_over_ranks(values, device="cuda"):
+    """Element-wise maximum over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, step_bytes: int, steps: int, max_ms: float) -> float:
+    """Whole-job GB/s: the bytes all ranks processed over the slowest rank's time."""
+    return world * step_bytes * steps / (max_ms * 1e-3) / 1e9
 
 
 # ---- workloads ----------------------------------------------------------------------
@@ -398,8 +420,8 @@ def run_ours(args):
     import rope_add_rms_b200 as nv
     nv.library()
 
-    case = Case("add_rms_norm", (WORKLOAD["rows"], WORKLOAD["D"]), WORKLOAD["dtype"], seed=rank,
-                eps=WORKLOAD["eps"])
+    case = Case("add_rms_norm", (WORKLOAD["rows"], WORKLOAD["D"]), WORKLOAD["dtype"],
+                seed=shard_seed(rank), eps=WORKLOAD["eps"])
     flush = l2_flush_buffer()
 
     def barrier():
@@ -420,10 +442,7 @@ def run_ours(args):
     te = time_steps(case, e2e_steps, 3, flush, e2e=True)
     barrier()
     e2e_ms = sum(te)
-    if pg:
-        t = torch.tensor([total_ms, e2e_ms], device="cuda", dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms, e2e_ms = t.tolist()
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms])
 
     extras = None
     if rank == 0 and not args.no_extras and world == 1:
@@ -435,11 +454,11 @@ def run_ours(args):
     if rank == 0:
         peak, peak_kind = measured_peak()
         step_bytes = case.bytes
-        value = world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9
+        value = job_throughput(world, step_bytes, args.steps, total_ms)
         per_launch_ms = total_ms / args.steps      # average launch duration, back to back
         achieved = step_bytes / (per_launch_ms * 1e-3) / 1e9
         bi, bo = case.e2e_bytes()
-        e2e_value = world * step_bytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
+        e2e_value = job_throughput(world, step_bytes, e2e_steps, e2e_ms)
         plan = nv.nv_describe_plan("add_rms_norm", WORKLOAD["rows"], WORKLOAD["D"],
                                    torch.bfloat16)
         line = {
@@ -464,7 +483,7 @@ def run_ours(args):
             "frac_of_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": ncu_traffic("add_rms_norm_bf16_8192x4096"),
+                         "traffic": ncu_traffic("add_rms_norm_bf16_8192x4096", plan),
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_kind == "measured" else "fallback 6650 GB/s",
                          "kernel": f"rms_rows_kernel<bf16, VPT={plan['vec_per_thread']}, ADD>",
@@ -483,6 +502,37 @@ def run_ours(args):
     if pg:
         pg.barrier()
         pg.destroy_process_group()
+    return 0
+
+
+WORKLOADS = {
+    "add_rms_norm": lambda: Case("add_rms_norm", (8192, 4096), "bf16", 0, eps=1e-5),
+    "rms_norm_small": lambda: Case("rms_norm", (64, 512), "f32", 0, eps=1e-6),
+    "layer_norm": lambda: Case("layer_norm", (16384, 8192), "bf16", 0, eps=1e-5),
+    "norm_rope_halves": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,
+                                     dims=128, traditional=0, base=10000.0, scale=1.0, offset=0),
+    "norm_rope_traditional": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,
+                                          dims=128, traditional=1, base=10000.0, scale=1.0,
+                                          offset=4096),
+}
+
+
+def run_workload(args):
+    """One named workload (not the headline metric): GB/s of algorithmic bytes."""
+    torch.cuda.set_device(dist_env()[2])
+    c = WORKLOADS[args.workload]()
+    flush = l2_flush_buffer()
+    peak, _ = measured_peak()
+    if c.rotating:
+        ms = time_span(c, args.steps, args.warmup) / args.steps
+    else:
+        ms = statistics.median(time_steps(c, args.steps, args.warmup, flush))
+    gbs = c.bytes / (ms * 1e-3) / 1e9
+    print(json.dumps({"workload": args.workload, "op": c.op, "rows": c.rows, "D": c.D,
+                      "dtype": c.dtype, "us_per_call": round(ms * 1e3, 3), "GB/s": round(gbs, 1),
+                      "frac_of_measured_hbm": round(gbs / peak, 4),
+                      "rows_per_s": round(c.rows / (ms * 1e-3), 1), "l2": c.l2_note()}),
+          flush=True)
     return 0
 
 
@@ -517,6 +567,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
+                    help="time one named workload instead of the headline step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -526,6 +578,8 @@ def main():
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.workload:
+        return run_workload(args)
     return run_ours(args)
 
 

@@ -193,10 +193,13 @@ bool rows_shape(Op op, int nvec, int vpt_req, int g_req, int* vpt, int* G) {
     int v = vpt_req;
     if (v == 0) {
         v = 0;
-        if (nvec <= 32 * 4) {
+        // layer_norm does more arithmetic per element and gains from longer rows per
+        // thread (eight vectors); the rms kernels from more threads (four)
+        const int pref = op == OP_LAYER ? 8 : 4;
+        if (nvec <= 32 * pref) {
             v = std::max(1, pow2_ceil((nvec + 31) / 32));
         } else {
-            for (int c = 4; c <= max_vpt(op); c *= 2)
+            for (int c = pref; c <= max_vpt(op); c *= 2)
                 if ((nvec + c - 1) / c <= max_threads(op, c)) { v = c; break; }
         }
         if (v == 0) return false;

@@ -44,6 +44,28 @@ def uniform(shape, lo, hi, seed, k, dtype="bf16") -> torch.Tensor:
     return t.to(DTYPES[dtype])
 
 
+def normal_device(shape, mean, std, seed, k, dtype="bf16", device="cuda") -> torch.Tensor:
+    """N(mean, std^2) drawn by torch's generator on `device` (for inputs too large to
+    draw on the host quickly), float32, rounded to ``dtype``."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) + int(k))
+    t = torch.randn(tuple(shape), generator=g, dtype=torch.float32, device=device)
+    if std != 1.0:
+        t.mul_(std)
+    if mean != 0.0:
+        t.add_(mean)
+    return t.to(DTYPES[dtype])
+
+
+def uniform_device(shape, lo, hi, seed, k, dtype="bf16", device="cuda") -> torch.Tensor:
+    """U(lo, hi) drawn by torch's generator on `device`, rounded to ``dtype``."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) + int(k))
+    t = torch.rand(tuple(shape), generator=g, dtype=torch.float32, device=device)
+    t.mul_(hi - lo).add_(lo)
+    return t.to(DTYPES[dtype])
+
+
 def to_numpy(t: torch.Tensor) -> np.ndarray:
     """The oracle's view of a CPU tensor: bfloat16 as raw uint16 bits, float32 as is."""
     t = t.contiguous()

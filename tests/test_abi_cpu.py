@@ -138,9 +138,10 @@ def test_plain_rope_ignores_eps():
     ("rms_norm", 512, "f32", dict(path=1, vec_per_thread=4, threads_per_row=32, rows_per_cta=4)),
     ("layer_norm", 512, "bf16", dict(path=1, vec_per_thread=2, threads_per_row=32, rows_per_cta=4)),
     ("layer_norm", 1024, "bf16", dict(path=1, vec_per_thread=4, threads_per_row=32, rows_per_cta=4)),
-    ("layer_norm", 2048, "bf16", dict(path=1, vec_per_thread=4, threads_per_row=64, rows_per_cta=1)),
-    ("layer_norm", 8192, "bf16", dict(path=1, vec_per_thread=4, threads_per_row=256)),
-    ("norm_rope", 128, "bf16", dict(path=1, vec_per_thread=1, threads_per_row=16)),
+    ("layer_norm", 2048, "bf16", dict(path=1, vec_per_thread=8, threads_per_row=32, rows_per_cta=4)),
+    ("layer_norm", 4096, "bf16", dict(path=1, vec_per_thread=8, threads_per_row=64, rows_per_cta=1)),
+    ("layer_norm", 8192, "bf16", dict(path=1, vec_per_thread=8, threads_per_row=128)),
+    ("norm_rope", 128, "bf16", dict(path=1, vec_per_thread=2, threads_per_row=8)),
     ("norm_rope", 1000, "bf16", dict(path=2)),
 ])
 def test_plan_selection(op, D, dtype, want):

@@ -1,0 +1,105 @@
+"""GPU parity at the benchmark workloads' full sizes, in the launch configuration the
+benchmark times (automatic plan, programmatic dependent launch).
+
+Element-by-element against the CPU oracle for:
+  - add_rms_norm bf16, x and r [8192, 4096] ~ N(0,1), w ~ U(0.5,1.5), eps 1e-5
+  - layer_norm bf16, x [16384, 8192] ~ N(0.5, 2^2), w ~ U(0.5,1.5), b ~ N(0, 0.1^2), eps 1e-5
+  - norm_rope bf16, x [8, 32, 2048, 128] ~ N(0,1), w ~ U(0.5,1.5), eps 1e-6, dims 128,
+    base 10000, scale 1: halves at offset 0, and traditional at offset 4096
+and on sampled rows for the add_rms_norm sweep D x rows x {bf16, f32} (eps 1e-6).
+Large outputs are compared in row chunks to bound host memory.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rope_add_rms_b200 as nv
+from rope_add_rms_b200 import synth
+from checks import check_bf16, check_exact, check_f32, sample_rows, to_host_bits
+
+pytestmark = pytest.mark.gpu
+
+CHUNK = 2048
+
+
+def host(t):
+    return None if t is None else synth.to_numpy(t)
+
+
+def compare_rows(y_dev, ref_fn, rows, what):
+    """Compare the device output with ref_fn(r0, r1) row chunk by row chunk."""
+    for r0 in range(0, rows, CHUNK):
+        r1 = min(rows, r0 + CHUNK)
+        got = to_host_bits(y_dev[r0:r1])
+        ref = ref_fn(r0, r1)
+        if got.dtype == np.uint16:
+            check_bf16(got, ref, f"{what} rows {r0}:{r1}")
+        else:
+            check_f32(got, ref, f"{what} rows {r0}:{r1}")
+
+
+def test_add_rms_norm_bf16_8192x4096():
+    inp = synth.add_rms_inputs(8192, 4096, "bf16", seed=0)
+    x, r, w = (inp[k].cuda() for k in ("x", "r", "w"))
+    y, h = nv.add_rms_norm(x, r, w, eps=1e-5)
+    torch.cuda.synchronize()
+    xh, rh, wh = host(inp["x"]), host(inp["r"]), host(inp["w"])
+    href_all = []
+
+    def ref(r0, r1):
+        yr, hr = oracle.add_rms_norm(xh[r0:r1], rh[r0:r1], wh, 1e-5)
+        href_all.append(hr)
+        return yr
+
+    compare_rows(y, ref, 8192, "y")
+    check_exact(h, np.concatenate(href_all), "h")
+
+
+def test_layer_norm_bf16_16384x8192():
+    inp = synth.layer_norm_inputs(16384, 8192, "bf16", seed=0)
+    x, w, b = (inp[k].cuda() for k in ("x", "w", "b"))
+    y = nv.layer_norm(x, w, b, eps=1e-5)
+    torch.cuda.synchronize()
+    xh, wh, bh = host(inp["x"]), host(inp["w"]), host(inp["b"])
+    compare_rows(y, lambda r0, r1: oracle.layer_norm(xh[r0:r1], wh, bh, 1e-5), 16384, "y")
+
+
+@pytest.mark.parametrize("trad,offset", [(0, 0), (1, 4096)])
+def test_norm_rope_bf16_8x32x2048x128(trad, offset):
+    B, H, L, D = 8, 32, 2048, 128
+    inp = synth.norm_rope_inputs(B, H, L, D, "bf16", seed=0)
+    x, w = inp["x"].cuda(), inp["w"].cuda()
+    y = nv.norm_rope(x.view(B, H, L, D), w, dims=D, traditional=bool(trad), base=10000.0,
+                     scale=1.0, offset=offset, eps=1e-6).view(-1, D)
+    torch.cuda.synchronize()
+    xh, wh = host(inp["x"]), host(inp["w"])
+    # row chunks are whole multiples of L, so l = k mod L is preserved
+    compare_rows(y, lambda r0, r1: oracle.norm_rope(xh[r0:r1], wh, L, D, trad, 10000.0, 1.0,
+                                                    offset, 1, 1e-6), B * H * L, "y")
+
+
+SWEEP = [(dt, D, rows) for dt in ("bf16", "f32") for D in (2048, 4096, 5120, 8192, 16384)
+         for rows in (1, 16, 256, 4096, 65536)]
+
+
+@pytest.mark.parametrize("dt,D,rows", SWEEP, ids=lambda v: str(v))
+def test_add_rms_norm_sweep(dt, D, rows):
+    seed = 0
+    if rows * D <= 4096 * 4096:
+        inp = synth.add_rms_inputs(rows, D, dt, seed)
+        x, r, w = (inp[k].cuda() for k in ("x", "r", "w"))
+    else:   # drawn on the device: hundreds of millions of values
+        x = synth.normal_device((rows, D), 0.0, 1.0, seed, synth.X, dt)
+        r = synth.normal_device((rows, D), 0.0, 1.0, seed, synth.R, dt)
+        w = synth.uniform_device((D,), 0.5, 1.5, seed, synth.W, dt)
+    y, h = nv.add_rms_norm(x, r, w, eps=1e-6)
+    torch.cuda.synchronize()
+    idx = torch.as_tensor(sample_rows(rows, 384, seed=D + rows), device="cuda")
+    xs, rs, ws = to_host_bits(x[idx]), to_host_bits(r[idx]), to_host_bits(w)
+    ref, href = oracle.add_rms_norm(xs, rs, ws, 1e-6)
+    check_exact(h[idx], href, "h")
+    got = to_host_bits(y[idx])
+    (check_bf16 if dt == "bf16" else check_f32)(got, ref, "y")
+    del x, r, y, h
+    torch.cuda.empty_cache()
