@@ -155,8 +155,8 @@ typedef enum {
     NV_PATH_ROWS = 1,    /* row held in registers, 16-byte vector loads */
     NV_PATH_GENERIC = 2, /* any D and alignment: scalar loop, two passes over the row */
     NV_PATH_STAGED = 3   /* persistent, rows staged in shared memory by bulk async copies;
-                            rms_norm and add_rms_norm only.  rows_per_cta = rows in flight
-                            per CTA (shared-memory stages), ctas_per_sm = CTAs per SM */
+                            rms_norm, add_rms_norm and layer_norm.  rows_per_cta = rows in
+                            flight per CTA (shared-memory stages), ctas_per_sm = CTAs per SM */
 } nv_path;
 
 typedef enum { NV_LAUNCH_DEFAULT = 0, NV_LAUNCH_PLAIN = 1 } nv_launch;

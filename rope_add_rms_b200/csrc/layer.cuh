@@ -58,39 +58,20 @@ __device__ __forceinline__ double row_sum_f64(double v, double* buf, int slot, i
     return v;
 }
 
-// Float32 output of one element and whether it passes the error test above.
-struct LnOut {
-    float mu_hi, mu_lo, rf, kmu;
-    bool two_sub;
-    __device__ __forceinline__ float y(float x, float w, float b, bool& ok) const {
-        const float A = __fmul_rn(rf, w);
-        const float d = two_sub ? __fsub_rn(__fsub_rn(x, mu_hi), mu_lo) : __fsub_rn(x, mu_hi);
-        const float v = __fmaf_rn(d, A, b);
-        ok = fabsf(v) > __fmaf_rn(kmu, fabsf(A), 0x1p-11f * fabsf(b));
-        return v;
-    }
-};
-
-// Recompute the elements of one output vector that fail the error test, in double
-// precision: y = (x - mean) * (rstd * w) + b, then round (via float32) to the I/O type.
+// Recompute one output vector in double precision, y = (x - mean) * (rstd * w) + b,
+// rounded (via float32) to the I/O type.  Called for the rare vectors holding an
+// element that fails the float32 error test.
 template <typename T>
-__device__ __noinline__ V16 fix_near_cancellation(V16 o, const LnOut f, V16 xv, V16 wv, V16 bv,
-                                                  double mean, double rstd) {
+__device__ __forceinline__ V16 layer_vector_f64(V16 xv, V16 wv, V16 bv, double mean, double rstd) {
     using E = Elem<T>;
+    V16 o;
 #pragma unroll 1
-    for (int e = 0; e < E::kVec; ++e) {
-        bool ok;
-        f.y(E::get(xv, e), E::get(wv, e), E::get(bv, e), ok);
-        if (ok) continue;
-        const double y = fma((double)E::get(xv, e) - mean, rstd * (double)E::get(wv, e),
-                             (double)E::get(bv, e));
-        const int e0 = e & ~1;
-        const float keep = E::get(o, e0 ^ (e & 1) ^ 1);  // the other element of the pair
-        const float yf = __double2float_rn(y);
-        if (e & 1)
-            E::put2(o, e0, keep, yf);
-        else
-            E::put2(o, e0, yf, keep);
+    for (int e = 0; e < E::kVec; e += 2) {
+        const double y0 = fma((double)E::get(xv, e) - mean, rstd * (double)E::get(wv, e),
+                              (double)E::get(bv, e));
+        const double y1 = fma((double)E::get(xv, e + 1) - mean, rstd * (double)E::get(wv, e + 1),
+                              (double)E::get(bv, e + 1));
+        E::put2(o, e, __double2float_rn(y0), __double2float_rn(y1));
     }
     return o;
 }
@@ -214,13 +195,15 @@ __global__ void __launch_bounds__(layer_max_threads(VPT)) layer_rows_kernel(cons
         const double rstd = rsqrt(var + eps);
         const float mu_hi = __double2float_rn(mean);
         const float mu_lo = __double2float_rn(mean - (double)mu_hi);
-        LnOut f;
-        f.mu_hi = mu_hi;
-        f.mu_lo = mu_lo;
-        f.rf = __double2float_rn(rstd);
-        // one subtraction unless the dropped mean_lo would flag more than ~2^-16 of the row
-        f.two_sub = 0x1p10f * fabsf(mu_lo) * f.rf > 0x1p-16f;
-        f.kmu = f.two_sub ? 0x1p-37f * fabsf(mu_hi) : 0x1p10f * fabsf(mu_lo);
+        const float rf = __double2float_rn(rstd);
+        // d = (x - mean_hi) + nlo: nlo = -mean_lo for rows whose mean is large against
+        // their spread, else +0 (exact); kmu is the matching mean-error term of the test
+        const bool two_sub = 0x1p10f * fabsf(mu_lo) * rf > 0x1p-16f;
+        const float kmu = two_sub ? 0x1p-37f * fabsf(mu_hi) : 0x1p10f * fabsf(mu_lo);
+        const float2 rf2 = make_float2(rf, rf);
+        const float2 nhi2 = make_float2(-mu_hi, -mu_hi);
+        const float nlo = two_sub ? -mu_lo : 0.f;
+        const float2 nlo2 = make_float2(nlo, nlo);
 
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
@@ -234,14 +217,17 @@ __global__ void __launch_bounds__(layer_max_threads(VPT)) layer_rows_kernel(cons
                 bool all_ok = true;
 #pragma unroll
                 for (int e = 0; e < VEC; e += 2) {
-                    bool ok0, ok1;
-                    const float y0 = f.y(E::get(xv[k], e), E::get(wv[k], e), E::get(bv[k], e), ok0);
-                    const float y1 =
-                        f.y(E::get(xv[k], e + 1), E::get(wv[k], e + 1), E::get(bv[k], e + 1), ok1);
-                    all_ok = all_ok && ok0 && ok1;
-                    E::put2(o, e, y0, y1);
+                    const float2 w2 = E::get2(wv[k], e);
+                    const float2 b2 = E::get2(bv[k], e);
+                    const float2 A2 = mul2(rf2, w2);
+                    const float2 d2 = add2(add2(E::get2(xv[k], e), nhi2), nlo2);
+                    const float2 y2 = fma2(d2, A2, b2);
+                    // bitwise: no short-circuit branches in the unrolled loop
+                    all_ok &= (fabsf(y2.x) > __fmaf_rn(kmu, fabsf(A2.x), 0x1p-11f * fabsf(b2.x))) &
+                              (fabsf(y2.y) > __fmaf_rn(kmu, fabsf(A2.y), 0x1p-11f * fabsf(b2.y)));
+                    E::put2(o, e, y2);
                 }
-                if (!all_ok) o = fix_near_cancellation<T>(o, f, xv[k], wv[k], bv[k], mean, rstd);
+                if (!all_ok) o = layer_vector_f64<T>(xv[k], wv[k], bv[k], mean, rstd);
                 st_stream(static_cast<char*>(a.y) + roff + (size_t)v * 16, o);
             }
         }

@@ -257,8 +257,6 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
         p.threads_per_row = 256;
         p.rows_per_cta = 1;
     } else if (p.path == NV_PATH_STAGED) {
-        if (op == OP_LAYER)
-            return fail(NV_ERR_UNSUPPORTED, "the staged path covers rms_norm and add_rms_norm");
         if (!vec_ok) return fail(NV_ERR_UNSUPPORTED, "staged path needs D %% %d == 0 and "
                                  "16-byte aligned pointers", vecw);
         int vpt = 0, G = 0;
@@ -377,6 +375,17 @@ template <typename T>
 nv_status run_layer(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs a) {
     if (p.path == NV_PATH_GENERIC)
         return launch(layer_generic_kernel<T>, a.rows, 256, 0, p.ctas_per_sm, di, s, a);
+    if (p.path == NV_PATH_STAGED) {
+        const size_t smem = staged_smem(OP_LAYER, a.D, sizeof(T) == 4 ? NV_F32 : NV_BF16,
+                                        p.rows_per_cta);
+        switch (p.vec_per_thread) {
+            case 1: return launch_staged(layer_staged_kernel<T, 1>, p, smem, di, s, a);
+            case 2: return launch_staged(layer_staged_kernel<T, 2>, p, smem, di, s, a);
+            case 4: return launch_staged(layer_staged_kernel<T, 4>, p, smem, di, s, a);
+            case 8: return launch_staged(layer_staged_kernel<T, 8>, p, smem, di, s, a);
+        }
+        return fail(NV_ERR_UNSUPPORTED, "vec_per_thread %d", p.vec_per_thread);
+    }
     a.G = p.threads_per_row;
     a.rows_per_cta = p.rows_per_cta;
     const int block = a.G * a.rows_per_cta;

@@ -24,6 +24,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "layer.cuh"
 #include "rms.cuh"
 
 namespace nvn {
@@ -232,6 +233,169 @@ __global__ void __launch_bounds__(512) rms_staged_kernel(const RowArgs a, const 
                 mbar_wait_bounded(bbase + 8u * (uint32_t)(j % stages),
                                   (uint32_t)((j / stages) & 1));
         }
+    }
+}
+
+// ---- layer_norm, staged ------------------------------------------------------------
+// Same arithmetic as layer_rows_kernel (double statistics from one widening per
+// element, float32 output with the error test and the double recompute), but the row
+// lives in a shared-memory stage filled by a bulk copy instead of in registers: each
+// thread reads its vectors from the stage in the statistics pass and again in the
+// output pass.  Registers then hold no row data across the reduction, so more warps fit
+// per SM, and the copies of the next `stages - 1` rows are in flight meanwhile.  Two
+// barriers per row: the reduction's, and one after the output pass that frees the stage.
+template <typename T, int VPT>
+__global__ void __launch_bounds__(512) layer_staged_kernel(const RowArgs a, const int stages) {
+    pdl_wait();
+    pdl_release();
+    using E = Elem<T>;
+    constexpr int VEC = E::kVec;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ double red[2][3][16];
+    __shared__ int abort_flag;
+
+    const int G = blockDim.x;
+    const int t = threadIdx.x;
+    const int wpr = G >> 5;
+    const uint32_t row_bytes = (uint32_t)a.nvec * 16u;
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t bbase = sbase + (uint32_t)stages * row_bytes;
+    const int64_t first = blockIdx.x;
+    const int64_t stride = gridDim.x;
+    const int64_t nmine = first < a.rows ? (a.rows - 1 - first) / stride + 1 : 0;
+
+    if (t == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < stages; ++s) mbar_init(bbase + 8u * s, 1);
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+    auto issue = [&](int64_t k) {
+        const int s = (int)(k % stages);
+        const int64_t row = first + k * stride;
+        const uint32_t bar = bbase + 8u * s;
+        mbar_arrive_expect_tx(bar, row_bytes);
+        bulk_load(sbase + (uint32_t)s * row_bytes,
+                  static_cast<const char*>(a.x) + (size_t)row * row_bytes, row_bytes, bar);
+    };
+    if (t == 0)
+        for (int64_t k = 0; k < nmine && k < stages; ++k) issue(k);
+
+    const double invD = 1.0 / (double)a.D;
+    const double eps = (double)a.eps;
+
+    int64_t k = 0;
+    for (; k < nmine; ++k) {
+        const int s = (int)(k % stages);
+        if (!mbar_wait_bounded(bbase + 8u * s, (uint32_t)((k / stages) & 1))) abort_flag = 1;
+        const unsigned char* stg = smem + (size_t)s * row_bytes;
+        const int64_t row = first + k * stride;
+        const size_t roff = (size_t)row * row_bytes;
+
+        double s1 = 0.0, s2 = 0.0, s1b = 0.0, s2b = 0.0;
+#pragma unroll
+        for (int kk = 0; kk < VPT; ++kk) {
+            const int v = t + kk * G;
+            if (v < a.nvec) {
+                const V16 xv = ld_shared16(stg + (size_t)v * 16);
+#pragma unroll
+                for (int e = 0; e < VEC; e += 2) {
+                    const double x0 = (double)E::get(xv, e);
+                    const double x1 = (double)E::get(xv, e + 1);
+                    s1 += x0;
+                    s1b += x1;
+                    s2 = fma(x0, x0, s2);
+                    s2b = fma(x1, x1, s2b);
+                }
+            }
+        }
+        s1 = warp_sum(s1 + s1b);
+        s2 = warp_sum(s2 + s2b);
+        double(*buf)[16] = red[k & 1];
+        if ((t & 31) == 0) {
+            buf[0][t >> 5] = s1;
+            buf[1][t >> 5] = s2;
+        }
+        __syncthreads();
+        if (abort_flag) break;
+        s1 = 0.0;
+        s2 = 0.0;
+        for (int i = 0; i < wpr; ++i) {
+            s1 += buf[0][i];
+            s2 += buf[1][i];
+        }
+        const double mean = s1 * invD;
+        double var = s2 * invD - mean * mean;
+        if (!(var > ldexp(mean * mean, -20))) {   // CTA-uniform: one row per CTA
+            double c2 = 0.0;
+#pragma unroll
+            for (int kk = 0; kk < VPT; ++kk) {
+                const int v = t + kk * G;
+                if (v < a.nvec) {
+                    const V16 xv = ld_shared16(stg + (size_t)v * 16);
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) {
+                        const double dd = (double)E::get(xv, e) - mean;
+                        c2 = fma(dd, dd, c2);
+                    }
+                }
+            }
+            c2 = warp_sum(c2);
+            if ((t & 31) == 0) buf[2][t >> 5] = c2;
+            __syncthreads();
+            c2 = 0.0;
+            for (int i = 0; i < wpr; ++i) c2 += buf[2][i];
+            var = c2 * invD;
+        }
+        const double rstd = rsqrt(var + eps);
+        const float mu_hi = __double2float_rn(mean);
+        const float mu_lo = __double2float_rn(mean - (double)mu_hi);
+        const float rf = __double2float_rn(rstd);
+        const bool two_sub = 0x1p10f * fabsf(mu_lo) * rf > 0x1p-16f;
+        const float kmu = two_sub ? 0x1p-37f * fabsf(mu_hi) : 0x1p10f * fabsf(mu_lo);
+        const float2 rf2 = make_float2(rf, rf);
+        const float2 nhi2 = make_float2(-mu_hi, -mu_hi);
+        const float nlo = two_sub ? -mu_lo : 0.f;
+        const float2 nlo2 = make_float2(nlo, nlo);
+#pragma unroll
+        for (int kk = 0; kk < VPT; ++kk) {
+            const int v = t + kk * G;
+            if (v < a.nvec) {
+                const V16 xv = ld_shared16(stg + (size_t)v * 16);
+                const V16 wv = a.w ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16)
+                                   : ones_vec<T>();
+                const V16 bv = a.b ? ld_param(static_cast<const char*>(a.b) + (size_t)v * 16)
+                                   : zeros_vec<T>();
+                V16 o;
+                bool all_ok = true;
+#pragma unroll
+                for (int e = 0; e < VEC; e += 2) {
+                    const float2 w2 = E::get2(wv, e);
+                    const float2 b2 = E::get2(bv, e);
+                    const float2 A2 = mul2(rf2, w2);
+                    const float2 d2 = add2(add2(E::get2(xv, e), nhi2), nlo2);
+                    const float2 y2 = fma2(d2, A2, b2);
+                    // bitwise: no short-circuit branches in the unrolled loop
+                    all_ok &= (fabsf(y2.x) > __fmaf_rn(kmu, fabsf(A2.x), 0x1p-11f * fabsf(b2.x))) &
+                              (fabsf(y2.y) > __fmaf_rn(kmu, fabsf(A2.y), 0x1p-11f * fabsf(b2.y)));
+                    E::put2(o, e, y2);
+                }
+                if (!all_ok) o = layer_vector_f64<T>(xv, wv, bv, mean, rstd);
+                st_stream(static_cast<char*>(a.y) + roff + (size_t)v * 16, o);
+            }
+        }
+        __syncthreads();  // every thread is done with stage s
+        if (t == 0 && k + stages < nmine) {
+            fence_proxy_async_smem();
+            issue(k + stages);
+        }
+    }
+
+    if (k < nmine && t == 0) {  // a wait ran out: count it, let the copies in flight land
+        atomicAdd(&nvn_fault_count, 1u);
+        for (int64_t j = k; j < nmine && j < k + stages; ++j)
+            mbar_wait_bounded(bbase + 8u * (uint32_t)(j % stages), (uint32_t)((j / stages) & 1));
     }
 }
 

@@ -269,16 +269,39 @@ def test_layer_norm(rows, D, wb, dt):
     check_out(g.t, oracle.layer_norm(host(inp["x"]), host(inp["w"]), host(inp["b"]), 1e-5))
 
 
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
 @pytest.mark.parametrize("plan", [dict(path=nv.PATH_GENERIC)] +
                          [dict(path=nv.PATH_ROWS, vec_per_thread=v) for v in (1, 2, 4, 8)] +
-                         [dict(path=nv.PATH_ROWS, vec_per_thread=4, ctas_per_sm=2)])
-def test_layer_norm_every_variant(plan):
-    inp = synth.layer_norm_inputs(211, 4096, "bf16", seed=2)
+                         [dict(path=nv.PATH_ROWS, vec_per_thread=4, ctas_per_sm=2),
+                          dict(path=nv.PATH_STAGED),
+                          dict(path=nv.PATH_STAGED, vec_per_thread=2, rows_per_cta=3, ctas_per_sm=2),
+                          dict(path=nv.PATH_STAGED, vec_per_thread=8, rows_per_cta=2, ctas_per_sm=3)],
+                         ids=lambda p: "-".join(f"{k}{v}" for k, v in p.items()))
+def test_layer_norm_every_variant(plan, dt):
+    inp = synth.layer_norm_inputs(211, 4096, dt, seed=2)
     x = dev(inp["x"])
     y = torch.empty_like(x)
-    nv.nv_layer_norm(x, dev(inp["w"]), dev(inp["b"]), y, 1e-5, plan=nv.Plan(**plan))
+    try:
+        nv.nv_layer_norm(x, dev(inp["w"]), dev(inp["b"]), y, 1e-5, plan=nv.Plan(**plan))
+    except nv.NvError as e:
+        assert e.status == nv.NV_ERR_UNSUPPORTED
+        pytest.skip(str(e))
     torch.cuda.synchronize()
+    assert nv.nv_fault_count() == 0
     check_out(y, oracle.layer_norm(host(inp["x"]), host(inp["w"]), host(inp["b"]), 1e-5))
+
+
+@pytest.mark.parametrize("dt,mean,std", [("bf16", 0.5, 2.0), ("f32", 1e4, 1.0), ("bf16", 3000.0, 0.25)])
+def test_layer_norm_staged_rows_and_means(dt, mean, std):
+    for rows, D in ((1, 8192), (300, 8192), (1000, 1024)):
+        x = synth.normal((rows, D), mean, std, 5, 0, dt)
+        w = synth.uniform((D,), 0.5, 1.5, 5, 2, dt)
+        b = synth.normal((D,), 0.0, 0.1, 5, 3, dt)
+        y = torch.empty_like(x).cuda()
+        nv.nv_layer_norm(x.cuda(), w.cuda(), b.cuda(), y, 1e-5, plan=nv.Plan(path=nv.PATH_STAGED))
+        torch.cuda.synchronize()
+        assert nv.nv_fault_count() == 0
+        check_out(y, oracle.layer_norm(host(x), host(w), host(b), 1e-5))
 
 
 @pytest.mark.parametrize("dt,mean,std", [("f32", 1e4, 1.0), ("f32", -3e5, 0.01), ("bf16", 3000.0, 40.0),
