@@ -599,6 +599,7 @@ nv_status rope_op(const void* x, const void* w, void* y, int64_t rows, int64_t L
     a.lpr = rp.lpr;
     a.bt = rp.bt;
     a.base = base;
+    a.log2_base = std::log2((double)base);
     a.scale = scale;
     a.eps = eps;
     a.normalize = normalize != 0;

@@ -42,6 +42,7 @@ struct RopeArgs {
     float eps;
     int normalize;
     int traditional;
+    double log2_base;   // log2((double)base), computed on the host
 };
 
 // z = a_o * c + a_t * s for c = c_hi + c_lo, s = s_hi + s_lo (hi/lo float splits).
@@ -57,10 +58,11 @@ __device__ __forceinline__ float rotate_pair(float a_o, float a_t, float c_hi, f
     return __fadd_rn(z1, c3);
 }
 
-// cos and sin of (pos * scale * base^(-2 i / dims)) in double, split into float hi/lo.
-__device__ __forceinline__ float4 angle_entry(double pos, double scale, double base, int i,
+// cos and sin of (pos * scale * base^(-2 i / dims)) in double, split into float hi/lo;
+// base^(-2 i / dims) = 2^(-2 i log2(base) / dims).
+__device__ __forceinline__ float4 angle_entry(double pos, double scale, double log2_base, int i,
                                               int dims) {
-    const double theta = pow(base, -2.0 * (double)i / (double)dims);
+    const double theta = exp2(-2.0 * (double)i / (double)dims * log2_base);
     const double phi = pos * scale * theta;
     double s, c;
     sincos(phi, &s, &c);
@@ -131,29 +133,28 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
     const char* xbase = static_cast<const char*>(a.x) + (size_t)l * row_bytes + (size_t)v * 16;
     char* ybase = static_cast<char*>(a.y) + (size_t)l * row_bytes + (size_t)v * 16;
 
-    // The angle table touches no global memory, so it is built before waiting on a
-    // preceding kernel (programmatic dependent launch).
-    const double pos = (double)(a.offset + l);
-    for (int i = threadIdx.x; i < a.half; i += blockDim.x)
-        tab[i] = angle_entry(pos, (double)a.scale, (double)a.base, i, a.dims);
     pdl_wait();
     pdl_release();
-
     // Every thread runs the same trip count (rows past bh_end are predicated off):
     // the shuffles below involve the whole warp, which may hold several rows.
+    // The first rows' loads go out before the angle table is built, so its latency
+    // (double exp2 and sincos) hides behind theirs.
     V16 xv[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
         const int64_t b = bh0 + slot + (int64_t)u * slots;
         if (has_vec && b < bh_end) xv[u] = ld_stream(xbase + (size_t)b * lstride);
     }
-    // per-column weights of this lane's elements and of their partners, as floats
+    // per-column weights of this lane's elements and of their partners
     const V16 w_own_v = (norm && a.w && has_vec)
                             ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16)
                             : ones_vec<T>();
     V16 w_par_v = w_own_v;
     if (!TRAD && pv != v && norm && a.w && pv < a.nvec)
         w_par_v = ld_param(static_cast<const char*>(a.w) + (size_t)pv * 16);
+    const double pos = (double)(a.offset + l);
+    for (int i = threadIdx.x; i < a.half; i += blockDim.x)
+        tab[i] = angle_entry(pos, (double)a.scale, a.log2_base, i, a.dims);
     float2 w_own[VEC / 2], w_par[VEC / 2];
 #pragma unroll
     for (int e = 0; e < VEC; e += 2) {
@@ -290,9 +291,6 @@ __global__ void __launch_bounds__(256) rope_pairs_kernel(const RopeArgs a) {
     const int v0 = lane, v1 = lane + hvec;
     const bool has_vec = lane < hvec;
 
-    const double pos = (double)(a.offset + l);
-    for (int i = threadIdx.x; i < a.half; i += blockDim.x)
-        tab[i] = angle_entry(pos, (double)a.scale, (double)a.base, i, a.dims);
     pdl_wait();
     pdl_release();
 
@@ -312,7 +310,6 @@ __global__ void __launch_bounds__(256) rope_pairs_kernel(const RopeArgs a) {
             xv[u][1] = ld_stream(xbase + (size_t)b * lstride + (size_t)v1 * 16);
         }
     }
-
     const bool norm = a.normalize != 0;
     float2 w0[VEC / 2], w1[VEC / 2];
     {
@@ -320,6 +317,10 @@ __global__ void __launch_bounds__(256) rope_pairs_kernel(const RopeArgs a) {
                            ? ld_param(static_cast<const char*>(a.w) + (size_t)v0 * 16) : ones_vec<T>();
         const V16 wb = (norm && a.w && has_vec)
                            ? ld_param(static_cast<const char*>(a.w) + (size_t)v1 * 16) : ones_vec<T>();
+        // the angle table is built while the first rows' loads are in flight
+        const double pos = (double)(a.offset + l);
+        for (int i = threadIdx.x; i < a.half; i += blockDim.x)
+            tab[i] = angle_entry(pos, (double)a.scale, a.log2_base, i, a.dims);
 #pragma unroll
         for (int e = 0; e < VEC; e += 2) {
             w0[e / 2] = E::get2(wa, e);
@@ -422,7 +423,7 @@ __global__ void __launch_bounds__(128) rope_generic_kernel(const RopeArgs a) {
             const float wq = (norm && a.w) ? E::load1(a.w, q) : 1.f;
             const float ap = __fmul_rn(E::load1(a.x, r0 + p), wp);
             const float aq = __fmul_rn(E::load1(a.x, r0 + q), wq);
-            const float4 t = angle_entry(pos, (double)a.scale, (double)a.base, i, a.dims);
+            const float4 t = angle_entry(pos, (double)a.scale, a.log2_base, i, a.dims);
             const float yp = rotate_pair(ap, aq, t.x, t.y, -t.z, -t.w);
             const float yq = rotate_pair(aq, ap, t.x, t.y, t.z, t.w);
             E::store1(a.y, r0 + p, __fmul_rn(yp, inv));
