@@ -103,8 +103,10 @@ class Oracle:
         lib.oracle_rope_f64.argtypes = [vp, vp, i64, i64, i64, i64, i64, i32, f32, f32, i64, i32]
         lib.oracle_norm_rope.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, f32,
                                          i64, i32, f32, i32]
+        lib.oracle_rope_ex.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, f32, f32,
+                                       i64, i32, i32, f32, i32]
         for name in ("oracle_rms_norm", "oracle_add_rms_norm", "oracle_layer_norm",
-                     "oracle_rope_f64", "oracle_norm_rope"):
+                     "oracle_rope_f64", "oracle_norm_rope", "oracle_rope_ex"):
             getattr(lib, name).restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -186,6 +188,26 @@ class Oracle:
         return y
 
 
+    def rope_ex(self, x, w, L, dims, traditional, base, scale, offset, normalize, eps,
+                forward=True, freqs=None, y=None, y_len=0, threads=None):
+        """General NormRope / Rope: freqs (dims/2 values) replace base^(-2i/dims);
+        forward=False rotates back; y_len > 0 writes rows into the float64 cache y
+        [rows/L * y_len, D] at positions offset + l (other cache rows untouched)."""
+        x, dt = _io(x, "x")
+        rows, D = x.shape
+        w = None if w is None else _io(w, "w")[0]
+        f = None if freqs is None else np.ascontiguousarray(freqs, dtype=np.float64)
+        if y_len:
+            assert y is not None and y.dtype == np.float64 and y.flags.c_contiguous
+            assert y.shape == (rows // L * y_len, D)
+        else:
+            y = np.empty((rows, D), np.float64)
+        self._run(lambda a, b: self.lib.oracle_rope_ex(
+            _ptr(x), _ptr(w), _ptr(f), _ptr(y), a, b, L, y_len, D, dims, int(traditional), base,
+            scale, offset, int(forward), int(normalize), eps, dt), rows, threads)
+        return y
+
+
 _default = None
 
 
@@ -220,3 +242,9 @@ def rope_f64(x, L, dims, traditional, base, scale, offset, forward=True, threads
 def norm_rope(x, w, L, dims, traditional, base, scale, offset, normalize, eps, threads=None):
     return get().norm_rope(x, w, L, dims, traditional, base, scale, offset, normalize, eps,
                            threads)
+
+
+def rope_ex(x, w, L, dims, traditional, base, scale, offset, normalize, eps, forward=True,
+            freqs=None, y=None, y_len=0, threads=None):
+    return get().rope_ex(x, w, L, dims, traditional, base, scale, offset, normalize, eps,
+                         forward, freqs, y, y_len, threads)

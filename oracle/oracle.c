@@ -139,15 +139,16 @@ static void layer_row(const double* x, const void* w, const void* b, int dt, int
 
 /*
  * Rope of one row at position pos: pair i (0 <= i < dims/2) turns by
- * phi_i = pos * scale * base^(-2 i / dims); forward = 0 turns by -phi_i.
- * Features from dims on are copied unchanged.
+ * phi_i = pos * scale * theta_i, theta_i = base^(-2 i / dims), or theta_i = freqs[i]
+ * when a frequency vector is given (FastOp::Rope: "base ... unused with freqs");
+ * forward = 0 turns by -phi_i.  Features from dims on are copied unchanged.
  */
-static void rope_row(const double* x, int64_t D, int64_t dims, int traditional, double base,
-                     double scale, double pos, int forward, double* y) {
+static void rope_row_freqs(const double* x, int64_t D, int64_t dims, int traditional, double base,
+                           const double* freqs, double scale, double pos, int forward, double* y) {
     int64_t half = dims / 2;
     for (int64_t j = 0; j < D; ++j) y[j] = x[j];
     for (int64_t i = 0; i < half; ++i) {
-        double theta = pow(base, -2.0 * (double)i / (double)dims);
+        double theta = freqs ? freqs[i] : pow(base, -2.0 * (double)i / (double)dims);
         double phi = pos * scale * theta;
         if (!forward) phi = -phi;
         int64_t p = traditional ? 2 * i : i;
@@ -156,6 +157,11 @@ static void rope_row(const double* x, int64_t D, int64_t dims, int traditional, 
         y[p] = x[p] * c - x[q] * s;
         y[q] = x[p] * s + x[q] * c;
     }
+}
+
+static void rope_row(const double* x, int64_t D, int64_t dims, int traditional, double base,
+                     double scale, double pos, int forward, double* y) {
+    rope_row_freqs(x, D, dims, traditional, base, NULL, scale, pos, forward, y);
 }
 
 static void load_row(const void* src, int dt, int64_t row, int64_t D, double* dst) {
@@ -241,6 +247,41 @@ int oracle_norm_rope(const void* x, const void* w, double* y, int64_t r0, int64_
             memcpy(nrm, row, (size_t)D * sizeof(double));
         double pos = (double)offset + (double)(k % L);
         rope_row(nrm, D, dims, traditional, (double)base, (double)scale, pos, 1, y + k * D);
+    }
+    free(row);
+    free(nrm);
+    return 0;
+}
+
+/*
+ * The general NormRope / Rope (FastOp::NormRope with its cache form, FastOp::Rope with
+ * freqs and forward): rows of x [B, H, L, D] (rows = B*H*L) are normalised when
+ * normalize != 0 and rotated at position offset + l (by -phi when forward == 0), with
+ * theta_i from freqs (dims/2 doubles) when freqs != NULL.  y_len == 0: y is
+ * [rows, D] like x.  y_len > 0: y is a cache [B*H, y_len, D] and row (bh, l) of x is
+ * written to cache row (bh, offset + l); no other cache row is touched.
+ */
+int oracle_rope_ex(const void* x, const void* w, const double* freqs, double* y, int64_t r0,
+                   int64_t r1, int64_t L, int64_t y_len, int64_t D, int64_t dims, int traditional,
+                   float base, float scale, int64_t offset, int forward, int normalize, float eps,
+                   int dt) {
+    double* row = (double*)malloc((size_t)D * sizeof(double));
+    double* nrm = (double*)malloc((size_t)D * sizeof(double));
+    if (!row || !nrm) {
+        free(row);
+        free(nrm);
+        return -1;
+    }
+    for (int64_t k = r0; k < r1; ++k) {
+        load_row(x, dt, k, D, row);
+        if (normalize)
+            rms_row(row, w, dt, D, (double)eps, nrm);
+        else
+            memcpy(nrm, row, (size_t)D * sizeof(double));
+        int64_t l = k % L;
+        int64_t out = y_len > 0 ? (k / L) * y_len + offset + l : k;
+        rope_row_freqs(nrm, D, dims, traditional, (double)base, freqs, (double)scale,
+                       (double)offset + (double)l, forward, y + out * D);
     }
     free(row);
     free(nrm);

@@ -323,6 +323,61 @@ def check_norm_rope_composition(o):
                what="normalize = 0")
 
 
+def check_rope_ex_matches_rope(o):
+    """The general entry with default settings equals NormRope / Rope."""
+    Bsz, H, L, D, dims = 2, 2, 6, 24, 16
+    x = _randn_bf16((Bsz * H * L, D), 36)
+    w = bf16_bits(_rng(37).uniform(0.5, 1.5, D))
+    for trad in (0, 1):
+        for norm in (0, 1):
+            a = o.norm_rope(x, w, L, dims, trad, 500.0, 0.5, 9, norm, 1e-6)
+            b = o.rope_ex(x, w, L, dims, trad, 500.0, 0.5, 9, norm, 1e-6)
+            assert (a == b).all(), "rope_ex default path differs"
+
+
+def check_rope_freqs(o):
+    """freqs replace base^(-2i/dims): the standard frequencies reproduce Rope, zero
+    frequencies leave the row unrotated, and a hand-picked quarter turn lands exactly."""
+    L, D, dims = 5, 8, 8
+    x = _randn_bf16((2 * L, D), 38)
+    std = 100.0 ** (-np.arange(dims // 2) * 2.0 / dims)
+    a = o.rope_ex(x, None, L, dims, 0, 100.0, 1.0, 3, 0, 0.0, freqs=std)
+    b = o.norm_rope(x, None, L, dims, 0, 100.0, 1.0, 3, 0, 0.0)
+    _close(a, b, 1e-14, atol=1e-15, what="freqs = standard")
+    z = o.rope_ex(x, None, L, dims, 1, 100.0, 1.0, 3, 0, 0.0, freqs=np.zeros(dims // 2))
+    assert (z == widen_bf16(x)).all(), "zero frequencies must not rotate"
+    e = bf16_bits([[1.0, 0.0, 0.0, 0.0]])
+    q = o.rope_ex(e, None, 1, 4, 0, 10000.0, 1.0, 1, 0, 0.0, freqs=[math.pi / 2, 0.0])
+    _close(q[0], [math.cos(math.pi / 2), 0.0, 1.0, 0.0], 0, atol=1e-15, what="quarter turn")
+
+
+def check_rope_ex_inverse(o):
+    """forward = false undoes forward = true on the general path (no normalisation)."""
+    L, D, dims = 4, 16, 12
+    xf = _rng(39).standard_normal((3 * L, D)).astype(np.float32)
+    for trad in (0, 1):
+        y = o.rope_ex(xf, None, L, dims, trad, 1000.0, 2.0, 77, 0, 0.0, forward=True)
+        back = o.rope_ex(y.astype(np.float32), None, L, dims, trad, 1000.0, 2.0, 77, 0, 0.0,
+                         forward=False)
+        _close(back, xf, 1e-5, atol=1e-6, what="inverse on rope_ex")
+
+
+def check_rope_cache_placement(o):
+    """Cache form: row (bh, l) lands at cache row (bh, offset + l); other rows untouched."""
+    Bsz, H, L, D, dims, y_len, off = 1, 3, 4, 8, 8, 11, 5
+    x = _randn_bf16((Bsz * H * L, D), 40)
+    cache = np.full((Bsz * H * y_len, D), 7.25)
+    o.rope_ex(x, None, L, dims, 0, 10000.0, 1.0, off, 1, 1e-6, y=cache, y_len=y_len)
+    plain = o.norm_rope(x, None, L, dims, 0, 10000.0, 1.0, off, 1, 1e-6)
+    for bh in range(Bsz * H):
+        for r in range(y_len):
+            got = cache[bh * y_len + r]
+            if off <= r < off + L:
+                assert (got == plain[bh * L + r - off]).all(), "cache row misplaced"
+            else:
+                assert (got == 7.25).all(), "a cache row outside [offset, offset+L) changed"
+
+
 # ---- hand-worked cases -----------------------------------------------------------------
 
 _MATH = {k: getattr(math, k) for k in ("sqrt", "cos", "sin", "pi")}

@@ -49,8 +49,16 @@ MUTANTS = {
                                  "double pos = (double)(k % L);\n        rope_row(nrm"),
     "norm_rope_position_k_div_L": ("double pos = (double)offset + (double)(k % L);\n        rope_row(nrm",
                                    "double pos = (double)offset + (double)(k / L);\n        rope_row(nrm"),
-    "norm_rope_skips_normalise": ("if (normalize)\n            rms_row(row, w, dt, D, (double)eps, nrm);",
-                                  "if (0)\n            rms_row(row, w, dt, D, (double)eps, nrm);"),
+    "norm_rope_skips_normalise": ("if (normalize)\n            rms_row(row, w, dt, D, (double)eps, nrm);\n        else\n            memcpy(nrm, row, (size_t)D * sizeof(double));\n        double pos",
+                                  "if (0)\n            rms_row(row, w, dt, D, (double)eps, nrm);\n        else\n            memcpy(nrm, row, (size_t)D * sizeof(double));\n        double pos"),
+    "rope_ex_skips_normalise": ("if (normalize)\n            rms_row(row, w, dt, D, (double)eps, nrm);\n        else\n            memcpy(nrm, row, (size_t)D * sizeof(double));\n        int64_t l",
+                                "if (0)\n            rms_row(row, w, dt, D, (double)eps, nrm);\n        else\n            memcpy(nrm, row, (size_t)D * sizeof(double));\n        int64_t l"),
+    "rope_ex_freqs_ignored": ("double theta = freqs ? freqs[i] : pow(base, -2.0 * (double)i / (double)dims);",
+                              "double theta = pow(base, -2.0 * (double)i / (double)dims);"),
+    "rope_ex_cache_row_ignores_offset": ("int64_t out = y_len > 0 ? (k / L) * y_len + offset + l : k;",
+                                         "int64_t out = y_len > 0 ? (k / L) * y_len + l : k;"),
+    "rope_ex_cache_row_uses_L": ("int64_t out = y_len > 0 ? (k / L) * y_len + offset + l : k;",
+                                 "int64_t out = y_len > 0 ? (k / L) * L + offset + l : k;"),
     "round_truncates": ("double n = rint(ldexp(a, -qexp));", "double n = trunc(ldexp(a, -qexp));"),
     "round_ties_away": ("double n = rint(ldexp(a, -qexp));", "double n = round(ldexp(a, -qexp));"),
     "round_subnormal_quantum": ("int qexp = (e < -125 ? -125 : e) - 8;", "int qexp = e - 8;"),
