@@ -113,6 +113,24 @@ NV_API nv_status nv_norm_rope(const void* x, const void* w, void* y, int64_t row
                        int32_t dims, int32_t traditional, float base, float scale, int64_t offset,
                        int32_t normalize, float eps, nv_dtype dt, nv_stream_t stream);
 
+/*
+ * rope -- the general form of norm_rope: docs.rs nuvec-core 0.5.0, Enum FastOp, variant
+ * NormRope with its cache form ("written into cache at the same positions") and
+ * variant Rope with an explicit frequency vector and a direction.
+ *   freqs    [dims/2] float32 device array of frequencies theta_i replacing
+ *            base^(-2 i / dims) ("base ... unused with freqs"), or NULL.
+ *   forward  != 0: turn by +phi_i; 0: the inverse rotation (-phi_i), the gradient of Rope.
+ *   y_len    0: y is [B, H, L, D] like x (may be x).  > 0: y is a cache [B, H, y_len, D]
+ *            and row (b, h, l) of x is written to cache row (b, h, offset + l), at the
+ *            same position offset + l it is rotated at; no other cache row is written.
+ *            Requires y_len >= offset + L; y must not overlap x then.
+ * Other arguments as nv_norm_rope; base is checked only when freqs is NULL.
+ */
+NV_API nv_status nv_rope(const void* x, const void* w, const float* freqs, void* y, int64_t rows,
+                         int64_t L, int64_t y_len, int64_t D, int32_t dims, int32_t traditional,
+                         float base, float scale, int64_t offset, int32_t forward,
+                         int32_t normalize, float eps, nv_dtype dt, nv_stream_t stream);
+
 /* Name of a status code (static storage). */
 NV_API const char* nv_status_string(nv_status status);
 
@@ -178,6 +196,11 @@ NV_API nv_status nv_add_rms_norm_ex(const void* x, const void* r, const void* w,
 NV_API nv_status nv_layer_norm_ex(const void* x, const void* w, const void* b, void* y, int64_t rows,
                            int64_t D, float eps, nv_dtype dt, nv_stream_t stream,
                            const nv_plan* plan);
+NV_API nv_status nv_rope_ex(const void* x, const void* w, const float* freqs, void* y,
+                            int64_t rows, int64_t L, int64_t y_len, int64_t D, int32_t dims,
+                            int32_t traditional, float base, float scale, int64_t offset,
+                            int32_t forward, int32_t normalize, float eps, nv_dtype dt,
+                            nv_stream_t stream, const nv_plan* plan);
 NV_API nv_status nv_norm_rope_ex(const void* x, const void* w, void* y, int64_t rows, int64_t L,
                           int64_t D, int32_t dims, int32_t traditional, float base, float scale,
                           int64_t offset, int32_t normalize, float eps, nv_dtype dt,

@@ -20,7 +20,8 @@ __all__ = [
     "NvError", "Plan", "library", "library_path",
     "nv_rms_norm", "nv_add_rms_norm", "nv_layer_norm", "nv_norm_rope", "nv_describe_plan",
     "nv_fault_count",
-    "rms_norm", "add_rms_norm", "layer_norm", "norm_rope",
+    "nv_rope", "rms_norm", "add_rms_norm", "layer_norm", "norm_rope", "norm_rope_into_cache",
+    "rope",
     "PATH_AUTO", "PATH_ROWS", "PATH_GENERIC", "PATH_STAGED", "LAUNCH_DEFAULT", "LAUNCH_PLAIN",
 ]
 
@@ -79,6 +80,10 @@ def library() -> ctypes.CDLL:
         "nv_norm_rope_ex": [vp, vp, vp, i64, i64, i64, i32, i32, f32, f32, i64, i32, f32, i32,
                             vp, pp],
         "nv_describe_plan": [i32, i64, i64, i32, pp],
+        "nv_rope": [vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, f32, f32, i64, i32, i32, f32, i32,
+                    vp],
+        "nv_rope_ex": [vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, f32, f32, i64, i32, i32, f32,
+                       i32, vp, pp],
     }
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -177,6 +182,21 @@ def nv_norm_rope(x, w, y, L, dims, traditional, base, scale, offset, normalize, 
     _check("nv_norm_rope", st)
 
 
+def nv_rope(x, w, y, L, dims, traditional, base, scale, offset, normalize, eps, freqs=None,
+            forward=True, y_len=0, stream=None, plan=None):
+    """General NormRope / Rope (cache output when y_len > 0, explicit float32 freqs,
+    forward=False for the inverse rotation); x is [rows, D] with rows = B*H*L."""
+    rows, D = _rows_D(x)
+    if freqs is not None and freqs.dtype != torch.float32:
+        raise TypeError("freqs must be float32")
+    lib = library()
+    args = (_ptr(x), _ptr(w), _ptr(freqs), _ptr(y), rows, L, y_len, D, dims,
+            int(bool(traditional)), base, scale, offset, int(bool(forward)), int(bool(normalize)),
+            eps, _dtype(x, w, y), _stream(stream))
+    st = lib.nv_rope(*args) if plan is None else lib.nv_rope_ex(*args, _plan(plan))
+    _check("nv_rope", st)
+
+
 def nv_describe_plan(op: str, rows: int, D: int, dtype) -> dict:
     """The kernel variant the library picks for op on [rows, D] (16-byte aligned data)."""
     ops = {"rms_norm": 0, "add_rms_norm": 1, "layer_norm": 2, "norm_rope": 3}
@@ -214,6 +234,28 @@ def layer_norm(x, w=None, b=None, eps=1e-5, stream=None):
     """y = (x - mean) / sqrt(var + eps) * w + b over the last axis."""
     y = torch.empty_like(x)
     nv_layer_norm(x, w, b, y, eps, stream)
+    return y
+
+
+def norm_rope_into_cache(x, cache, w=None, dims=None, traditional=False, base=10000.0,
+                         scale=1.0, offset=0, eps=1e-6, freqs=None, stream=None):
+    """Normalise (eps None: skip) and rotate x [..., L, D]; write row l into
+    cache [..., Lc, D] at row offset + l (the cache form of NormRope)."""
+    L, D = x.shape[-2], x.shape[-1]
+    normalize = eps is not None
+    nv_rope(x, w, cache, L, D if dims is None else dims, traditional, base, scale, offset,
+            normalize, eps if normalize else 0.0, freqs=freqs, y_len=cache.shape[-2],
+            stream=stream)
+    return cache
+
+
+def rope(x, dims=None, traditional=False, base=10000.0, scale=1.0, offset=0, freqs=None,
+         forward=True, stream=None):
+    """Plain rotary embedding of x [..., L, D] (forward=False: the inverse rotation)."""
+    L, D = x.shape[-2], x.shape[-1]
+    y = torch.empty_like(x)
+    nv_rope(x, None, y, L, D if dims is None else dims, traditional, base, scale, offset, False,
+            0.0, freqs=freqs, forward=forward, stream=stream)
     return y
 
 

@@ -540,10 +540,10 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
     return NV_OK;
 }
 
-nv_status rope_op(const void* x, const void* w, void* y, int64_t rows, int64_t L, int64_t D,
-                  int32_t dims, int32_t traditional, float base, float scale, int64_t offset,
-                  int32_t normalize, float eps, nv_dtype dt, nv_stream_t stream,
-                  const nv_plan* req) {
+nv_status rope_op(const void* x, const void* w, const float* freqs, void* y, int64_t rows,
+                  int64_t L, int64_t y_len, int64_t D, int32_t dims, int32_t traditional,
+                  float base, float scale, int64_t offset, int32_t forward, int32_t normalize,
+                  float eps, nv_dtype dt, nv_stream_t stream, const nv_plan* req) {
     nv_status st = check_common(rows, D, eps, dt, normalize != 0);
     if (st != NV_OK) return st;
     if (L < 1) return fail(NV_ERR_INVALID_ARG, "L = %lld < 1", (long long)L);
@@ -553,12 +553,16 @@ nv_status rope_op(const void* x, const void* w, void* y, int64_t rows, int64_t L
     if (dims <= 0 || dims % 2 != 0 || dims > D)
         return fail(NV_ERR_INVALID_ARG, "dims = %d must be even with 0 < dims <= D = %lld", dims,
                     (long long)D);
-    if (!(base > 0.f) || !std::isfinite(base))
+    if (!freqs && (!(base > 0.f) || !std::isfinite(base)))
         return fail(NV_ERR_INVALID_ARG, "base = %g must be finite and > 0", (double)base);
     if (!std::isfinite(scale)) return fail(NV_ERR_INVALID_ARG, "scale must be finite");
     if (offset < 0) return fail(NV_ERR_INVALID_ARG, "offset = %lld < 0", (long long)offset);
     if (offset > ((int64_t)1 << 52) - L)
         return fail(NV_ERR_INVALID_ARG, "offset + L must stay below 2^52");
+    if (y_len < 0) return fail(NV_ERR_INVALID_ARG, "y_len = %lld < 0", (long long)y_len);
+    if (y_len > 0 && y_len < offset + L)
+        return fail(NV_ERR_INVALID_ARG, "cache length y_len = %lld < offset + L = %lld",
+                    (long long)y_len, (long long)(offset + L));
     if (rows == 0) return NV_OK;
     if (!x) return fail(NV_ERR_INVALID_ARG, "x is NULL");
     if (!y) return fail(NV_ERR_INVALID_ARG, "y is NULL");
@@ -569,12 +573,16 @@ nv_status rope_op(const void* x, const void* w, void* y, int64_t rows, int64_t L
     if (st != NV_OK) return st;
     const size_t s = elem_size(dt);
     const size_t nbytes = (size_t)rows * (size_t)D * s;
+    const bool cache = y_len > 0;
+    const size_t ybytes = cache ? (size_t)(rows / L) * (size_t)y_len * (size_t)D * s : nbytes;
     const Buf bufs[] = {
-        {x, nbytes, "x", false, true},
+        // a cache has another layout than x: then y may not even alias x
+        {x, nbytes, "x", false, !cache},
         {normalize ? w : nullptr, (size_t)D * s, "w", false, false},
-        {y, nbytes, "y", true, false},
+        {freqs, (size_t)(dims / 2) * sizeof(float), "freqs", false, false},
+        {y, ybytes, "y", true, false},
     };
-    st = check_buffers(bufs, 3, dev);
+    st = check_buffers(bufs, 4, dev);
     if (st != NV_OK) return st;
 
     const bool al = aligned16(x) && aligned16(y) && (!w || !normalize || aligned16(w));
@@ -599,11 +607,15 @@ nv_status rope_op(const void* x, const void* w, void* y, int64_t rows, int64_t L
     a.lpr = rp.lpr;
     a.bt = rp.bt;
     a.base = base;
-    a.log2_base = std::log2((double)base);
+    a.log2_base = freqs ? 0.0 : std::log2((double)base);
     a.scale = scale;
     a.eps = eps;
     a.normalize = normalize != 0;
     a.traditional = traditional != 0;
+    a.freqs = freqs;
+    a.forward = forward != 0;
+    a.y_len = cache ? y_len : L;
+    a.y_off = cache ? offset : 0;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     const bool bf = dt == NV_BF16;
     if (rp.rows) {
@@ -658,8 +670,24 @@ nv_status nv_norm_rope_ex(const void* x, const void* w, void* y, int64_t rows, i
                           int64_t D, int32_t dims, int32_t traditional, float base, float scale,
                           int64_t offset, int32_t normalize, float eps, nv_dtype dt,
                           nv_stream_t stream, const nv_plan* plan) {
-    return rope_op(x, w, y, rows, L, D, dims, traditional, base, scale, offset, normalize, eps,
-                   dt, stream, plan);
+    return rope_op(x, w, nullptr, y, rows, L, 0, D, dims, traditional, base, scale, offset, 1,
+                   normalize, eps, dt, stream, plan);
+}
+
+nv_status nv_rope_ex(const void* x, const void* w, const float* freqs, void* y, int64_t rows,
+                     int64_t L, int64_t y_len, int64_t D, int32_t dims, int32_t traditional,
+                     float base, float scale, int64_t offset, int32_t forward, int32_t normalize,
+                     float eps, nv_dtype dt, nv_stream_t stream, const nv_plan* plan) {
+    return rope_op(x, w, freqs, y, rows, L, y_len, D, dims, traditional, base, scale, offset,
+                   forward, normalize, eps, dt, stream, plan);
+}
+
+nv_status nv_rope(const void* x, const void* w, const float* freqs, void* y, int64_t rows,
+                  int64_t L, int64_t y_len, int64_t D, int32_t dims, int32_t traditional,
+                  float base, float scale, int64_t offset, int32_t forward, int32_t normalize,
+                  float eps, nv_dtype dt, nv_stream_t stream) {
+    return rope_op(x, w, freqs, y, rows, L, y_len, D, dims, traditional, base, scale, offset,
+                   forward, normalize, eps, dt, stream, nullptr);
 }
 
 nv_status nv_norm_rope(const void* x, const void* w, void* y, int64_t rows, int64_t L, int64_t D,

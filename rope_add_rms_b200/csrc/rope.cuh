@@ -43,6 +43,10 @@ struct RopeArgs {
     int normalize;
     int traditional;
     double log2_base;   // log2((double)base), computed on the host
+    const float* freqs; // [dims/2] frequencies replacing base^(-2i/dims), or NULL
+    int forward;        // 0: inverse rotation (-phi)
+    int64_t y_len;      // rows per (b, h) in y: L, or the cache length
+    int64_t y_off;      // first y row of a (b, h): 0, or offset in the cache form
 };
 
 // z = a_o * c + a_t * s for c = c_hi + c_lo, s = s_hi + s_lo (hi/lo float splits).
@@ -58,14 +62,16 @@ __device__ __forceinline__ float rotate_pair(float a_o, float a_t, float c_hi, f
     return __fadd_rn(z1, c3);
 }
 
-// cos and sin of (pos * scale * base^(-2 i / dims)) in double, split into float hi/lo;
-// base^(-2 i / dims) = 2^(-2 i log2(base) / dims).
-__device__ __forceinline__ float4 angle_entry(double pos, double scale, double log2_base, int i,
-                                              int dims) {
-    const double theta = exp2(-2.0 * (double)i / (double)dims * log2_base);
-    const double phi = pos * scale * theta;
+// cos and sin of phi_i = pos * scale * theta_i in double, split into float hi/lo, where
+// theta_i = freqs[i] if a frequency vector is given, else base^(-2 i / dims) =
+// 2^(-2 i log2(base) / dims).  The inverse rotation negates sin (exact).
+__device__ __forceinline__ float4 angle_entry(const RopeArgs& a, double pos, int i) {
+    const double theta = a.freqs ? (double)a.freqs[i]
+                                 : exp2(-2.0 * (double)i / (double)a.dims * a.log2_base);
+    const double phi = pos * (double)a.scale * theta;
     double s, c;
     sincos(phi, &s, &c);
+    if (!a.forward) s = -s;
     const float ch = __double2float_rn(c);
     const float sh = __double2float_rn(s);
     return make_float4(ch, __double2float_rn(c - (double)ch), sh, __double2float_rn(s - (double)sh));
@@ -131,7 +137,9 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
     const size_t row_bytes = (size_t)a.D * sizeof(T);
     const size_t lstride = (size_t)a.L * row_bytes;  // between consecutive bh at fixed l
     const char* xbase = static_cast<const char*>(a.x) + (size_t)l * row_bytes + (size_t)v * 16;
-    char* ybase = static_cast<char*>(a.y) + (size_t)l * row_bytes + (size_t)v * 16;
+    // y row of (b, h, l): b * y_len + y_off + l (y_len = L, y_off = 0 unless a cache)
+    const size_t ystride = (size_t)a.y_len * row_bytes;
+    char* ybase = static_cast<char*>(a.y) + (size_t)(a.y_off + l) * row_bytes + (size_t)v * 16;
 
     pdl_wait();
     pdl_release();
@@ -154,7 +162,7 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
         w_par_v = ld_param(static_cast<const char*>(a.w) + (size_t)pv * 16);
     const double pos = (double)(a.offset + l);
     for (int i = threadIdx.x; i < a.half; i += blockDim.x)
-        tab[i] = angle_entry(pos, (double)a.scale, a.log2_base, i, a.dims);
+        tab[i] = angle_entry(a, pos, i);
     float2 w_own[VEC / 2], w_par[VEC / 2];
 #pragma unroll
     for (int e = 0; e < VEC; e += 2) {
@@ -263,7 +271,7 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const RopeArgs a) {
                             E::put2(o, e, y, 0.f);
                     }
                 }
-                st_stream(ybase + (size_t)b * lstride, o);
+                st_stream(ybase + (size_t)b * ystride, o);
             }
         }
     }
@@ -299,7 +307,8 @@ __global__ void __launch_bounds__(256) rope_pairs_kernel(const RopeArgs a) {
     const size_t row_bytes = (size_t)a.D * sizeof(T);
     const size_t lstride = (size_t)a.L * row_bytes;
     const char* xbase = static_cast<const char*>(a.x) + (size_t)l * row_bytes;
-    char* ybase = static_cast<char*>(a.y) + (size_t)l * row_bytes;
+    const size_t ystride = (size_t)a.y_len * row_bytes;
+    char* ybase = static_cast<char*>(a.y) + (size_t)(a.y_off + l) * row_bytes;
 
     V16 xv[kUnroll][2];
 #pragma unroll
@@ -320,7 +329,7 @@ __global__ void __launch_bounds__(256) rope_pairs_kernel(const RopeArgs a) {
         // the angle table is built while the first rows' loads are in flight
         const double pos = (double)(a.offset + l);
         for (int i = threadIdx.x; i < a.half; i += blockDim.x)
-            tab[i] = angle_entry(pos, (double)a.scale, a.log2_base, i, a.dims);
+            tab[i] = angle_entry(a, pos, i);
 #pragma unroll
         for (int e = 0; e < VEC; e += 2) {
             w0[e / 2] = E::get2(wa, e);
@@ -377,8 +386,8 @@ __global__ void __launch_bounds__(256) rope_pairs_kernel(const RopeArgs a) {
                     E::put2(o0, e, mul2(z0, inv2));
                     E::put2(o1, e, mul2(z1, inv2));
                 }
-                st_stream(ybase + (size_t)b * lstride + (size_t)v0 * 16, o0);
-                st_stream(ybase + (size_t)b * lstride + (size_t)v1 * 16, o1);
+                st_stream(ybase + (size_t)b * ystride + (size_t)v0 * 16, o0);
+                st_stream(ybase + (size_t)b * ystride + (size_t)v1 * 16, o1);
             }
         }
     }
@@ -416,6 +425,7 @@ __global__ void __launch_bounds__(128) rope_generic_kernel(const RopeArgs a) {
             inv = rsqrtf(__fmaf_rn(ss, 1.0f / (float)a.D, a.eps));
         }
         const double pos = (double)(a.offset + row % a.L);
+        const int64_t o0 = ((row / a.L) * a.y_len + a.y_off + row % a.L) * (int64_t)a.D;
         for (int i = threadIdx.x; i < a.half; i += blockDim.x) {
             const int p = a.traditional ? 2 * i : i;
             const int q = a.traditional ? 2 * i + 1 : i + a.half;
@@ -423,15 +433,15 @@ __global__ void __launch_bounds__(128) rope_generic_kernel(const RopeArgs a) {
             const float wq = (norm && a.w) ? E::load1(a.w, q) : 1.f;
             const float ap = __fmul_rn(E::load1(a.x, r0 + p), wp);
             const float aq = __fmul_rn(E::load1(a.x, r0 + q), wq);
-            const float4 t = angle_entry(pos, (double)a.scale, a.log2_base, i, a.dims);
+            const float4 t = angle_entry(a, pos, i);
             const float yp = rotate_pair(ap, aq, t.x, t.y, -t.z, -t.w);
             const float yq = rotate_pair(aq, ap, t.x, t.y, t.z, t.w);
-            E::store1(a.y, r0 + p, __fmul_rn(yp, inv));
-            E::store1(a.y, r0 + q, __fmul_rn(yq, inv));
+            E::store1(a.y, o0 + p, __fmul_rn(yp, inv));
+            E::store1(a.y, o0 + q, __fmul_rn(yq, inv));
         }
         for (int j = a.dims + threadIdx.x; j < a.D; j += blockDim.x) {
             const float wj = (norm && a.w) ? E::load1(a.w, j) : 1.f;
-            E::store1(a.y, r0 + j, __fmul_rn(__fmul_rn(E::load1(a.x, r0 + j), wj), inv));
+            E::store1(a.y, o0 + j, __fmul_rn(__fmul_rn(E::load1(a.x, r0 + j), wj), inv));
         }
     }
 }

@@ -77,6 +77,12 @@ def rope(x=FAKE, w=None, y=FAKE, rows=8, L=4, D=8, dims=8, trad=0, base=10000.0,
                                      normalize, eps, dt, None)
 
 
+def rope_general(x=FAKE, w=None, freqs=None, y=FAKE, rows=8, L=4, y_len=0, D=8, dims=8, trad=0,
+                 base=10000.0, scale=1.0, offset=0, forward=1, normalize=1, eps=1e-6, dt=BF16):
+    return nv.library().nv_rope(x, w, freqs, y, rows, L, y_len, D, dims, trad, base, scale, offset,
+                                forward, normalize, eps, dt, None)
+
+
 def last_error():
     return nv.library().nv_last_error().decode()
 
@@ -109,6 +115,11 @@ def last_error():
     (lambda: rope(offset=-1), INVALID, "offset"),
     (lambda: rope(eps=-1.0), INVALID, "eps"),
     (lambda: rope(x=None), INVALID, "x is NULL"),
+    (lambda: rope_general(y_len=-1), INVALID, "y_len"),
+    (lambda: rope_general(y_len=5, offset=2, L=4), INVALID, "cache length"),
+    (lambda: rope_general(base=0.0), INVALID, "base"),
+    (lambda: rope_general(base=0.0, freqs=FAKE, x=None), INVALID, "x is NULL"),
+    (lambda: rope_general(dims=3), INVALID, "dims"),
 ])
 def test_invalid_arguments_are_rejected_on_the_host(call, status, words):
     assert call() == status

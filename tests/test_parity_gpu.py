@@ -471,3 +471,81 @@ def test_dependent_chain_across_ops_in_place():
     check_out(stages[2], oracle.norm_rope(to_host_bits(stages[1]), wh, L, D, 0, 10000.0, 1.0, 4096,
                                           1, 1e-6), "norm_rope")
     check_out(stages[3], oracle.rms_norm(to_host_bits(stages[2]), None, 1e-6), "rms_norm")
+
+
+# ---- general rope: cache form, explicit frequencies, inverse ----------------------------------
+
+ROPE_PLANS = [None, dict(path=nv.PATH_GENERIC), dict(path=nv.PATH_ROWS, vec_per_thread=1),
+              dict(path=nv.PATH_ROWS, vec_per_thread=2)]
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("trad", [0, 1])
+@pytest.mark.parametrize("plan", ROPE_PLANS, ids=lambda p: "auto" if p is None else
+                         "-".join(f"{k}{v}" for k, v in p.items()))
+def test_norm_rope_into_cache(plan, trad, dt):
+    """Row (b, h, l) lands in cache row (b, h, offset + l); every other row is untouched."""
+    B, H, L, D, Lc, off = 2, 3, 16, 128, 50, 20
+    inp = synth.norm_rope_inputs(B, H, L, D, dt, seed=31)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    cache = torch.full((B * H * Lc, D), 7.25, dtype=x.dtype, device="cuda")
+    try:
+        nv.nv_rope(x, w, cache, L, D, trad, 10000.0, 1.0, off, 1, 1e-6, y_len=Lc,
+                   plan=None if plan is None else nv.Plan(**plan))
+    except nv.NvError as e:
+        assert e.status == nv.NV_ERR_UNSUPPORTED
+        pytest.skip(str(e))
+    torch.cuda.synchronize()
+    ref = np.full((B * H * Lc, D), 7.25)
+    oracle.rope_ex(host(inp["x"]), host(inp["w"]), L, D, trad, 10000.0, 1.0, off, 1, 1e-6,
+                   y=ref, y_len=Lc)
+    inside = np.zeros(B * H * Lc, bool)
+    for bh in range(B * H):
+        inside[bh * Lc + off: bh * Lc + off + L] = True
+    got = cache.float().cpu().numpy()
+    assert (got[~inside] == 7.25).all(), "a cache row outside [offset, offset + L) changed"
+    check_out(cache[torch.as_tensor(inside, device="cuda")], ref[inside])
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("trad", [0, 1])
+@pytest.mark.parametrize("plan", ROPE_PLANS, ids=lambda p: "auto" if p is None else
+                         "-".join(f"{k}{v}" for k, v in p.items()))
+def test_rope_freqs_and_inverse(plan, trad, dt):
+    B, H, L, D = 2, 4, 32, 128
+    inp = synth.norm_rope_inputs(B, H, L, D, dt, seed=32)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    freqs = synth.uniform((D // 2,), 0.0, 0.5, 32, 5, "f32")
+    p = None if plan is None else nv.Plan(**plan)
+    for normalize in (0, 1):
+        for forward in (True, False):
+            for f in (None, freqs):
+                y = torch.empty_like(x)
+                try:
+                    nv.nv_rope(x, w, y, L, D, trad, 500.0, 0.75, 4095, normalize, 1e-6,
+                               freqs=None if f is None else f.cuda(), forward=forward, plan=p)
+                except nv.NvError as e:
+                    assert e.status == nv.NV_ERR_UNSUPPORTED
+                    pytest.skip(str(e))
+                torch.cuda.synchronize()
+                ref = oracle.rope_ex(host(inp["x"]), host(inp["w"]), L, D, trad, 500.0, 0.75,
+                                     4095, normalize, 1e-6, forward=forward,
+                                     freqs=None if f is None else f.numpy().astype(np.float64))
+                check_out(y, ref, f"normalize={normalize} forward={forward} freqs={f is not None}")
+
+
+def test_rope_round_trip_and_cache_rules():
+    B, H, L, D = 1, 2, 8, 64
+    x = synth.normal((B * H * L, D), 0.0, 1.0, 33, 0, "f32").cuda()
+    y = nv.rope(x.view(B, H, L, D), offset=100).view(-1, D)
+    back = nv.rope(y.view(B, H, L, D), offset=100, forward=False).view(-1, D)
+    torch.cuda.synchronize()
+    assert torch.allclose(back, x, rtol=1e-5, atol=1e-5)
+    cache = torch.zeros(B * H * 20, D, device="cuda")
+    with pytest.raises(nv.NvError, match="cache length"):
+        nv.nv_rope(x, None, cache, L, D, 0, 10000.0, 1.0, 15, 0, 0.0, y_len=20)
+    big = torch.zeros(B * H * L * D + B * H * 20 * D, device="cuda")
+    xs = big[:B * H * L * D].view(-1, D)
+    with pytest.raises(nv.NvError, match="overlaps"):
+        nv.nv_rope(xs, None, big[B * H * L * D // 2:][:B * H * 20 * D].view(-1, D), L, D, 0,
+                   10000.0, 1.0, 0, 0, 0.0, y_len=20)
