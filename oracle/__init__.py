@@ -105,8 +105,12 @@ class Oracle:
                                          i64, i32, f32, i32]
         lib.oracle_rope_ex.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, f32, f32,
                                        i64, i32, i32, f32, i32]
+        lib.oracle_rms_norm_vjp.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, f32, i32]
+        lib.oracle_layer_norm_vjp.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64,
+                                              f32, i32]
         for name in ("oracle_rms_norm", "oracle_add_rms_norm", "oracle_layer_norm",
-                     "oracle_rope_f64", "oracle_norm_rope", "oracle_rope_ex"):
+                     "oracle_rope_f64", "oracle_norm_rope", "oracle_rope_ex",
+                     "oracle_rms_norm_vjp", "oracle_layer_norm_vjp"):
             getattr(lib, name).restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -208,6 +212,53 @@ class Oracle:
         return y
 
 
+    def _vjp(self, fn, nsums, x, g, w, threads):
+        x, dt = _io(x, "x")
+        g = _io(g, "g")[0]
+        rows, D = x.shape
+        w = None if w is None else _io(w, "w")[0]
+        dx = np.empty((rows, D), np.float64)
+        mdx = np.empty((rows, D), np.float64)
+        chunks = _chunks(rows, threads)
+        parts = [np.zeros((2 * nsums, D), np.float64) for _ in chunks]
+
+        def one(i):
+            a, b = chunks[i]
+            p = parts[i]
+            return fn(x, w, g, dx, mdx, p, a, b, D, dt)
+
+        if len(chunks) == 1:
+            rcs = [one(0)]
+        else:
+            with ThreadPoolExecutor(len(chunks)) as ex:
+                rcs = list(ex.map(one, range(len(chunks))))
+        if any(rc != 0 for rc in rcs):
+            raise MemoryError("oracle: row buffer allocation failed")
+        self.last_threads = len(chunks)
+        tot = np.zeros((2 * nsums, D), np.float64)
+        for p in parts:            # chunk order: a fixed summation order
+            tot += p
+        return dx, mdx, tot
+
+    def rms_norm_vjp(self, x, w, g, eps, threads=None):
+        """RmsNormVjp: (dx, dw or None, mag_dx, mag_dw) -- mag_* are the magnitude sums
+        bounding a float32 evaluation's rounding error."""
+        def fn(x, w, g, dx, mdx, p, a, b, D, dt):
+            return self.lib.oracle_rms_norm_vjp(_ptr(x), _ptr(w), _ptr(g), _ptr(dx), _ptr(p[0]),
+                                                _ptr(mdx), _ptr(p[1]), a, b, D, eps, dt)
+        dx, mdx, tot = self._vjp(fn, 1, x, g, w, threads)
+        return dx, (tot[0] if w is not None else None), mdx, tot[1]
+
+    def layer_norm_vjp(self, x, w, g, eps, threads=None):
+        """LayerNormVjp: (dx, dw, db, mag_dx, mag_dw, mag_db); dw is None without w."""
+        def fn(x, w, g, dx, mdx, p, a, b, D, dt):
+            return self.lib.oracle_layer_norm_vjp(_ptr(x), _ptr(w), _ptr(g), _ptr(dx), _ptr(p[0]),
+                                                  _ptr(p[1]), _ptr(mdx), _ptr(p[2]), _ptr(p[3]),
+                                                  a, b, D, eps, dt)
+        dx, mdx, tot = self._vjp(fn, 2, x, g, w, threads)
+        return dx, (tot[0] if w is not None else None), tot[1], mdx, tot[2], tot[3]
+
+
 _default = None
 
 
@@ -248,3 +299,11 @@ def rope_ex(x, w, L, dims, traditional, base, scale, offset, normalize, eps, for
             freqs=None, y=None, y_len=0, threads=None):
     return get().rope_ex(x, w, L, dims, traditional, base, scale, offset, normalize, eps,
                          forward, freqs, y, y_len, threads)
+
+
+def rms_norm_vjp(x, w, g, eps, threads=None):
+    return get().rms_norm_vjp(x, w, g, eps, threads)
+
+
+def layer_norm_vjp(x, w, g, eps, threads=None):
+    return get().layer_norm_vjp(x, w, g, eps, threads)

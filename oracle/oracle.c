@@ -287,3 +287,85 @@ int oracle_rope_ex(const void* x, const void* w, const double* freqs, double* y,
     free(nrm);
     return 0;
 }
+
+/*
+ * RmsNormVjp (x, w, g): the gradients of RmsNorm for x and w (docs.rs nuvec-core 0.5.0,
+ * Enum FastOp, variant RmsNormVjp).  With r = 1 / sqrt(mean(x^2) + eps) and
+ * y_j = x_j r w_j:
+ *   dx_j = r w_j g_j - x_j r^3 (sum_k g_k w_k x_k) / D
+ *   dw_j = sum over rows of g_j x_j r            (accumulated into dw, rows r0..r1)
+ * mag_dx / mag_dw receive the same expressions with every term replaced by its
+ * magnitude (the scale of the rounding error of a float32 evaluation).
+ */
+int oracle_rms_norm_vjp(const void* x, const void* w, const void* g, double* dx, double* dw,
+                        double* mag_dx, double* mag_dw, int64_t r0, int64_t r1, int64_t D,
+                        float eps, int dt) {
+    for (int64_t k = r0; k < r1; ++k) {
+        double sumsq = 0.0, c = 0.0, cmag = 0.0;
+        for (int64_t j = 0; j < D; ++j) {
+            double xj = widen(x, dt, k * D + j);
+            double wj = w ? widen(w, dt, j) : 1.0;
+            double gj = widen(g, dt, k * D + j);
+            sumsq += xj * xj;
+            c += gj * wj * xj;
+            cmag += fabs(gj * wj * xj);
+        }
+        double r = 1.0 / sqrt(sumsq / (double)D + (double)eps);
+        for (int64_t j = 0; j < D; ++j) {
+            double xj = widen(x, dt, k * D + j);
+            double wj = w ? widen(w, dt, j) : 1.0;
+            double gj = widen(g, dt, k * D + j);
+            dx[k * D + j] = r * wj * gj - xj * r * r * r * c / (double)D;
+            mag_dx[k * D + j] = fabs(r * wj * gj) + fabs(xj) * r * r * r * cmag / (double)D;
+            dw[j] += gj * xj * r;
+            mag_dw[j] += fabs(gj * xj * r);
+        }
+    }
+    return 0;
+}
+
+/*
+ * LayerNormVjp (x, w, b, g): the gradients of LayerNorm for x, w and b (docs.rs
+ * nuvec-core 0.5.0, Enum FastOp, variant LayerNormVjp).  With mean, var (population),
+ * r = 1 / sqrt(var + eps), xh_j = (x_j - mean) r, a_j = w_j g_j:
+ *   dx_j = r (a_j - mean_k(a_k) - xh_j mean_k(a_k xh_k))
+ *   dw_j = sum over rows of g_j xh_j,   db_j = sum over rows of g_j
+ * (accumulated into dw and db for rows r0..r1); mag_* as for RmsNormVjp.
+ */
+int oracle_layer_norm_vjp(const void* x, const void* w, const void* g, double* dx, double* dw,
+                          double* db, double* mag_dx, double* mag_dw, double* mag_db, int64_t r0,
+                          int64_t r1, int64_t D, float eps, int dt) {
+    for (int64_t k = r0; k < r1; ++k) {
+        double sum = 0.0;
+        for (int64_t j = 0; j < D; ++j) sum += widen(x, dt, k * D + j);
+        double mean = sum / (double)D;
+        double sqdev = 0.0;
+        for (int64_t j = 0; j < D; ++j) {
+            double d = widen(x, dt, k * D + j) - mean;
+            sqdev += d * d;
+        }
+        double r = 1.0 / sqrt(sqdev / (double)D + (double)eps);
+        double sa = 0.0, sax = 0.0, sa_mag = 0.0, sax_mag = 0.0;
+        for (int64_t j = 0; j < D; ++j) {
+            double xh = (widen(x, dt, k * D + j) - mean) * r;
+            double a = (w ? widen(w, dt, j) : 1.0) * widen(g, dt, k * D + j);
+            sa += a;
+            sax += a * xh;
+            sa_mag += fabs(a);
+            sax_mag += fabs(a * xh);
+        }
+        for (int64_t j = 0; j < D; ++j) {
+            double gj = widen(g, dt, k * D + j);
+            double xh = (widen(x, dt, k * D + j) - mean) * r;
+            double a = (w ? widen(w, dt, j) : 1.0) * gj;
+            dx[k * D + j] = r * (a - sa / (double)D - xh * sax / (double)D);
+            mag_dx[k * D + j] =
+                r * (fabs(a) + sa_mag / (double)D + fabs(xh) * sax_mag / (double)D);
+            dw[j] += gj * xh;
+            db[j] += gj;
+            mag_dw[j] += fabs(gj * xh);
+            mag_db[j] += fabs(gj);
+        }
+    }
+    return 0;
+}

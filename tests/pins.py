@@ -378,6 +378,80 @@ def check_rope_cache_placement(o):
                 assert (got == 7.25).all(), "a cache row outside [offset, offset+L) changed"
 
 
+# ---- backward (vector-Jacobian products) ---------------------------------------------
+
+def _fd_grad(f, v, h):
+    """Central differences of the scalar f at v (float32 array on a dyadic grid), one
+    coordinate at a time; v + h and v - h are exact in float32."""
+    out = np.zeros(v.size)
+    flat = v.reshape(-1)
+    for i in range(flat.size):
+        up, dn = flat.copy(), flat.copy()
+        up[i] += np.float32(h)
+        dn[i] -= np.float32(h)
+        out[i] = (f(up.reshape(v.shape)) - f(dn.reshape(v.shape))) / (2 * h)
+    return out.reshape(v.shape)
+
+
+def _grid(shape, seed, lo=-2.0, hi=2.0):
+    return (np.round(_rng(seed).uniform(lo, hi, shape) * 64) / 64).astype(np.float32)
+
+
+def check_rms_norm_vjp_finite_differences(o):
+    """dx and dw match central differences of the oracle's own RmsNorm."""
+    x, g = _grid((3, 6), 41), _grid((3, 6), 42)
+    w = _grid((6,), 43, 0.5, 1.5)
+    eps = float(np.float32(1e-3))
+    dx, dw, _, _ = o.rms_norm_vjp(x, w, g, eps)
+    loss = lambda xx, ww: float((o.rms_norm(xx, ww, eps) * g).sum())  # noqa: E731
+    _close(dx, _fd_grad(lambda xx: loss(xx, w), x, 2.0 ** -10), 1e-5, atol=1e-6, what="rms dx")
+    _close(dw, _fd_grad(lambda ww: loss(x, ww), w, 2.0 ** -10), 1e-5, atol=1e-6, what="rms dw")
+
+
+def check_layer_norm_vjp_finite_differences(o):
+    """dx, dw and db match central differences of the oracle's own LayerNorm."""
+    x, g = _grid((3, 6), 44), _grid((3, 6), 45)
+    w = _grid((6,), 46, 0.5, 1.5)
+    b = _grid((6,), 47, -0.5, 0.5)
+    eps = float(np.float32(1e-3))
+    dx, dw, db, _, _, _ = o.layer_norm_vjp(x, w, g, eps)
+    loss = lambda xx, ww, bb: float((o.layer_norm(xx, ww, bb, eps) * g).sum())  # noqa: E731
+    _close(dx, _fd_grad(lambda xx: loss(xx, w, b), x, 2.0 ** -10), 1e-5, atol=1e-6, what="ln dx")
+    _close(dw, _fd_grad(lambda ww: loss(x, ww, b), w, 2.0 ** -10), 1e-5, atol=1e-6, what="ln dw")
+    _close(db, _fd_grad(lambda bb: loss(x, w, bb), b, 2.0 ** -10), 1e-5, atol=1e-6, what="ln db")
+
+
+def check_vjp_invariances(o):
+    """eps = 0: RmsNorm is scale invariant (sum x dx = 0); LayerNorm is shift and scale
+    invariant (sum dx = 0, sum (x - mean) dx = 0); db is the column sum of g."""
+    x = _randn_bf16((7, 40), 48)
+    g = _randn_bf16((7, 40), 49)
+    w = bf16_bits(_rng(50).uniform(0.5, 1.5, 40))
+    xv = widen_bf16(x)
+    dx, _, _, _ = o.rms_norm_vjp(x, w, g, 0.0)
+    scale = np.abs(dx).max(axis=1) * np.abs(xv).max(axis=1) * 40
+    assert (np.abs((xv * dx).sum(axis=1)) <= 1e-13 * scale).all(), "rms: x . dx != 0"
+    dx, _, db, _, _, _ = o.layer_norm_vjp(x, w, g, 0.0)
+    s = np.abs(dx).max(axis=1) * 40
+    assert (np.abs(dx.sum(axis=1)) <= 1e-13 * s).all(), "layer: sum dx != 0"
+    xc = xv - xv.mean(axis=1, keepdims=True)
+    assert (np.abs((xc * dx).sum(axis=1)) <= 1e-12 * s * np.abs(xc).max()).all(), \
+        "layer: (x - mean) . dx != 0"
+    _close(db, widen_bf16(g).sum(axis=0), 1e-14, atol=1e-14, what="db")
+
+
+def check_vjp_without_weight(o):
+    """w = None is w = 1 and has no gradient of its own."""
+    x, g = _randn_bf16((5, 24), 51), _randn_bf16((5, 24), 52)
+    ones = bf16_bits(np.ones(24))
+    a = o.rms_norm_vjp(x, None, g, 1e-5)
+    b = o.rms_norm_vjp(x, ones, g, 1e-5)
+    assert a[1] is None and (a[0] == b[0]).all(), "rms vjp with w = None"
+    a = o.layer_norm_vjp(x, None, g, 1e-5)
+    b = o.layer_norm_vjp(x, ones, g, 1e-5)
+    assert a[1] is None and (a[0] == b[0]).all() and (a[2] == b[2]).all(), "layer vjp w = None"
+
+
 # ---- hand-worked cases -----------------------------------------------------------------
 
 _MATH = {k: getattr(math, k) for k in ("sqrt", "cos", "sin", "pi")}

@@ -59,6 +59,19 @@ MUTANTS = {
                                          "int64_t out = y_len > 0 ? (k / L) * y_len + l : k;"),
     "rope_ex_cache_row_uses_L": ("int64_t out = y_len > 0 ? (k / L) * y_len + offset + l : k;",
                                  "int64_t out = y_len > 0 ? (k / L) * L + offset + l : k;"),
+    "rms_vjp_drops_projection": ("dx[k * D + j] = r * wj * gj - xj * r * r * r * c / (double)D;",
+                                 "dx[k * D + j] = r * wj * gj;"),
+    "rms_vjp_r_squared": ("dx[k * D + j] = r * wj * gj - xj * r * r * r * c / (double)D;",
+                          "dx[k * D + j] = r * wj * gj - xj * r * r * c / (double)D;"),
+    "rms_vjp_sum_not_mean": ("dx[k * D + j] = r * wj * gj - xj * r * r * r * c / (double)D;",
+                             "dx[k * D + j] = r * wj * gj - xj * r * r * r * c;"),
+    "rms_vjp_dw_without_r": ("dw[j] += gj * xj * r;", "dw[j] += gj * xj;"),
+    "layer_vjp_drops_mean_a": ("dx[k * D + j] = r * (a - sa / (double)D - xh * sax / (double)D);",
+                               "dx[k * D + j] = r * (a - xh * sax / (double)D);"),
+    "layer_vjp_drops_xh_term": ("dx[k * D + j] = r * (a - sa / (double)D - xh * sax / (double)D);",
+                                "dx[k * D + j] = r * (a - sa / (double)D);"),
+    "layer_vjp_dw_uses_x": ("dw[j] += gj * xh;", "dw[j] += gj * widen(x, dt, k * D + j);"),
+    "layer_vjp_db_weighted": ("db[j] += gj;", "db[j] += a;"),
     "round_truncates": ("double n = rint(ldexp(a, -qexp));", "double n = trunc(ldexp(a, -qexp));"),
     "round_ties_away": ("double n = rint(ldexp(a, -qexp));", "double n = round(ldexp(a, -qexp));"),
     "round_subnormal_quantum": ("int qexp = (e < -125 ? -125 : e) - 8;", "int qexp = e - 8;"),
