@@ -34,6 +34,7 @@
 #ifndef NVNORM_H
 #define NVNORM_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)
@@ -130,6 +131,40 @@ NV_API nv_status nv_rope(const void* x, const void* w, const float* freqs, void*
                          int64_t L, int64_t y_len, int64_t D, int32_t dims, int32_t traditional,
                          float base, float scale, int64_t offset, int32_t forward,
                          int32_t normalize, float eps, nv_dtype dt, nv_stream_t stream);
+
+/*
+ * rms_norm_vjp -- docs.rs nuvec-core 0.5.0, Enum FastOp, variant RmsNormVjp: the
+ * gradients of rms_norm for x and w.  With r = 1/sqrt(mean(x^2) + eps):
+ *   dx_j = r w_j g_j - x_j r^3 (sum_k g_k w_k x_k) / D,   dw_j = sum over rows of g_j x_j r.
+ * x, g [rows, D] in (g = the gradient of y); w [D] in or NULL (w = 1); dx [rows, D] out
+ * (may be x or g); dw [D] out, given exactly when w is (w = 1 has no gradient).
+ * workspace: device memory of at least nv_norm_vjp_workspace_size(0, rows, D) bytes when
+ * dw is requested (per-CTA partial sums of the columns; contents are overwritten), else
+ * may be NULL.  dw is deterministic: the partials are added in a fixed order in double.
+ * rows == 0 with dw requested writes dw = 0.  Needs D a multiple of 16 bytes of elements,
+ * D <= 16384 (bf16) / 8192 (f32), and 16-byte aligned x, g, dx, w.
+ */
+NV_API nv_status nv_rms_norm_vjp(const void* x, const void* w, const void* g, void* dx, void* dw,
+                                 void* workspace, size_t workspace_bytes, int64_t rows, int64_t D,
+                                 float eps, nv_dtype dt, nv_stream_t stream);
+
+/*
+ * layer_norm_vjp -- docs.rs nuvec-core 0.5.0, Enum FastOp, variant LayerNormVjp: the
+ * gradients of layer_norm for x, w and b (b itself does not enter them).  With
+ * r = 1/sqrt(var + eps), xh = (x - mean) r, a = w g:
+ *   dx_j = r (a_j - mean(a) - xh_j mean(a xh)),  dw_j = sum_rows g_j xh_j,  db_j = sum_rows g_j.
+ * dw given exactly when w is; db [D] out or NULL.  workspace: at least
+ * nv_norm_vjp_workspace_size(2, rows, D) bytes when dw or db is requested.  Otherwise as
+ * nv_rms_norm_vjp.
+ */
+NV_API nv_status nv_layer_norm_vjp(const void* x, const void* w, const void* g, void* dx,
+                                   void* dw, void* db, void* workspace, size_t workspace_bytes,
+                                   int64_t rows, int64_t D, float eps, nv_dtype dt,
+                                   nv_stream_t stream);
+
+/* Workspace bytes for the vjp column sums (op 0 rms_norm_vjp, 2 layer_norm_vjp; 0 for
+ * invalid arguments). */
+NV_API size_t nv_norm_vjp_workspace_size(int32_t op, int64_t rows, int64_t D);
 
 /* Name of a status code (static storage). */
 NV_API const char* nv_status_string(nv_status status);

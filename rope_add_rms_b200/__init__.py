@@ -21,7 +21,8 @@ __all__ = [
     "nv_rms_norm", "nv_add_rms_norm", "nv_layer_norm", "nv_norm_rope", "nv_describe_plan",
     "nv_fault_count",
     "nv_rope", "rms_norm", "add_rms_norm", "layer_norm", "norm_rope", "norm_rope_into_cache",
-    "rope",
+    "rope", "nv_rms_norm_vjp", "nv_layer_norm_vjp", "nv_norm_vjp_workspace_size", "rms_norm_vjp",
+    "layer_norm_vjp",
     "PATH_AUTO", "PATH_ROWS", "PATH_GENERIC", "PATH_STAGED", "LAUNCH_DEFAULT", "LAUNCH_PLAIN",
 ]
 
@@ -97,6 +98,13 @@ def library() -> ctypes.CDLL:
     lib.nv_version.restype = ctypes.c_int32
     lib.nv_fault_count.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]
     lib.nv_fault_count.restype = ctypes.c_int
+    sz = ctypes.c_size_t
+    lib.nv_rms_norm_vjp.argtypes = [vp, vp, vp, vp, vp, vp, sz, i64, i64, f32, i32, vp]
+    lib.nv_rms_norm_vjp.restype = ctypes.c_int
+    lib.nv_layer_norm_vjp.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, i64, i64, f32, i32, vp]
+    lib.nv_layer_norm_vjp.restype = ctypes.c_int
+    lib.nv_norm_vjp_workspace_size.argtypes = [i32, i64, i64]
+    lib.nv_norm_vjp_workspace_size.restype = sz
     _lib = lib
     return lib
 
@@ -213,6 +221,39 @@ def nv_fault_count(reset: bool = False) -> int:
     return c.value
 
 
+def nv_norm_vjp_workspace_size(op: str, rows: int, D: int) -> int:
+    """Bytes of workspace the vjp column sums need (op 'rms_norm' or 'layer_norm')."""
+    return library().nv_norm_vjp_workspace_size({"rms_norm": 0, "layer_norm": 2}[op], rows, D)
+
+
+def _workspace(op, x, need, workspace):
+    if not need:
+        return None, 0
+    rows, D = _rows_D(x)
+    n = nv_norm_vjp_workspace_size(op, rows, D)
+    if workspace is None:
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=x.device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def nv_rms_norm_vjp(x, w, g, dx, dw, eps, workspace=None, stream=None):
+    """Gradients of rms_norm: dx, and dw (exactly when w is given)."""
+    rows, D = _rows_D(x)
+    ws, nbytes = _workspace("rms_norm", x, dw is not None, workspace)
+    _check("nv_rms_norm_vjp", library().nv_rms_norm_vjp(
+        _ptr(x), _ptr(w), _ptr(g), _ptr(dx), _ptr(dw), _ptr(ws), nbytes, rows, D, eps,
+        _dtype(x, w, g, dx, dw), _stream(stream)))
+
+
+def nv_layer_norm_vjp(x, w, g, dx, dw, db, eps, workspace=None, stream=None):
+    """Gradients of layer_norm: dx, dw (exactly when w is given), db (or None)."""
+    rows, D = _rows_D(x)
+    ws, nbytes = _workspace("layer_norm", x, dw is not None or db is not None, workspace)
+    _check("nv_layer_norm_vjp", library().nv_layer_norm_vjp(
+        _ptr(x), _ptr(w), _ptr(g), _ptr(dx), _ptr(dw), _ptr(db), _ptr(ws), nbytes, rows, D, eps,
+        _dtype(x, w, g, dx, dw, db), _stream(stream)))
+
+
 # ---- allocating wrappers ---------------------------------------------------------------
 
 def rms_norm(x, w=None, eps=1e-5, stream=None):
@@ -271,3 +312,20 @@ def norm_rope(x, w=None, dims=None, traditional=False, base=10000.0, scale=1.0, 
     nv_norm_rope(x, w, y, L, D if dims is None else dims, traditional, base, scale, offset,
                  normalize, eps if normalize else 0.0, stream)
     return y
+
+
+def rms_norm_vjp(x, w, g, eps=1e-5, stream=None):
+    """(dx, dw) of rms_norm for upstream gradient g; dw is None when w is None."""
+    dx = torch.empty_like(x)
+    dw = None if w is None else torch.empty_like(w)
+    nv_rms_norm_vjp(x, w, g, dx, dw, eps, stream=stream)
+    return dx, dw
+
+
+def layer_norm_vjp(x, w, g, eps=1e-5, with_db=True, stream=None):
+    """(dx, dw, db) of layer_norm for upstream gradient g; dw None when w is None."""
+    dx = torch.empty_like(x)
+    dw = None if w is None else torch.empty_like(w)
+    db = torch.empty(x.shape[-1], dtype=x.dtype, device=x.device) if with_db else None
+    nv_layer_norm_vjp(x, w, g, dx, dw, db, eps, stream=stream)
+    return dx, dw, db

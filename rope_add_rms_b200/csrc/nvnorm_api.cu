@@ -19,6 +19,7 @@
 #include "rms.cuh"
 #include "rope.cuh"
 #include "staged.cuh"
+#include "vjp.cuh"
 
 namespace {
 
@@ -629,6 +630,115 @@ nv_status rope_op(const void* x, const void* w, const float* freqs, void* y, int
               : launch_rope_generic<float>(di, p.ctas_per_sm, cs, a);
 }
 
+// ---- backward (vjp) -------------------------------------------------------------------------
+constexpr int kMaxVjpParts = 512;
+
+int vjp_parts(int64_t rows) { return (int)std::min<int64_t>(rows, kMaxVjpParts); }
+
+// Vectors per thread for the vjp kernels: 2, or 4 when the row needs more than 512 threads.
+int vjp_vpt(int nvec) {
+    if ((nvec + 1) / 2 <= 512) return 2;
+    if ((nvec + 3) / 4 <= 512) return 4;
+    return 0;
+}
+
+size_t vjp_workspace(Op op, int64_t rows, int64_t D) {
+    return (size_t)(op == OP_LAYER ? 2 : 1) * (size_t)vjp_parts(rows) * (size_t)D * sizeof(float);
+}
+
+template <typename T>
+nv_status run_vjp(Op op, const VjpArgs& a, int vpt, cudaStream_t s, void* dw, void* db) {
+    const int G = ((a.nvec + vpt - 1) / vpt + 31) / 32 * 32;
+    nv_status st = NV_OK;
+    if (a.rows > 0) {
+        if (op == OP_RMS)
+            st = vpt == 2 ? launch_kernel(rms_vjp_kernel<T, 2>, a.parts, G, 0, s, a)
+                          : launch_kernel(rms_vjp_kernel<T, 4>, a.parts, G, 0, s, a);
+        else
+            st = vpt == 2 ? launch_kernel(layer_vjp_kernel<T, 2>, a.parts, G, 0, s, a)
+                          : launch_kernel(layer_vjp_kernel<T, 4>, a.parts, G, 0, s, a);
+        if (st != NV_OK) return st;
+    }
+    const int64_t grid = (a.D + 255) / 256;
+    const int parts = a.rows > 0 ? a.parts : 0;
+    const float* pw = a.part;
+    const float* pb = a.part ? a.part + (size_t)a.parts * a.D : nullptr;
+    if (dw) {
+        st = launch_kernel(vjp_reduce_kernel<T>, grid, 256, 0, s, pw, parts, a.D, dw);
+        if (st != NV_OK) return st;
+    }
+    if (db) st = launch_kernel(vjp_reduce_kernel<T>, grid, 256, 0, s, pb, parts, a.D, db);
+    return st;
+}
+
+nv_status vjp_op(Op op, const void* x, const void* w, const void* g, void* dx, void* dw, void* db,
+                 void* ws, size_t ws_bytes, int64_t rows, int64_t D, float eps, nv_dtype dt,
+                 nv_stream_t stream) {
+    nv_status st = check_common(rows, D, eps, dt);
+    if (st != NV_OK) return st;
+    if ((dw != nullptr) != (w != nullptr))
+        return fail(NV_ERR_INVALID_ARG, "dw must be given exactly when w is (w = NULL is the "
+                    "scalar 1, which has no gradient)");
+    const size_t s = elem_size(dt);
+    const int vecw = 16 / (int)s;
+    if (D % vecw != 0 || vjp_vpt((int)(D / vecw)) == 0)
+        return fail(NV_ERR_UNSUPPORTED, "vjp needs D %% %d == 0 and D <= %d", vecw,
+                    2048 * vecw);
+    const bool sums = dw || db;
+    const size_t need = sums ? vjp_workspace(op, rows, D) : 0;
+    if (sums && rows > 0) {
+        if (!ws) return fail(NV_ERR_INVALID_ARG, "workspace is NULL (%zu bytes needed)", need);
+        if (ws_bytes < need)
+            return fail(NV_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed", ws_bytes, need);
+    }
+    if (rows > 0) {
+        if (!x) return fail(NV_ERR_INVALID_ARG, "x is NULL");
+        if (!g) return fail(NV_ERR_INVALID_ARG, "g is NULL");
+        if (!dx) return fail(NV_ERR_INVALID_ARG, "dx is NULL");
+    }
+    if (rows == 0 && !sums) return NV_OK;
+
+    int dev = 0;
+    DevInfo di;
+    st = current_device(&dev, &di);
+    if (st != NV_OK) return st;
+    const size_t nbytes = (size_t)rows * (size_t)D * s;
+    const Buf bufs[] = {
+        {rows ? x : nullptr, nbytes, "x", false, true},
+        {rows ? g : nullptr, nbytes, "g", false, true},
+        {w, (size_t)D * s, "w", false, false},
+        {rows ? dx : nullptr, nbytes, "dx", true, false},
+        {dw, (size_t)D * s, "dw", true, false},
+        {db, (size_t)D * s, "db", true, false},
+        {(sums && rows) ? ws : nullptr, need, "workspace", true, false},
+    };
+    st = check_buffers(bufs, 7, dev);
+    if (st != NV_OK) return st;
+    const bool al = (!rows || (aligned16(x) && aligned16(g) && aligned16(dx))) &&
+                    (!w || aligned16(w));
+    if (!al) return fail(NV_ERR_UNSUPPORTED, "vjp needs 16-byte aligned x, g, dx and w");
+
+    VjpArgs a{};
+    a.x = x;
+    a.w = w;
+    a.g = g;
+    a.dx = dx;
+    a.part = (sums && rows) ? static_cast<float*>(ws) : nullptr;
+    a.rows = rows;
+    a.D = (int)D;
+    a.nvec = (int)(D / vecw);
+    a.parts = rows > 0 ? (sums ? vjp_parts(rows) : (int)std::min<int64_t>(rows, (int64_t)di.sms * 8))
+                       : 0;
+    a.want_dw = dw != nullptr;
+    a.want_db = db != nullptr;
+    a.eps = eps;
+    g_pdl = true;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const int vpt = vjp_vpt(a.nvec);
+    return dt == NV_BF16 ? run_vjp<__nv_bfloat16>(op, a, vpt, cs, dw, db)
+                         : run_vjp<float>(op, a, vpt, cs, dw, db);
+}
+
 }  // namespace
 
 // ---- exported C ABI -------------------------------------------------------------------------
@@ -708,6 +818,25 @@ nv_status nv_describe_plan(int32_t op, int64_t rows, int64_t D, nv_dtype dt, nv_
         return rope_plan(rows, 1, D, (int)(D - D % 2), false, dt, true, 148, nullptr, plan, &rp);
     }
     return make_plan((Op)op, rows, D, dt, true, nullptr, plan);
+}
+
+size_t nv_norm_vjp_workspace_size(int32_t op, int64_t rows, int64_t D) {
+    if ((op != OP_RMS && op != OP_LAYER) || rows <= 0 || D <= 0) return 0;
+    return vjp_workspace((Op)op, rows, D);
+}
+
+nv_status nv_rms_norm_vjp(const void* x, const void* w, const void* g, void* dx, void* dw,
+                          void* workspace, size_t workspace_bytes, int64_t rows, int64_t D,
+                          float eps, nv_dtype dt, nv_stream_t stream) {
+    return vjp_op(OP_RMS, x, w, g, dx, dw, nullptr, workspace, workspace_bytes, rows, D, eps, dt,
+                  stream);
+}
+
+nv_status nv_layer_norm_vjp(const void* x, const void* w, const void* g, void* dx, void* dw,
+                            void* db, void* workspace, size_t workspace_bytes, int64_t rows,
+                            int64_t D, float eps, nv_dtype dt, nv_stream_t stream) {
+    return vjp_op(OP_LAYER, x, w, g, dx, dw, db, workspace, workspace_bytes, rows, D, eps, dt,
+                  stream);
 }
 
 const char* nv_status_string(nv_status status) {

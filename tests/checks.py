@@ -120,3 +120,29 @@ def sample_rows(rows: int, k: int, seed: int = 0) -> np.ndarray:
     rng = np.random.default_rng(seed)
     mid = rng.choice(np.arange(1, rows - 1), size=k - 2, replace=False)
     return np.unique(np.concatenate([[0, rows - 1], mid]))
+
+
+# ---- gradients ------------------------------------------------------------------------
+# The vjp outputs are formed in float32 from terms that can cancel; their bar, derived
+# from that arithmetic: the bfloat16 (float32) bar above, or an absolute error of at
+# most 2^-16 times the sum of the magnitudes of the terms (the oracle's mag_* output).
+
+VJP_MAG = 2.0 ** -16
+
+
+def check_grad(y_dev, ref, mag, what="grad"):
+    host = to_host_bits(y_dev).reshape(-1)
+    ref = np.asarray(ref, np.float64).reshape(-1)
+    mag = np.asarray(mag, np.float64).reshape(-1)
+    if host.dtype == np.uint16:
+        got = (host.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        dist = np.abs(bf16_ordinal(host) - bf16_ordinal(oracle.round_bf16(ref)))
+        ok = (dist <= 1) | (np.abs(got - ref) <= VJP_MAG * mag)
+    else:
+        got = host.astype(np.float64)
+        ok = (np.abs(got - ref) <= F32_TOL * (1 + np.abs(ref))) | \
+             (np.abs(got - ref) <= VJP_MAG * mag)
+    if not ok.all():
+        i = np.argmax(~ok)
+        raise AssertionError(f"{what}: {int((~ok).sum())} of {ok.size} elements off; first at "
+                             f"{i}: got {got[i]!r}, oracle {ref[i]!r}, magnitude {mag[i]!r}")

@@ -83,6 +83,14 @@ def rope_general(x=FAKE, w=None, freqs=None, y=FAKE, rows=8, L=4, y_len=0, D=8, 
                                 forward, normalize, eps, dt, None)
 
 
+def vjp(op="rms", x=FAKE, w=None, g=FAKE, dx=FAKE, dw=None, db=None, ws=None, ws_bytes=0, rows=4,
+        D=64, eps=1e-5, dt=BF16):
+    lib = nv.library()
+    if op == "rms":
+        return lib.nv_rms_norm_vjp(x, w, g, dx, dw, ws, ws_bytes, rows, D, eps, dt, None)
+    return lib.nv_layer_norm_vjp(x, w, g, dx, dw, db, ws, ws_bytes, rows, D, eps, dt, None)
+
+
 def last_error():
     return nv.library().nv_last_error().decode()
 
@@ -120,6 +128,15 @@ def last_error():
     (lambda: rope_general(base=0.0), INVALID, "base"),
     (lambda: rope_general(base=0.0, freqs=FAKE, x=None), INVALID, "x is NULL"),
     (lambda: rope_general(dims=3), INVALID, "dims"),
+    (lambda: vjp(w=FAKE), INVALID, "dw must be given"),
+    (lambda: vjp(dw=FAKE), INVALID, "dw must be given"),
+    (lambda: vjp(op="layer", w=FAKE), INVALID, "dw must be given"),
+    (lambda: vjp(w=FAKE, dw=FAKE), INVALID, "workspace is NULL"),
+    (lambda: vjp(w=FAKE, dw=FAKE, ws=FAKE, ws_bytes=16), INVALID, "workspace of 16 bytes"),
+    (lambda: vjp(op="layer", db=FAKE, ws=FAKE, ws_bytes=16), INVALID, "workspace of 16"),
+    (lambda: vjp(D=7), UNSUPPORTED, "vjp needs D"),
+    (lambda: vjp(D=32768), UNSUPPORTED, "vjp needs D"),
+    (lambda: vjp(g=None), INVALID, "g is NULL"),
 ])
 def test_invalid_arguments_are_rejected_on_the_host(call, status, words):
     assert call() == status
@@ -160,3 +177,11 @@ def test_plan_selection(op, D, dtype, want):
     p = nv.nv_describe_plan(op, 8192, D, {"bf16": torch.bfloat16, "f32": torch.float32}[dtype])
     for k, v in want.items():
         assert p[k] == v, (op, D, dtype, p)
+
+
+def test_vjp_workspace_size():
+    lib = nv.library()
+    assert lib.nv_norm_vjp_workspace_size(0, 8192, 4096) == 512 * 4096 * 4
+    assert lib.nv_norm_vjp_workspace_size(2, 100, 1024) == 2 * 100 * 1024 * 4
+    assert lib.nv_norm_vjp_workspace_size(1, 100, 1024) == 0
+    assert lib.nv_norm_vjp_workspace_size(0, 0, 1024) == 0

@@ -549,3 +549,71 @@ def test_rope_round_trip_and_cache_rules():
     with pytest.raises(nv.NvError, match="overlaps"):
         nv.nv_rope(xs, None, big[B * H * L * D // 2:][:B * H * 20 * D].view(-1, D), L, D, 0,
                    10000.0, 1.0, 0, 0, 0.0, y_len=20)
+
+
+# ---- gradients -----------------------------------------------------------------------------
+
+from checks import check_grad  # noqa: E402
+
+VJP_SHAPES = [(256, 4096), (1000, 2048), (33, 8192), (1, 512), (2000, 1024), (7, 16384)]
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("weight", [True, False])
+@pytest.mark.parametrize("rows,D", VJP_SHAPES)
+def test_rms_norm_vjp(rows, D, weight, dt):
+    if dt == "f32" and D > 8192:
+        pytest.skip("float32 rows are limited to 8192")
+    inp = synth.rms_inputs(rows, D, dt, seed=rows + D, weight=weight)
+    g = synth.normal((rows, D), 0.0, 1.0, rows + D, 4, dt)
+    x, w, gd = dev(inp["x"]), dev(inp["w"]), dev(g)
+    dx, dw = nv.rms_norm_vjp(x, w, gd, eps=1e-5)
+    torch.cuda.synchronize()
+    ref_dx, ref_dw, mag_dx, mag_dw = oracle.rms_norm_vjp(host(inp["x"]), host(inp["w"]), host(g),
+                                                         1e-5)
+    check_grad(dx, ref_dx, mag_dx, "dx")
+    if weight:
+        check_grad(dw, ref_dw, mag_dw, "dw")
+    else:
+        assert dw is None
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("weight", [True, False])
+@pytest.mark.parametrize("rows,D", VJP_SHAPES)
+def test_layer_norm_vjp(rows, D, weight, dt):
+    if dt == "f32" and D > 8192:
+        pytest.skip("float32 rows are limited to 8192")
+    inp = synth.layer_norm_inputs(rows, D, dt, seed=rows * 3 + D, weight=weight, bias=False)
+    g = synth.normal((rows, D), 0.0, 1.0, rows * 3 + D, 4, dt)
+    x, w, gd = dev(inp["x"]), dev(inp["w"]), dev(g)
+    dx, dw, db = nv.layer_norm_vjp(x, w, gd, eps=1e-5)
+    torch.cuda.synchronize()
+    ref = oracle.layer_norm_vjp(host(inp["x"]), host(inp["w"]), host(g), 1e-5)
+    check_grad(dx, ref[0], ref[3], "dx")
+    if weight:
+        check_grad(dw, ref[1], ref[4], "dw")
+    check_grad(db, ref[2], ref[5], "db")
+
+
+def test_vjp_deterministic_in_place_and_empty():
+    inp = synth.rms_inputs(3000, 4096, "bf16", seed=9)
+    g = synth.normal((3000, 4096), 0.0, 1.0, 9, 4, "bf16").cuda()
+    x, w = dev(inp["x"]), dev(inp["w"])
+    a = nv.rms_norm_vjp(x, w, g)
+    b = nv.rms_norm_vjp(x, w, g)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
+    assert torch.equal(a[1].view(torch.int16), b[1].view(torch.int16)), "dw must be deterministic"
+    gg = g.clone()
+    dw = torch.empty_like(w)
+    nv.nv_rms_norm_vjp(x, w, gg, gg, dw, 1e-5)         # dx written over g
+    torch.cuda.synchronize()
+    assert torch.equal(gg.view(torch.int16), a[0].view(torch.int16))
+    empty = torch.empty(0, 4096, dtype=torch.bfloat16, device="cuda")
+    dw0 = torch.full_like(w, 3.0)
+    nv.nv_rms_norm_vjp(empty, w, empty, empty, dw0, 1e-5)
+    db0 = torch.full_like(w, 3.0)
+    nv.nv_layer_norm_vjp(empty, None, empty, empty, None, db0, 1e-5)
+    torch.cuda.synchronize()
+    assert (dw0 == 0).all() and (db0 == 0).all(), "an empty batch has zero column gradients"
