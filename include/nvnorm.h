@@ -166,6 +166,31 @@ NV_API nv_status nv_layer_norm_vjp(const void* x, const void* w, const void* g, 
  * invalid arguments). */
 NV_API size_t nv_norm_vjp_workspace_size(int32_t op, int64_t rows, int64_t D);
 
+/*
+ * rms_norm_vjp_static -- nv_rms_norm_vjp for callers that cannot allocate device memory.
+ * The op definitions this library follows have no counterpart of this entry point: it
+ * exists for callers that are handed their input and output buffers and may not allocate
+ * more -- a plugin inside an inference engine or graph runtime that owns all memory, code
+ * under a fixed memory budget, or a hot loop where cudaMalloc would synchronise the
+ * device.  The caller passes x, w, g, dx and dw exactly as for nv_rms_norm_vjp, but no
+ * workspace: the per-CTA partial sums of dw go to a fixed 4 MiB array in device memory
+ * that the library declares (every GPU that loads the library holds it until the process
+ * exits).  Nothing is allocated, and nothing needs clearing: each call writes every
+ * partial row it later reads.
+ *   - Limit: D <= 16384 (and the limits of nv_rms_norm_vjp); a larger D returns
+ *     NV_ERR_UNSUPPORTED.  The number of partial rows is min(rows, 512, 2^20 / D), so dw
+ *     can differ from nv_rms_norm_vjp's in the last bits (another summation grouping);
+ *     dx is the same.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls share the one array: two calls whose kernels overlap on the GPU (on
+ *     different streams without ordering) race and may corrupt each other's dw.
+ */
+NV_API nv_status nv_rms_norm_vjp_static(const void* x, const void* w, const void* g, void* dx,
+                                        void* dw, int64_t rows, int64_t D, float eps,
+                                        nv_dtype dt, nv_stream_t stream);
+
 /* Name of a status code (static storage). */
 NV_API const char* nv_status_string(nv_status status);
 

@@ -739,6 +739,96 @@ nv_status vjp_op(Op op, const void* x, const void* w, const void* g, void* dx, v
                          : run_vjp<float>(op, a, vpt, cs, dw, db);
 }
 
+// ---- rms_norm_vjp without caller-provided workspace -------------------------------------------
+// Scratch for the dw partials of nv_rms_norm_vjp_static: a fixed array in device memory
+// that every GPU loading the library holds until the process exits.  Host code must not
+// use the symbol as an address; the device address comes from cudaGetSymbolAddress.
+constexpr int64_t kStaticScratchFloats = (int64_t)1 << 20;  // 4 MiB
+constexpr int64_t kStaticMaxD = 16384;
+static __device__ __align__(256) float nvn_static_scratch[kStaticScratchFloats];
+
+float* g_static_scratch[kMaxDevices] = {};
+std::mutex g_static_mu;
+
+// Device address of the scratch array on the current device, fetched on first use.
+nv_status static_scratch(int dev, float** out) {
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    if (!g_static_scratch[dev]) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, nvn_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+        g_static_scratch[dev] = static_cast<float*>(p);
+    }
+    *out = g_static_scratch[dev];
+    return NV_OK;
+}
+
+nv_status rms_vjp_static(const void* x, const void* w, const void* g, void* dx, void* dw,
+                         int64_t rows, int64_t D, float eps, nv_dtype dt, nv_stream_t stream) {
+    nv_status st = check_common(rows, D, eps, dt);
+    if (st != NV_OK) return st;
+    if (D > kStaticMaxD)
+        return fail(NV_ERR_UNSUPPORTED, "nv_rms_norm_vjp_static: D = %lld exceeds %lld, the "
+                    "widest row its fixed %lld-float scratch is sized for", (long long)D,
+                    (long long)kStaticMaxD, (long long)kStaticScratchFloats);
+    if ((dw != nullptr) != (w != nullptr))
+        return fail(NV_ERR_INVALID_ARG, "dw must be given exactly when w is (w = NULL is the "
+                    "scalar 1, which has no gradient)");
+    const size_t s = elem_size(dt);
+    const int vecw = 16 / (int)s;
+    if (D % vecw != 0 || vjp_vpt((int)(D / vecw)) == 0)
+        return fail(NV_ERR_UNSUPPORTED, "vjp needs D %% %d == 0 and D <= %d", vecw,
+                    2048 * vecw);
+    if (rows > 0 && (!x || !g || !dx))
+        return fail(NV_ERR_INVALID_ARG, "x, g and dx must not be NULL");
+    if (rows == 0 && !dw) return NV_OK;
+
+    int dev = 0;
+    DevInfo di;
+    st = current_device(&dev, &di);
+    if (st != NV_OK) return st;
+    float* scratch = nullptr;
+    if (dw) {
+        st = static_scratch(dev, &scratch);
+        if (st != NV_OK) return st;
+    }
+    const size_t nbytes = (size_t)rows * (size_t)D * s;
+    const Buf bufs[] = {
+        {rows ? x : nullptr, nbytes, "x", false, true},
+        {rows ? g : nullptr, nbytes, "g", false, true},
+        {w, (size_t)D * s, "w", false, false},
+        {rows ? dx : nullptr, nbytes, "dx", true, false},
+        {dw, (size_t)D * s, "dw", true, false},
+    };
+    st = check_buffers(bufs, 5, dev);
+    if (st != NV_OK) return st;
+    if (!((!rows || (aligned16(x) && aligned16(g) && aligned16(dx))) && (!w || aligned16(w))))
+        return fail(NV_ERR_UNSUPPORTED, "vjp needs 16-byte aligned x, g, dx and w");
+
+    VjpArgs a{};
+    a.x = x;
+    a.w = w;
+    a.g = g;
+    a.dx = dx;
+    a.rows = rows;
+    a.D = (int)D;
+    a.nvec = (int)(D / vecw);
+    // as many partial rows as the scratch holds (at least 64 at the widest D)
+    const int64_t fit = kStaticScratchFloats / D;
+    a.parts = rows > 0 ? (dw ? (int)std::min<int64_t>(std::min<int64_t>(rows, kMaxVjpParts), fit)
+                              : (int)std::min<int64_t>(rows, (int64_t)di.sms * 8))
+                       : 0;
+    a.part = (dw && rows) ? scratch : nullptr;
+    a.want_dw = dw != nullptr;
+    a.want_db = 0;
+    a.eps = eps;
+    g_pdl = true;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const int vpt = vjp_vpt(a.nvec);
+    return dt == NV_BF16 ? run_vjp<__nv_bfloat16>(OP_RMS, a, vpt, cs, dw, nullptr)
+                         : run_vjp<float>(OP_RMS, a, vpt, cs, dw, nullptr);
+}
+
 }  // namespace
 
 // ---- exported C ABI -------------------------------------------------------------------------
@@ -818,6 +908,12 @@ nv_status nv_describe_plan(int32_t op, int64_t rows, int64_t D, nv_dtype dt, nv_
         return rope_plan(rows, 1, D, (int)(D - D % 2), false, dt, true, 148, nullptr, plan, &rp);
     }
     return make_plan((Op)op, rows, D, dt, true, nullptr, plan);
+}
+
+nv_status nv_rms_norm_vjp_static(const void* x, const void* w, const void* g, void* dx, void* dw,
+                                 int64_t rows, int64_t D, float eps, nv_dtype dt,
+                                 nv_stream_t stream) {
+    return rms_vjp_static(x, w, g, dx, dw, rows, D, eps, dt, stream);
 }
 
 size_t nv_norm_vjp_workspace_size(int32_t op, int64_t rows, int64_t D) {
