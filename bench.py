@@ -179,6 +179,10 @@ def algorithmic_bytes(op, rows, D, s):
         return 2 * rows * D * s + 2 * D * s
     if op == "norm_rope":
         return 2 * rows * D * s + D * s
+    if op == "rms_norm_vjp":          # read x, g, w; write dx, dw
+        return 3 * rows * D * s + 2 * D * s
+    if op == "layer_norm_vjp":        # read x, g, w; write dx, dw, db
+        return 3 * rows * D * s + 3 * D * s
     raise ValueError(op)
 
 
@@ -204,16 +208,27 @@ class Case:
         else:
             rows, D = shape
             self.rows, self.D = rows, D
-            if op == "add_rms_norm":
+            if op == "add_rms_norm" and rows * D > (1 << 27):
+                # hundreds of millions of values: drawn on the device (same recipe)
+                inp = {"x": synth.normal_device((rows, D), 0.0, 1.0, seed, synth.X, dtype),
+                       "r": synth.normal_device((rows, D), 0.0, 1.0, seed, synth.R, dtype),
+                       "w": synth.uniform_device((D,), 0.5, 1.5, seed, synth.W, dtype)}
+            elif op == "add_rms_norm":
                 inp = synth.add_rms_inputs(rows, D, dtype, seed)
-            elif op == "rms_norm":
+            elif op in ("rms_norm", "rms_norm_vjp"):
                 inp = synth.rms_inputs(rows, D, dtype, seed)
             else:
                 inp = synth.layer_norm_inputs(rows, D, dtype, seed)
-        self.host = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+            if op.endswith("_vjp"):
+                inp["r"] = synth.normal((rows, D), 0.0, 1.0, seed, synth.R, dtype)  # g
+        on_dev = any(v is not None and v.is_cuda for v in inp.values())
+        self.host = {k: (v.pin_memory() if v is not None and not on_dev else None)
+                     for k, v in inp.items()}
+        self.device_drawn = on_dev
+        src = inp if on_dev else self.host
         self.bytes = algorithmic_bytes(op, self.rows, self.D, self.s)
         l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
-        n_row_tensors = 4 if op == "add_rms_norm" else 2
+        n_row_tensors = 4 if op == "add_rms_norm" else (3 if op.endswith("_vjp") else 2)
         set_bytes = n_row_tensors * self.rows * self.D * self.s
         if set_bytes >= l2:
             self.nsets = max(2, min(8, -(-3 * l2 // set_bytes)))
@@ -221,13 +236,20 @@ class Case:
             self.nsets = 1
         self.sets = []
         for _ in range(self.nsets):
-            d = {k: (v.cuda() if v is not None else None) for k, v in self.host.items()}
+            d = {k: (v.clone() if on_dev else v.cuda()) if v is not None else None
+                 for k, v in src.items()}
             d["y"] = torch.empty_like(d["x"])
             d["h"] = torch.empty_like(d["x"]) if op == "add_rms_norm" else None
+            if op.endswith("_vjp"):
+                d["dw"] = torch.empty_like(d["w"])
+                d["db"] = torch.empty_like(d["w"])
+                d["ws"] = torch.empty(max(1, nv.nv_norm_vjp_workspace_size(
+                    op[:-4], rows, D)), dtype=torch.uint8, device="cuda")
             self.sets.append(d)
         self.nv = nv
         n_out = 2 if op == "add_rms_norm" else 1
-        self.host_out = [torch.empty_like(self.host["x"]).pin_memory() for _ in range(n_out)]
+        self.host_out = [] if on_dev else \
+            [torch.empty_like(self.host["x"]).pin_memory() for _ in range(n_out)]
         self.plan = None
 
     @property
@@ -236,7 +258,9 @@ class Case:
 
     def l2_note(self):
         if self.rotating:
-            mb = self.nsets * (4 if self.op == "add_rms_norm" else 2) * self.rows * self.D * self.s
+            mb = self.nsets * (4 if self.op == "add_rms_norm" else (3 if self.op.endswith("_vjp")
+                                                                  else 2)) \
+            * self.rows * self.D * self.s
             return (f"inputs larger than L2: {self.nsets} buffer sets ({mb / 1e6:.0f} MB) "
                     "rotated, steps back to back, no flush")
         return "L2 flushed before every step (write of 2x L2)"
@@ -249,6 +273,11 @@ class Case:
             nv.nv_rms_norm(d["x"], d["w"], d["y"], k["eps"], stream, self.plan)
         elif self.op == "layer_norm":
             nv.nv_layer_norm(d["x"], d["w"], d["b"], d["y"], k["eps"], stream, self.plan)
+        elif self.op == "rms_norm_vjp":
+            nv.nv_rms_norm_vjp(d["x"], d["w"], d["r"], d["y"], d["dw"], k["eps"], d["ws"], stream)
+        elif self.op == "layer_norm_vjp":
+            nv.nv_layer_norm_vjp(d["x"], d["w"], d["r"], d["y"], d["dw"], d["db"], k["eps"],
+                                 d["ws"], stream)
         else:
             nv.nv_norm_rope(d["x"], d["w"], d["y"], self.L, k["dims"], k["traditional"], k["base"],
                             k["scale"], k["offset"], 1, k["eps"], stream, self.plan)
@@ -514,6 +543,8 @@ WORKLOADS = {
     "norm_rope_traditional": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,
                                           dims=128, traditional=1, base=10000.0, scale=1.0,
                                           offset=4096),
+    "rms_norm_vjp": lambda: Case("rms_norm_vjp", (8192, 4096), "bf16", 0, eps=1e-5),
+    "layer_norm_vjp": lambda: Case("layer_norm_vjp", (16384, 8192), "bf16", 0, eps=1e-5),
 }
 
 

@@ -519,7 +519,7 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
         int64_t bt = p.rows_per_cta;
         if (bt <= 0) {
             const int64_t target = (rows + 8LL * sms - 1) / (8LL * sms);
-            bt = std::max<int64_t>(slots * (rp->pairs ? 2 : 4), std::min<int64_t>(target, 256));
+            bt = std::max<int64_t>(slots * (rp->pairs ? 3 : 4), std::min<int64_t>(target, 256));
             bt = std::min<int64_t>(bt, std::max<int64_t>(BH, 1));
         }
         rp->lpr = lpr;
