@@ -631,43 +631,57 @@ nv_status rope_op(const void* x, const void* w, const float* freqs, void* y, int
 }
 
 // ---- backward (vjp) -------------------------------------------------------------------------
-constexpr int kMaxVjpParts = 512;
+// Partial rows kept for the column sums: enough CTAs to fill the GPU at every D (up to
+// 148 SMs x 32 CTAs for the narrowest rows) while the workspace stays <= 8 MiB per sum
+// at D <= 4096 (512 x D x 4 bytes beyond that).
+int vjp_parts_cap(int64_t D) {
+    return (int)std::max<int64_t>(512, ((int64_t)1 << 21) / std::max<int64_t>(D, 1));
+}
 
-int vjp_parts(int64_t rows) { return (int)std::min<int64_t>(rows, kMaxVjpParts); }
+int vjp_parts(int64_t rows, int64_t D) {
+    return (int)std::min<int64_t>(rows, vjp_parts_cap(D));
+}
 
-// Vectors per thread for the vjp kernels: 2, or 4 when the row needs more than 512 threads.
+// Vectors per thread for the vjp kernels: 1 (one thread per vector, next row in flight)
+// up to 1024 vectors a row, 2 up to 2048.
 int vjp_vpt(int nvec) {
-    if ((nvec + 1) / 2 <= 512) return 2;
-    if ((nvec + 3) / 4 <= 512) return 4;
+    if (nvec <= kVjpThreads) return 1;
+    if ((nvec + 1) / 2 <= kVjpThreads) return 2;
     return 0;
 }
 
 size_t vjp_workspace(Op op, int64_t rows, int64_t D) {
-    return (size_t)(op == OP_LAYER ? 2 : 1) * (size_t)vjp_parts(rows) * (size_t)D * sizeof(float);
+    return (size_t)(op == OP_LAYER ? 2 : 1) * (size_t)vjp_parts(rows, D) * (size_t)D *
+           sizeof(float);
 }
 
+// Kernel 1 runs one wave: `parts` = min(rows, cap, SMs x resident CTAs per SM), so no
+// SM idles through a partial second wave.
 template <typename T>
-nv_status run_vjp(Op op, const VjpArgs& a, int vpt, cudaStream_t s, void* dw, void* db) {
+nv_status run_vjp(Op op, VjpArgs a, int vpt, int cap, const DevInfo& di, cudaStream_t s,
+                  void* dw, void* db) {
     const int G = ((a.nvec + vpt - 1) / vpt + 31) / 32 * 32;
+    auto k1 = op == OP_RMS ? (vpt == 1 ? rms_vjp_kernel<T, 1> : rms_vjp_kernel<T, 2>)
+                           : (vpt == 1 ? layer_vjp_kernel<T, 1> : layer_vjp_kernel<T, 2>);
     nv_status st = NV_OK;
     if (a.rows > 0) {
-        if (op == OP_RMS)
-            st = vpt == 2 ? launch_kernel(rms_vjp_kernel<T, 2>, a.parts, G, 0, s, a)
-                          : launch_kernel(rms_vjp_kernel<T, 4>, a.parts, G, 0, s, a);
-        else
-            st = vpt == 2 ? launch_kernel(layer_vjp_kernel<T, 2>, a.parts, G, 0, s, a)
-                          : launch_kernel(layer_vjp_kernel<T, 4>, a.parts, G, 0, s, a);
+        const int64_t wave = (int64_t)di.sms * occupancy(k1, G, 0);
+        a.parts = (int)std::min<int64_t>(std::min<int64_t>(a.rows, cap), wave);
+        st = launch_kernel(k1, a.parts, G, 0, s, a);
         if (st != NV_OK) return st;
     }
-    const int64_t grid = (a.D + 255) / 256;
+    const int64_t grid = (a.D + 31) / 32;
     const int parts = a.rows > 0 ? a.parts : 0;
     const float* pw = a.part;
     const float* pb = a.part ? a.part + (size_t)a.parts * a.D : nullptr;
     if (dw) {
-        st = launch_kernel(vjp_reduce_kernel<T>, grid, 256, 0, s, pw, parts, a.D, dw);
+        st = launch_kernel(vjp_reduce_kernel<T>, grid, kReduceWarps * 32, 0, s, pw, parts,
+                           a.D, dw);
         if (st != NV_OK) return st;
     }
-    if (db) st = launch_kernel(vjp_reduce_kernel<T>, grid, 256, 0, s, pb, parts, a.D, db);
+    if (db)
+        st = launch_kernel(vjp_reduce_kernel<T>, grid, kReduceWarps * 32, 0, s, pb, parts, a.D,
+                           db);
     return st;
 }
 
@@ -727,16 +741,16 @@ nv_status vjp_op(Op op, const void* x, const void* w, const void* g, void* dx, v
     a.rows = rows;
     a.D = (int)D;
     a.nvec = (int)(D / vecw);
-    a.parts = rows > 0 ? (sums ? vjp_parts(rows) : (int)std::min<int64_t>(rows, (int64_t)di.sms * 8))
-                       : 0;
+    a.parts = 0;  // set from the occupancy in run_vjp
     a.want_dw = dw != nullptr;
     a.want_db = db != nullptr;
     a.eps = eps;
     g_pdl = true;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     const int vpt = vjp_vpt(a.nvec);
-    return dt == NV_BF16 ? run_vjp<__nv_bfloat16>(op, a, vpt, cs, dw, db)
-                         : run_vjp<float>(op, a, vpt, cs, dw, db);
+    const int cap = vjp_parts_cap(D);
+    return dt == NV_BF16 ? run_vjp<__nv_bfloat16>(op, a, vpt, cap, di, cs, dw, db)
+                         : run_vjp<float>(op, a, vpt, cap, di, cs, dw, db);
 }
 
 // ---- rms_norm_vjp without caller-provided workspace -------------------------------------------
@@ -814,10 +828,8 @@ nv_status rms_vjp_static(const void* x, const void* w, const void* g, void* dx, 
     a.D = (int)D;
     a.nvec = (int)(D / vecw);
     // as many partial rows as the scratch holds (at least 64 at the widest D)
-    const int64_t fit = kStaticScratchFloats / D;
-    a.parts = rows > 0 ? (dw ? (int)std::min<int64_t>(std::min<int64_t>(rows, kMaxVjpParts), fit)
-                              : (int)std::min<int64_t>(rows, (int64_t)di.sms * 8))
-                       : 0;
+    const int cap = (int)std::min<int64_t>(vjp_parts_cap(D), kStaticScratchFloats / D);
+    a.parts = 0;
     a.part = (dw && rows) ? scratch : nullptr;
     a.want_dw = dw != nullptr;
     a.want_db = 0;
@@ -825,8 +837,8 @@ nv_status rms_vjp_static(const void* x, const void* w, const void* g, void* dx, 
     g_pdl = true;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     const int vpt = vjp_vpt(a.nvec);
-    return dt == NV_BF16 ? run_vjp<__nv_bfloat16>(OP_RMS, a, vpt, cs, dw, nullptr)
-                         : run_vjp<float>(OP_RMS, a, vpt, cs, dw, nullptr);
+    return dt == NV_BF16 ? run_vjp<__nv_bfloat16>(OP_RMS, a, vpt, cap, di, cs, dw, nullptr)
+                         : run_vjp<float>(OP_RMS, a, vpt, cap, di, cs, dw, nullptr);
 }
 
 }  // namespace

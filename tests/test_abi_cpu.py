@@ -185,3 +185,6 @@ def test_vjp_workspace_size():
     assert lib.nv_norm_vjp_workspace_size(2, 100, 1024) == 2 * 100 * 1024 * 4
     assert lib.nv_norm_vjp_workspace_size(1, 100, 1024) == 0
     assert lib.nv_norm_vjp_workspace_size(0, 0, 1024) == 0
+    # narrow rows keep more partial sums (up to 2^21 / D of them)
+    assert lib.nv_norm_vjp_workspace_size(0, 100000, 512) == 4096 * 512 * 4
+    assert lib.nv_norm_vjp_workspace_size(2, 100000, 16384) == 2 * 512 * 16384 * 4

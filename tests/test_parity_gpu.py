@@ -596,6 +596,40 @@ def test_layer_norm_vjp(rows, D, weight, dt):
     check_grad(db, ref[2], ref[5], "db")
 
 
+@pytest.mark.parametrize("dt,mean,std", [("bf16", 300.0, 0.5), ("bf16", 3000.0, 40.0),
+                                         ("f32", 300.0, 0.5), ("f32", -2.0e4, 3.0)])
+def test_layer_norm_vjp_large_mean(dt, mean, std):
+    # |mean| / std up to ~7000: the row mean has to be carried past float32 rounding of |mean|
+    rows, D = 96, 4096
+    x = synth.normal((rows, D), mean, std, 31, 0, dt)
+    w = synth.normal((D,), 1.0, 0.1, 31, 2, dt)
+    g = synth.normal((rows, D), 0.0, 1.0, 31, 4, dt)
+    dx, dw, db = nv.layer_norm_vjp(dev(x), dev(w), dev(g), eps=1e-5)
+    torch.cuda.synchronize()
+    ref = oracle.layer_norm_vjp(host(x), host(w), host(g), 1e-5)
+    check_grad(dx, ref[0], ref[3], "dx")
+    check_grad(dw, ref[1], ref[4], "dw")
+    check_grad(db, ref[2], ref[5], "db")
+
+
+@pytest.mark.parametrize("rows,D", [(20000, 512), (5000, 64), (3001, 1024)])
+def test_vjp_many_narrow_rows(rows, D):
+    # more rows than partial sums: every CTA walks many rows
+    inp = synth.layer_norm_inputs(rows, D, "bf16", seed=rows, weight=True, bias=False)
+    g = synth.normal((rows, D), 0.0, 1.0, rows, 4, "bf16")
+    x, w, gd = dev(inp["x"]), dev(inp["w"]), dev(g)
+    dx, dw, db = nv.layer_norm_vjp(x, w, gd, eps=1e-5)
+    rdx, rdw = nv.rms_norm_vjp(x, w, gd, eps=1e-5)
+    torch.cuda.synchronize()
+    ref = oracle.layer_norm_vjp(host(inp["x"]), host(inp["w"]), host(g), 1e-5)
+    check_grad(dx, ref[0], ref[3], "dx")
+    check_grad(dw, ref[1], ref[4], "dw")
+    check_grad(db, ref[2], ref[5], "db")
+    rref = oracle.rms_norm_vjp(host(inp["x"]), host(inp["w"]), host(g), 1e-5)
+    check_grad(rdx, rref[0], rref[2], "rms dx")
+    check_grad(rdw, rref[1], rref[3], "rms dw")
+
+
 def test_vjp_deterministic_in_place_and_empty():
     inp = synth.rms_inputs(3000, 4096, "bf16", seed=9)
     g = synth.normal((3000, 4096), 0.0, 1.0, 9, 4, "bf16").cuda()
