@@ -642,11 +642,14 @@ int vjp_parts(int64_t rows, int64_t D) {
     return (int)std::min<int64_t>(rows, vjp_parts_cap(D));
 }
 
-// Vectors per thread for the vjp kernels: 1 (one thread per vector, next row in flight)
-// up to 1024 vectors a row, 2 up to 2048.
-int vjp_vpt(int nvec) {
-    if (nvec <= kVjpThreads) return 1;
-    if ((nvec + 1) / 2 <= kVjpThreads) return 2;
+// Vectors per thread for the vjp kernels (measured on B200, bf16, 2^26 elements):
+// rms_norm_vjp runs one thread per vector up to 1024 vectors a row; layer_norm_vjp, with
+// five row sums and two reductions a row, is faster with 2 vectors a thread from 129
+// vectors on (fewer warps per row to reduce).  4 vectors a thread up to 2048.
+int vjp_vpt(Op op, int nvec) {
+    if (nvec <= (op == OP_LAYER ? 128 : vjp_max_threads(1))) return 1;
+    if (op == OP_LAYER && (nvec + 1) / 2 <= vjp_max_threads(2)) return 2;
+    if ((nvec + 3) / 4 <= vjp_max_threads(4)) return 4;
     return 0;
 }
 
@@ -661,8 +664,11 @@ template <typename T>
 nv_status run_vjp(Op op, VjpArgs a, int vpt, int cap, const DevInfo& di, cudaStream_t s,
                   void* dw, void* db) {
     const int G = ((a.nvec + vpt - 1) / vpt + 31) / 32 * 32;
-    auto k1 = op == OP_RMS ? (vpt == 1 ? rms_vjp_kernel<T, 1> : rms_vjp_kernel<T, 2>)
-                           : (vpt == 1 ? layer_vjp_kernel<T, 1> : layer_vjp_kernel<T, 2>);
+    auto k1 = op == OP_RMS
+                  ? (vpt == 1 ? rms_vjp_kernel<T, 1>
+                              : vpt == 2 ? rms_vjp_kernel<T, 2> : rms_vjp_kernel<T, 4>)
+                  : (vpt == 1 ? layer_vjp_kernel<T, 1>
+                              : vpt == 2 ? layer_vjp_kernel<T, 2> : layer_vjp_kernel<T, 4>);
     nv_status st = NV_OK;
     if (a.rows > 0) {
         const int64_t wave = (int64_t)di.sms * occupancy(k1, G, 0);
@@ -695,7 +701,7 @@ nv_status vjp_op(Op op, const void* x, const void* w, const void* g, void* dx, v
                     "scalar 1, which has no gradient)");
     const size_t s = elem_size(dt);
     const int vecw = 16 / (int)s;
-    if (D % vecw != 0 || vjp_vpt((int)(D / vecw)) == 0)
+    if (D % vecw != 0 || vjp_vpt(op, (int)(D / vecw)) == 0)
         return fail(NV_ERR_UNSUPPORTED, "vjp needs D %% %d == 0 and D <= %d", vecw,
                     2048 * vecw);
     const bool sums = dw || db;
@@ -747,7 +753,7 @@ nv_status vjp_op(Op op, const void* x, const void* w, const void* g, void* dx, v
     a.eps = eps;
     g_pdl = true;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    const int vpt = vjp_vpt(a.nvec);
+    const int vpt = vjp_vpt(op, a.nvec);
     const int cap = vjp_parts_cap(D);
     return dt == NV_BF16 ? run_vjp<__nv_bfloat16>(op, a, vpt, cap, di, cs, dw, db)
                          : run_vjp<float>(op, a, vpt, cap, di, cs, dw, db);
@@ -790,7 +796,7 @@ nv_status rms_vjp_static(const void* x, const void* w, const void* g, void* dx, 
                     "scalar 1, which has no gradient)");
     const size_t s = elem_size(dt);
     const int vecw = 16 / (int)s;
-    if (D % vecw != 0 || vjp_vpt((int)(D / vecw)) == 0)
+    if (D % vecw != 0 || vjp_vpt(OP_RMS, (int)(D / vecw)) == 0)
         return fail(NV_ERR_UNSUPPORTED, "vjp needs D %% %d == 0 and D <= %d", vecw,
                     2048 * vecw);
     if (rows > 0 && (!x || !g || !dx))
@@ -836,7 +842,7 @@ nv_status rms_vjp_static(const void* x, const void* w, const void* g, void* dx, 
     a.eps = eps;
     g_pdl = true;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    const int vpt = vjp_vpt(a.nvec);
+    const int vpt = vjp_vpt(OP_RMS, a.nvec);
     return dt == NV_BF16 ? run_vjp<__nv_bfloat16>(OP_RMS, a, vpt, cap, di, cs, dw, nullptr)
                          : run_vjp<float>(OP_RMS, a, vpt, cap, di, cs, dw, nullptr);
 }

@@ -48,25 +48,72 @@ struct VjpArgs {
     float eps;
 };
 
-// Largest CTA of kernel 1: one thread per vector for VPT = 1 up to 1024 vectors a row.
-constexpr int kVjpThreads = 1024;
+// CTA size bound of kernel 1 by vectors per thread: one thread per vector up to 1024
+// vectors a row (64 registers a thread); 2 or 4 vectors a thread at up to 512 threads
+// (128 registers).
+constexpr int vjp_max_threads(int vpt) { return vpt == 1 ? 1024 : 512; }
 
-// Sum of N floats across the CTA with one barrier: warp butterflies, one partial per warp
-// in `buf`, then every warp reduces the partials itself with the same butterfly, so all
-// threads end with bit-identical totals.  `buf` holds N x 32 floats.
+// Warp sums of N (2 or 3) values at once: the first levels of the butterfly halve the set
+// of sums each lane carries (a lane keeps one half and sends the other to its partner),
+// so N sums cost 5 (N = 2) or 6 (N = 3) shuffles rather than 5 N.  On return lane l holds
+// the warp total of sum l / kLanesPerSum<N> (N = 3: lanes 24-31 hold a zero pad sum);
+// lanes holding the same sum hold bit-identical values.
 template <int N>
-__device__ __forceinline__ void cta_sum(float (&v)[N], float (*buf)[32]) {
-#pragma unroll
-    for (int i = 0; i < N; ++i) v[i] = warp_sum(v[i]);
-    const int nw = blockDim.x >> 5;
-    if (nw == 1) return;
+constexpr int kLanesPerSum = N == 2 ? 16 : 8;
+
+template <int N>
+__device__ __forceinline__ float warp_sums(const float (&v)[N]) {
+    static_assert(N == 2 || N == 3, "two or three sums");
     const int lane = threadIdx.x & 31;
-    if (lane == 0)
+    float keep;
+    if constexpr (N == 2) {
+        const bool hi = lane & 16;
+        keep = hi ? v[1] : v[0];
+        keep += __shfl_xor_sync(0xFFFFFFFFu, hi ? v[0] : v[1], 16);
+    } else {
+        const bool b4 = lane & 16, b3 = lane & 8;
+        float k0 = b4 ? v[2] : v[0], k1 = b4 ? 0.f : v[1];
+        k0 += __shfl_xor_sync(0xFFFFFFFFu, b4 ? v[0] : v[2], 16);
+        k1 += __shfl_xor_sync(0xFFFFFFFFu, b4 ? v[1] : 0.f, 16);
+        keep = b3 ? k1 : k0;
+        keep += __shfl_xor_sync(0xFFFFFFFFu, b3 ? k0 : k1, 8);
+    }
 #pragma unroll
-        for (int i = 0; i < N; ++i) buf[i][threadIdx.x >> 5] = v[i];
+    for (int off = kLanesPerSum<N> / 2; off >= 1; off >>= 1)
+        keep += __shfl_xor_sync(0xFFFFFFFFu, keep, off);
+    return keep;
+}
+
+template <int N>
+struct CtaSums {
+    float part[N][32];  // per-warp partials
+    float tot[N];
+};
+
+// Sum of N floats across the CTA; every thread receives the totals.  Each warp reduces
+// its own values, warp 0 reduces the warps' partials the same way and publishes the
+// totals: two barriers, a fixed order of additions (the same totals in every thread and
+// on every run).  One CtaSums may be reused by consecutive calls.
+template <int N>
+__device__ __forceinline__ void cta_sum(float (&v)[N], CtaSums<N>& b) {
+    constexpr int L = kLanesPerSum<N>;
+    const int lane = threadIdx.x & 31;
+    const int wid = threadIdx.x >> 5;
+    const bool writer = (lane & (L - 1)) == 0 && lane / L < N;
+    const float s = warp_sums<N>(v);
+    if (writer) b.part[lane / L][wid] = s;
+    __syncthreads();
+    if (wid == 0) {
+        const bool in = lane < (int)(blockDim.x >> 5);
+        float p[N];
+#pragma unroll
+        for (int i = 0; i < N; ++i) p[i] = in ? b.part[i][lane] : 0.f;
+        const float t = warp_sums<N>(p);
+        if (writer) b.tot[lane / L] = t;
+    }
     __syncthreads();
 #pragma unroll
-    for (int i = 0; i < N; ++i) v[i] = warp_sum(lane < nw ? buf[i][lane] : 0.f);
+    for (int i = 0; i < N; ++i) v[i] = b.tot[i];
 }
 
 // This thread's x and g vectors of `row` (zeros past the row's end or past the last row).
@@ -93,199 +140,229 @@ __device__ __forceinline__ V16 load_w(const VjpArgs& a, int k) {
                                : ones_vec<T>();
 }
 
-// ---- RmsNormVjp, kernel 1 ---------------------------------------------------------------
-template <typename T, int VPT>
-__global__ void __launch_bounds__(kVjpThreads) rms_vjp_kernel(const VjpArgs a) {
-    pdl_wait();
-    pdl_release();
-    using E = Elem<T>;
-    constexpr int VEC = E::kVec;
-    constexpr bool kAhead = VPT == 1;  // next row in flight
-    __shared__ float red[2][2][32];
-    const int G = blockDim.x;
-    const int t = threadIdx.x;
-    const float invD = 1.f / (float)a.D;
-
-    V16 wv[VPT];
-    float acc[VPT][VEC];
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-        wv[k] = load_w<T>(a, k);
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[k][e] = 0.f;
-    }
-    V16 xv[VPT], gv[VPT];
-    if (kAhead) load_xg<T, VPT>(a, blockIdx.x, xv, gv);
-
-    int it = 0;
-    for (int64_t row = blockIdx.x; row < a.rows; row += a.parts, ++it) {
-        V16 xn[VPT], gn[VPT];
-        if (kAhead)
-            load_xg<T, VPT>(a, row + a.parts, xn, gn);
-        else
+// Rows of kernel 1: CTA p takes rows p, p + parts, ...  With VPT <= 2 two register sets
+// alternate, so row i + 1's loads are in flight while row i is reduced and written (and no
+// register copy waits on them); with VPT = 4 each row is loaded where it is used.
+template <int VPT, typename Row>
+__device__ __forceinline__ void walk_rows(const VjpArgs& a, Row&& row_step) {
+    using T = typename Row::T;
+    if constexpr (VPT <= 2) {
+        V16 xa[VPT], ga[VPT], xb[VPT], gb[VPT];
+        load_xg<T, VPT>(a, blockIdx.x, xa, ga);
+        const int64_t step = a.parts;
+        for (int64_t row = blockIdx.x; row < a.rows; row += 2 * step) {
+            load_xg<T, VPT>(a, row + step, xb, gb);
+            row_step(row, xa, ga);
+            if (row + step >= a.rows) break;
+            load_xg<T, VPT>(a, row + 2 * step, xa, ga);
+            row_step(row + step, xb, gb);
+        }
+    } else {
+        for (int64_t row = blockIdx.x; row < a.rows; row += a.parts) {
+            V16 xv[VPT], gv[VPT];
             load_xg<T, VPT>(a, row, xv, gv);
+            row_step(row, xv, gv);
+        }
+    }
+}
+
+// The element work runs on float32 pairs (packed FFMA2 / FADD2 / FMUL2, IEEE per lane):
+// each of a thread's row sums is two interleaved chains, added at the end.
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
+// ---- RmsNormVjp, kernel 1 ---------------------------------------------------------------
+template <typename TT, int VPT>
+struct RmsVjpRow {
+    using T = TT;
+    using E = Elem<T>;
+    static constexpr int VEC = E::kVec;
+    static constexpr int NP = VEC / 2;  // float pairs per vector
+    const VjpArgs& a;
+    const float2 (&wf)[VPT][NP];
+    float2 (&acc)[VPT][NP];
+    CtaSums<2>& red;
+    float invD;
+
+    __device__ __forceinline__ void operator()(int64_t row, const V16 (&xv)[VPT],
+                                               const V16 (&gv)[VPT]) const {
         // sum x^2 (the scale) and sum g w x (the projection)
-        float s[2] = {0.f, 0.f};
+        float2 s0 = splat2(0.f), s1 = splat2(0.f);
 #pragma unroll
         for (int k = 0; k < VPT; ++k)
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-                const float xf = E::get(xv[k], e);
-                s[0] = __fmaf_rn(xf, xf, s[0]);
-                s[1] = __fmaf_rn(__fmul_rn(E::get(gv[k], e), E::get(wv[k], e)), xf, s[1]);
+            for (int e = 0; e < VEC; e += 2) {
+                const float2 x2 = E::get2(xv[k], e);
+                const float2 u2 = mul2(E::get2(gv[k], e), wf[k][e / 2]);
+                s0 = fma2(x2, x2, s0);
+                s1 = fma2(u2, x2, s1);
             }
-        cta_sum<2>(s, red[it & 1]);
+        float s[2] = {__fadd_rn(s0.x, s0.y), __fadd_rn(s1.x, s1.y)};
+        cta_sum<2>(s, red);
         const float r = rsqrtf(__fmaf_rn(s[0], invD, a.eps));
         const float vr = __fmul_rn(__fmul_rn(r, r), __fmul_rn(s[1], invD));
+        const float2 r2 = splat2(r), nv2 = splat2(-vr);
         const size_t roff = (size_t)row * (size_t)a.nvec * 16;
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
-            const int v = t + k * G;
+            const int v = threadIdx.x + k * blockDim.x;
             if (v < a.nvec) {
                 V16 o;
 #pragma unroll
                 for (int e = 0; e < VEC; e += 2) {
-                    float d[2];
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const float xf = E::get(xv[k], e + q);
-                        const float gf = E::get(gv[k], e + q);
-                        const float u = __fmul_rn(gf, E::get(wv[k], e + q));
-                        d[q] = __fmul_rn(r, __fmaf_rn(-xf, vr, u));   // r (g w - x v)
-                        acc[k][e + q] = __fmaf_rn(__fmul_rn(gf, xf), r, acc[k][e + q]);
-                    }
-                    E::put2(o, e, d[0], d[1]);
+                    const float2 x2 = E::get2(xv[k], e);
+                    const float2 g2 = E::get2(gv[k], e);
+                    const float2 u2 = mul2(g2, wf[k][e / 2]);
+                    E::put2(o, e, mul2(r2, fma2(x2, nv2, u2)));        // r (g w - x v)
+                    acc[k][e / 2] = fma2(mul2(g2, x2), r2, acc[k][e / 2]);
                 }
                 st_stream(static_cast<char*>(a.dx) + roff + (size_t)v * 16, o);
             }
         }
-        if (kAhead)
-#pragma unroll
-            for (int k = 0; k < VPT; ++k) {
-                xv[k] = xn[k];
-                gv[k] = gn[k];
-            }
     }
+};
+
+template <typename T, int VPT>
+__device__ __forceinline__ void load_wf(const VjpArgs& a, float2 (&wf)[VPT][Elem<T>::kVec / 2]) {
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+        const V16 w = load_w<T>(a, k);
+#pragma unroll
+        for (int e = 0; e < Elem<T>::kVec; e += 2) wf[k][e / 2] = Elem<T>::get2(w, e);
+    }
+}
+
+template <typename T, int VPT>
+__global__ void __launch_bounds__(vjp_max_threads(VPT)) rms_vjp_kernel(const VjpArgs a) {
+    pdl_wait();
+    pdl_release();
+    constexpr int NP = Elem<T>::kVec / 2;
+    __shared__ CtaSums<2> red;
+    float2 wf[VPT][NP], acc[VPT][NP];
+    load_wf<T, VPT>(a, wf);
+#pragma unroll
+    for (int k = 0; k < VPT; ++k)
+#pragma unroll
+        for (int i = 0; i < NP; ++i) acc[k][i] = splat2(0.f);
+    walk_rows<VPT>(a, RmsVjpRow<T, VPT>{a, wf, acc, red, 1.f / (float)a.D});
     if (a.want_dw) {
         float* out = a.part + (size_t)blockIdx.x * a.D;
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
-            const int v = t + k * G;
+            const int v = threadIdx.x + k * blockDim.x;
             if (v < a.nvec)
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) out[v * VEC + e] = acc[k][e];
+                for (int i = 0; i < NP; ++i)
+                    reinterpret_cast<float2*>(out)[v * NP + i] = acc[k][i];
         }
     }
 }
 
 // ---- LayerNormVjp, kernel 1 ---------------------------------------------------------------
-template <typename T, int VPT>
-__global__ void __launch_bounds__(kVjpThreads) layer_vjp_kernel(const VjpArgs a) {
-    pdl_wait();
-    pdl_release();
+template <typename TT, int VPT>
+struct LayerVjpRow {
+    using T = TT;
     using E = Elem<T>;
-    constexpr int VEC = E::kVec;
-    constexpr bool kAhead = VPT == 1;  // next row in flight; w kept in registers
-    __shared__ float red[2][3][32];    // [pass][sum][warp]
-    const int G = blockDim.x;
-    const int t = threadIdx.x;
-    const float invD = 1.f / (float)a.D;
+    static constexpr int VEC = E::kVec;
+    static constexpr int NP = VEC / 2;
+    const VjpArgs& a;
+    V16 (&wv)[VPT];         // VPT <= 2: held for the whole walk; VPT = 4: reloaded per row
+    float2 (&accw)[VPT][NP];
+    float2 (&accb)[VPT][NP];
+    CtaSums<2>& red1;       // pass 1
+    CtaSums<3>& red2;       // pass 2
+    float invD;
 
-    V16 wv[VPT];
-    float accw[VPT][VEC], accb[VPT][VEC];
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-        if (kAhead) wv[k] = load_w<T>(a, k);
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) accw[k][e] = accb[k][e] = 0.f;
-    }
-    V16 xv[VPT], gv[VPT];
-    if (kAhead) load_xg<T, VPT>(a, blockIdx.x, xv, gv);
-
-    for (int64_t row = blockIdx.x; row < a.rows; row += a.parts) {
-        V16 xn[VPT], gn[VPT];
-        if (kAhead) {
-            load_xg<T, VPT>(a, row + a.parts, xn, gn);
-        } else {
-            load_xg<T, VPT>(a, row, xv, gv);
+    __device__ __forceinline__ void operator()(int64_t row, const V16 (&xv)[VPT],
+                                               const V16 (&gv)[VPT]) const {
+        if (VPT > 2)
 #pragma unroll
             for (int k = 0; k < VPT; ++k) wv[k] = load_w<T>(a, k);
-        }
         // pass 1: sum x and sum a (a = w g)
-        float p[2] = {0.f, 0.f};
+        float2 p0 = splat2(0.f), p1 = splat2(0.f);
 #pragma unroll
         for (int k = 0; k < VPT; ++k)
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-                p[0] = __fadd_rn(p[0], E::get(xv[k], e));
-                p[1] = __fadd_rn(p[1], __fmul_rn(E::get(wv[k], e), E::get(gv[k], e)));
+            for (int e = 0; e < VEC; e += 2) {
+                p0 = add2(p0, E::get2(xv[k], e));
+                p1 = add2(p1, mul2(E::get2(wv[k], e), E::get2(gv[k], e)));
             }
-        cta_sum<2>(p, red[0]);
+        float p[2] = {__fadd_rn(p0.x, p0.y), __fadd_rn(p1.x, p1.y)};
+        cta_sum<2>(p, red1);
         const float m1 = __fmul_rn(p[0], invD);
         const float ma = __fmul_rn(p[1], invD);
+        const float2 nm1 = splat2(-m1);
         // pass 2: sum c', sum c'^2 and sum a c' around m1 (c' = x - m1)
-        float q[3] = {0.f, 0.f, 0.f};
+        float2 q0 = splat2(0.f), q1 = splat2(0.f), q2 = splat2(0.f);
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
-            const int v = t + k * G;
+            const int v = threadIdx.x + k * blockDim.x;
             if (v < a.nvec)   // c' of a padding lane would be -m1
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    const float cp = __fsub_rn(E::get(xv[k], e), m1);
-                    const float af = __fmul_rn(E::get(wv[k], e), E::get(gv[k], e));
-                    q[0] = __fadd_rn(q[0], cp);
-                    q[1] = __fmaf_rn(cp, cp, q[1]);
-                    q[2] = __fmaf_rn(af, cp, q[2]);
+                for (int e = 0; e < VEC; e += 2) {
+                    const float2 cp = add2(E::get2(xv[k], e), nm1);
+                    const float2 a2 = mul2(E::get2(wv[k], e), E::get2(gv[k], e));
+                    q0 = add2(q0, cp);
+                    q1 = fma2(cp, cp, q1);
+                    q2 = fma2(a2, cp, q2);
                 }
         }
-        cta_sum<3>(q, red[1]);
+        float q[3] = {__fadd_rn(q0.x, q0.y), __fadd_rn(q1.x, q1.y), __fadd_rn(q2.x, q2.y)};
+        cta_sum<3>(q, red2);
         const float dm = __fmul_rn(q[0], invD);                             // mean = m1 + dm
         const float var = fmaxf(__fmaf_rn(q[1], invD, -__fmul_rn(dm, dm)), 0.f);
         const float r = rsqrtf(__fadd_rn(var, a.eps));
         // dx = r (a - mean(a) - c B) with B = r^2 sum(a c) / D
         const float B = __fmul_rn(__fmul_rn(r, r), __fmul_rn(__fmaf_rn(-dm, p[1], q[2]), invD));
+        const float2 r2 = splat2(r), ndm = splat2(-dm), nB = splat2(-B), nma = splat2(-ma);
         const size_t roff = (size_t)row * (size_t)a.nvec * 16;
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
-            const int v = t + k * G;
+            const int v = threadIdx.x + k * blockDim.x;
             if (v < a.nvec) {
                 V16 o;
 #pragma unroll
                 for (int e = 0; e < VEC; e += 2) {
-                    float d[2];
-#pragma unroll
-                    for (int q2 = 0; q2 < 2; ++q2) {
-                        const float xf = E::get(xv[k], e + q2);
-                        const float gf = E::get(gv[k], e + q2);
-                        const float af = __fmul_rn(E::get(wv[k], e + q2), gf);
-                        const float c = __fsub_rn(__fsub_rn(xf, m1), dm);
-                        d[q2] = __fmul_rn(r, __fmaf_rn(-c, B, __fsub_rn(af, ma)));
-                        accw[k][e + q2] = __fmaf_rn(gf, __fmul_rn(c, r), accw[k][e + q2]);
-                        accb[k][e + q2] = __fadd_rn(accb[k][e + q2], gf);
-                    }
-                    E::put2(o, e, d[0], d[1]);
+                    const float2 g2 = E::get2(gv[k], e);
+                    const float2 a2 = mul2(E::get2(wv[k], e), g2);
+                    const float2 c2 = add2(add2(E::get2(xv[k], e), nm1), ndm);
+                    E::put2(o, e, mul2(r2, fma2(c2, nB, add2(a2, nma))));
+                    accw[k][e / 2] = fma2(g2, mul2(c2, r2), accw[k][e / 2]);
+                    accb[k][e / 2] = add2(accb[k][e / 2], g2);
                 }
                 st_stream(static_cast<char*>(a.dx) + roff + (size_t)v * 16, o);
             }
         }
-        if (kAhead)
-#pragma unroll
-            for (int k = 0; k < VPT; ++k) {
-                xv[k] = xn[k];
-                gv[k] = gn[k];
-            }
     }
+};
+
+template <typename T, int VPT>
+__global__ void __launch_bounds__(vjp_max_threads(VPT)) layer_vjp_kernel(const VjpArgs a) {
+    pdl_wait();
+    pdl_release();
+    constexpr int NP = Elem<T>::kVec / 2;
+    __shared__ CtaSums<2> red1;
+    __shared__ CtaSums<3> red2;
+    V16 wv[VPT];
+    float2 accw[VPT][NP], accb[VPT][NP];
+    if (VPT <= 2)
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) wv[k] = load_w<T>(a, k);
+#pragma unroll
+    for (int k = 0; k < VPT; ++k)
+#pragma unroll
+        for (int i = 0; i < NP; ++i) accw[k][i] = accb[k][i] = splat2(0.f);
+    walk_rows<VPT>(a, LayerVjpRow<T, VPT>{a, wv, accw, accb, red1, red2, 1.f / (float)a.D});
     if (a.part) {
-        float* outw = a.part + (size_t)blockIdx.x * a.D;
-        float* outb = a.part + ((size_t)a.parts + blockIdx.x) * a.D;
+        float2* outw = reinterpret_cast<float2*>(a.part + (size_t)blockIdx.x * a.D);
+        float2* outb = reinterpret_cast<float2*>(a.part + ((size_t)a.parts + blockIdx.x) * a.D);
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
-            const int v = t + k * G;
+            const int v = threadIdx.x + k * blockDim.x;
             if (v < a.nvec)
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    if (a.want_dw) outw[v * VEC + e] = accw[k][e];
-                    if (a.want_db) outb[v * VEC + e] = accb[k][e];
+                for (int i = 0; i < NP; ++i) {
+                    if (a.want_dw) outw[v * NP + i] = accw[k][i];
+                    if (a.want_db) outb[v * NP + i] = accb[k][i];
                 }
         }
     }
