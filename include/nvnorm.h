@@ -219,7 +219,8 @@ NV_API nv_status nv_fault_count(uint32_t* count, int32_t reset);
  *                   per lane, which needs halves pairing and dims == D)
  *   threads_per_row threads that share one row (multiple of 32, <= 1024; 0 = auto)
  *   rows_per_cta    rows one CTA works on at a time (0 = auto)
- *   ctas_per_sm     0: one CTA per row group (register and generic paths) or one CTA
+ *   ctas_per_sm     0: one CTA per row group (rms_norm register path, generic paths),
+ *                   as many CTAs per SM as fit (layer_norm register path) or one CTA
  *                   per SM (staged path); > 0: a persistent grid of that many CTAs per
  *                   SM walking the rows
  *   launch          NV_LAUNCH_DEFAULT: programmatic dependent launch -- the kernel may

@@ -284,6 +284,24 @@ __global__ void __launch_bounds__(512) layer_staged_kernel(const RowArgs a, cons
 
     const double invD = 1.0 / (double)a.D;
     const double eps = (double)a.eps;
+    // largest |w| and 2^-11 |b| over this thread's columns (bounds of the error test)
+    float wmax = 0.f, bmax = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < VPT; ++kk) {
+        const int v = t + kk * G;
+        if (v < a.nvec) {
+            const V16 wv = a.w ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16)
+                               : ones_vec<T>();
+            const V16 bv = a.b ? ld_param(static_cast<const char*>(a.b) + (size_t)v * 16)
+                               : zeros_vec<T>();
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                wmax = fmaxf(wmax, fabsf(E::get(wv, e)));
+                bmax = fmaxf(bmax, fabsf(E::get(bv, e)));
+            }
+        }
+    }
+    bmax *= 0x1p-11f;
 
     int64_t k = 0;
     for (; k < nmine; ++k) {
@@ -358,6 +376,7 @@ __global__ void __launch_bounds__(512) layer_staged_kernel(const RowArgs a, cons
         const float2 nhi2 = make_float2(-mu_hi, -mu_hi);
         const float nlo = two_sub ? -mu_lo : 0.f;
         const float2 nlo2 = make_float2(nlo, nlo);
+        const float tmax = __fmaf_rn(__fmul_rn(kmu, rf), wmax, bmax);
 #pragma unroll
         for (int kk = 0; kk < VPT; ++kk) {
             const int v = t + kk * G;
@@ -368,7 +387,7 @@ __global__ void __launch_bounds__(512) layer_staged_kernel(const RowArgs a, cons
                 const V16 bv = a.b ? ld_param(static_cast<const char*>(a.b) + (size_t)v * 16)
                                    : zeros_vec<T>();
                 V16 o;
-                bool all_ok = true;
+                float ymin = INFINITY;
 #pragma unroll
                 for (int e = 0; e < VEC; e += 2) {
                     const float2 w2 = E::get2(wv, e);
@@ -376,12 +395,10 @@ __global__ void __launch_bounds__(512) layer_staged_kernel(const RowArgs a, cons
                     const float2 A2 = mul2(rf2, w2);
                     const float2 d2 = add2(add2(E::get2(xv, e), nhi2), nlo2);
                     const float2 y2 = fma2(d2, A2, b2);
-                    // bitwise: no short-circuit branches in the unrolled loop
-                    all_ok &= (fabsf(y2.x) > __fmaf_rn(kmu, fabsf(A2.x), 0x1p-11f * fabsf(b2.x))) &
-                              (fabsf(y2.y) > __fmaf_rn(kmu, fabsf(A2.y), 0x1p-11f * fabsf(b2.y)));
+                    ymin = fminf(ymin, fminf(fabsf(y2.x), fabsf(y2.y)));
                     E::put2(o, e, y2);
                 }
-                if (!all_ok) o = layer_vector_f64<T>(xv, wv, bv, mean, rstd);
+                if (!(ymin > tmax)) o = layer_vector_f64<T>(xv, wv, bv, mean, rstd);
                 st_stream(static_cast<char*>(a.y) + roff + (size_t)v * 16, o);
             }
         }

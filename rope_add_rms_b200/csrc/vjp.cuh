@@ -369,34 +369,44 @@ __global__ void __launch_bounds__(vjp_max_threads(VPT)) layer_vjp_kernel(const V
 }
 
 // ---- kernel 2: column sums of the partials --------------------------------------------------
-// out[j] = sum_{p < parts} part[p][j] in double.  A CTA owns 32 columns; warp w adds parts
-// w, w + 8, w + 16, ... in that order, then lane j of warp 0 adds the 8 warp sums in warp
-// order: a fixed order, so the result does not depend on timing.
-constexpr int kReduceWarps = 8;
+// out[y][j] = sum_{p < parts} part[first + y][p][j] in double, y = blockIdx.y.
+// A CTA owns 32 columns; warp w adds parts w, w + 32, w + 64, ... in that order (eight
+// loads in flight per lane), then the 32 warp sums are added pairwise in a fixed tree:
+// a fixed order, so the result does not depend on timing.
+constexpr int kReduceWarps = 32;
+
+struct ReduceArgs {
+    const float* part;  // [nsum][parts][D]
+    void* out[2];       // [D] for sums first, first + 1
+    int first;          // slice of the first sum reduced (0: dw, 1: db)
+    int parts;
+    int D;
+};
 
 template <typename T>
-__global__ void __launch_bounds__(kReduceWarps * 32) vjp_reduce_kernel(const float* part,
-                                                                       int parts, int D,
-                                                                       void* out) {
+__global__ void __launch_bounds__(kReduceWarps * 32) vjp_reduce_kernel(const ReduceArgs a) {
     pdl_wait();
     pdl_release();
     __shared__ double sw[kReduceWarps][32];
     const int lane = threadIdx.x & 31;
     const int w = threadIdx.x >> 5;
     const int j = blockIdx.x * 32 + lane;
+    const float* part =
+        a.part ? a.part + (size_t)(a.first + blockIdx.y) * a.parts * a.D : nullptr;
     double s = 0.0;
-    if (j < D) {
-#pragma unroll 4
-        for (int p = w; p < parts; p += kReduceWarps) s += (double)part[(size_t)p * D + j];
+    if (j < a.D && part) {
+#pragma unroll 8
+        for (int p = w; p < a.parts; p += kReduceWarps) s += (double)part[(size_t)p * a.D + j];
     }
     sw[w][lane] = s;
     __syncthreads();
-    if (w == 0 && j < D) {
-        double tot = 0.0;
 #pragma unroll
-        for (int i = 0; i < kReduceWarps; ++i) tot += sw[i][lane];
-        Elem<T>::store1(out, j, __double2float_rn(tot));
+    for (int stride = kReduceWarps / 2; stride >= 1; stride >>= 1) {
+        if (w < stride) sw[w][lane] += sw[w + stride][lane];
+        __syncthreads();
     }
+    if (w == 0 && j < a.D)
+        Elem<T>::store1(blockIdx.y ? a.out[1] : a.out[0], j, __double2float_rn(sw[0][lane]));
 }
 
 }  // namespace nvn
