@@ -65,7 +65,7 @@ typedef enum {
 
 /*
  * rms_norm -- docs.rs nuvec-core 0.5.0, Enum FastOp, variant RmsNorm:
- *   y = x / sqrt(mean(x^2) + eps) * w over the last axis; w is 1-D or the scalar 1
+ *   y = x / sqrt(mean(x^2) + eps) * w over the last axis; w is a length-D vector, or NULL for 1
  *   (nuvec-nn src/layers.rs, RmsNorm::forward; miniVLLM Layers page, LayerNorm with
  *   residual = None).
  * x [rows, D] in; w [D] in, or NULL for w = 1; y [rows, D] out (may be x).
@@ -88,8 +88,8 @@ NV_API nv_status nv_add_rms_norm(const void* x, const void* r, const void* w, vo
 
 /*
  * layer_norm -- docs.rs nuvec-core 0.5.0, Enum FastOp, variant LayerNorm:
- *   y = (x - mean) / sqrt(var + eps) * w + b over the last axis, w and b 1-D or the
- *   scalars 1 and 0 (nuvec-nn src/layers.rs, LayerNorm: affine / without_bias).
+ *   y = (x - mean) / sqrt(var + eps) * w + b over the last axis, w and b length-D
+ *   vectors or NULL for 1 and 0 (nuvec-nn src/layers.rs, LayerNorm: affine / without_bias).
  * var is the population variance (sum of squared deviations / D).
  * x [rows, D] in; w [D] or NULL (w = 1); b [D] or NULL (b = 0); y [rows, D] out.
  */
@@ -98,7 +98,7 @@ NV_API nv_status nv_layer_norm(const void* x, const void* w, const void* b, void
 
 /*
  * norm_rope -- docs.rs nuvec-core 0.5.0, Enum FastOp, variants NormRope and Rope
- * (non-cache form): each [b, h, l] row of x [B, H, L, D] is RMS-normalised with eps
+ * (non-cache form): every row (b, h, l) of x [B, H, L, D] is RMS-normalised with eps
  * and w, then its first dims features are rotated at position offset + l:
  *   theta_i = base^(-2 i / dims), phi_i = (offset + l) * scale * theta_i,
  *   (y_p, y_q) = (n_p cos phi_i - n_q sin phi_i, n_p sin phi_i + n_q cos phi_i)
@@ -116,10 +116,10 @@ NV_API nv_status nv_norm_rope(const void* x, const void* w, void* y, int64_t row
 
 /*
  * rope -- the general form of norm_rope: docs.rs nuvec-core 0.5.0, Enum FastOp, variant
- * NormRope with its cache form ("written into cache at the same positions") and
+ * NormRope with its cache form (rotated rows land in the cache at their own positions) and
  * variant Rope with an explicit frequency vector and a direction.
  *   freqs    [dims/2] float32 device array of frequencies theta_i replacing
- *            base^(-2 i / dims) ("base ... unused with freqs"), or NULL.
+ *            base^(-2 i / dims) (base is then ignored), or NULL.
  *   forward  != 0: turn by +phi_i; 0: the inverse rotation (-phi_i), the gradient of Rope.
  *   y_len    0: y is [B, H, L, D] like x (may be x).  > 0: y is a cache [B, H, y_len, D]
  *            and row (b, h, l) of x is written to cache row (b, h, offset + l), at the

@@ -15,8 +15,8 @@
  *   AddRmsNorm  (x, r, w): h = x + r, then RmsNorm of h; the updated residual h is
  *               returned next to the normalised row (miniVLLM LayerNorm.forward,
  *               steps 1-3: x_new = x + residual, normalise x_new, return both).
- *   LayerNorm   (x, w, b): (x - mean) / sqrt(var + eps) * w + b over the last axis,
- *               w and b are 1-D or the scalars 1 and 0.
+ *   LayerNorm   (x, w, b): (x - mean) / sqrt(var + eps) * w + b over the last axis;
+ *               w and b are length-D vectors, or absent (1 and 0).
  *   Rope        rotary embedding of the first dims features (dims even), as the two
  *               halves or as interleaved pairs ("traditional"); base and a position
  *               scale; forward = false is the inverse rotation.
@@ -289,7 +289,7 @@ int oracle_rope_ex(const void* x, const void* w, const double* freqs, double* y,
 }
 
 /*
- * RmsNormVjp (x, w, g): the gradients of RmsNorm for x and w (docs.rs nuvec-core 0.5.0,
+ * RmsNormVjp (x, w, g): gradients of rms_norm with respect to x and w (docs.rs nuvec-core 0.5.0,
  * Enum FastOp, variant RmsNormVjp).  With r = 1 / sqrt(mean(x^2) + eps) and
  * y_j = x_j r w_j:
  *   dx_j = r w_j g_j - x_j r^3 (sum_k g_k w_k x_k) / D
@@ -325,7 +325,7 @@ int oracle_rms_norm_vjp(const void* x, const void* w, const void* g, double* dx,
 }
 
 /*
- * LayerNormVjp (x, w, b, g): the gradients of LayerNorm for x, w and b (docs.rs
+ * LayerNormVjp (x, w, b, g): gradients of layer_norm with respect to x, w and b (docs.rs
  * nuvec-core 0.5.0, Enum FastOp, variant LayerNormVjp).  With mean, var (population),
  * r = 1 / sqrt(var + eps), xh_j = (x_j - mean) r, a_j = w_j g_j:
  *   dx_j = r (a_j - mean_k(a_k) - xh_j mean_k(a_k xh_k))

@@ -1,8 +1,8 @@
 // layer.cuh -- layer_norm kernels.
 //
 // Definition: docs.rs nuvec-core 0.5.0, Enum FastOp, variant LayerNorm:
-// y = (x - mean) / sqrt(var + eps) * w + b over the last axis, w and b 1-D or the
-// scalars 1 and 0; var is the population variance.
+// y = (x - mean) / sqrt(var + eps) * w + b for every row (last axis), with the
+// population variance; w and b are length-D vectors, or absent and standing for 1 and 0.
 //
 // Precision: the output y = a + b with a = (x - mean) * rstd * w can cancel (a close
 // to -b).  A float32 error in mean or rstd is an absolute error of about 2^-24 |a| in
