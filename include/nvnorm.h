@@ -167,6 +167,27 @@ NV_API nv_status nv_layer_norm_vjp(const void* x, const void* w, const void* g, 
 NV_API size_t nv_norm_vjp_workspace_size(int32_t op, int64_t rows, int64_t D);
 
 /*
+ * add_rms_norm_host -- add_rms_norm (as nv_add_rms_norm) on rows that live in host
+ * memory: x and r are copied in, the op runs, y and h are copied back, pipelined over
+ * chunks of chunk_rows rows (0 = about eight chunks) on internal streams so that copies in
+ * and out and the compute of different chunks overlap.
+ * x_host, r_host [rows, D] in, y_host, h_host [rows, D] out: page-locked host memory
+ * (cudaHostAlloc / cudaHostRegister); y_host may be x_host and h_host may be r_host, other
+ * host buffers may not overlap.  x_dev, r_dev, y_dev, h_dev [rows, D]: device buffers of
+ * the current device owned by the caller, used as the staging area (on return their
+ * contents are the inputs and outputs of the op; y_dev may be x_dev, h_dev may be r_dev).
+ * w [D] device or NULL.  Asynchronous with respect to the host like the other calls: the
+ * work starts after what is already queued on `stream`, and `stream` waits for all of it.
+ * Calls from several host threads are serialised while they enqueue.  Errors as
+ * nv_add_rms_norm, plus NV_ERR_INVALID_ARG for host buffers that are not page-locked.
+ */
+NV_API nv_status nv_add_rms_norm_host(const void* x_host, const void* r_host, const void* w,
+                                      void* y_host, void* h_host, void* x_dev, void* r_dev,
+                                      void* y_dev, void* h_dev, int64_t rows, int64_t D,
+                                      float eps, nv_dtype dt, int64_t chunk_rows,
+                                      nv_stream_t stream);
+
+/*
  * rms_norm_vjp_static -- nv_rms_norm_vjp for callers that cannot allocate device memory.
  * The op definitions this library follows have no counterpart of this entry point: it
  * exists for callers that are handed their input and output buffers and may not allocate

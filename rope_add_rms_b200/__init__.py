@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "NvError", "Plan", "library", "library_path",
-    "nv_rms_norm", "nv_add_rms_norm", "nv_layer_norm", "nv_norm_rope", "nv_describe_plan",
+    "nv_rms_norm", "nv_add_rms_norm", "nv_add_rms_norm_host", "nv_layer_norm", "nv_norm_rope",
+    "nv_describe_plan",
     "nv_fault_count",
     "nv_rope", "rms_norm", "add_rms_norm", "layer_norm", "norm_rope", "norm_rope_into_cache",
     "rope", "nv_rms_norm_vjp", "nv_layer_norm_vjp", "nv_norm_vjp_workspace_size", "rms_norm_vjp",
@@ -73,6 +74,8 @@ def library() -> ctypes.CDLL:
     sigs = {
         "nv_rms_norm": [vp, vp, vp, i64, i64, f32, i32, vp],
         "nv_add_rms_norm": [vp, vp, vp, vp, vp, i64, i64, f32, i32, vp],
+        "nv_add_rms_norm_host": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, f32, i32, i64,
+                                 vp],
         "nv_layer_norm": [vp, vp, vp, vp, i64, i64, f32, i32, vp],
         "nv_norm_rope": [vp, vp, vp, i64, i64, i64, i32, i32, f32, f32, i64, i32, f32, i32, vp],
         "nv_rms_norm_ex": [vp, vp, vp, i64, i64, f32, i32, vp, pp],
@@ -170,6 +173,24 @@ def nv_add_rms_norm(x, r, w, y, h, eps, stream=None, plan=None):
             _stream(stream))
     st = lib.nv_add_rms_norm(*args) if plan is None else lib.nv_add_rms_norm_ex(*args, _plan(plan))
     _check("nv_add_rms_norm", st)
+
+
+def nv_add_rms_norm_host(x_host, r_host, w, y_host, h_host, x_dev, r_dev, y_dev, h_dev, eps,
+                         chunk_rows=0, stream=None):
+    """add_rms_norm on rows in page-locked host tensors (``pin_memory()``), staged through
+    the caller's device tensors; copies in, compute and copies out pipelined over row
+    chunks.  Asynchronous like the other calls (synchronise ``stream`` to read y_host)."""
+    rows, D = _rows_D(x_host)
+    for t in (x_host, r_host, y_host, h_host):
+        if t.is_cuda:
+            raise ValueError("x_host, r_host, y_host and h_host must be host tensors")
+    lib = library()
+    st = lib.nv_add_rms_norm_host(_ptr(x_host), _ptr(r_host), _ptr(w), _ptr(y_host),
+                                  _ptr(h_host), _ptr(x_dev), _ptr(r_dev), _ptr(y_dev),
+                                  _ptr(h_dev), rows, D, eps,
+                                  _dtype(x_host, r_host, w, y_host, h_host, x_dev, r_dev,
+                                         y_dev, h_dev), chunk_rows, _stream(stream))
+    _check("nv_add_rms_norm_host", st)
 
 
 def nv_layer_norm(x, w, b, y, eps, stream=None, plan=None):

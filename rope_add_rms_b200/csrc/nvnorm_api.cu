@@ -406,6 +406,9 @@ nv_status run_layer(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs
     return fail(NV_ERR_UNSUPPORTED, "vec_per_thread %d", p.vec_per_thread);
 }
 
+nv_status row_dispatch(Op op, const nv_plan& p, const DevInfo& di, nv_dtype dt, cudaStream_t cs,
+                       const RowArgs& a);
+
 nv_status row_op(Op op, const void* x, const void* r, const void* w, const void* b, void* y,
                  void* h, int64_t rows, int64_t D, float eps, nv_dtype dt, nv_stream_t stream,
                  const nv_plan* req) {
@@ -455,7 +458,11 @@ nv_status row_op(Op op, const void* x, const void* r, const void* w, const void*
     a.D = (int)D;
     a.nvec = (int)(D * (int64_t)s / 16);
     a.eps = eps;
-    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    return row_dispatch(op, p, di, dt, reinterpret_cast<cudaStream_t>(stream), a);
+}
+
+nv_status row_dispatch(Op op, const nv_plan& p, const DevInfo& di, nv_dtype dt, cudaStream_t cs,
+                       const RowArgs& a) {
     const bool bf = dt == NV_BF16;
     switch (op) {
         case OP_RMS:
@@ -634,6 +641,164 @@ nv_status rope_op(const void* x, const void* w, const float* freqs, void* y, int
     }
     return bf ? launch_rope_generic<__nv_bfloat16>(di, p.ctas_per_sm, cs, a)
               : launch_rope_generic<float>(di, p.ctas_per_sm, cs, a);
+}
+
+// ---- host-resident rows: copies and compute pipelined over row chunks ---------------------
+// Chunk k goes to internal stream k % kPipeStreams: host -> device copies of its x and r
+// rows, the add_rms_norm launch on those rows, device -> host copies of its y and h.  The
+// copy engines move chunk k + 1 in while chunk k - 1 moves out, so the PCIe link runs in
+// both directions at once.  The internal streams start after the work already queued on
+// the caller's stream and the caller's stream waits for all of them, so the call is
+// ordered like any other launch on `stream`.
+constexpr int kPipeStreams = 3;
+
+struct Pipe {
+    cudaStream_t s[kPipeStreams] = {};
+    cudaEvent_t start = nullptr;
+    cudaEvent_t done[kPipeStreams] = {};
+};
+Pipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mu;  // guards creation and the enqueue sequence (events are reused)
+
+nv_status pipe_for(int dev, Pipe** out) {
+    Pipe& pp = g_pipe[dev];
+    if (!pp.start) {
+        cudaError_t e = cudaEventCreateWithFlags(&pp.start, cudaEventDisableTiming);
+        for (int i = 0; e == cudaSuccess && i < kPipeStreams; ++i) {
+            e = cudaStreamCreateWithFlags(&pp.s[i], cudaStreamNonBlocking);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&pp.done[i], cudaEventDisableTiming);
+        }
+        if (e != cudaSuccess) {
+            pp = Pipe{};  // a later call retries; objects made so far are left to the context
+            return cuda_fail(e, "creating the pipeline streams");
+        }
+    }
+    *out = &pp;
+    return NV_OK;
+}
+
+// Page-locked host memory (cudaHostAlloc or cudaHostRegister) holding `bytes` bytes.
+nv_status check_host(const void* p, size_t bytes, const char* name) {
+    cudaPointerAttributes at;
+    cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess || at.type != cudaMemoryTypeHost) {
+        cudaGetLastError();
+        return fail(NV_ERR_INVALID_ARG, "%s (%p) is not page-locked host memory", name, p);
+    }
+    RangeFn fn = range_fn();
+    if (fn && at.devicePointer) {
+        CUdeviceptr base = 0;
+        size_t size = 0;
+        if (fn(&base, &size, (CUdeviceptr)(uintptr_t)at.devicePointer) == CUDA_SUCCESS &&
+            (uintptr_t)at.devicePointer + bytes > (uintptr_t)base + size)
+            return fail(NV_ERR_INVALID_ARG, "%s (%p): %zu bytes run past the end of its "
+                        "page-locked allocation", name, p, bytes);
+    }
+    return NV_OK;
+}
+
+nv_status add_rms_norm_host(const void* x_host, const void* r_host, const void* w,
+                            void* y_host, void* h_host, void* x_dev, void* r_dev, void* y_dev,
+                            void* h_dev, int64_t rows, int64_t D, float eps, nv_dtype dt,
+                            int64_t chunk_rows, nv_stream_t stream) {
+    nv_status st = check_common(rows, D, eps, dt);
+    if (st != NV_OK) return st;
+    if (chunk_rows < 0) return fail(NV_ERR_INVALID_ARG, "chunk_rows = %lld < 0", (long long)chunk_rows);
+    if (rows == 0) return NV_OK;
+    const void* ptrs[] = {x_host, r_host, y_host, h_host, x_dev, r_dev, y_dev, h_dev};
+    const char* names[] = {"x_host", "r_host", "y_host", "h_host", "x_dev", "r_dev", "y_dev", "h_dev"};
+    for (int i = 0; i < 8; ++i)
+        if (!ptrs[i]) return fail(NV_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (y_dev == h_dev || y_host == h_host)
+        return fail(NV_ERR_INVALID_ARG, "y and h are the same buffer");
+    const size_t s = elem_size(dt);
+    const size_t nbytes = (size_t)rows * (size_t)D * s;
+    for (int i = 0; i < 4; ++i) {
+        st = check_host(ptrs[i], nbytes, names[i]);
+        if (st != NV_OK) return st;
+    }
+    // host outputs: each may be exactly its own row input (chunk k is read before it is
+    // written, and no other chunk touches its rows), otherwise disjoint from the rest
+    const struct { const void* p; bool out; const void* may_equal; } hb[] = {
+        {x_host, false, nullptr}, {r_host, false, nullptr},
+        {y_host, true, x_host}, {h_host, true, r_host}};
+    for (int i = 0; i < 4; ++i) {
+        if (!hb[i].out) continue;
+        const uintptr_t a0 = (uintptr_t)hb[i].p, a1 = a0 + nbytes;
+        for (int j = 0; j < 4; ++j) {
+            if (j == i || hb[j].p == hb[i].may_equal) continue;
+            const uintptr_t b0 = (uintptr_t)hb[j].p, b1 = b0 + nbytes;
+            if (a0 < b1 && b0 < a1)
+                return fail(NV_ERR_INVALID_ARG, "host output %s overlaps %s", names[i],
+                            names[j]);
+        }
+    }
+
+    int dev = 0;
+    DevInfo di;
+    st = current_device(&dev, &di);
+    if (st != NV_OK) return st;
+    const Buf bufs[] = {
+        {x_dev, nbytes, "x_dev", false, true},  {r_dev, nbytes, "r_dev", false, true},
+        {w, (size_t)D * s, "w", false, false},  {y_dev, nbytes, "y_dev", true, false},
+        {h_dev, nbytes, "h_dev", true, false},
+    };
+    st = check_buffers(bufs, 5, dev);
+    if (st != NV_OK) return st;
+    const int64_t chunk =
+        chunk_rows > 0 ? chunk_rows : std::max<int64_t>(1, (rows + 7) / 8);  // ~8 chunks
+    const int64_t row_bytes = D * (int64_t)s;
+    bool al = aligned16(x_dev) && aligned16(r_dev) && aligned16(y_dev) && aligned16(h_dev) &&
+              (!w || aligned16(w)) && (chunk * row_bytes) % 16 == 0;
+    nv_plan p;
+    st = make_plan(OP_ADD, std::min(rows, chunk), D, dt, al, nullptr, &p, &di);
+    if (st != NV_OK) return st;
+    g_pdl = true;
+
+    std::lock_guard<std::mutex> lk(g_pipe_mu);
+    Pipe* pp = nullptr;
+    st = pipe_for(dev, &pp);
+    if (st != NV_OK) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaEventRecord(pp->start, cs);
+    for (int i = 0; e == cudaSuccess && i < kPipeStreams; ++i)
+        e = cudaStreamWaitEvent(pp->s[i], pp->start, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "pipeline start");
+    const int64_t nchunks = (rows + chunk - 1) / chunk;
+    for (int64_t k = 0; k < nchunks; ++k) {
+        cudaStream_t sk = pp->s[k % kPipeStreams];
+        const int64_t r0 = k * chunk, n = std::min(chunk, rows - r0);
+        const size_t off = (size_t)r0 * (size_t)row_bytes, len = (size_t)n * (size_t)row_bytes;
+        auto at = [off](const void* base) {
+            return static_cast<char*>(const_cast<void*>(base)) + off;
+        };
+        e = cudaMemcpyAsync(at(x_dev), at(x_host), len, cudaMemcpyHostToDevice, sk);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(at(r_dev), at(r_host), len, cudaMemcpyHostToDevice, sk);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (host to device)");
+        RowArgs a{};
+        a.x = at(x_dev);
+        a.r = at(r_dev);
+        a.w = w;
+        a.y = at(y_dev);
+        a.h = at(h_dev);
+        a.rows = n;
+        a.D = (int)D;
+        a.nvec = (int)(row_bytes / 16);
+        a.eps = eps;
+        st = row_dispatch(OP_ADD, p, di, dt, sk, a);
+        if (st != NV_OK) return st;
+        e = cudaMemcpyAsync(at(y_host), at(y_dev), len, cudaMemcpyDeviceToHost, sk);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(at(h_host), at(h_dev), len, cudaMemcpyDeviceToHost, sk);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (device to host)");
+    }
+    for (int i = 0; e == cudaSuccess && i < kPipeStreams; ++i) {
+        e = cudaEventRecord(pp->done[i], pp->s[i]);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, pp->done[i], 0);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "pipeline end");
+    return NV_OK;
 }
 
 // ---- backward (vjp) -------------------------------------------------------------------------
@@ -930,6 +1095,14 @@ nv_status nv_describe_plan(int32_t op, int64_t rows, int64_t D, nv_dtype dt, nv_
         return rope_plan(rows, 1, D, (int)(D - D % 2), false, dt, true, 148, nullptr, plan, &rp);
     }
     return make_plan((Op)op, rows, D, dt, true, nullptr, plan);
+}
+
+nv_status nv_add_rms_norm_host(const void* x_host, const void* r_host, const void* w,
+                               void* y_host, void* h_host, void* x_dev, void* r_dev, void* y_dev,
+                               void* h_dev, int64_t rows, int64_t D, float eps, nv_dtype dt,
+                               int64_t chunk_rows, nv_stream_t stream) {
+    return add_rms_norm_host(x_host, r_host, w, y_host, h_host, x_dev, r_dev, y_dev, h_dev, rows,
+                             D, eps, dt, chunk_rows, stream);
 }
 
 nv_status nv_rms_norm_vjp_static(const void* x, const void* w, const void* g, void* dx, void* dw,

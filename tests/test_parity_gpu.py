@@ -406,6 +406,55 @@ def test_norm_rope_in_place():
     check_out(x, ref)
 
 
+# ---- host-resident rows --------------------------------------------------------------------
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,D,chunk", [(3000, 4096, 0), (1000, 1024, 333), (7, 512, 1),
+                                          (513, 2048, 1000), (64, 100, 10)])
+def test_add_rms_norm_host(rows, D, chunk, dt):
+    """Copies in, compute and copies out pipelined over row chunks: bit-identical to the
+    device call, and the device staging buffers end up holding inputs and outputs."""
+    inp = synth.add_rms_inputs(rows, D, dt, seed=rows + chunk)
+    xh, rh = inp["x"].pin_memory(), inp["r"].pin_memory()
+    w = dev(inp["w"])
+    yh, hh = torch.empty_like(xh).pin_memory(), torch.empty_like(xh).pin_memory()
+    xd, rd, yd, hd = (torch.empty(rows, D, dtype=xh.dtype, device="cuda") for _ in range(4))
+    nv.nv_add_rms_norm_host(xh, rh, w, yh, hh, xd, rd, yd, hd, 1e-5, chunk_rows=chunk)
+    torch.cuda.synchronize()
+    y_ref, h_ref = torch.empty_like(xd), torch.empty_like(xd)
+    nv.nv_add_rms_norm(dev(inp["x"]), dev(inp["r"]), w, y_ref, h_ref, 1e-5)
+    torch.cuda.synchronize()
+    bits = torch.int16 if dt == "bf16" else torch.int32
+    assert torch.equal(yh.view(bits), y_ref.cpu().view(bits))
+    assert torch.equal(hh.view(bits), h_ref.cpu().view(bits))
+    assert torch.equal(yd.view(bits), y_ref.view(bits))
+    ref, href = oracle.add_rms_norm(host(inp["x"]), host(inp["r"]), host(inp["w"]), 1e-5)
+    check_exact(hh, href, "h")
+    check_out(yh, ref, "y")
+
+
+def test_add_rms_norm_host_in_place_and_errors():
+    rows, D = 2048, 4096
+    inp = synth.add_rms_inputs(rows, D, "bf16", seed=5)
+    xh, rh = inp["x"].clone().pin_memory(), inp["r"].clone().pin_memory()
+    w = dev(inp["w"])
+    xd, rd = (torch.empty(rows, D, dtype=xh.dtype, device="cuda") for _ in range(2))
+    nv.nv_add_rms_norm_host(xh, rh, w, xh, rh, xd, rd, xd, rd, 1e-5)   # y over x, h over r
+    torch.cuda.synchronize()
+    ref, href = oracle.add_rms_norm(host(inp["x"]), host(inp["r"]), host(inp["w"]), 1e-5)
+    check_exact(rh, href, "h in place")
+    check_out(xh, ref, "y in place")
+    pageable = inp["x"].clone()
+    with pytest.raises(nv.NvError, match="page-locked"):
+        nv.nv_add_rms_norm_host(pageable, rh, w, xh, rh, xd, rd, xd, rd, 1e-5)
+    other = torch.empty_like(xh).pin_memory()
+    with pytest.raises(nv.NvError, match="overlaps"):
+        nv.nv_add_rms_norm_host(xh, rh, w, other, xh, xd, rd, xd, rd, 1e-5)   # h over x
+    with pytest.raises(nv.NvError, match="past the end"):
+        small = torch.empty(100, D, dtype=xh.dtype, device="cuda")
+        nv.nv_add_rms_norm_host(xh, rh, w, xh, rh, small, rd, small, rd, 1e-5)
+
+
 # ---- programmatic dependent launch ---------------------------------------------------------
 
 @pytest.mark.parametrize("launch", [nv.LAUNCH_DEFAULT, nv.LAUNCH_PLAIN])
