@@ -99,6 +99,8 @@ class Oracle:
         lib.oracle_round_bf16.restype = None
         lib.oracle_rms_norm.argtypes = [vp, vp, vp, i64, i64, i64, f32, i32]
         lib.oracle_add_rms_norm.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, f32, i32]
+        lib.oracle_allreduce_add_rms_norm.argtypes = [vp, i32, vp, vp, vp, vp, vp, i64, i64, i64,
+                                                      f32, i32]
         lib.oracle_layer_norm.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, i32]
         lib.oracle_rope_f64.argtypes = [vp, vp, i64, i64, i64, i64, i64, i32, f32, f32, i64, i32]
         lib.oracle_norm_rope.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, f32,
@@ -156,6 +158,28 @@ class Oracle:
                                                             _ptr(h), a, b, D, eps, dt),
                   rows, threads)
         return y, h
+
+    def allreduce_add_rms_norm(self, parts, r, w, eps, threads=None):
+        """(y, h, x): x = the sum of the partial tensors (in order, in double) rounded once
+        to the I/O type, then add_rms_norm(x, r)."""
+        ps = [_io(p, "part") for p in parts]
+        if not ps:
+            raise ValueError("at least one partial tensor")
+        dt = ps[0][1]
+        ps = [p for p, _ in ps]
+        r = _io(r, "r")[0]
+        rows, D = r.shape
+        if any(p.shape != (rows, D) or p.dtype != r.dtype for p in ps):
+            raise ValueError("partial tensors must match r in shape and dtype")
+        w = None if w is None else _io(w, "w")[0]
+        y = np.empty((rows, D), np.float64)
+        h = np.empty((rows, D), r.dtype)
+        x = np.empty((rows, D), r.dtype)
+        table = (ctypes.c_void_p * len(ps))(*[p.ctypes.data for p in ps])
+        self._run(lambda a, b: self.lib.oracle_allreduce_add_rms_norm(
+            ctypes.cast(table, ctypes.c_void_p), len(ps), _ptr(r), _ptr(w), _ptr(y), _ptr(x),
+            _ptr(h), a, b, D, eps, dt), rows, threads)
+        return y, h, x
 
     def layer_norm(self, x, w, b, eps, threads=None):
         """y = (x - mean) / sqrt(var + eps) * w + b per row; w None means 1, b None 0."""
@@ -280,6 +304,10 @@ def rms_norm(x, w, eps, threads=None):
 
 def add_rms_norm(x, r, w, eps, threads=None):
     return get().add_rms_norm(x, r, w, eps, threads)
+
+
+def allreduce_add_rms_norm(parts, r, w, eps, threads=None):
+    return get().allreduce_add_rms_norm(parts, r, w, eps, threads)
 
 
 def layer_norm(x, w, b, eps, threads=None):

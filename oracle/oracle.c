@@ -200,6 +200,49 @@ int oracle_add_rms_norm(const void* x, const void* r, const void* w, double* y, 
     return 0;
 }
 
+/*
+ * AllReduce + AddRmsNorm: the step a tensor-parallel decoder takes after a row-parallel
+ * linear layer (miniVLLM Layers page, section Linear layers, RowParallelLinear: the
+ * forward pass sums the ranks' partial outputs with an all_reduce), followed by the fused
+ * residual add + RMSNorm (same page, section LayerNorm, forward with a residual; docs.rs
+ * nuvec-core 0.5.0, Enum FastOp, variant AddRmsNorm).
+ *   x = the sum over the nparts partial tensors, taken in part order in double and rounded
+ *       once to the I/O type (written to x_out when it is not NULL);
+ *   then add_rms_norm(x, r): h = x + r rounded to the I/O type, y = RmsNorm(h) * w.
+ * parts: nparts pointers to [rows, D] arrays of the I/O type.
+ */
+int oracle_allreduce_add_rms_norm(const void* const* parts, int nparts, const void* r,
+                                  const void* w, double* y, void* x_out, void* h, int64_t r0,
+                                  int64_t r1, int64_t D, float eps, int dt) {
+    if (nparts < 1) return -1;
+    void* xb = malloc((size_t)(r1 - r0) * (size_t)D * (dt == ORACLE_BF16 ? 2 : 4));
+    if (!xb) return -1;
+    for (int64_t k = r0; k < r1; ++k)
+        for (int64_t j = 0; j < D; ++j) {
+            const int64_t i = k * D + j;
+            double s = 0.0;
+            for (int p = 0; p < nparts; ++p) s += widen(parts[p], dt, i);
+            const int64_t o = (k - r0) * D + j;
+            if (dt == ORACLE_BF16)
+                ((uint16_t*)xb)[o] = oracle_bf16_from_f64(s);
+            else
+                ((float*)xb)[o] = (float)s;
+            if (x_out) {
+                if (dt == ORACLE_BF16)
+                    ((uint16_t*)x_out)[i] = ((uint16_t*)xb)[o];
+                else
+                    ((float*)x_out)[i] = ((float*)xb)[o];
+            }
+        }
+    /* add_rms_norm on the rounded x, rows r0..r1 (xb holds only those rows) */
+    const size_t off = (size_t)r0 * (size_t)D;
+    const size_t esz = dt == ORACLE_BF16 ? 2 : 4;
+    int rc = oracle_add_rms_norm(xb, (const char*)r + off * esz, w, y + off, (char*)h + off * esz,
+                                 0, r1 - r0, D, eps, dt);
+    free(xb);
+    return rc;
+}
+
 int oracle_layer_norm(const void* x, const void* w, const void* b, double* y, int64_t r0,
                       int64_t r1, int64_t D, float eps, int dt) {
     double* row = (double*)malloc((size_t)D * sizeof(double));

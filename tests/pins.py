@@ -118,6 +118,73 @@ def check_add_rms_is_rms_of_h(o):
     _close(y, o.rms_norm(h, w, 1e-5), 1e-15, what="add_rms_norm vs rms_norm(h)")
 
 
+# ---- all-reduce + add_rms_norm --------------------------------------------------------
+
+def _bf16_round_exact(v: float) -> float:
+    """bfloat16 nearest-even of a double in one rounding (Python's round() ties to even
+    on the exactly representable half-way value); normal range only."""
+    if v == 0.0:
+        return 0.0
+    m, e = math.frexp(v)                 # v = m 2^e, 0.5 <= |m| < 1
+    q = round(math.ldexp(m, 8))          # 8 significant bits
+    return math.ldexp(q, e - 8)
+
+
+def check_allreduce_rounds_exact_sum_once(o):
+    """x = the sum of the partials (in double, exact here) rounded once: 1 + 2^-8 + 2^-30
+    is above the bf16 tie 1 + 2^-8 and rounds up, and 1 + 2^-24 + 2^-40 above the binary32
+    tie; binary32 accumulation would drop the last term and round both down to 1."""
+    parts = [bf16_bits([[1.0, 3.0]]), bf16_bits([[2.0 ** -8, 2.0 ** -7]]),
+             bf16_bits([[2.0 ** -30, -2.0 ** -30]])]
+    r = bf16_bits([[0.0, 0.0]])
+    _, _, x = o.allreduce_add_rms_norm(parts, r, None, 1e-5)
+    assert widen_bf16(x).tolist() == [[1.0 + 2.0 ** -7, 3.0]], widen_bf16(x).tolist()
+    pf = [np.array([[1.0]], np.float32), np.array([[2.0 ** -24]], np.float32),
+          np.array([[2.0 ** -40]], np.float32)]     # exact in double, above the f32 tie
+    _, _, xf = o.allreduce_add_rms_norm(pf, np.zeros((1, 1), np.float32), None, 1e-5)
+    assert float(xf[0, 0]) == 1.0 + 2.0 ** -23, float(xf[0, 0])
+    ps = [_randn_bf16((13, 40), 42 + i, scale=4.0 ** i) for i in range(5)]
+    _, _, x = o.allreduce_add_rms_norm(ps, _randn_bf16((13, 40), 50), None, 1e-5)
+    exact = sum(widen_bf16(p) for p in ps)          # exact: 8-bit significands, 10 binades
+    want = np.vectorize(_bf16_round_exact)(exact)
+    assert (widen_bf16(x) == want).all(), "x is not the exact sum rounded once"
+
+
+def check_allreduce_order_and_cancellation(o):
+    """The sum does not depend on the order of the parts (exact for bf16 data); parts
+    that cancel leave x = the remaining part, h = RNE(x + r) and y = RmsNorm(h)."""
+    ps = [_randn_bf16((11, 64), 60 + i) for i in range(4)]
+    r = _randn_bf16((11, 64), 65)
+    w = bf16_bits(_rng(66).uniform(0.5, 1.5, 64))
+    y1, h1, x1 = o.allreduce_add_rms_norm(ps, r, w, 1e-5)
+    y2, h2, x2 = o.allreduce_add_rms_norm(ps[::-1], r, w, 1e-5)
+    assert (x1 == x2).all() and (h1 == h2).all() and (y1 == y2).all()
+    p = ps[0]
+    neg = p ^ np.uint16(0x8000)                      # -p exactly
+    y, h, x = o.allreduce_add_rms_norm([p, neg, ps[1]], r, w, 1e-5)
+    assert (x == ps[1]).all(), "p + (-p) + q must be q"
+    s = widen_bf16(ps[1]).astype(np.float32) + widen_bf16(r).astype(np.float32)
+    assert (h == bf16_bits(s)).all(), "h must be RNE(x + r)"
+    hd = widen_bf16(h)
+    want = hd / np.sqrt((hd * hd).mean(axis=1, keepdims=True) + 1e-5) * widen_bf16(w)
+    _close(y, want, 1e-13, what="y = RmsNorm(h) * w")
+
+
+def check_allreduce_hand_case(o):
+    """parts [1, 2] and [3, 4], r = [0.5, 0.5]: x = [4, 6], h = [4.5, 6.5],
+    y = h / sqrt((4.5^2 + 6.5^2) / 2 + eps); one part alone is add_rms_norm itself."""
+    y, h, x = o.allreduce_add_rms_norm([bf16_bits([[1.0, 2.0]]), bf16_bits([[3.0, 4.0]])],
+                                       bf16_bits([[0.5, 0.5]]), None, 1e-5)
+    assert widen_bf16(x).tolist() == [[4.0, 6.0]] and widen_bf16(h).tolist() == [[4.5, 6.5]]
+    den = math.sqrt((4.5 ** 2 + 6.5 ** 2) / 2 + float(np.float32(1e-5)))   # eps is binary32
+    _close(y, [[4.5 / den, 6.5 / den]], 1e-15, what="hand case")
+    p = _randn_bf16((7, 48), 70)
+    r = _randn_bf16((7, 48), 71)
+    y1, h1, x1 = o.allreduce_add_rms_norm([p], r, None, 1e-6)
+    y2, h2 = o.add_rms_norm(p, r, None, 1e-6)
+    assert (x1 == p).all() and (h1 == h2).all() and (y1 == y2).all()
+
+
 # ---- rms_norm -------------------------------------------------------------------------
 
 def check_rms_constant_rows(o):

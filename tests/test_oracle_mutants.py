@@ -22,6 +22,14 @@ MUTANTS = {
     "add_normalises_unrounded_h": ("row[j] = widen(h, dt, i);", "row[j] = (double)sum;"),
     "add_drops_residual": ("float sum = (float)widen(x, dt, i) + (float)widen(r, dt, i);",
                            "float sum = (float)widen(x, dt, i);"),
+    "allreduce_float_accumulation": ("double s = 0.0;\n            for (int p = 0; p < nparts; ++p)",
+                                     "float s = 0.0f;\n            for (int p = 0; p < nparts; ++p)"),
+    "allreduce_drops_last_part": ("for (int p = 0; p < nparts; ++p) s +=",
+                                  "for (int p = 0; p < nparts - 1; ++p) s +="),
+    "allreduce_rounds_through_binary32": ("((uint16_t*)xb)[o] = oracle_bf16_from_f64(s);",
+                                          "((uint16_t*)xb)[o] = oracle_bf16_from_f64((double)(float)s);"),
+    "allreduce_skips_residual": ("int rc = oracle_add_rms_norm(xb, (const char*)r + off * esz,",
+                                 "int rc = oracle_add_rms_norm(xb, (const char*)xb,"),
     "layer_unbiased_variance": ("double var = sqdev / (double)D;",
                                 "double var = sqdev / (double)(D - 1);"),
     "layer_drops_mean_in_output": ("y[j] = (x[j] - mean) / denom * wj + bj;",
