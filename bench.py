@@ -170,7 +170,9 @@ def job_throughput(world: int, step_bytes: int, steps: int, max_ms: float) -> fl
 
 # ---- workloads ----------------------------------------------------------------------
 
-def algorithmic_bytes(op, rows, D, s):
+def algorithmic_bytes(op, rows, D, s, nparts=0):
+    if op == "allreduce_add_rms_norm":  # read the parts, r, w; write y, h
+        return (nparts + 3) * rows * D * s + D * s
     if op == "add_rms_norm":
         return 4 * rows * D * s + D * s
     if op == "rms_norm":
@@ -215,6 +217,10 @@ class Case:
                        "w": synth.uniform_device((D,), 0.5, 1.5, seed, synth.W, dtype)}
             elif op == "add_rms_norm":
                 inp = synth.add_rms_inputs(rows, D, dtype, seed)
+            elif op == "allreduce_add_rms_norm":
+                a = synth.allreduce_inputs(rows, D, kw["nparts"], dtype, seed)
+                inp = {"r": a["r"], "w": a["w"]}
+                inp.update({f"p{i}": p for i, p in enumerate(a["parts"])})
             elif op in ("rms_norm", "rms_norm_vjp"):
                 inp = synth.rms_inputs(rows, D, dtype, seed)
             else:
@@ -226,9 +232,13 @@ class Case:
                      for k, v in inp.items()}
         self.device_drawn = on_dev
         src = inp if on_dev else self.host
-        self.bytes = algorithmic_bytes(op, self.rows, self.D, self.s)
+        self.nparts = kw.get("nparts", 0)
+        self.bytes = algorithmic_bytes(op, self.rows, self.D, self.s, self.nparts)
         l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
         n_row_tensors = 4 if op == "add_rms_norm" else (3 if op.endswith("_vjp") else 2)
+        if op == "allreduce_add_rms_norm":
+            n_row_tensors = self.nparts + 3
+        self.n_row_tensors = n_row_tensors
         set_bytes = n_row_tensors * self.rows * self.D * self.s
         if set_bytes >= l2:
             self.nsets = max(2, min(8, -(-3 * l2 // set_bytes)))
@@ -238,8 +248,8 @@ class Case:
         for _ in range(self.nsets):
             d = {k: (v.clone() if on_dev else v.cuda()) if v is not None else None
                  for k, v in src.items()}
-            d["y"] = torch.empty_like(d["x"])
-            d["h"] = torch.empty_like(d["x"]) if op == "add_rms_norm" else None
+            d["y"] = torch.empty_like(d["r"] if op == "allreduce_add_rms_norm" else d["x"])
+            d["h"] = torch.empty_like(d["y"]) if "add_rms_norm" in op else None
             if op.endswith("_vjp"):
                 d["dw"] = torch.empty_like(d["w"])
                 d["db"] = torch.empty_like(d["w"])
@@ -248,7 +258,7 @@ class Case:
             self.sets.append(d)
         self.nv = nv
         n_out = 2 if op == "add_rms_norm" else 1
-        self.host_out = [] if on_dev else \
+        self.host_out = [] if on_dev or "x" not in self.host else \
             [torch.empty_like(self.host["x"]).pin_memory() for _ in range(n_out)]
         self.plan = None
 
@@ -258,9 +268,7 @@ class Case:
 
     def l2_note(self):
         if self.rotating:
-            mb = self.nsets * (4 if self.op == "add_rms_norm" else (3 if self.op.endswith("_vjp")
-                                                                  else 2)) \
-            * self.rows * self.D * self.s
+            mb = self.nsets * self.n_row_tensors * self.rows * self.D * self.s
             return (f"inputs larger than L2: {self.nsets} buffer sets ({mb / 1e6:.0f} MB) "
                     "rotated, steps back to back, no flush")
         return "L2 flushed before every step (write of 2x L2)"
@@ -269,6 +277,9 @@ class Case:
         d, nv, k = self.sets[i % self.nsets], self.nv, self.kw
         if self.op == "add_rms_norm":
             nv.nv_add_rms_norm(d["x"], d["r"], d["w"], d["y"], d["h"], k["eps"], stream, self.plan)
+        elif self.op == "allreduce_add_rms_norm":
+            nv.nv_allreduce_add_rms_norm([d[f"p{j}"] for j in range(self.nparts)], d["r"], d["w"],
+                                         d["y"], d["h"], k["eps"], stream=stream)
         elif self.op == "rms_norm":
             nv.nv_rms_norm(d["x"], d["w"], d["y"], k["eps"], stream, self.plan)
         elif self.op == "layer_norm":
@@ -549,6 +560,10 @@ WORKLOADS = {
                                           offset=4096),
     "rms_norm_vjp": lambda: Case("rms_norm_vjp", (8192, 4096), "bf16", 0, eps=1e-5),
     "layer_norm_vjp": lambda: Case("layer_norm_vjp", (16384, 8192), "bf16", 0, eps=1e-5),
+    # a TP8 decoder's all-reduce + residual add + RMSNorm, the 8 partial outputs already
+    # in this GPU's memory (the reduction half of a one-shot all-reduce)
+    "allreduce_add_rms_norm": lambda: Case("allreduce_add_rms_norm", (8192, 4096), "bf16", 0,
+                                           eps=1e-5, nparts=8),
 }
 
 

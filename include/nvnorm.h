@@ -167,6 +167,30 @@ NV_API nv_status nv_layer_norm_vjp(const void* x, const void* w, const void* g, 
 NV_API size_t nv_norm_vjp_workspace_size(int32_t op, int64_t rows, int64_t D);
 
 /*
+ * allreduce_add_rms_norm -- the step a tensor-parallel decoder takes after a row-parallel
+ * layer: miniVLLM Layers page, section Linear layers, RowParallelLinear (the forward pass
+ * sums the ranks' partial outputs with an all_reduce), then the fused residual add +
+ * RMSNorm (same page, section LayerNorm; docs.rs nuvec-core 0.5.0, Enum FastOp, variant
+ * AddRmsNorm).  This call is the reduction half of a one-shot all-reduce fused with the
+ * norm: given every rank's partial output it computes
+ *   x = sum of parts[0..nparts) in that order, in double, rounded once to dt;
+ *   h = x + r in float32 rounded to dt;  y = h / sqrt(mean(h^2) + eps) * w.
+ * Every rank that calls it with the same parts gets bit-identical x, h and y.
+ * parts: host array of nparts (1..8) device pointers, each [rows, D] in: this GPU's memory
+ * (for example the slots of an all-gather) or another GPU's buffer mapped into this
+ * process (peer access / IPC; the call reads it directly).  r [rows, D] in (the residual);
+ * w [D] or NULL; y [rows, D] out; h [rows, D] out (may be r); x_out [rows, D] out or NULL
+ * (may be one of the parts).  r, w, y, h and x_out must be memory of the current device.
+ * The caller orders the producers of remote parts before this call (e.g. a barrier or a
+ * collective on `stream`).  Errors: NV_ERR_INVALID_ARG for bad pointers, sizes, overlaps or
+ * nparts outside 1..8.
+ */
+NV_API nv_status nv_allreduce_add_rms_norm(const void* const* parts, int32_t nparts,
+                                           const void* r, const void* w, void* y, void* h,
+                                           void* x_out, int64_t rows, int64_t D, float eps,
+                                           nv_dtype dt, nv_stream_t stream);
+
+/*
  * add_rms_norm_host -- add_rms_norm (as nv_add_rms_norm) on rows that live in host
  * memory: x and r are copied in, the op runs, y and h are copied back, pipelined over
  * chunks of chunk_rows rows (0 = about eight chunks) on internal streams so that copies in

@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "NvError", "Plan", "library", "library_path",
-    "nv_rms_norm", "nv_add_rms_norm", "nv_add_rms_norm_host", "nv_layer_norm", "nv_norm_rope",
+    "nv_rms_norm", "nv_add_rms_norm", "nv_add_rms_norm_host", "nv_allreduce_add_rms_norm",
+    "allreduce_add_rms_norm", "nv_layer_norm", "nv_norm_rope",
     "nv_describe_plan",
     "nv_fault_count",
     "nv_rope", "rms_norm", "add_rms_norm", "layer_norm", "norm_rope", "norm_rope_into_cache",
@@ -76,6 +77,8 @@ def library() -> ctypes.CDLL:
         "nv_add_rms_norm": [vp, vp, vp, vp, vp, i64, i64, f32, i32, vp],
         "nv_add_rms_norm_host": [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, f32, i32, i64,
                                  vp],
+        "nv_allreduce_add_rms_norm": [ctypes.POINTER(vp), i32, vp, vp, vp, vp, vp, i64, i64,
+                                      f32, i32, vp],
         "nv_layer_norm": [vp, vp, vp, vp, i64, i64, f32, i32, vp],
         "nv_norm_rope": [vp, vp, vp, i64, i64, i64, i32, i32, f32, f32, i64, i32, f32, i32, vp],
         "nv_rms_norm_ex": [vp, vp, vp, i64, i64, f32, i32, vp, pp],
@@ -191,6 +194,25 @@ def nv_add_rms_norm_host(x_host, r_host, w, y_host, h_host, x_dev, r_dev, y_dev,
                                   _dtype(x_host, r_host, w, y_host, h_host, x_dev, r_dev,
                                          y_dev, h_dev), chunk_rows, _stream(stream))
     _check("nv_add_rms_norm_host", st)
+
+
+def nv_allreduce_add_rms_norm(parts, r, w, y, h, eps, x_out=None, stream=None):
+    """x = sum(parts) (in order, in double, rounded once), h = x + r, y = RmsNorm(h) * w.
+    ``parts`` are device tensors shaped like r (this GPU's, or peers' mapped buffers)."""
+    rows, D = _rows_D(r)
+    table = (ctypes.c_void_p * len(parts))(*[t.data_ptr() for t in parts])
+    lib = library()
+    st = lib.nv_allreduce_add_rms_norm(table, len(parts), _ptr(r), _ptr(w), _ptr(y), _ptr(h),
+                                       _ptr(x_out), rows, D, eps,
+                                       _dtype(*parts, r, w, y, h, x_out), _stream(stream))
+    _check("nv_allreduce_add_rms_norm", st)
+
+
+def allreduce_add_rms_norm(parts, r, w, eps=1e-5):
+    """Allocating form: returns (y, h, x) for device tensors."""
+    y, h, x = torch.empty_like(r), torch.empty_like(r), torch.empty_like(r)
+    nv_allreduce_add_rms_norm(parts, r, w, y, h, eps, x_out=x)
+    return y, h, x
 
 
 def nv_layer_norm(x, w, b, y, eps, stream=None, plan=None):

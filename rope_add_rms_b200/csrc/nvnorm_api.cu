@@ -14,6 +14,7 @@
 
 #include "nvnorm.h"
 
+#include "allreduce.cuh"
 #include "common.cuh"
 #include "layer.cuh"
 #include "rms.cuh"
@@ -643,6 +644,109 @@ nv_status rope_op(const void* x, const void* w, const float* freqs, void* y, int
               : launch_rope_generic<float>(di, p.ctas_per_sm, cs, a);
 }
 
+// ---- all-reduce of partial sums + add_rms_norm ---------------------------------------------
+// A part may live on another GPU (mapped into this process): it must be device memory of
+// some device and lie inside one allocation; the other buffers belong to the current one.
+nv_status check_part(const void* p, size_t bytes, int i) {
+    cudaPointerAttributes at;
+    cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess || (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)) {
+        cudaGetLastError();
+        return fail(NV_ERR_INVALID_ARG, "parts[%d] (%p) is not device memory", i, p);
+    }
+    RangeFn fn = range_fn();
+    if (fn) {
+        CUdeviceptr base = 0;
+        size_t size = 0;
+        if (fn(&base, &size, (CUdeviceptr)(uintptr_t)p) == CUDA_SUCCESS &&
+            (uintptr_t)p + bytes > (uintptr_t)base + size)
+            return fail(NV_ERR_INVALID_ARG, "parts[%d] (%p): %zu bytes run past the end of its "
+                        "allocation", i, p, bytes);
+    }
+    return NV_OK;
+}
+
+nv_status allreduce_add_rms_norm(const void* const* parts, int32_t nparts, const void* r,
+                                 const void* w, void* y, void* h, void* x_out, int64_t rows,
+                                 int64_t D, float eps, nv_dtype dt, nv_stream_t stream) {
+    nv_status st = check_common(rows, D, eps, dt);
+    if (st != NV_OK) return st;
+    if (nparts < 1 || nparts > kMaxParts)
+        return fail(NV_ERR_INVALID_ARG, "nparts = %d must be 1..%d", nparts, kMaxParts);
+    if (rows == 0) return NV_OK;
+    if (!parts) return fail(NV_ERR_INVALID_ARG, "parts is NULL");
+    for (int i = 0; i < nparts; ++i)
+        if (!parts[i]) return fail(NV_ERR_INVALID_ARG, "parts[%d] is NULL", i);
+    if (!r) return fail(NV_ERR_INVALID_ARG, "r is NULL");
+    if (!y) return fail(NV_ERR_INVALID_ARG, "y is NULL");
+    if (!h) return fail(NV_ERR_INVALID_ARG, "h is NULL");
+    const size_t s = elem_size(dt);
+    const size_t nbytes = (size_t)rows * (size_t)D * s;
+    for (int i = 0; i < nparts; ++i) {
+        st = check_part(parts[i], nbytes, i);
+        if (st != NV_OK) return st;
+    }
+    int dev = 0;
+    DevInfo di;
+    st = current_device(&dev, &di);
+    if (st != NV_OK) return st;
+    // outputs may be exactly a row input (h over r, x_out over a part), nothing else
+    Buf bufs[kMaxParts + 5];
+    int nb = 0;
+    bufs[nb++] = {r, nbytes, "r", false, true};
+    bufs[nb++] = {w, (size_t)D * s, "w", false, false};
+    bufs[nb++] = {y, nbytes, "y", true, false};
+    bufs[nb++] = {h, nbytes, "h", true, false};
+    bufs[nb++] = {x_out, nbytes, "x_out", true, false};
+    st = check_buffers(bufs, nb, dev);
+    if (st != NV_OK) return st;
+    for (int i = 0; i < nparts; ++i) {  // parts are inputs: only x_out may be one of them
+        const uintptr_t p0 = (uintptr_t)parts[i], p1 = p0 + nbytes;
+        const void* outs[] = {y, h, x_out};
+        const char* names[] = {"y", "h", "x_out"};
+        for (int o = 0; o < 3; ++o) {
+            if (!outs[o]) continue;
+            const uintptr_t o0 = (uintptr_t)outs[o], o1 = o0 + nbytes;
+            if (o0 >= p1 || p0 >= o1) continue;
+            if (o == 2 && o0 == p0) continue;
+            return fail(NV_ERR_INVALID_ARG, "output %s overlaps parts[%d]", names[o], i);
+        }
+    }
+
+    ReduceNormArgs a{};
+    for (int i = 0; i < nparts; ++i) a.parts[i] = parts[i];
+    a.nparts = nparts;
+    a.r = r;
+    a.w = w;
+    a.y = y;
+    a.h = h;
+    a.x_out = x_out;
+    a.rows = rows;
+    a.D = (int)D;
+    a.eps = eps;
+    g_pdl = true;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf = dt == NV_BF16;
+    const int vecw = 16 / (int)s;
+    bool al = aligned16(r) && aligned16(y) && aligned16(h) && (!w || aligned16(w)) &&
+              (!x_out || aligned16(x_out)) && D % vecw == 0;
+    for (int i = 0; i < nparts; ++i) al = al && aligned16(parts[i]);
+    const int64_t nvec = D / vecw;
+    const int64_t grid = std::min<int64_t>(rows, INT32_MAX);
+    if (al && nvec <= 2048) {
+        const int vpt = nvec <= 1024 ? 1 : 2;
+        a.nvec = (int)nvec;
+        a.G = (int)(((nvec + vpt - 1) / vpt + 31) / 32 * 32);
+        if (vpt == 1)
+            return bf ? launch_kernel(allreduce_rms_rows_kernel<__nv_bfloat16, 1>, grid, a.G, 0, cs, a)
+                      : launch_kernel(allreduce_rms_rows_kernel<float, 1>, grid, a.G, 0, cs, a);
+        return bf ? launch_kernel(allreduce_rms_rows_kernel<__nv_bfloat16, 2>, grid, a.G, 0, cs, a)
+                  : launch_kernel(allreduce_rms_rows_kernel<float, 2>, grid, a.G, 0, cs, a);
+    }
+    return bf ? launch_kernel(allreduce_rms_generic_kernel<__nv_bfloat16>, grid, 256, 0, cs, a)
+              : launch_kernel(allreduce_rms_generic_kernel<float>, grid, 256, 0, cs, a);
+}
+
 // ---- host-resident rows: copies and compute pipelined over row chunks ---------------------
 // Chunk k goes to internal stream k % kPipeStreams: host -> device copies of its x and r
 // rows, the add_rms_norm launch on those rows, device -> host copies of its y and h.  The
@@ -1095,6 +1199,12 @@ nv_status nv_describe_plan(int32_t op, int64_t rows, int64_t D, nv_dtype dt, nv_
         return rope_plan(rows, 1, D, (int)(D - D % 2), false, dt, true, 148, nullptr, plan, &rp);
     }
     return make_plan((Op)op, rows, D, dt, true, nullptr, plan);
+}
+
+nv_status nv_allreduce_add_rms_norm(const void* const* parts, int32_t nparts, const void* r,
+                                    const void* w, void* y, void* h, void* x_out, int64_t rows,
+                                    int64_t D, float eps, nv_dtype dt, nv_stream_t stream) {
+    return allreduce_add_rms_norm(parts, nparts, r, w, y, h, x_out, rows, D, eps, dt, stream);
 }
 
 nv_status nv_add_rms_norm_host(const void* x_host, const void* r_host, const void* w,

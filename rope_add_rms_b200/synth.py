@@ -91,6 +91,15 @@ def add_rms_inputs(rows, D, dtype="bf16", seed=0, weight=True):
             "w": uniform((D,), 0.5, 1.5, seed, W, dtype) if weight else None}
 
 
+def allreduce_inputs(rows, D, nparts, dtype="bf16", seed=0, weight=True):
+    """all-reduce + add_rms_norm: nparts partial outputs ~ N(0, 1/nparts) each (their sum
+    ~ N(0, 1), like the shards of a row-parallel layer), r ~ N(0,1), w ~ U(0.5,1.5)."""
+    sd = 1.0 / nparts ** 0.5
+    return {"parts": [normal((rows, D), 0.0, sd, seed, 16 + i, dtype) for i in range(nparts)],
+            "r": normal((rows, D), 0.0, 1.0, seed, R, dtype),
+            "w": uniform((D,), 0.5, 1.5, seed, W, dtype) if weight else None}
+
+
 def layer_norm_inputs(rows, D, dtype="bf16", seed=0, weight=True, bias=True):
     """layer_norm: x ~ N(0.5, 2^2), w ~ U(0.5,1.5), b ~ N(0, 0.1^2)."""
     return {"x": normal((rows, D), 0.5, 2.0, seed, X, dtype),

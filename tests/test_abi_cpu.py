@@ -91,6 +91,18 @@ def vjp(op="rms", x=FAKE, w=None, g=FAKE, dx=FAKE, dw=None, db=None, ws=None, ws
     return lib.nv_layer_norm_vjp(x, w, g, dx, dw, db, ws, ws_bytes, rows, D, eps, dt, None)
 
 
+def allreduce(parts=(FAKE, FAKE), n=None, r=FAKE, w=None, y=FAKE, h=ctypes.c_void_p(0x20000),
+              x_out=None, rows=4, D=8, eps=1e-5, dt=BF16):
+    table = None if parts is None else (ctypes.c_void_p * max(len(parts), 1))(*parts)
+    return nv.library().nv_allreduce_add_rms_norm(table, len(parts or ()) if n is None else n,
+                                                  r, w, y, h, x_out, rows, D, eps, dt, None)
+
+
+def host_add(x=FAKE, r=FAKE, y=FAKE, h=ctypes.c_void_p(0x20000), rows=4, D=8, chunk=0):
+    return nv.library().nv_add_rms_norm_host(x, r, None, y, h, FAKE, FAKE, FAKE, FAKE, rows, D,
+                                             1e-5, BF16, chunk, None)
+
+
 def last_error():
     return nv.library().nv_last_error().decode()
 
@@ -137,6 +149,16 @@ def last_error():
     (lambda: vjp(D=7), UNSUPPORTED, "vjp needs D"),
     (lambda: vjp(D=32768), UNSUPPORTED, "vjp needs D"),
     (lambda: vjp(g=None), INVALID, "g is NULL"),
+    (lambda: allreduce(n=0), INVALID, "nparts"),
+    (lambda: allreduce(parts=(FAKE,) * 9), INVALID, "nparts"),
+    (lambda: allreduce(parts=None, n=2), INVALID, "parts is NULL"),
+    (lambda: allreduce(parts=(FAKE, None)), INVALID, "parts[1] is NULL"),
+    (lambda: allreduce(r=None), INVALID, "r is NULL"),
+    (lambda: allreduce(h=None), INVALID, "h is NULL"),
+    (lambda: allreduce(dt=F16), UNSUPPORTED, "F16"),
+    (lambda: host_add(x=None), INVALID, "x_host is NULL"),
+    (lambda: host_add(h=FAKE), INVALID, "same buffer"),
+    (lambda: host_add(chunk=-1), INVALID, "chunk_rows"),
 ])
 def test_invalid_arguments_are_rejected_on_the_host(call, status, words):
     assert call() == status
@@ -148,6 +170,8 @@ def test_zero_rows_is_a_no_op():
     assert add(x=None, r=None, y=None, h=None, rows=0) == OK
     assert layer(x=None, y=None, rows=0) == OK
     assert rope(x=None, y=None, rows=0) == OK
+    assert allreduce(parts=None, n=1, r=None, y=None, h=None, rows=0) == OK
+    assert host_add(x=None, r=None, y=None, h=None, rows=0) == OK
 
 
 def test_plain_rope_ignores_eps():

@@ -1,7 +1,10 @@
-"""Multi-process host logic of the benchmark, on CPU with gloo (world size 2).
+"""Multi-process host logic, on CPU with gloo (world size 2).
 
-The path shards by rows with no data-path collective; what crosses ranks is the
-barrier and the max-over-ranks time.  These tests run that logic in two processes.
+The benchmark shards by rows with no data-path collective; what crosses ranks is the
+barrier and the max-over-ranks time.  The tensor-parallel all-reduce + add_rms_norm
+gathers every rank's partial output in rank order before the fused kernel; here the
+kernel is stood in for by the oracle (CPU tensors), which checks the gather, the order
+and that every rank computes the same result.
 """
 import os
 import socket
@@ -54,3 +57,40 @@ def test_single_process_is_identity_and_throughput_formula():
     # two ranks, 268,443,648 bytes per step, 1000 steps, slowest rank 41.79 ms in total
     v = bench.job_throughput(2, 268443648, 1000, 41.79)
     assert v == pytest.approx(2 * 268443648 * 1000 / 0.04179 / 1e9)
+
+
+def _tp_worker(rank, world, port, out):
+    import numpy as np
+    import oracle
+    from rope_add_rms_b200 import synth, tp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        inp = synth.allreduce_inputs(6, 32, world, "f32", seed=3)
+        seen = {}
+
+        def fake_kernel(parts, r, w, y, h, eps, x_out=None, stream=None):
+            seen["parts"] = [p.clone() for p in parts]
+            yy, hh, _ = oracle.allreduce_add_rms_norm([p.numpy() for p in parts], r.numpy(),
+                                                      w.numpy(), eps)
+            y.copy_(torch.from_numpy(yy.astype(np.float32)))
+            h.copy_(torch.from_numpy(hh))
+
+        tp.nv_allreduce_add_rms_norm = fake_kernel
+        y, h = tp.allreduce_add_rms_norm(inp["parts"][rank], inp["r"], inp["w"], 1e-5)
+        for i, p in enumerate(seen["parts"]):
+            assert torch.equal(p, inp["parts"][i]), f"part {i} is not rank {i}'s partial"
+        out[rank] = (y.numpy().tobytes(), h.numpy().tobytes())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_tp_allreduce_gathers_in_rank_order_two_processes():
+    world = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_tp_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0] == res[1], "every rank must compute the same y and h"
