@@ -6,6 +6,10 @@ Element-by-element against the CPU oracle for:
   - layer_norm bf16, x [16384, 8192] ~ N(0.5, 2^2), w ~ U(0.5,1.5), b ~ N(0, 0.1^2), eps 1e-5
   - norm_rope bf16, x [8, 32, 2048, 128] ~ N(0,1), w ~ U(0.5,1.5), eps 1e-6, dims 128,
     base 10000, scale 1: halves at offset 0, and traditional at offset 4096
+  - allreduce_add_rms_norm bf16, 8 parts [8192, 4096] ~ N(0, 1/8), r ~ N(0,1),
+    w ~ U(0.5,1.5), eps 1e-5 (the TP8 workload of the benchmark)
+  - the gradients: rms_norm_vjp bf16 [8192, 4096] and layer_norm_vjp bf16 [16384, 8192]
+    on sampled rows (dx) and every column (dw, db) summed over all rows
 and on sampled rows for the add_rms_norm sweep D x rows x {bf16, f32} (eps 1e-6).
 Large outputs are compared in row chunks to bound host memory.
 """
@@ -16,7 +20,7 @@ import torch
 import oracle
 import rope_add_rms_b200 as nv
 from rope_add_rms_b200 import synth
-from checks import check_bf16, check_exact, check_f32, sample_rows, to_host_bits
+from checks import check_bf16, check_exact, check_f32, check_grad, sample_rows, to_host_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -103,3 +107,61 @@ def test_add_rms_norm_sweep(dt, D, rows):
     (check_bf16 if dt == "bf16" else check_f32)(got, ref, "y")
     del x, r, y, h
     torch.cuda.empty_cache()
+
+
+def test_allreduce_add_rms_norm_tp8_bf16_8192x4096():
+    inp = synth.allreduce_inputs(8192, 4096, 8, "bf16", seed=0)
+    parts = [p.cuda() for p in inp["parts"]]
+    r, w = inp["r"].cuda(), inp["w"].cuda()
+    y, h, x = nv.allreduce_add_rms_norm(parts, r, w, eps=1e-5)
+    torch.cuda.synchronize()
+    ph = [host(p) for p in inp["parts"]]
+    rh, wh = host(inp["r"]), host(inp["w"])
+    xs, hs = [], []
+
+    def ref(r0, r1):
+        yr, hr, xr = oracle.allreduce_add_rms_norm([p[r0:r1] for p in ph], rh[r0:r1], wh, 1e-5)
+        xs.append(xr)
+        hs.append(hr)
+        return yr
+
+    compare_rows(y, ref, 8192, "y")
+    check_exact(h, np.concatenate(hs), "h")
+    check_exact(x, np.concatenate(xs), "x")
+
+
+@pytest.mark.parametrize("op,rows,D", [("rms", 8192, 4096), ("layer", 16384, 8192)])
+def test_gradients_full_size(op, rows, D):
+    """dx of every row chunk by chunk; dw (and db) of every column, the oracle's column sums
+    accumulated over the chunks (the bar is relative to the magnitude sums, so the
+    order of that accumulation does not matter)."""
+    if op == "rms":
+        inp = synth.rms_inputs(rows, D, "bf16", seed=0)
+    else:
+        inp = synth.layer_norm_inputs(rows, D, "bf16", seed=0, bias=False)
+    g = synth.normal((rows, D), 0.0, 1.0, 0, synth.R, "bf16")
+    x, w, gd = inp["x"].cuda(), inp["w"].cuda(), g.cuda()
+    if op == "rms":
+        dx, dw = nv.rms_norm_vjp(x, w, gd, eps=1e-5)
+        db = None
+    else:
+        dx, dw, db = nv.layer_norm_vjp(x, w, gd, eps=1e-5)
+    torch.cuda.synchronize()
+    xh, wh, gh = host(inp["x"]), host(inp["w"]), host(g)
+    sums = None
+    for r0 in range(0, rows, CHUNK):
+        r1 = min(rows, r0 + CHUNK)
+        if op == "rms":
+            rdx, rdw, mdx, mdw = oracle.rms_norm_vjp(xh[r0:r1], wh, gh[r0:r1], 1e-5)
+            parts = [rdw, mdw]
+        else:
+            rdx, rdw, rdb, mdx, mdw, mdb = oracle.layer_norm_vjp(xh[r0:r1], wh, gh[r0:r1], 1e-5)
+            parts = [rdw, rdb, mdw, mdb]
+        check_grad(dx[r0:r1], rdx, mdx, f"dx rows {r0}:{r1}")
+        parts = [np.asarray(p, np.float64) for p in parts]
+        sums = parts if sums is None else [a + b for a, b in zip(sums, parts)]
+    if op == "rms":
+        check_grad(dw, sums[0], sums[1], "dw")
+    else:
+        check_grad(dw, sums[0], sums[2], "dw")
+        check_grad(db, sums[1], sums[3], "db")

@@ -459,6 +459,50 @@ def test_allreduce_in_place_ranks_agree_and_errors():
                                      torch.empty_like(r), 1e-5)
 
 
+# ---- CUDA graphs ------------------------------------------------------------------------------
+
+def test_cuda_graph_capture_and_replay():
+    """A chain of the ops (with programmatic dependent launch) captured into one CUDA graph
+    and replayed on new inputs gives the same bits as running the calls directly."""
+    B, H, L, D = 2, 8, 64, 128
+    rows = B * H * L
+    inp = synth.add_rms_inputs(rows, D, "bf16", seed=23)
+    x, r, w = dev(inp["x"]), dev(inp["r"]), dev(inp["w"])
+    y, h, z, q = (torch.empty_like(x) for _ in range(4))
+    parts = [dev(inp["x"]), dev(inp["r"])]
+    a_y, a_h = torch.empty_like(x), torch.empty_like(x)
+
+    def chain():
+        nv.nv_add_rms_norm(x, r, w, y, h, 1e-5)
+        nv.nv_layer_norm(y, w, None, z, 1e-5)
+        nv.nv_norm_rope(z, w, q, L, D, 0, 10000.0, 1.0, 4096, 1, 1e-6)
+        nv.nv_allreduce_add_rms_norm(parts, q, w, a_y, a_h, 1e-5)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        chain()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        chain()
+    new = synth.add_rms_inputs(rows, D, "bf16", seed=24)
+    x.copy_(dev(new["x"]))
+    r.copy_(dev(new["r"]))
+    graph.replay()
+    torch.cuda.synchronize()
+    got = [t.clone() for t in (y, h, z, q, a_y, a_h)]
+    chain()
+    torch.cuda.synchronize()
+    for name, gt, et in zip("y h z q a_y a_h".split(), got, (y, h, z, q, a_y, a_h)):
+        assert torch.equal(gt.view(torch.int16), et.view(torch.int16)), f"{name} differs"
+    ref, href = oracle.add_rms_norm(host(new["x"]), host(new["r"]), host(inp["w"]), 1e-5)
+    check_exact(got[1], href, "h from the graph")
+    check_out(got[0], ref, "y from the graph")
+    del graph
+
+
 # ---- host-resident rows --------------------------------------------------------------------
 
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
