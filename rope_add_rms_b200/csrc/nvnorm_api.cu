@@ -489,7 +489,7 @@ struct RopePlan {
 template <typename T, bool TRAD>
 nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a, bool pairs) {
     const size_t smem = (size_t)a.half * sizeof(float4);
-    auto kern = (pairs && !TRAD) ? rope_pairs_kernel<T> : rope_rows_kernel<T, TRAD>;
+    auto kern = pairs ? rope_pairs_kernel<T, TRAD> : rope_rows_kernel<T, TRAD>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -515,8 +515,9 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
     const int64_t nvec = D / vecw;
     const bool vec_ok = aligned && D % vecw == 0 && nvec <= 32 &&
                         (trad || (dims / 2) % vecw == 0);
-    // both halves per lane: every feature rotated, an even number of vectors
-    const bool pairs_ok = !trad && aligned && D % vecw == 0 && dims == D && nvec % 2 == 0 &&
+    // two vectors per lane (both halves of the rotation, or two vectors of interleaved
+    // pairs): every feature rotated, an even number of vectors
+    const bool pairs_ok = aligned && D % vecw == 0 && dims == D && nvec % 2 == 0 &&
                           nvec / 2 <= 32;
     if (p.path == NV_PATH_AUTO) p.path = (vec_ok || pairs_ok) ? NV_PATH_ROWS : NV_PATH_GENERIC;
     rp->rows = p.path == NV_PATH_ROWS;

@@ -279,17 +279,81 @@ __global__ void __launch_bounds__(256, TRAD ? 3 : 2) rope_rows_kernel(const Rope
     }
 }
 
-// ---- register path, both halves per lane (halves pairing, dims == D) -----------------------
-// Each lane holds vectors v and v + nvec/2 of a row (16-byte vectors, nvec even).  With
-// halves pairing and dims == D these are exactly the p and q members of the pairs
-// i = v*VEC .. v*VEC + VEC - 1, so the partner of every element is in the lane's own
-// registers (no shuffles) and one table entry serves both of its elements.
-template <typename T>
-__global__ void __launch_bounds__(256) rope_pairs_kernel(const RopeArgs a) {
+// ---- register path, two vectors per lane (every feature rotated: dims == D) ---------------
+// Each lane holds vectors v and v + nvec/2 of a row (16-byte vectors, nvec even) and keeps
+// its elements as float pairs of rotation partners: p[k] holds the first members (the
+// cos-side inputs of y_p = a_p cos - a_q sin) of two pairs and q[k] their second members,
+// so one packed rotation serves two pairs and no partner is in another lane.
+//   halves:      vector v holds the p members of pairs v*VEC .. v*VEC + VEC - 1 and
+//                vector v + nvec/2 their q members;
+//   traditional: each vector holds VEC/2 whole pairs (2i, 2i + 1).
+// The angle table stays in shared memory, transposed so that the lanes of a row read
+// consecutive entries, and is read per row: without it in registers three CTAs fit per SM
+// (halves, bf16 [8, 32, 2048, 128]: 59.5 us against 69.5 us with the table in registers).
+template <typename T, bool TRAD>
+struct PairLayout {
     using E = Elem<T>;
-    constexpr int VEC = E::kVec;
-    constexpr int kUnroll = 3;  // rows in flight per lane group (measured best of 2..4)
-    extern __shared__ float4 tab[];  // [half]: (cos_hi, cos_lo, sin_hi, sin_lo)
+    static constexpr int VEC = E::kVec;
+    static constexpr int NP = VEC / 2;  // float pairs per side
+    // vector (0: v, 1: v + nvec/2) and element of the .x (h = 0) or .y (h = 1) member of
+    // slot k on side s (0: p, 1: q)
+    __device__ __forceinline__ static void where(int k, int h, int s, int& vec, int& e) {
+        if (!TRAD) {
+            vec = s;
+            e = 2 * k + h;
+        } else {
+            vec = k < NP / 2 ? 0 : 1;
+            e = 2 * (2 * (k % (NP / 2)) + h) + s;
+        }
+    }
+    // index in the transposed table of the pair of slot (k, h); the table has rows of
+    // `lanes` entries (halves: nvec/2, one per lane; traditional: nvec, one per vector)
+    __device__ __forceinline__ static int entry(int v0, int v1, int k, int h, int hvec) {
+        if (!TRAD) return (2 * k + h) * hvec + v0;
+        const int v = k < NP / 2 ? v0 : v1;
+        return (2 * (k % (NP / 2)) + h) * (2 * hvec) + v;
+    }
+    // the table slot of rotation pair i
+    __device__ __forceinline__ static int slot_of(int i, int hvec) {
+        return TRAD ? (i % NP) * (2 * hvec) + i / NP : (i % VEC) * hvec + i / VEC;
+    }
+    __device__ __forceinline__ static void split(const V16& a, const V16& b, float2 (&p)[NP],
+                                                 float2 (&q)[NP]) {
+#pragma unroll
+        for (int k = 0; k < NP; ++k)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                int vp, ep, vq, eq;
+                where(k, h, 0, vp, ep);
+                where(k, h, 1, vq, eq);
+                reinterpret_cast<float*>(&p[k])[h] = E::get(vp ? b : a, ep);
+                reinterpret_cast<float*>(&q[k])[h] = E::get(vq ? b : a, eq);
+            }
+    }
+    __device__ __forceinline__ static void join(const float2 (&p)[NP], const float2 (&q)[NP],
+                                                V16& a, V16& b) {
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+            if (!TRAD) {
+                E::put2(a, 2 * k, p[k]);
+                E::put2(b, 2 * k, q[k]);
+            } else {  // pair (2i, 2i + 1) is elements (e, e + 1) of one vector
+                V16& v = k < NP / 2 ? a : b;
+                const int e0 = 4 * (k % (NP / 2));
+                E::put2(v, e0, p[k].x, q[k].x);
+                E::put2(v, e0 + 2, p[k].y, q[k].y);
+            }
+        }
+    }
+};
+
+template <typename T, bool TRAD>
+__global__ void __launch_bounds__(256, 3) rope_pairs_kernel(const RopeArgs a) {
+    using E = Elem<T>;
+    using PL = PairLayout<T, TRAD>;
+    constexpr int NP = PL::NP;
+    constexpr int kUnroll = 2;  // rows in flight per lane group (measured best of 2..4)
+    extern __shared__ float4 tab[];  // transposed: (cos_hi, cos_lo, sin_hi, sin_lo)
 
     const int64_t chunk = blockIdx.x % a.n_chunks;
     const int64_t l = blockIdx.x / a.n_chunks;
@@ -322,7 +386,7 @@ __global__ void __launch_bounds__(256) rope_pairs_kernel(const RopeArgs a) {
         }
     }
     const bool norm = a.normalize != 0;
-    float2 w0[VEC / 2], w1[VEC / 2];
+    float2 wp[NP], wq[NP];
     {
         const V16 wa = (norm && a.w && has_vec)
                            ? ld_param(static_cast<const char*>(a.w) + (size_t)v0 * 16) : ones_vec<T>();
@@ -331,25 +395,10 @@ __global__ void __launch_bounds__(256) rope_pairs_kernel(const RopeArgs a) {
         // the angle table is built while the first rows' loads are in flight
         const double pos = (double)(a.offset + l);
         for (int i = threadIdx.x; i < a.half; i += blockDim.x)
-            tab[i] = angle_entry(a, pos, i);
-#pragma unroll
-        for (int e = 0; e < VEC; e += 2) {
-            w0[e / 2] = E::get2(wa, e);
-            w1[e / 2] = E::get2(wb, e);
-        }
+            tab[PL::slot_of(i, hvec)] = angle_entry(a, pos, i);
+        PL::split(wa, wb, wp, wq);
     }
     __syncthreads();
-
-    float2 c_hi[VEC / 2], c_lo[VEC / 2], s_hi[VEC / 2], s_lo[VEC / 2];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-        float4 t4 = make_float4(1.f, 0.f, 0.f, 0.f);
-        if (has_vec) t4 = tab[v0 * VEC + e];
-        reinterpret_cast<float*>(&c_hi[e / 2])[e & 1] = t4.x;
-        reinterpret_cast<float*>(&c_lo[e / 2])[e & 1] = t4.y;
-        reinterpret_cast<float*>(&s_hi[e / 2])[e & 1] = t4.z;
-        reinterpret_cast<float*>(&s_lo[e / 2])[e & 1] = t4.w;
-    }
 
     const float invD = 1.0f / (float)a.D;
     for (int64_t base = bh0; base < bh_end; base += (int64_t)kUnroll * slots) {
@@ -364,30 +413,32 @@ __global__ void __launch_bounds__(256) rope_pairs_kernel(const RopeArgs a) {
                 xv[u][0] = ld_stream(xbase + (size_t)bn * lstride + (size_t)v0 * 16);
                 xv[u][1] = ld_stream(xbase + (size_t)bn * lstride + (size_t)v1 * 16);
             }
-            float2 x0[VEC / 2], x1[VEC / 2];
+            float2 p[NP], q[NP];
+            PL::split(xa, xb, p, q);
             float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < VEC; e += 2) {
-                x0[e / 2] = E::get2(xa, e);
-                x1[e / 2] = E::get2(xb, e);
-                ss2 = fma2(x0[e / 2], x0[e / 2], ss2);
-                ss2 = fma2(x1[e / 2], x1[e / 2], ss2);
+            for (int k = 0; k < NP; ++k) {
+                ss2 = fma2(p[k], p[k], ss2);
+                ss2 = fma2(q[k], q[k], ss2);
             }
             const float ss = group_sum(__fadd_rn(ss2.x, ss2.y), lpr);
             const float inv = norm ? rsqrtf(__fmaf_rn(ss, invD, a.eps)) : 1.f;
             const float2 inv2 = make_float2(inv, inv);
-            if (live) {
-                V16 o0, o1;
+            if (live) {  // only lanes holding vectors read the table
+                float2 yp[NP], yq[NP];
 #pragma unroll
-                for (int e = 0; e < VEC; e += 2) {
-                    const int q = e / 2;
-                    const float2 a0 = mul2(x0[q], w0[q]);  // exact for bfloat16 data
-                    const float2 a1 = mul2(x1[q], w1[q]);
-                    const float2 z0 = rotate_sub2(a0, a1, c_hi[q], c_lo[q], s_hi[q], s_lo[q]);
-                    const float2 z1 = rotate_pair2(a1, a0, c_hi[q], c_lo[q], s_hi[q], s_lo[q]);
-                    E::put2(o0, e, mul2(z0, inv2));
-                    E::put2(o1, e, mul2(z1, inv2));
+                for (int k = 0; k < NP; ++k) {
+                    const float4 t0 = tab[PL::entry(v0, v1, k, 0, hvec)];
+                    const float4 t1 = tab[PL::entry(v0, v1, k, 1, hvec)];
+                    const float2 ch = make_float2(t0.x, t1.x), cl = make_float2(t0.y, t1.y);
+                    const float2 sh = make_float2(t0.z, t1.z), sl = make_float2(t0.w, t1.w);
+                    const float2 ap = mul2(p[k], wp[k]);  // exact for bfloat16 data
+                    const float2 aq = mul2(q[k], wq[k]);
+                    yp[k] = mul2(rotate_sub2(ap, aq, ch, cl, sh, sl), inv2);
+                    yq[k] = mul2(rotate_pair2(aq, ap, ch, cl, sh, sl), inv2);
                 }
+                V16 o0, o1;
+                PL::join(yp, yq, o0, o1);
                 st_stream(ybase + (size_t)b * ystride + (size_t)v0 * 16, o0);
                 st_stream(ybase + (size_t)b * ystride + (size_t)v1 * 16, o1);
             }
