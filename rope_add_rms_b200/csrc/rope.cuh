@@ -352,7 +352,9 @@ __global__ void __launch_bounds__(256, 3) rope_pairs_kernel(const RopeArgs a) {
     using E = Elem<T>;
     using PL = PairLayout<T, TRAD>;
     constexpr int NP = PL::NP;
-    constexpr int kUnroll = 2;  // rows in flight per lane group (measured best of 2..4)
+    // rows in flight per lane group (measured best of 2..4 at three CTAs per SM: 2 for
+    // bfloat16, 4 for the float32 rows that carry twice the bytes per element)
+    constexpr int kUnroll = sizeof(T) == 4 ? 4 : 2;
     extern __shared__ float4 tab[];  // transposed: (cos_hi, cos_lo, sin_hi, sin_lo)
 
     const int64_t chunk = blockIdx.x % a.n_chunks;
