@@ -260,8 +260,9 @@ NV_API nv_status nv_fault_count(uint32_t* count, int32_t reset);
  * that forces one.  A plan that the shape cannot use returns NV_ERR_UNSUPPORTED.
  *   path            NV_PATH_AUTO, or one of the kernel families below
  *   vec_per_thread  16-byte vectors per thread and row (register paths; 0 = auto; for
- *                   norm_rope 1 = one vector per lane, 2 = both halves of the rotation
- *                   per lane, which needs halves pairing and dims == D)
+ *                   norm_rope 1 = one vector per lane, 2 = two vectors per lane (both
+ *                   halves of a rotation, or two vectors of interleaved pairs), which
+ *                   needs dims == D)
  *   threads_per_row threads that share one row (multiple of 32, <= 1024; 0 = auto)
  *   rows_per_cta    rows one CTA works on at a time (0 = auto)
  *   ctas_per_sm     0: one CTA per row group (rms_norm register path, generic paths),

@@ -480,7 +480,7 @@ nv_status row_dispatch(Op op, const nv_plan& p, const DevInfo& di, nv_dtype dt, 
 // ---- norm_rope -------------------------------------------------------------------------------
 struct RopePlan {
     bool rows;
-    bool pairs;  // both halves of the rotation in one lane (dims == D)
+    bool pairs;  // two vectors per lane: rope_pairs_kernel (dims == D)
     int lpr;
     int bt;
     int64_t n_chunks;
