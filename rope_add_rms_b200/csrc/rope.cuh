@@ -287,9 +287,11 @@ __global__ void __launch_bounds__(256, TRAD ? 3 : 2) rope_rows_kernel(const Rope
 //   halves:      vector v holds the p members of pairs v*VEC .. v*VEC + VEC - 1 and
 //                vector v + nvec/2 their q members;
 //   traditional: each vector holds VEC/2 whole pairs (2i, 2i + 1).
-// The angle table stays in shared memory, transposed so that the lanes of a row read
-// consecutive entries, and is read per row: without it in registers three CTAs fit per SM
-// (halves, bf16 [8, 32, 2048, 128]: 59.5 us against 69.5 us with the table in registers).
+// The angle table stays in shared memory as records of two pairs, transposed so that the
+// lanes of a row read consecutive records, and is read per row: without it in registers
+// three CTAs fit per SM, and a record load yields the float pairs the packed rotation takes
+// (halves, bf16 [8, 32, 2048, 128]: 54.3 us; 59.2 us with one entry per pair, 69.5 us with
+// the table in registers).
 template <typename T, bool TRAD>
 struct PairLayout {
     using E = Elem<T>;
@@ -306,16 +308,24 @@ struct PairLayout {
             e = 2 * (2 * (k % (NP / 2)) + h) + s;
         }
     }
-    // index in the transposed table of the pair of slot (k, h); the table has rows of
-    // `lanes` entries (halves: nvec/2, one per lane; traditional: nvec, one per vector)
-    __device__ __forceinline__ static int entry(int v0, int v1, int k, int h, int hvec) {
-        if (!TRAD) return (2 * k + h) * hvec + v0;
-        const int v = k < NP / 2 ? v0 : v1;
-        return (2 * (k % (NP / 2)) + h) * (2 * hvec) + v;
+    // The table holds one record per two pairs served by one packed rotation: C =
+    // (cos_hi, cos_hi', cos_lo, cos_lo') and S = (sin_hi, sin_hi', sin_lo, sin_lo'), so one
+    // 16-byte load gives the float pairs directly.  Records are transposed (row k of
+    // `lanes` records), so the lanes of a row read consecutive records:
+    //   halves:      slot k of lane v  -> record k * nvec/2 + v;
+    //   traditional: slot k of lane v  -> record (k mod NP/2) * nvec + (v or v + nvec/2).
+    __device__ __forceinline__ static int record(int v0, int v1, int k, int hvec) {
+        if (!TRAD) return k * hvec + v0;
+        return (k % (NP / 2)) * (2 * hvec) + (k < NP / 2 ? v0 : v1);
     }
-    // the table slot of rotation pair i
-    __device__ __forceinline__ static int slot_of(int i, int hvec) {
-        return TRAD ? (i % NP) * (2 * hvec) + i / NP : (i % VEC) * hvec + i / VEC;
+    // record of rotation pair i and which member (.x / .y of each half) it is
+    __device__ __forceinline__ static int record_of(int i, int hvec, int& h) {
+        if (!TRAD) {
+            h = (i % VEC) & 1;
+            return ((i % VEC) >> 1) * hvec + i / VEC;
+        }
+        h = (i % NP) & 1;
+        return ((i % NP) >> 1) * (2 * hvec) + i / NP;
     }
     __device__ __forceinline__ static void split(const V16& a, const V16& b, float2 (&p)[NP],
                                                  float2 (&q)[NP]) {
@@ -355,7 +365,7 @@ __global__ void __launch_bounds__(256, 3) rope_pairs_kernel(const RopeArgs a) {
     // rows in flight per lane group (measured best of 2..4 at three CTAs per SM: 2 for
     // bfloat16, 4 for the float32 rows that carry twice the bytes per element)
     constexpr int kUnroll = sizeof(T) == 4 ? 4 : 2;
-    extern __shared__ float4 tab[];  // transposed: (cos_hi, cos_lo, sin_hi, sin_lo)
+    extern __shared__ float4 tab[];  // records: C [half / 2], then S [half / 2]
 
     const int64_t chunk = blockIdx.x % a.n_chunks;
     const int64_t l = blockIdx.x / a.n_chunks;
@@ -396,8 +406,17 @@ __global__ void __launch_bounds__(256, 3) rope_pairs_kernel(const RopeArgs a) {
                            ? ld_param(static_cast<const char*>(a.w) + (size_t)v1 * 16) : ones_vec<T>();
         // the angle table is built while the first rows' loads are in flight
         const double pos = (double)(a.offset + l);
-        for (int i = threadIdx.x; i < a.half; i += blockDim.x)
-            tab[PL::slot_of(i, hvec)] = angle_entry(a, pos, i);
+        float* tabf = reinterpret_cast<float*>(tab);
+        const int nrec = a.half / 2;
+        for (int i = threadIdx.x; i < a.half; i += blockDim.x) {
+            int h = 0;
+            const int rec = PL::record_of(i, hvec, h);
+            const float4 t = angle_entry(a, pos, i);
+            tabf[rec * 4 + h] = t.x;               // C: cos_hi, cos_lo
+            tabf[rec * 4 + 2 + h] = t.y;
+            tabf[(nrec + rec) * 4 + h] = t.z;      // S: sin_hi, sin_lo
+            tabf[(nrec + rec) * 4 + 2 + h] = t.w;
+        }
         PL::split(wa, wb, wp, wq);
     }
     __syncthreads();
@@ -430,10 +449,10 @@ __global__ void __launch_bounds__(256, 3) rope_pairs_kernel(const RopeArgs a) {
                 float2 yp[NP], yq[NP];
 #pragma unroll
                 for (int k = 0; k < NP; ++k) {
-                    const float4 t0 = tab[PL::entry(v0, v1, k, 0, hvec)];
-                    const float4 t1 = tab[PL::entry(v0, v1, k, 1, hvec)];
-                    const float2 ch = make_float2(t0.x, t1.x), cl = make_float2(t0.y, t1.y);
-                    const float2 sh = make_float2(t0.z, t1.z), sl = make_float2(t0.w, t1.w);
+                    const int rec = PL::record(v0, v1, k, hvec);
+                    const float4 c4 = tab[rec], s4 = tab[a.half / 2 + rec];
+                    const float2 ch = make_float2(c4.x, c4.y), cl = make_float2(c4.z, c4.w);
+                    const float2 sh = make_float2(s4.x, s4.y), sl = make_float2(s4.z, s4.w);
                     const float2 ap = mul2(p[k], wp[k]);  // exact for bfloat16 data
                     const float2 aq = mul2(q[k], wq[k]);
                     yp[k] = mul2(rotate_sub2(ap, aq, ch, cl, sh, sl), inv2);
