@@ -488,7 +488,10 @@ struct RopePlan {
 
 template <typename T, bool TRAD>
 nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a, bool pairs) {
-    const size_t smem = (size_t)a.half * sizeof(float4);
+    // the pairs kernel keeps its lanes' weights after the table: VEC/2 records per lane
+    const size_t smem = (size_t)a.half * sizeof(float4) +
+                        (pairs ? (size_t)Elem<T>::kVec / 2 * (size_t)(a.nvec / 2) * sizeof(float4)
+                               : 0);
     auto kern = pairs ? rope_pairs_kernel<T, TRAD> : rope_rows_kernel<T, TRAD>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

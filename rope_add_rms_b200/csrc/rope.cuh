@@ -287,11 +287,12 @@ __global__ void __launch_bounds__(256, TRAD ? 3 : 2) rope_rows_kernel(const Rope
 //   halves:      vector v holds the p members of pairs v*VEC .. v*VEC + VEC - 1 and
 //                vector v + nvec/2 their q members;
 //   traditional: each vector holds VEC/2 whole pairs (2i, 2i + 1).
-// The angle table stays in shared memory as records of two pairs, transposed so that the
-// lanes of a row read consecutive records, and is read per row: without it in registers
-// three CTAs fit per SM, and a record load yields the float pairs the packed rotation takes
-// (halves, bf16 [8, 32, 2048, 128]: 54.3 us; 59.2 us with one entry per pair, 69.5 us with
-// the table in registers).
+// The angle table and the lane's weights stay in shared memory as records of two pairs,
+// transposed so that the lanes of a row read consecutive records, and are read per row:
+// with neither in registers four CTAs fit per SM (three for float32), and a record load
+// yields the float pairs the packed rotation takes.  Halves, bf16 [8, 32, 2048, 128]:
+// 51.7 us; 54.3 us with the weights in registers (3 CTAs/SM), 59.2 us with one table
+// entry per pair, 69.5 us with the table in registers (2 CTAs/SM).
 template <typename T, bool TRAD>
 struct PairLayout {
     using E = Elem<T>;
@@ -358,14 +359,15 @@ struct PairLayout {
 };
 
 template <typename T, bool TRAD>
-__global__ void __launch_bounds__(256, 3) rope_pairs_kernel(const RopeArgs a) {
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 4 : 3) rope_pairs_kernel(const RopeArgs a) {
     using E = Elem<T>;
     using PL = PairLayout<T, TRAD>;
     constexpr int NP = PL::NP;
     // rows in flight per lane group (measured best of 2..4 at three CTAs per SM: 2 for
     // bfloat16, 4 for the float32 rows that carry twice the bytes per element)
     constexpr int kUnroll = sizeof(T) == 4 ? 4 : 2;
-    extern __shared__ float4 tab[];  // records: C [half / 2], then S [half / 2]
+    // records: C [half / 2], S [half / 2], then the lanes' weights W [NP][nvec / 2]
+    extern __shared__ float4 tab[];
 
     const int64_t chunk = blockIdx.x % a.n_chunks;
     const int64_t l = blockIdx.x / a.n_chunks;
@@ -398,7 +400,6 @@ __global__ void __launch_bounds__(256, 3) rope_pairs_kernel(const RopeArgs a) {
         }
     }
     const bool norm = a.normalize != 0;
-    float2 wp[NP], wq[NP];
     {
         const V16 wa = (norm && a.w && has_vec)
                            ? ld_param(static_cast<const char*>(a.w) + (size_t)v0 * 16) : ones_vec<T>();
@@ -417,7 +418,12 @@ __global__ void __launch_bounds__(256, 3) rope_pairs_kernel(const RopeArgs a) {
             tabf[(nrec + rec) * 4 + h] = t.z;      // S: sin_hi, sin_lo
             tabf[(nrec + rec) * 4 + 2 + h] = t.w;
         }
+        float2 wp[NP], wq[NP];
         PL::split(wa, wb, wp, wq);
+        if (slot == 0 && has_vec)
+#pragma unroll
+            for (int k = 0; k < NP; ++k)
+                tab[a.half + k * hvec + v0] = make_float4(wp[k].x, wp[k].y, wq[k].x, wq[k].y);
     }
     __syncthreads();
 
@@ -453,8 +459,9 @@ __global__ void __launch_bounds__(256, 3) rope_pairs_kernel(const RopeArgs a) {
                     const float4 c4 = tab[rec], s4 = tab[a.half / 2 + rec];
                     const float2 ch = make_float2(c4.x, c4.y), cl = make_float2(c4.z, c4.w);
                     const float2 sh = make_float2(s4.x, s4.y), sl = make_float2(s4.z, s4.w);
-                    const float2 ap = mul2(p[k], wp[k]);  // exact for bfloat16 data
-                    const float2 aq = mul2(q[k], wq[k]);
+                    const float4 w4 = tab[a.half + k * hvec + v0];
+                    const float2 ap = mul2(p[k], make_float2(w4.x, w4.y));  // exact for bf16 data
+                    const float2 aq = mul2(q[k], make_float2(w4.z, w4.w));
                     yp[k] = mul2(rotate_sub2(ap, aq, ch, cl, sh, sl), inv2);
                     yq[k] = mul2(rotate_pair2(aq, ap, ch, cl, sh, sl), inv2);
                 }
