@@ -402,7 +402,10 @@ nv_status run_layer(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs
         case 1: return go(layer_rows_kernel<T, 1>);
         case 2: return go(layer_rows_kernel<T, 2>);
         case 4: return go(layer_rows_kernel<T, 4>);
-        case 8: return go(layer_rows_kernel<T, 8>);
+        case 8:
+            return block <= 128   ? go(layer_rows_kernel<T, 8, 128>)
+                   : block <= 256 ? go(layer_rows_kernel<T, 8, 256>)
+                                  : go(layer_rows_kernel<T, 8>);
     }
     return fail(NV_ERR_UNSUPPORTED, "vec_per_thread %d", p.vec_per_thread);
 }
