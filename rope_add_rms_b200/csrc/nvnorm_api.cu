@@ -953,9 +953,19 @@ nv_status run_vjp(Op op, VjpArgs a, int vpt, int cap, const DevInfo& di, cudaStr
                               : vpt == 2 ? layer_vjp_kernel<T, 2> : layer_vjp_kernel<T, 4>);
     nv_status st = NV_OK;
     if (a.rows > 0) {
-        const int64_t wave = (int64_t)di.sms * occupancy(k1, G, 0);
+        // VPT = 4 keeps its column partial sums in shared memory (ColAcc)
+        constexpr int NP = Elem<T>::kVec / 2;
+        const size_t smem = vpt < 4 ? 0
+                            : op == OP_RMS ? ColAcc<4, NP, 1>::smem_bytes(G)
+                                           : ColAcc<4, NP, 2>::smem_bytes(G);
+        if (smem > 48 * 1024) {
+            cudaError_t e =
+                cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        }
+        const int64_t wave = (int64_t)di.sms * occupancy(k1, G, smem);
         a.parts = (int)std::min<int64_t>(std::min<int64_t>(a.rows, cap), wave);
-        st = launch_kernel(k1, a.parts, G, 0, s, a);
+        st = launch_kernel(k1, a.parts, G, smem, s, a);
         if (st != NV_OK) return st;
     }
     if (!dw && !db) return st;
