@@ -109,7 +109,9 @@ __device__ __forceinline__ float2 rotate_sub2(float2 a_o, float2 a_t, float2 c_h
 // wholly the q side or wholly past dims, and its partner vector sits hv = half/VEC
 // lanes away (one shuffle per word).  Traditional pairs live inside one vector and need
 // fewer registers: three CTAs per SM (measured 7% faster than two on bf16
-// [8, 32, 2048, 128]; the halves form loses at three, its spills cost more).
+// [8, 32, 2048, 128] with this kernel; the halves form loses at three, its spills cost
+// more).  When every feature is rotated, rope_pairs_kernel below serves both pairings;
+// this kernel takes dims < D and plans that ask for one vector per lane.
 template <typename T, bool TRAD>
 __global__ void __launch_bounds__(256, TRAD ? 3 : 2) rope_rows_kernel(const RopeArgs a) {
     using E = Elem<T>;
