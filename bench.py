@@ -249,6 +249,9 @@ class Case:
             d = {k: (v.clone() if on_dev else v.cuda()) if v is not None else None
                  for k, v in src.items()}
             d["y"] = torch.empty_like(d["r"] if op == "allreduce_add_rms_norm" else d["x"])
+            if op == "norm_rope" and kw.get("y_len"):   # a KV cache [B, H, y_len, D]
+                d["y"] = torch.empty((self.rows // self.L * kw["y_len"], self.D),
+                                     dtype=d["x"].dtype, device="cuda")
             d["h"] = torch.empty_like(d["y"]) if "add_rms_norm" in op else None
             if op.endswith("_vjp"):
                 d["dw"] = torch.empty_like(d["w"])
@@ -289,6 +292,10 @@ class Case:
         elif self.op == "layer_norm_vjp":
             nv.nv_layer_norm_vjp(d["x"], d["w"], d["r"], d["y"], d["dw"], d["db"], k["eps"],
                                  d["ws"], stream)
+        elif k.get("y_len"):
+            nv.nv_rope(d["x"], d["w"], d["y"], self.L, k["dims"], k["traditional"], k["base"],
+                       k["scale"], k["offset"], 1, k["eps"], y_len=k["y_len"], stream=stream,
+                       plan=self.plan)
         else:
             nv.nv_norm_rope(d["x"], d["w"], d["y"], self.L, k["dims"], k["traditional"], k["base"],
                             k["scale"], k["offset"], 1, k["eps"], stream, self.plan)
@@ -558,6 +565,11 @@ WORKLOADS = {
     "norm_rope_traditional": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,
                                           dims=128, traditional=1, base=10000.0, scale=1.0,
                                           offset=4096),
+    # NormRope's cache form: the 2048 new positions of every (b, h) written into a KV cache
+    # of 8192 positions at offset 4096
+    "norm_rope_cache": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,
+                                    dims=128, traditional=0, base=10000.0, scale=1.0,
+                                    offset=4096, y_len=8192),
     "rms_norm_vjp": lambda: Case("rms_norm_vjp", (8192, 4096), "bf16", 0, eps=1e-5),
     "layer_norm_vjp": lambda: Case("layer_norm_vjp", (16384, 8192), "bf16", 0, eps=1e-5),
     # a TP8 decoder's all-reduce + residual add + RMSNorm, the 8 partial outputs already
