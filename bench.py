@@ -559,6 +559,7 @@ def run_ours(args):
 WORKLOADS = {
     "add_rms_norm": lambda: Case("add_rms_norm", (8192, 4096), "bf16", 0, eps=1e-5),
     "rms_norm_small": lambda: Case("rms_norm", (64, 512), "f32", 0, eps=1e-6),
+    "rms_norm": lambda: Case("rms_norm", (8192, 4096), "bf16", 0, eps=1e-5),
     "layer_norm": lambda: Case("layer_norm", (16384, 8192), "bf16", 0, eps=1e-5),
     "norm_rope_halves": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,
                                      dims=128, traditional=0, base=10000.0, scale=1.0, offset=0),
