@@ -12,6 +12,8 @@
 // rounded to the I/O type.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "rms.cuh"
 
@@ -209,43 +211,52 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 256 ? 768 / MAXT : 1)
         const float mu_hi = __double2float_rn(mean);
         const float mu_lo = __double2float_rn(mean - (double)mu_hi);
         const float rf = __double2float_rn(rstd);
-        // d = (x - mean_hi) + nlo: nlo = -mean_lo for rows whose mean is large against
-        // their spread, else +0 (exact); kmu is the matching mean-error term of the test
+        // d = x - mean_hi, and for rows whose mean is large against their spread
+        // (two_sub) also - mean_lo; kmu is the matching mean-error term of the test
         const bool two_sub = 0x1p10f * fabsf(mu_lo) * rf > 0x1p-16f;
         const float kmu = two_sub ? 0x1p-37f * fabsf(mu_hi) : 0x1p10f * fabsf(mu_lo);
         const float2 rf2 = make_float2(rf, rf);
         const float2 nhi2 = make_float2(-mu_hi, -mu_hi);
-        const float nlo = two_sub ? -mu_lo : 0.f;
-        const float2 nlo2 = make_float2(nlo, nlo);
+        const float2 nlo2 = make_float2(-mu_lo, -mu_lo);  // used when two_sub
         // kmu |A| + 2^-11 |b| <= kmu rf wmax + bmax =: tmax for every element of the thread
         const float tmax = __fmaf_rn(__fmul_rn(kmu, rf), wmax, bmax);
 
+        // the output loop, compiled twice: with the second subtraction of the mean
+        // (two_sub) and without it, chosen once per row (CTA-uniform)
+        auto output = [&](auto two) {
+            constexpr bool TWO = decltype(two)::value;
 #pragma unroll
-        for (int k = 0; k < VPT; ++k) {
-            const int v = t + k * G;
-            if (active && v < a.nvec) {
-                if constexpr (!kPRegs) {
-                    wv[k] = a.w ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16) : ones_vec<T>();
-                    bv[k] = a.b ? ld_param(static_cast<const char*>(a.b) + (size_t)v * 16) : zeros_vec<T>();
-                }
-                V16 o;
-                float ymin = INFINITY;
+            for (int k = 0; k < VPT; ++k) {
+                const int v = t + k * G;
+                if (active && v < a.nvec) {
+                    if constexpr (!kPRegs) {
+                        wv[k] = a.w ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16) : ones_vec<T>();
+                        bv[k] = a.b ? ld_param(static_cast<const char*>(a.b) + (size_t)v * 16) : zeros_vec<T>();
+                    }
+                    V16 o;
+                    float ymin = INFINITY;
 #pragma unroll
-                for (int e = 0; e < VEC; e += 2) {
-                    const float2 w2 = E::get2(wv[k], e);
-                    const float2 b2 = E::get2(bv[k], e);
-                    const float2 A2 = mul2(rf2, w2);
-                    const float2 d2 = add2(add2(E::get2(xv[k], e), nhi2), nlo2);
-                    const float2 y2 = fma2(d2, A2, b2);
-                    ymin = fminf(ymin, fminf(fabsf(y2.x), fabsf(y2.y)));
-                    E::put2(o, e, y2);
+                    for (int e = 0; e < VEC; e += 2) {
+                        const float2 w2 = E::get2(wv[k], e);
+                        const float2 b2 = E::get2(bv[k], e);
+                        const float2 A2 = mul2(rf2, w2);
+                        const float2 d2 = TWO ? add2(add2(E::get2(xv[k], e), nhi2), nlo2)
+                                                  : add2(E::get2(xv[k], e), nhi2);
+                        const float2 y2 = fma2(d2, A2, b2);
+                        ymin = fminf(ymin, fminf(fabsf(y2.x), fabsf(y2.y)));
+                        E::put2(o, e, y2);
+                    }
+                    // the vector passes when its smallest |y| clears the thread's bound (a NaN
+                    // y is skipped by fminf and kept: the double form gives NaN too)
+                    if (!(ymin > tmax)) o = layer_vector_f64<T>(xv[k], wv[k], bv[k], mean, rstd);
+                    st_stream(static_cast<char*>(a.y) + roff + (size_t)v * 16, o);
                 }
-                // the vector passes when its smallest |y| clears the thread's bound (a NaN
-                // y is skipped by fminf and kept: the double form gives NaN too)
-                if (!(ymin > tmax)) o = layer_vector_f64<T>(xv[k], wv[k], bv[k], mean, rstd);
-                st_stream(static_cast<char*>(a.y) + roff + (size_t)v * 16, o);
             }
-        }
+        };
+        if (two_sub)
+            output(std::true_type{});
+        else
+            output(std::false_type{});
     }
 }
 
