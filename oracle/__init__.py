@@ -99,6 +99,8 @@ class Oracle:
         lib.oracle_round_bf16.restype = None
         lib.oracle_rms_norm.argtypes = [vp, vp, vp, i64, i64, i64, f32, i32]
         lib.oracle_add_rms_norm.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, f32, i32]
+        f64 = ctypes.c_double
+        lib.oracle_llama3_freqs.argtypes = [i64, f64, f64, f64, f64, f64, vp]
         lib.oracle_allreduce_add_rms_norm.argtypes = [vp, i32, vp, vp, vp, vp, vp, i64, i64, i64,
                                                       f32, i32]
         lib.oracle_layer_norm.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, i32]
@@ -158,6 +160,14 @@ class Oracle:
                                                             _ptr(h), a, b, D, eps, dt),
                   rows, threads)
         return y, h
+
+    def llama3_freqs(self, dims, base, factor, low_freq_factor, high_freq_factor, orig):
+        """Llama 3 NTK-by-parts scaled frequencies theta_i, i < dims/2 (float64)."""
+        out = np.empty(dims // 2, np.float64)
+        if self.lib.oracle_llama3_freqs(dims, base, factor, low_freq_factor, high_freq_factor,
+                                        orig, _ptr(out)) != 0:
+            raise ValueError("arguments outside the Llama 3 scaling's domain")
+        return out
 
     def allreduce_add_rms_norm(self, parts, r, w, eps, threads=None):
         """(y, h, x): x = the sum of the partial tensors (in order, in double) rounded once
@@ -304,6 +314,10 @@ def rms_norm(x, w, eps, threads=None):
 
 def add_rms_norm(x, r, w, eps, threads=None):
     return get().add_rms_norm(x, r, w, eps, threads)
+
+
+def llama3_freqs(dims, base, factor, low_freq_factor, high_freq_factor, orig):
+    return get().llama3_freqs(dims, base, factor, low_freq_factor, high_freq_factor, orig)
 
 
 def allreduce_add_rms_norm(parts, r, w, eps, threads=None):

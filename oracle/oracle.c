@@ -297,6 +297,43 @@ int oracle_norm_rope(const void* x, const void* w, double* y, int64_t r0, int64_
 }
 
 /*
+ * Llama 3 long-context frequency scaling ("NTK-by-parts"): miniVLLM Layers page, section
+ * RotaryEmbedding, constructor parameters llama3_rope_factor, llama3_rope_high_freq_factor,
+ * llama3_rope_low_freq_factor and llama3_rope_original_max_position_embeddings; docs.rs
+ * nuvec-core 0.5.0, Enum FastOp, variant Rope (frequency scaling by mlx-lm's Llama3RoPE).
+ * The pages give the parameters: `factor` scales the low-frequency components; the two
+ * other factors set wavelength thresholds (orig / low_freq_factor and orig / high_freq_factor)
+ * beyond which the scaling is full or absent.  Reading (the pages print no formula): with
+ * theta_i = base^(-2i/dims) and wavelength 2 pi / theta_i,
+ *   wavelength < orig / high_freq_factor  ->  theta_i unchanged            (high frequency)
+ *   wavelength > orig / low_freq_factor   ->  theta_i / factor             (low frequency)
+ *   otherwise, with s = (orig / wavelength - low_freq_factor)
+ *                       / (high_freq_factor - low_freq_factor) in [0, 1],
+ *                                         ->  (1 - s) theta_i / factor + s theta_i
+ * out: dims / 2 doubles.  Returns -1 for arguments outside the reading's domain.
+ */
+int oracle_llama3_freqs(int64_t dims, double base, double factor, double low_freq_factor,
+                        double high_freq_factor, double orig, double* out) {
+    if (dims < 2 || dims % 2 || !(base > 0.0) || !(factor >= 1.0) || !(low_freq_factor > 0.0) ||
+        !(high_freq_factor > low_freq_factor) || !(orig > 0.0))
+        return -1;
+    const double two_pi = 2.0 * acos(-1.0);
+    for (int64_t i = 0; i < dims / 2; ++i) {
+        const double theta = pow(base, -(double)(2 * i) / (double)dims);
+        const double wavelen = two_pi / theta;
+        if (wavelen < orig / high_freq_factor) {
+            out[i] = theta;
+        } else if (wavelen > orig / low_freq_factor) {
+            out[i] = theta / factor;
+        } else {
+            const double s = (orig / wavelen - low_freq_factor) / (high_freq_factor - low_freq_factor);
+            out[i] = (1.0 - s) * theta / factor + s * theta;
+        }
+    }
+    return 0;
+}
+
+/*
  * The general NormRope / Rope (FastOp::NormRope with its cache form, FastOp::Rope with
  * freqs and forward): rows of x [B, H, L, D] (rows = B*H*L) are normalised when
  * normalize != 0 and rotated at position offset + l (by -phi when forward == 0), with

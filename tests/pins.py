@@ -185,6 +185,37 @@ def check_allreduce_hand_case(o):
     assert (x1 == p).all() and (h1 == h2).all() and (y1 == y2).all()
 
 
+# ---- Llama 3 frequency scaling (reading of the pages' four parameters) ----------------
+
+def check_llama3_freqs_regions(o):
+    """factor 1 changes nothing; wavelengths below orig/high keep theta exactly, those above
+    orig/low get exactly theta/factor, the band between lies strictly between the two; the
+    scaled frequencies fall strictly with i (the blend joins both ends continuously)."""
+    dims, base = 128, 500000.0
+    theta = np.array([base ** (-2.0 * i / dims) for i in range(dims // 2)])
+    # (1 - s) theta + s theta rounds to within an ulp or two of theta in the band
+    _close(o.llama3_freqs(dims, base, 1.0, 1.0, 4.0, 8192.0), theta, 1e-15, what="factor 1")
+    for factor, low, high, orig in ((32.0, 1.0, 4.0, 8192.0), (8.0, 2.0, 16.0, 4096.0)):
+        f = o.llama3_freqs(dims, base, factor, low, high, orig)
+        lam = 2 * math.pi / theta
+        hi, lo = lam < orig / high, lam > orig / low
+        mid = ~(hi | lo)
+        assert (f[hi] == theta[hi]).all(), "high frequencies must be unchanged"
+        assert (f[lo] == theta[lo] / factor).all(), "low frequencies must be divided by factor"
+        assert hi.any() and lo.any() and mid.any()
+        assert ((f[mid] < theta[mid]) & (f[mid] > theta[mid] / factor)).all()
+        assert (np.diff(f) < 0).all(), "scaled frequencies must fall strictly with i"
+
+
+def check_llama3_freqs_hand_case(o):
+    """dims 4, base 16: theta = [1, 1/4], wavelengths [2 pi, 8 pi]; orig 16 pi, low 1,
+    high 4: thresholds 4 pi and 16 pi, so theta_0 stays and theta_1 sits in the band at
+    orig / wavelength = 2, s = 1/3: (2/3)(1/4)/8 + (1/3)(1/4) = 5/48 with factor 8."""
+    f = o.llama3_freqs(4, 16.0, 8.0, 1.0, 4.0, 16 * math.pi)
+    assert f[0] == 1.0
+    assert abs(f[1] - 5.0 / 48.0) < 1e-15, f[1]
+
+
 # ---- rms_norm -------------------------------------------------------------------------
 
 def check_rms_constant_rows(o):

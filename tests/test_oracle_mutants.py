@@ -30,6 +30,14 @@ MUTANTS = {
                                           "((uint16_t*)xb)[o] = oracle_bf16_from_f64((double)(float)s);"),
     "allreduce_skips_residual": ("int rc = oracle_add_rms_norm(xb, (const char*)r + off * esz,",
                                  "int rc = oracle_add_rms_norm(xb, (const char*)xb,"),
+    "llama3_thresholds_swapped": ("if (wavelen < orig / high_freq_factor) {",
+                                  "if (wavelen < orig / low_freq_factor) {"),
+    "llama3_ramp_reversed": ("const double s = (orig / wavelen - low_freq_factor) / (high_freq_factor - low_freq_factor);",
+                             "const double s = (high_freq_factor - orig / wavelen) / (high_freq_factor - low_freq_factor);"),
+    "llama3_multiplies_by_factor": ("            out[i] = theta / factor;\n",
+                                    "            out[i] = theta * factor;\n"),
+    "llama3_theta_over_dims_half": ("const double theta = pow(base, -(double)(2 * i) / (double)dims);",
+                                    "const double theta = pow(base, -(double)i / (double)dims);"),
     "layer_unbiased_variance": ("double var = sqdev / (double)D;",
                                 "double var = sqdev / (double)(D - 1);"),
     "layer_drops_mean_in_output": ("y[j] = (x[j] - mean) / denom * wj + bj;",
