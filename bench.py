@@ -260,6 +260,9 @@ class Case:
                     op[:-4], rows, D)), dtype=torch.uint8, device="cuda")
             self.sets.append(d)
         self.nv = nv
+        # explicit frequencies (the Llama 3 scaling) for the general rope call
+        self.freqs = (nv.rope_llama3_freqs(self.D).cuda() if op == "norm_rope" and kw.get("llama3")
+                      else None)
         n_out = 2 if op == "add_rms_norm" else 1
         self.host_out = [] if on_dev or "x" not in self.host else \
             [torch.empty_like(self.host["x"]).pin_memory() for _ in range(n_out)]
@@ -292,10 +295,10 @@ class Case:
         elif self.op == "layer_norm_vjp":
             nv.nv_layer_norm_vjp(d["x"], d["w"], d["r"], d["y"], d["dw"], d["db"], k["eps"],
                                  d["ws"], stream)
-        elif k.get("y_len"):
+        elif k.get("y_len") or self.freqs is not None:
             nv.nv_rope(d["x"], d["w"], d["y"], self.L, k["dims"], k["traditional"], k["base"],
-                       k["scale"], k["offset"], 1, k["eps"], y_len=k["y_len"], stream=stream,
-                       plan=self.plan)
+                       k["scale"], k["offset"], 1, k["eps"], freqs=self.freqs,
+                       y_len=k.get("y_len", 0), stream=stream, plan=self.plan)
         else:
             nv.nv_norm_rope(d["x"], d["w"], d["y"], self.L, k["dims"], k["traditional"], k["base"],
                             k["scale"], k["offset"], 1, k["eps"], stream, self.plan)
@@ -571,6 +574,10 @@ WORKLOADS = {
     "norm_rope_cache": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,
                                     dims=128, traditional=0, base=10000.0, scale=1.0,
                                     offset=4096, y_len=8192),
+    # NormRope with the Llama 3 scaled frequencies (base 500000), past the original context
+    "norm_rope_llama3": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-5,
+                                     dims=128, traditional=0, base=500000.0, scale=1.0,
+                                     offset=16384, llama3=True),
     "rms_norm_vjp": lambda: Case("rms_norm_vjp", (8192, 4096), "bf16", 0, eps=1e-5),
     "layer_norm_vjp": lambda: Case("layer_norm_vjp", (16384, 8192), "bf16", 0, eps=1e-5),
     # a TP8 decoder's all-reduce + residual add + RMSNorm, the 8 partial outputs already

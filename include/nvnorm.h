@@ -167,6 +167,26 @@ NV_API nv_status nv_layer_norm_vjp(const void* x, const void* w, const void* g, 
 NV_API size_t nv_norm_vjp_workspace_size(int32_t op, int64_t rows, int64_t D);
 
 /*
+ * rope_llama3_freqs -- the Llama 3 long-context frequency scaling ("NTK-by-parts") for
+ * nv_rope's `freqs`: miniVLLM Layers page, section RotaryEmbedding, parameters
+ * llama3_rope_factor (scales the low-frequency components), llama3_rope_low_freq_factor and
+ * llama3_rope_high_freq_factor (wavelength thresholds original_max_position / factor) and
+ * llama3_rope_original_max_position_embeddings; docs.rs nuvec-core 0.5.0, Enum FastOp,
+ * variant Rope (frequency scaling by Llama3RoPE).  The pages print no formula; read as:
+ * with theta_i = base^(-2i/dims) and wavelength 2 pi / theta_i, wavelengths below
+ * original_max_position / high_freq_factor keep theta_i, those above
+ * original_max_position / low_freq_factor get theta_i / factor, and between them
+ * (1 - s) theta_i / factor + s theta_i with s = (original_max_position / wavelength -
+ * low_freq_factor) / (high_freq_factor - low_freq_factor).  Computed in double on the host,
+ * rounded once: freqs [dims / 2] is HOST memory (copy it to the device for nv_rope).
+ * Needs dims even >= 2, base > 0, factor >= 1, 0 < low_freq_factor < high_freq_factor,
+ * original_max_position > 0 (else NV_ERR_INVALID_ARG).  Needs no GPU.
+ */
+NV_API nv_status nv_rope_llama3_freqs(int32_t dims, float base, float factor,
+                                      float low_freq_factor, float high_freq_factor,
+                                      int64_t original_max_position, float* freqs);
+
+/*
  * allreduce_add_rms_norm -- the step a tensor-parallel decoder takes after a row-parallel
  * layer: miniVLLM Layers page, section Linear layers, RowParallelLinear (the forward pass
  * sums the ranks' partial outputs with an all_reduce), then the fused residual add +

@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "NvError", "Plan", "library", "library_path",
     "nv_rms_norm", "nv_add_rms_norm", "nv_add_rms_norm_host", "nv_allreduce_add_rms_norm",
-    "allreduce_add_rms_norm", "nv_layer_norm", "nv_norm_rope",
+    "allreduce_add_rms_norm", "rope_llama3_freqs", "nv_layer_norm", "nv_norm_rope",
     "nv_describe_plan",
     "nv_fault_count",
     "nv_rope", "rms_norm", "add_rms_norm", "layer_norm", "norm_rope", "norm_rope_into_cache",
@@ -109,6 +109,8 @@ def library() -> ctypes.CDLL:
     lib.nv_rms_norm_vjp.restype = ctypes.c_int
     lib.nv_layer_norm_vjp.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, i64, i64, f32, i32, vp]
     lib.nv_layer_norm_vjp.restype = ctypes.c_int
+    lib.nv_rope_llama3_freqs.argtypes = [i32, f32, f32, f32, f32, i64, vp]
+    lib.nv_rope_llama3_freqs.restype = ctypes.c_int
     lib.nv_norm_vjp_workspace_size.argtypes = [i32, i64, i64]
     lib.nv_norm_vjp_workspace_size.restype = sz
     _lib = lib
@@ -194,6 +196,17 @@ def nv_add_rms_norm_host(x_host, r_host, w, y_host, h_host, x_dev, r_dev, y_dev,
                                   _dtype(x_host, r_host, w, y_host, h_host, x_dev, r_dev,
                                          y_dev, h_dev), chunk_rows, _stream(stream))
     _check("nv_add_rms_norm_host", st)
+
+
+def rope_llama3_freqs(dims, base=500000.0, factor=32.0, low_freq_factor=1.0,
+                      high_freq_factor=4.0, original_max_position=8192):
+    """Llama 3 scaled RoPE frequencies theta_i (i < dims/2) as a float32 host tensor, for
+    ``nv_rope(..., freqs=...)`` after ``.cuda()``."""
+    out = torch.empty(dims // 2, dtype=torch.float32)
+    st = library().nv_rope_llama3_freqs(dims, base, factor, low_freq_factor, high_freq_factor,
+                                        original_max_position, ctypes.c_void_p(out.data_ptr()))
+    _check("nv_rope_llama3_freqs", st)
+    return out
 
 
 def nv_allreduce_add_rms_norm(parts, r, w, y, h, eps, x_out=None, stream=None):

@@ -1218,6 +1218,45 @@ nv_status nv_describe_plan(int32_t op, int64_t rows, int64_t D, nv_dtype dt, nv_
     return make_plan((Op)op, rows, D, dt, true, nullptr, plan);
 }
 
+nv_status nv_rope_llama3_freqs(int32_t dims, float base, float factor, float low_freq_factor,
+                               float high_freq_factor, int64_t original_max_position,
+                               float* freqs) {
+    if (dims < 2 || dims % 2 != 0)
+        return fail(NV_ERR_INVALID_ARG, "dims = %d must be even and >= 2", dims);
+    if (!(base > 0.f) || !std::isfinite(base))
+        return fail(NV_ERR_INVALID_ARG, "base = %g must be finite and > 0", (double)base);
+    if (!(factor >= 1.f) || !std::isfinite(factor))
+        return fail(NV_ERR_INVALID_ARG, "factor = %g must be finite and >= 1", (double)factor);
+    if (!(low_freq_factor > 0.f) || !(high_freq_factor > low_freq_factor) ||
+        !std::isfinite(high_freq_factor))
+        return fail(NV_ERR_INVALID_ARG, "need 0 < low_freq_factor (%g) < high_freq_factor (%g)",
+                    (double)low_freq_factor, (double)high_freq_factor);
+    if (original_max_position <= 0)
+        return fail(NV_ERR_INVALID_ARG, "original_max_position = %lld must be > 0",
+                    (long long)original_max_position);
+    if (!freqs) return fail(NV_ERR_INVALID_ARG, "freqs is NULL");
+    const double orig = (double)original_max_position, f = factor;
+    const double short_wave = orig / high_freq_factor;  // shorter: unchanged
+    const double long_wave = orig / low_freq_factor;    // longer: divided by factor
+    const double pi2 = 2.0 * 3.14159265358979323846;
+    for (int32_t i = 0; i < dims / 2; ++i) {
+        const double th = std::pow((double)base, -2.0 * (double)i / (double)dims);
+        const double lambda = pi2 / th;
+        double out;
+        if (lambda < short_wave) {
+            out = th;
+        } else if (lambda > long_wave) {
+            out = th / f;
+        } else {  // blend linearly in orig / lambda between the two thresholds
+            const double t = (orig / lambda - low_freq_factor) /
+                             ((double)high_freq_factor - (double)low_freq_factor);
+            out = (1.0 - t) * (th / f) + t * th;
+        }
+        freqs[i] = (float)out;
+    }
+    return NV_OK;
+}
+
 nv_status nv_allreduce_add_rms_norm(const void* const* parts, int32_t nparts, const void* r,
                                     const void* w, void* y, void* h, void* x_out, int64_t rows,
                                     int64_t D, float eps, nv_dtype dt, nv_stream_t stream) {

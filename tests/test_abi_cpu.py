@@ -212,3 +212,31 @@ def test_vjp_workspace_size():
     # narrow rows keep more partial sums (up to 2^21 / D of them)
     assert lib.nv_norm_vjp_workspace_size(0, 100000, 512) == 4096 * 512 * 4
     assert lib.nv_norm_vjp_workspace_size(2, 100000, 16384) == 2 * 512 * 16384 * 4
+
+
+# ---- Llama 3 frequency scaling: a host-side helper, testable without a GPU ------------------
+
+@pytest.mark.parametrize("args", [(128, 500000.0, 32.0, 1.0, 4.0, 8192),
+                                  (64, 10000.0, 8.0, 2.0, 16.0, 4096),
+                                  (256, 1000000.0, 16.0, 1.0, 8.0, 131072),
+                                  (4, 16.0, 8.0, 1.0, 4.0, 50), (128, 500000.0, 1.0, 1.0, 4.0, 8192)])
+def test_rope_llama3_freqs_matches_the_oracle(args):
+    import numpy as np
+    import oracle
+    got = nv.rope_llama3_freqs(*args).numpy()
+    want = oracle.llama3_freqs(args[0], args[1], args[2], args[3], args[4],
+                               float(args[5])).astype(np.float32)
+    ulps = np.abs(got.view(np.int32).astype(np.int64) - want.view(np.int32).astype(np.int64))
+    assert ulps.max() <= 1, f"{int(ulps.max())} float ulps apart"
+
+
+@pytest.mark.parametrize("kw, words", [
+    (dict(dims=7), "dims"), (dict(dims=0), "dims"), (dict(base=0.0), "base"),
+    (dict(factor=0.5), "factor"), (dict(low_freq_factor=4.0, high_freq_factor=4.0), "low_freq"),
+    (dict(original_max_position=0), "original_max_position")])
+def test_rope_llama3_freqs_rejects(kw, words):
+    args = dict(dims=128, base=500000.0, factor=32.0, low_freq_factor=1.0, high_freq_factor=4.0,
+                original_max_position=8192)
+    args.update(kw)
+    with pytest.raises(nv.NvError, match=words):
+        nv.rope_llama3_freqs(**args)

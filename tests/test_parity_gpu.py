@@ -680,6 +680,23 @@ def test_rope_freqs_and_inverse(plan, trad, dt):
                 check_out(y, ref, f"normalize={normalize} forward={forward} freqs={f is not None}")
 
 
+@pytest.mark.parametrize("trad", [0, 1])
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_rope_llama3_scaled_frequencies(trad, dt):
+    """NormRope with the Llama 3 scaled frequencies at positions past the original context."""
+    B, H, L, D = 2, 4, 64, 128
+    inp = synth.norm_rope_inputs(B, H, L, D, dt, seed=41)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    freqs = nv.rope_llama3_freqs(D, 500000.0, 32.0, 1.0, 4.0, 8192)
+    for offset in (0, 20000):
+        y = torch.empty_like(x)
+        nv.nv_rope(x, w, y, L, D, trad, 500000.0, 1.0, offset, 1, 1e-5, freqs=freqs.cuda())
+        torch.cuda.synchronize()
+        ref = oracle.rope_ex(host(inp["x"]), host(inp["w"]), L, D, trad, 500000.0, 1.0, offset, 1,
+                             1e-5, freqs=freqs.numpy().astype(np.float64))
+        check_out(y, ref, f"offset {offset}")
+
+
 def test_rope_round_trip_and_cache_rules():
     B, H, L, D = 1, 2, 8, 64
     x = synth.normal((B * H * L, D), 0.0, 1.0, 33, 0, "f32").cuda()
