@@ -545,7 +545,7 @@ def run_ours(args):
                     "d2h_bytes_per_step": bo,
                     "ms_per_step": round(e2e_ms / e2e_steps, 4), "steps": e2e_steps,
                     "how": "nv_add_rms_norm_host: pinned host x, r -> device, add_rms_norm, "
-                           "y, h -> pinned host, pipelined over 8 row chunks on 3 streams; "
+                           "y, h -> pinned host, 8 row chunks through copy-in/compute/copy-out streams; "
                            "events on the caller's stream around each step"},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),

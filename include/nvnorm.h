@@ -213,8 +213,9 @@ NV_API nv_status nv_allreduce_add_rms_norm(const void* const* parts, int32_t npa
 /*
  * add_rms_norm_host -- add_rms_norm (as nv_add_rms_norm) on rows that live in host
  * memory: x and r are copied in, the op runs, y and h are copied back, pipelined over
- * chunks of chunk_rows rows (0 = about eight chunks) on internal streams so that copies in
- * and out and the compute of different chunks overlap.
+ * chunks of chunk_rows rows (0 = about eight chunks, at most 64) through three internal
+ * streams -- copies in, compute, copies out, linked per chunk by events -- so that copies
+ * in and out and the compute of different chunks overlap.
  * x_host, r_host [rows, D] in, y_host, h_host [rows, D] out: page-locked host memory
  * (cudaHostAlloc / cudaHostRegister); y_host may be x_host and h_host may be r_host, other
  * host buffers may not overlap.  x_dev, r_dev, y_dev, h_dev [rows, D]: device buffers of

@@ -755,18 +755,22 @@ nv_status allreduce_add_rms_norm(const void* const* parts, int32_t nparts, const
 }
 
 // ---- host-resident rows: copies and compute pipelined over row chunks ---------------------
-// Chunk k goes to internal stream k % kPipeStreams: host -> device copies of its x and r
-// rows, the add_rms_norm launch on those rows, device -> host copies of its y and h.  The
-// copy engines move chunk k + 1 in while chunk k - 1 moves out, so the PCIe link runs in
-// both directions at once.  The internal streams start after the work already queued on
-// the caller's stream and the caller's stream waits for all of them, so the call is
-// ordered like any other launch on `stream`.
-constexpr int kPipeStreams = 3;
+// A three-stage pipeline over row chunks, one internal stream per stage: stream IN copies
+// chunk after chunk of x and r to the device, stream COMPUTE runs add_rms_norm on chunk k
+// once IN has recorded it, stream OUT copies chunk k's y and h back once COMPUTE has
+// recorded it.  No stage waits on a later one, so uploads run back to back while the
+// downloads of earlier chunks proceed: the PCIe link works in both directions at once.
+// The stages start after the work already queued on the caller's stream and the caller's
+// stream waits for all of them, so the call is ordered like any other launch on `stream`.
+constexpr int kPipeStreams = 3;  // IN, COMPUTE, OUT
+constexpr int kPipeMaxChunks = 64;
 
 struct Pipe {
     cudaStream_t s[kPipeStreams] = {};
     cudaEvent_t start = nullptr;
     cudaEvent_t done[kPipeStreams] = {};
+    cudaEvent_t in[kPipeMaxChunks] = {};    // chunk k is on the device
+    cudaEvent_t comp[kPipeMaxChunks] = {};  // chunk k's outputs are written
 };
 Pipe g_pipe[kMaxDevices];
 std::mutex g_pipe_mu;  // guards creation and the enqueue sequence (events are reused)
@@ -778,6 +782,10 @@ nv_status pipe_for(int dev, Pipe** out) {
         for (int i = 0; e == cudaSuccess && i < kPipeStreams; ++i) {
             e = cudaStreamCreateWithFlags(&pp.s[i], cudaStreamNonBlocking);
             if (e == cudaSuccess) e = cudaEventCreateWithFlags(&pp.done[i], cudaEventDisableTiming);
+        }
+        for (int k = 0; e == cudaSuccess && k < kPipeMaxChunks; ++k) {
+            e = cudaEventCreateWithFlags(&pp.in[k], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&pp.comp[k], cudaEventDisableTiming);
         }
         if (e != cudaSuccess) {
             pp = Pipe{};  // a later call retries; objects made so far are left to the context
@@ -856,8 +864,9 @@ nv_status add_rms_norm_host(const void* x_host, const void* r_host, const void* 
     };
     st = check_buffers(bufs, 5, dev);
     if (st != NV_OK) return st;
-    const int64_t chunk =
+    int64_t chunk =
         chunk_rows > 0 ? chunk_rows : std::max<int64_t>(1, (rows + 7) / 8);  // ~8 chunks
+    chunk = std::max(chunk, (rows + kPipeMaxChunks - 1) / kPipeMaxChunks);  // <= 64 chunks
     const int64_t row_bytes = D * (int64_t)s;
     bool al = aligned16(x_dev) && aligned16(r_dev) && aligned16(y_dev) && aligned16(h_dev) &&
               (!w || aligned16(w)) && (chunk * row_bytes) % 16 == 0;
@@ -876,17 +885,19 @@ nv_status add_rms_norm_host(const void* x_host, const void* r_host, const void* 
         e = cudaStreamWaitEvent(pp->s[i], pp->start, 0);
     if (e != cudaSuccess) return cuda_fail(e, "pipeline start");
     const int64_t nchunks = (rows + chunk - 1) / chunk;
+    cudaStream_t s_in = pp->s[0], s_comp = pp->s[1], s_out = pp->s[2];
     for (int64_t k = 0; k < nchunks; ++k) {
-        cudaStream_t sk = pp->s[k % kPipeStreams];
         const int64_t r0 = k * chunk, n = std::min(chunk, rows - r0);
         const size_t off = (size_t)r0 * (size_t)row_bytes, len = (size_t)n * (size_t)row_bytes;
         auto at = [off](const void* base) {
             return static_cast<char*>(const_cast<void*>(base)) + off;
         };
-        e = cudaMemcpyAsync(at(x_dev), at(x_host), len, cudaMemcpyHostToDevice, sk);
+        e = cudaMemcpyAsync(at(x_dev), at(x_host), len, cudaMemcpyHostToDevice, s_in);
         if (e == cudaSuccess)
-            e = cudaMemcpyAsync(at(r_dev), at(r_host), len, cudaMemcpyHostToDevice, sk);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (host to device)");
+            e = cudaMemcpyAsync(at(r_dev), at(r_host), len, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess) e = cudaEventRecord(pp->in[k], s_in);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_comp, pp->in[k], 0);
+        if (e != cudaSuccess) return cuda_fail(e, "pipeline: copy in");
         RowArgs a{};
         a.x = at(x_dev);
         a.r = at(r_dev);
@@ -897,12 +908,15 @@ nv_status add_rms_norm_host(const void* x_host, const void* r_host, const void* 
         a.D = (int)D;
         a.nvec = (int)(row_bytes / 16);
         a.eps = eps;
-        st = row_dispatch(OP_ADD, p, di, dt, sk, a);
+        st = row_dispatch(OP_ADD, p, di, dt, s_comp, a);
         if (st != NV_OK) return st;
-        e = cudaMemcpyAsync(at(y_host), at(y_dev), len, cudaMemcpyDeviceToHost, sk);
+        e = cudaEventRecord(pp->comp[k], s_comp);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, pp->comp[k], 0);
         if (e == cudaSuccess)
-            e = cudaMemcpyAsync(at(h_host), at(h_dev), len, cudaMemcpyDeviceToHost, sk);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (device to host)");
+            e = cudaMemcpyAsync(at(y_host), at(y_dev), len, cudaMemcpyDeviceToHost, s_out);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(at(h_host), at(h_dev), len, cudaMemcpyDeviceToHost, s_out);
+        if (e != cudaSuccess) return cuda_fail(e, "pipeline: copy out");
     }
     for (int i = 0; e == cudaSuccess && i < kPipeStreams; ++i) {
         e = cudaEventRecord(pp->done[i], pp->s[i]);
