@@ -775,6 +775,28 @@ def test_layer_norm_vjp_large_mean(dt, mean, std):
     check_grad(db, ref[2], ref[5], "db")
 
 
+@pytest.mark.parametrize("dt,D", [("bf16", 1024), ("bf16", 4096), ("bf16", 16384), ("f32", 512),
+                                  ("f32", 4096), ("f32", 8192)])
+def test_layer_norm_vjp_rows_starting_far_from_their_mean(dt, D):
+    """Rows whose leading elements sit far from the row mean (1000, 2.5 or 3.0 followed by
+    N(0, 1) values), plain N(0, 1) rows and constant rows (variance 0), mixed within one
+    CTA's rows: statistics that lean on a row's first elements, or on E[x^2] - mean^2,
+    lose precision exactly here."""
+    rows = 64
+    x = synth.normal((rows, D), 0.0, 1.0, 43, 0, dt)
+    for i, v in enumerate((1000.0, 2.5, 3.0)):
+        x[i::5, :2] = v
+    x[4::5] = 7.0
+    w = synth.normal((D,), 1.0, 0.1, 43, 2, dt)
+    g = synth.normal((rows, D), 0.0, 1.0, 43, 4, dt)
+    dx, dw, db = nv.layer_norm_vjp(dev(x), dev(w), dev(g), eps=1e-5)
+    torch.cuda.synchronize()
+    ref = oracle.layer_norm_vjp(host(x), host(w), host(g), 1e-5)
+    check_grad(dx, ref[0], ref[3], "dx")
+    check_grad(dw, ref[1], ref[4], "dw")
+    check_grad(db, ref[2], ref[5], "db")
+
+
 @pytest.mark.parametrize("rows,D", [(20000, 512), (5000, 64), (3001, 1024)])
 def test_vjp_many_narrow_rows(rows, D):
     # more rows than partial sums: every CTA walks many rows
