@@ -276,6 +276,17 @@ NV_API int32_t nv_version(void);
 NV_API nv_status nv_fault_count(uint32_t* count, int32_t reset);
 
 /*
+ * Check of the failure path of those bounded waits, for tests: launches `ctas` CTAs of
+ * 32 threads on `stream`, each waiting on an mbarrier that nothing ever completes (no
+ * copy is issued).  Every wait gives up after about one second and each CTA counts one
+ * fault, so nv_fault_count then reports `ctas` more; nothing else is touched and the
+ * context stays usable.  Takes about a second of GPU time.
+ * ctas: 1..64.  Errors: NV_ERR_INVALID_ARG outside that range (nothing launched);
+ * NV_ERR_CUDA on a launch error.
+ */
+NV_API nv_status nv_selftest_bounded_wait(int32_t ctas, nv_stream_t stream);
+
+/*
  * Kernel-variant control, for tests and benchmarks.  The plain entry points above
  * pick a variant from (op, dtype, D, rows, alignment); the *_ex forms take a plan
  * that forces one.  A plan that the shape cannot use returns NV_ERR_UNSUPPORTED.

@@ -21,7 +21,7 @@ __all__ = [
     "nv_rms_norm", "nv_add_rms_norm", "nv_add_rms_norm_host", "nv_allreduce_add_rms_norm",
     "allreduce_add_rms_norm", "rope_llama3_freqs", "nv_layer_norm", "nv_norm_rope",
     "nv_describe_plan",
-    "nv_fault_count",
+    "nv_fault_count", "nv_selftest_bounded_wait",
     "nv_rope", "rms_norm", "add_rms_norm", "layer_norm", "norm_rope", "norm_rope_into_cache",
     "rope", "nv_rms_norm_vjp", "nv_layer_norm_vjp", "nv_norm_vjp_workspace_size", "rms_norm_vjp",
     "layer_norm_vjp",
@@ -104,6 +104,8 @@ def library() -> ctypes.CDLL:
     lib.nv_version.restype = ctypes.c_int32
     lib.nv_fault_count.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]
     lib.nv_fault_count.restype = ctypes.c_int
+    lib.nv_selftest_bounded_wait.argtypes = [ctypes.c_int32, ctypes.c_void_p]
+    lib.nv_selftest_bounded_wait.restype = ctypes.c_int
     sz = ctypes.c_size_t
     lib.nv_rms_norm_vjp.argtypes = [vp, vp, vp, vp, vp, vp, sz, i64, i64, f32, i32, vp]
     lib.nv_rms_norm_vjp.restype = ctypes.c_int
@@ -275,6 +277,12 @@ def nv_fault_count(reset: bool = False) -> int:
     c = ctypes.c_uint32(0)
     _check("nv_fault_count", library().nv_fault_count(ctypes.byref(c), int(bool(reset))))
     return c.value
+
+
+def nv_selftest_bounded_wait(ctas: int = 1, stream=None):
+    """Launch `ctas` CTAs whose device-side bounded waits run out (about one second);
+    each counts one fault in nv_fault_count.  A check of the failure path."""
+    _check("nv_selftest_bounded_wait", library().nv_selftest_bounded_wait(int(ctas), _stream(stream)))
 
 
 def nv_norm_vjp_workspace_size(op: str, rows: int, D: int) -> int:

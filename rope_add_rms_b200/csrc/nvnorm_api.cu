@@ -27,6 +27,7 @@ namespace {
 using namespace nvn;
 
 constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxSelftestCtas = 64;  // nv_selftest_bounded_wait: one resident wave
 
 // ---- error reporting ------------------------------------------------------------------
 thread_local char g_msg[512] = "";
@@ -1331,6 +1332,15 @@ nv_status nv_fault_count(uint32_t* count, int32_t reset) {
         e = cudaMemcpyToSymbol(nvn::nvn_fault_count, &zero, sizeof(uint32_t));
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
     }
+    return NV_OK;
+}
+
+nv_status nv_selftest_bounded_wait(int32_t ctas, nv_stream_t stream) {
+    if (ctas < 1 || ctas > kMaxSelftestCtas)
+        return fail(NV_ERR_INVALID_ARG, "ctas = %d outside 1..%d", ctas, kMaxSelftestCtas);
+    bounded_wait_selftest_kernel<<<ctas, 32, 0, (cudaStream_t)stream>>>();
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "bounded_wait_selftest_kernel launch");
     return NV_OK;
 }
 

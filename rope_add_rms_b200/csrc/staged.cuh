@@ -88,6 +88,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     return false;
 }
 
+// Check of the bounded wait itself: each CTA waits on an mbarrier that nothing arrives on
+// (its first phase never completes), so every thread gives up after ~kWaitLimitNs, and
+// the CTA counts one fault, as a staged kernel does when its copies never land.  No copy
+// is in flight, so the CTA may leave at once.
+__global__ void __launch_bounds__(32) bounded_wait_selftest_kernel() {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_addr(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const bool ok = mbar_wait_bounded(b, 0);
+    if (__syncthreads_count(ok ? 0 : 1) > 0 && threadIdx.x == 0) atomicAdd(&nvn_fault_count, 1u);
+}
+
 __device__ __forceinline__ V16 ld_shared16(const unsigned char* p) {
     const uint4 t = *reinterpret_cast<const uint4*>(p);
     return V16{{t.x, t.y, t.z, t.w}};

@@ -158,6 +158,8 @@ def last_error():
     (lambda: allreduce(dt=F16), UNSUPPORTED, "F16"),
     (lambda: host_add(x=None), INVALID, "x_host is NULL"),
     (lambda: host_add(h=FAKE), INVALID, "same buffer"),
+    (lambda: nv.library().nv_selftest_bounded_wait(0, None), INVALID, "ctas"),
+    (lambda: nv.library().nv_selftest_bounded_wait(65, None), INVALID, "ctas"),
     (lambda: host_add(chunk=-1), INVALID, "chunk_rows"),
 ])
 def test_invalid_arguments_are_rejected_on_the_host(call, status, words):

@@ -836,3 +836,21 @@ def test_vjp_deterministic_in_place_and_empty():
     nv.nv_layer_norm_vjp(empty, None, empty, empty, None, db0, 1e-5)
     torch.cuda.synchronize()
     assert (dw0 == 0).all() and (db0 == 0).all(), "an empty batch has zero column gradients"
+
+
+def test_bounded_wait_runs_out_is_counted_and_leaves_the_context_usable():
+    """The failure path of the device-side bounded waits: waits on an mbarrier that nothing
+    completes give up after about a second, each CTA counts one fault, the host reads the
+    count, and the next kernels run normally."""
+    import time
+    nv.nv_fault_count(reset=True)
+    t0 = time.monotonic()
+    nv.nv_selftest_bounded_wait(3)
+    assert nv.nv_fault_count(reset=True) == 3
+    assert 0.5 < time.monotonic() - t0 < 60
+    inp = synth.rms_inputs(64, 512, "f32", seed=5)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    y = nv.rms_norm(x, w, eps=1e-6)
+    torch.cuda.synchronize()
+    check_out(y, oracle.rms_norm(host(inp["x"]), host(inp["w"]), 1e-6), "after the timed-out waits")
+    assert nv.nv_fault_count() == 0
