@@ -120,7 +120,6 @@ __global__ void __launch_bounds__(512) rms_staged_kernel(const RowArgs a, const 
     constexpr int NT = ADD ? 2 : 1;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ float red[2][32];
-    __shared__ int abort_flag;
 
     const int G = blockDim.x;
     const int t = threadIdx.x;
@@ -134,7 +133,6 @@ __global__ void __launch_bounds__(512) rms_staged_kernel(const RowArgs a, const 
     const int64_t nmine = first < a.rows ? (a.rows - 1 - first) / stride + 1 : 0;
 
     if (t == 0) {
-        abort_flag = 0;
         for (int s = 0; s < stages; ++s) mbar_init(bbase + 8u * s, 1);
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -172,7 +170,7 @@ __global__ void __launch_bounds__(512) rms_staged_kernel(const RowArgs a, const 
     for (; k < nmine; ++k) {
         const int s = (int)(k % stages);
         const uint32_t parity = (uint32_t)((k / stages) & 1);
-        if (!mbar_wait_bounded(bbase + 8u * s, parity)) abort_flag = 1;
+        const bool bad = !mbar_wait_bounded(bbase + 8u * s, parity);
         const int64_t row = first + k * stride;
         const size_t roff = (size_t)row * row_bytes;
         const unsigned char* stg = smem + (size_t)s * stage_bytes;
@@ -211,8 +209,8 @@ __global__ void __launch_bounds__(512) rms_staged_kernel(const RowArgs a, const 
         ss = warp_sum(ss);
         float* buf = red[k & 1];
         if ((t & 31) == 0) buf[t >> 5] = ss;
-        __syncthreads();  // every thread has consumed stage s; abort_flag is settled
-        if (abort_flag) break;
+        // every thread has consumed stage s; a wait that ran out anywhere stops every thread
+        if (__syncthreads_or(bad ? 1 : 0)) break;
         if (t == 0 && k + stages < nmine) {
             fence_proxy_async_smem();
             issue(k + stages);
@@ -268,7 +266,6 @@ __global__ void __launch_bounds__(512) layer_staged_kernel(const RowArgs a, cons
     constexpr int VEC = E::kVec;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ double red[2][3][16];
-    __shared__ int abort_flag;
 
     const int G = blockDim.x;
     const int t = threadIdx.x;
@@ -281,7 +278,6 @@ __global__ void __launch_bounds__(512) layer_staged_kernel(const RowArgs a, cons
     const int64_t nmine = first < a.rows ? (a.rows - 1 - first) / stride + 1 : 0;
 
     if (t == 0) {
-        abort_flag = 0;
         for (int s = 0; s < stages; ++s) mbar_init(bbase + 8u * s, 1);
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -322,7 +318,7 @@ __global__ void __launch_bounds__(512) layer_staged_kernel(const RowArgs a, cons
     int64_t k = 0;
     for (; k < nmine; ++k) {
         const int s = (int)(k % stages);
-        if (!mbar_wait_bounded(bbase + 8u * s, (uint32_t)((k / stages) & 1))) abort_flag = 1;
+        const bool bad = !mbar_wait_bounded(bbase + 8u * s, (uint32_t)((k / stages) & 1));
         const unsigned char* stg = smem + (size_t)s * row_bytes;
         const int64_t row = first + k * stride;
         const size_t roff = (size_t)row * row_bytes;
@@ -351,8 +347,7 @@ __global__ void __launch_bounds__(512) layer_staged_kernel(const RowArgs a, cons
             buf[0][t >> 5] = s1;
             buf[1][t >> 5] = s2;
         }
-        __syncthreads();
-        if (abort_flag) break;
+        if (__syncthreads_or(bad ? 1 : 0)) break;  // the same verdict in every thread
         s1 = 0.0;
         s2 = 0.0;
         for (int i = 0; i < wpr; ++i) {
