@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(512) layer_staged_kernel(const RowArgs a, cons
             buf[0][t >> 5] = s1;
             buf[1][t >> 5] = s2;
         }
-        if (__syncthreads_or(bad ? 1 : 0)) break;  // the same verdict in every thread
+        if (__syncthreads_or(bad ? 1 : 0)) break;  // the same decision in every thread
         s1 = 0.0;
         s2 = 0.0;
         for (int i = 0; i < wpr; ++i) {
