@@ -4,7 +4,8 @@ The benchmark shards by rows with no data-path collective; what crosses ranks is
 barrier and the max-over-ranks time.  The tensor-parallel all-reduce + add_rms_norm
 gathers every rank's partial output in rank order before the fused kernel; here the
 kernel is stood in for by the oracle (CPU tensors), which checks the gather, the order
-and that every rank computes the same result.
+and that every rank computes the same result.  A rank that leaves between steps makes the
+remaining rank's next gather fail (short process-group timeout) instead of hanging.
 """
 import os
 import socket
@@ -94,3 +95,50 @@ def test_tp_allreduce_gathers_in_rank_order_two_processes():
         mp.spawn(_tp_worker, args=(world, _free_port(), out), nprocs=world, join=True)
         res = dict(out)
     assert res[0] == res[1], "every rank must compute the same y and h"
+
+
+def _leaving_worker(rank, world, port, out):
+    import datetime
+    import time
+    from rope_add_rms_b200 import tp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    dist.barrier()              # one step completes on every rank
+    if rank == 1:
+        os._exit(0)             # rank 1 leaves between steps, with nothing in flight
+    t0 = time.monotonic()
+    try:
+        tp.gather_parts(torch.ones(4, 8))
+        out[rank] = ("no error", time.monotonic() - t0)
+    except Exception as e:  # noqa: BLE001 -- the error is what is checked
+        out[rank] = (type(e).__name__, time.monotonic() - t0)
+    finally:
+        try:
+            dist.destroy_process_group()
+        except Exception:  # noqa: BLE001
+            pass
+
+
+def test_a_rank_that_leaves_ends_the_next_gather_with_an_error():
+    """A rank that leaves between steps: the remaining rank's next gather of the partial
+    outputs ends with an error within the process group's short timeout, not a hang."""
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_leaving_worker, args=(r, 2, port, out)) for r in range(2)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+        hung = [p for p in procs if p.is_alive()]
+        for p in hung:
+            p.kill()
+            p.join()
+        res = dict(out)
+    assert not hung, "a rank is still waiting in its collective"
+    name, took = res[0]
+    print(f"remaining rank: {name} after {took:.2f} s")
+    assert name != "no error", "the gather with a departed rank must fail"
+    assert took < 60
