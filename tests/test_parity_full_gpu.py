@@ -10,7 +10,8 @@ Element-by-element against the CPU oracle for:
     w ~ U(0.5,1.5), eps 1e-5 (the TP8 workload of the benchmark)
   - the gradients: rms_norm_vjp bf16 [8192, 4096] and layer_norm_vjp bf16 [16384, 8192]
     on sampled rows (dx) and every column (dw, db) summed over all rows
-and on sampled rows for the add_rms_norm sweep D x rows x {bf16, f32} (eps 1e-6).
+and on sampled rows for the add_rms_norm sweep D x rows x {bf16, f32} (eps 1e-6) and for
+tensors past 2^31 elements (add_rms_norm, layer_norm, norm_rope, rms_norm_vjp).
 Large outputs are compared in row chunks to bound host memory.
 """
 import numpy as np
@@ -165,3 +166,62 @@ def test_gradients_full_size(op, rows, D):
     else:
         check_grad(dw, sums[0], sums[2], "dw")
         check_grad(db, sums[1], sums[3], "db")
+
+
+# ---- past 2^31 elements ---------------------------------------------------------------------
+# Row offsets are 64-bit throughout the kernels; these runs place rows beyond element 2^31
+# (byte 2^32 of a bf16 tensor) and compare sampled rows -- the rows straddling that boundary
+# and the last row always among them -- with the oracle.  About 26 GB of device memory at
+# the peak (four 4.3 GB tensors and the float32 draw of one).
+def _rows_past(rows, D, seed, k=64):
+    edge = (1 << 31) // D
+    return np.unique(np.concatenate([sample_rows(rows, k, seed),
+                                     np.arange(edge - 2, min(rows, edge + 3)), [rows - 1]]))
+
+
+def test_add_rms_norm_and_layer_norm_past_2_31_elements():
+    rows, D = (1 << 31) // 4096 + 5, 4096
+    x = synth.normal_device((rows, D), 0.0, 1.0, 7, synth.X, "bf16")
+    r = synth.normal_device((rows, D), 0.0, 1.0, 7, synth.R, "bf16")
+    w = synth.uniform_device((D,), 0.5, 1.5, 7, synth.W, "bf16")
+    b = synth.normal_device((D,), 0.0, 0.1, 7, synth.B, "bf16")
+    y, h = nv.add_rms_norm(x, r, w, eps=1e-5)
+    torch.cuda.synchronize()
+    idx = torch.as_tensor(_rows_past(rows, D, 1), device="cuda")
+    xs, rs, ws, bs = to_host_bits(x[idx]), to_host_bits(r[idx]), to_host_bits(w), to_host_bits(b)
+    ref, href = oracle.add_rms_norm(xs, rs, ws, 1e-5)
+    check_exact(h[idx], href, "h")
+    check_bf16(to_host_bits(y[idx]), ref, "y")
+    del r, y, h
+    torch.cuda.empty_cache()
+    yl = nv.layer_norm(x, w, b, eps=1e-5)
+    torch.cuda.synchronize()
+    check_bf16(to_host_bits(yl[idx]), oracle.layer_norm(xs, ws, bs, 1e-5), "layer_norm y")
+    del x, yl
+    torch.cuda.empty_cache()
+
+
+def test_norm_rope_and_rms_norm_vjp_past_2_31_elements():
+    H, L, D = 256, 65537, 128            # 16 777 472 rows of 128: 2^31 + 32 768 elements
+    rows = H * L
+    x = synth.normal_device((rows, D), 0.0, 1.0, 8, synth.X, "bf16")
+    w = synth.uniform_device((D,), 0.5, 1.5, 8, synth.W, "bf16")
+    y = nv.norm_rope(x.view(1, H, L, D), w, dims=D, traditional=False, base=10000.0,
+                     scale=1.0, offset=0, eps=1e-6).view(rows, D)
+    torch.cuda.synchronize()
+    ks = _rows_past(rows, D, 2)
+    idx = torch.as_tensor(ks, device="cuda")
+    xs, ws, ys = to_host_bits(x[idx]), to_host_bits(w), to_host_bits(y[idx])
+    for i, k in enumerate(ks):       # row k sits at position k mod L
+        ref = oracle.norm_rope(xs[i:i + 1], ws, 1, D, 0, 10000.0, 1.0, int(k % L), 1, 1e-6)
+        check_bf16(ys[i:i + 1], ref, f"norm_rope row {k}")
+    del y
+    torch.cuda.empty_cache()
+    g = synth.normal_device((rows, D), 0.0, 1.0, 8, synth.R, "bf16")
+    dx, dw = nv.rms_norm_vjp(x, w, g, eps=1e-5)
+    torch.cuda.synchronize()
+    rdx, _, mdx, _ = oracle.rms_norm_vjp(xs, ws, to_host_bits(g[idx]), 1e-5)
+    check_grad(dx[idx], rdx, mdx, "rms_norm_vjp dx")
+    assert torch.isfinite(dw.float()).all()
+    del x, g, dx, dw
+    torch.cuda.empty_cache()
