@@ -690,14 +690,14 @@ nv_status allreduce_add_rms_norm(const void* const* parts, int32_t nparts, const
     if (!h) return fail(NV_ERR_INVALID_ARG, "h is NULL");
     const size_t s = elem_size(dt);
     const size_t nbytes = (size_t)rows * (size_t)D * s;
+    int dev = 0;
+    DevInfo di;
+    st = current_device(&dev, &di);  // first, as in every entry: no usable device is NV_ERR_CUDA
+    if (st != NV_OK) return st;
     for (int i = 0; i < nparts; ++i) {
         st = check_part(parts[i], nbytes, i);
         if (st != NV_OK) return st;
     }
-    int dev = 0;
-    DevInfo di;
-    st = current_device(&dev, &di);
-    if (st != NV_OK) return st;
     // outputs may be exactly a row input (h over r, x_out over a part), nothing else
     Buf bufs[kMaxParts + 5];
     int nb = 0;
@@ -833,6 +833,10 @@ nv_status add_rms_norm_host(const void* x_host, const void* r_host, const void* 
         return fail(NV_ERR_INVALID_ARG, "y and h are the same buffer");
     const size_t s = elem_size(dt);
     const size_t nbytes = (size_t)rows * (size_t)D * s;
+    int dev = 0;
+    DevInfo di;
+    st = current_device(&dev, &di);  // first, as in every entry: no usable device is NV_ERR_CUDA
+    if (st != NV_OK) return st;
     for (int i = 0; i < 4; ++i) {
         st = check_host(ptrs[i], nbytes, names[i]);
         if (st != NV_OK) return st;
@@ -854,10 +858,6 @@ nv_status add_rms_norm_host(const void* x_host, const void* r_host, const void* 
         }
     }
 
-    int dev = 0;
-    DevInfo di;
-    st = current_device(&dev, &di);
-    if (st != NV_OK) return st;
     const Buf bufs[] = {
         {x_dev, nbytes, "x_dev", false, true},  {r_dev, nbytes, "r_dev", false, true},
         {w, (size_t)D * s, "w", false, false},  {y_dev, nbytes, "y_dev", true, false},

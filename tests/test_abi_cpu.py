@@ -242,3 +242,29 @@ def test_rope_llama3_freqs_rejects(kw, words):
     args.update(kw)
     with pytest.raises(nv.NvError, match=words):
         nv.rope_llama3_freqs(**args)
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="checks the path taken when no CUDA device can be used")
+@pytest.mark.parametrize("name, call", [
+    ("rms_norm", lambda: rms()),
+    ("add_rms_norm", lambda: add()),
+    ("layer_norm", lambda: layer()),
+    ("norm_rope", lambda: rope()),
+    ("rope", lambda: rope_general()),
+    ("rms_norm_vjp", lambda: vjp("rms")),
+    ("layer_norm_vjp", lambda: vjp("layer")),
+    ("allreduce_add_rms_norm", lambda: allreduce()),
+    ("add_rms_norm_host", lambda: nv.library().nv_add_rms_norm_host(   # x, r, w=NULL, y, h
+        *[ctypes.c_void_p(0x10000 * (i + 1)) for i in range(2)], None,  # on the host, then
+        *[ctypes.c_void_p(0x10000 * (i + 3)) for i in range(6)], 4, 8,  # the four staging
+        1e-5, BF16, 0, None)),                                            # device buffers
+    ("selftest_bounded_wait", lambda: nv.library().nv_selftest_bounded_wait(1, None)),
+])
+def test_cuda_failures_are_reported_as_nv_err_cuda(name, call):
+    """With no usable CUDA device, a well-formed call fails at its first CUDA runtime call:
+    the status is NV_ERR_CUDA, the message names that call and the runtime's error, and no
+    exception crosses the boundary (the process carries on)."""
+    assert call() == nv.NV_ERR_CUDA, name
+    msg = last_error()
+    assert re.match(r"^\w[\w ]*: cudaError\w+ \(", msg), msg
