@@ -328,20 +328,48 @@ def l2_flush_buffer():
     return torch.empty(2 * max(l2, 64 << 20), dtype=torch.uint8, device="cuda")
 
 
+class nvtx_range:
+    """An NVTX range around a phase of the bench (for nsys timelines and ncu's --nvtx
+    filters); a no-op where NVTX is unavailable."""
+
+    def __init__(self, name):
+        self.name = name
+        self.open = False
+
+    def __enter__(self):
+        try:
+            torch.cuda.nvtx.range_push(self.name)
+            self.open = True
+        except Exception:  # noqa: BLE001 -- tracing must never stop the bench
+            pass
+        return self
+
+    def __exit__(self, *exc):
+        if self.open:
+            try:
+                torch.cuda.nvtx.range_pop()
+            except Exception:  # noqa: BLE001
+                pass
+        return False
+
+
 def time_span(case, steps, warmup):
     """K back-to-back steps over rotating buffer sets, bracketed by one pair of CUDA
-    events on the launching stream; returns the span in ms."""
+    events on the launching stream; returns the span in ms.  NVTX ranges mark the
+    warm-up and the timed steps (one range each: nothing is added between launches)."""
     stream = torch.cuda.current_stream()
-    for i in range(warmup):
-        case.run(stream, i)
-    torch.cuda.synchronize()
+    with nvtx_range(f"{case.op} warmup x{warmup}"):
+        for i in range(warmup):
+            case.run(stream, i)
+        torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(steps):
-        case.run(stream, i)
-    end.record(stream)
-    torch.cuda.synchronize()
+    with nvtx_range(f"{case.op} timed x{steps}"):
+        start.record(stream)
+        for i in range(steps):
+            case.run(stream, i)
+        end.record(stream)
+        torch.cuda.synchronize()
     return start.elapsed_time(end)
 
 
@@ -360,9 +388,10 @@ def time_steps(case, steps, warmup, flush, e2e=False):
     for i in range(steps):
         if use_flush:
             flush.zero_()
-        starts[i].record(stream)
-        fn(stream, i)
-        ends[i].record(stream)
+        with nvtx_range(f"{case.op}{' e2e' if e2e else ''} step {i}"):
+            starts[i].record(stream)
+            fn(stream, i)
+            ends[i].record(stream)
     torch.cuda.synchronize()
     return [s.elapsed_time(e) for s, e in zip(starts, ends)]
 

@@ -57,3 +57,14 @@ def test_reference_arm_prints_one_contract_line():
     assert cb["sample"] and cb["unit"] == d["unit"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_nvtx_ranges_nest_and_never_raise():
+    with bench.nvtx_range("outer"):
+        with bench.nvtx_range("inner") as r:
+            assert r.open in (True, False)
+    try:
+        with bench.nvtx_range("failing body"):
+            raise KeyError("body")
+    except KeyError:
+        pass   # the body's exception propagates; the range is closed on the way out
