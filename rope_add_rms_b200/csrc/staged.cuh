@@ -10,16 +10,16 @@
 //
 // Per row k of this CTA (rows blockIdx.x, blockIdx.x + gridDim.x, ...):
 //   wait full[k % S] -> read x, r from the stage into registers -> h = RNE(x + r),
-//   store h, sum of squares -> CTA reduction (one __syncthreads: after it every thread
-//   has consumed the stage) -> thread 0 refills the stage with row k + S -> y = h*inv*w,
-//   store y.
+//   store h, sum of squares -> CTA reduction (one barrier, __syncthreads_or: after it
+//   every thread has consumed the stage, and all know whether any wait ran out) ->
+//   thread 0 refills the stage with row k + S -> y = h*inv*w, store y.
 // The copies are plain (non-multicast) 1-D bulk copies from this GPU's own memory into
 // the issuing CTA's shared memory.
 //
 // Every wait on an mbarrier is bounded (about one second of %globaltimer).  If a wait
-// runs out, the CTA counts a fault in nvn_fault_count (read by nv_fault_count()),
-// stops consuming rows, waits (again bounded) for the copies it has in flight and
-// returns.  A correct launch never gets there: the bytes expected per stage equal the
+// runs out, every thread of the CTA learns it at the row's barrier, the CTA counts a
+// fault in nvn_fault_count (read by nv_fault_count()), stops consuming rows, waits (again
+// bounded) for the copies it has in flight and returns.  A correct launch never gets there: the bytes expected per stage equal the
 // bytes copied into it.
 #pragma once
 
