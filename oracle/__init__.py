@@ -101,6 +101,7 @@ class Oracle:
         lib.oracle_add_rms_norm.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, f32, i32]
         f64 = ctypes.c_double
         lib.oracle_llama3_freqs.argtypes = [i64, f64, f64, f64, f64, f64, vp]
+        lib.oracle_yarn_freqs.argtypes = [i64, f64, f64, f64, f64, f64, vp, vp]
         lib.oracle_allreduce_add_rms_norm.argtypes = [vp, i32, vp, vp, vp, vp, vp, i64, i64, i64,
                                                       f32, i32]
         lib.oracle_layer_norm.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, i32]
@@ -168,6 +169,16 @@ class Oracle:
                                         orig, _ptr(out)) != 0:
             raise ValueError("arguments outside the Llama 3 scaling's domain")
         return out
+
+    def yarn_freqs(self, dims, base, s, L, alpha=1.0, beta=32.0):
+        """(frequencies h(theta_d), d < dims/2, float64; temperature factor sqrt(1/t)) of
+        YaRN with extension factor s over original context length L."""
+        out = np.empty(dims // 2, np.float64)
+        mscale = ctypes.c_double(0.0)
+        if self.lib.oracle_yarn_freqs(dims, base, s, L, alpha, beta, _ptr(out),
+                                      ctypes.byref(mscale)) != 0:
+            raise ValueError("arguments outside YaRN's domain")
+        return out, mscale.value
 
     def allreduce_add_rms_norm(self, parts, r, w, eps, threads=None):
         """(y, h, x): x = the sum of the partial tensors (in order, in double) rounded once
@@ -318,6 +329,10 @@ def add_rms_norm(x, r, w, eps, threads=None):
 
 def llama3_freqs(dims, base, factor, low_freq_factor, high_freq_factor, orig):
     return get().llama3_freqs(dims, base, factor, low_freq_factor, high_freq_factor, orig)
+
+
+def yarn_freqs(dims, base, s, L, alpha=1.0, beta=32.0):
+    return get().yarn_freqs(dims, base, s, L, alpha, beta)
 
 
 def allreduce_add_rms_norm(parts, r, w, eps, threads=None):

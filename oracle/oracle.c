@@ -334,6 +334,44 @@ int oracle_llama3_freqs(int64_t dims, double base, double factor, double low_fre
 }
 
 /*
+ * YaRN frequency scaling: named on docs.rs nuvec-core 0.5.0, Enum FastOp, variant Rope
+ * (frequency scaling by mlx-lm's YarnRoPE); the pages give neither parameters nor formula.
+ * Reading: the published YaRN method (Peng, Quesnelle, Fan and Shippole, "YaRN: Efficient
+ * Context Window Extension of Large Language Models", 2023), its "NTK-by-parts"
+ * interpolation and its attention temperature, in the paper's notation.  For pair d,
+ * theta_d = base^(-2d/dims), wavelength lambda_d = 2 pi / theta_d, and r_d = L / lambda_d
+ * the turns pair d makes over the original context length L.  With the ramp
+ *   gamma(r) = 0 (r < alpha),  1 (r > beta),  (r - alpha) / (beta - alpha) otherwise,
+ * the scaled frequency is h(theta_d) = (1 - gamma(r_d)) theta_d / s + gamma(r_d) theta_d
+ * (s the extension factor): pairs turning many times keep theta_d, pairs turning less than
+ * once are interpolated to theta_d / s.  The temperature scales q and k each by
+ * sqrt(1/t) = 0.1 ln(s) + 1.  out: dims / 2 doubles; *mscale: sqrt(1/t).  Returns -1
+ * outside the method's domain (dims even >= 2, base > 0, s >= 1, L > 0, 0 < alpha < beta).
+ */
+int oracle_yarn_freqs(int64_t dims, double base, double s, double L, double alpha, double beta,
+                      double* out, double* mscale) {
+    if (dims < 2 || dims % 2 || !(base > 0.0) || !(s >= 1.0) || !(L > 0.0) || !(alpha > 0.0) ||
+        !(beta > alpha))
+        return -1;
+    const double pi = acos(-1.0);
+    for (int64_t d = 0; d < dims / 2; ++d) {
+        const double theta_d = pow(base, -2.0 * (double)d / (double)dims);
+        const double lambda_d = 2.0 * pi / theta_d;
+        const double r = L / lambda_d;
+        double gamma;
+        if (r < alpha)
+            gamma = 0.0;
+        else if (r > beta)
+            gamma = 1.0;
+        else
+            gamma = (r - alpha) / (beta - alpha);
+        out[d] = (1.0 - gamma) * theta_d / s + gamma * theta_d;
+    }
+    *mscale = 0.1 * log(s) + 1.0;
+    return 0;
+}
+
+/*
  * The general NormRope / Rope (FastOp::NormRope with its cache form, FastOp::Rope with
  * freqs and forward): rows of x [B, H, L, D] (rows = B*H*L) are normalised when
  * normalize != 0 and rotated at position offset + l (by -phi when forward == 0), with

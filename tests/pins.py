@@ -216,6 +216,52 @@ def check_llama3_freqs_hand_case(o):
     assert abs(f[1] - 5.0 / 48.0) < 1e-15, f[1]
 
 
+# ---- YaRN frequency scaling (reading: the published method, in its own notation) --------
+
+def check_yarn_freqs_regions(o):
+    """s = 1 changes nothing and gives temperature 1; pairs turning more than beta times over
+    the original context keep theta exactly, those turning fewer than alpha times get exactly
+    theta / s, those between lie strictly between; the frequencies fall strictly with d."""
+    dims, base = 128, 10000.0
+    theta = np.array([base ** (-2.0 * d / dims) for d in range(dims // 2)])
+    f, m = o.yarn_freqs(dims, base, 1.0, 4096.0, 1.0, 32.0)
+    _close(f, theta, 1e-15, what="s = 1")
+    assert m == 1.0
+    for s, L, alpha, beta in ((16.0, 4096.0, 1.0, 32.0), (4.0, 2048.0, 2.0, 8.0)):
+        f, _ = o.yarn_freqs(dims, base, s, L, alpha, beta)
+        turns = L * theta / (2 * math.pi)
+        keep, interp = turns > beta, turns < alpha
+        mid = ~(keep | interp)
+        assert keep.any() and interp.any() and mid.any()
+        assert (f[keep] == theta[keep]).all(), "fast pairs must keep their frequency"
+        assert (f[interp] == theta[interp] / s).all(), "slow pairs must be divided by s"
+        assert ((f[mid] < theta[mid]) & (f[mid] > theta[mid] / s)).all()
+        assert (np.diff(f) < 0).all(), "scaled frequencies must fall strictly with d"
+
+
+def check_yarn_freqs_hand_case(o):
+    """dims 8, base 10^4: theta = 1, 0.1, 0.01, 0.001; over L = 4096 the pairs turn
+    4096 theta / (2 pi) = 651.90, 65.190, 6.518986, 0.65190 times.  With alpha 1, beta 32,
+    s 4: the first two keep theta, the last gets 0.001 / 4, and the third has
+    gamma = 5.518986469 / 31 = 0.1780318216, so 0.01 (0.1780318216 + 0.8219681784 / 4)
+    = 0.003835238662.  Temperature 0.1 ln 4 + 1 = 1.138629436."""
+    f, m = o.yarn_freqs(8, 10000.0, 4.0, 4096.0, 1.0, 32.0)
+    assert f[0] == 1.0 and abs(f[1] - 0.1) < 1e-17
+    assert abs(f[2] / 0.003835238662 - 1) < 1e-9, f[2]
+    assert abs(f[3] - 0.00025) < 1e-19, f[3]
+    assert abs(m - 1.138629436) < 1e-9, m
+
+
+def check_yarn_ramp_is_the_llama3_rule(o):
+    """The two readings, written separately, agree where they should: Llama 3's rule with
+    low / high frequency factors (alpha, beta) and original context L is YaRN's ramp
+    with those bounds (only the temperature differs)."""
+    for dims, base, s, L, alpha, beta in ((128, 500000.0, 32.0, 8192.0, 1.0, 4.0),
+                                          (64, 10000.0, 8.0, 4096.0, 1.0, 32.0)):
+        f, _ = o.yarn_freqs(dims, base, s, L, alpha, beta)
+        _close(f, o.llama3_freqs(dims, base, s, alpha, beta, L), 1e-14, what="YaRN vs Llama 3")
+
+
 # ---- rms_norm -------------------------------------------------------------------------
 
 def check_rms_constant_rows(o):

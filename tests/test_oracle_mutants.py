@@ -38,6 +38,16 @@ MUTANTS = {
                                     "            out[i] = theta * factor;\n"),
     "llama3_theta_over_dims_half": ("const double theta = pow(base, -(double)(2 * i) / (double)dims);",
                                     "const double theta = pow(base, -(double)i / (double)dims);"),
+    "yarn_ramp_reversed": ("gamma = (r - alpha) / (beta - alpha);",
+                           "gamma = (beta - r) / (beta - alpha);"),
+    "yarn_multiplies_by_s": ("out[d] = (1.0 - gamma) * theta_d / s + gamma * theta_d;",
+                             "out[d] = (1.0 - gamma) * theta_d * s + gamma * theta_d;"),
+    "yarn_ramp_roles_swapped": ("out[d] = (1.0 - gamma) * theta_d / s + gamma * theta_d;",
+                                "out[d] = gamma * theta_d / s + (1.0 - gamma) * theta_d;"),
+    "yarn_turns_inverted": ("const double r = L / lambda_d;", "const double r = lambda_d / L;"),
+    "yarn_temperature_log10": ("*mscale = 0.1 * log(s) + 1.0;", "*mscale = 0.1 * log10(s) + 1.0;"),
+    "yarn_temperature_squared": ("*mscale = 0.1 * log(s) + 1.0;",
+                                 "*mscale = (0.1 * log(s) + 1.0) * (0.1 * log(s) + 1.0);"),
     "layer_unbiased_variance": ("double var = sqdev / (double)D;",
                                 "double var = sqdev / (double)(D - 1);"),
     "layer_drops_mean_in_output": ("y[j] = (x[j] - mean) / denom * wj + bj;",
