@@ -187,6 +187,26 @@ NV_API nv_status nv_rope_llama3_freqs(int32_t dims, float base, float factor,
                                       int64_t original_max_position, float* freqs);
 
 /*
+ * rope_yarn_freqs -- YaRN frequency scaling for nv_rope's `freqs`: docs.rs nuvec-core 0.5.0,
+ * Enum FastOp, variant Rope names it (frequency scaling by YarnRoPE) without parameters or
+ * formula; read as the published method (Peng, Quesnelle, Fan and Shippole, "YaRN:
+ * Efficient Context Window Extension of Large Language Models", 2023).  With
+ * theta_i = base^(-2i/dims), pair i turns r_i = original_max_position * theta_i / (2 pi)
+ * times over the original context; pairs with r_i > beta keep theta_i, pairs with
+ * r_i < alpha get theta_i / factor, and between them theta_i / factor is blended linearly
+ * toward theta_i by (r_i - alpha) / (beta - alpha) ("NTK-by-parts").  YaRN also scales the
+ * rotated q and k each by the temperature factor mscale = 0.1 ln(factor) + 1; this library
+ * does not apply it: multiply the attention logits by mscale^2 (or q and k by mscale).
+ * The paper's values for LLaMA are alpha = 1, beta = 32.  Computed in double on the host,
+ * rounded once: freqs [dims / 2] and mscale are HOST memory (copy freqs to the device for
+ * nv_rope); mscale may be NULL.  Needs dims even >= 2, base > 0, factor >= 1,
+ * 0 < alpha < beta, original_max_position > 0 (else NV_ERR_INVALID_ARG).  Needs no GPU.
+ */
+NV_API nv_status nv_rope_yarn_freqs(int32_t dims, float base, float factor,
+                                    int64_t original_max_position, float alpha, float beta,
+                                    float* freqs, float* mscale);
+
+/*
  * allreduce_add_rms_norm -- the step a tensor-parallel decoder takes after a row-parallel
  * layer: miniVLLM Layers page, section Linear layers, RowParallelLinear (the forward pass
  * sums the ranks' partial outputs with an all_reduce), then the fused residual add +

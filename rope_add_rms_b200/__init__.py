@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "NvError", "Plan", "library", "library_path",
     "nv_rms_norm", "nv_add_rms_norm", "nv_add_rms_norm_host", "nv_allreduce_add_rms_norm",
-    "allreduce_add_rms_norm", "rope_llama3_freqs", "nv_layer_norm", "nv_norm_rope",
+    "allreduce_add_rms_norm", "rope_llama3_freqs", "rope_yarn_freqs", "nv_layer_norm", "nv_norm_rope",
     "nv_describe_plan",
     "nv_fault_count", "nv_selftest_bounded_wait",
     "nv_rope", "rms_norm", "add_rms_norm", "layer_norm", "norm_rope", "norm_rope_into_cache",
@@ -113,6 +113,8 @@ def library() -> ctypes.CDLL:
     lib.nv_layer_norm_vjp.restype = ctypes.c_int
     lib.nv_rope_llama3_freqs.argtypes = [i32, f32, f32, f32, f32, i64, vp]
     lib.nv_rope_llama3_freqs.restype = ctypes.c_int
+    lib.nv_rope_yarn_freqs.argtypes = [i32, f32, f32, i64, f32, f32, vp, vp]
+    lib.nv_rope_yarn_freqs.restype = ctypes.c_int
     lib.nv_norm_vjp_workspace_size.argtypes = [i32, i64, i64]
     lib.nv_norm_vjp_workspace_size.restype = sz
     _lib = lib
@@ -209,6 +211,19 @@ def rope_llama3_freqs(dims, base=500000.0, factor=32.0, low_freq_factor=1.0,
                                         original_max_position, ctypes.c_void_p(out.data_ptr()))
     _check("nv_rope_llama3_freqs", st)
     return out
+
+
+def rope_yarn_freqs(dims, base=10000.0, factor=4.0, original_max_position=4096, alpha=1.0,
+                    beta=32.0):
+    """YaRN scaled RoPE frequencies (a float32 host tensor of dims/2, for
+    ``nv_rope(..., freqs=...)`` after ``.cuda()``) and its temperature factor mscale, which
+    the caller applies (attention logits times mscale**2)."""
+    out = torch.empty(dims // 2, dtype=torch.float32)
+    m = ctypes.c_float(0.0)
+    st = library().nv_rope_yarn_freqs(dims, base, factor, original_max_position, alpha, beta,
+                                      ctypes.c_void_p(out.data_ptr()), ctypes.byref(m))
+    _check("nv_rope_yarn_freqs", st)
+    return out, m.value
 
 
 def nv_allreduce_add_rms_norm(parts, r, w, y, h, eps, x_out=None, stream=None):

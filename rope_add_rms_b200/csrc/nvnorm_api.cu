@@ -1272,6 +1272,42 @@ nv_status nv_rope_llama3_freqs(int32_t dims, float base, float factor, float low
     return NV_OK;
 }
 
+nv_status nv_rope_yarn_freqs(int32_t dims, float base, float factor,
+                             int64_t original_max_position, float alpha, float beta,
+                             float* freqs, float* mscale) {
+    if (dims < 2 || dims % 2 != 0)
+        return fail(NV_ERR_INVALID_ARG, "dims = %d must be even and >= 2", dims);
+    if (!(base > 0.f) || !std::isfinite(base))
+        return fail(NV_ERR_INVALID_ARG, "base = %g must be finite and > 0", (double)base);
+    if (!(factor >= 1.f) || !std::isfinite(factor))
+        return fail(NV_ERR_INVALID_ARG, "factor = %g must be finite and >= 1", (double)factor);
+    if (!(alpha > 0.f) || !(beta > alpha) || !std::isfinite(beta))
+        return fail(NV_ERR_INVALID_ARG, "need 0 < alpha (%g) < beta (%g)", (double)alpha,
+                    (double)beta);
+    if (original_max_position <= 0)
+        return fail(NV_ERR_INVALID_ARG, "original_max_position = %lld must be > 0",
+                    (long long)original_max_position);
+    if (!freqs) return fail(NV_ERR_INVALID_ARG, "freqs is NULL");
+    const double ctx = (double)original_max_position, s = factor;
+    const double per_turn = 1.0 / (2.0 * 3.14159265358979323846);
+    for (int32_t i = 0; i < dims / 2; ++i) {
+        const double th = std::pow((double)base, -2.0 * (double)i / (double)dims);
+        const double turns = ctx * th * per_turn;  // rotations of pair i over the context
+        double out;
+        if (turns > beta) {
+            out = th;                                 // fast pairs: extrapolate
+        } else if (turns < alpha) {
+            out = th / s;                             // slow pairs: interpolate
+        } else {
+            const double g = (turns - alpha) / ((double)beta - (double)alpha);
+            out = th / s + g * (th - th / s);
+        }
+        freqs[i] = (float)out;
+    }
+    if (mscale) *mscale = (float)(1.0 + 0.1 * std::log(s));
+    return NV_OK;
+}
+
 nv_status nv_allreduce_add_rms_norm(const void* const* parts, int32_t nparts, const void* r,
                                     const void* w, void* y, void* h, void* x_out, int64_t rows,
                                     int64_t D, float eps, nv_dtype dt, nv_stream_t stream) {

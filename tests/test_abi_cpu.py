@@ -244,6 +244,36 @@ def test_rope_llama3_freqs_rejects(kw, words):
         nv.rope_llama3_freqs(**args)
 
 
+# ---- YaRN frequency scaling: also a host-side helper ------------------------------------------
+
+@pytest.mark.parametrize("args", [(128, 10000.0, 4.0, 4096, 1.0, 32.0),
+                                  (128, 500000.0, 16.0, 8192, 1.0, 32.0),
+                                  (64, 10000.0, 8.0, 2048, 2.0, 8.0),
+                                  (8, 10000.0, 4.0, 4096, 1.0, 32.0),
+                                  (128, 10000.0, 1.0, 4096, 1.0, 32.0)])
+def test_rope_yarn_freqs_matches_the_oracle(args):
+    import numpy as np
+    import oracle
+    got, m = nv.rope_yarn_freqs(*args)
+    want, want_m = oracle.yarn_freqs(args[0], args[1], args[2], float(args[3]), args[4], args[5])
+    got, want = got.numpy(), want.astype(np.float32)
+    ulps = np.abs(got.view(np.int32).astype(np.int64) - want.view(np.int32).astype(np.int64))
+    assert ulps.max() <= 1, f"{int(ulps.max())} float ulps apart"
+    assert abs(m - want_m) <= 2.0 ** -23 * want_m
+
+
+@pytest.mark.parametrize("kw, words", [
+    (dict(dims=5), "dims"), (dict(base=-1.0), "base"), (dict(factor=0.9), "factor"),
+    (dict(alpha=0.0), "alpha"), (dict(alpha=32.0, beta=32.0), "alpha"),
+    (dict(original_max_position=-4), "original_max_position")])
+def test_rope_yarn_freqs_rejects(kw, words):
+    args = dict(dims=128, base=10000.0, factor=4.0, original_max_position=4096, alpha=1.0,
+                beta=32.0)
+    args.update(kw)
+    with pytest.raises(nv.NvError, match=words):
+        nv.rope_yarn_freqs(**args)
+
+
 @pytest.mark.skipif(__import__("torch").cuda.is_available(),
                     reason="checks the path taken when no CUDA device can be used")
 @pytest.mark.parametrize("name, call", [

@@ -697,6 +697,23 @@ def test_rope_llama3_scaled_frequencies(trad, dt):
         check_out(y, ref, f"offset {offset}")
 
 
+@pytest.mark.parametrize("trad", [0, 1])
+def test_rope_yarn_scaled_frequencies(trad):
+    """NormRope with YaRN frequencies (factor 8 over an original context of 4096) at
+    positions past that context."""
+    B, H, L, D = 2, 4, 64, 128
+    inp = synth.norm_rope_inputs(B, H, L, D, "bf16", seed=47)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    freqs, _ = nv.rope_yarn_freqs(D, 10000.0, 8.0, 4096, 1.0, 32.0)
+    for offset in (0, 30000):
+        y = torch.empty_like(x)
+        nv.nv_rope(x, w, y, L, D, trad, 10000.0, 1.0, offset, 1, 1e-6, freqs=freqs.cuda())
+        torch.cuda.synchronize()
+        ref = oracle.rope_ex(host(inp["x"]), host(inp["w"]), L, D, trad, 10000.0, 1.0, offset, 1,
+                             1e-6, freqs=freqs.numpy().astype(np.float64))
+        check_out(y, ref, f"offset {offset}")
+
+
 def test_rope_round_trip_and_cache_rules():
     B, H, L, D = 1, 2, 8, 64
     x = synth.normal((B * H * L, D), 0.0, 1.0, 33, 0, "f32").cuda()
