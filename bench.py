@@ -260,9 +260,12 @@ class Case:
                     op[:-4], rows, D)), dtype=torch.uint8, device="cuda")
             self.sets.append(d)
         self.nv = nv
-        # explicit frequencies (the Llama 3 scaling) for the general rope call
-        self.freqs = (nv.rope_llama3_freqs(self.D).cuda() if op == "norm_rope" and kw.get("llama3")
-                      else None)
+        # explicit frequencies (the Llama 3 or the YaRN scaling) for the general rope call
+        self.freqs = None
+        if op == "norm_rope" and kw.get("llama3"):
+            self.freqs = nv.rope_llama3_freqs(self.D).cuda()
+        elif op == "norm_rope" and kw.get("yarn"):
+            self.freqs = nv.rope_yarn_freqs(self.D, 10000.0, 8.0, 4096)[0].cuda()
         n_out = 2 if op == "add_rms_norm" else 1
         self.host_out = [] if on_dev or "x" not in self.host else \
             [torch.empty_like(self.host["x"]).pin_memory() for _ in range(n_out)]
@@ -607,6 +610,10 @@ WORKLOADS = {
     "norm_rope_llama3": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-5,
                                      dims=128, traditional=0, base=500000.0, scale=1.0,
                                      offset=16384, llama3=True),
+    # NormRope with YaRN frequencies (factor 8 over an original context of 4096), past it
+    "norm_rope_yarn": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,
+                                   dims=128, traditional=0, base=10000.0, scale=1.0,
+                                   offset=16384, yarn=True),
     "rms_norm_vjp": lambda: Case("rms_norm_vjp", (8192, 4096), "bf16", 0, eps=1e-5),
     "layer_norm_vjp": lambda: Case("layer_norm_vjp", (16384, 8192), "bf16", 0, eps=1e-5),
     # a TP8 decoder's all-reduce + residual add + RMSNorm, the 8 partial outputs already
