@@ -48,6 +48,15 @@ MUTANTS = {
     "yarn_temperature_log10": ("*mscale = 0.1 * log(s) + 1.0;", "*mscale = 0.1 * log10(s) + 1.0;"),
     "yarn_temperature_squared": ("*mscale = 0.1 * log(s) + 1.0;",
                                  "*mscale = (0.1 * log(s) + 1.0) * (0.1 * log(s) + 1.0);"),
+    "layer_mean_over_D_minus_1": ("double mean = sum / (double)D;\n    double sqdev = 0.0;\n    for (int64_t j = 0; j < D; ++j) sqdev +=",
+                                  "double mean = sum / (double)(D - 1);\n    double sqdev = 0.0;\n    for (int64_t j = 0; j < D; ++j) sqdev +="),
+    "layer_eps_outside_sqrt": ("double denom = sqrt(var + eps);", "double denom = sqrt(var) + eps;"),
+    "rms_eps_outside_sqrt": ("sqrt(sumsq / (double)D + eps)", "(sqrt(sumsq / (double)D) + eps)"),
+    "rms_no_sqrt": ("sqrt(sumsq / (double)D + eps)", "(sumsq / (double)D + eps)"),
+    "rms_weight_squared": ("y[j] = x[j] / denom * wj;", "y[j] = x[j] / denom * wj * wj;"),
+    "rope_theta_index_shifted": ("double theta = freqs ? freqs[i] : pow(base, -2.0 * (double)i / (double)dims);",
+                                 "double theta = freqs ? freqs[i] : pow(base, -2.0 * (double)(i + 1) / (double)dims);"),
+    "rms_vjp_dw_weighted": ("dw[j] += gj * xj * r;", "dw[j] += gj * wj * xj * r;"),
     "layer_unbiased_variance": ("double var = sqdev / (double)D;",
                                 "double var = sqdev / (double)(D - 1);"),
     "layer_drops_mean_in_output": ("y[j] = (x[j] - mean) / denom * wj + bj;",
