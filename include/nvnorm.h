@@ -288,9 +288,10 @@ NV_API int32_t nv_version(void);
 
 /*
  * Device-side bounded waits that ran out, on the current device, since the library
- * was loaded (or last reset).  Only the staged kernels wait on the copy engine; each
- * wait gives up after about one second, counts a fault here, lets its copies in
- * flight land and leaves the rest of its rows unwritten.  Synchronises the device.
+ * was loaded (or last reset).  Only the staged kernels wait on the copy engine (and
+ * nv_selftest_bounded_wait, on purpose, on a barrier nothing completes); each wait gives
+ * up after about one second, counts a fault here, lets its copies in flight land and
+ * leaves the rest of its rows unwritten.  Synchronises the device.
  * count: out, non-NULL.  reset != 0 sets the counter back to zero after reading it.
  */
 NV_API nv_status nv_fault_count(uint32_t* count, int32_t reset);
