@@ -102,6 +102,7 @@ class Oracle:
         f64 = ctypes.c_double
         lib.oracle_llama3_freqs.argtypes = [i64, f64, f64, f64, f64, f64, vp]
         lib.oracle_yarn_freqs.argtypes = [i64, f64, f64, f64, f64, f64, vp, vp]
+        lib.oracle_suscaled_freqs.argtypes = [i64, f64, vp, vp, f64, f64, f64, vp, vp]
         lib.oracle_allreduce_add_rms_norm.argtypes = [vp, i32, vp, vp, vp, vp, vp, i64, i64, i64,
                                                       f32, i32]
         lib.oracle_layer_norm.argtypes = [vp, vp, vp, vp, i64, i64, i64, f32, i32]
@@ -178,6 +179,21 @@ class Oracle:
         if self.lib.oracle_yarn_freqs(dims, base, s, L, alpha, beta, _ptr(out),
                                       ctypes.byref(mscale)) != 0:
             raise ValueError("arguments outside YaRN's domain")
+        return out, mscale.value
+
+    def suscaled_freqs(self, dims, base, short_factors, long_factors, seq_len, max_pos, orig):
+        """(frequencies theta_i / lambda_i, i < dims/2, float64; attention factor) of the
+        LongRoPE / SuScaled scaling: lambda the long factors when seq_len exceeds the
+        original context orig, else the short ones."""
+        sf = np.ascontiguousarray(short_factors, np.float64)
+        lf = np.ascontiguousarray(long_factors, np.float64)
+        if sf.shape != (dims // 2,) or lf.shape != (dims // 2,):
+            raise ValueError("factor lists must hold dims / 2 values")
+        out = np.empty(dims // 2, np.float64)
+        mscale = ctypes.c_double(0.0)
+        if self.lib.oracle_suscaled_freqs(dims, base, _ptr(sf), _ptr(lf), seq_len, max_pos, orig,
+                                          _ptr(out), ctypes.byref(mscale)) != 0:
+            raise ValueError("arguments outside the SuScaled scaling's domain")
         return out, mscale.value
 
     def allreduce_add_rms_norm(self, parts, r, w, eps, threads=None):
@@ -333,6 +349,10 @@ def llama3_freqs(dims, base, factor, low_freq_factor, high_freq_factor, orig):
 
 def yarn_freqs(dims, base, s, L, alpha=1.0, beta=32.0):
     return get().yarn_freqs(dims, base, s, L, alpha, beta)
+
+
+def suscaled_freqs(dims, base, short_factors, long_factors, seq_len, max_pos, orig):
+    return get().suscaled_freqs(dims, base, short_factors, long_factors, seq_len, max_pos, orig)
 
 
 def allreduce_add_rms_norm(parts, r, w, eps, threads=None):

@@ -372,6 +372,39 @@ int oracle_yarn_freqs(int64_t dims, double base, double s, double L, double alph
 }
 
 /*
+ * SuScaled (LongRoPE) frequency scaling: named on docs.rs nuvec-core 0.5.0, Enum FastOp,
+ * variant Rope (frequency scaling by mlx-lm's SuScaledRoPE); the pages give neither
+ * parameters nor formula.  Reading: the published LongRoPE method (Ding, Zhang, Zhang, Xu,
+ * Shang, Xu, Yang and Yang, "LongRoPE: Extending LLM Context Window Beyond 2 Million
+ * Tokens", 2024) in the form the Phi-3 models use it (Abdin et al., "Phi-3 Technical
+ * Report", 2024): every pair i has its own rescale factor lambda_i and turns at
+ * theta_i / lambda_i, theta_i = base^(-2i/dims).  Two factor sets are searched, a short
+ * one for sequences within the original context L and a long one beyond it:
+ * lambda = long_factors when seq_len > L, else short_factors.  Extending L to the model's
+ * maximum context L' (s = L' / L) also scales q and k by the attention factor
+ * sqrt(1 + ln s / ln L) when s > 1 (1 otherwise).
+ * out: dims / 2 doubles; *mscale: the attention factor.  Returns -1 outside the method's
+ * domain (dims even >= 2, base > 0, every factor > 0, L > 1, L' > 0, seq_len >= 0).
+ */
+int oracle_suscaled_freqs(int64_t dims, double base, const double* short_factors,
+                          const double* long_factors, double seq_len, double max_pos,
+                          double orig, double* out, double* mscale) {
+    if (dims < 2 || dims % 2 || !(base > 0.0) || !(orig > 1.0) || !(max_pos > 0.0) ||
+        !(seq_len >= 0.0))
+        return -1;
+    const double* lambda = seq_len > orig ? long_factors : short_factors;
+    for (int64_t i = 0; i < dims / 2; ++i)
+        if (!(lambda[i] > 0.0)) return -1;
+    for (int64_t i = 0; i < dims / 2; ++i) {
+        const double theta_i = 1.0 / pow(base, 2.0 * (double)i / (double)dims);
+        out[i] = theta_i / lambda[i];
+    }
+    const double s = max_pos / orig;
+    *mscale = s > 1.0 ? sqrt(1.0 + log(s) / log(orig)) : 1.0;
+    return 0;
+}
+
+/*
  * The general NormRope / Rope (FastOp::NormRope with its cache form, FastOp::Rope with
  * freqs and forward): rows of x [B, H, L, D] (rows = B*H*L) are normalised when
  * normalize != 0 and rotated at position offset + l (by -phi when forward == 0), with

@@ -262,6 +262,42 @@ def check_yarn_ramp_is_the_llama3_rule(o):
         _close(f, o.llama3_freqs(dims, base, s, alpha, beta, L), 1e-14, what="YaRN vs Llama 3")
 
 
+# ---- SuScaled (LongRoPE) frequency scaling (reading: the published method) ---------------
+
+def check_suscaled_identity_and_selection(o):
+    """Factors of 1 leave the base frequencies exactly, and a maximum context within the
+    original one gives attention factor 1; the short factors serve sequences up to the
+    original context L, the long ones from L + 1 on; each pair's frequency is divided by
+    its own factor (the ratio of the long to the short result is short / long, pair by pair)."""
+    dims, base = 64, 10000.0
+    half = dims // 2
+    theta = np.array([base ** (-2.0 * i / dims) for i in range(half)])
+    ones = np.ones(half)
+    f, m = o.suscaled_freqs(dims, base, ones, ones, 100000.0, 4096.0, 4096.0)
+    _close(f, theta, 1e-15, what="factors 1")
+    assert m == 1.0
+    rng = _rng(21)
+    short, long_ = rng.uniform(1.0, 1.5, half), rng.uniform(1.0, 40.0, half)
+    fs, ms = o.suscaled_freqs(dims, base, short, long_, 4096.0, 131072.0, 4096.0)
+    fl, ml = o.suscaled_freqs(dims, base, short, long_, 4097.0, 131072.0, 4096.0)
+    _close(fs, theta / short, 1e-15, what="short factors at seq_len = L")
+    _close(fl, theta / long_, 1e-15, what="long factors at seq_len = L + 1")
+    _close(fl / fs, short / long_, 1e-14, what="per-pair ratio")
+    assert ms == ml > 1.0, "the attention factor depends on the contexts, not on seq_len"
+
+
+def check_suscaled_hand_case(o):
+    """dims 4, base 10^4: theta = (1, 0.01).  Short factors (1, 2) give (1, 0.005); long
+    factors (4, 8) give (0.25, 0.00125).  L = 4096 = 2^12 extended to L' = 131072 = 2^17:
+    s = 32, ln s / ln L = 5/12, attention factor sqrt(17/12) = 1.190238071."""
+    f, m = o.suscaled_freqs(4, 10000.0, [1.0, 2.0], [4.0, 8.0], 1000.0, 131072.0, 4096.0)
+    assert f[0] == 1.0 and abs(f[1] - 0.005) < 1e-18, f
+    f, m2 = o.suscaled_freqs(4, 10000.0, [1.0, 2.0], [4.0, 8.0], 8192.0, 131072.0, 4096.0)
+    assert f[0] == 0.25 and abs(f[1] - 0.00125) < 1e-18, f
+    assert m == m2 and abs(m - math.sqrt(17.0 / 12.0)) < 1e-15, m
+    assert abs(m - 1.190238071) < 1e-9
+
+
 # ---- rms_norm -------------------------------------------------------------------------
 
 def check_rms_constant_rows(o):

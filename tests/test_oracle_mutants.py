@@ -46,6 +46,19 @@ MUTANTS = {
                                 "out[d] = gamma * theta_d / s + (1.0 - gamma) * theta_d;"),
     "yarn_turns_inverted": ("const double r = L / lambda_d;", "const double r = lambda_d / L;"),
     "yarn_temperature_log10": ("*mscale = 0.1 * log(s) + 1.0;", "*mscale = 0.1 * log10(s) + 1.0;"),
+    "suscaled_multiplies_by_factor": ("out[i] = theta_i / lambda[i];", "out[i] = theta_i * lambda[i];"),
+    "suscaled_long_from_L": ("const double* lambda = seq_len > orig ? long_factors : short_factors;",
+                             "const double* lambda = seq_len >= orig ? long_factors : short_factors;"),
+    "suscaled_factor_sets_swapped": ("const double* lambda = seq_len > orig ? long_factors : short_factors;",
+                                     "const double* lambda = seq_len > orig ? short_factors : long_factors;"),
+    "suscaled_factor_index_reversed": ("out[i] = theta_i / lambda[i];",
+                                       "out[i] = theta_i / lambda[dims / 2 - 1 - i];"),
+    "suscaled_attention_no_sqrt": ("*mscale = s > 1.0 ? sqrt(1.0 + log(s) / log(orig)) : 1.0;",
+                                   "*mscale = s > 1.0 ? 1.0 + log(s) / log(orig) : 1.0;"),
+    "suscaled_attention_ratio_inverted": ("*mscale = s > 1.0 ? sqrt(1.0 + log(s) / log(orig)) : 1.0;",
+                                          "*mscale = s > 1.0 ? sqrt(1.0 + log(orig) / log(s)) : 1.0;"),
+    "suscaled_attention_log_of_max": ("*mscale = s > 1.0 ? sqrt(1.0 + log(s) / log(orig)) : 1.0;",
+                                      "*mscale = s > 1.0 ? sqrt(1.0 + log(max_pos) / log(orig)) : 1.0;"),
     "yarn_temperature_squared": ("*mscale = 0.1 * log(s) + 1.0;",
                                  "*mscale = (0.1 * log(s) + 1.0) * (0.1 * log(s) + 1.0);"),
     "layer_mean_over_D_minus_1": ("double mean = sum / (double)D;\n    double sqdev = 0.0;\n    for (int64_t j = 0; j < D; ++j) sqdev +=",
