@@ -627,6 +627,9 @@ def run_workload(args):
     """One named workload (not the headline metric): GB/s of algorithmic bytes."""
     torch.cuda.set_device(dist_env()[2])
     c = WORKLOADS[args.workload]()
+    import rope_add_rms_b200 as nv
+    if args.plan:
+        c.plan = nv.Plan(**json.loads(args.plan))
     flush = l2_flush_buffer()
     peak, _ = measured_peak()
     if c.rotating:
@@ -634,7 +637,8 @@ def run_workload(args):
     else:
         ms = statistics.median(time_steps(c, args.steps, args.warmup, flush))
     gbs = c.bytes / (ms * 1e-3) / 1e9
-    print(json.dumps({"workload": args.workload, "op": c.op, "rows": c.rows, "D": c.D,
+    plan = c.plan.as_dict() if c.plan is not None else None
+    print(json.dumps({"workload": args.workload, "op": c.op, "rows": c.rows, "D": c.D, "plan": plan,
                       "dtype": c.dtype, "us_per_call": round(ms * 1e3, 3), "GB/s": round(gbs, 1),
                       "frac_of_measured_hbm": round(gbs / peak, 4),
                       "rows_per_s": round(c.rows / (ms * 1e-3), 1), "l2": c.l2_note()}),
@@ -642,25 +646,88 @@ def run_workload(args):
     return 0
 
 
+# Forced plans the sweep compares with the automatic one (register path at every vector
+# count, with one or two rows per CTA, persistent grids, and the staged path).
+SWEEP_PLANS = (
+    [{"path": 1, "vec_per_thread": v} for v in (1, 2, 4, 8)]
+    + [{"path": 1, "vec_per_thread": v, "rows_per_cta": 2} for v in (2, 4, 8)]
+    + [{"path": 1, "vec_per_thread": 4, "ctas_per_sm": c} for c in (2, 4)]
+    + [{"path": 3}, {"path": 3, "ctas_per_sm": 2}]
+)
+
+
+def host_cost(op, rows, D, dtype, iters=200):
+    """Host time inside one C-ABI call and device time per call (tests/c/host_cost.c,
+    compiled here with gcc): the decode-size story, where the call's host cost can exceed
+    the kernel.  None if the program cannot be built."""
+    import shutil
+    from rope_add_rms_b200 import library_path
+    if shutil.which("gcc") is None:
+        return None
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    exe = os.path.join(tempfile.gettempdir(), f"nv_host_cost_{os.getpid()}")
+    if not os.path.exists(exe):
+        libdir = os.path.dirname(library_path)
+        cmd = ["gcc", "-std=c99", "-O2", "-I", os.path.join(ROOT, "include"),
+               "-I", os.path.join(cuda, "include"), os.path.join(ROOT, "tests", "c", "host_cost.c"),
+               "-o", exe, "-L", libdir, "-lnvnorm", "-L", os.path.join(cuda, "lib64"), "-lcudart",
+               f"-Wl,-rpath,{libdir}", f"-Wl,-rpath,{os.path.join(cuda, 'lib64')}"]
+        if subprocess.run(cmd, capture_output=True).returncode != 0:
+            return None
+    res = subprocess.run([exe, "add" if op == "add_rms_norm" else "rms", str(rows), str(D),
+                          dtype, str(iters)], capture_output=True, text=True, timeout=120)
+    if res.returncode != 0:
+        return None
+    return json.loads(res.stdout)
+
+
 def run_sweep(args):
-    """add_rms_norm over D x rows x dtype (eps 1e-6): one JSON line per point."""
+    """add_rms_norm over D x rows x dtype (eps 1e-6): one JSON line per point.  Points of
+    >= 4096 rows also time every forced plan of SWEEP_PLANS and report the best next to the
+    automatic plan; points of <= 256 rows add the host cost of one call through the C ABI
+    (latency-bound: the kernel time is not an HBM figure there)."""
+    import rope_add_rms_b200 as nv
     torch.cuda.set_device(dist_env()[2])
     flush = l2_flush_buffer()
     peak, _ = measured_peak()
+
+    def timed(c):
+        if c.rotating:
+            return time_span(c, args.steps, args.warmup) / args.steps
+        return statistics.median(time_steps(c, args.steps, args.warmup, flush))
+
     for dtype in ("bf16", "f32"):
         for D in (2048, 4096, 5120, 8192, 16384):
             for rows in (1, 16, 256, 4096, 65536):
                 c = Case("add_rms_norm", (rows, D), dtype, 0, eps=1e-6)
-                if c.rotating:
-                    med = time_span(c, args.steps, args.warmup) / args.steps
-                else:
-                    med = statistics.median(time_steps(c, args.steps, args.warmup, flush))
+                med = timed(c)
                 gbs = c.bytes / (med * 1e-3) / 1e9
-                print(json.dumps({"op": "add_rms_norm", "dtype": dtype, "rows": rows, "D": D,
-                                  "median_us": round(med * 1e3, 2), "GB/s": round(gbs, 1),
-                                  "frac": round(gbs / peak, 4),
-                                  "rows_per_s": round(rows / (med * 1e-3), 1),
-                                  "bound": "hbm" if rows >= 4096 else "latency"}), flush=True)
+                auto = nv.nv_describe_plan("add_rms_norm", rows, D,
+                                           torch.bfloat16 if dtype == "bf16" else torch.float32)
+                line = {"op": "add_rms_norm", "dtype": dtype, "rows": rows, "D": D,
+                        "median_us": round(med * 1e3, 2), "GB/s": round(gbs, 1),
+                        "frac": round(gbs / peak, 4),
+                        "rows_per_s": round(rows / (med * 1e-3), 1),
+                        "bound": "hbm" if rows >= 4096 else "latency", "plan": auto}
+                if rows >= 4096 and args.plans:
+                    best = None
+                    for p in SWEEP_PLANS:
+                        c.plan = nv.Plan(**p)
+                        try:
+                            m = timed(c)
+                        except nv.NvError:
+                            continue
+                        if best is None or m < best[0]:
+                            best = (m, p)
+                    c.plan = None
+                    if best:
+                        bg = c.bytes / (best[0] * 1e-3) / 1e9
+                        line["best_forced"] = {"plan": best[1], "median_us": round(best[0] * 1e3, 2),
+                                               "GB/s": round(bg, 1)}
+                        line["auto_over_best"] = round(gbs / bg, 4)
+                if rows <= 256:
+                    line["host_call"] = host_cost("add_rms_norm", rows, D, dtype)
+                print(json.dumps(line), flush=True)
                 del c
                 torch.cuda.empty_cache()
     return 0
@@ -673,8 +740,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--plans", action="store_true",
+                    help="with --sweep: also time the forced plans at each large point")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
                     help="time one named workload instead of the headline step")
+    ap.add_argument("--plan", default=None,
+                    help="with --workload: a forced nv_plan as JSON, e.g. '{\"path\": 4}'")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -141,8 +141,10 @@ NV_API nv_status nv_rope(const void* x, const void* w, const float* freqs, void*
  * workspace: device memory of at least nv_norm_vjp_workspace_size(0, rows, D) bytes when
  * dw is requested (per-CTA partial sums of the columns; contents are overwritten), else
  * may be NULL.  dw is deterministic: the partials are added in a fixed order in double.
- * rows == 0 with dw requested writes dw = 0.  Needs D a multiple of 16 bytes of elements,
- * D <= 16384 (bf16) / 8192 (f32), and 16-byte aligned x, g, dx, w.
+ * rows == 0 with dw requested writes dw = 0.  Any D >= 1 and any element alignment: rows
+ * of whole 16-byte vectors with D <= 16384 (bf16) / 8192 (f32) and 16-byte aligned x, g, dx
+ * and w take the register kernels; other rows a generic kernel (scalar accesses, row
+ * statistics in double; slower).
  */
 NV_API nv_status nv_rms_norm_vjp(const void* x, const void* w, const void* g, void* dx, void* dw,
                                  void* workspace, size_t workspace_bytes, int64_t rows, int64_t D,
@@ -207,6 +209,28 @@ NV_API nv_status nv_rope_yarn_freqs(int32_t dims, float base, float factor,
                                     float* freqs, float* mscale);
 
 /*
+ * rope_suscaled_freqs -- SuScaled (LongRoPE) frequency scaling for nv_rope's `freqs`:
+ * docs.rs nuvec-core 0.5.0, Enum FastOp, variant Rope names it (frequency scaling by
+ * SuScaledRoPE) without parameters or formula; read as the published method (Ding et al.,
+ * "LongRoPE: Extending LLM Context Window Beyond 2 Million Tokens", 2024) in the form of the
+ * Phi-3 models (Abdin et al., "Phi-3 Technical Report", 2024).  Every pair i has its own
+ * rescale factor lambda_i and turns at theta_i / lambda_i, theta_i = base^(-2i/dims); the
+ * factors are long_factors when seq_len > original_max_position, else short_factors.
+ * Extending the original context L to max_position L' also scales the rotated q and k by
+ * the attention factor mscale = sqrt(1 + ln(L'/L) / ln L) when L' > L (1 otherwise); this
+ * library does not apply it (multiply q and k, or the logits by its square).
+ * short_factors, long_factors [dims / 2], freqs [dims / 2] and mscale are HOST memory
+ * (copy freqs to the device for nv_rope); mscale may be NULL.  Computed in double on the
+ * host, rounded once.  Needs dims even >= 2, base > 0, the chosen factors finite and > 0,
+ * original_max_position >= 2, max_position >= 1, seq_len >= 0 (else NV_ERR_INVALID_ARG).
+ * Needs no GPU.
+ */
+NV_API nv_status nv_rope_suscaled_freqs(int32_t dims, float base, const float* short_factors,
+                                        const float* long_factors, int64_t seq_len,
+                                        int64_t max_position, int64_t original_max_position,
+                                        float* freqs, float* mscale);
+
+/*
  * allreduce_add_rms_norm -- the step a tensor-parallel decoder takes after a row-parallel
  * layer: miniVLLM Layers page, section Linear layers, RowParallelLinear (the forward pass
  * sums the ranks' partial outputs with an all_reduce), then the fused residual add +
@@ -229,6 +253,62 @@ NV_API nv_status nv_allreduce_add_rms_norm(const void* const* parts, int32_t npa
                                            const void* r, const void* w, void* y, void* h,
                                            void* x_out, int64_t rows, int64_t D, float eps,
                                            nv_dtype dt, nv_stream_t stream);
+
+/*
+ * allreduce_add_rms_norm_peers -- the one-shot form of nv_allreduce_add_rms_norm for ranks
+ * that read each other's partials directly (same page and sections).  Every rank keeps its
+ * partial output in its own device buffer, which the other ranks have mapped into their
+ * processes (nv_ipc_export / nv_ipc_import), and a flag array of one int64 per rank in its
+ * own device memory, also mapped by the others.  Per step `epoch` (1, 2, 3, ... on every
+ * rank in lockstep) each rank, after producing its partial on `stream`, calls
+ * nv_tp_publish, which stores `epoch` into its slot of every rank's flag array; then this
+ * call waits on the device until every slot of this rank's `flags` [nparts] has reached
+ * `epoch` and computes exactly what nv_allreduce_add_rms_norm computes, reading the parts
+ * (this rank's own buffer and the mapped peers', in rank order) with plain loads.  The wait
+ * is bounded (about a second per CTA): if a peer never publishes, each CTA that gave up
+ * counts a fault (nv_fault_count) and leaves its rows unwritten; no error is returned by the
+ * launch itself.  A rank must not overwrite the partial of step e before every rank's call
+ * of step e has read it: write step e + 1 into a second buffer (double buffering) on the
+ * same stream, after this call -- a peer then publishes e + 1 only after its own step-e call
+ * has finished, and this rank's step e + 1 call waits for that before step e + 2 reuses the
+ * first buffer.  flags: 8-byte aligned device memory of the current device, zero before the
+ * first step.  Errors: as nv_allreduce_add_rms_norm, plus NV_ERR_INVALID_ARG for a NULL or
+ * misaligned flags array or epoch < 1.
+ */
+NV_API nv_status nv_allreduce_add_rms_norm_peers(const void* const* parts, int32_t nparts,
+                                                 const void* r, const void* w, void* y, void* h,
+                                                 void* x_out, int64_t rows, int64_t D, float eps,
+                                                 nv_dtype dt, const int64_t* flags, int64_t epoch,
+                                                 nv_stream_t stream);
+
+/*
+ * tp_publish -- the publishing half of nv_allreduce_add_rms_norm_peers: after everything
+ * queued on `stream` before it (this rank's partial of step `epoch`) has completed, a
+ * system-scope fence and then one release store of `epoch` into slot `rank` of each of the
+ * `world` flag arrays (flags[p]: rank p's array of `world` int64, this rank's own or a mapped
+ * peer's).  world 1..8, 0 <= rank < world, epoch >= 1, each flags[p] 8-byte aligned device
+ * memory (else NV_ERR_INVALID_ARG).
+ */
+NV_API nv_status nv_tp_publish(int64_t* const* flags, int32_t world, int32_t rank, int64_t epoch,
+                               nv_stream_t stream);
+
+/* Bytes of a device-memory handle for another process (cudaIpcMemHandle_t). */
+#define NV_IPC_HANDLE_BYTES 64
+
+/*
+ * ipc_export / ipc_import / ipc_close -- sharing device buffers between the processes of
+ * one node (CUDA IPC), for nv_allreduce_add_rms_norm_peers.  nv_ipc_export writes the
+ * handle (NV_IPC_HANDLE_BYTES bytes, host memory) of the allocation holding `ptr` and the
+ * offset of `ptr` inside it; another process passes both to nv_ipc_import, which maps the
+ * allocation (with peer access enabled on demand) and returns the matching pointer there,
+ * and later to nv_ipc_close with that pointer.  The handle is plain bytes: send it over
+ * any channel (for example a process-group all-gather of objects).  Errors: NV_ERR_INVALID_ARG
+ * for NULL arguments or a pointer outside any allocation, NV_ERR_CUDA when the runtime
+ * refuses (for example importing a handle in the process that exported it).
+ */
+NV_API nv_status nv_ipc_export(const void* ptr, void* handle, uint64_t* offset);
+NV_API nv_status nv_ipc_import(const void* handle, uint64_t offset, void** ptr);
+NV_API nv_status nv_ipc_close(void* ptr, uint64_t offset);
 
 /*
  * add_rms_norm_host -- add_rms_norm (as nv_add_rms_norm) on rows that live in host
@@ -263,13 +343,16 @@ NV_API nv_status nv_add_rms_norm_host(const void* x_host, const void* r_host, co
  * that the library declares (every GPU that loads the library holds it until the process
  * exits).  Nothing is allocated, and nothing needs clearing: each call writes every
  * partial row it later reads.
- *   - Limit: D <= 16384 (and the limits of nv_rms_norm_vjp); a larger D returns
- *     NV_ERR_UNSUPPORTED.  The number of partial rows is min(rows, 512, 2^20 / D), so dw
- *     can differ from nv_rms_norm_vjp's in the last bits (another summation grouping);
- *     dx is the same.
+ *   - Limits: D <= 16384, D a multiple of 16 bytes of elements (8 bf16, 4 float32),
+ *     float32 D <= 8192, 16-byte aligned x, g, dx and w (the register kernels only);
+ *     other shapes return NV_ERR_UNSUPPORTED.  The number of partial rows is
+ *     min(rows, SMs x resident CTAs per SM, max(512, 2^21 / D), 2^20 / D) -- at most
+ *     2^20 / D, which is 64 at D = 16384 -- so dw can differ from nv_rms_norm_vjp's in the
+ *     last bits (another summation grouping); dx is the same.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call before any
- *     stream capture.
+ *     stream capture.  The address is kept per device and CUDA context: after a device
+ *     reset (a new context) the next call looks it up again.
  *   - All calls share the one array: two calls whose kernels overlap on the GPU (on
  *     different streams without ordering) race and may corrupt each other's dw.
  */
@@ -327,14 +410,26 @@ NV_API nv_status nv_selftest_bounded_wait(int32_t ctas, nv_stream_t stream);
  *                   it waits for that kernel (griddepcontrol.wait) before reading or
  *                   writing any global memory, so results are the same as with a plain
  *                   launch; NV_LAUNCH_PLAIN: ordinary stream-ordered launch.
+ *   stages          NV_PATH_RING: shared-memory row buffers per CTA (0 = as many as fit,
+ *                   at most 32; a multiple of rows_per_cta, at least 2 x rows_per_cta).  norm_rope, two vectors per
+ *                   lane: 1 = the compensated (error-free) rotation on every pair instead
+ *                   of the float32 rotation with a per-pair error test and compensated
+ *                   recomputation of the pairs that fail it (same results within the
+ *                   tolerance).  Other paths: must be 0.
+ * For NV_PATH_RING, threads_per_row is the size of a row group (32 x warps, <= 256),
+ * rows_per_cta the row groups of a CTA (rows reduced at once), ctas_per_sm the CTAs per
+ * SM (0 = 1), vec_per_thread must be 0.
  */
 typedef enum {
     NV_PATH_AUTO = 0,
     NV_PATH_ROWS = 1,    /* row held in registers, 16-byte vector loads */
     NV_PATH_GENERIC = 2, /* any D and alignment: scalar loop, two passes over the row */
-    NV_PATH_STAGED = 3   /* persistent, rows staged in shared memory by bulk async copies;
+    NV_PATH_STAGED = 3,  /* persistent, rows staged in shared memory by bulk async copies;
                             rms_norm, add_rms_norm and layer_norm.  rows_per_cta = rows in
                             flight per CTA (shared-memory stages), ctas_per_sm = CTAs per SM */
+    NV_PATH_RING = 4     /* layer_norm: persistent CTAs of several row groups (a few warps
+                            each, reducing one row at a time) fed by a ring of shared-memory
+                            row buffers that bulk async copies refill as rows finish */
 } nv_path;
 
 typedef enum { NV_LAUNCH_DEFAULT = 0, NV_LAUNCH_PLAIN = 1 } nv_launch;
@@ -346,6 +441,7 @@ typedef struct {
     int32_t rows_per_cta;
     int32_t ctas_per_sm;
     int32_t launch;
+    int32_t stages;
 } nv_plan;
 
 NV_API nv_status nv_rms_norm_ex(const void* x, const void* w, void* y, int64_t rows, int64_t D,

@@ -19,13 +19,16 @@ import torch
 __all__ = [
     "NvError", "Plan", "library", "library_path",
     "nv_rms_norm", "nv_add_rms_norm", "nv_add_rms_norm_host", "nv_allreduce_add_rms_norm",
-    "allreduce_add_rms_norm", "rope_llama3_freqs", "rope_yarn_freqs", "nv_layer_norm", "nv_norm_rope",
+    "nv_allreduce_add_rms_norm_peers", "nv_tp_publish", "ipc_export", "ipc_import", "ipc_close",
+    "allreduce_add_rms_norm", "rope_llama3_freqs", "rope_yarn_freqs", "rope_suscaled_freqs",
+    "nv_layer_norm", "nv_norm_rope",
     "nv_describe_plan",
     "nv_fault_count", "nv_selftest_bounded_wait",
     "nv_rope", "rms_norm", "add_rms_norm", "layer_norm", "norm_rope", "norm_rope_into_cache",
     "rope", "nv_rms_norm_vjp", "nv_layer_norm_vjp", "nv_norm_vjp_workspace_size", "rms_norm_vjp",
     "layer_norm_vjp",
-    "PATH_AUTO", "PATH_ROWS", "PATH_GENERIC", "PATH_STAGED", "LAUNCH_DEFAULT", "LAUNCH_PLAIN",
+    "PATH_AUTO", "PATH_ROWS", "PATH_GENERIC", "PATH_STAGED", "PATH_RING", "LAUNCH_DEFAULT",
+    "LAUNCH_PLAIN",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,7 +36,7 @@ library_path = os.path.join(_HERE, "libnvnorm.so")
 
 NV_F32, NV_BF16, NV_F16 = 0, 1, 2
 NV_OK, NV_ERR_INVALID_ARG, NV_ERR_UNSUPPORTED, NV_ERR_CUDA = 0, 1, 2, 3
-PATH_AUTO, PATH_ROWS, PATH_GENERIC, PATH_STAGED = 0, 1, 2, 3
+PATH_AUTO, PATH_ROWS, PATH_GENERIC, PATH_STAGED, PATH_RING = 0, 1, 2, 3, 4
 LAUNCH_DEFAULT, LAUNCH_PLAIN = 0, 1
 
 _DT = {torch.float32: NV_F32, torch.bfloat16: NV_BF16, torch.float16: NV_F16}
@@ -52,7 +55,8 @@ class Plan(ctypes.Structure):
     """nv_plan: kernel-variant selection (0 fields mean automatic)."""
     _fields_ = [("path", ctypes.c_int32), ("vec_per_thread", ctypes.c_int32),
                 ("threads_per_row", ctypes.c_int32), ("rows_per_cta", ctypes.c_int32),
-                ("ctas_per_sm", ctypes.c_int32), ("launch", ctypes.c_int32)]
+                ("ctas_per_sm", ctypes.c_int32), ("launch", ctypes.c_int32),
+                ("stages", ctypes.c_int32)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_}
@@ -111,10 +115,26 @@ def library() -> ctypes.CDLL:
     lib.nv_rms_norm_vjp.restype = ctypes.c_int
     lib.nv_layer_norm_vjp.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, i64, i64, f32, i32, vp]
     lib.nv_layer_norm_vjp.restype = ctypes.c_int
+    lib.nv_allreduce_add_rms_norm_peers.argtypes = [ctypes.POINTER(vp), i32, vp, vp, vp, vp, vp,
+                                                    i64, i64, f32, i32, vp, i64, vp]
+    lib.nv_allreduce_add_rms_norm_peers.restype = ctypes.c_int
+    lib.nv_tp_publish.argtypes = [ctypes.POINTER(vp), i32, i32, i64, vp]
+    lib.nv_tp_publish.restype = ctypes.c_int
+    u64 = ctypes.c_uint64
+    lib.nv_ipc_export.argtypes = [vp, vp, ctypes.POINTER(u64)]
+    lib.nv_ipc_export.restype = ctypes.c_int
+    lib.nv_ipc_import.argtypes = [vp, u64, ctypes.POINTER(vp)]
+    lib.nv_ipc_import.restype = ctypes.c_int
+    lib.nv_ipc_close.argtypes = [vp, u64]
+    lib.nv_ipc_close.restype = ctypes.c_int
+    lib.nv_rms_norm_vjp_static.argtypes = [vp, vp, vp, vp, vp, i64, i64, f32, i32, vp]
+    lib.nv_rms_norm_vjp_static.restype = ctypes.c_int
     lib.nv_rope_llama3_freqs.argtypes = [i32, f32, f32, f32, f32, i64, vp]
     lib.nv_rope_llama3_freqs.restype = ctypes.c_int
     lib.nv_rope_yarn_freqs.argtypes = [i32, f32, f32, i64, f32, f32, vp, vp]
     lib.nv_rope_yarn_freqs.restype = ctypes.c_int
+    lib.nv_rope_suscaled_freqs.argtypes = [i32, f32, vp, vp, i64, i64, i64, vp, vp]
+    lib.nv_rope_suscaled_freqs.restype = ctypes.c_int
     lib.nv_norm_vjp_workspace_size.argtypes = [i32, i64, i64]
     lib.nv_norm_vjp_workspace_size.restype = sz
     _lib = lib
@@ -226,6 +246,26 @@ def rope_yarn_freqs(dims, base=10000.0, factor=4.0, original_max_position=4096, 
     return out, m.value
 
 
+def rope_suscaled_freqs(dims, short_factors, long_factors, seq_len, base=10000.0,
+                        max_position=131072, original_max_position=4096):
+    """SuScaled (LongRoPE) RoPE frequencies (a float32 host tensor of dims/2, for
+    ``nv_rope(..., freqs=...)`` after ``.cuda()``): the long factors when seq_len exceeds
+    the original context, else the short ones; and the attention factor mscale, which the
+    caller applies to q and k."""
+    sf = torch.as_tensor(short_factors, dtype=torch.float32).contiguous()
+    lf = torch.as_tensor(long_factors, dtype=torch.float32).contiguous()
+    if sf.numel() != dims // 2 or lf.numel() != dims // 2:
+        raise ValueError("short_factors and long_factors must hold dims / 2 values")
+    out = torch.empty(dims // 2, dtype=torch.float32)
+    m = ctypes.c_float(0.0)
+    st = library().nv_rope_suscaled_freqs(dims, base, ctypes.c_void_p(sf.data_ptr()),
+                                          ctypes.c_void_p(lf.data_ptr()), seq_len, max_position,
+                                          original_max_position, ctypes.c_void_p(out.data_ptr()),
+                                          ctypes.byref(m))
+    _check("nv_rope_suscaled_freqs", st)
+    return out, m.value
+
+
 def nv_allreduce_add_rms_norm(parts, r, w, y, h, eps, x_out=None, stream=None):
     """x = sum(parts) (in order, in double, rounded once), h = x + r, y = RmsNorm(h) * w.
     ``parts`` are device tensors shaped like r (this GPU's, or peers' mapped buffers)."""
@@ -236,6 +276,55 @@ def nv_allreduce_add_rms_norm(parts, r, w, y, h, eps, x_out=None, stream=None):
                                        _ptr(x_out), rows, D, eps,
                                        _dtype(*parts, r, w, y, h, x_out), _stream(stream))
     _check("nv_allreduce_add_rms_norm", st)
+
+
+def nv_allreduce_add_rms_norm_peers(part_ptrs, r, w, y, h, eps, flags, epoch, x_out=None,
+                                    stream=None):
+    """The one-shot form: ``part_ptrs`` are device addresses (ints) of every rank's partial,
+    shaped and typed like r (this rank's own buffer and peers' mapped ones, rank order);
+    waits on the device until every slot of ``flags`` (an int64 device tensor, one slot per
+    rank) reaches ``epoch``, then computes as nv_allreduce_add_rms_norm."""
+    rows, D = _rows_D(r)
+    table = (ctypes.c_void_p * len(part_ptrs))(*[int(p) for p in part_ptrs])
+    st = library().nv_allreduce_add_rms_norm_peers(
+        table, len(part_ptrs), _ptr(r), _ptr(w), _ptr(y), _ptr(h), _ptr(x_out), rows, D, eps,
+        _dtype(r, w, y, h, x_out), _ptr(flags), epoch, _stream(stream))
+    _check("nv_allreduce_add_rms_norm_peers", st)
+
+
+def nv_tp_publish(flag_ptrs, rank, epoch, stream=None):
+    """Store ``epoch`` into slot ``rank`` of every rank's flag array (device addresses, rank
+    order) once the work queued before on the stream is complete."""
+    table = (ctypes.c_void_p * len(flag_ptrs))(*[int(p) for p in flag_ptrs])
+    _check("nv_tp_publish", library().nv_tp_publish(table, len(flag_ptrs), rank, epoch,
+                                                     _stream(stream)))
+
+
+IPC_HANDLE_BYTES = 64
+
+
+def ipc_export(t):
+    """(handle bytes, offset) that another process of this node passes to ipc_import to map
+    the device memory of tensor ``t``."""
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    off = ctypes.c_uint64(0)
+    _check("nv_ipc_export", library().nv_ipc_export(ctypes.c_void_p(t.data_ptr()), buf,
+                                                    ctypes.byref(off)))
+    return buf.raw, off.value
+
+
+def ipc_import(handle, offset):
+    """Device address, in this process, of the memory another process exported."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle is 64 bytes")
+    out = ctypes.c_void_p(0)
+    _check("nv_ipc_import", library().nv_ipc_import(ctypes.create_string_buffer(handle, 64),
+                                                    offset, ctypes.byref(out)))
+    return out.value
+
+
+def ipc_close(ptr, offset):
+    _check("nv_ipc_close", library().nv_ipc_close(ctypes.c_void_p(ptr), offset))
 
 
 def allreduce_add_rms_norm(parts, r, w, eps=1e-5):

@@ -11,14 +11,64 @@
 // memory (an all-gather), or other GPUs' buffers mapped into this process.  Each element
 // of every part is read once and x is never re-read, so one pass reads (nparts + 1) rows
 // and writes two or three.
+//
+// One-shot form over peers' memory: each rank keeps its partial in its own buffer, which
+// the other ranks have mapped (CUDA IPC).  After producing the partial of step `epoch`, a
+// rank publishes that epoch into a flag slot of every rank (tp_publish_kernel: a
+// system-scope fence, then a release store per rank); the fused kernel of every rank first
+// waits until all flags of its own array have reached the epoch (acquire loads, bounded to
+// about a second, one thread per CTA), then reads the peers' partials directly with plain
+// loads -- no copy, no multicast.  A wait that runs out counts a fault (nv_fault_count)
+// and the CTA leaves without touching its rows.
 #pragma once
 
 #include "common.cuh"
 #include "rms.cuh"
+#include "staged.cuh"
 
 namespace nvn {
 
 constexpr int kMaxParts = 8;
+
+__device__ __forceinline__ long long ld_acquire_sys(const long long* p) {
+    long long v;
+    asm volatile("ld.acquire.sys.global.s64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_sys(long long* p, long long v) {
+    asm volatile("st.release.sys.global.s64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Wait until flags[0..n) all reach `epoch`; false once ~kWaitLimitNs have passed (or after
+// an iteration cap).  One thread.
+__device__ __forceinline__ bool wait_flags(const long long* flags, int n, long long epoch) {
+    const uint64_t t0 = global_ns();
+    uint32_t i = 0;
+    for (int p = 0; p < n; ++p) {
+        while (ld_acquire_sys(flags + p) < epoch) {
+            if (++i >= (1u << 26)) return false;
+            if ((i & 63u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
+            __nanosleep(64);
+        }
+    }
+    return true;
+}
+
+struct PublishArgs {
+    long long* flags[kMaxParts];  // every rank's flag array (this rank's own, and mapped)
+    int world;
+    int rank;
+    long long epoch;
+};
+
+// Publish `epoch` in slot `rank` of every rank's flag array, after everything queued
+// before on the stream (the partial) is complete and visible system-wide.
+__global__ void __launch_bounds__(32) tp_publish_kernel(const PublishArgs a) {
+    pdl_wait();
+    if (threadIdx.x != 0) return;
+    __threadfence_system();
+    for (int p = 0; p < a.world; ++p) st_release_sys(a.flags[p] + a.rank, a.epoch);
+}
 
 struct ReduceNormArgs {
     const void* parts[kMaxParts];
@@ -33,7 +83,21 @@ struct ReduceNormArgs {
     int nvec;     // 16-byte vectors per row (register path)
     int G;        // threads per row (register path)
     float eps;
+    const long long* flags;  // NULL, or this rank's flag array [nparts]: wait for `epoch`
+    long long epoch;
 };
+
+// The one-shot form's wait (a no-op without flags): false when this CTA must leave.
+__device__ __forceinline__ bool peers_ready(const ReduceNormArgs& a) {
+    if (!a.flags) return true;
+    bool ok = true;
+    if (threadIdx.x == 0) ok = wait_flags(a.flags, a.nparts, a.epoch);
+    if (__syncthreads_or(ok ? 0 : 1)) {
+        if (threadIdx.x == 0) atomicAdd(&nvn_fault_count, 1u);
+        return false;
+    }
+    return true;
+}
 
 template <typename T>
 __device__ __forceinline__ float round_io(double v);
@@ -51,6 +115,7 @@ template <typename T, int VPT>
 __global__ void __launch_bounds__(1024) allreduce_rms_rows_kernel(const ReduceNormArgs a) {
     pdl_wait();
     pdl_release();
+    if (!peers_ready(a)) return;
     using E = Elem<T>;
     constexpr int VEC = E::kVec;
     __shared__ float red[2][32];
@@ -127,6 +192,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) allreduce_rms_generic_kernel(const ReduceNormArgs a) {
     pdl_wait();
     pdl_release();
+    if (!peers_ready(a)) return;
     using E = Elem<T>;
     __shared__ float red[2][32];
     const int nw = blockDim.x >> 5;

@@ -17,6 +17,7 @@
 #include "allreduce.cuh"
 #include "common.cuh"
 #include "layer.cuh"
+#include "layer_ring.cuh"
 #include "rms.cuh"
 #include "rope.cuh"
 #include "staged.cuh"
@@ -76,20 +77,31 @@ nv_status current_device(int* dev, DevInfo* info) {
 }
 
 // ---- pointer checks ----------------------------------------------------------------------
-// cuMemGetAddressRange, fetched through the runtime so the library needs no libcuda link.
+// Driver entry points, fetched through the runtime so the library needs no libcuda link.
+template <typename F>
+F driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    F fn = nullptr;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        fn = reinterpret_cast<F>(p);
+    cudaGetLastError();
+    return fn;
+}
+
+// cuPointerGetAttributes answers every question the check asks (memory type, device,
+// managed or not, the allocation's range) in one driver call per pointer.
+using AttrsFn = CUresult (*)(unsigned int, CUpointer_attribute*, void**, CUdeviceptr);
+AttrsFn attrs_fn() {
+    static AttrsFn fn = driver_fn<AttrsFn>("cuPointerGetAttributes");
+    return fn;
+}
+
+// cuMemGetAddressRange, for the checks of peers' parts and of page-locked host buffers.
 using RangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
 RangeFn range_fn() {
-    static RangeFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<RangeFn>(p);
-        cudaGetLastError();
-    });
+    static RangeFn fn = driver_fn<RangeFn>("cuMemGetAddressRange");
     return fn;
 }
 
@@ -104,31 +116,35 @@ struct Buf {
 // The buffer must be device (or managed) memory of the current device and lie inside
 // one allocation.
 nv_status check_pointer(const Buf& b, int dev) {
-    cudaPointerAttributes at;
-    cudaError_t e = cudaPointerGetAttributes(&at, b.p);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return fail(NV_ERR_INVALID_ARG, "%s (%p) is not a CUDA pointer: %s", b.name, b.p,
-                    cudaGetErrorString(e));
-    }
-    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged)
+    AttrsFn fn = attrs_fn();
+    if (!fn) return fail(NV_ERR_CUDA, "the driver does not provide cuPointerGetAttributes");
+    unsigned int mtype = 0;
+    int ordinal = -1;
+    uint64_t managed = 0;  // the driver writes a bool into the first byte
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    CUpointer_attribute which[5] = {CU_POINTER_ATTRIBUTE_MEMORY_TYPE,
+                                    CU_POINTER_ATTRIBUTE_DEVICE_ORDINAL,
+                                    CU_POINTER_ATTRIBUTE_IS_MANAGED,
+                                    CU_POINTER_ATTRIBUTE_RANGE_START_ADDR,
+                                    CU_POINTER_ATTRIBUTE_RANGE_SIZE};
+    void* out[5] = {&mtype, &ordinal, &managed, &base, &size};
+    // an address the driver does not know comes back as success with empty attributes
+    if (fn(5, which, out, (CUdeviceptr)(uintptr_t)b.p) != CUDA_SUCCESS || mtype == 0)
+        return fail(NV_ERR_INVALID_ARG, "%s (%p) is not a CUDA pointer", b.name, b.p);
+    const bool is_managed = (managed & 0xFFu) != 0;
+    if (!is_managed && mtype != CU_MEMORYTYPE_DEVICE)
         return fail(NV_ERR_INVALID_ARG, "%s (%p) is not device memory", b.name, b.p);
-    if (at.type == cudaMemoryTypeDevice && at.device != dev)
+    if (!is_managed && ordinal != dev)
         return fail(NV_ERR_INVALID_ARG, "%s (%p) belongs to device %d, current device is %d",
-                    b.name, b.p, at.device, dev);
-    RangeFn fn = range_fn();
-    if (fn) {
-        CUdeviceptr base = 0;
-        size_t size = 0;
-        if (fn(&base, &size, (CUdeviceptr)(uintptr_t)b.p) != CUDA_SUCCESS)
-            return fail(NV_ERR_INVALID_ARG, "%s (%p): allocation not found", b.name, b.p);
-        const uintptr_t lo = (uintptr_t)b.p;
-        if (lo + b.bytes > (uintptr_t)base + size)
-            return fail(NV_ERR_INVALID_ARG,
-                        "%s (%p): %zu bytes run past the end of its allocation "
-                        "(%zu bytes at %p)",
-                        b.name, b.p, b.bytes, size, (void*)(uintptr_t)base);
-    }
+                    b.name, b.p, ordinal, dev);
+    if (size == 0)
+        return fail(NV_ERR_INVALID_ARG, "%s (%p): allocation not found", b.name, b.p);
+    const uintptr_t lo = (uintptr_t)b.p;
+    if (lo + b.bytes > (uintptr_t)base + size)
+        return fail(NV_ERR_INVALID_ARG,
+                    "%s (%p): %zu bytes run past the end of its allocation (%zu bytes at %p)",
+                    b.name, b.p, b.bytes, size, (void*)(uintptr_t)base);
     return NV_OK;
 }
 
@@ -225,6 +241,60 @@ size_t staged_smem(Op op, int64_t D, nv_dtype dt, int stages) {
 }
 constexpr int kStaticSmemReserve = 2048;  // static shared memory + per-CTA system use
 
+// Ring path shape (layer_norm): R warps per row group so that a thread holds about eight
+// 16-byte vectors of a row; 16 warps per CTA in row groups; then as many row buffers as
+// the shared memory holds (at most 32) in a multiple of the group count, at least two per
+// group, with w and b as a float32 table when it takes at most 64 KB.  Requested fields
+// are kept.  The multiple matters for correctness: row k uses buffer k mod stages and
+// belongs to group k mod groups, so each buffer serves one group only, and that group
+// waits on the buffer's phases strictly in order -- a parity wait can never be answered by
+// the completion of an earlier phase meant for another group.
+bool ring_shape(int nvec, int vecw, const nv_plan& p, const DevInfo* di, RingArgs* out) {
+    RingArgs r{};
+    if (p.vec_per_thread != 0) return false;
+    if (p.threads_per_row != 0) {
+        if (p.threads_per_row % 32 != 0 || p.threads_per_row < 32 || p.threads_per_row > 256)
+            return false;
+        r.R = p.threads_per_row / 32;
+    } else {
+        r.R = std::min(8, std::max(1, (nvec + 255) / 256));
+    }
+    const int optin = di ? di->smem_optin : 232448;
+    const int per_sm = di ? di->smem_per_sm : 233472;
+    const int cps = p.ctas_per_sm > 0 ? p.ctas_per_sm : 1;
+    const int64_t budget = std::min(optin, per_sm / cps) - kStaticSmemReserve;
+    const int64_t row = (int64_t)nvec * 16;
+    const int64_t table = (int64_t)ring_table_bytes(nvec, vecw);
+    const int want_groups = p.rows_per_cta > 0 ? p.rows_per_cta : std::max(1, 16 / r.R);
+    if (want_groups * r.R > 16) return false;  // CTAs of at most 512 threads
+    // fixed bytes besides the buffers and the table (barriers, counts, reduction slots)
+    auto fixed = [&](int groups, int stages) {
+        RingArgs t{r.R, groups, stages, 0};
+        return (int64_t)ring_smem_bytes(nvec, vecw, t) - (int64_t)stages * row;
+    };
+    for (int wb = 1; wb >= 0; --wb) {
+        if (wb && table > 64 * 1024) continue;
+        const int64_t room = budget - (wb ? table : 0) - fixed(want_groups, 32);
+        int64_t smax = std::min<int64_t>(room / row, 32);
+        int groups = want_groups;
+        if (p.stages > 0) {
+            if (p.stages > smax || p.stages % groups != 0 || p.stages < 2 * groups) continue;
+            smax = p.stages;
+        } else {
+            if (p.rows_per_cta == 0) groups = (int)std::min<int64_t>(groups, smax / 2);
+            if (groups < 1) continue;
+            smax = smax / groups * groups;
+        }
+        if (smax < 2 * groups) continue;
+        r.groups = groups;
+        r.stages = (int)smax;
+        r.wb_smem = wb;
+        *out = r;
+        return true;
+    }
+    return false;
+}
+
 nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, const nv_plan* req,
                     nv_plan* out, const DevInfo* di = nullptr) {
     nv_plan p{};
@@ -277,9 +347,24 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
         if (p.rows_per_cta < 2 || staged_smem(op, D, dt, p.rows_per_cta) > (size_t)budget)
             return fail(NV_ERR_UNSUPPORTED, "staged path: %d stages of %zu bytes do not fit "
                         "%d bytes of shared memory", p.rows_per_cta, one, budget);
+    } else if (p.path == NV_PATH_RING && op == OP_LAYER) {
+        if (!vec_ok) return fail(NV_ERR_UNSUPPORTED, "ring path needs D %% %d == 0 and "
+                                 "16-byte aligned pointers", vecw);
+        RingArgs rg{};
+        if (!ring_shape(nvec, vecw, p, di, &rg))
+            return fail(NV_ERR_UNSUPPORTED, "ring path: no shape for D = %lld (group %d threads, "
+                        "%d groups, %d stages)", (long long)D, p.threads_per_row, p.rows_per_cta,
+                        p.stages);
+        p.vec_per_thread = 0;
+        p.threads_per_row = 32 * rg.R;
+        p.rows_per_cta = rg.groups;
+        p.stages = rg.stages;
+        if (p.ctas_per_sm == 0) p.ctas_per_sm = 1;
     } else {
         return fail(NV_ERR_UNSUPPORTED, "path %d is not available for this op", p.path);
     }
+    if (p.path != NV_PATH_RING && p.stages != 0)
+        return fail(NV_ERR_UNSUPPORTED, "stages is for the ring path only");
     if (p.ctas_per_sm < 0) return fail(NV_ERR_INVALID_ARG, "ctas_per_sm < 0");
     (void)rows;
     *out = p;
@@ -378,6 +463,19 @@ template <typename T>
 nv_status run_layer(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs a) {
     if (p.path == NV_PATH_GENERIC)
         return launch(layer_generic_kernel<T>, a.rows, 256, 0, p.ctas_per_sm, di, s, a);
+    if (p.path == NV_PATH_RING) {
+        constexpr int vecw = 16 / sizeof(T);
+        RingArgs rg{};
+        if (!ring_shape(a.nvec, vecw, p, &di, &rg))
+            return fail(NV_ERR_UNSUPPORTED, "ring path: no shape");
+        const size_t smem = ring_smem_bytes(a.nvec, vecw, rg);
+        auto kern = rg.wb_smem ? layer_ring_kernel<T, true> : layer_ring_kernel<T, false>;
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        const int64_t grid = grid_for(a.rows, di.sms, std::max(1, p.ctas_per_sm));
+        return launch_kernel(kern, grid, 32 * rg.R * rg.groups, smem, s, a, rg);
+    }
     if (p.path == NV_PATH_STAGED) {
         const size_t smem = staged_smem(OP_LAYER, a.D, sizeof(T) == 4 ? NV_F32 : NV_BF16,
                                         p.rows_per_cta);
@@ -485,18 +583,21 @@ nv_status row_dispatch(Op op, const nv_plan& p, const DevInfo& di, nv_dtype dt, 
 struct RopePlan {
     bool rows;
     bool pairs;  // two vectors per lane: rope_pairs_kernel (dims == D)
+    bool exact;  // pairs kernel: the compensated rotation on every pair
     int lpr;
     int bt;
     int64_t n_chunks;
 };
 
 template <typename T, bool TRAD>
-nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a, bool pairs) {
+nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a, bool pairs,
+                           bool exact) {
     // the pairs kernel keeps its lanes' weights after the table: VEC/2 records per lane
     const size_t smem = (size_t)a.half * sizeof(float4) +
                         (pairs ? (size_t)Elem<T>::kVec / 2 * (size_t)(a.nvec / 2) * sizeof(float4)
                                : 0);
-    auto kern = pairs ? rope_pairs_kernel<T, TRAD> : rope_rows_kernel<T, TRAD>;
+    auto kern = !pairs ? rope_rows_kernel<T, TRAD>
+                       : exact ? rope_pairs_kernel<T, TRAD, true> : rope_pairs_kernel<T, TRAD, false>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -529,6 +630,10 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
     if (p.path == NV_PATH_AUTO) p.path = (vec_ok || pairs_ok) ? NV_PATH_ROWS : NV_PATH_GENERIC;
     rp->rows = p.path == NV_PATH_ROWS;
     rp->pairs = rp->rows && pairs_ok && p.vec_per_thread != 1;
+    if (p.stages != 0 && !(p.stages == 1 && rp->pairs))
+        return fail(NV_ERR_UNSUPPORTED, "norm_rope: stages = 1 (the compensated rotation on "
+                    "every pair) needs the two-vectors-per-lane register path");
+    rp->exact = p.stages == 1;
     if (p.path == NV_PATH_ROWS) {
         if (!vec_ok && !rp->pairs)
             return fail(NV_ERR_UNSUPPORTED, "norm_rope register path needs D %% %d == 0, "
@@ -643,10 +748,10 @@ nv_status rope_op(const void* x, const void* w, const float* freqs, void* y, int
     const bool bf = dt == NV_BF16;
     if (rp.rows) {
         if (traditional)
-            return bf ? launch_rope_rows<__nv_bfloat16, true>(di, cs, a, rp.pairs)
-                      : launch_rope_rows<float, true>(di, cs, a, rp.pairs);
-        return bf ? launch_rope_rows<__nv_bfloat16, false>(di, cs, a, rp.pairs)
-                  : launch_rope_rows<float, false>(di, cs, a, rp.pairs);
+            return bf ? launch_rope_rows<__nv_bfloat16, true>(di, cs, a, rp.pairs, rp.exact)
+                      : launch_rope_rows<float, true>(di, cs, a, rp.pairs, rp.exact);
+        return bf ? launch_rope_rows<__nv_bfloat16, false>(di, cs, a, rp.pairs, rp.exact)
+                  : launch_rope_rows<float, false>(di, cs, a, rp.pairs, rp.exact);
     }
     return bf ? launch_rope_generic<__nv_bfloat16>(di, p.ctas_per_sm, cs, a)
               : launch_rope_generic<float>(di, p.ctas_per_sm, cs, a);
@@ -676,11 +781,16 @@ nv_status check_part(const void* p, size_t bytes, int i) {
 
 nv_status allreduce_add_rms_norm(const void* const* parts, int32_t nparts, const void* r,
                                  const void* w, void* y, void* h, void* x_out, int64_t rows,
-                                 int64_t D, float eps, nv_dtype dt, nv_stream_t stream) {
+                                 int64_t D, float eps, nv_dtype dt, nv_stream_t stream,
+                                 const int64_t* flags = nullptr, int64_t epoch = 0) {
     nv_status st = check_common(rows, D, eps, dt);
     if (st != NV_OK) return st;
     if (nparts < 1 || nparts > kMaxParts)
         return fail(NV_ERR_INVALID_ARG, "nparts = %d must be 1..%d", nparts, kMaxParts);
+    if (flags && epoch < 1)
+        return fail(NV_ERR_INVALID_ARG, "epoch = %lld must be >= 1", (long long)epoch);
+    if (flags && ((uintptr_t)flags & 7u))
+        return fail(NV_ERR_INVALID_ARG, "flags must be 8-byte aligned");
     if (rows == 0) return NV_OK;
     if (!parts) return fail(NV_ERR_INVALID_ARG, "parts is NULL");
     for (int i = 0; i < nparts; ++i)
@@ -706,6 +816,7 @@ nv_status allreduce_add_rms_norm(const void* const* parts, int32_t nparts, const
     bufs[nb++] = {y, nbytes, "y", true, false};
     bufs[nb++] = {h, nbytes, "h", true, false};
     bufs[nb++] = {x_out, nbytes, "x_out", true, false};
+    bufs[nb++] = {flags, (size_t)nparts * sizeof(int64_t), "flags", false, false};
     st = check_buffers(bufs, nb, dev);
     if (st != NV_OK) return st;
     for (int i = 0; i < nparts; ++i) {  // parts are inputs: only x_out may be one of them
@@ -732,6 +843,8 @@ nv_status allreduce_add_rms_norm(const void* const* parts, int32_t nparts, const
     a.rows = rows;
     a.D = (int)D;
     a.eps = eps;
+    a.flags = reinterpret_cast<const long long*>(flags);
+    a.epoch = epoch;
     g_pdl = true;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     const bool bf = dt == NV_BF16;
@@ -960,8 +1073,9 @@ size_t vjp_workspace(Op op, int64_t rows, int64_t D) {
 template <typename T>
 nv_status run_vjp(Op op, VjpArgs a, int vpt, int cap, const DevInfo& di, cudaStream_t s,
                   void* dw, void* db) {
-    const int G = ((a.nvec + vpt - 1) / vpt + 31) / 32 * 32;
-    auto k1 = op == OP_RMS
+    const int G = vpt == 0 ? 256 : ((a.nvec + vpt - 1) / vpt + 31) / 32 * 32;
+    auto k1 = vpt == 0 ? (op == OP_RMS ? vjp_generic_kernel<T, false> : vjp_generic_kernel<T, true>)
+              : op == OP_RMS
                   ? (vpt == 1 ? rms_vjp_kernel<T, 1>
                               : vpt == 2 ? rms_vjp_kernel<T, 2> : rms_vjp_kernel<T, 4>)
                   : (vpt == 1 ? layer_vjp_kernel<T, 1>
@@ -1006,9 +1120,9 @@ nv_status vjp_op(Op op, const void* x, const void* w, const void* g, void* dx, v
                     "scalar 1, which has no gradient)");
     const size_t s = elem_size(dt);
     const int vecw = 16 / (int)s;
-    if (D % vecw != 0 || vjp_vpt(op, (int)(D / vecw)) == 0)
-        return fail(NV_ERR_UNSUPPORTED, "vjp needs D %% %d == 0 and D <= %d", vecw,
-                    2048 * vecw);
+    // the register kernels need whole 16-byte vectors (and aligned pointers, below); any
+    // other row goes to the generic kernel
+    const bool vec_ok = D % vecw == 0 && vjp_vpt(op, (int)(D / vecw)) != 0;
     const bool sums = dw || db;
     const size_t need = sums ? vjp_workspace(op, rows, D) : 0;
     if (sums && rows > 0) {
@@ -1041,7 +1155,6 @@ nv_status vjp_op(Op op, const void* x, const void* w, const void* g, void* dx, v
     if (st != NV_OK) return st;
     const bool al = (!rows || (aligned16(x) && aligned16(g) && aligned16(dx))) &&
                     (!w || aligned16(w));
-    if (!al) return fail(NV_ERR_UNSUPPORTED, "vjp needs 16-byte aligned x, g, dx and w");
 
     VjpArgs a{};
     a.x = x;
@@ -1058,7 +1171,7 @@ nv_status vjp_op(Op op, const void* x, const void* w, const void* g, void* dx, v
     a.eps = eps;
     g_pdl = true;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    const int vpt = vjp_vpt(op, a.nvec);
+    const int vpt = (vec_ok && al) ? vjp_vpt(op, a.nvec) : 0;  // 0: the generic kernel
     const int cap = vjp_parts_cap(D);
     return dt == NV_BF16 ? run_vjp<__nv_bfloat16>(op, a, vpt, cap, di, cs, dw, db)
                          : run_vjp<float>(op, a, vpt, cap, di, cs, dw, db);
@@ -1072,19 +1185,37 @@ constexpr int64_t kStaticScratchFloats = (int64_t)1 << 20;  // 4 MiB
 constexpr int64_t kStaticMaxD = 16384;
 static __device__ __align__(256) float nvn_static_scratch[kStaticScratchFloats];
 
-float* g_static_scratch[kMaxDevices] = {};
+// The address is looked up once per device and context: a device reset tears down the
+// primary context (and the module holding the array), and the next context loads it anew.
+struct StaticSlot {
+    CUcontext ctx = nullptr;
+    float* ptr = nullptr;
+};
+StaticSlot g_static_scratch[kMaxDevices];
 std::mutex g_static_mu;
 
-// Device address of the scratch array on the current device, fetched on first use.
+using CtxFn = CUresult (*)(CUcontext*);
+
+// Device address of the scratch array on the current device (and context), fetched on the
+// first call there.
 nv_status static_scratch(int dev, float** out) {
+    static CtxFn ctx_fn = driver_fn<CtxFn>("cuCtxGetCurrent");
+    if (!ctx_fn) return fail(NV_ERR_CUDA, "the driver does not provide cuCtxGetCurrent");
+    CUcontext ctx = nullptr;
+    if (ctx_fn(&ctx) != CUDA_SUCCESS) ctx = nullptr;
     std::lock_guard<std::mutex> lk(g_static_mu);
-    if (!g_static_scratch[dev]) {
+    StaticSlot& slot = g_static_scratch[dev];
+    if (!slot.ptr || !ctx || slot.ctx != ctx) {
+        // the lookup also makes the runtime's context current if nothing has yet
         void* p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, nvn_static_scratch);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
-        g_static_scratch[dev] = static_cast<float*>(p);
+        if (ctx_fn(&ctx) != CUDA_SUCCESS || !ctx)
+            return fail(NV_ERR_CUDA, "no current CUDA context on device %d", dev);
+        slot.ptr = static_cast<float*>(p);
+        slot.ctx = ctx;
     }
-    *out = g_static_scratch[dev];
+    *out = slot.ptr;
     return NV_OK;
 }
 
@@ -1308,10 +1439,122 @@ nv_status nv_rope_yarn_freqs(int32_t dims, float base, float factor,
     return NV_OK;
 }
 
+nv_status nv_rope_suscaled_freqs(int32_t dims, float base, const float* short_factors,
+                                 const float* long_factors, int64_t seq_len,
+                                 int64_t max_position, int64_t original_max_position,
+                                 float* freqs, float* mscale) {
+    if (dims < 2 || dims % 2 != 0)
+        return fail(NV_ERR_INVALID_ARG, "dims = %d must be even and >= 2", dims);
+    if (!(base > 0.f) || !std::isfinite(base))
+        return fail(NV_ERR_INVALID_ARG, "base = %g must be finite and > 0", (double)base);
+    if (original_max_position < 2)
+        return fail(NV_ERR_INVALID_ARG, "original_max_position = %lld must be >= 2",
+                    (long long)original_max_position);
+    if (max_position < 1)
+        return fail(NV_ERR_INVALID_ARG, "max_position = %lld must be >= 1", (long long)max_position);
+    if (seq_len < 0) return fail(NV_ERR_INVALID_ARG, "seq_len = %lld < 0", (long long)seq_len);
+    if (!short_factors || !long_factors)
+        return fail(NV_ERR_INVALID_ARG, "short_factors and long_factors must not be NULL");
+    if (!freqs) return fail(NV_ERR_INVALID_ARG, "freqs is NULL");
+    // the long factors once the sequence runs past the original context
+    const float* lam = seq_len > original_max_position ? long_factors : short_factors;
+    for (int32_t i = 0; i < dims / 2; ++i)
+        if (!(lam[i] > 0.f) || !std::isfinite(lam[i]))
+            return fail(NV_ERR_INVALID_ARG, "factor %d = %g must be finite and > 0", i,
+                        (double)lam[i]);
+    for (int32_t i = 0; i < dims / 2; ++i) {
+        const double th = 1.0 / std::pow((double)base, 2.0 * (double)i / (double)dims);
+        freqs[i] = (float)(th / (double)lam[i]);
+    }
+    if (mscale) {
+        const double ratio = (double)max_position / (double)original_max_position;
+        *mscale = ratio > 1.0
+                      ? (float)std::sqrt(1.0 + std::log(ratio) / std::log((double)original_max_position))
+                      : 1.f;
+    }
+    return NV_OK;
+}
+
 nv_status nv_allreduce_add_rms_norm(const void* const* parts, int32_t nparts, const void* r,
                                     const void* w, void* y, void* h, void* x_out, int64_t rows,
                                     int64_t D, float eps, nv_dtype dt, nv_stream_t stream) {
     return allreduce_add_rms_norm(parts, nparts, r, w, y, h, x_out, rows, D, eps, dt, stream);
+}
+
+nv_status nv_allreduce_add_rms_norm_peers(const void* const* parts, int32_t nparts,
+                                          const void* r, const void* w, void* y, void* h,
+                                          void* x_out, int64_t rows, int64_t D, float eps,
+                                          nv_dtype dt, const int64_t* flags, int64_t epoch,
+                                          nv_stream_t stream) {
+    if (!flags) return fail(NV_ERR_INVALID_ARG, "flags is NULL");
+    return allreduce_add_rms_norm(parts, nparts, r, w, y, h, x_out, rows, D, eps, dt, stream,
+                                  flags, epoch);
+}
+
+nv_status nv_tp_publish(int64_t* const* flags, int32_t world, int32_t rank, int64_t epoch,
+                        nv_stream_t stream) {
+    if (world < 1 || world > kMaxParts)
+        return fail(NV_ERR_INVALID_ARG, "world = %d must be 1..%d", world, kMaxParts);
+    if (rank < 0 || rank >= world)
+        return fail(NV_ERR_INVALID_ARG, "rank = %d outside 0..%d", rank, world - 1);
+    if (epoch < 1) return fail(NV_ERR_INVALID_ARG, "epoch = %lld must be >= 1", (long long)epoch);
+    if (!flags) return fail(NV_ERR_INVALID_ARG, "flags is NULL");
+    PublishArgs a{};
+    for (int p = 0; p < world; ++p) {
+        if (!flags[p]) return fail(NV_ERR_INVALID_ARG, "flags[%d] is NULL", p);
+        if ((uintptr_t)flags[p] & 7u)
+            return fail(NV_ERR_INVALID_ARG, "flags[%d] must be 8-byte aligned", p);
+        a.flags[p] = reinterpret_cast<long long*>(flags[p]);
+    }
+    int dev = 0;
+    DevInfo di;
+    nv_status st = current_device(&dev, &di);
+    if (st != NV_OK) return st;
+    for (int p = 0; p < world; ++p) {
+        st = check_part(flags[p], (size_t)world * sizeof(int64_t), p);
+        if (st != NV_OK) return st;
+    }
+    a.world = world;
+    a.rank = rank;
+    a.epoch = epoch;
+    g_pdl = true;
+    return launch_kernel(tp_publish_kernel, 1, 32, 0, reinterpret_cast<cudaStream_t>(stream), a);
+}
+
+nv_status nv_ipc_export(const void* ptr, void* handle, uint64_t* offset) {
+    if (!ptr || !handle || !offset)
+        return fail(NV_ERR_INVALID_ARG, "ptr, handle and offset must not be NULL");
+    RangeFn fn = range_fn();
+    if (!fn) return fail(NV_ERR_CUDA, "the driver does not provide cuMemGetAddressRange");
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (fn(&base, &size, (CUdeviceptr)(uintptr_t)ptr) != CUDA_SUCCESS)
+        return fail(NV_ERR_INVALID_ARG, "ptr (%p): allocation not found", ptr);
+    cudaIpcMemHandle_t hd;
+    cudaError_t e = cudaIpcGetMemHandle(&hd, (void*)(uintptr_t)base);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaIpcGetMemHandle");
+    static_assert(sizeof(hd) == NV_IPC_HANDLE_BYTES, "IPC handle size");
+    std::memcpy(handle, &hd, sizeof(hd));
+    *offset = (uint64_t)((uintptr_t)ptr - (uintptr_t)base);
+    return NV_OK;
+}
+
+nv_status nv_ipc_import(const void* handle, uint64_t offset, void** ptr) {
+    if (!handle || !ptr) return fail(NV_ERR_INVALID_ARG, "handle and ptr must not be NULL");
+    cudaIpcMemHandle_t hd;
+    std::memcpy(&hd, handle, sizeof(hd));
+    void* base = nullptr;
+    cudaError_t e = cudaIpcOpenMemHandle(&base, hd, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaIpcOpenMemHandle");
+    *ptr = static_cast<char*>(base) + offset;
+    return NV_OK;
+}
+
+nv_status nv_ipc_close(void* ptr, uint64_t offset) {
+    if (!ptr) return fail(NV_ERR_INVALID_ARG, "ptr is NULL");
+    cudaError_t e = cudaIpcCloseMemHandle(static_cast<char*>(ptr) - offset);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaIpcCloseMemHandle");
+    return NV_OK;
 }
 
 nv_status nv_add_rms_norm_host(const void* x_host, const void* r_host, const void* w,

@@ -397,6 +397,86 @@ __global__ void __launch_bounds__(vjp_max_threads(VPT)) layer_vjp_kernel(const V
     }
 }
 
+// ---- generic kernel 1: any D, any alignment ----------------------------------------------------
+// One CTA per partial row p, walking rows p, p + parts, ...: scalar accesses, three passes
+// over the row (x and g are re-read from global memory / L1), row statistics in double.
+// The CTA's column partial sums live in its own row of the workspace, updated in place
+// after each row (it is the only writer of that row).  dx may be x or g: each thread reads
+// index j in every pass before it writes index j in the last one, and the passes of a row
+// are separated by the barriers of the reductions.
+template <int N>
+__device__ __forceinline__ void cta_sum_f64(double (&v)[N], double (*buf)[32]) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        v[i] = warp_sum(v[i]);
+        if (lane == 0) buf[i][wid] = v[i];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        double t = 0.0;
+        for (int k = 0; k < nw; ++k) t += buf[i][k];
+        v[i] = t;
+    }
+    __syncthreads();  // the buffer may be reused at once
+}
+
+template <typename T, bool LAYER>
+__global__ void __launch_bounds__(256) vjp_generic_kernel(const VjpArgs a) {
+    pdl_wait();
+    pdl_release();
+    using E = Elem<T>;
+    __shared__ double buf[3][32];
+    const int D = a.D;
+    const double invD = 1.0 / (double)D;
+    float* pdw = a.part ? a.part + (size_t)blockIdx.x * D : nullptr;
+    float* pdb = (a.part && LAYER) ? a.part + ((size_t)a.parts + blockIdx.x) * D : nullptr;
+    bool first = true;
+    for (int64_t row = blockIdx.x; row < a.rows; row += a.parts, first = false) {
+        const int64_t r0 = row * (int64_t)D;
+        double mean = 0.0;
+        if constexpr (LAYER) {
+            double s[1] = {0.0};
+            for (int j = threadIdx.x; j < D; j += blockDim.x) s[0] += (double)E::load1(a.x, r0 + j);
+            cta_sum_f64<1>(s, buf);
+            mean = s[0] * invD;
+        }
+        // RMS: sum x^2, sum g w x.  Layer: sum c^2, sum a, sum a c with c = x - mean, a = w g.
+        double s[3] = {0.0, 0.0, 0.0};
+        for (int j = threadIdx.x; j < D; j += blockDim.x) {
+            const double x = (double)E::load1(a.x, r0 + j) - mean;
+            const double wj = a.w ? (double)E::load1(a.w, j) : 1.0;
+            const double u = wj * (double)E::load1(a.g, r0 + j);
+            s[0] = fma(x, x, s[0]);
+            if constexpr (LAYER) {
+                s[1] += u;
+                s[2] = fma(u, x, s[2]);
+            } else {
+                s[1] = fma(u, x, s[1]);
+            }
+        }
+        cta_sum_f64<3>(s, buf);
+        const double r = 1.0 / sqrt(s[0] * invD + (double)a.eps);
+        // RMS: dx = r (u - x v), v = r^2 sum(u x) / D.
+        // Layer: dx = r (u - mean(a) - xh mean(a xh)), xh = c r, mean(a xh) = r sum(a c) / D.
+        const double ma = LAYER ? s[1] * invD : 0.0;
+        const double k = LAYER ? r * r * s[2] * invD : r * r * s[1] * invD;
+        for (int j = threadIdx.x; j < D; j += blockDim.x) {
+            const double x = (double)E::load1(a.x, r0 + j) - mean;
+            const double gj = (double)E::load1(a.g, r0 + j);
+            const double wj = a.w ? (double)E::load1(a.w, j) : 1.0;
+            E::store1(a.dx, r0 + j, (float)(r * (wj * gj - ma - x * k)));
+            if (pdw) {
+                const float c = (float)(gj * x * r);
+                pdw[j] = first ? c : __fadd_rn(pdw[j], c);
+            }
+            if constexpr (LAYER)
+                if (pdb) pdb[j] = first ? (float)gj : __fadd_rn(pdb[j], (float)gj);
+        }
+    }
+}
+
 // ---- kernel 2: column sums of the partials --------------------------------------------------
 // out[y][j] = sum_{p < parts} part[first + y][p][j] in double, y = blockIdx.y.
 // A CTA owns 32 columns; warp w adds parts w, w + 32, w + 64, ... in that order (eight

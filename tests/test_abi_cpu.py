@@ -91,6 +91,10 @@ def vjp(op="rms", x=FAKE, w=None, g=FAKE, dx=FAKE, dw=None, db=None, ws=None, ws
     return lib.nv_layer_norm_vjp(x, w, g, dx, dw, db, ws, ws_bytes, rows, D, eps, dt, None)
 
 
+def vjp_static(x=FAKE, w=None, g=FAKE, dx=FAKE, dw=None, rows=4, D=64, eps=1e-5, dt=BF16):
+    return nv.library().nv_rms_norm_vjp_static(x, w, g, dx, dw, rows, D, eps, dt, None)
+
+
 def allreduce(parts=(FAKE, FAKE), n=None, r=FAKE, w=None, y=FAKE, h=ctypes.c_void_p(0x20000),
               x_out=None, rows=4, D=8, eps=1e-5, dt=BF16):
     table = None if parts is None else (ctypes.c_void_p * max(len(parts), 1))(*parts)
@@ -146,8 +150,9 @@ def last_error():
     (lambda: vjp(w=FAKE, dw=FAKE), INVALID, "workspace is NULL"),
     (lambda: vjp(w=FAKE, dw=FAKE, ws=FAKE, ws_bytes=16), INVALID, "workspace of 16 bytes"),
     (lambda: vjp(op="layer", db=FAKE, ws=FAKE, ws_bytes=16), INVALID, "workspace of 16"),
-    (lambda: vjp(D=7), UNSUPPORTED, "vjp needs D"),
-    (lambda: vjp(D=32768), UNSUPPORTED, "vjp needs D"),
+    (lambda: vjp_static(D=7), UNSUPPORTED, "vjp needs D"),
+    (lambda: vjp_static(D=32768), UNSUPPORTED, "16384"),
+    (lambda: vjp_static(dw=FAKE), INVALID, "dw must be given"),
     (lambda: vjp(g=None), INVALID, "g is NULL"),
     (lambda: allreduce(n=0), INVALID, "nparts"),
     (lambda: allreduce(parts=(FAKE,) * 9), INVALID, "nparts"),
@@ -272,6 +277,45 @@ def test_rope_yarn_freqs_rejects(kw, words):
     args.update(kw)
     with pytest.raises(nv.NvError, match=words):
         nv.rope_yarn_freqs(**args)
+
+
+# ---- SuScaled (LongRoPE) frequency scaling: also a host-side helper ----------------------------
+
+def _factors(n, lo, hi, seed):
+    import numpy as np
+    return np.random.default_rng(seed).uniform(lo, hi, n).astype(np.float32)
+
+
+@pytest.mark.parametrize("dims, seq_len, max_pos, orig", [(128, 4096, 131072, 4096),
+                                                          (128, 4097, 131072, 4096),
+                                                          (96, 100000, 131072, 4096),
+                                                          (64, 10, 2048, 2048),
+                                                          (4, 0, 8192, 4096)])
+def test_rope_suscaled_freqs_matches_the_oracle(dims, seq_len, max_pos, orig):
+    import numpy as np
+    import oracle
+    sf, lf = _factors(dims // 2, 1.0, 1.2, 1), _factors(dims // 2, 1.0, 60.0, 2)
+    got, m = nv.rope_suscaled_freqs(dims, sf, lf, seq_len, 10000.0, max_pos, orig)
+    want, want_m = oracle.suscaled_freqs(dims, 10000.0, sf.astype(np.float64),
+                                         lf.astype(np.float64), float(seq_len), float(max_pos),
+                                         float(orig))
+    got, want = got.numpy(), want.astype(np.float32)
+    ulps = np.abs(got.view(np.int32).astype(np.int64) - want.view(np.int32).astype(np.int64))
+    assert ulps.max() <= 1, f"{int(ulps.max())} float ulps apart"
+    assert abs(m - want_m) <= 2.0 ** -23 * want_m
+
+
+@pytest.mark.parametrize("kw, words", [
+    (dict(dims=5), "dims"), (dict(base=-1.0), "base"), (dict(original_max_position=1), "original"),
+    (dict(max_position=0), "max_position"), (dict(seq_len=-1), "seq_len"),
+    (dict(long_factors=[1.0, 0.0]), "factor 1"), (dict(short_factors=[float("nan"), 1.0], seq_len=5),
+                                                  "factor 0")])
+def test_rope_suscaled_freqs_rejects(kw, words):
+    args = dict(dims=4, short_factors=[1.0, 1.0], long_factors=[2.0, 2.0], seq_len=9000,
+                base=10000.0, max_position=131072, original_max_position=4096)
+    args.update(kw)
+    with pytest.raises(nv.NvError, match=words):
+        nv.rope_suscaled_freqs(**args)
 
 
 @pytest.mark.skipif(__import__("torch").cuda.is_available(),

@@ -142,3 +142,74 @@ def test_a_rank_that_leaves_ends_the_next_gather_with_an_error():
     print(f"remaining rank: {name} after {took:.2f} s")
     assert name != "no error", "the gather with a departed rank must fail"
     assert took < 60
+
+
+def _peer_worker(rank, world, port, out):
+    """PeerAllReduce's host protocol on CPU: the device calls are fakes that record what
+    they are given."""
+    import datetime
+    from rope_add_rms_b200 import tp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        calls = []
+        fake_base = {r: 0x7000_0000_0000 + (r << 32) for r in range(world)}  # peers' mappings
+
+        def export(t):
+            calls.append(("export", t.data_ptr(), t.numel()))
+            return (f"handle-of-rank-{rank}".encode().ljust(64, b"\0"), 0)
+
+        def imp(handle, offset):
+            peer = int(handle.rstrip(b"\0").decode().rsplit("-", 1)[1])
+            calls.append(("import", peer, offset))
+            return fake_base[peer] + offset
+
+        lib = {"export": export, "import": imp,
+               "publish": lambda ptrs, rk, ep, stream=None: calls.append(("publish", list(ptrs), rk, ep)),
+               "reduce": lambda parts, r, w, y, h, eps, flags, ep, stream=None:
+                   calls.append(("reduce", list(parts), flags.data_ptr(), ep)),
+               "close": lambda ptr, off: calls.append(("close", ptr, off))}
+        shape = (6, 32)
+        par = tp.PeerAllReduce(shape, torch.bfloat16, device="cpu", lib=lib)
+        slots = []
+        for step in range(3):
+            slots.append(par.partial().data_ptr())
+            par(torch.zeros(shape, dtype=torch.bfloat16), None, 1e-5)
+        par.close()
+        out[rank] = (calls, par.raw.data_ptr(), par.slot_bytes, par.flags_off, slots,
+                     int(par.flags.abs().sum()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_allreduce_host_protocol_two_processes():
+    """Handles exchanged once in rank order (own memory used directly, each peer mapped
+    once and closed at the end); per step the epoch grows by one, is published into every
+    rank's flag slot before the reduction runs, and the parts are the epoch's slot of every
+    rank's buffer in rank order, the slots alternating between steps (double buffering)."""
+    world = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_peer_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    for rank in range(world):
+        calls, own, slot_bytes, flags_off, slots, flag_sum = res[rank]
+        peer = 1 - rank
+        peer_base = 0x7000_0000_0000 + (peer << 32)
+        assert flag_sum == 0, "flags start at zero"
+        assert slot_bytes == 6 * 32 * 2 and flags_off >= 2 * slot_bytes
+        assert [c[0] for c in calls[:2]] == ["export", "import"] and calls[1][1] == peer
+        bases = {rank: own, peer: peer_base}
+        steps = [c for c in calls if c[0] in ("publish", "reduce")]
+        assert [c[0] for c in steps] == ["publish", "reduce"] * 3
+        for i in range(3):
+            pub, red = steps[2 * i], steps[2 * i + 1]
+            epoch = i + 1
+            assert pub[3] == epoch and red[3] == epoch and pub[2] == rank
+            assert pub[1] == [bases[r] + flags_off for r in range(world)]
+            assert red[1] == [bases[r] + (epoch & 1) * slot_bytes for r in range(world)]
+            assert red[2] == own + flags_off, "the reduction waits on this rank's own flags"
+            assert slots[i] == own + (epoch & 1) * slot_bytes, "partial() is this step's slot"
+        assert calls[-1] == ("close", peer_base, 0)

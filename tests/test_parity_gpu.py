@@ -326,6 +326,55 @@ def test_layer_norm_in_place_and_large_mean():
     check_out(xd, ref)
 
 
+RING = [dict(path=nv.PATH_RING),
+        dict(path=nv.PATH_RING, threads_per_row=32, rows_per_cta=4),
+        dict(path=nv.PATH_RING, threads_per_row=64, rows_per_cta=3, stages=6),
+        dict(path=nv.PATH_RING, threads_per_row=128, rows_per_cta=2, stages=4),
+        dict(path=nv.PATH_RING, threads_per_row=96, rows_per_cta=1, stages=2, ctas_per_sm=2),
+        dict(path=nv.PATH_RING, threads_per_row=32, rows_per_cta=5, stages=15),
+        dict(path=nv.PATH_RING, threads_per_row=256, rows_per_cta=2)]
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("plan", RING, ids=lambda p: "-".join(f"{k}{v}" for k, v in p.items()))
+@pytest.mark.parametrize("rows,D,wb", [(147, 8192, (1, 1)), (149, 5120, (1, 0)), (33, 4096, (0, 0)),
+                                        (5, 16384, (1, 1)), (64, 512, (1, 1)), (300, 256, (0, 1)),
+                                        (1000, 2048, (1, 1)), (1, 8192, (1, 1)), (2, 8, (1, 1))])
+def test_layer_norm_ring(rows, D, wb, plan, dt):
+    """The ring path: row groups of a few warps fed by a ring of bulk-copied row buffers."""
+    inp = synth.layer_norm_inputs(rows, D, dt, seed=D + 3 * rows, weight=bool(wb[0]),
+                                  bias=bool(wb[1]))
+    x, w, b = dev(inp["x"]), dev(inp["w"]), dev(inp["b"])
+    g = Guarded(x.shape, x.dtype)
+    try:
+        nv.nv_layer_norm(x, w, b, g.t, 1e-5, plan=nv.Plan(**plan))
+    except nv.NvError as e:
+        assert e.status == nv.NV_ERR_UNSUPPORTED
+        pytest.skip(str(e))
+    torch.cuda.synchronize()
+    assert nv.nv_fault_count() == 0
+    assert g.bands_intact()
+    check_out(g.t, oracle.layer_norm(host(inp["x"]), host(inp["w"]), host(inp["b"]), 1e-5))
+
+
+@pytest.mark.parametrize("dt,mean,std", [("f32", 1e4, 1.0), ("f32", -3e5, 0.01), ("bf16", 3000.0, 40.0),
+                                          ("bf16", 3000.0, 0.25), ("f32", 0.0, 1e-30),
+                                          ("bf16", 0.5, 2.0)])
+def test_layer_norm_ring_means_and_in_place(dt, mean, std):
+    """The ring path on rows whose mean is far from zero (centred second pass, two-step
+    subtraction of the mean) and in place (y == x)."""
+    for rows, D in ((33, 4096), (300, 8192), (7, 64)):
+        x = synth.normal((rows, D), mean, std, 4, 0, dt)
+        w = synth.uniform((D,), 0.5, 1.5, 4, 2, dt)
+        b = synth.normal((D,), 0.0, 0.1, 4, 3, dt)
+        ref = oracle.layer_norm(host(x), host(w), host(b), 1e-5)
+        xd = x.cuda()
+        nv.nv_layer_norm(xd, w.cuda(), b.cuda(), xd, 1e-5, plan=nv.Plan(path=nv.PATH_RING))
+        torch.cuda.synchronize()
+        assert nv.nv_fault_count() == 0
+        check_out(xd, ref)
+
+
 # ---- norm_rope ---------------------------------------------------------------------------
 
 ROPE_CASES = [
@@ -381,7 +430,8 @@ def test_norm_rope_every_variant(D, dt):
     inp = synth.norm_rope_inputs(2, 4, 64, D, dt, seed=1)
     x, w = dev(inp["x"]), dev(inp["w"])
     plans = [dict(path=nv.PATH_GENERIC), dict(path=nv.PATH_ROWS, vec_per_thread=1),
-             dict(path=nv.PATH_ROWS, vec_per_thread=2), dict(path=nv.PATH_ROWS, rows_per_cta=3)]
+             dict(path=nv.PATH_ROWS, vec_per_thread=2), dict(path=nv.PATH_ROWS, rows_per_cta=3),
+             dict(path=nv.PATH_ROWS, vec_per_thread=2, stages=1)]
     for trad in (0, 1):
         ref = oracle.norm_rope(host(inp["x"]), host(inp["w"]), 64, D, trad, 10000.0, 1.0, 4096,
                                1, 1e-6)
@@ -395,6 +445,40 @@ def test_norm_rope_every_variant(D, dt):
                 continue
             torch.cuda.synchronize()
             check_out(y, ref, f"{p} trad={trad}")
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("trad", [0, 1])
+def test_norm_rope_near_cancellation(trad, dt):
+    """Rows built so that many rotated outputs nearly cancel: every pair (p, q) of a row is
+    a multiple of (cos phi, sin phi) of its own angle, so y_p = a_p cos - a_q sin is
+    (nearly) zero before rounding.  The float32 rotation's error test must send these pairs
+    to the compensated rotation; the results meet the same bar as everywhere."""
+    B, H, L, D = 2, 8, 64, 128
+    half = D // 2
+    offset = 4096
+    pos = offset + np.arange(L)[:, None]
+    theta = 10000.0 ** (-2.0 * np.arange(half) / D)
+    phi = pos * theta                                   # [L, half], double
+    rng = np.random.default_rng(5)
+    r = rng.uniform(0.5, 2.0, size=(B, H, L, half))
+    # (x_p, x_q) = r (sin phi, cos phi) turns to (0, r): y_p cancels
+    xp, xq = r * np.sin(phi), r * np.cos(phi)
+    x = np.empty((B, H, L, D))
+    if trad:
+        x[..., 0::2], x[..., 1::2] = xp, xq
+    else:
+        x[..., :half], x[..., half:] = xp, xq
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    xt = torch.from_numpy(x.reshape(-1, D)).to(tdt)
+    w = torch.ones(D, dtype=tdt)
+    ref = oracle.norm_rope(host(xt), host(w), L, D, trad, 10000.0, 1.0, offset, 1, 1e-6)
+    for p in (None, dict(path=nv.PATH_ROWS, vec_per_thread=2, stages=1)):
+        y = torch.empty_like(xt).cuda()
+        nv.nv_norm_rope(xt.cuda(), w.cuda(), y, L, D, trad, 10000.0, 1.0, offset, 1, 1e-6,
+                        plan=None if p is None else nv.Plan(**p))
+        torch.cuda.synchronize()
+        check_out(y, ref, f"near cancellation {p}")
 
 
 def test_norm_rope_in_place():
@@ -427,6 +511,53 @@ def test_allreduce_add_rms_norm(rows, D, nparts, dt):
     check_exact(gx.t, x, "x")
     check_exact(gh.t, h, "h")
     check_out(gy.t, y, "y")
+
+
+def test_peer_allreduce_one_rank_and_a_flag_that_never_comes():
+    """The one-shot form on one GPU (a world of one rank, where nothing waits on another
+    kernel): three steps through PeerAllReduce (publish, flag wait, slots alternating), each
+    matching the oracle; then a call whose epoch no rank ever publishes -- its bounded waits
+    run out (about a second), every CTA counts a fault and leaves its rows unwritten, and the
+    next step runs normally on the same context."""
+    import socket
+    import torch.distributed as dist
+    from rope_add_rms_b200 import tp
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        rows, D = 300, 4096
+        par = tp.PeerAllReduce((rows, D), torch.bfloat16)
+        nv.nv_fault_count(reset=True)
+
+        def step(seed):
+            inp = synth.allreduce_inputs(rows, D, 1, "bf16", seed=seed)
+            par.partial().copy_(dev(inp["parts"][0]))
+            y, h = par(dev(inp["r"]), dev(inp["w"]), 1e-5)
+            torch.cuda.synchronize()
+            y_ref, h_ref, _ = oracle.allreduce_add_rms_norm([host(inp["parts"][0])],
+                                                            host(inp["r"]), host(inp["w"]), 1e-5)
+            check_exact(h, h_ref, f"h, step {seed}")
+            check_out(y, y_ref, f"y, step {seed}")
+
+        for seed in range(3):
+            step(seed)
+        assert par.epoch == 3 and nv.nv_fault_count() == 0
+        r = torch.zeros(4, D, dtype=torch.bfloat16, device="cuda")
+        y = torch.full_like(r, 7.0)
+        h = torch.full_like(r, 7.0)
+        nv.nv_allreduce_add_rms_norm_peers([par.buf_ptrs[0]], r, None, y, h, 1e-5, par.flags,
+                                           par.epoch + 5)
+        torch.cuda.synchronize()
+        assert nv.nv_fault_count(reset=True) == 4, "one fault per CTA (one CTA per row)"
+        assert (y == 7).all() and (h == 7).all(), "rows of a CTA that gave up stay unwritten"
+        step(3)
+        assert nv.nv_fault_count() == 0
+        par.close()
+    finally:
+        dist.destroy_process_group()
 
 
 def test_allreduce_in_place_ranks_agree_and_errors():
@@ -622,7 +753,8 @@ def test_dependent_chain_across_ops_in_place():
 # ---- general rope: cache form, explicit frequencies, inverse ----------------------------------
 
 ROPE_PLANS = [None, dict(path=nv.PATH_GENERIC), dict(path=nv.PATH_ROWS, vec_per_thread=1),
-              dict(path=nv.PATH_ROWS, vec_per_thread=2)]
+              dict(path=nv.PATH_ROWS, vec_per_thread=2),
+              dict(path=nv.PATH_ROWS, vec_per_thread=2, stages=1)]
 
 
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
@@ -714,6 +846,27 @@ def test_rope_yarn_scaled_frequencies(trad):
         check_out(y, ref, f"offset {offset}")
 
 
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("trad", [0, 1])
+def test_rope_suscaled_frequencies(trad, dt):
+    """NormRope with SuScaled (LongRoPE) frequencies: the short factors within the original
+    context of 4096, the long ones past it (positions up to ~100000)."""
+    B, H, L, D = 2, 4, 64, 128
+    inp = synth.norm_rope_inputs(B, H, L, D, dt, seed=53)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    rng = np.random.default_rng(53)
+    short, long_ = rng.uniform(1.0, 1.2, D // 2), rng.uniform(1.0, 60.0, D // 2)
+    for offset in (0, 100000):
+        freqs, m = nv.rope_suscaled_freqs(D, short, long_, offset + L, 10000.0, 131072, 4096)
+        assert m > 1.0
+        y = torch.empty_like(x)
+        nv.nv_rope(x, w, y, L, D, trad, 10000.0, 1.0, offset, 1, 1e-6, freqs=freqs.cuda())
+        torch.cuda.synchronize()
+        ref = oracle.rope_ex(host(inp["x"]), host(inp["w"]), L, D, trad, 10000.0, 1.0, offset, 1,
+                             1e-6, freqs=freqs.numpy().astype(np.float64))
+        check_out(y, ref, f"offset {offset}")
+
+
 def test_rope_round_trip_and_cache_rules():
     B, H, L, D = 1, 2, 8, 64
     x = synth.normal((B * H * L, D), 0.0, 1.0, 33, 0, "f32").cuda()
@@ -742,8 +895,6 @@ VJP_SHAPES = [(256, 4096), (1000, 2048), (33, 8192), (1, 512), (2000, 1024), (7,
 @pytest.mark.parametrize("weight", [True, False])
 @pytest.mark.parametrize("rows,D", VJP_SHAPES)
 def test_rms_norm_vjp(rows, D, weight, dt):
-    if dt == "f32" and D > 8192:
-        pytest.skip("float32 rows are limited to 8192")
     inp = synth.rms_inputs(rows, D, dt, seed=rows + D, weight=weight)
     g = synth.normal((rows, D), 0.0, 1.0, rows + D, 4, dt)
     x, w, gd = dev(inp["x"]), dev(inp["w"]), dev(g)
@@ -762,8 +913,6 @@ def test_rms_norm_vjp(rows, D, weight, dt):
 @pytest.mark.parametrize("weight", [True, False])
 @pytest.mark.parametrize("rows,D", VJP_SHAPES)
 def test_layer_norm_vjp(rows, D, weight, dt):
-    if dt == "f32" and D > 8192:
-        pytest.skip("float32 rows are limited to 8192")
     inp = synth.layer_norm_inputs(rows, D, dt, seed=rows * 3 + D, weight=weight, bias=False)
     g = synth.normal((rows, D), 0.0, 1.0, rows * 3 + D, 4, dt)
     x, w, gd = dev(inp["x"]), dev(inp["w"]), dev(g)
@@ -774,6 +923,42 @@ def test_layer_norm_vjp(rows, D, weight, dt):
     if weight:
         check_grad(dw, ref[1], ref[4], "dw")
     check_grad(db, ref[2], ref[5], "db")
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,D,shift", [(37, 1001, 0), (300, 7, 0), (5, 40000, 0), (64, 4096, 1),
+                                          (3, 1, 0), (1000, 333, 3), (9, 32768, 0)])
+def test_vjp_generic_rows(rows, D, shift, dt):
+    """Rows the register kernels cannot take -- D not a whole number of 16-byte vectors,
+    rows wider than they are built for, pointers off the 16-byte grid (shift elements into
+    a larger buffer) -- go to the generic kernel, and meet the same bar."""
+    inp = synth.layer_norm_inputs(rows, D, dt, seed=rows + D, weight=True, bias=False)
+    g = synth.normal((rows, D), 0.0, 1.0, rows + D, 4, dt)
+    tdt = DT[dt]
+
+    def placed(t):  # t as a view starting `shift` elements into a device buffer
+        flat = torch.zeros(t.numel() + shift, dtype=tdt, device="cuda")
+        flat[shift:] = t.reshape(-1).cuda()
+        return flat[shift:].view(t.shape)
+
+    x, w, gd = placed(inp["x"]), placed(inp["w"]), placed(g)
+    for op in ("rms", "layer"):
+        dx = placed(torch.zeros(rows, D, dtype=tdt))
+        dw = placed(torch.zeros(D, dtype=tdt))
+        db = placed(torch.zeros(D, dtype=tdt))
+        if op == "rms":
+            nv.nv_rms_norm_vjp(x, w, gd, dx, dw, 1e-5)
+            torch.cuda.synchronize()
+            ref = oracle.rms_norm_vjp(host(inp["x"]), host(inp["w"]), host(g), 1e-5)
+            check_grad(dx, ref[0], ref[2], "rms dx")
+            check_grad(dw, ref[1], ref[3], "rms dw")
+        else:
+            nv.nv_layer_norm_vjp(x, w, gd, dx, dw, db, 1e-5)
+            torch.cuda.synchronize()
+            ref = oracle.layer_norm_vjp(host(inp["x"]), host(inp["w"]), host(g), 1e-5)
+            check_grad(dx, ref[0], ref[3], "layer dx")
+            check_grad(dw, ref[1], ref[4], "layer dw")
+            check_grad(db, ref[2], ref[5], "layer db")
 
 
 @pytest.mark.parametrize("dt,mean,std", [("bf16", 300.0, 0.5), ("bf16", 3000.0, 40.0),

@@ -63,6 +63,44 @@ def test_static_scratch_vjp_matches_workspace_vjp_twice(dt):
         check_grad(dw, ref_vals, 2 * mag_dw, "static vs workspace dw")
 
 
+def test_static_scratch_vjp_widest_row_twice():
+    """D = 16384: the scratch holds only 2^20 / D = 64 partial rows, so each CTA walks
+    many rows; checked on two calls in a row against the workspace entry point."""
+    fn = _static_vjp()
+    rows, D = 4096, 16384
+    inp = synth.rms_inputs(rows, D, "bf16", seed=3)
+    g = synth.normal((rows, D), 0.0, 1.0, 3, 4, "bf16").cuda()
+    x, w = inp["x"].cuda(), inp["w"].cuda()
+    ref_dx, ref_dw = nv.rms_norm_vjp(x, w, g, eps=1e-6)
+    o_dx, o_dw, mag_dx, mag_dw = oracle.rms_norm_vjp(synth.to_numpy(inp["x"]),
+                                                     synth.to_numpy(inp["w"]),
+                                                     to_host_bits(g), 1e-6)
+    for _ in range(2):
+        dx, dw = torch.full_like(x, float("nan")), torch.full_like(w, float("nan"))
+        _call(fn, x, w, g, dx, dw, 1e-6, nv.NV_BF16)
+        torch.cuda.synchronize()
+        assert torch.equal(dx, ref_dx), "dx must equal the workspace entry point's"
+        check_grad(dw, o_dw, mag_dw, "static dw, D = 16384")
+        check_grad(dw, ref_dw.double().cpu().numpy(), 2 * mag_dw, "static vs workspace dw")
+
+
+def test_static_scratch_vjp_zero_rows_gives_zero_dw():
+    """rows = 0 with dw requested: dw is the sum over no rows, zero -- also right after a
+    call that left partial sums in the scratch."""
+    fn = _static_vjp()
+    D = 4096
+    inp = synth.rms_inputs(64, D, "bf16", seed=5)
+    x, w = inp["x"].cuda(), inp["w"].cuda()
+    g = synth.normal((64, D), 0.0, 1.0, 5, 4, "bf16").cuda()
+    _call(fn, x, w, g, torch.empty_like(x), torch.empty_like(w), 1e-5, nv.NV_BF16)
+    empty = torch.empty(0, D, dtype=torch.bfloat16, device="cuda")
+    for _ in range(2):
+        dw = torch.full_like(w, float("nan"))
+        _call(fn, empty, w, empty, empty, dw, 1e-5, nv.NV_BF16)
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(dw).item() == 0 and not torch.isnan(dw).any()
+
+
 def test_static_scratch_vjp_rejects_wide_rows():
     fn = _static_vjp()
     x = torch.zeros(2, 32768, dtype=torch.bfloat16, device="cuda")
