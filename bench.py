@@ -532,6 +532,14 @@ def run_ours(args):
     extras = None
     if rank == 0 and not args.no_extras and world == 1:
         extras = other_configs(flush, max(5, min(args.steps, 50)))
+    decode = None
+    if rank == 0 and not args.no_extras and world == 1:
+        # decode-sized calls are host-bound: the host time inside one C-ABI call next to
+        # the kernel time, with the per-pointer driver queries on and off
+        decode = {f"{op} {dt} [{r},{d}] checks={'on' if ck else 'off'}":
+                  host_cost(op, r, d, dt, checks=ck)
+                  for op, r, d, dt in (("rms_norm", 64, 512, "f32"), ("add_rms_norm", 1, 4096, "bf16"))
+                  for ck in (True, False)}
     baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         baseline = cpu_baseline(args.cpu_seconds)
@@ -583,6 +591,7 @@ def run_ours(args):
             "clocks": clk.summary(),
             "cpu_baseline": baseline,
             "other_configs": extras,
+            "decode_host_us": decode,
         }
         print(json.dumps(line), flush=True)
     if pg:
@@ -656,10 +665,11 @@ SWEEP_PLANS = (
 )
 
 
-def host_cost(op, rows, D, dtype, iters=200):
+def host_cost(op, rows, D, dtype, iters=200, checks=True):
     """Host time inside one C-ABI call and device time per call (tests/c/host_cost.c,
     compiled here with gcc): the decode-size story, where the call's host cost can exceed
-    the kernel.  None if the program cannot be built."""
+    the kernel.  checks=False turns the library's per-pointer driver queries off first.
+    None if the program cannot be built."""
     import shutil
     from rope_add_rms_b200 import library_path
     if shutil.which("gcc") is None:
@@ -675,7 +685,8 @@ def host_cost(op, rows, D, dtype, iters=200):
         if subprocess.run(cmd, capture_output=True).returncode != 0:
             return None
     res = subprocess.run([exe, "add" if op == "add_rms_norm" else "rms", str(rows), str(D),
-                          dtype, str(iters)], capture_output=True, text=True, timeout=120)
+                          dtype, str(iters)] + ([] if checks else ["nochecks"]),
+                         capture_output=True, text=True, timeout=120)
     if res.returncode != 0:
         return None
     return json.loads(res.stdout)
@@ -727,6 +738,8 @@ def run_sweep(args):
                         line["auto_over_best"] = round(gbs / bg, 4)
                 if rows <= 256:
                     line["host_call"] = host_cost("add_rms_norm", rows, D, dtype)
+                    line["host_call_nochecks"] = host_cost("add_rms_norm", rows, D, dtype,
+                                                           checks=False)
                 print(json.dumps(line), flush=True)
                 del c
                 torch.cuda.empty_cache()

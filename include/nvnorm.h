@@ -370,6 +370,20 @@ NV_API const char* nv_last_error(void);
 NV_API int32_t nv_version(void);
 
 /*
+ * Pointer checks -- by default every call asks the driver, for each pointer, whether it
+ * is device memory of the current device and how far its allocation extends (one query per
+ * pointer, a few tenths of a microsecond each; together most of the host time of a call on
+ * a decode-sized batch).  A caller that guarantees its pointers -- buffers it allocated
+ * itself, sized for the call, on the current device -- may turn these queries off for the
+ * whole process with enabled = 0, and back on with 1.  Everything else is still checked:
+ * sizes, NULL pointers, and the overlap of outputs with other buffers.  With the queries
+ * off, a wrong pointer is no longer caught on the host: the kernel then reads or writes
+ * whatever memory it is given.  previous: out, the former setting (1 on, 0 off), or NULL.
+ * Always NV_OK.
+ */
+NV_API nv_status nv_set_pointer_checks(int32_t enabled, int32_t* previous);
+
+/*
  * Device-side bounded waits that ran out, on the current device, since the library
  * was loaded (or last reset).  Only the staged kernels wait on the copy engine (and
  * nv_selftest_bounded_wait, on purpose, on a barrier nothing completes); each wait gives
@@ -411,7 +425,9 @@ NV_API nv_status nv_selftest_bounded_wait(int32_t ctas, nv_stream_t stream);
  *                   writing any global memory, so results are the same as with a plain
  *                   launch; NV_LAUNCH_PLAIN: ordinary stream-ordered launch.
  *   stages          NV_PATH_RING: shared-memory row buffers per CTA (0 = as many as fit,
- *                   at most 32; a multiple of rows_per_cta, at least 2 x rows_per_cta).  norm_rope, two vectors per
+ *                   at most 32; a multiple of rows_per_cta, at least 2 x rows_per_cta).
+ *                   NV_PATH_SLOTS: 0 or 1 = each row slot asks L2 for its next row while
+ *                   it works on the current one (one bulk prefetch a row); -1 = no prefetch.  norm_rope, two vectors per
  *                   lane: 1 = the compensated (error-free) rotation on every pair instead
  *                   of the float32 rotation with a per-pair error test and compensated
  *                   recomputation of the pairs that fail it (same results within the
@@ -427,9 +443,13 @@ typedef enum {
     NV_PATH_STAGED = 3,  /* persistent, rows staged in shared memory by bulk async copies;
                             rms_norm, add_rms_norm and layer_norm.  rows_per_cta = rows in
                             flight per CTA (shared-memory stages), ctas_per_sm = CTAs per SM */
-    NV_PATH_RING = 4     /* layer_norm: persistent CTAs of several row groups (a few warps
+    NV_PATH_RING = 4,    /* layer_norm: persistent CTAs of several row groups (a few warps
                             each, reducing one row at a time) fed by a ring of shared-memory
                             row buffers that bulk async copies refill as rows finish */
+    NV_PATH_SLOTS = 5    /* layer_norm, bfloat16: rows in registers, rows_per_cta of them per
+                            persistent CTA sharing a float32 table of w and b in shared
+                            memory; x consumed packed (bfloat16 -> double conversions and
+                            mixed-precision fma, no unpacking) */
 } nv_path;
 
 typedef enum { NV_LAUNCH_DEFAULT = 0, NV_LAUNCH_PLAIN = 1 } nv_launch;

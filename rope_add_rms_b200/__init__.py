@@ -23,11 +23,11 @@ __all__ = [
     "allreduce_add_rms_norm", "rope_llama3_freqs", "rope_yarn_freqs", "rope_suscaled_freqs",
     "nv_layer_norm", "nv_norm_rope",
     "nv_describe_plan",
-    "nv_fault_count", "nv_selftest_bounded_wait",
+    "nv_fault_count", "nv_selftest_bounded_wait", "nv_set_pointer_checks",
     "nv_rope", "rms_norm", "add_rms_norm", "layer_norm", "norm_rope", "norm_rope_into_cache",
     "rope", "nv_rms_norm_vjp", "nv_layer_norm_vjp", "nv_norm_vjp_workspace_size", "rms_norm_vjp",
     "layer_norm_vjp",
-    "PATH_AUTO", "PATH_ROWS", "PATH_GENERIC", "PATH_STAGED", "PATH_RING", "LAUNCH_DEFAULT",
+    "PATH_AUTO", "PATH_ROWS", "PATH_GENERIC", "PATH_STAGED", "PATH_RING", "PATH_SLOTS", "LAUNCH_DEFAULT",
     "LAUNCH_PLAIN",
 ]
 
@@ -36,7 +36,7 @@ library_path = os.path.join(_HERE, "libnvnorm.so")
 
 NV_F32, NV_BF16, NV_F16 = 0, 1, 2
 NV_OK, NV_ERR_INVALID_ARG, NV_ERR_UNSUPPORTED, NV_ERR_CUDA = 0, 1, 2, 3
-PATH_AUTO, PATH_ROWS, PATH_GENERIC, PATH_STAGED, PATH_RING = 0, 1, 2, 3, 4
+PATH_AUTO, PATH_ROWS, PATH_GENERIC, PATH_STAGED, PATH_RING, PATH_SLOTS = 0, 1, 2, 3, 4, 5
 LAUNCH_DEFAULT, LAUNCH_PLAIN = 0, 1
 
 _DT = {torch.float32: NV_F32, torch.bfloat16: NV_BF16, torch.float16: NV_F16}
@@ -106,6 +106,8 @@ def library() -> ctypes.CDLL:
     lib.nv_last_error.restype = ctypes.c_char_p
     lib.nv_version.argtypes = []
     lib.nv_version.restype = ctypes.c_int32
+    lib.nv_set_pointer_checks.argtypes = [ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
+    lib.nv_set_pointer_checks.restype = ctypes.c_int
     lib.nv_fault_count.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int32]
     lib.nv_fault_count.restype = ctypes.c_int
     lib.nv_selftest_bounded_wait.argtypes = [ctypes.c_int32, ctypes.c_void_p]
@@ -374,6 +376,15 @@ def nv_describe_plan(op: str, rows: int, D: int, dtype) -> dict:
     _check("nv_describe_plan", library().nv_describe_plan(ops[op], rows, D, _DT[dtype],
                                                            ctypes.byref(p)))
     return p.as_dict()
+
+
+def nv_set_pointer_checks(enabled: bool) -> bool:
+    """Turn the per-pointer driver queries of every call on or off (process-wide); returns
+    the former setting.  Off is for callers that vouch for their pointers."""
+    prev = ctypes.c_int32(0)
+    _check("nv_set_pointer_checks", library().nv_set_pointer_checks(int(bool(enabled)),
+                                                                     ctypes.byref(prev)))
+    return bool(prev.value)
 
 
 def nv_fault_count(reset: bool = False) -> int:

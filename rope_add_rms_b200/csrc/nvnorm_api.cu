@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -18,6 +19,7 @@
 #include "common.cuh"
 #include "layer.cuh"
 #include "layer_ring.cuh"
+#include "layer_slots.cuh"
 #include "rms.cuh"
 #include "rope.cuh"
 #include "staged.cuh"
@@ -27,7 +29,7 @@ namespace {
 
 using namespace nvn;
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0 (nv_plan gained `stages`)
 constexpr int kMaxSelftestCtas = 64;  // nv_selftest_bounded_wait: one resident wave
 
 // ---- error reporting ------------------------------------------------------------------
@@ -60,6 +62,12 @@ nv_status current_device(int* dev, DevInfo* info) {
     cudaError_t e = cudaGetDevice(dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (*dev < 0 || *dev >= kMaxDevices) return fail(NV_ERR_UNSUPPORTED, "device %d", *dev);
+    // each thread keeps its own copy of the (immutable) facts: no lock after the first call
+    thread_local DevInfo tl_dev[kMaxDevices];
+    if (tl_dev[*dev].ready) {
+        *info = tl_dev[*dev];
+        return NV_OK;
+    }
     std::lock_guard<std::mutex> lk(g_dev_mu);
     DevInfo& d = g_dev[*dev];
     if (!d.ready) {
@@ -72,6 +80,7 @@ nv_status current_device(int* dev, DevInfo* info) {
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
         d.ready = true;
     }
+    tl_dev[*dev] = d;
     *info = d;
     return NV_OK;
 }
@@ -148,11 +157,16 @@ nv_status check_pointer(const Buf& b, int dev) {
     return NV_OK;
 }
 
+// Process-wide switch for the driver queries of check_pointer (nv_set_pointer_checks).
+std::atomic<int> g_pointer_checks{1};
+
 nv_status check_buffers(const Buf* bufs, int n, int dev) {
-    for (int i = 0; i < n; ++i) {
-        if (!bufs[i].p) continue;
-        nv_status st = check_pointer(bufs[i], dev);
-        if (st != NV_OK) return st;
+    if (g_pointer_checks.load(std::memory_order_relaxed)) {
+        for (int i = 0; i < n; ++i) {
+            if (!bufs[i].p) continue;
+            nv_status st = check_pointer(bufs[i], dev);
+            if (st != NV_OK) return st;
+        }
     }
     // an output may not overlap anything, except that it may be exactly a row input
     for (int i = 0; i < n; ++i) {
@@ -240,6 +254,34 @@ size_t staged_smem(Op op, int64_t D, nv_dtype dt, int stages) {
     return (size_t)stages * (stage + 8);
 }
 constexpr int kStaticSmemReserve = 2048;  // static shared memory + per-CTA system use
+
+// Slots path shape (bfloat16 layer_norm): VPT vectors a thread (8, or 4 for narrow rows),
+// G threads a row, as many row slots as make 768 threads (24 warps per SM, one CTA per SM),
+// at most 15 when a row spans several warps (one named barrier each); the float32 w/b table
+// (64 bytes a vector) must fit the shared memory.
+bool slots_shape(int nvec, const nv_plan& req, const DevInfo* di, nv_plan* out) {
+    nv_plan p = req;
+    int v = p.vec_per_thread ? p.vec_per_thread : (nvec >= 256 ? 8 : 4);
+    if (v != 4 && v != 8) return false;
+    int g = p.threads_per_row ? p.threads_per_row : ((nvec + v - 1) / v + 31) / 32 * 32;
+    if (g % 32 || g < 32 || (int64_t)g * v < nvec || g > kSlotsMaxThreads) return false;
+    int slots = p.rows_per_cta ? p.rows_per_cta : kSlotsMaxThreads / g;
+    if (g > 32) slots = std::min(slots, 15);
+    if (slots < 1 || slots * g > kSlotsMaxThreads || (g > 32 && slots > 15)) return false;
+    const size_t optin = (size_t)(di ? di->smem_optin : 232448) - kStaticSmemReserve;
+    if (slots_table_bytes(nvec) > optin) return false;
+    if (p.ctas_per_sm > 1) return false;  // one table per SM
+    // stages: 0 or 1 = each slot prefetches its next row into L2 (one bulk prefetch a row),
+    // -1 = no prefetch
+    if (p.stages != 0 && p.stages != 1 && p.stages != -1) return false;
+    p.stages = p.stages == 0 ? 1 : p.stages;
+    p.vec_per_thread = v;
+    p.threads_per_row = g;
+    p.rows_per_cta = slots;
+    p.ctas_per_sm = 1;
+    *out = p;
+    return true;
+}
 
 // Ring path shape (layer_norm): R warps per row group so that a thread holds about eight
 // 16-byte vectors of a row; 16 warps per CTA in row groups; then as many row buffers as
@@ -347,6 +389,14 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
         if (p.rows_per_cta < 2 || staged_smem(op, D, dt, p.rows_per_cta) > (size_t)budget)
             return fail(NV_ERR_UNSUPPORTED, "staged path: %d stages of %zu bytes do not fit "
                         "%d bytes of shared memory", p.rows_per_cta, one, budget);
+    } else if (p.path == NV_PATH_SLOTS && op == OP_LAYER) {
+        if (!vec_ok || dt != NV_BF16)
+            return fail(NV_ERR_UNSUPPORTED, "slots path: bfloat16 layer_norm with D %% 8 == 0 "
+                        "and 16-byte aligned pointers");
+        if (!slots_shape(nvec, p, di, &p))
+            return fail(NV_ERR_UNSUPPORTED, "slots path: no shape for D = %lld (vpt %d, G %d, "
+                        "slots %d)", (long long)D, p.vec_per_thread, p.threads_per_row,
+                        p.rows_per_cta);
     } else if (p.path == NV_PATH_RING && op == OP_LAYER) {
         if (!vec_ok) return fail(NV_ERR_UNSUPPORTED, "ring path needs D %% %d == 0 and "
                                  "16-byte aligned pointers", vecw);
@@ -363,8 +413,8 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
     } else {
         return fail(NV_ERR_UNSUPPORTED, "path %d is not available for this op", p.path);
     }
-    if (p.path != NV_PATH_RING && p.stages != 0)
-        return fail(NV_ERR_UNSUPPORTED, "stages is for the ring path only");
+    if (p.path != NV_PATH_RING && p.path != NV_PATH_SLOTS && p.stages != 0)
+        return fail(NV_ERR_UNSUPPORTED, "stages is for the ring and slots paths only");
     if (p.ctas_per_sm < 0) return fail(NV_ERR_INVALID_ARG, "ctas_per_sm < 0");
     (void)rows;
     *out = p;
@@ -463,6 +513,25 @@ template <typename T>
 nv_status run_layer(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs a) {
     if (p.path == NV_PATH_GENERIC)
         return launch(layer_generic_kernel<T>, a.rows, 256, 0, p.ctas_per_sm, di, s, a);
+    if (p.path == NV_PATH_SLOTS) {
+        if constexpr (sizeof(T) == 2) {
+            a.G = p.threads_per_row;
+            a.rows_per_cta = p.rows_per_cta;
+            const bool pf = p.stages == 1;
+            const size_t smem = slots_table_bytes(a.nvec);
+            auto kern = p.vec_per_thread == 8
+                            ? (pf ? layer_slots_kernel<8, true> : layer_slots_kernel<8, false>)
+                            : (pf ? layer_slots_kernel<4, true> : layer_slots_kernel<4, false>);
+            cudaError_t e =
+                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+            const int64_t units = (a.rows + a.rows_per_cta - 1) / a.rows_per_cta;
+            const int64_t grid = grid_for(units, di.sms, 1);
+            return launch_kernel(kern, grid, a.G * a.rows_per_cta, smem, s, a);
+        } else {
+            return fail(NV_ERR_UNSUPPORTED, "slots path: bfloat16 only");
+        }
+    }
     if (p.path == NV_PATH_RING) {
         constexpr int vecw = 16 / sizeof(T);
         RingArgs rg{};
@@ -1624,5 +1693,11 @@ nv_status nv_selftest_bounded_wait(int32_t ctas, nv_stream_t stream) {
 }
 
 int32_t nv_version(void) { return kVersion; }
+
+nv_status nv_set_pointer_checks(int32_t enabled, int32_t* previous) {
+    const int old = g_pointer_checks.exchange(enabled ? 1 : 0);
+    if (previous) *previous = old;
+    return NV_OK;
+}
 
 }  // extern "C"

@@ -5,7 +5,10 @@
  * to back on one stream.  For decode-sized batches (a few rows) the host cost is the
  * whole story: when it exceeds the kernel time the stream runs dry between calls.
  *
- *   host_cost OP ROWS D DTYPE ITERS     OP: rms | add;  DTYPE: bf16 | f32
+ *   host_cost OP ROWS D DTYPE ITERS [nochecks]     OP: rms | add;  DTYPE: bf16 | f32
+ *
+ * With `nochecks` the library's per-pointer driver queries are turned off first
+ * (nv_set_pointer_checks(0)): the host cost of a caller that vouches for its pointers.
  *
  * Prints one JSON object: {"op", "rows", "D", "dtype", "iters", "host_us_per_call",
  * "device_us_per_call", "empty_launch_us"}: the host time inside one call; the device time
@@ -48,10 +51,12 @@ static double now_us(void) {
 }
 
 int main(int argc, char** argv) {
-    if (argc != 6) {
-        fprintf(stderr, "usage: %s rms|add ROWS D bf16|f32 ITERS\n", argv[0]);
+    if (argc != 6 && argc != 7) {
+        fprintf(stderr, "usage: %s rms|add ROWS D bf16|f32 ITERS [nochecks]\n", argv[0]);
         return 1;
     }
+    const int checks = !(argc == 7 && strcmp(argv[6], "nochecks") == 0);
+    nv_set_pointer_checks(checks, NULL);
     const int add = strcmp(argv[1], "add") == 0;
     const int64_t rows = atoll(argv[2]), D = atoll(argv[3]);
     const int bf = strcmp(argv[4], "bf16") == 0;
@@ -116,9 +121,10 @@ int main(int argc, char** argv) {
     CK(cudaStreamSynchronize(st));
 
     printf("{\"op\": \"%s\", \"rows\": %lld, \"D\": %lld, \"dtype\": \"%s\", \"iters\": %d, "
+           "\"pointer_checks\": %d, "
            "\"host_us_per_call\": %.3f, \"device_us_per_call\": %.3f, "
            "\"empty_launch_us\": %.3f}\n",
            add ? "add_rms_norm" : "rms_norm", (long long)rows, (long long)D, bf ? "bf16" : "f32",
-           iters, (t1 - t0) / iters, 1e3 * span_ms / iters, (m1 - m0) / iters);
+           iters, checks, (t1 - t0) / iters, 1e3 * span_ms / iters, (m1 - m0) / iters);
     return 0;
 }

@@ -342,3 +342,15 @@ def test_cuda_failures_are_reported_as_nv_err_cuda(name, call):
     assert call() == nv.NV_ERR_CUDA, name
     msg = last_error()
     assert re.match(r"^\w[\w ]*: cudaError\w+ \(", msg), msg
+
+
+def test_pointer_checks_switch_reports_the_former_setting():
+    assert nv.nv_set_pointer_checks(False) is True     # on by default
+    try:
+        assert nv.nv_set_pointer_checks(False) is False
+        # argument checks that need no driver query still apply with the queries off
+        assert rms(D=0) == INVALID and "D" in last_error()
+        assert add(h=FAKE) == INVALID and "same buffer" in last_error()
+    finally:
+        assert nv.nv_set_pointer_checks(True) is False
+    assert nv.nv_set_pointer_checks(True) is True

@@ -207,6 +207,27 @@ def test_host_memory_undersized_and_overlapping_buffers_are_rejected():
         nv.nv_rms_norm(xs, w, ys, 1e-5)      # partial overlap of input and output
 
 
+def test_pointer_checks_off_same_results_overlaps_still_rejected():
+    """With the per-pointer driver queries off the ops give the same bits; a host buffer is
+    caught only with them on; an output overlapping an input is rejected either way."""
+    inp = synth.add_rms_inputs(300, 4096, "bf16", seed=21)
+    x, r, w = dev(inp["x"]), dev(inp["r"]), dev(inp["w"])
+    y0, h0 = nv.add_rms_norm(x, r, w, 1e-5)
+    prev = nv.nv_set_pointer_checks(False)
+    try:
+        y1, h1 = nv.add_rms_norm(x, r, w, 1e-5)
+        torch.cuda.synchronize()
+        assert torch.equal(y0, y1) and torch.equal(h0, h1)
+        big = torch.zeros(3 * 2048, dtype=torch.bfloat16, device="cuda")
+        xs, ys = big[:2048].view(8, 256), big[128:128 + 2048].view(8, 256)
+        with pytest.raises(nv.NvError, match="overlaps"):
+            nv.nv_rms_norm(xs, w[:256], ys, 1e-5)
+    finally:
+        nv.nv_set_pointer_checks(prev)
+    with pytest.raises(nv.NvError, match="not device memory"):
+        nv.nv_rms_norm(x.cpu().pin_memory(), w, torch.empty_like(x), 1e-5)
+
+
 # ---- staged (bulk-copy) path ----------------------------------------------------------------
 
 STAGED = [dict(path=nv.PATH_STAGED),
@@ -324,6 +345,50 @@ def test_layer_norm_in_place_and_large_mean():
     nv.nv_layer_norm(xd, None, None, xd, 1e-5)
     torch.cuda.synchronize()
     check_out(xd, ref)
+
+
+SLOTS = [dict(path=nv.PATH_SLOTS), dict(path=nv.PATH_SLOTS, vec_per_thread=4),
+         dict(path=nv.PATH_SLOTS, rows_per_cta=1), dict(path=nv.PATH_SLOTS, rows_per_cta=5),
+         dict(path=nv.PATH_SLOTS, vec_per_thread=8, threads_per_row=64),
+         dict(path=nv.PATH_SLOTS, stages=-1)]
+
+
+@pytest.mark.parametrize("plan", SLOTS, ids=lambda p: "-".join(f"{k}{v}" for k, v in p.items()))
+@pytest.mark.parametrize("rows,D,wb", [(147, 8192, (1, 1)), (149, 5120, (1, 0)), (33, 4096, (0, 0)),
+                                        (5, 16384, (1, 1)), (64, 512, (1, 1)), (300, 256, (0, 1)),
+                                        (1000, 2048, (1, 1)), (1, 8192, (1, 1)), (2, 8, (1, 1)),
+                                        (77, 24576, (1, 1))])
+def test_layer_norm_slots(rows, D, wb, plan):
+    """The slots path (bfloat16): rows in registers, several per CTA sharing a float32 table
+    of w and b, x consumed packed by bfloat16 -> double conversions and mixed-precision fma."""
+    inp = synth.layer_norm_inputs(rows, D, "bf16", seed=D + 5 * rows, weight=bool(wb[0]),
+                                  bias=bool(wb[1]))
+    x, w, b = dev(inp["x"]), dev(inp["w"]), dev(inp["b"])
+    g = Guarded(x.shape, x.dtype)
+    try:
+        nv.nv_layer_norm(x, w, b, g.t, 1e-5, plan=nv.Plan(**plan))
+    except nv.NvError as e:
+        assert e.status == nv.NV_ERR_UNSUPPORTED
+        pytest.skip(str(e))
+    torch.cuda.synchronize()
+    assert g.bands_intact()
+    check_out(g.t, oracle.layer_norm(host(inp["x"]), host(inp["w"]), host(inp["b"]), 1e-5))
+
+
+@pytest.mark.parametrize("mean,std", [(3000.0, 40.0), (3000.0, 0.25), (0.5, 2.0), (-7.0e4, 3.0),
+                                      (1.0, 1e-30)])
+def test_layer_norm_slots_means_and_in_place(mean, std):
+    """The slots path on rows whose mean is far from zero (centred second pass, two-step
+    subtraction of the mean), near-constant rows, and in place (y == x)."""
+    for rows, D in ((33, 4096), (300, 8192), (7, 64)):
+        x = synth.normal((rows, D), mean, std, 6, 0, "bf16")
+        w = synth.uniform((D,), 0.5, 1.5, 6, 2, "bf16")
+        b = synth.normal((D,), 0.0, 0.1, 6, 3, "bf16")
+        ref = oracle.layer_norm(host(x), host(w), host(b), 1e-5)
+        xd = x.cuda()
+        nv.nv_layer_norm(xd, w.cuda(), b.cuda(), xd, 1e-5, plan=nv.Plan(path=nv.PATH_SLOTS))
+        torch.cuda.synchronize()
+        check_out(xd, ref)
 
 
 RING = [dict(path=nv.PATH_RING),
