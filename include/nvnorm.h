@@ -426,12 +426,9 @@ NV_API nv_status nv_selftest_bounded_wait(int32_t ctas, nv_stream_t stream);
  *                   launch; NV_LAUNCH_PLAIN: ordinary stream-ordered launch.
  *   stages          NV_PATH_RING: shared-memory row buffers per CTA (0 = as many as fit,
  *                   at most 32; a multiple of rows_per_cta, at least 2 x rows_per_cta).
- *                   NV_PATH_SLOTS: 0 or 1 = each row slot asks L2 for its next row while
- *                   it works on the current one (one bulk prefetch a row); -1 = no prefetch.  norm_rope, two vectors per
- *                   lane: 1 = the compensated (error-free) rotation on every pair instead
- *                   of the float32 rotation with a per-pair error test and compensated
- *                   recomputation of the pairs that fail it (same results within the
- *                   tolerance).  Other paths: must be 0.
+ *                   NV_PATH_SLOTS: 1 = each row slot asks L2 for its next row while it
+ *                   works on the current one (one bulk prefetch a row); -1 = no prefetch;
+ *                   0 = prefetch when a row spans several warps.  Other paths: must be 0.
  * For NV_PATH_RING, threads_per_row is the size of a row group (32 x warps, <= 256),
  * rows_per_cta the row groups of a CTA (rows reduced at once), ctas_per_sm the CTAs per
  * SM (0 = 1), vec_per_thread must be 0.

@@ -73,7 +73,9 @@ __device__ __forceinline__ void slot_bar(int id, int nthreads) {
 __host__ __device__ constexpr size_t slots_table_bytes(int nvec) {
     return (size_t)nvec * 8u * 2u * sizeof(float);
 }
-constexpr int kSlotsMaxThreads = 768;
+// CTA sizes the kernel is built for: 768 threads (24 warps, up to 80 registers) and 1024
+// (32 warps, up to 64 registers).
+constexpr int kSlotsMaxThreads = 1024;
 
 // Bulk prefetch of `bytes` (a multiple of 16) at global address p (16-byte aligned) into L2.
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
@@ -82,15 +84,15 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 
 // Launch: blockDim.x = a.G * a.rows_per_cta (rows_per_cta = slots <= 15 when G > 32),
 // dynamic shared memory = slots_table_bytes(a.nvec); persistent grid.
-template <int VPT, bool PREFETCH>
-__global__ void __launch_bounds__(kSlotsMaxThreads, 1) layer_slots_kernel(const RowArgs a) {
+template <int VPT, bool PREFETCH, int MAXT>
+__global__ void __launch_bounds__(MAXT, 1) layer_slots_kernel(const RowArgs a) {
     pdl_wait();
     pdl_release();
     using T = __nv_bfloat16;
     using E = Elem<T>;
     constexpr int VEC = 8;
     extern __shared__ float4 tab[];  // [4][nvec]: w 0-3, w 4-7, b 0-3, b 4-7
-    __shared__ double red[2][kSlotsMaxThreads / 32][3];
+    __shared__ double red[2][MAXT / 32][3];
 
     const int G = a.G;
     const int slots = a.rows_per_cta;

@@ -265,16 +265,18 @@ bool slots_shape(int nvec, const nv_plan& req, const DevInfo* di, nv_plan* out) 
     if (v != 4 && v != 8) return false;
     int g = p.threads_per_row ? p.threads_per_row : ((nvec + v - 1) / v + 31) / 32 * 32;
     if (g % 32 || g < 32 || (int64_t)g * v < nvec || g > kSlotsMaxThreads) return false;
-    int slots = p.rows_per_cta ? p.rows_per_cta : kSlotsMaxThreads / g;
+    // 768 threads (24 warps, 80 registers) unless asked for more rows per CTA
+    int slots = p.rows_per_cta ? p.rows_per_cta : 768 / g;
     if (g > 32) slots = std::min(slots, 15);
     if (slots < 1 || slots * g > kSlotsMaxThreads || (g > 32 && slots > 15)) return false;
     const size_t optin = (size_t)(di ? di->smem_optin : 232448) - kStaticSmemReserve;
     if (slots_table_bytes(nvec) > optin) return false;
     if (p.ctas_per_sm > 1) return false;  // one table per SM
-    // stages: 0 or 1 = each slot prefetches its next row into L2 (one bulk prefetch a row),
-    // -1 = no prefetch
+    // stages: 1 = each slot prefetches its next row into L2 (one bulk prefetch a row),
+    // -1 = no prefetch, 0 = prefetch when a row spans several warps (measured: it gains
+    // 1-5 % from D = 4096 on, and loses 3 % at D = 2048, a warp per row)
     if (p.stages != 0 && p.stages != 1 && p.stages != -1) return false;
-    p.stages = p.stages == 0 ? 1 : p.stages;
+    p.stages = p.stages == 0 ? (g > 32 ? 1 : -1) : p.stages;
     p.vec_per_thread = v;
     p.threads_per_row = g;
     p.rows_per_cta = slots;
@@ -346,9 +348,17 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
     const int nvec = vec_ok ? (int)(D / vecw) : 0;
     if (p.path == NV_PATH_AUTO) {
         int v = 0, g = 0;
-        p.path = vec_ok && rows_shape(op, nvec, p.vec_per_thread, p.threads_per_row, &v, &g)
-                     ? NV_PATH_ROWS
-                     : NV_PATH_GENERIC;
+        nv_plan sp{};
+        // bfloat16 layer_norm: the slots kernel (measured 10-20 % faster than the register
+        // kernel over D = 2048..16384 on B200) from rows of 256 vectors on, whenever its
+        // w/b table fits
+        if (op == OP_LAYER && dt == NV_BF16 && vec_ok && nvec >= 256 && p.vec_per_thread == 0 &&
+            p.threads_per_row == 0 && p.rows_per_cta == 0 && slots_shape(nvec, p, di, &sp))
+            p.path = NV_PATH_SLOTS;
+        else
+            p.path = vec_ok && rows_shape(op, nvec, p.vec_per_thread, p.threads_per_row, &v, &g)
+                         ? NV_PATH_ROWS
+                         : NV_PATH_GENERIC;
     }
     if (p.path == NV_PATH_ROWS) {
         if (!vec_ok) return fail(NV_ERR_UNSUPPORTED, "register path needs D %% %d == 0 and "
@@ -519,9 +529,14 @@ nv_status run_layer(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs
             a.rows_per_cta = p.rows_per_cta;
             const bool pf = p.stages == 1;
             const size_t smem = slots_table_bytes(a.nvec);
-            auto kern = p.vec_per_thread == 8
-                            ? (pf ? layer_slots_kernel<8, true> : layer_slots_kernel<8, false>)
-                            : (pf ? layer_slots_kernel<4, true> : layer_slots_kernel<4, false>);
+            const bool big = a.G * a.rows_per_cta > 768;
+            auto pick = [&](auto vpt) {
+                constexpr int V = decltype(vpt)::value;
+                return big ? (pf ? layer_slots_kernel<V, true, 1024> : layer_slots_kernel<V, false, 1024>)
+                           : (pf ? layer_slots_kernel<V, true, 768> : layer_slots_kernel<V, false, 768>);
+            };
+            auto kern = p.vec_per_thread == 8 ? pick(std::integral_constant<int, 8>{})
+                                              : pick(std::integral_constant<int, 4>{});
             cudaError_t e =
                 cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -652,21 +667,18 @@ nv_status row_dispatch(Op op, const nv_plan& p, const DevInfo& di, nv_dtype dt, 
 struct RopePlan {
     bool rows;
     bool pairs;  // two vectors per lane: rope_pairs_kernel (dims == D)
-    bool exact;  // pairs kernel: the compensated rotation on every pair
     int lpr;
     int bt;
     int64_t n_chunks;
 };
 
 template <typename T, bool TRAD>
-nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a, bool pairs,
-                           bool exact) {
+nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a, bool pairs) {
     // the pairs kernel keeps its lanes' weights after the table: VEC/2 records per lane
     const size_t smem = (size_t)a.half * sizeof(float4) +
                         (pairs ? (size_t)Elem<T>::kVec / 2 * (size_t)(a.nvec / 2) * sizeof(float4)
                                : 0);
-    auto kern = !pairs ? rope_rows_kernel<T, TRAD>
-                       : exact ? rope_pairs_kernel<T, TRAD, true> : rope_pairs_kernel<T, TRAD, false>;
+    auto kern = pairs ? rope_pairs_kernel<T, TRAD> : rope_rows_kernel<T, TRAD>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -699,10 +711,7 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
     if (p.path == NV_PATH_AUTO) p.path = (vec_ok || pairs_ok) ? NV_PATH_ROWS : NV_PATH_GENERIC;
     rp->rows = p.path == NV_PATH_ROWS;
     rp->pairs = rp->rows && pairs_ok && p.vec_per_thread != 1;
-    if (p.stages != 0 && !(p.stages == 1 && rp->pairs))
-        return fail(NV_ERR_UNSUPPORTED, "norm_rope: stages = 1 (the compensated rotation on "
-                    "every pair) needs the two-vectors-per-lane register path");
-    rp->exact = p.stages == 1;
+    if (p.stages != 0) return fail(NV_ERR_UNSUPPORTED, "norm_rope takes no stages");
     if (p.path == NV_PATH_ROWS) {
         if (!vec_ok && !rp->pairs)
             return fail(NV_ERR_UNSUPPORTED, "norm_rope register path needs D %% %d == 0, "
@@ -817,10 +826,10 @@ nv_status rope_op(const void* x, const void* w, const float* freqs, void* y, int
     const bool bf = dt == NV_BF16;
     if (rp.rows) {
         if (traditional)
-            return bf ? launch_rope_rows<__nv_bfloat16, true>(di, cs, a, rp.pairs, rp.exact)
-                      : launch_rope_rows<float, true>(di, cs, a, rp.pairs, rp.exact);
-        return bf ? launch_rope_rows<__nv_bfloat16, false>(di, cs, a, rp.pairs, rp.exact)
-                  : launch_rope_rows<float, false>(di, cs, a, rp.pairs, rp.exact);
+            return bf ? launch_rope_rows<__nv_bfloat16, true>(di, cs, a, rp.pairs)
+                      : launch_rope_rows<float, true>(di, cs, a, rp.pairs);
+        return bf ? launch_rope_rows<__nv_bfloat16, false>(di, cs, a, rp.pairs)
+                  : launch_rope_rows<float, false>(di, cs, a, rp.pairs);
     }
     return bf ? launch_rope_generic<__nv_bfloat16>(di, p.ctas_per_sm, cs, a)
               : launch_rope_generic<float>(di, p.ctas_per_sm, cs, a);

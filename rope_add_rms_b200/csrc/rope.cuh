@@ -360,33 +360,7 @@ struct PairLayout {
     }
 };
 
-// Plain float32 rotation of two pairs and the test that it meets the output tolerance.
-// With c = c_hi + c_lo and s = s_hi + s_lo, z_p = a_p c_hi - RN(a_q s_hi) (one fma) is
-// off by at most 2^-23 (|a_p c| + |a_q s|) + 2^-24 |z_p| <= 2^-23 |a| + 2^-24 |z_p| (|a| the
-// pair's norm, Cauchy-Schwarz; 1.5 x 2^-23 |a| for float32 data, where a = x w is itself
-// rounded), and likewise z_q.  The rotation keeps the norm, so |a| <= sqrt(2) max|z|.
-//   bfloat16: half a bfloat16 step (2^-9 |y|, with 2^-21.5 |y| left for the common factor
-//   inv) holds whenever |z| > 2^-12 max(|z_p|, |z_q|) for both members (a factor ~1.9 of
-//   margin); only a near cancellation fails it (about 1 pair in 10^4).
-//   float32: the absolute error 2^-22.4 |a| inv stays below the 1e-5 bar of the outputs
-//   while max|z| inv < 16, true for every normalised row of ordinary width.
-// Returns false when the pairs must be recomputed with the compensated rotation.
-template <typename T>
-__device__ __forceinline__ bool rotate_plain2(float2 ap, float2 aq, float2 ch, float2 sh,
-                                              float inv, float2& zp, float2& zq) {
-    zp = fma2(ap, ch, neg2(mul2(aq, sh)));
-    zq = fma2(aq, ch, mul2(ap, sh));
-    if constexpr (sizeof(T) == 2) {
-        const float m0 = fminf(fabsf(zp.x), fabsf(zq.x)), M0 = fmaxf(fabsf(zp.x), fabsf(zq.x));
-        const float m1 = fminf(fabsf(zp.y), fabsf(zq.y)), M1 = fmaxf(fabsf(zp.y), fabsf(zq.y));
-        return m0 > 0x1p-12f * M0 && m1 > 0x1p-12f * M1;
-    } else {
-        const float M = fmaxf(fmaxf(fabsf(zp.x), fabsf(zp.y)), fmaxf(fabsf(zq.x), fabsf(zq.y)));
-        return M * inv < 16.f;
-    }
-}
-
-template <typename T, bool TRAD, bool EXACT = false>
+template <typename T, bool TRAD>
 __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 4 : 3) rope_pairs_kernel(const RopeArgs a) {
     using E = Elem<T>;
     using PL = PairLayout<T, TRAD>;
@@ -490,13 +464,8 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 4 : 3) rope_pairs_kernel
                     const float4 w4 = tab[a.half + k * hvec + v0];
                     const float2 ap = mul2(p[k], make_float2(w4.x, w4.y));  // exact for bf16 data
                     const float2 aq = mul2(q[k], make_float2(w4.z, w4.w));
-                    float2 zp, zq;
-                    if (EXACT || !rotate_plain2<T>(ap, aq, ch, sh, inv, zp, zq)) {
-                        zp = rotate_sub2(ap, aq, ch, cl, sh, sl);
-                        zq = rotate_pair2(aq, ap, ch, cl, sh, sl);
-                    }
-                    yp[k] = mul2(zp, inv2);
-                    yq[k] = mul2(zq, inv2);
+                    yp[k] = mul2(rotate_sub2(ap, aq, ch, cl, sh, sl), inv2);
+                    yq[k] = mul2(rotate_pair2(aq, ap, ch, cl, sh, sl), inv2);
                 }
                 V16 o0, o1;
                 PL::join(yp, yq, o0, o1);
