@@ -478,6 +478,10 @@ def other_configs(flush, steps):
                  base=10000.0, scale=1.0, offset=4096),
         "rms_norm f32 [64,512] eps 1e-6":
             Case("rms_norm", (64, 512), "f32", 0, eps=1e-6),
+        "rms_norm_vjp bf16 [8192,4096] eps 1e-5 (dx, dw)":
+            Case("rms_norm_vjp", (8192, 4096), "bf16", 0, eps=1e-5),
+        "layer_norm_vjp bf16 [16384,8192] eps 1e-5 (dx, dw, db)":
+            Case("layer_norm_vjp", (16384, 8192), "bf16", 0, eps=1e-5),
     }
     for name, c in cases.items():
         if c.rotating:

@@ -78,6 +78,20 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
 
+// ---- bfloat16 pairs consumed packed (sm_100 mixed-precision fma) ----------------------
+// (lo(u) lo(v) + c.x, hi(u) hi(v) + c.y): each a float32 fma of the bfloat16 halves of two
+// packed words -- the exact product plus c, rounded once, as the float32 fma of the unpacked
+// values would give -- with no unpacking.
+__device__ __forceinline__ float2 bf16x2_mac(uint32_t u, uint32_t v, float2 c) {
+    float lo, hi;
+    asm("{\n\t.reg .b16 ul, uh, vl, vh;\n\tmov.b32 {ul, uh}, %2;\n\tmov.b32 {vl, vh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, ul, vl, %4;\n\tfma.rn.f32.bf16 %1, uh, vh, %5;\n}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(u), "r"(v), "f"(c.x), "f"(c.y));
+    return make_float2(lo, hi);
+}
+constexpr uint32_t kBf16x2One = 0x3F803F80u;  // (1, 1)
+
 // ---- 16-byte global memory access -------------------------------------------------
 // Streaming loads (read once: evict-first) and stores for the row data; plain cached
 // loads for the per-column parameters that every row reuses.

@@ -261,12 +261,16 @@ constexpr int kStaticSmemReserve = 2048;  // static shared memory + per-CTA syst
 // (64 bytes a vector) must fit the shared memory.
 bool slots_shape(int nvec, const nv_plan& req, const DevInfo* di, nv_plan* out) {
     nv_plan p = req;
-    int v = p.vec_per_thread ? p.vec_per_thread : (nvec >= 256 ? 8 : 4);
+    // measured on B200 (bf16, 2^27 elements): 8 vectors a thread in CTAs of 768 threads,
+    // except rows of 257..512 vectors (D = 4096), which run 4 % faster with 4 vectors a
+    // thread in CTAs of 1024 threads (32 warps at 64 registers)
+    const bool mid = nvec > 256 && nvec <= 512;
+    int v = p.vec_per_thread ? p.vec_per_thread : (nvec >= 256 && !mid ? 8 : 4);
     if (v != 4 && v != 8) return false;
     int g = p.threads_per_row ? p.threads_per_row : ((nvec + v - 1) / v + 31) / 32 * 32;
     if (g % 32 || g < 32 || (int64_t)g * v < nvec || g > kSlotsMaxThreads) return false;
     // 768 threads (24 warps, 80 registers) unless asked for more rows per CTA
-    int slots = p.rows_per_cta ? p.rows_per_cta : 768 / g;
+    int slots = p.rows_per_cta ? p.rows_per_cta : ((mid && v == 4) ? 1024 : 768) / g;
     if (g > 32) slots = std::min(slots, 15);
     if (slots < 1 || slots * g > kSlotsMaxThreads || (g > 32 && slots > 15)) return false;
     const size_t optin = (size_t)(di ? di->smem_optin : 232448) - kStaticSmemReserve;
@@ -1152,7 +1156,11 @@ template <typename T>
 nv_status run_vjp(Op op, VjpArgs a, int vpt, int cap, const DevInfo& di, cudaStream_t s,
                   void* dw, void* db) {
     const int G = vpt == 0 ? 256 : ((a.nvec + vpt - 1) / vpt + 31) / 32 * 32;
+    // rms_norm_vjp with one vector a thread and CTAs of at most 512 threads reduces two rows
+    // at a time (half the barriers per row)
+    const bool pairs = op == OP_RMS && vpt == 1 && G <= kVjpPairsMaxThreads;
     auto k1 = vpt == 0 ? (op == OP_RMS ? vjp_generic_kernel<T, false> : vjp_generic_kernel<T, true>)
+              : pairs ? rms_vjp_pairs_kernel<T, 1>
               : op == OP_RMS
                   ? (vpt == 1 ? rms_vjp_kernel<T, 1>
                               : vpt == 2 ? rms_vjp_kernel<T, 2> : rms_vjp_kernel<T, 4>)

@@ -63,7 +63,7 @@ constexpr int kLanesPerSum = N == 2 ? 16 : 8;
 
 template <int N>
 __device__ __forceinline__ float warp_sums(const float (&v)[N]) {
-    static_assert(N == 2 || N == 3, "two or three sums");
+    static_assert(N >= 2 && N <= 4, "two to four sums");
     const int lane = threadIdx.x & 31;
     float keep;
     if constexpr (N == 2) {
@@ -71,10 +71,12 @@ __device__ __forceinline__ float warp_sums(const float (&v)[N]) {
         keep = hi ? v[1] : v[0];
         keep += __shfl_xor_sync(0xFFFFFFFFu, hi ? v[0] : v[1], 16);
     } else {
+        // four slots (the fourth a zero pad when N = 3)
+        const float v3 = N == 4 ? v[N - 1] : 0.f;
         const bool b4 = lane & 16, b3 = lane & 8;
-        float k0 = b4 ? v[2] : v[0], k1 = b4 ? 0.f : v[1];
+        float k0 = b4 ? v[2] : v[0], k1 = b4 ? v3 : v[1];
         k0 += __shfl_xor_sync(0xFFFFFFFFu, b4 ? v[0] : v[2], 16);
-        k1 += __shfl_xor_sync(0xFFFFFFFFu, b4 ? v[1] : 0.f, 16);
+        k1 += __shfl_xor_sync(0xFFFFFFFFu, b4 ? v[1] : v3, 16);
         keep = b3 ? k1 : k0;
         keep += __shfl_xor_sync(0xFFFFFFFFu, b3 ? k0 : k1, 8);
     }
@@ -215,16 +217,23 @@ struct RmsVjpRow {
 
     __device__ __forceinline__ void operator()(int64_t row, const V16 (&xv)[VPT],
                                                const V16 (&gv)[VPT]) const {
-        // sum x^2 (the scale) and sum g w x (the projection)
+        // sum x^2 (the scale) and sum g w x (the projection); bfloat16 pairs consumed packed
+        // (x x and g x exact products, (g x) w exact too: 8 + 8 + 8 significant bits)
         float2 s0 = splat2(0.f), s1 = splat2(0.f);
 #pragma unroll
         for (int k = 0; k < VPT; ++k)
 #pragma unroll
             for (int e = 0; e < VEC; e += 2) {
-                const float2 x2 = E::get2(xv[k], e);
-                const float2 u2 = mul2(E::get2(gv[k], e), wf[k][e / 2]);
-                s0 = fma2(x2, x2, s0);
-                s1 = fma2(u2, x2, s1);
+                if constexpr (sizeof(T) == 2) {
+                    s0 = bf16x2_mac(xv[k].u[e / 2], xv[k].u[e / 2], s0);
+                    s1 = fma2(bf16x2_mac(gv[k].u[e / 2], xv[k].u[e / 2], splat2(0.f)),
+                              wf[k][e / 2], s1);
+                } else {
+                    const float2 x2 = E::get2(xv[k], e);
+                    const float2 u2 = mul2(E::get2(gv[k], e), wf[k][e / 2]);
+                    s0 = fma2(x2, x2, s0);
+                    s1 = fma2(u2, x2, s1);
+                }
             }
         float s[2] = {__fadd_rn(s0.x, s0.y), __fadd_rn(s1.x, s1.y)};
         cta_sum<2>(s, red);
@@ -287,6 +296,127 @@ __global__ void __launch_bounds__(vjp_max_threads(VPT)) rms_vjp_kernel(const Vjp
     }
 }
 
+// ---- RmsNormVjp, kernel 1, two rows per reduction -------------------------------------------
+// The same arithmetic as RmsVjpRow, but each CTA reduces the sums of two rows at once (four
+// values in one butterfly and one cta_sum): half the barriers per row.  Rows p, p + parts,
+// p + 2 parts, ... are taken in pairs; while one pair is reduced and written, the next
+// pair's loads are in flight (four register sets).
+template <typename TT, int VPT>
+struct RmsVjpPair {
+    using T = TT;
+    using E = Elem<T>;
+    static constexpr int VEC = E::kVec;
+    static constexpr int NP = VEC / 2;
+    const VjpArgs& a;
+    const float2 (&wf)[VPT][NP];
+    ColAcc<VPT, NP, 1>& acc;
+    CtaSums<4>& red;
+    float invD;
+
+    __device__ __forceinline__ void sums(const V16 (&xv)[VPT], const V16 (&gv)[VPT], float& ss,
+                                         float& sp) const {
+        float2 s0 = splat2(0.f), s1 = splat2(0.f);
+#pragma unroll
+        for (int k = 0; k < VPT; ++k)
+#pragma unroll
+            for (int e = 0; e < VEC; e += 2) {
+                if constexpr (sizeof(T) == 2) {
+                    s0 = bf16x2_mac(xv[k].u[e / 2], xv[k].u[e / 2], s0);
+                    s1 = fma2(bf16x2_mac(gv[k].u[e / 2], xv[k].u[e / 2], splat2(0.f)),
+                              wf[k][e / 2], s1);
+                } else {
+                    const float2 x2 = E::get2(xv[k], e);
+                    const float2 u2 = mul2(E::get2(gv[k], e), wf[k][e / 2]);
+                    s0 = fma2(x2, x2, s0);
+                    s1 = fma2(u2, x2, s1);
+                }
+            }
+        ss = __fadd_rn(s0.x, s0.y);
+        sp = __fadd_rn(s1.x, s1.y);
+    }
+    __device__ __forceinline__ void write(int64_t row, const V16 (&xv)[VPT], const V16 (&gv)[VPT],
+                                          float ss, float sp) const {
+        const float r = rsqrtf(__fmaf_rn(ss, invD, a.eps));
+        const float vr = __fmul_rn(__fmul_rn(r, r), __fmul_rn(sp, invD));
+        const float2 r2 = splat2(r), nv2 = splat2(-vr);
+        const bool live = row < a.rows;
+        const size_t roff = (size_t)row * (size_t)a.nvec * 16;
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            const int v = threadIdx.x + k * blockDim.x;
+            if (v < a.nvec) {
+                V16 o;
+#pragma unroll
+                for (int e = 0; e < VEC; e += 2) {
+                    const float2 x2 = E::get2(xv[k], e);
+                    const float2 g2 = E::get2(gv[k], e);
+                    const float2 u2 = mul2(g2, wf[k][e / 2]);
+                    E::put2(o, e, mul2(r2, fma2(x2, nv2, u2)));        // r (g w - x v)
+                    float2& ac = acc.at(0, k * NP + e / 2);
+                    ac = fma2(mul2(g2, x2), r2, ac);  // a row past the end holds zeros
+                }
+                if (live) st_stream(static_cast<char*>(a.dx) + roff + (size_t)v * 16, o);
+            }
+        }
+    }
+    __device__ __forceinline__ void operator()(int64_t r0, const V16 (&x0)[VPT], const V16 (&g0)[VPT],
+                                               int64_t r1, const V16 (&x1)[VPT],
+                                               const V16 (&g1)[VPT]) const {
+        float s[4];
+        sums(x0, g0, s[0], s[1]);
+        sums(x1, g1, s[2], s[3]);
+        cta_sum<4>(s, red);
+        write(r0, x0, g0, s[0], s[1]);
+        write(r1, x1, g1, s[2], s[3]);
+    }
+};
+
+template <int VPT, typename Pair>
+__device__ __forceinline__ void walk_row_pairs(const VjpArgs& a, Pair&& pair_step) {
+    using T = typename Pair::T;
+    V16 xa[VPT], ga[VPT], xb[VPT], gb[VPT], xc[VPT], gc[VPT], xd[VPT], gd[VPT];
+    const int64_t step = a.parts;
+    load_xg<T, VPT>(a, blockIdx.x, xa, ga);
+    load_xg<T, VPT>(a, blockIdx.x + step, xb, gb);
+    for (int64_t row = blockIdx.x; row < a.rows; row += 4 * step) {
+        load_xg<T, VPT>(a, row + 2 * step, xc, gc);
+        load_xg<T, VPT>(a, row + 3 * step, xd, gd);
+        pair_step(row, xa, ga, row + step, xb, gb);
+        if (row + 2 * step >= a.rows) break;
+        load_xg<T, VPT>(a, row + 4 * step, xa, ga);
+        load_xg<T, VPT>(a, row + 5 * step, xb, gb);
+        pair_step(row + 2 * step, xc, gc, row + 3 * step, xd, gd);
+    }
+}
+
+// CTAs of at most 512 threads: the four register sets need up to 128 registers.
+constexpr int kVjpPairsMaxThreads = 512;
+
+template <typename T, int VPT>
+__global__ void __launch_bounds__(kVjpPairsMaxThreads) rms_vjp_pairs_kernel(const VjpArgs a) {
+    pdl_wait();
+    pdl_release();
+    constexpr int NP = Elem<T>::kVec / 2;
+    __shared__ CtaSums<4> red;
+    extern __shared__ float2 acc_smem[];
+    float2 wf[VPT][NP];
+    load_wf<T, VPT>(a, wf);
+    ColAcc<VPT, NP, 1> acc;
+    acc.init(acc_smem);
+    walk_row_pairs<VPT>(a, RmsVjpPair<T, VPT>{a, wf, acc, red, 1.f / (float)a.D});
+    if (a.want_dw) {
+        float* out = a.part + (size_t)blockIdx.x * a.D;
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            const int v = threadIdx.x + k * blockDim.x;
+            if (v < a.nvec)
+#pragma unroll
+                for (int i = 0; i < NP; ++i)
+                    reinterpret_cast<float2*>(out)[v * NP + i] = acc.at(0, k * NP + i);
+        }
+    }
+}
+
 // ---- LayerNormVjp, kernel 1 ---------------------------------------------------------------
 template <typename TT, int VPT>
 struct LayerVjpRow {
@@ -306,14 +436,22 @@ struct LayerVjpRow {
         if (VPT > 2)
 #pragma unroll
             for (int k = 0; k < VPT; ++k) wv[k] = load_w<T>(a, k);
+        // bfloat16 pairs are consumed packed (bf16x2_mac: the same single roundings as the
+        // float32 arithmetic on the unpacked values, without the unpacking)
+        constexpr bool kPacked = sizeof(T) == 2;
         // pass 1: sum x and sum a (a = w g)
         float2 p0 = splat2(0.f), p1 = splat2(0.f);
 #pragma unroll
         for (int k = 0; k < VPT; ++k)
 #pragma unroll
             for (int e = 0; e < VEC; e += 2) {
-                p0 = add2(p0, E::get2(xv[k], e));
-                p1 = add2(p1, mul2(E::get2(wv[k], e), E::get2(gv[k], e)));
+                if constexpr (kPacked) {
+                    p0 = bf16x2_mac(xv[k].u[e / 2], kBf16x2One, p0);
+                    p1 = bf16x2_mac(wv[k].u[e / 2], gv[k].u[e / 2], p1);
+                } else {
+                    p0 = add2(p0, E::get2(xv[k], e));
+                    p1 = add2(p1, mul2(E::get2(wv[k], e), E::get2(gv[k], e)));
+                }
             }
         float p[2] = {__fadd_rn(p0.x, p0.y), __fadd_rn(p1.x, p1.y)};
         cta_sum<2>(p, red1);
@@ -328,8 +466,14 @@ struct LayerVjpRow {
             if (v < a.nvec)   // c' of a padding lane would be -m1
 #pragma unroll
                 for (int e = 0; e < VEC; e += 2) {
-                    const float2 cp = add2(E::get2(xv[k], e), nm1);
-                    const float2 a2 = mul2(E::get2(wv[k], e), E::get2(gv[k], e));
+                    float2 cp, a2;
+                    if constexpr (kPacked) {
+                        cp = bf16x2_mac(xv[k].u[e / 2], kBf16x2One, nm1);
+                        a2 = bf16x2_mac(wv[k].u[e / 2], gv[k].u[e / 2], splat2(0.f));
+                    } else {
+                        cp = add2(E::get2(xv[k], e), nm1);
+                        a2 = mul2(E::get2(wv[k], e), E::get2(gv[k], e));
+                    }
                     q0 = add2(q0, cp);
                     q1 = fma2(cp, cp, q1);
                     q2 = fma2(a2, cp, q2);
@@ -352,8 +496,14 @@ struct LayerVjpRow {
 #pragma unroll
                 for (int e = 0; e < VEC; e += 2) {
                     const float2 g2 = E::get2(gv[k], e);
-                    const float2 a2 = mul2(E::get2(wv[k], e), g2);
-                    const float2 c2 = add2(add2(E::get2(xv[k], e), nm1), ndm);
+                    float2 a2, c2;
+                    if constexpr (kPacked) {
+                        a2 = bf16x2_mac(wv[k].u[e / 2], gv[k].u[e / 2], splat2(0.f));
+                        c2 = add2(bf16x2_mac(xv[k].u[e / 2], kBf16x2One, nm1), ndm);
+                    } else {
+                        a2 = mul2(E::get2(wv[k], e), g2);
+                        c2 = add2(add2(E::get2(xv[k], e), nm1), ndm);
+                    }
                     E::put2(o, e, mul2(r2, fma2(c2, nB, add2(a2, nma))));
                     float2& aw = acc.at(0, k * NP + e / 2);
                     float2& ab = acc.at(1, k * NP + e / 2);
