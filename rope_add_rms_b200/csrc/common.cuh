@@ -72,6 +72,11 @@ struct Elem<__nv_bfloat16> {
     __device__ __forceinline__ static void put2(V16& v, int e, float2 p) { put2(v, e, p.x, p.y); }
 };
 
+// Bulk prefetch of `bytes` (a multiple of 16) at global address p (16-byte aligned) into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // ---- packed float32 pairs (Blackwell FFMA2 / FADD2 / FMUL2; IEEE per lane) ------------
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }

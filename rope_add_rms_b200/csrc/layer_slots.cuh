@@ -77,11 +77,6 @@ __host__ __device__ constexpr size_t slots_table_bytes(int nvec) {
 // (32 warps, up to 64 registers).
 constexpr int kSlotsMaxThreads = 1024;
 
-// Bulk prefetch of `bytes` (a multiple of 16) at global address p (16-byte aligned) into L2.
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // Launch: blockDim.x = a.G * a.rows_per_cta (rows_per_cta = slots <= 15 when G > 32),
 // dynamic shared memory = slots_table_bytes(a.nvec); persistent grid.
 template <int VPT, bool PREFETCH, int MAXT>

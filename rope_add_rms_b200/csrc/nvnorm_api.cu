@@ -682,14 +682,20 @@ nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a,
     const size_t smem = (size_t)a.half * sizeof(float4) +
                         (pairs ? (size_t)Elem<T>::kVec / 2 * (size_t)(a.nvec / 2) * sizeof(float4)
                                : 0);
-    auto kern = pairs ? rope_pairs_kernel<T, TRAD> : rope_rows_kernel<T, TRAD>;
+    // the pairs kernel with lanes per row fixed at compile time where hvec is 4, 8 or 16
+    const int hv = pairs && a.lpr == a.nvec / 2 ? a.nvec / 2 : 0;
+    auto kern = !pairs   ? rope_rows_kernel<T, TRAD>
+                : hv == 8  ? rope_pairs_kernel<T, TRAD, 8>
+                : hv == 16 ? rope_pairs_kernel<T, TRAD, 16>
+                : hv == 4  ? rope_pairs_kernel<T, TRAD, 4>
+                           : rope_pairs_kernel<T, TRAD, 0>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     }
     (void)di;
-    return launch_kernel(kern, a.L * a.n_chunks, 256, smem, s, a);
+    return launch_kernel(kern, a.L * a.n_chunks, kRopeThreads, smem, s, a);
 }
 
 template <typename T>
@@ -723,7 +729,7 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
                         vecw, 32 * vecw, vecw);
         const int lanes_needed = rp->pairs ? (int)(nvec / 2) : (int)nvec;
         const int lpr = pow2_ceil(std::max(lanes_needed, 1));
-        const int slots = 256 / lpr;
+        const int slots = kRopeThreads / lpr;
         const int64_t BH = rows / L;
         int64_t bt = p.rows_per_cta;
         if (bt <= 0) {
@@ -1193,7 +1199,7 @@ nv_status run_vjp(Op op, VjpArgs a, int vpt, int cap, const DevInfo& di, cudaStr
     r.out[0] = dw ? dw : db;
     r.out[1] = db;
     const dim3 grid((unsigned)((a.D + 31) / 32), (dw && db) ? 2u : 1u);
-    return launch_kernel(vjp_reduce_kernel<T>, grid, kReduceWarps * 32, 0, s, r);
+    return launch_kernel(vjp_reduce_kernel<T>, grid, reduce_warps(r.parts) * 32, 0, s, r);
 }
 
 nv_status vjp_op(Op op, const void* x, const void* w, const void* g, void* dx, void* dw, void* db,

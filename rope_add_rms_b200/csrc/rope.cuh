@@ -360,26 +360,118 @@ struct PairLayout {
     }
 };
 
+// The angle records of position offset + l, written by threads t = 0, n, 2n, ... < half:
+// C [half / 2] then S [half / 2], each record serving two pairs (PairLayout::record_of).
 template <typename T, bool TRAD>
-__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 4 : 3) rope_pairs_kernel(const RopeArgs a) {
-    using E = Elem<T>;
+__device__ __forceinline__ void build_angle_records(const RopeArgs& a, float4* ctab, int64_t l,
+                                                    int t, int n) {
+    using PL = PairLayout<T, TRAD>;
+    const double pos = (double)(a.offset + l);
+    float* tabf = reinterpret_cast<float*>(ctab);
+    const int nrec = a.half / 2;
+    const int hvec = a.nvec / 2;
+    for (int i = t; i < a.half; i += n) {
+        int h = 0;
+        const int rec = PL::record_of(i, hvec, h);
+        const float4 e = angle_entry(a, pos, i);
+        tabf[rec * 4 + h] = e.x;               // C: cos_hi, cos_lo
+        tabf[rec * 4 + 2 + h] = e.y;
+        tabf[(nrec + rec) * 4 + h] = e.z;      // S: sin_hi, sin_lo
+        tabf[(nrec + rec) * 4 + 2 + h] = e.w;
+    }
+}
+
+// The lanes' weight records W [NP][nvec / 2]; lanes with a vector (has_vec) read w and
+// those of slot 0 (write) store the records.
+template <typename T, bool TRAD>
+__device__ __forceinline__ void store_weight_records(const RopeArgs& a, float4* wtab, int v0,
+                                                     int v1, bool has_vec, bool write) {
     using PL = PairLayout<T, TRAD>;
     constexpr int NP = PL::NP;
-    // rows in flight per lane group (measured best of 2..4 at three CTAs per SM: 2 for
-    // bfloat16, 4 for the float32 rows that carry twice the bytes per element)
-    constexpr int kUnroll = sizeof(T) == 4 ? 4 : 2;
-    // records: C [half / 2], S [half / 2], then the lanes' weights W [NP][nvec / 2]
+    const bool has_w = a.normalize != 0 && a.w != nullptr && has_vec;
+    const V16 wa = has_w ? ld_param(static_cast<const char*>(a.w) + (size_t)v0 * 16) : ones_vec<T>();
+    const V16 wb = has_w ? ld_param(static_cast<const char*>(a.w) + (size_t)v1 * 16) : ones_vec<T>();
+    float2 wp[NP], wq[NP];
+    PL::split(wa, wb, wp, wq);
+    if (write)
+#pragma unroll
+        for (int k = 0; k < NP; ++k)
+            wtab[k * (a.nvec / 2) + v0] = make_float4(wp[k].x, wp[k].y, wq[k].x, wq[k].y);
+}
+
+// One row of the two-vectors-per-lane layout: sum of squares over the lane group, then the
+// rotation of this lane's pairs, weights applied first and the row's 1/rms last.  Every
+// lane of the group takes part (the group sum); lanes with live == false store nothing.
+// hvec = nvec / 2 vectors a lane group covers per side, lpr lanes per row; with dims == D
+// the table holds hvec * NP C records, then as many S records.
+template <typename T, bool TRAD>
+__device__ __forceinline__ void rope_pairs_row(const RopeArgs& a, const float4* ctab,
+                                               const float4* wtab, const V16& xa, const V16& xb,
+                                               bool live, int v0, int v1, int hvec, int lpr,
+                                               float invD, char* yrow) {
+    using PL = PairLayout<T, TRAD>;
+    constexpr int NP = PL::NP;
+    float2 p[NP], q[NP];
+    PL::split(xa, xb, p, q);
+    float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < NP; ++k) {
+        ss2 = fma2(p[k], p[k], ss2);
+        ss2 = fma2(q[k], q[k], ss2);
+    }
+    const float ss = group_sum(__fadd_rn(ss2.x, ss2.y), lpr);
+    const float inv = a.normalize ? rsqrtf(__fmaf_rn(ss, invD, a.eps)) : 1.f;
+    const float2 inv2 = make_float2(inv, inv);
+    if (live) {  // only lanes holding vectors read the table
+        float2 yp[NP], yq[NP];
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+            const int rec = PL::record(v0, v1, k, hvec);
+            const float4 c4 = ctab[rec], s4 = ctab[hvec * NP + rec];
+            const float2 ch = make_float2(c4.x, c4.y), cl = make_float2(c4.z, c4.w);
+            const float2 sh = make_float2(s4.x, s4.y), sl = make_float2(s4.z, s4.w);
+            const float4 w4 = wtab[k * hvec + v0];
+            const float2 ap = mul2(p[k], make_float2(w4.x, w4.y));  // exact for bf16 data
+            const float2 aq = mul2(q[k], make_float2(w4.z, w4.w));
+            yp[k] = mul2(rotate_sub2(ap, aq, ch, cl, sh, sl), inv2);
+            yq[k] = mul2(rotate_pair2(aq, ap, ch, cl, sh, sl), inv2);
+        }
+        V16 o0, o1;
+        PL::join(yp, yq, o0, o1);
+        st_stream(yrow + (size_t)v0 * 16, o0);
+        st_stream(yrow + (size_t)v1 * 16, o1);
+    }
+}
+
+// rows in flight per lane group (measured best of 2..4 at three or four CTAs per SM: 2 for
+// bfloat16, 4 for the float32 rows that carry twice the bytes per element)
+template <typename T>
+__host__ __device__ constexpr int rope_pairs_unroll() { return sizeof(T) == 4 ? 4 : 2; }
+
+// One CTA of kRopeThreads per (position l, chunk of bt rows): the table of l is built while
+// the chunk's first rows load.  HV > 0 fixes hvec = nvec / 2 = lanes per row at compile time
+// (4, 8 or 16: D = 128 in bfloat16 is 8), so every table and row offset is a constant and
+// the group sum a fixed butterfly; HV = 0 takes them from the arguments.
+constexpr int kRopeThreads = 256;
+
+template <typename T, bool TRAD, int HV>
+__global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
+    rope_pairs_kernel(const RopeArgs a) {
+    constexpr int kUnroll = rope_pairs_unroll<T>();
+    constexpr int NP = PairLayout<T, TRAD>::NP;
+    // records: C [hvec NP], S [hvec NP], then the lanes' weights W [NP][hvec]
     extern __shared__ float4 tab[];
 
     const int64_t chunk = blockIdx.x % a.n_chunks;
     const int64_t l = blockIdx.x / a.n_chunks;
-    const int lpr = a.lpr;
+    const int hvec = HV > 0 ? HV : a.nvec / 2;
+    const int lpr = HV > 0 ? HV : a.lpr;
     const int lane = threadIdx.x & (lpr - 1);
     const int slot = threadIdx.x / lpr;
-    const int slots = blockDim.x / lpr;
-    const int hvec = a.nvec / 2;
+    const int slots = kRopeThreads / lpr;
     const int v0 = lane, v1 = lane + hvec;
-    const bool has_vec = lane < hvec;
+    // with HV fixed every lane of a group holds vectors (lpr == hvec)
+    const bool has_vec = HV > 0 || lane < hvec;
 
     pdl_wait();
     pdl_release();
@@ -396,37 +488,28 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 4 : 3) rope_pairs_kernel
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
         const int64_t b = bh0 + slot + (int64_t)u * slots;
+        xv[u][0] = zeros_vec<T>();
+        xv[u][1] = zeros_vec<T>();
         if (has_vec && b < bh_end) {
             xv[u][0] = ld_stream(xbase + (size_t)b * lstride + (size_t)v0 * 16);
             xv[u][1] = ld_stream(xbase + (size_t)b * lstride + (size_t)v1 * 16);
         }
     }
-    const bool norm = a.normalize != 0;
-    {
-        const V16 wa = (norm && a.w && has_vec)
-                           ? ld_param(static_cast<const char*>(a.w) + (size_t)v0 * 16) : ones_vec<T>();
-        const V16 wb = (norm && a.w && has_vec)
-                           ? ld_param(static_cast<const char*>(a.w) + (size_t)v1 * 16) : ones_vec<T>();
-        // the angle table is built while the first rows' loads are in flight
-        const double pos = (double)(a.offset + l);
-        float* tabf = reinterpret_cast<float*>(tab);
-        const int nrec = a.half / 2;
-        for (int i = threadIdx.x; i < a.half; i += blockDim.x) {
-            int h = 0;
-            const int rec = PL::record_of(i, hvec, h);
-            const float4 t = angle_entry(a, pos, i);
-            tabf[rec * 4 + h] = t.x;               // C: cos_hi, cos_lo
-            tabf[rec * 4 + 2 + h] = t.y;
-            tabf[(nrec + rec) * 4 + h] = t.z;      // S: sin_hi, sin_lo
-            tabf[(nrec + rec) * 4 + 2 + h] = t.w;
-        }
-        float2 wp[NP], wq[NP];
-        PL::split(wa, wb, wp, wq);
-        if (slot == 0 && has_vec)
+    // The next kUnroll rows of each slot are asked of L2 now (one bulk prefetch per row, by
+    // the group's lane 0), so the first round after the table finds them on chip: a CTA's
+    // start costs one DRAM latency instead of two.  Measured on bf16 [8, 32, 2048, 128]:
+    // 47.7 us against 48.2 us without; asking for the whole chunk at once 54.0, two rounds
+    // ahead 49.5, and a rolling prefetch two rounds ahead of every row 50.7.
+    if (has_vec && lane == 0)
 #pragma unroll
-            for (int k = 0; k < NP; ++k)
-                tab[a.half + k * hvec + v0] = make_float4(wp[k].x, wp[k].y, wq[k].x, wq[k].y);
-    }
+        for (int u = kUnroll; u < 2 * kUnroll; ++u) {
+            const int64_t b = bh0 + slot + (int64_t)u * slots;
+            if (b < bh_end) prefetch_l2(xbase + (size_t)b * lstride, (uint32_t)row_bytes);
+        }
+    // the angle table is built while the first rows' loads are in flight
+    float4* wtab = tab + 2 * hvec * NP;
+    build_angle_records<T, TRAD>(a, tab, l, threadIdx.x, kRopeThreads);
+    store_weight_records<T, TRAD>(a, wtab, v0, v1, has_vec, slot == 0 && has_vec);
     __syncthreads();
 
     const float invD = 1.0f / (float)a.D;
@@ -435,43 +518,17 @@ __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 4 : 3) rope_pairs_kernel
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t b = base + slot + (int64_t)u * slots;
             const bool live = has_vec && b < bh_end;
-            V16 xa = live ? xv[u][0] : zeros_vec<T>();
-            V16 xb = live ? xv[u][1] : zeros_vec<T>();
+            // a row past the chunk is reduced from stale registers and not stored; lanes
+            // without a vector keep the zeros they started with, so add nothing to the sum
+            const V16 xa = xv[u][0];
+            const V16 xb = xv[u][1];
             const int64_t bn = b + (int64_t)kUnroll * slots;
             if (has_vec && bn < bh_end) {
                 xv[u][0] = ld_stream(xbase + (size_t)bn * lstride + (size_t)v0 * 16);
                 xv[u][1] = ld_stream(xbase + (size_t)bn * lstride + (size_t)v1 * 16);
             }
-            float2 p[NP], q[NP];
-            PL::split(xa, xb, p, q);
-            float2 ss2 = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int k = 0; k < NP; ++k) {
-                ss2 = fma2(p[k], p[k], ss2);
-                ss2 = fma2(q[k], q[k], ss2);
-            }
-            const float ss = group_sum(__fadd_rn(ss2.x, ss2.y), lpr);
-            const float inv = norm ? rsqrtf(__fmaf_rn(ss, invD, a.eps)) : 1.f;
-            const float2 inv2 = make_float2(inv, inv);
-            if (live) {  // only lanes holding vectors read the table
-                float2 yp[NP], yq[NP];
-#pragma unroll
-                for (int k = 0; k < NP; ++k) {
-                    const int rec = PL::record(v0, v1, k, hvec);
-                    const float4 c4 = tab[rec], s4 = tab[a.half / 2 + rec];
-                    const float2 ch = make_float2(c4.x, c4.y), cl = make_float2(c4.z, c4.w);
-                    const float2 sh = make_float2(s4.x, s4.y), sl = make_float2(s4.z, s4.w);
-                    const float4 w4 = tab[a.half + k * hvec + v0];
-                    const float2 ap = mul2(p[k], make_float2(w4.x, w4.y));  // exact for bf16 data
-                    const float2 aq = mul2(q[k], make_float2(w4.z, w4.w));
-                    yp[k] = mul2(rotate_sub2(ap, aq, ch, cl, sh, sl), inv2);
-                    yq[k] = mul2(rotate_pair2(aq, ap, ch, cl, sh, sl), inv2);
-                }
-                V16 o0, o1;
-                PL::join(yp, yq, o0, o1);
-                st_stream(ybase + (size_t)b * ystride + (size_t)v0 * 16, o0);
-                st_stream(ybase + (size_t)b * ystride + (size_t)v1 * 16, o1);
-            }
+            rope_pairs_row<T, TRAD>(a, tab, wtab, xa, xb, live, v0, v1, hvec, lpr, invD,
+                                    ybase + (size_t)b * ystride);
         }
     }
 }

@@ -629,10 +629,13 @@ __global__ void __launch_bounds__(256) vjp_generic_kernel(const VjpArgs a) {
 
 // ---- kernel 2: column sums of the partials --------------------------------------------------
 // out[y][j] = sum_{p < parts} part[first + y][p][j] in double, y = blockIdx.y.
-// A CTA owns 32 columns; warp w adds parts w, w + 32, w + 64, ... in that order (eight
-// loads in flight per lane), then the 32 warp sums are added pairwise in a fixed tree:
-// a fixed order, so the result does not depend on timing.
-constexpr int kReduceWarps = 32;
+// A CTA of nw = blockDim.x / 32 warps owns 32 columns.  Warp w adds the contiguous run of
+// parts [w per, (w + 1) per) in order, per = ceil(parts / nw), with up to kReduceBatch loads
+// in flight per lane; the host picks nw = ceil(parts / kReduceBatch) (at most 32), so a warp
+// waits for one batch of loads.  After one barrier warp 0 adds the warps' sums in warp
+// order.  The order is fixed, so the result does not depend on timing.
+constexpr int kReduceBatch = 16;
+constexpr int kReduceMaxWarps = 32;
 
 struct ReduceArgs {
     const float* part;  // [nsum][parts][D]
@@ -642,30 +645,53 @@ struct ReduceArgs {
     int D;
 };
 
+// warps per CTA of vjp_reduce_kernel for `parts` partial rows
+__host__ __device__ constexpr int reduce_warps(int parts) {
+    return parts <= kReduceBatch ? 1
+           : (parts + kReduceBatch - 1) / kReduceBatch > kReduceMaxWarps
+               ? kReduceMaxWarps
+               : (parts + kReduceBatch - 1) / kReduceBatch;
+}
+
 template <typename T>
-__global__ void __launch_bounds__(kReduceWarps * 32) vjp_reduce_kernel(const ReduceArgs a) {
+__global__ void __launch_bounds__(kReduceMaxWarps * 32) vjp_reduce_kernel(const ReduceArgs a) {
     pdl_wait();
     pdl_release();
-    __shared__ double sw[kReduceWarps][32];
+    __shared__ double sw[kReduceMaxWarps][32];
     const int lane = threadIdx.x & 31;
     const int w = threadIdx.x >> 5;
+    const int nw = blockDim.x >> 5;
     const int j = blockIdx.x * 32 + lane;
     const float* part =
         a.part ? a.part + (size_t)(a.first + blockIdx.y) * a.parts * a.D : nullptr;
+    const int per = (a.parts + nw - 1) / nw;
+    const int p0 = min(w * per, a.parts);
+    const int p1 = min(p0 + per, a.parts);
     double s = 0.0;
     if (j < a.D && part) {
-#pragma unroll 8
-        for (int p = w; p < a.parts; p += kReduceWarps) s += (double)part[(size_t)p * a.D + j];
+        const float* col = part + (size_t)p0 * a.D + j;
+        int n = p1 - p0;
+        for (; n >= kReduceBatch; n -= kReduceBatch, col += (size_t)kReduceBatch * a.D) {
+            float v[kReduceBatch];
+#pragma unroll
+            for (int i = 0; i < kReduceBatch; ++i) v[i] = col[(size_t)i * a.D];
+#pragma unroll
+            for (int i = 0; i < kReduceBatch; ++i) s += (double)v[i];
+        }
+        float v[kReduceBatch];
+#pragma unroll
+        for (int i = 0; i < kReduceBatch; ++i) v[i] = i < n ? col[(size_t)i * a.D] : 0.f;
+#pragma unroll
+        for (int i = 0; i < kReduceBatch; ++i)
+            if (i < n) s += (double)v[i];
     }
     sw[w][lane] = s;
     __syncthreads();
-#pragma unroll
-    for (int stride = kReduceWarps / 2; stride >= 1; stride >>= 1) {
-        if (w < stride) sw[w][lane] += sw[w + stride][lane];
-        __syncthreads();
+    if (w == 0 && j < a.D) {
+        double t = sw[0][lane];
+        for (int i = 1; i < nw; ++i) t += sw[i][lane];
+        Elem<T>::store1(blockIdx.y ? a.out[1] : a.out[0], j, __double2float_rn(t));
     }
-    if (w == 0 && j < a.D)
-        Elem<T>::store1(blockIdx.y ? a.out[1] : a.out[0], j, __double2float_rn(sw[0][lane]));
 }
 
 }  // namespace nvn

@@ -456,6 +456,9 @@ ROPE_CASES = [
     (1, 2, 12, 1000, 96, 1, 2, 1, True),     # D > 256: generic path
     (1, 1, 6, 6, 4, 0, 1, 1, True),
     (1, 600, 1, 128, 128, 0, 4095, 1, True),  # decode-like: one position, many rows
+    (2, 3, 40, 96, 96, 0, 11, 1, True),      # two vectors per lane, lanes without a vector
+    (2, 3, 40, 96, 96, 1, 11, 1, True),
+    (1, 2, 30, 192, 192, 0, 5, 1, True),
 ]
 
 
