@@ -1043,6 +1043,27 @@ def test_layer_norm_vjp_large_mean(dt, mean, std):
     check_grad(db, ref[2], ref[5], "db")
 
 
+@pytest.mark.parametrize("dt,D", [("bf16", 1024), ("bf16", 8192), ("f32", 4096)])
+def test_layer_norm_vjp_mixed_conditioning(dt, D):
+    """Every CTA walks rows of several kinds in turn: means small against the spread, means
+    that dwarf it (mean / std = 150) and means of the order of the spread (|mean| around
+    std / 2 and above): any statistic that leans on E[x^2] - mean^2, or on a mean carried
+    over from another row, fails on some of them."""
+    rows = 1500
+    x = synth.normal((rows, D), 0.5, 2.0, 47, 0, dt)
+    x[1::3] += 300.0                 # mean / std = 150
+    x[2::6] = x[2::6] * 0.5 + 0.25   # mean 0.5, std 1
+    x[5::6] = x[5::6] * 0.25 + 0.5   # mean 0.625, std 0.5
+    w = synth.normal((D,), 1.0, 0.1, 47, 2, dt)
+    g = synth.normal((rows, D), 0.0, 1.0, 47, 4, dt)
+    dx, dw, db = nv.layer_norm_vjp(dev(x), dev(w), dev(g), eps=1e-5)
+    torch.cuda.synchronize()
+    ref = oracle.layer_norm_vjp(host(x), host(w), host(g), 1e-5)
+    check_grad(dx, ref[0], ref[3], "dx")
+    check_grad(dw, ref[1], ref[4], "dw")
+    check_grad(db, ref[2], ref[5], "db")
+
+
 @pytest.mark.parametrize("dt,D", [("bf16", 1024), ("bf16", 4096), ("bf16", 16384), ("f32", 512),
                                   ("f32", 4096), ("f32", 8192)])
 def test_layer_norm_vjp_rows_starting_far_from_their_mean(dt, D):
