@@ -6,9 +6,10 @@ Default workload (one step = one add_rms_norm call through the C ABI):
     eps = 1e-5; outputs y and h = x + r.
 Metric: achieved HBM GB/s of algorithmic bytes (4 N s + D s per call, s = 2) and rows/s,
 against B200's HBM peak.  Each step is timed with CUDA events on the launching stream.
-Steps rotate over device buffer sets that together exceed L2 several times and run back
-to back, so no step reads data a previous step left in L2 and every step pays the
-write-back of its predecessor's output (workloads smaller than L2 flush it instead).
+Steps rotate over device buffer sets and run back to back; between two uses of one set the
+other sets move at least 3x L2 through the cache, so no step reads data a previous step
+left in L2, and every step pays the write-back of its predecessor's output (workloads
+smaller than L2 flush it instead).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --sweep        # add_rms_norm over D x rows x dtype, one line per point
@@ -192,9 +193,13 @@ class Case:
     """Device-resident inputs/outputs of one workload and a callable that runs it once.
 
     Large workloads keep `nsets` copies of their device buffers and step i uses copy
-    i % nsets, so consecutive steps touch disjoint memory larger than L2 and run back to
-    back (each step then also pays the write-back of the previous step's dirty lines,
-    as in a steady stream).  Workloads too small for that are timed after an L2 flush.
+    i % nsets; the other nsets - 1 copies, which the steps in between touch, hold at least
+    3x L2, so no line a step reads survives in L2 from the last use of its copy (with 2
+    copies of the 268 MB norm_rope set, lines that an L2 bulk prefetch had brought in --
+    at normal eviction priority, unlike the streamed rows -- still made up ~5% of a
+    step's reads).  Steps run back to back (each then also pays the write-back of the
+    previous step's dirty lines, as in a steady stream).  Workloads too small for that
+    are timed after an L2 flush.
     """
 
     def __init__(self, op, shape, dtype, seed, **kw):
@@ -241,7 +246,7 @@ class Case:
         self.n_row_tensors = n_row_tensors
         set_bytes = n_row_tensors * self.rows * self.D * self.s
         if set_bytes >= l2:
-            self.nsets = max(2, min(8, -(-3 * l2 // set_bytes)))
+            self.nsets = max(2, min(9, 1 + -(-3 * l2 // set_bytes)))
         else:
             self.nsets = 1
         self.sets = []

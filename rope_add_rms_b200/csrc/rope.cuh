@@ -495,17 +495,6 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
             xv[u][1] = ld_stream(xbase + (size_t)b * lstride + (size_t)v1 * 16);
         }
     }
-    // The next kUnroll rows of each slot are asked of L2 now (one bulk prefetch per row, by
-    // the group's lane 0), so the first round after the table finds them on chip: a CTA's
-    // start costs one DRAM latency instead of two.  Measured on bf16 [8, 32, 2048, 128]:
-    // 47.7 us against 48.2 us without; asking for the whole chunk at once 54.0, two rounds
-    // ahead 49.5, and a rolling prefetch two rounds ahead of every row 50.7.
-    if (has_vec && lane == 0)
-#pragma unroll
-        for (int u = kUnroll; u < 2 * kUnroll; ++u) {
-            const int64_t b = bh0 + slot + (int64_t)u * slots;
-            if (b < bh_end) prefetch_l2(xbase + (size_t)b * lstride, (uint32_t)row_bytes);
-        }
     // the angle table is built while the first rows' loads are in flight
     float4* wtab = tab + 2 * hvec * NP;
     build_angle_records<T, TRAD>(a, tab, l, threadIdx.x, kRopeThreads);
