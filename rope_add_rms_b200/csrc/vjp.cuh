@@ -484,9 +484,12 @@ struct LayerVjpRow {
         const float dm = __fmul_rn(q[0], invD);                             // mean = m1 + dm
         const float var = fmaxf(__fmaf_rn(q[1], invD, -__fmul_rn(dm, dm)), 0.f);
         const float r = rsqrtf(__fadd_rn(var, a.eps));
-        // dx = r (a - mean(a) - c B) with B = r^2 sum(a c) / D
+        // dx = r (a - mean(a) - c B) with B = r^2 sum(a c) / D, evaluated as
+        // r a + (c (-r B) - r mean(a)): two packed fmas a pair, each rounding relative to one
+        // of the cancelling terms
         const float B = __fmul_rn(__fmul_rn(r, r), __fmul_rn(__fmaf_rn(-dm, p[1], q[2]), invD));
-        const float2 r2 = splat2(r), ndm = splat2(-dm), nB = splat2(-B), nma = splat2(-ma);
+        const float2 r2 = splat2(r), ndm = splat2(-dm), nrB = splat2(-__fmul_rn(r, B)),
+                     nrma = splat2(-__fmul_rn(r, ma));
         const size_t roff = (size_t)row * (size_t)a.nvec * 16;
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
@@ -504,7 +507,7 @@ struct LayerVjpRow {
                         a2 = mul2(E::get2(wv[k], e), g2);
                         c2 = add2(add2(E::get2(xv[k], e), nm1), ndm);
                     }
-                    E::put2(o, e, mul2(r2, fma2(c2, nB, add2(a2, nma))));
+                    E::put2(o, e, fma2(r2, a2, fma2(c2, nrB, nrma)));
                     float2& aw = acc.at(0, k * NP + e / 2);
                     float2& ab = acc.at(1, k * NP + e / 2);
                     aw = fma2(g2, mul2(c2, r2), aw);
