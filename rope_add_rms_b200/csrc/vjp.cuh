@@ -484,12 +484,15 @@ struct LayerVjpRow {
         const float dm = __fmul_rn(q[0], invD);                             // mean = m1 + dm
         const float var = fmaxf(__fmaf_rn(q[1], invD, -__fmul_rn(dm, dm)), 0.f);
         const float r = rsqrtf(__fadd_rn(var, a.eps));
-        // dx = r (a - mean(a) - c B) with B = r^2 sum(a c) / D, evaluated as
-        // r a + (c (-r B) - r mean(a)): two packed fmas a pair, each rounding relative to one
-        // of the cancelling terms
+        // dx = r (a - mean(a) - c B) with B = r^2 sum(a c) / D and c = c' - dm, evaluated as
+        // r a + (c' (-r B) + (r B dm - r mean(a))), and xhat = c r as c' r - dm r: each
+        // rounding relative to one of the terms, two packed fmas a pair for dx and one for
+        // xhat
         const float B = __fmul_rn(__fmul_rn(r, r), __fmul_rn(__fmaf_rn(-dm, p[1], q[2]), invD));
-        const float2 r2 = splat2(r), ndm = splat2(-dm), nrB = splat2(-__fmul_rn(r, B)),
-                     nrma = splat2(-__fmul_rn(r, ma));
+        const float rB = __fmul_rn(r, B);
+        const float2 r2 = splat2(r), nrB = splat2(-rB),
+                     k0 = splat2(__fmaf_rn(rB, dm, -__fmul_rn(r, ma))),
+                     ndmr = splat2(-__fmul_rn(dm, r));
         const size_t roff = (size_t)row * (size_t)a.nvec * 16;
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
@@ -499,18 +502,18 @@ struct LayerVjpRow {
 #pragma unroll
                 for (int e = 0; e < VEC; e += 2) {
                     const float2 g2 = E::get2(gv[k], e);
-                    float2 a2, c2;
+                    float2 a2, cp;  // cp = c' = x - m1
                     if constexpr (kPacked) {
                         a2 = bf16x2_mac(wv[k].u[e / 2], gv[k].u[e / 2], splat2(0.f));
-                        c2 = add2(bf16x2_mac(xv[k].u[e / 2], kBf16x2One, nm1), ndm);
+                        cp = bf16x2_mac(xv[k].u[e / 2], kBf16x2One, nm1);
                     } else {
                         a2 = mul2(E::get2(wv[k], e), g2);
-                        c2 = add2(add2(E::get2(xv[k], e), nm1), ndm);
+                        cp = add2(E::get2(xv[k], e), nm1);
                     }
-                    E::put2(o, e, fma2(r2, a2, fma2(c2, nrB, nrma)));
+                    E::put2(o, e, fma2(r2, a2, fma2(cp, nrB, k0)));
                     float2& aw = acc.at(0, k * NP + e / 2);
                     float2& ab = acc.at(1, k * NP + e / 2);
-                    aw = fma2(g2, mul2(c2, r2), aw);
+                    aw = fma2(g2, fma2(cp, r2, ndmr), aw);
                     ab = add2(ab, g2);
                 }
                 st_stream(static_cast<char*>(a.dx) + roff + (size_t)v * 16, o);
