@@ -292,9 +292,11 @@ __global__ void __launch_bounds__(256, TRAD ? 3 : 2) rope_rows_kernel(const Rope
 // The angle table and the lane's weights stay in shared memory as records of two pairs,
 // transposed so that the lanes of a row read consecutive records, and are read per row:
 // with neither in registers four CTAs fit per SM (three for float32), and a record load
-// yields the float pairs the packed rotation takes.  Halves, bf16 [8, 32, 2048, 128]:
-// 51.7 us; 54.3 us with the weights in registers (3 CTAs/SM), 59.2 us with one table
-// entry per pair, 69.5 us with the table in registers (2 CTAs/SM).
+// yields the float pairs the packed rotation takes.  Halves, bf16 [8, 32, 2048, 128], with
+// the lanes per row taken from the arguments: 51.7 us; 54.3 us with the weights in registers
+// (3 CTAs/SM), 59.2 us with one table entry per pair, 69.5 us with the table in registers
+// (2 CTAs/SM).  With the lanes per row fixed at compile time (rope_pairs_kernel's HV):
+// 48.1-48.3 us.
 template <typename T, bool TRAD>
 struct PairLayout {
     using E = Elem<T>;
