@@ -189,6 +189,15 @@ def algorithmic_bytes(op, rows, D, s, nparts=0):
     raise ValueError(op)
 
 
+def rotation_sets(set_bytes, l2_bytes):
+    """Copies of a workload's buffers to rotate over: enough that the other copies, which
+    the steps between two uses of one copy touch, hold at least 3x L2 (at least 2 copies,
+    at most 9); 1 (and an L2 flush before each step) when one copy is smaller than L2."""
+    if set_bytes < l2_bytes:
+        return 1
+    return max(2, min(9, 1 + -(-3 * l2_bytes // set_bytes)))
+
+
 class Case:
     """Device-resident inputs/outputs of one workload and a callable that runs it once.
 
@@ -244,11 +253,7 @@ class Case:
         if op == "allreduce_add_rms_norm":
             n_row_tensors = self.nparts + 3
         self.n_row_tensors = n_row_tensors
-        set_bytes = n_row_tensors * self.rows * self.D * self.s
-        if set_bytes >= l2:
-            self.nsets = max(2, min(9, 1 + -(-3 * l2 // set_bytes)))
-        else:
-            self.nsets = 1
+        self.nsets = rotation_sets(n_row_tensors * self.rows * self.D * self.s, l2)
         self.sets = []
         for _ in range(self.nsets):
             d = {k: (v.clone() if on_dev else v.cuda()) if v is not None else None

@@ -68,3 +68,21 @@ def test_nvtx_ranges_nest_and_never_raise():
             raise KeyError("body")
     except KeyError:
         pass   # the body's exception propagates; the range is closed on the way out
+
+
+def test_rotation_keeps_three_l2_between_uses_of_a_buffer_set():
+    """Between two uses of one buffer set the other sets hold at least 3x L2, so no line a
+    step reads can have survived in L2 from that set's last use."""
+    l2 = 126 * 2 ** 20
+    for set_bytes, want in [(268435456, 3),      # add_rms_norm / norm_rope bf16 sets
+                            (536870912, 2),      # layer_norm bf16 [16384, 8192]
+                            (201326592, 3),      # rms_norm_vjp
+                            (134217728, 4),      # rms_norm bf16 [8192, 4096]
+                            (l2, 4), (l2 - 1, 1), (10 * l2, 2), (l2 // 2 + 2 ** 20, 1)]:
+        n = bench.rotation_sets(set_bytes, l2)
+        assert n == want, (set_bytes, n, want)
+        if n > 1:
+            assert (n - 1) * set_bytes >= 3 * l2 or n == 9
+    assert bench.rotation_sets(l2 + 1, l2) == 4     # just over L2: 3 more copies
+    assert bench.rotation_sets(l2 // 4 + l2, l2) == 4
+
