@@ -627,6 +627,52 @@ def test_peer_allreduce_one_rank_and_a_flag_that_never_comes():
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("world", [2, 4])
+def test_peer_allreduce_emulated_ranks_on_one_gpu(world):
+    """The one-shot form with `world` ranks emulated in one process on one GPU: each rank's
+    buffer (two partial slots, then its flag array) is local memory, so every part pointer is
+    an ordinary device address.  Per step, every rank publishes the step's epoch into every
+    rank's flag array first, and only then does each rank's reduce run, so every flag it
+    checks is already set and no kernel waits on another.  The slot of the other parity
+    holds NaNs: a reduce that read it would show.  All ranks get the oracle's y and h
+    bit-identically."""
+    rows, D = 257, 4096
+    esz = 2
+    slot = rows * D * esz
+    flags_off = (2 * slot + 255) // 256 * 256
+    raws = [torch.zeros(flags_off + 8 * world, dtype=torch.uint8, device="cuda")
+            for _ in range(world)]
+    bufs = [r[:2 * slot].view(torch.bfloat16).view(2, rows, D) for r in raws]
+    flags = [r[flags_off:].view(torch.int64) for r in raws]
+    flag_ptrs = [f.data_ptr() for f in flags]
+    nv.nv_fault_count(reset=True)
+    for epoch in (1, 2, 3):
+        inp = synth.allreduce_inputs(rows, D, world, "bf16", seed=40 + epoch)
+        for k in range(world):
+            bufs[k][epoch & 1].copy_(dev(inp["parts"][k]))
+            bufs[k][(epoch + 1) & 1].fill_(float("nan"))
+        for k in range(world):
+            nv.nv_tp_publish(flag_ptrs, k, epoch)
+        parts = [bufs[k][epoch & 1].data_ptr() for k in range(world)]
+        r, w = dev(inp["r"]), dev(inp["w"])
+        outs = []
+        for k in range(world):
+            y, h = torch.empty_like(r), torch.empty_like(r)
+            nv.nv_allreduce_add_rms_norm_peers(parts, r, w, y, h, 1e-5, flags[k], epoch)
+            outs.append((y, h))
+        torch.cuda.synchronize()
+        for k in range(world):
+            assert (flags[k].cpu() == epoch).all(), f"rank {k}'s flags after epoch {epoch}"
+        y_ref, h_ref, _ = oracle.allreduce_add_rms_norm([host(p) for p in inp["parts"]],
+                                                        host(inp["r"]), host(inp["w"]), 1e-5)
+        check_exact(outs[0][1], h_ref, f"h, epoch {epoch}")
+        check_out(outs[0][0], y_ref, f"y, epoch {epoch}")
+        for k in range(1, world):
+            assert torch.equal(outs[k][0].view(torch.int16), outs[0][0].view(torch.int16))
+            assert torch.equal(outs[k][1].view(torch.int16), outs[0][1].view(torch.int16))
+    assert nv.nv_fault_count() == 0
+
+
 def test_allreduce_in_place_ranks_agree_and_errors():
     rows, D, n = 300, 4096, 4
     inp = synth.allreduce_inputs(rows, D, n, "bf16", seed=77)
