@@ -428,7 +428,11 @@ NV_API nv_status nv_selftest_bounded_wait(int32_t ctas, nv_stream_t stream);
  *                   at most 32; a multiple of rows_per_cta, at least 2 x rows_per_cta).
  *                   NV_PATH_SLOTS: 1 = each row slot asks L2 for its next row while it
  *                   works on the current one (one bulk prefetch a row); -1 = no prefetch;
- *                   0 = prefetch when a row spans several warps.  Other paths: must be 0.
+ *                   0 = prefetch when a row spans several warps.  norm_rope register path
+ *                   with two vectors per lane of 4, 8 or 16 lanes: 2..6 = that many rounds
+ *                   of rows in flight per lane group, staged by per-thread asynchronous
+ *                   copies into shared memory; -1 = rows in flight in registers; 0 = 2
+ *                   rounds for bfloat16, registers otherwise.  Other paths: must be 0.
  * For NV_PATH_RING, threads_per_row is the size of a row group (32 x warps, <= 256),
  * rows_per_cta the row groups of a CTA (rows reduced at once), ctas_per_sm the CTAs per
  * SM (0 = 1), vec_per_thread must be 0.

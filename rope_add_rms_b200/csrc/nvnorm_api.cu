@@ -671,13 +671,39 @@ nv_status row_dispatch(Op op, const nv_plan& p, const DevInfo& di, nv_dtype dt, 
 struct RopePlan {
     bool rows;
     bool pairs;  // two vectors per lane: rope_pairs_kernel (dims == D)
+    int depth;   // > 0: rope_pairs_async_kernel with this many rounds in flight
     int lpr;
     int bt;
     int64_t n_chunks;
 };
 
+template <typename T, bool TRAD, int HV>
+nv_status launch_rope_async(cudaStream_t s, const RopeArgs& a, int depth) {
+    const size_t smem = (size_t)a.half * sizeof(float4) +
+                        (size_t)Elem<T>::kVec / 2 * (size_t)HV * sizeof(float4) +
+                        rope_async_ring_bytes(depth);
+    auto kern = depth == 4   ? rope_pairs_async_kernel<T, TRAD, HV, 4>
+                : depth == 6 ? rope_pairs_async_kernel<T, TRAD, HV, 6>
+                : depth == 2 ? rope_pairs_async_kernel<T, TRAD, HV, 2>
+                : depth == 5 ? rope_pairs_async_kernel<T, TRAD, HV, 5>
+                             : rope_pairs_async_kernel<T, TRAD, HV, 3>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    }
+    return launch_kernel(kern, a.L * a.n_chunks, kRopeThreads, smem, s, a);
+}
+
 template <typename T, bool TRAD>
-nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a, bool pairs) {
+nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a, bool pairs,
+                           int depth) {
+    if (depth > 0) {
+        const int hv = a.nvec / 2;
+        return hv == 8    ? launch_rope_async<T, TRAD, 8>(s, a, depth)
+               : hv == 16 ? launch_rope_async<T, TRAD, 16>(s, a, depth)
+                          : launch_rope_async<T, TRAD, 4>(s, a, depth);
+    }
     // the pairs kernel keeps its lanes' weights after the table: VEC/2 records per lane
     const size_t smem = (size_t)a.half * sizeof(float4) +
                         (pairs ? (size_t)Elem<T>::kVec / 2 * (size_t)(a.nvec / 2) * sizeof(float4)
@@ -721,7 +747,18 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
     if (p.path == NV_PATH_AUTO) p.path = (vec_ok || pairs_ok) ? NV_PATH_ROWS : NV_PATH_GENERIC;
     rp->rows = p.path == NV_PATH_ROWS;
     rp->pairs = rp->rows && pairs_ok && p.vec_per_thread != 1;
-    if (p.stages != 0) return fail(NV_ERR_UNSUPPORTED, "norm_rope takes no stages");
+    // stages: rounds of rows in flight per lane group through the shared-memory ring of
+    // rope_pairs_async_kernel (2..6; two vectors per lane of 4, 8 or 16 lanes), -1: the
+    // register kernel, 0: automatic -- 2 rounds for bfloat16 where the ring kernel exists
+    // (measured on bf16 [8, 32, 2048, 128]: 45.6 us against 48.3 for the register kernel;
+    // 3 rounds 46.0, 4 rounds 46.2; float32 rows gain nothing and keep the register kernel)
+    const int hv = (int)(nvec / 2);
+    const bool ring_ok = rp->pairs && (hv == 4 || hv == 8 || hv == 16);
+    if (p.stages != 0 && p.stages != -1 &&
+        (!(p.stages >= 2 && p.stages <= 6) || !ring_ok || p.vec_per_thread == 1))
+        return fail(NV_ERR_UNSUPPORTED, "norm_rope stages = %d: 2 to 6 rounds of the "
+                    "two-vectors-per-lane kernel at 4, 8 or 16 lanes per row, or -1", p.stages);
+    rp->depth = p.stages > 0 ? p.stages : (p.stages == 0 && ring_ok && dt == NV_BF16 ? 2 : 0);
     if (p.path == NV_PATH_ROWS) {
         if (!vec_ok && !rp->pairs)
             return fail(NV_ERR_UNSUPPORTED, "norm_rope register path needs D %% %d == 0, "
@@ -745,6 +782,7 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
         p.vec_per_thread = rp->pairs ? 2 : 1;
         p.threads_per_row = lpr;
         p.rows_per_cta = (int)bt;
+        p.stages = rp->depth > 0 ? rp->depth : -1;
     } else if (p.path == NV_PATH_GENERIC) {
         p.vec_per_thread = 0;
         p.threads_per_row = 128;
@@ -836,10 +874,10 @@ nv_status rope_op(const void* x, const void* w, const float* freqs, void* y, int
     const bool bf = dt == NV_BF16;
     if (rp.rows) {
         if (traditional)
-            return bf ? launch_rope_rows<__nv_bfloat16, true>(di, cs, a, rp.pairs)
-                      : launch_rope_rows<float, true>(di, cs, a, rp.pairs);
-        return bf ? launch_rope_rows<__nv_bfloat16, false>(di, cs, a, rp.pairs)
-                  : launch_rope_rows<float, false>(di, cs, a, rp.pairs);
+            return bf ? launch_rope_rows<__nv_bfloat16, true>(di, cs, a, rp.pairs, rp.depth)
+                      : launch_rope_rows<float, true>(di, cs, a, rp.pairs, rp.depth);
+        return bf ? launch_rope_rows<__nv_bfloat16, false>(di, cs, a, rp.pairs, rp.depth)
+                  : launch_rope_rows<float, false>(di, cs, a, rp.pairs, rp.depth);
     }
     return bf ? launch_rope_generic<__nv_bfloat16>(di, p.ctas_per_sm, cs, a)
               : launch_rope_generic<float>(di, p.ctas_per_sm, cs, a);

@@ -524,6 +524,92 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
     }
 }
 
+// The same rows with DEPTH rounds of loads in flight per lane group, staged by per-thread
+// asynchronous copies (cp.async, 16 bytes, L2 only) into a ring of shared memory instead of
+// registers, so rows in flight cost shared memory (DEPTH x 8 KB a CTA) rather than the
+// registers that hold four CTAs per SM.  Each thread copies, waits for and reads back only
+// its own two vectors of a round (slot [round % DEPTH][vector][thread]: consecutive
+// threads, consecutive 16 bytes), so no barrier is needed: cp.async.wait_group orders a
+// thread's own copies, one commit group per round (empty past the chunk's last row).  A
+// slot is refilled only after the row read from it has been computed.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    const uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// shared memory of rope_pairs_async_kernel: the table and weight records, then the ring
+__host__ __device__ constexpr size_t rope_async_ring_bytes(int depth) {
+    return (size_t)depth * 2 * kRopeThreads * 16;
+}
+
+template <typename T, bool TRAD, int HV, int DEPTH>
+__global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
+    rope_pairs_async_kernel(const RopeArgs a) {
+    static_assert(HV > 0, "lanes per row fixed at compile time");
+    constexpr int NP = PairLayout<T, TRAD>::NP;
+    constexpr int kSlots = kRopeThreads / HV;
+    // records: C [HV NP], S [HV NP], the lanes' weights W [NP][HV], then the ring
+    extern __shared__ float4 tab[];
+    float4* wtab = tab + 2 * HV * NP;
+    V16* ring = reinterpret_cast<V16*>(wtab + NP * HV);
+
+    const int64_t chunk = blockIdx.x % a.n_chunks;
+    const int64_t l = blockIdx.x / a.n_chunks;
+    const int lane = threadIdx.x & (HV - 1);
+    const int slot = threadIdx.x / HV;
+    const int v0 = lane, v1 = lane + HV;
+
+    pdl_wait();
+    pdl_release();
+
+    const int64_t bh0 = chunk * (int64_t)a.bt;
+    const int64_t bh_end = min(bh0 + (int64_t)a.bt, a.BH);
+    const size_t row_bytes = (size_t)a.D * sizeof(T);
+    const size_t lstride = (size_t)a.L * row_bytes;
+    const char* xbase = static_cast<const char*>(a.x) + (size_t)l * row_bytes;
+    const size_t ystride = (size_t)a.y_len * row_bytes;
+    char* ybase = static_cast<char*>(a.y) + (size_t)(a.y_off + l) * row_bytes;
+    const int rounds = (a.bt + kSlots - 1) / kSlots;
+
+    auto issue = [&](int r) {
+        const int64_t b = bh0 + slot + (int64_t)r * kSlots;
+        if (r < rounds && b < bh_end) {
+            const char* src = xbase + (size_t)b * lstride;
+            V16* dst = ring + (size_t)(r % DEPTH) * 2 * kRopeThreads + threadIdx.x;
+            cp_async16(dst, src + (size_t)v0 * 16);
+            cp_async16(dst + kRopeThreads, src + (size_t)v1 * 16);
+        }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int r = 0; r < DEPTH; ++r) issue(r);
+    // the angle table is built while the first rounds load
+    build_angle_records<T, TRAD>(a, tab, l, threadIdx.x, kRopeThreads);
+    store_weight_records<T, TRAD>(a, wtab, v0, v1, true, slot == 0);
+    __syncthreads();
+
+    const float invD = 1.0f / (float)a.D;
+    for (int r = 0; r < rounds; ++r) {
+        cp_async_wait<DEPTH - 1>();  // this thread's copies of round r have landed
+        const V16* src = ring + (size_t)(r % DEPTH) * 2 * kRopeThreads + threadIdx.x;
+        const V16 xa = src[0];
+        const V16 xb = src[kRopeThreads];
+        const int64_t b = bh0 + slot + (int64_t)r * kSlots;
+        // a row past the chunk is reduced from stale shared memory and not stored
+        rope_pairs_row<T, TRAD>(a, tab, wtab, xa, xb, b < bh_end, v0, v1, HV, HV, invD,
+                                ybase + (size_t)b * ystride);
+        issue(r + DEPTH);
+    }
+    cp_async_wait<0>();
+}
+
 // ---- generic path ---------------------------------------------------------------------
 // Any D, dims and alignment: one CTA per row.  Pass 1: sum of squares.  Pass 2: each
 // thread takes whole pairs (reads both members, then writes both, so y may be x) with

@@ -498,7 +498,9 @@ def test_norm_rope_every_variant(D, dt):
     inp = synth.norm_rope_inputs(2, 4, 64, D, dt, seed=1)
     x, w = dev(inp["x"]), dev(inp["w"])
     plans = [dict(path=nv.PATH_GENERIC), dict(path=nv.PATH_ROWS, vec_per_thread=1),
-             dict(path=nv.PATH_ROWS, vec_per_thread=2), dict(path=nv.PATH_ROWS, rows_per_cta=3)]
+             dict(path=nv.PATH_ROWS, vec_per_thread=2), dict(path=nv.PATH_ROWS, rows_per_cta=3),
+             dict(path=nv.PATH_ROWS, stages=6), dict(path=nv.PATH_ROWS, stages=4, rows_per_cta=40),
+             dict(path=nv.PATH_ROWS, stages=-1), dict(path=nv.PATH_ROWS, stages=2)]
     for trad in (0, 1):
         ref = oracle.norm_rope(host(inp["x"]), host(inp["w"]), 64, D, trad, 10000.0, 1.0, 4096,
                                1, 1e-6)
@@ -540,12 +542,54 @@ def test_norm_rope_near_cancellation(trad, dt):
     xt = torch.from_numpy(x.reshape(-1, D)).to(tdt)
     w = torch.ones(D, dtype=tdt)
     ref = oracle.norm_rope(host(xt), host(w), L, D, trad, 10000.0, 1.0, offset, 1, 1e-6)
-    for p in (None, dict(path=nv.PATH_ROWS, vec_per_thread=1), dict(path=nv.PATH_GENERIC)):
+    for p in (None, dict(path=nv.PATH_ROWS, vec_per_thread=1), dict(path=nv.PATH_GENERIC),
+              dict(path=nv.PATH_ROWS, stages=3), dict(path=nv.PATH_ROWS, stages=-1)):
         y = torch.empty_like(xt).cuda()
         nv.nv_norm_rope(xt.cuda(), w.cuda(), y, L, D, trad, 10000.0, 1.0, offset, 1, 1e-6,
                         plan=None if p is None else nv.Plan(**p))
         torch.cuda.synchronize()
         check_out(y, ref, f"near cancellation {p}")
+
+
+@pytest.mark.parametrize("stages", [2, 3, 4, 6])
+@pytest.mark.parametrize("case", [(3, 100, 9, 128, "bf16", 0), (3, 100, 9, 128, "bf16", 70),
+                                  (2, 5, 30, 64, "bf16", 0), (2, 9, 20, 256, "bf16", 0),
+                                  (3, 100, 9, 128, "f32", 0), (1, 600, 2, 128, "bf16", 96)],
+                         ids=lambda c: "x".join(map(str, c)))
+def test_norm_rope_async_rounds(case, stages):
+    """Rows staged through the per-thread asynchronous-copy ring (stages = rounds in flight),
+    ragged chunks (BH = 300 or 600 in chunks of 70 or 96) included, both pairings, in place
+    too."""
+    B, H, L, D, dt, bt = case
+    inp = synth.norm_rope_inputs(B, H, L, D, dt, seed=L + D + stages)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    for trad in (0, 1):
+        ref = oracle.norm_rope(host(inp["x"]), host(inp["w"]), L, D, trad, 10000.0, 1.0, 2047, 1,
+                               1e-6)
+        plan = nv.Plan(path=nv.PATH_ROWS, stages=stages, rows_per_cta=bt)
+        g = Guarded(x.shape, x.dtype)
+        nv.nv_norm_rope(x, w, g.t, L, D, trad, 10000.0, 1.0, 2047, 1, 1e-6, plan=plan)
+        torch.cuda.synchronize()
+        assert g.bands_intact()
+        check_out(g.t, ref, f"async rounds {case} stages={stages} trad={trad}")
+        xi = x.clone()
+        nv.nv_norm_rope(xi, w, xi, L, D, trad, 10000.0, 1.0, 2047, 1, 1e-6, plan=plan)
+        torch.cuda.synchronize()
+        check_out(xi, ref, f"async rounds in place {case} stages={stages} trad={trad}")
+
+
+def test_norm_rope_async_rounds_rejects():
+    x = torch.zeros(2 * 4 * 16, 128, dtype=torch.bfloat16, device="cuda")
+    w = torch.ones(128, dtype=torch.bfloat16, device="cuda")
+    for p, dims in ((dict(path=nv.PATH_ROWS, stages=7), 128),
+                    (dict(path=nv.PATH_ROWS, stages=1), 128),
+                    (dict(path=nv.PATH_ROWS, stages=-2), 128),
+                    (dict(path=nv.PATH_ROWS, stages=4, vec_per_thread=1), 128),
+                    (dict(path=nv.PATH_ROWS, stages=4), 64),
+                    (dict(path=nv.PATH_GENERIC, stages=4), 128)):
+        with pytest.raises(nv.NvError) as e:
+            nv.nv_norm_rope(x, w, x, 16, dims, 0, 10000.0, 1.0, 0, 1, 1e-6, plan=nv.Plan(**p))
+        assert e.value.status == nv.NV_ERR_UNSUPPORTED, p
 
 
 def test_norm_rope_in_place():
@@ -866,7 +910,9 @@ def test_dependent_chain_across_ops_in_place():
 # ---- general rope: cache form, explicit frequencies, inverse ----------------------------------
 
 ROPE_PLANS = [None, dict(path=nv.PATH_GENERIC), dict(path=nv.PATH_ROWS, vec_per_thread=1),
-              dict(path=nv.PATH_ROWS, vec_per_thread=2)]
+              dict(path=nv.PATH_ROWS, vec_per_thread=2),
+              dict(path=nv.PATH_ROWS, vec_per_thread=2, stages=4),
+              dict(path=nv.PATH_ROWS, vec_per_thread=2, stages=-1)]
 
 
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
