@@ -19,6 +19,7 @@
 //     error, harmless).
 #pragma once
 
+#include "async_copy.cuh"
 #include "common.cuh"
 
 namespace nvn {
@@ -532,18 +533,6 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
 // threads, consecutive 16 bytes), so no barrier is needed: cp.async.wait_group orders a
 // thread's own copies, one commit group per round (empty past the chunk's last row).  A
 // slot is refilled only after the row read from it has been computed.
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-    const uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // shared memory of rope_pairs_async_kernel: the table and weight records, then the ring
 __host__ __device__ constexpr size_t rope_async_ring_bytes(int depth) {
     return (size_t)depth * 2 * kRopeThreads * 16;
