@@ -624,6 +624,11 @@ WORKLOADS = {
     "norm_rope_traditional": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,
                                           dims=128, traditional=1, base=10000.0, scale=1.0,
                                           offset=4096),
+    # partial rotary: only the first 64 of the 128 features rotate (halves (i, i + 32)), the
+    # rest are normalised and weighted only
+    "norm_rope_partial": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,
+                                      dims=64, traditional=0, base=10000.0, scale=1.0,
+                                      offset=0),
     # NormRope's cache form: the 2048 new positions of every (b, h) written into a KV cache
     # of 8192 positions at offset 4096
     "norm_rope_cache": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,

@@ -412,7 +412,8 @@ NV_API nv_status nv_selftest_bounded_wait(int32_t ctas, nv_stream_t stream);
  *   vec_per_thread  16-byte vectors per thread and row (register paths; 0 = auto; for
  *                   norm_rope 1 = one vector per lane, 2 = two vectors per lane (both
  *                   halves of a rotation, or two vectors of interleaved pairs), which
- *                   needs dims == D)
+ *                   needs dims == D, or with dims < D rotated features that fill an even
+ *                   number of whole 16-byte vectors and 4, 8 or 16 lanes per row)
  *   threads_per_row threads that share one row (multiple of 32, <= 1024; 0 = auto)
  *   rows_per_cta    rows one CTA works on at a time (0 = auto)
  *   ctas_per_sm     0: one CTA per row group (rms_norm register path, generic paths),
@@ -431,8 +432,10 @@ NV_API nv_status nv_selftest_bounded_wait(int32_t ctas, nv_stream_t stream);
  *                   0 = prefetch when a row spans several warps.  norm_rope register path
  *                   with two vectors per lane of 4, 8 or 16 lanes: 2..6 = that many rounds
  *                   of rows in flight per lane group, staged by per-thread asynchronous
- *                   copies into shared memory; -1 = rows in flight in registers; 0 = 2
- *                   rounds for bfloat16, registers otherwise.  Other paths: must be 0.
+ *                   copies into shared memory; -1 = rows in flight in registers; 0 =
+ *                   automatic: with dims == D 2 rounds for bfloat16, registers for
+ *                   float32; with dims < D 3 rounds for bfloat16, 4 for float32.
+ *                   Other paths: must be 0.
  * For NV_PATH_RING, threads_per_row is the size of a row group (32 x warps, <= 256),
  * rows_per_cta the row groups of a CTA (rows reduced at once), ctas_per_sm the CTAs per
  * SM (0 = 1), vec_per_thread must be 0.

@@ -670,23 +670,23 @@ nv_status row_dispatch(Op op, const nv_plan& p, const DevInfo& di, nv_dtype dt, 
 // ---- norm_rope -------------------------------------------------------------------------------
 struct RopePlan {
     bool rows;
-    bool pairs;  // two vectors per lane: rope_pairs_kernel (dims == D)
+    bool pairs;  // two vectors per lane: rope_pairs_kernel
     int depth;   // > 0: rope_pairs_async_kernel with this many rounds in flight
     int lpr;
     int bt;
     int64_t n_chunks;
 };
 
-template <typename T, bool TRAD, int HV>
+template <typename T, bool TRAD, int HV, bool PART>
 nv_status launch_rope_async(cudaStream_t s, const RopeArgs& a, int depth) {
     const size_t smem = (size_t)a.half * sizeof(float4) +
                         (size_t)Elem<T>::kVec / 2 * (size_t)HV * sizeof(float4) +
                         rope_async_ring_bytes(depth);
-    auto kern = depth == 4   ? rope_pairs_async_kernel<T, TRAD, HV, 4>
-                : depth == 6 ? rope_pairs_async_kernel<T, TRAD, HV, 6>
-                : depth == 2 ? rope_pairs_async_kernel<T, TRAD, HV, 2>
-                : depth == 5 ? rope_pairs_async_kernel<T, TRAD, HV, 5>
-                             : rope_pairs_async_kernel<T, TRAD, HV, 3>;
+    auto kern = depth == 4   ? rope_pairs_async_kernel<T, TRAD, HV, 4, PART>
+                : depth == 6 ? rope_pairs_async_kernel<T, TRAD, HV, 6, PART>
+                : depth == 2 ? rope_pairs_async_kernel<T, TRAD, HV, 2, PART>
+                : depth == 5 ? rope_pairs_async_kernel<T, TRAD, HV, 5, PART>
+                             : rope_pairs_async_kernel<T, TRAD, HV, 3, PART>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -698,11 +698,17 @@ nv_status launch_rope_async(cudaStream_t s, const RopeArgs& a, int depth) {
 template <typename T, bool TRAD>
 nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a, bool pairs,
                            int depth) {
+    // dims < D (the plan only takes the pairs kernels there at 4, 8 or 16 lanes per row)
+    const bool part = a.dims < a.D;
     if (depth > 0) {
         const int hv = a.nvec / 2;
-        return hv == 8    ? launch_rope_async<T, TRAD, 8>(s, a, depth)
-               : hv == 16 ? launch_rope_async<T, TRAD, 16>(s, a, depth)
-                          : launch_rope_async<T, TRAD, 4>(s, a, depth);
+        if (part)
+            return hv == 8    ? launch_rope_async<T, TRAD, 8, true>(s, a, depth)
+                   : hv == 16 ? launch_rope_async<T, TRAD, 16, true>(s, a, depth)
+                              : launch_rope_async<T, TRAD, 4, true>(s, a, depth);
+        return hv == 8    ? launch_rope_async<T, TRAD, 8, false>(s, a, depth)
+               : hv == 16 ? launch_rope_async<T, TRAD, 16, false>(s, a, depth)
+                          : launch_rope_async<T, TRAD, 4, false>(s, a, depth);
     }
     // the pairs kernel keeps its lanes' weights after the table: VEC/2 records per lane
     const size_t smem = (size_t)a.half * sizeof(float4) +
@@ -710,11 +716,14 @@ nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a,
                                : 0);
     // the pairs kernel with lanes per row fixed at compile time where hvec is 4, 8 or 16
     const int hv = pairs && a.lpr == a.nvec / 2 ? a.nvec / 2 : 0;
-    auto kern = !pairs   ? rope_rows_kernel<T, TRAD>
-                : hv == 8  ? rope_pairs_kernel<T, TRAD, 8>
-                : hv == 16 ? rope_pairs_kernel<T, TRAD, 16>
-                : hv == 4  ? rope_pairs_kernel<T, TRAD, 4>
-                           : rope_pairs_kernel<T, TRAD, 0>;
+    auto kern = !pairs           ? rope_rows_kernel<T, TRAD>
+                : part && hv == 8  ? rope_pairs_kernel<T, TRAD, 8, true>
+                : part && hv == 16 ? rope_pairs_kernel<T, TRAD, 16, true>
+                : part             ? rope_pairs_kernel<T, TRAD, 4, true>
+                : hv == 8          ? rope_pairs_kernel<T, TRAD, 8>
+                : hv == 16         ? rope_pairs_kernel<T, TRAD, 16>
+                : hv == 4          ? rope_pairs_kernel<T, TRAD, 4>
+                                   : rope_pairs_kernel<T, TRAD, 0>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -741,24 +750,34 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
     const bool vec_ok = aligned && D % vecw == 0 && nvec <= 32 &&
                         (trad || (dims / 2) % vecw == 0);
     // two vectors per lane (both halves of the rotation, or two vectors of interleaved
-    // pairs): every feature rotated, an even number of vectors
-    const bool pairs_ok = aligned && D % vecw == 0 && dims == D && nvec % 2 == 0 &&
-                          nvec / 2 <= 32;
+    // pairs), an even number of vectors; with dims < D the rotated features fill an even
+    // number of whole vectors (halves: dims / 2 of them on each side) and the lanes per row
+    // are 4, 8 or 16 (the kernels with the lanes fixed at compile time)
+    const int64_t hv_all = nvec / 2;
+    const bool part_ok = (trad ? dims % (2 * vecw) == 0 : (dims / 2) % vecw == 0) &&
+                         (hv_all == 4 || hv_all == 8 || hv_all == 16);
+    const bool pairs_ok = aligned && D % vecw == 0 && nvec % 2 == 0 && nvec / 2 <= 32 &&
+                          (dims == D || part_ok);
     if (p.path == NV_PATH_AUTO) p.path = (vec_ok || pairs_ok) ? NV_PATH_ROWS : NV_PATH_GENERIC;
     rp->rows = p.path == NV_PATH_ROWS;
     rp->pairs = rp->rows && pairs_ok && p.vec_per_thread != 1;
     // stages: rounds of rows in flight per lane group through the shared-memory ring of
     // rope_pairs_async_kernel (2..6; two vectors per lane of 4, 8 or 16 lanes), -1: the
-    // register kernel, 0: automatic -- 2 rounds for bfloat16 where the ring kernel exists
-    // (measured on bf16 [8, 32, 2048, 128]: 45.6 us against 48.3 for the register kernel;
-    // 3 rounds 46.0, 4 rounds 46.2; float32 rows gain nothing and keep the register kernel)
+    // register kernel, 0: automatic.  Measured on [8, 32, 2048, 128]:
+    //   dims == D, bfloat16: 2 rounds, 45.4-45.7 us (register kernel 48.2, 3 rounds 45.8);
+    //   dims == D, float32:  the register kernel, 86.8 us (the ring 87.0-87.5);
+    //   dims < D,  bfloat16: 3 rounds, 45.9 / 51.6 / 48.7 us at dims 32 / 64 / 96 (2 rounds
+    //                        46.9 / 52.2 / 49.6, register kernel 57-69);
+    //   dims < D,  float32:  4 rounds, 87.6-88.6 us (register kernel 104-107).
     const int hv = (int)(nvec / 2);
     const bool ring_ok = rp->pairs && (hv == 4 || hv == 8 || hv == 16);
     if (p.stages != 0 && p.stages != -1 &&
         (!(p.stages >= 2 && p.stages <= 6) || !ring_ok || p.vec_per_thread == 1))
         return fail(NV_ERR_UNSUPPORTED, "norm_rope stages = %d: 2 to 6 rounds of the "
                     "two-vectors-per-lane kernel at 4, 8 or 16 lanes per row, or -1", p.stages);
-    rp->depth = p.stages > 0 ? p.stages : (p.stages == 0 && ring_ok && dt == NV_BF16 ? 2 : 0);
+    const bool part = dims < D;
+    const int auto_depth = !ring_ok ? 0 : part ? (dt == NV_BF16 ? 3 : 4) : (dt == NV_BF16 ? 2 : 0);
+    rp->depth = p.stages > 0 ? p.stages : (p.stages == 0 ? auto_depth : 0);
     if (p.path == NV_PATH_ROWS) {
         if (!vec_ok && !rp->pairs)
             return fail(NV_ERR_UNSUPPORTED, "norm_rope register path needs D %% %d == 0, "

@@ -111,8 +111,9 @@ __device__ __forceinline__ float2 rotate_sub2(float2 a_o, float2 a_t, float2 c_h
 // lanes away (one shuffle per word).  Traditional pairs live inside one vector and need
 // fewer registers: three CTAs per SM (measured 7% faster than two on bf16
 // [8, 32, 2048, 128] with this kernel; the halves form loses at three, its spills cost
-// more).  When every feature is rotated, rope_pairs_kernel below serves both pairings;
-// this kernel takes dims < D and plans that ask for one vector per lane.
+// more).  rope_pairs_kernel below serves both pairings where the rotated features fill an
+// even number of whole vectors; this kernel takes the other shapes with dims < D and plans
+// that ask for one vector per lane.
 template <typename T, bool TRAD>
 __global__ void __launch_bounds__(256, TRAD ? 3 : 2) rope_rows_kernel(const RopeArgs a) {
     using E = Elem<T>;
@@ -282,11 +283,13 @@ __global__ void __launch_bounds__(256, TRAD ? 3 : 2) rope_rows_kernel(const Rope
     }
 }
 
-// ---- register path, two vectors per lane (every feature rotated: dims == D) ---------------
+// ---- register path, two vectors per lane ---------------------------------------------------
 // Each lane holds vectors v and v + nvec/2 of a row (16-byte vectors, nvec even) and keeps
 // its elements as float pairs of rotation partners: p[k] holds the first members (the
 // cos-side inputs of y_p = a_p cos - a_q sin) of two pairs and q[k] their second members,
-// so one packed rotation serves two pairs and no partner is in another lane.
+// so one packed rotation serves two pairs and no partner is in another lane.  With dims < D
+// (pair_lane_vectors) the rotated lanes pair vectors v and v + dims/(2 VEC) instead and the
+// other lanes hold the features past dims.
 //   halves:      vector v holds the p members of pairs v*VEC .. v*VEC + VEC - 1 and
 //                vector v + nvec/2 their q members;
 //   traditional: each vector holds VEC/2 whole pairs (2i, 2i + 1).
@@ -372,10 +375,10 @@ __device__ __forceinline__ void build_angle_records(const RopeArgs& a, float4* c
     const double pos = (double)(a.offset + l);
     float* tabf = reinterpret_cast<float*>(ctab);
     const int nrec = a.half / 2;
-    const int hvec = a.nvec / 2;
+    const int hr = a.half / PL::VEC;  // lanes of a row that rotate (all of them when dims == D)
     for (int i = t; i < a.half; i += n) {
         int h = 0;
-        const int rec = PL::record_of(i, hvec, h);
+        const int rec = PL::record_of(i, hr, h);
         const float4 e = angle_entry(a, pos, i);
         tabf[rec * 4 + h] = e.x;               // C: cos_hi, cos_lo
         tabf[rec * 4 + 2 + h] = e.y;
@@ -384,11 +387,12 @@ __device__ __forceinline__ void build_angle_records(const RopeArgs& a, float4* c
     }
 }
 
-// The lanes' weight records W [NP][nvec / 2]; lanes with a vector (has_vec) read w and
-// those of slot 0 (write) store the records.
+// The lanes' weight records W [NP][lanes], record k * lanes + lane; lanes with a vector
+// (has_vec) read w at their vectors v0 and v1, and those of slot 0 (write) store the records.
 template <typename T, bool TRAD>
-__device__ __forceinline__ void store_weight_records(const RopeArgs& a, float4* wtab, int v0,
-                                                     int v1, bool has_vec, bool write) {
+__device__ __forceinline__ void store_weight_records(const RopeArgs& a, float4* wtab, int lane,
+                                                     int lanes, int v0, int v1, bool has_vec,
+                                                     bool write) {
     using PL = PairLayout<T, TRAD>;
     constexpr int NP = PL::NP;
     const bool has_w = a.normalize != 0 && a.w != nullptr && has_vec;
@@ -399,19 +403,22 @@ __device__ __forceinline__ void store_weight_records(const RopeArgs& a, float4* 
     if (write)
 #pragma unroll
         for (int k = 0; k < NP; ++k)
-            wtab[k * (a.nvec / 2) + v0] = make_float4(wp[k].x, wp[k].y, wq[k].x, wq[k].y);
+            wtab[k * lanes + lane] = make_float4(wp[k].x, wp[k].y, wq[k].x, wq[k].y);
 }
 
 // One row of the two-vectors-per-lane layout: sum of squares over the lane group, then the
 // rotation of this lane's pairs, weights applied first and the row's 1/rms last.  Every
 // lane of the group takes part (the group sum); lanes with live == false store nothing.
-// hvec = nvec / 2 vectors a lane group covers per side, lpr lanes per row; with dims == D
-// the table holds hvec * NP C records, then as many S records.
+// hvec = nvec / 2 vectors a lane group covers per side (the weight records' stride: record
+// k * hvec + lane), lpr lanes per row; hr of the lanes rotate (hr = hvec when dims == D) and
+// the table holds hr * NP C records, then as many S records; a lane with rot == false holds
+// two vectors past dims, which keep a = x w and take the row's 1/rms.
 template <typename T, bool TRAD>
 __device__ __forceinline__ void rope_pairs_row(const RopeArgs& a, const float4* ctab,
                                                const float4* wtab, const V16& xa, const V16& xb,
-                                               bool live, int v0, int v1, int hvec, int lpr,
-                                               float invD, char* yrow) {
+                                               bool live, int lane, int v0, int v1, int hvec,
+                                               int hr, bool rot, int lpr, float invD,
+                                               char* yrow) {
     using PL = PairLayout<T, TRAD>;
     constexpr int NP = PL::NP;
     float2 p[NP], q[NP];
@@ -427,17 +434,26 @@ __device__ __forceinline__ void rope_pairs_row(const RopeArgs& a, const float4* 
     const float2 inv2 = make_float2(inv, inv);
     if (live) {  // only lanes holding vectors read the table
         float2 yp[NP], yq[NP];
+        if (rot) {
 #pragma unroll
-        for (int k = 0; k < NP; ++k) {
-            const int rec = PL::record(v0, v1, k, hvec);
-            const float4 c4 = ctab[rec], s4 = ctab[hvec * NP + rec];
-            const float2 ch = make_float2(c4.x, c4.y), cl = make_float2(c4.z, c4.w);
-            const float2 sh = make_float2(s4.x, s4.y), sl = make_float2(s4.z, s4.w);
-            const float4 w4 = wtab[k * hvec + v0];
-            const float2 ap = mul2(p[k], make_float2(w4.x, w4.y));  // exact for bf16 data
-            const float2 aq = mul2(q[k], make_float2(w4.z, w4.w));
-            yp[k] = mul2(rotate_sub2(ap, aq, ch, cl, sh, sl), inv2);
-            yq[k] = mul2(rotate_pair2(aq, ap, ch, cl, sh, sl), inv2);
+            for (int k = 0; k < NP; ++k) {
+                const int rec = PL::record(v0, v1, k, hr);
+                const float4 c4 = ctab[rec], s4 = ctab[hr * NP + rec];
+                const float2 ch = make_float2(c4.x, c4.y), cl = make_float2(c4.z, c4.w);
+                const float2 sh = make_float2(s4.x, s4.y), sl = make_float2(s4.z, s4.w);
+                const float4 w4 = wtab[k * hvec + lane];
+                const float2 ap = mul2(p[k], make_float2(w4.x, w4.y));  // exact for bf16 data
+                const float2 aq = mul2(q[k], make_float2(w4.z, w4.w));
+                yp[k] = mul2(rotate_sub2(ap, aq, ch, cl, sh, sl), inv2);
+                yq[k] = mul2(rotate_pair2(aq, ap, ch, cl, sh, sl), inv2);
+            }
+        } else {  // past dims: a = x w, then the row's 1/rms
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+                const float4 w4 = wtab[k * hvec + lane];
+                yp[k] = mul2(mul2(p[k], make_float2(w4.x, w4.y)), inv2);
+                yq[k] = mul2(mul2(q[k], make_float2(w4.z, w4.w)), inv2);
+            }
         }
         V16 o0, o1;
         PL::join(yp, yq, o0, o1);
@@ -457,7 +473,27 @@ __host__ __device__ constexpr int rope_pairs_unroll() { return sizeof(T) == 4 ? 
 // the group sum a fixed butterfly; HV = 0 takes them from the arguments.
 constexpr int kRopeThreads = 256;
 
-template <typename T, bool TRAD, int HV>
+// PART (HV > 0 only): dims < D.  The first hr = dims / (2 VEC) lanes of a row hold the
+// rotated vectors as partner pairs (lane j: vectors j and j + hr), the others two of the
+// vectors past dims each (lane j: R + j - hr and that plus (nvec - R) / 2, R = dims / VEC).
+template <bool PART, int HV>
+__device__ __forceinline__ void pair_lane_vectors(const RopeArgs& a, int lane, int hvec, int vec,
+                                                  int& hr, int& v0, int& v1, bool& rot) {
+    if (!PART) {
+        hr = hvec;
+        v0 = lane;
+        v1 = lane + hvec;
+        rot = true;
+        return;
+    }
+    hr = a.half / vec;
+    rot = lane < hr;
+    const int R = 2 * hr;
+    v0 = rot ? lane : R + lane - hr;
+    v1 = rot ? lane + hr : v0 + (a.nvec - R) / 2;
+}
+
+template <typename T, bool TRAD, int HV, bool PART = false>
 __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
     rope_pairs_kernel(const RopeArgs a) {
     constexpr int kUnroll = rope_pairs_unroll<T>();
@@ -472,7 +508,10 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
     const int lane = threadIdx.x & (lpr - 1);
     const int slot = threadIdx.x / lpr;
     const int slots = kRopeThreads / lpr;
-    const int v0 = lane, v1 = lane + hvec;
+    static_assert(!PART || HV > 0, "dims < D takes the fixed-lane kernels");
+    int hr, v0, v1;
+    bool rot;
+    pair_lane_vectors<PART, HV>(a, lane, hvec, Elem<T>::kVec, hr, v0, v1, rot);
     // with HV fixed every lane of a group holds vectors (lpr == hvec)
     const bool has_vec = HV > 0 || lane < hvec;
 
@@ -498,10 +537,10 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
             xv[u][1] = ld_stream(xbase + (size_t)b * lstride + (size_t)v1 * 16);
         }
     }
-    // the angle table is built while the first rows' loads are in flight
-    float4* wtab = tab + 2 * hvec * NP;
+    // the angle table (half records) is built while the first rows' loads are in flight
+    float4* wtab = tab + 2 * hr * NP;
     build_angle_records<T, TRAD>(a, tab, l, threadIdx.x, kRopeThreads);
-    store_weight_records<T, TRAD>(a, wtab, v0, v1, has_vec, slot == 0 && has_vec);
+    store_weight_records<T, TRAD>(a, wtab, lane, hvec, v0, v1, has_vec, slot == 0 && has_vec);
     __syncthreads();
 
     const float invD = 1.0f / (float)a.D;
@@ -519,8 +558,8 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
                 xv[u][0] = ld_stream(xbase + (size_t)bn * lstride + (size_t)v0 * 16);
                 xv[u][1] = ld_stream(xbase + (size_t)bn * lstride + (size_t)v1 * 16);
             }
-            rope_pairs_row<T, TRAD>(a, tab, wtab, xa, xb, live, v0, v1, hvec, lpr, invD,
-                                    ybase + (size_t)b * ystride);
+            rope_pairs_row<T, TRAD>(a, tab, wtab, xa, xb, live, lane, v0, v1, hvec, hr, rot, lpr,
+                                    invD, ybase + (size_t)b * ystride);
         }
     }
 }
@@ -538,22 +577,24 @@ __host__ __device__ constexpr size_t rope_async_ring_bytes(int depth) {
     return (size_t)depth * 2 * kRopeThreads * 16;
 }
 
-template <typename T, bool TRAD, int HV, int DEPTH>
+template <typename T, bool TRAD, int HV, int DEPTH, bool PART = false>
 __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
     rope_pairs_async_kernel(const RopeArgs a) {
     static_assert(HV > 0, "lanes per row fixed at compile time");
     constexpr int NP = PairLayout<T, TRAD>::NP;
     constexpr int kSlots = kRopeThreads / HV;
-    // records: C [HV NP], S [HV NP], the lanes' weights W [NP][HV], then the ring
+    const int lane = threadIdx.x & (HV - 1);
+    const int slot = threadIdx.x / HV;
+    int hr, v0, v1;
+    bool rot;
+    pair_lane_vectors<PART, HV>(a, lane, HV, Elem<T>::kVec, hr, v0, v1, rot);
+    // records: C [hr NP], S [hr NP], the lanes' weights W [NP][HV], then the ring
     extern __shared__ float4 tab[];
-    float4* wtab = tab + 2 * HV * NP;
+    float4* wtab = tab + 2 * hr * NP;
     V16* ring = reinterpret_cast<V16*>(wtab + NP * HV);
 
     const int64_t chunk = blockIdx.x % a.n_chunks;
     const int64_t l = blockIdx.x / a.n_chunks;
-    const int lane = threadIdx.x & (HV - 1);
-    const int slot = threadIdx.x / HV;
-    const int v0 = lane, v1 = lane + HV;
 
     pdl_wait();
     pdl_release();
@@ -581,7 +622,7 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
     for (int r = 0; r < DEPTH; ++r) issue(r);
     // the angle table is built while the first rounds load
     build_angle_records<T, TRAD>(a, tab, l, threadIdx.x, kRopeThreads);
-    store_weight_records<T, TRAD>(a, wtab, v0, v1, true, slot == 0);
+    store_weight_records<T, TRAD>(a, wtab, lane, HV, v0, v1, true, slot == 0);
     __syncthreads();
 
     const float invD = 1.0f / (float)a.D;
@@ -592,8 +633,8 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
         const V16 xb = src[kRopeThreads];
         const int64_t b = bh0 + slot + (int64_t)r * kSlots;
         // a row past the chunk is reduced from stale shared memory and not stored
-        rope_pairs_row<T, TRAD>(a, tab, wtab, xa, xb, b < bh_end, v0, v1, HV, HV, invD,
-                                ybase + (size_t)b * ystride);
+        rope_pairs_row<T, TRAD>(a, tab, wtab, xa, xb, b < bh_end, lane, v0, v1, HV, hr, rot,
+                                HV, invD, ybase + (size_t)b * ystride);
         issue(r + DEPTH);
     }
     cp_async_wait<0>();

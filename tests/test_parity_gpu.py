@@ -585,11 +585,71 @@ def test_norm_rope_async_rounds_rejects():
                     (dict(path=nv.PATH_ROWS, stages=1), 128),
                     (dict(path=nv.PATH_ROWS, stages=-2), 128),
                     (dict(path=nv.PATH_ROWS, stages=4, vec_per_thread=1), 128),
-                    (dict(path=nv.PATH_ROWS, stages=4), 64),
+                    (dict(path=nv.PATH_ROWS, stages=4), 24),
+                    (dict(path=nv.PATH_ROWS, stages=4), 40),
                     (dict(path=nv.PATH_GENERIC, stages=4), 128)):
         with pytest.raises(nv.NvError) as e:
             nv.nv_norm_rope(x, w, x, 16, dims, 0, 10000.0, 1.0, 0, 1, 1e-6, plan=nv.Plan(**p))
         assert e.value.status == nv.NV_ERR_UNSUPPORTED, p
+
+
+def _partial_pairs_ok(D, dims, trad, dt):
+    """Whether the two-vectors-per-lane kernels take rotary dims < D: the rotated features
+    fill an even number of whole 16-byte vectors (halves: dims / 2 of them on each side) and
+    a row is 4, 8 or 16 lanes of two vectors."""
+    vec = 8 if dt == "bf16" else 4
+    whole = dims % (2 * vec) == 0 if trad else (dims // 2) % vec == 0
+    return whole and (D // vec) // 2 in (4, 8, 16)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("D,dims_list", [(128, (16, 32, 48, 64, 96, 112, 120)),
+                                         (64, (16, 32, 48, 8)), (256, (32, 64, 128, 192, 240))],
+                         ids=lambda v: str(v) if isinstance(v, int) else "-".join(map(str, v)))
+def test_norm_rope_partial_rotary_pairs(D, dims_list, dt):
+    """Rotary dims < D through the two-vectors-per-lane kernels (register and ring forms):
+    the rotated lanes hold partner vectors, the others the features past dims, which are
+    only normalised and weighted.  Ragged chunks of rows, without weights, without
+    normalisation, and in place too; a plan the shape cannot take is refused."""
+    B, H, L = 2, 5, 21
+    inp = synth.norm_rope_inputs(B, H, L, D, dt, seed=D + 17)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    plans = [None, dict(path=nv.PATH_ROWS, stages=-1), dict(path=nv.PATH_ROWS, stages=2),
+             dict(path=nv.PATH_ROWS, stages=4, rows_per_cta=7),
+             dict(path=nv.PATH_ROWS, stages=-1, rows_per_cta=3),
+             dict(path=nv.PATH_ROWS, vec_per_thread=1)]
+    for dims in dims_list:
+        for trad in (0, 1):
+            ok = _partial_pairs_ok(D, dims, trad, dt)
+            for normalize, wt in ((1, w), (0, w), (1, None)):
+                wh = host(inp["w"]) if wt is not None else None
+                ref = oracle.norm_rope(host(inp["x"]), wh, L, dims, trad, 10000.0, 1.0, 300,
+                                       normalize, 1e-6)
+                for p in plans:
+                    tag = f"D={D} dims={dims} trad={trad} norm={normalize} w={wt is not None} {p}"
+                    g = Guarded(x.shape, x.dtype)
+                    # where the pairs kernels take the shape no plan is refused; where they
+                    # do not, every ring plan is
+                    ring = p is not None and p.get("stages", 0) >= 2
+                    try:
+                        nv.nv_norm_rope(x, wt, g.t, L, dims, trad, 10000.0, 1.0, 300, normalize,
+                                        1e-6, plan=None if p is None else nv.Plan(**p))
+                    except nv.NvError as e:
+                        assert e.status == nv.NV_ERR_UNSUPPORTED, tag
+                        assert not ok, tag
+                        continue
+                    assert ok or not ring, tag
+                    torch.cuda.synchronize()
+                    assert g.bands_intact(), tag
+                    check_out(g.t, ref, tag)
+            if ok:
+                xi = x.clone()
+                nv.nv_norm_rope(xi, w, xi, L, dims, trad, 10000.0, 1.0, 300, 1, 1e-6,
+                                plan=nv.Plan(path=nv.PATH_ROWS, stages=3))
+                torch.cuda.synchronize()
+                ref = oracle.norm_rope(host(inp["x"]), host(inp["w"]), L, dims, trad, 10000.0,
+                                       1.0, 300, 1, 1e-6)
+                check_out(xi, ref, f"in place D={D} dims={dims} trad={trad}")
 
 
 def test_norm_rope_in_place():
