@@ -677,7 +677,7 @@ struct RopePlan {
     int64_t n_chunks;
 };
 
-template <typename T, bool TRAD, int HV, bool PART>
+template <typename T, bool TRAD, int HV, int PART>
 nv_status launch_rope_async(cudaStream_t s, const RopeArgs& a, int depth) {
     const size_t smem = (size_t)a.half * sizeof(float4) +
                         (size_t)Elem<T>::kVec / 2 * (size_t)HV * sizeof(float4) +
@@ -698,17 +698,22 @@ nv_status launch_rope_async(cudaStream_t s, const RopeArgs& a, int depth) {
 template <typename T, bool TRAD>
 nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a, bool pairs,
                            int depth) {
-    // dims < D (the plan only takes the pairs kernels there at 4, 8 or 16 lanes per row)
-    const bool part = a.dims < a.D;
+    // dims < D (the plan only takes the pairs kernels there at 4, 8 or 16 lanes per row):
+    // PART 1 while fewer than half the lanes of a row rotate, else 2
+    const int part = a.dims == a.D ? 0 : (2 * (a.half / Elem<T>::kVec) < a.nvec / 2 ? 1 : 2);
     if (depth > 0) {
         const int hv = a.nvec / 2;
-        if (part)
-            return hv == 8    ? launch_rope_async<T, TRAD, 8, true>(s, a, depth)
-                   : hv == 16 ? launch_rope_async<T, TRAD, 16, true>(s, a, depth)
-                              : launch_rope_async<T, TRAD, 4, true>(s, a, depth);
-        return hv == 8    ? launch_rope_async<T, TRAD, 8, false>(s, a, depth)
-               : hv == 16 ? launch_rope_async<T, TRAD, 16, false>(s, a, depth)
-                          : launch_rope_async<T, TRAD, 4, false>(s, a, depth);
+        if (part == 1)
+            return hv == 8    ? launch_rope_async<T, TRAD, 8, 1>(s, a, depth)
+                   : hv == 16 ? launch_rope_async<T, TRAD, 16, 1>(s, a, depth)
+                              : launch_rope_async<T, TRAD, 4, 1>(s, a, depth);
+        if (part == 2)
+            return hv == 8    ? launch_rope_async<T, TRAD, 8, 2>(s, a, depth)
+                   : hv == 16 ? launch_rope_async<T, TRAD, 16, 2>(s, a, depth)
+                              : launch_rope_async<T, TRAD, 4, 2>(s, a, depth);
+        return hv == 8    ? launch_rope_async<T, TRAD, 8, 0>(s, a, depth)
+               : hv == 16 ? launch_rope_async<T, TRAD, 16, 0>(s, a, depth)
+                          : launch_rope_async<T, TRAD, 4, 0>(s, a, depth);
     }
     // the pairs kernel keeps its lanes' weights after the table: VEC/2 records per lane
     const size_t smem = (size_t)a.half * sizeof(float4) +
@@ -716,14 +721,17 @@ nv_status launch_rope_rows(const DevInfo& di, cudaStream_t s, const RopeArgs& a,
                                : 0);
     // the pairs kernel with lanes per row fixed at compile time where hvec is 4, 8 or 16
     const int hv = pairs && a.lpr == a.nvec / 2 ? a.nvec / 2 : 0;
-    auto kern = !pairs           ? rope_rows_kernel<T, TRAD>
-                : part && hv == 8  ? rope_pairs_kernel<T, TRAD, 8, true>
-                : part && hv == 16 ? rope_pairs_kernel<T, TRAD, 16, true>
-                : part             ? rope_pairs_kernel<T, TRAD, 4, true>
-                : hv == 8          ? rope_pairs_kernel<T, TRAD, 8>
-                : hv == 16         ? rope_pairs_kernel<T, TRAD, 16>
-                : hv == 4          ? rope_pairs_kernel<T, TRAD, 4>
-                                   : rope_pairs_kernel<T, TRAD, 0>;
+    auto kern = !pairs                ? rope_rows_kernel<T, TRAD>
+                : part == 1 && hv == 8  ? rope_pairs_kernel<T, TRAD, 8, 1>
+                : part == 1 && hv == 16 ? rope_pairs_kernel<T, TRAD, 16, 1>
+                : part == 1             ? rope_pairs_kernel<T, TRAD, 4, 1>
+                : part == 2 && hv == 8  ? rope_pairs_kernel<T, TRAD, 8, 2>
+                : part == 2 && hv == 16 ? rope_pairs_kernel<T, TRAD, 16, 2>
+                : part == 2             ? rope_pairs_kernel<T, TRAD, 4, 2>
+                : hv == 8               ? rope_pairs_kernel<T, TRAD, 8>
+                : hv == 16              ? rope_pairs_kernel<T, TRAD, 16>
+                : hv == 4               ? rope_pairs_kernel<T, TRAD, 4>
+                                        : rope_pairs_kernel<T, TRAD, 0>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -766,8 +774,8 @@ nv_status rope_plan(int64_t rows, int64_t L, int64_t D, int dims, bool trad, nv_
     // register kernel, 0: automatic.  Measured on [8, 32, 2048, 128]:
     //   dims == D, bfloat16: 2 rounds, 45.4-45.7 us (register kernel 48.2, 3 rounds 45.8);
     //   dims == D, float32:  the register kernel, 86.8 us (the ring 87.0-87.5);
-    //   dims < D,  bfloat16: 3 rounds, 45.9 / 51.6 / 48.7 us at dims 32 / 64 / 96 (2 rounds
-    //                        46.9 / 52.2 / 49.6, register kernel 57-69);
+    //   dims < D,  bfloat16: 3 rounds, 45.9 / 47.6 / 47.8 us at dims 32 / 64 / 96 (2 rounds
+    //                        46.7 / 48.3 / 48.2, register kernel 57-61);
     //   dims < D,  float32:  4 rounds, 87.6-88.6 us (register kernel 104-107).
     const int hv = (int)(nvec / 2);
     const bool ring_ok = rp->pairs && (hv == 4 || hv == 8 || hv == 16);

@@ -412,8 +412,17 @@ __device__ __forceinline__ void store_weight_records(const RopeArgs& a, float4* 
 // hvec = nvec / 2 vectors a lane group covers per side (the weight records' stride: record
 // k * hvec + lane), lpr lanes per row; hr of the lanes rotate (hr = hvec when dims == D) and
 // the table holds hr * NP C records, then as many S records; a lane with rot == false holds
-// two vectors past dims, which keep a = x w and take the row's 1/rms.
-template <typename T, bool TRAD>
+// two vectors past dims, which keep a = x w and take the row's 1/rms.  PART selects how:
+//   0  dims == D, every lane rotates;
+//   1  the lanes past dims branch off to a scaling loop (cheaper while fewer than half the
+//      lanes of a row rotate: the rotating loop then runs on few lanes);
+//   2  every lane runs the rotating loop, those past dims on lane 0's records (a broadcast)
+//      and keeping their weighted inputs by a select, so the result is exactly a = x w
+//      whatever the discarded rotation gives; one instruction stream, each weight record
+//      read once.
+// Measured, bf16 [8, 32, 2048, 128], ring of 3 rounds: dims 32 / 64 / 96 with form 1
+// 45.9 / 51.6 / 48.7 us, with form 2 47.6 / 47.7 / 47.8 us.
+template <typename T, bool TRAD, int PART>
 __device__ __forceinline__ void rope_pairs_row(const RopeArgs& a, const float4* ctab,
                                                const float4* wtab, const V16& xa, const V16& xb,
                                                bool live, int lane, int v0, int v1, int hvec,
@@ -434,7 +443,24 @@ __device__ __forceinline__ void rope_pairs_row(const RopeArgs& a, const float4* 
     const float2 inv2 = make_float2(inv, inv);
     if (live) {  // only lanes holding vectors read the table
         float2 yp[NP], yq[NP];
-        if (rot) {
+        if (PART == 2) {
+            // every lane rotates: a lane past dims reads lane 0's records of the slot (a
+            // broadcast) and keeps its weighted inputs by a select
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+                const int rec = PL::record(rot ? v0 : 0, rot ? v1 : hr, k, hr);
+                const float4 c4 = ctab[rec], s4 = ctab[hr * NP + rec];
+                const float2 ch = make_float2(c4.x, c4.y), cl = make_float2(c4.z, c4.w);
+                const float2 sh = make_float2(s4.x, s4.y), sl = make_float2(s4.z, s4.w);
+                const float4 w4 = wtab[k * hvec + lane];
+                const float2 ap = mul2(p[k], make_float2(w4.x, w4.y));
+                const float2 aq = mul2(q[k], make_float2(w4.z, w4.w));
+                const float2 rp = rotate_sub2(ap, aq, ch, cl, sh, sl);
+                const float2 rq = rotate_pair2(aq, ap, ch, cl, sh, sl);
+                yp[k] = mul2(rot ? rp : ap, inv2);
+                yq[k] = mul2(rot ? rq : aq, inv2);
+            }
+        } else if (rot) {
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
                 const int rec = PL::record(v0, v1, k, hr);
@@ -447,7 +473,7 @@ __device__ __forceinline__ void rope_pairs_row(const RopeArgs& a, const float4* 
                 yp[k] = mul2(rotate_sub2(ap, aq, ch, cl, sh, sl), inv2);
                 yq[k] = mul2(rotate_pair2(aq, ap, ch, cl, sh, sl), inv2);
             }
-        } else {  // past dims: a = x w, then the row's 1/rms
+        } else {  // past dims, lanes diverged from the rotating ones: a = x w, then 1/rms
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
                 const float4 w4 = wtab[k * hvec + lane];
@@ -473,7 +499,7 @@ __host__ __device__ constexpr int rope_pairs_unroll() { return sizeof(T) == 4 ? 
 // the group sum a fixed butterfly; HV = 0 takes them from the arguments.
 constexpr int kRopeThreads = 256;
 
-// PART (HV > 0 only): dims < D.  The first hr = dims / (2 VEC) lanes of a row hold the
+// PART (dims < D, HV > 0 only): the first hr = dims / (2 VEC) lanes of a row hold the
 // rotated vectors as partner pairs (lane j: vectors j and j + hr), the others two of the
 // vectors past dims each (lane j: R + j - hr and that plus (nvec - R) / 2, R = dims / VEC).
 template <bool PART, int HV>
@@ -493,7 +519,7 @@ __device__ __forceinline__ void pair_lane_vectors(const RopeArgs& a, int lane, i
     v1 = rot ? lane + hr : v0 + (a.nvec - R) / 2;
 }
 
-template <typename T, bool TRAD, int HV, bool PART = false>
+template <typename T, bool TRAD, int HV, int PART = 0>
 __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
     rope_pairs_kernel(const RopeArgs a) {
     constexpr int kUnroll = rope_pairs_unroll<T>();
@@ -508,10 +534,10 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
     const int lane = threadIdx.x & (lpr - 1);
     const int slot = threadIdx.x / lpr;
     const int slots = kRopeThreads / lpr;
-    static_assert(!PART || HV > 0, "dims < D takes the fixed-lane kernels");
+    static_assert(PART == 0 || HV > 0, "dims < D takes the fixed-lane kernels");
     int hr, v0, v1;
     bool rot;
-    pair_lane_vectors<PART, HV>(a, lane, hvec, Elem<T>::kVec, hr, v0, v1, rot);
+    pair_lane_vectors<PART != 0, HV>(a, lane, hvec, Elem<T>::kVec, hr, v0, v1, rot);
     // with HV fixed every lane of a group holds vectors (lpr == hvec)
     const bool has_vec = HV > 0 || lane < hvec;
 
@@ -558,8 +584,8 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
                 xv[u][0] = ld_stream(xbase + (size_t)bn * lstride + (size_t)v0 * 16);
                 xv[u][1] = ld_stream(xbase + (size_t)bn * lstride + (size_t)v1 * 16);
             }
-            rope_pairs_row<T, TRAD>(a, tab, wtab, xa, xb, live, lane, v0, v1, hvec, hr, rot, lpr,
-                                    invD, ybase + (size_t)b * ystride);
+            rope_pairs_row<T, TRAD, PART>(a, tab, wtab, xa, xb, live, lane, v0, v1, hvec, hr, rot,
+                                          lpr, invD, ybase + (size_t)b * ystride);
         }
     }
 }
@@ -577,7 +603,7 @@ __host__ __device__ constexpr size_t rope_async_ring_bytes(int depth) {
     return (size_t)depth * 2 * kRopeThreads * 16;
 }
 
-template <typename T, bool TRAD, int HV, int DEPTH, bool PART = false>
+template <typename T, bool TRAD, int HV, int DEPTH, int PART = 0>
 __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
     rope_pairs_async_kernel(const RopeArgs a) {
     static_assert(HV > 0, "lanes per row fixed at compile time");
@@ -587,7 +613,7 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
     const int slot = threadIdx.x / HV;
     int hr, v0, v1;
     bool rot;
-    pair_lane_vectors<PART, HV>(a, lane, HV, Elem<T>::kVec, hr, v0, v1, rot);
+    pair_lane_vectors<PART != 0, HV>(a, lane, HV, Elem<T>::kVec, hr, v0, v1, rot);
     // records: C [hr NP], S [hr NP], the lanes' weights W [NP][HV], then the ring
     extern __shared__ float4 tab[];
     float4* wtab = tab + 2 * hr * NP;
@@ -633,8 +659,8 @@ __global__ void __launch_bounds__(kRopeThreads, sizeof(T) == 2 ? 4 : 3)
         const V16 xb = src[kRopeThreads];
         const int64_t b = bh0 + slot + (int64_t)r * kSlots;
         // a row past the chunk is reduced from stale shared memory and not stored
-        rope_pairs_row<T, TRAD>(a, tab, wtab, xa, xb, b < bh_end, lane, v0, v1, HV, hr, rot,
-                                HV, invD, ybase + (size_t)b * ystride);
+        rope_pairs_row<T, TRAD, PART>(a, tab, wtab, xa, xb, b < bh_end, lane, v0, v1, HV, hr,
+                                      rot, HV, invD, ybase + (size_t)b * ystride);
         issue(r + DEPTH);
     }
     cp_async_wait<0>();

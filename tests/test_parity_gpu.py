@@ -652,6 +652,40 @@ def test_norm_rope_partial_rotary_pairs(D, dims_list, dt):
                 check_out(xi, ref, f"in place D={D} dims={dims} trad={trad}")
 
 
+@pytest.mark.parametrize("dims", [32, 64, 96])
+def test_norm_rope_partial_rotary_non_finite(dims):
+    """A non-finite input stays in its row, and a lane past dims keeps exactly x w (times the
+    row's 1/rms) whatever its partner vector holds: with normalize an Inf anywhere in a row
+    makes its 1/rms zero, so the oracle's row is NaN at the Inf and its pair partner and
+    zero elsewhere; without normalize an Inf past dims passes through as Inf and leaves every
+    other element of its row alone.  Every kernel form, both ways of running the lanes past
+    dims (dims 32: branched, 64 and 96: one instruction stream)."""
+    B, H, L, D = 1, 4, 12, 128
+    inp = synth.norm_rope_inputs(B, H, L, D, "bf16", seed=dims)
+    xh = inp["x"].clone()
+    rows = xh.shape[0]
+    xh[3, D - 5] = float("inf")                # past dims, normalize and plain
+    xh[7, dims + 1] = -float("inf")
+    xh[20, 1] = float("inf")                   # rotated: normalize only
+    w = dev(inp["w"])
+    plans = [None, dict(path=nv.PATH_ROWS, stages=2), dict(path=nv.PATH_ROWS, stages=-1),
+             dict(path=nv.PATH_ROWS, vec_per_thread=1), dict(path=nv.PATH_GENERIC)]
+    for normalize in (1, 0):
+        xn = xh.clone()
+        if not normalize:
+            xn[20, 1] = 0.0
+        ref = oracle.norm_rope(host(xn), host(inp["w"]), L, dims, 0, 10000.0, 1.0, 5, normalize,
+                               1e-6)
+        x = dev(xn)
+        for p in plans:
+            y = torch.empty_like(x)
+            nv.nv_norm_rope(x, w, y, L, dims, 0, 10000.0, 1.0, 5, normalize, 1e-6,
+                            plan=None if p is None else nv.Plan(**p))
+            torch.cuda.synchronize()
+            check_out(y, ref, f"dims={dims} normalize={normalize} {p}")
+        assert rows == B * H * L
+
+
 def test_norm_rope_in_place():
     inp = synth.norm_rope_inputs(2, 4, 16, 128, "bf16", seed=4)
     ref = oracle.norm_rope(host(inp["x"]), host(inp["w"]), 16, 128, 1, 10000.0, 1.0, 4096, 1, 1e-6)
