@@ -9,7 +9,8 @@ against B200's HBM peak.  Each step is timed with CUDA events on the launching s
 Steps rotate over device buffer sets and run back to back; between two uses of one set the
 other sets move at least 3x L2 through the cache, so no step reads data a previous step
 left in L2, and every step pays the write-back of its predecessor's output (workloads
-smaller than L2 flush it instead).
+whose buffers are too small for that -- under 3/8 of L2 -- are timed one step at a time
+after an L2 flush instead).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --sweep        # add_rms_norm over D x rows x dtype, one line per point
@@ -192,8 +193,9 @@ def algorithmic_bytes(op, rows, D, s, nparts=0):
 def rotation_sets(set_bytes, l2_bytes):
     """Copies of a workload's buffers to rotate over: enough that the other copies, which
     the steps between two uses of one copy touch, hold at least 3x L2 (at least 2 copies,
-    at most 9); 1 (and an L2 flush before each step) when one copy is smaller than L2."""
-    if set_bytes < l2_bytes:
+    at most 9); 1 (and an L2 flush before each step) when even 8 other copies would hold
+    less than that."""
+    if 8 * set_bytes < 3 * l2_bytes:
         return 1
     return max(2, min(9, 1 + -(-3 * l2_bytes // set_bytes)))
 
@@ -208,7 +210,7 @@ class Case:
     at normal eviction priority, unlike the streamed rows -- still made up ~5% of a
     step's reads).  Steps run back to back (each then also pays the write-back of the
     previous step's dirty lines, as in a steady stream).  Workloads too small for that
-    are timed after an L2 flush.
+    are timed one step at a time after an L2 flush.
     """
 
     def __init__(self, op, shape, dtype, seed, **kw):
@@ -290,7 +292,7 @@ class Case:
             mb = self.nsets * self.n_row_tensors * self.rows * self.D * self.s
             return (f"inputs larger than L2: {self.nsets} buffer sets ({mb / 1e6:.0f} MB) "
                     "rotated, steps back to back, no flush")
-        return "L2 flushed before every step (write of 2x L2)"
+        return "L2 flushed before every step (read of 2x L2)"
 
     def run(self, stream=None, i=0):
         d, nv, k = self.sets[i % self.nsets], self.nv, self.kw
@@ -338,7 +340,15 @@ class Case:
 
 def l2_flush_buffer():
     l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
-    return torch.empty(2 * max(l2, 64 << 20), dtype=torch.uint8, device="cuda")
+    return torch.zeros(2 * max(l2, 64 << 20), dtype=torch.uint8, device="cuda")
+
+
+def flush_l2(buf):
+    """Evict the cache by reading a buffer of twice its size.  A read leaves clean lines
+    behind: writing the buffer instead would leave 2x L2 of dirty lines whose write-back
+    the next kernel pays (a 67 MB add_rms_norm step timed 18.5 us after a write flush
+    against 12.8 us back to back in steady state)."""
+    torch.amax(buf)
 
 
 class nvtx_range:
@@ -393,14 +403,14 @@ def time_steps(case, steps, warmup, flush, e2e=False):
     use_flush = e2e or not case.rotating
     for i in range(warmup):
         if use_flush:
-            flush.zero_()
+            flush_l2(flush)
         fn(stream, i)
     torch.cuda.synchronize()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     for i in range(steps):
         if use_flush:
-            flush.zero_()
+            flush_l2(flush)
         with nvtx_range(f"{case.op}{' e2e' if e2e else ''} step {i}"):
             starts[i].record(stream)
             fn(stream, i)

@@ -72,13 +72,16 @@ def test_nvtx_ranges_nest_and_never_raise():
 
 def test_rotation_keeps_three_l2_between_uses_of_a_buffer_set():
     """Between two uses of one buffer set the other sets hold at least 3x L2, so no line a
-    step reads can have survived in L2 from that set's last use."""
+    step reads can have survived in L2 from that set's last use; sets too small for that
+    within 9 copies (under 3/8 of L2) are flushed instead."""
     l2 = 126 * 2 ** 20
     for set_bytes, want in [(268435456, 3),      # add_rms_norm / norm_rope bf16 sets
                             (536870912, 2),      # layer_norm bf16 [16384, 8192]
                             (201326592, 3),      # rms_norm_vjp
                             (134217728, 4),      # rms_norm bf16 [8192, 4096]
-                            (l2, 4), (l2 - 1, 1), (10 * l2, 2), (l2 // 2 + 2 ** 20, 1)]:
+                            (l2, 4), (l2 - 1, 5), (10 * l2, 2), (l2 // 2 + 2 ** 20, 7),
+                            (67108864 * 2 // 2, 7),  # add_rms_norm bf16 [4096, 2048]
+                            (3 * l2 // 8, 9), (3 * l2 // 8 - 1, 1), (l2 // 4, 1)]:
         n = bench.rotation_sets(set_bytes, l2)
         assert n == want, (set_bytes, n, want)
         if n > 1:
