@@ -427,9 +427,9 @@ NV_API nv_status nv_selftest_bounded_wait(int32_t ctas, nv_stream_t stream);
  *                   launch; NV_LAUNCH_PLAIN: ordinary stream-ordered launch.
  *   stages          NV_PATH_RING: shared-memory row buffers per CTA (0 = as many as fit,
  *                   at most 32; a multiple of rows_per_cta, at least 2 x rows_per_cta).
- *                   NV_PATH_SLOTS: 1 = each row slot asks L2 for its next row while it
- *                   works on the current one (one bulk prefetch a row); -1 = no prefetch;
- *                   0 = prefetch when a row spans several warps.  norm_rope register path
+ *                   NV_PATH_SLOTS: 1 or 0 = each row slot asks L2 for its next row once
+ *                   its current row has landed (one bulk prefetch a row); -1 = no
+ *                   prefetch.  norm_rope register path
  *                   with two vectors per lane of 4, 8 or 16 lanes: 2..6 = that many rounds
  *                   of rows in flight per lane group, staged by per-thread asynchronous
  *                   copies into shared memory; -1 = rows in flight in registers; 0 =

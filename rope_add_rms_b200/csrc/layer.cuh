@@ -168,6 +168,16 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 256 ? 768 / MAXT : 1)
         s2 += s2b;
         s1 = warp_sum(s1);
         s2 = warp_sum(s2);
+        // bfloat16: the row's loads have landed, so ask L2 for this slot's next row (one bulk
+        // prefetch of the whole row from this GPU's own memory, nothing to wait on).
+        // Measured: [65536, 1024] 70.3 -> 65.0 us, [131072, 512] 82.4 -> 72.1 us; float32
+        // rows gain nothing ([65536, 1024] 95.4 -> 99.1 us) and go without.
+        if constexpr (sizeof(T) == 2) {
+            const int64_t next = row + (int64_t)gridDim.x * a.rows_per_cta;
+            if (t == 0 && next < a.rows)
+                prefetch_l2(static_cast<const char*>(a.x) + (size_t)next * (size_t)a.D * sizeof(T),
+                            (uint32_t)((size_t)a.D * sizeof(T)));
+        }
         if (wpr > 1) {
             double* b1 = red[it & 1][0];
             double* b2 = red[it & 1][1];

@@ -261,26 +261,26 @@ constexpr int kStaticSmemReserve = 2048;  // static shared memory + per-CTA syst
 // (64 bytes a vector) must fit the shared memory.
 bool slots_shape(int nvec, const nv_plan& req, const DevInfo* di, nv_plan* out) {
     nv_plan p = req;
-    // measured on B200 (bf16, 2^27 elements): 8 vectors a thread in CTAs of 768 threads,
-    // except rows of 257..512 vectors (D = 4096), which run 4 % faster with 4 vectors a
-    // thread in CTAs of 1024 threads (32 warps at 64 registers)
-    const bool mid = nvec > 256 && nvec <= 512;
-    int v = p.vec_per_thread ? p.vec_per_thread : (nvec >= 256 && !mid ? 8 : 4);
+    // measured on B200 (bf16, 2^26-2^27 elements, the prefetch after the warp sums): 8
+    // vectors a thread in CTAs of 768 threads from 256 vectors a row on (D = 4096: 51.9 us
+    // against 52.7 with 4 vectors in CTAs of 1024 threads, the better form while the
+    // prefetch came at the row's start), 4 below (D = 1024: 48.1 us, with 8 vectors 67.1)
+    int v = p.vec_per_thread ? p.vec_per_thread : (nvec >= 256 ? 8 : 4);
     if (v != 4 && v != 8) return false;
     int g = p.threads_per_row ? p.threads_per_row : ((nvec + v - 1) / v + 31) / 32 * 32;
     if (g % 32 || g < 32 || (int64_t)g * v < nvec || g > kSlotsMaxThreads) return false;
     // 768 threads (24 warps, 80 registers) unless asked for more rows per CTA
-    int slots = p.rows_per_cta ? p.rows_per_cta : ((mid && v == 4) ? 1024 : 768) / g;
+    int slots = p.rows_per_cta ? p.rows_per_cta : 768 / g;
     if (g > 32) slots = std::min(slots, 15);
     if (slots < 1 || slots * g > kSlotsMaxThreads || (g > 32 && slots > 15)) return false;
     const size_t optin = (size_t)(di ? di->smem_optin : 232448) - kStaticSmemReserve;
     if (slots_table_bytes(nvec) > optin) return false;
     if (p.ctas_per_sm > 1) return false;  // one table per SM
-    // stages: 1 = each slot prefetches its next row into L2 (one bulk prefetch a row),
-    // -1 = no prefetch, 0 = prefetch when a row spans several warps (measured: it gains
-    // 1-5 % from D = 4096 on, and loses 3 % at D = 2048, a warp per row)
+    // stages: 1 (and 0, automatic) = each slot prefetches its next row into L2 once its
+    // current row has landed (one bulk prefetch a row), -1 = no prefetch.  Measured, bf16:
+    // D = 1024 48.1 against 53.9 us, D = 2048 49.5 against 51.5, D = 4096 52.6 against 56.8
     if (p.stages != 0 && p.stages != 1 && p.stages != -1) return false;
-    p.stages = p.stages == 0 ? (g > 32 ? 1 : -1) : p.stages;
+    p.stages = p.stages == 0 ? 1 : p.stages;
     p.vec_per_thread = v;
     p.threads_per_row = g;
     p.rows_per_cta = slots;
@@ -353,10 +353,10 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
     if (p.path == NV_PATH_AUTO) {
         int v = 0, g = 0;
         nv_plan sp{};
-        // bfloat16 layer_norm: the slots kernel (measured 10-20 % faster than the register
-        // kernel over D = 2048..16384 on B200) from rows of 256 vectors on, whenever its
-        // w/b table fits
-        if (op == OP_LAYER && dt == NV_BF16 && vec_ok && nvec >= 256 && p.vec_per_thread == 0 &&
+        // bfloat16 layer_norm: the slots kernel from rows of 128 vectors on, whenever its
+        // w/b table fits.  Measured against the register kernel on B200: D = 1024 48.1
+        // against 64.6 us, D = 2048..16384 10-20 % faster; at D = 512 the two tie
+        if (op == OP_LAYER && dt == NV_BF16 && vec_ok && nvec >= 128 && p.vec_per_thread == 0 &&
             p.threads_per_row == 0 && p.rows_per_cta == 0 && slots_shape(nvec, p, di, &sp))
             p.path = NV_PATH_SLOTS;
         else
