@@ -264,8 +264,12 @@ bool slots_shape(int nvec, const nv_plan& req, const DevInfo* di, nv_plan* out) 
     // measured on B200 (bf16, 2^26-2^27 elements, the prefetch after the warp sums): 8
     // vectors a thread in CTAs of 768 threads from 256 vectors a row on (D = 4096: 51.9 us
     // against 52.7 with 4 vectors in CTAs of 1024 threads, the better form while the
-    // prefetch came at the row's start), 4 below (D = 1024: 48.1 us, with 8 vectors 67.1)
-    int v = p.vec_per_thread ? p.vec_per_thread : (nvec >= 256 ? 8 : 4);
+    // prefetch came at the row's start); below, whichever of 4 and 8 leaves fewer lanes of
+    // a row without a vector, 8 on a tie (fewer threads a row): D = 768 and 1024 take 4
+    // (56.3 and 48.1 us; with 8, 81.9 and 67.3), D = 1536 takes 8 (54.1 us; with 4, 61.4)
+    const auto lanes = [nvec](int vv) { return ((nvec + vv - 1) / vv + 31) / 32 * 32 * vv; };
+    int v = p.vec_per_thread ? p.vec_per_thread
+                             : (nvec >= 256 || lanes(8) <= lanes(4) ? 8 : 4);
     if (v != 4 && v != 8) return false;
     int g = p.threads_per_row ? p.threads_per_row : ((nvec + v - 1) / v + 31) / 32 * 32;
     if (g % 32 || g < 32 || (int64_t)g * v < nvec || g > kSlotsMaxThreads) return false;
@@ -353,10 +357,11 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
     if (p.path == NV_PATH_AUTO) {
         int v = 0, g = 0;
         nv_plan sp{};
-        // bfloat16 layer_norm: the slots kernel from rows of 128 vectors on, whenever its
-        // w/b table fits.  Measured against the register kernel on B200: D = 1024 48.1
-        // against 64.6 us, D = 2048..16384 10-20 % faster; at D = 512 the two tie
-        if (op == OP_LAYER && dt == NV_BF16 && vec_ok && nvec >= 128 && p.vec_per_thread == 0 &&
+        // bfloat16 layer_norm: the slots kernel for rows of more than 64 vectors, whenever
+        // its w/b table fits.  Measured against the register kernel on B200: D = 768 56.3
+        // against 77.6 us, D = 1024 48.1 against 64.6, D = 1536 54.1 against 67.0,
+        // D = 2048..16384 10-20 % faster; at D = 512 the two tie
+        if (op == OP_LAYER && dt == NV_BF16 && vec_ok && nvec > 64 && p.vec_per_thread == 0 &&
             p.threads_per_row == 0 && p.rows_per_cta == 0 && slots_shape(nvec, p, di, &sp))
             p.path = NV_PATH_SLOTS;
         else

@@ -196,7 +196,11 @@ def test_plain_rope_ignores_eps():
     ("add_rms_norm", 2 ** 17, "bf16", dict(path=2)),
     ("rms_norm", 512, "f32", dict(path=1, vec_per_thread=4, threads_per_row=32, rows_per_cta=4)),
     ("layer_norm", 512, "bf16", dict(path=1, vec_per_thread=2, threads_per_row=32, rows_per_cta=4)),
+    ("layer_norm", 768, "bf16", dict(path=5, vec_per_thread=4, threads_per_row=32, rows_per_cta=24,
+                                     stages=1)),
     ("layer_norm", 1024, "bf16", dict(path=5, vec_per_thread=4, threads_per_row=32, rows_per_cta=24,
+                                      stages=1)),
+    ("layer_norm", 1536, "bf16", dict(path=5, vec_per_thread=8, threads_per_row=32, rows_per_cta=24,
                                       stages=1)),
     ("layer_norm", 2048, "bf16", dict(path=5, vec_per_thread=8, threads_per_row=32, rows_per_cta=24,
                                       stages=1)),
