@@ -17,7 +17,8 @@
 //     shared by the CTA's row slots (16-byte words, word q of every vector contiguous, so
 //     the lanes of a warp read consecutive words);
 //   - a CTA holds `slots` rows at a time (G threads each); a row's cross-warp reduction
-//     uses a named barrier of its slot alone;
+//     uses a named barrier of its slot alone, and rows narrower than a warp (G = 2, 4, 8 or
+//     16) share warps, reducing over their own lanes;
 //   - prefetching form (PREFETCH): once a row's loads have landed (after its warp sums, before
 //     the cross-warp step), one thread of the slot asks L2 for the slot's next row
 //     (cp.async.bulk.prefetch.L2, one bulk prefetch of the whole row from this GPU's own
@@ -80,7 +81,8 @@ __host__ __device__ constexpr size_t slots_table_bytes(int nvec) {
 // (32 warps, up to 64 registers).
 constexpr int kSlotsMaxThreads = 1024;
 
-// Launch: blockDim.x = a.G * a.rows_per_cta (rows_per_cta = slots <= 15 when G > 32),
+// Launch: blockDim.x = a.G * a.rows_per_cta, a multiple of 32 (rows_per_cta = slots <= 15
+// when G > 32; G a multiple of 32 or a power of two up to 16),
 // dynamic shared memory = slots_table_bytes(a.nvec); persistent grid.
 template <int VPT, bool PREFETCH, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1) layer_slots_kernel(const RowArgs a) {
@@ -97,6 +99,7 @@ __global__ void __launch_bounds__(MAXT, 1) layer_slots_kernel(const RowArgs a) {
     const int slot = threadIdx.x / G;
     const int t = threadIdx.x - slot * G;
     const int wpr = G >> 5;
+    const int gw = G < 32 ? G : 32;  // lanes of a row within a warp
     const int warp = threadIdx.x >> 5;
     const int nvec = a.nvec;
     const uint32_t row_bytes = (uint32_t)nvec * 16u;
@@ -158,8 +161,8 @@ __global__ void __launch_bounds__(MAXT, 1) layer_slots_kernel(const RowArgs a) {
                 else
                     bf16x2_stats(xv[k].u[q], s1, s1b, s2, s2b);
             }
-        s1 = warp_sum((s1 + s1b) + (t1 + t1b));
-        s2 = warp_sum((s2 + s2b) + (t2 + t2b));
+        s1 = group_sum((s1 + s1b) + (t1 + t1b), gw);
+        s2 = group_sum((s2 + s2b) + (t2 + t2b), gw);
         // the row is in registers: ask L2 for the slot's next row (see the header)
         if constexpr (PREFETCH) {
             if (t == 0 && row + row_step < a.rows)
@@ -182,7 +185,11 @@ __global__ void __launch_bounds__(MAXT, 1) layer_slots_kernel(const RowArgs a) {
         }
         const double mean = s1 * invD;
         double var = s2 * invD - mean * mean;
-        if (!(var > ldexp(mean * mean, -20))) {
+        // centred second pass: uniform over a slot, and for slots narrower than a warp
+        // taken by the whole warp when any of its slots needs it (its shuffles are
+        // warp-wide), each slot keeping its own result only if it asked for it
+        const bool centre = !(var > ldexp(mean * mean, -20));
+        if (G < 32 ? __any_sync(0xFFFFFFFFu, centre) : centre) {
             // centred second pass (uniform over the slot's threads)
             double c2 = 0.0;
 #pragma unroll
@@ -190,14 +197,14 @@ __global__ void __launch_bounds__(MAXT, 1) layer_slots_kernel(const RowArgs a) {
                 if (t + k * G < nvec)
 #pragma unroll
                     for (int q = 0; q < 4; ++q) bf16x2_centred(xv[k].u[q], mean, c2);
-            c2 = warp_sum(c2);
+            c2 = group_sum(c2, gw);
             if (wpr > 1) {
                 if ((threadIdx.x & 31) == 0) rb[warp][2] = c2;
                 slot_bar(bar_id, G);
                 c2 = 0.0;
                 for (int i = 0; i < wpr; ++i) c2 += rb[slot * wpr + i][2];
             }
-            var = c2 * invD;
+            if (centre) var = c2 * invD;
         }
         const double rstd = rsqrt(var + eps);
         const float mu_hi = __double2float_rn(mean);

@@ -256,27 +256,43 @@ size_t staged_smem(Op op, int64_t D, nv_dtype dt, int stages) {
 constexpr int kStaticSmemReserve = 2048;  // static shared memory + per-CTA system use
 
 // Slots path shape (bfloat16 layer_norm): VPT vectors a thread (8, or 4 for narrow rows),
-// G threads a row, as many row slots as make 768 threads (24 warps per SM, one CTA per SM),
+// G threads a row (a multiple of 32, or 8 or 16), as many row slots as make 768 threads
+// (24 warps per SM, one CTA per SM),
 // at most 15 when a row spans several warps (one named barrier each); the float32 w/b table
 // (64 bytes a vector) must fit the shared memory.
 bool slots_shape(int nvec, const nv_plan& req, const DevInfo* di, nv_plan* out) {
     nv_plan p = req;
-    // measured on B200 (bf16, 2^26-2^27 elements, the prefetch after the warp sums): 8
-    // vectors a thread in CTAs of 768 threads from 256 vectors a row on (D = 4096: 51.9 us
-    // against 52.7 with 4 vectors in CTAs of 1024 threads, the better form while the
-    // prefetch came at the row's start); below, whichever of 4 and 8 leaves fewer lanes of
-    // a row without a vector, 8 on a tie (fewer threads a row): D = 768 and 1024 take 4
-    // (56.3 and 48.1 us; with 8, 81.9 and 67.3), D = 1536 takes 8 (54.1 us; with 4, 61.4)
-    const auto lanes = [nvec](int vv) { return ((nvec + vv - 1) / vv + 31) / 32 * 32 * vv; };
+    // threads a row: a multiple of 32, or a power of two up to 16 when that covers the row
+    // (several rows to a warp)
+    const auto threads = [nvec](int vv) {
+        const int n = (nvec + vv - 1) / vv;
+        int p2 = 1;
+        while (p2 < n) p2 *= 2;
+        return n <= 16 ? p2 : (n + 31) / 32 * 32;
+    };
+    const auto lanes = [&](int vv) { return threads(vv) * vv; };
+    // vectors a thread, measured on B200 (bf16, 2^26-2^27 elements, the prefetch after the
+    // warp sums): 8 in CTAs of 768 threads from 256 vectors a row on (D = 4096: 51.9 us
+    // against 52.7 with 4 in CTAs of 1024 threads); below, 4 where they cover the row with
+    // no idle lane (D = 256, 512, 1024: 53.6, 54.2, 52.4 us; with 8, -, 57.8, 54.6), else
+    // whichever leaves fewer lanes idle, 8 on a tie (D = 768: 57.1 against 62.4 with 4;
+    // D = 1536: 54.1 against 61.4)
     int v = p.vec_per_thread ? p.vec_per_thread
-                             : (nvec >= 256 || lanes(8) <= lanes(4) ? 8 : 4);
+                             : nvec >= 256 ? 8
+                             : lanes(4) == nvec ? 4
+                             : lanes(8) == nvec || lanes(8) <= lanes(4) ? 8 : 4;
     if (v != 4 && v != 8) return false;
-    int g = p.threads_per_row ? p.threads_per_row : ((nvec + v - 1) / v + 31) / 32 * 32;
-    if (g % 32 || g < 32 || (int64_t)g * v < nvec || g > kSlotsMaxThreads) return false;
+    int g = p.threads_per_row ? p.threads_per_row : threads(v);
+    if (g < 1 || (g % 32 && (g > 16 || (g & (g - 1)))) || (int64_t)g * v < nvec ||
+        g > kSlotsMaxThreads)
+        return false;
     // 768 threads (24 warps, 80 registers) unless asked for more rows per CTA
     int slots = p.rows_per_cta ? p.rows_per_cta : 768 / g;
     if (g > 32) slots = std::min(slots, 15);
-    if (slots < 1 || slots * g > kSlotsMaxThreads || (g > 32 && slots > 15)) return false;
+    // whole warps only: the row sums and the centred pass's vote are warp-wide shuffles
+    if (slots < 1 || slots * g > kSlotsMaxThreads || (g > 32 && slots > 15) ||
+        (slots * g) % 32 != 0)
+        return false;
     const size_t optin = (size_t)(di ? di->smem_optin : 232448) - kStaticSmemReserve;
     if (slots_table_bytes(nvec) > optin) return false;
     if (p.ctas_per_sm > 1) return false;  // one table per SM
@@ -357,11 +373,13 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
     if (p.path == NV_PATH_AUTO) {
         int v = 0, g = 0;
         nv_plan sp{};
-        // bfloat16 layer_norm: the slots kernel for rows of more than 64 vectors, whenever
-        // its w/b table fits.  Measured against the register kernel on B200: D = 768 56.3
-        // against 77.6 us, D = 1024 48.1 against 64.6, D = 1536 54.1 against 67.0,
-        // D = 2048..16384 10-20 % faster; at D = 512 the two tie
-        if (op == OP_LAYER && dt == NV_BF16 && vec_ok && nvec > 64 && p.vec_per_thread == 0 &&
+        // bfloat16 layer_norm: the slots kernel for rows of 8 vectors or more, whenever its
+        // w/b table fits.  Measured against the register kernel on B200 (2^26 elements):
+        // D = 64 143.6 against 368.1 us and D = 128 80.8 against 188.6 (with 8 threads a
+        // row), D = 256 53.6 against 101.3, D = 512 54.2 against 71.8, D = 768 56.3
+        // against 77.6, D = 1024 48.1 against 64.6, D = 1536 54.1 against 67.0,
+        // D = 2048..16384 10-20 % faster
+        if (op == OP_LAYER && dt == NV_BF16 && vec_ok && nvec >= 8 && p.vec_per_thread == 0 &&
             p.threads_per_row == 0 && p.rows_per_cta == 0 && slots_shape(nvec, p, di, &sp))
             p.path = NV_PATH_SLOTS;
         else

@@ -358,7 +358,8 @@ SLOTS = [dict(path=nv.PATH_SLOTS), dict(path=nv.PATH_SLOTS, vec_per_thread=4),
                                         (5, 16384, (1, 1)), (64, 512, (1, 1)), (300, 256, (0, 1)),
                                         (1000, 2048, (1, 1)), (1, 8192, (1, 1)), (2, 8, (1, 1)),
                                         (77, 24576, (1, 1)), (500, 1024, (1, 1)),
-                                        (129, 1536, (0, 1)), (311, 768, (1, 1))])
+                                        (129, 1536, (0, 1)), (311, 768, (1, 1)), (1001, 128, (1, 1)),
+                                        (999, 64, (1, 0)), (77, 32, (1, 1))])
 def test_layer_norm_slots(rows, D, wb, plan):
     """The slots path (bfloat16): rows in registers, several per CTA sharing a float32 table
     of w and b, x consumed packed by bfloat16 -> double conversions and mixed-precision fma."""
