@@ -222,14 +222,20 @@ int max_threads(Op op, int vpt) {
 // 16-byte vectors per thread and tensor -- enough loads in flight per thread while
 // keeping several CTAs per SM -- unless the row would then need more threads than
 // the kernel is built for; short rows use fewer vectors so a warp is not mostly idle.
-bool rows_shape(Op op, int nvec, int vpt_req, int g_req, int* vpt, int* G) {
+bool rows_shape(Op op, int nvec, int vpt_req, int g_req, int* vpt, int* G,
+                bool narrow_rows = false) {
     int v = vpt_req;
     if (v == 0) {
         v = 0;
         // layer_norm does more arithmetic per element and gains from longer rows per
         // thread (eight vectors); the rms kernels from more threads (four)
         const int pref = op == OP_LAYER ? 8 : 4;
-        if (nvec <= 32 * pref) {
+        if (narrow_rows && op == OP_RMS && nvec <= 128) {
+            // rms_norm rows of up to 128 vectors: four vectors a thread, rows narrower than
+            // a warp sharing warps (measured, bf16 2^26 elements, CTAs of 128 threads:
+            // D = 64 44.4 us, 128 41.4, 256 42.0, 512 42.1; one vector a thread 57-69 us)
+            v = std::min(4, pow2_ceil(nvec));
+        } else if (nvec <= 32 * pref) {
             v = std::max(1, pow2_ceil((nvec + 31) / 32));
         } else {
             for (int c = pref; c <= max_vpt(op); c *= 2)
@@ -240,8 +246,16 @@ bool rows_shape(Op op, int nvec, int vpt_req, int g_req, int* vpt, int* G) {
     if (v != 1 && v != 2 && v != 4 && v != 8) return false;
     if (v > max_vpt(op)) return false;
     int g = g_req;
-    if (g == 0) g = ((nvec + v - 1) / v + 31) / 32 * 32;
-    if (g % 32 != 0 || g < 32 || g > max_threads(op, v)) return false;
+    // register-path (narrow_rows) rms_norm / add_rms_norm rows of at most 16 x v vectors: a
+    // power of two of threads, several rows to a warp (their one reduction runs over the
+    // row's own lanes); every other row takes whole warps
+    const bool sub = narrow_rows && op != OP_LAYER;
+    if (g == 0) {
+        const int n = (nvec + v - 1) / v;
+        g = (sub && n <= 16) ? pow2_ceil(std::max(n, 1)) : (n + 31) / 32 * 32;
+    }
+    const bool sub_ok = sub && g >= 1 && g <= 16 && (g & (g - 1)) == 0;
+    if ((!sub_ok && (g % 32 != 0 || g < 32)) || g > max_threads(op, v)) return false;
     if ((int64_t)g * v < nvec) return false;
     *vpt = v;
     *G = g;
@@ -383,7 +397,8 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
             p.threads_per_row == 0 && p.rows_per_cta == 0 && slots_shape(nvec, p, di, &sp))
             p.path = NV_PATH_SLOTS;
         else
-            p.path = vec_ok && rows_shape(op, nvec, p.vec_per_thread, p.threads_per_row, &v, &g)
+            p.path = vec_ok && rows_shape(op, nvec, p.vec_per_thread, p.threads_per_row, &v, &g,
+                                          true)
                          ? NV_PATH_ROWS
                          : NV_PATH_GENERIC;
     }
@@ -391,7 +406,7 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
         if (!vec_ok) return fail(NV_ERR_UNSUPPORTED, "register path needs D %% %d == 0 and "
                                  "16-byte aligned pointers", vecw);
         int vpt = 0, G = 0;
-        if (!rows_shape(op, nvec, p.vec_per_thread, p.threads_per_row, &vpt, &G))
+        if (!rows_shape(op, nvec, p.vec_per_thread, p.threads_per_row, &vpt, &G, true))
             return fail(NV_ERR_UNSUPPORTED, "no register-path shape for D = %lld (vpt %d, G %d)",
                         (long long)D, p.vec_per_thread, p.threads_per_row);
         p.vec_per_thread = vpt;
@@ -399,7 +414,9 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
         // CTAs of at least 128 threads; a layer_norm row spanning several warps is alone
         if (p.rows_per_cta == 0)
             p.rows_per_cta = (op == OP_LAYER && G > 32) ? 1 : std::max(1, 128 / G);
-        if (p.rows_per_cta * G > max_threads(op, vpt) || p.rows_per_cta < 1)
+        // whole warps only (a row of fewer than 32 lanes reduces with warp-wide shuffles)
+        if (p.rows_per_cta * G > max_threads(op, vpt) || p.rows_per_cta < 1 ||
+            (G < 32 && (p.rows_per_cta * G) % 32 != 0))
             return fail(NV_ERR_UNSUPPORTED, "rows_per_cta %d x G %d", p.rows_per_cta, G);
         if (op == OP_LAYER && G > 32 && p.rows_per_cta != 1)
             return fail(NV_ERR_UNSUPPORTED, "layer_norm: a row spanning several warps is alone "

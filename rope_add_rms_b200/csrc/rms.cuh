@@ -27,7 +27,8 @@ struct RowArgs {
 };
 
 // ---- register path ------------------------------------------------------------------
-// G threads share one row; thread t holds vectors t, t + G, ..., t + (VPT-1) G of the
+// G threads share one row (a multiple of 32, or for narrow rows a power of two up to 16,
+// several rows to a warp); thread t holds vectors t, t + G, ..., t + (VPT-1) G of the
 // row in registers (coalesced: consecutive threads read consecutive 16-byte vectors).
 // All loads of a row are issued before any arithmetic; the sum of squares is reduced
 // with warp shuffles and, when a row spans several warps, one shared-memory step.
@@ -106,7 +107,7 @@ __global__ void __launch_bounds__(rms_max_threads(VPT)) rms_rows_kernel(const Ro
             }
         }
 
-        ss = warp_sum(ss);
+        ss = group_sum(ss, G < 32 ? G : 32);  // a row of fewer than 32 lanes: its own lanes
         if (wpr > 1) {
             float* buf = red[it & 1];
             if ((threadIdx.x & 31) == 0) buf[threadIdx.x >> 5] = ss;

@@ -195,6 +195,10 @@ def test_plain_rope_ignores_eps():
     ("add_rms_norm", 7, "bf16", dict(path=2)),
     ("add_rms_norm", 2 ** 17, "bf16", dict(path=2)),
     ("rms_norm", 512, "f32", dict(path=1, vec_per_thread=4, threads_per_row=32, rows_per_cta=4)),
+    ("rms_norm", 128, "bf16", dict(path=1, vec_per_thread=4, threads_per_row=4, rows_per_cta=32)),
+    ("rms_norm", 512, "bf16", dict(path=1, vec_per_thread=4, threads_per_row=16, rows_per_cta=8)),
+    ("add_rms_norm", 128, "bf16", dict(path=1, vec_per_thread=1, threads_per_row=16, rows_per_cta=8)),
+    ("add_rms_norm", 512, "bf16", dict(path=1, vec_per_thread=2, threads_per_row=32, rows_per_cta=4)),
     ("layer_norm", 32, "bf16", dict(path=1)),
     ("layer_norm", 64, "bf16", dict(path=5, vec_per_thread=4, threads_per_row=2, rows_per_cta=384,
                                     stages=1)),

@@ -58,6 +58,41 @@ def test_add_rms_norm(rows, D, dt):
     check_out(y, ref)
 
 
+NARROW_PLANS = [None] + [dict(path=nv.PATH_ROWS, vec_per_thread=v, threads_per_row=g,
+                               rows_per_cta=c)
+                          for v, g, c in ((1, 8, 16), (2, 4, 64), (4, 2, 16), (4, 1, 32),
+                                          (1, 16, 8), (2, 16, 2), (4, 4, 8))]
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("D", [8, 16, 32, 64, 128, 256, 512])
+def test_rms_rows_narrower_than_a_warp(D, dt):
+    """rms_norm and add_rms_norm rows of fewer than 32 lanes, several rows to a warp, each
+    reduced over its own lanes: automatic and forced shapes, a ragged row count (the last
+    CTA partly empty), h bit-exact and guard bands around the outputs.  A shape whose CTA is
+    not whole warps, or that does not cover the row, is refused."""
+    rows = 1237
+    inp = synth.add_rms_inputs(rows, D, dt, seed=D + 11)
+    ref, href = oracle.add_rms_norm(host(inp["x"]), host(inp["r"]), host(inp["w"]), 1e-5)
+    rref = oracle.rms_norm(host(inp["x"]), host(inp["w"]), 1e-5)
+    x, w = dev(inp["x"]), dev(inp["w"])
+    for p in NARROW_PLANS:
+        plan = None if p is None else nv.Plan(**p)
+        tag = f"D={D} {dt} {p}"
+        try:
+            y, h = run_add(inp, 1e-5, plan=plan)
+        except nv.NvError as e:
+            assert e.status == nv.NV_ERR_UNSUPPORTED, tag
+            continue
+        check_exact(h, href, "h " + tag)
+        check_out(y, ref, tag)
+        g = Guarded(x.shape, x.dtype)
+        nv.nv_rms_norm(x, w, g.t, 1e-5, plan=plan)
+        torch.cuda.synchronize()
+        assert g.bands_intact(), tag
+        check_out(g.t, rref, "rms " + tag)
+
+
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
 @pytest.mark.parametrize("rows,D", [(17, 7), (3, 127), (2, 129), (9, 1), (5, 33), (4, 1001)])
 def test_add_rms_norm_ragged_D_takes_generic_path(rows, D, dt):
