@@ -1278,7 +1278,37 @@ nv_status run_vjp(Op op, VjpArgs a, int vpt, int cap, const DevInfo& di, cudaStr
                   : (vpt == 1 ? layer_vjp_kernel<T, 1>
                               : vpt == 2 ? layer_vjp_kernel<T, 2> : layer_vjp_kernel<T, 4>);
     nv_status st = NV_OK;
-    if (a.rows > 0) {
+    // narrow rows: row groups of a power-of-two G <= 32 threads, several to a CTA of 256,
+    // each reducing with shuffles alone (vjp_narrow_kernel).  Taken where it measured
+    // faster than the kernels above (bf16, 2^26 elements, the same box):
+    //   rms_norm_vjp   D = 64 206.0 -> 86.2 us, 128 111.5 -> 87.1 (256: 75.3 against 88.3,
+    //                  512: 71.6 against 95.7 -- kept on the kernels above);
+    //   layer_norm_vjp D = 64 366.9 -> 94.5 us, 128 191.1 -> 100.4, 512 100.6 -> 83.8
+    //                  (256: 103.4 against 107.3 -- kept)
+    const bool narrow =
+        vpt != 0 && (a.nvec <= 16 || (op == OP_LAYER && a.nvec > 32 && a.nvec <= 64));
+    if (narrow && a.rows > 0) {
+        const int nvpt = a.nvec <= 32 ? 1 : 2;
+        a.G = pow2_ceil(std::max(1, (a.nvec + nvpt - 1) / nvpt));
+        constexpr int kThreads = 256;
+        constexpr int NP = Elem<T>::kVec / 2;
+        const int R = kThreads / a.G;
+        const size_t smem = (size_t)R * (size_t)a.nvec * NP * sizeof(float2);
+        auto kn = op == OP_RMS ? (nvpt == 1 ? vjp_narrow_kernel<T, 1, false>
+                                            : vjp_narrow_kernel<T, 2, false>)
+                               : (nvpt == 1 ? vjp_narrow_kernel<T, 1, true>
+                                            : vjp_narrow_kernel<T, 2, true>);
+        if (smem > 48 * 1024) {
+            cudaError_t e =
+                cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        }
+        const int64_t wave = (int64_t)di.sms * occupancy(kn, kThreads, smem);
+        const int64_t groups_needed = (a.rows + R - 1) / R;
+        a.parts = (int)std::min<int64_t>(std::min<int64_t>(groups_needed, cap), wave);
+        st = launch_kernel(kn, a.parts, kThreads, smem, s, a);
+        if (st != NV_OK) return st;
+    } else if (a.rows > 0) {
         // VPT = 4 keeps its column partial sums in shared memory (ColAcc)
         constexpr int NP = Elem<T>::kVec / 2;
         const size_t smem = vpt < 4 ? 0

@@ -46,6 +46,7 @@ struct VjpArgs {
     int want_dw;
     int want_db;
     float eps;
+    int G;           // vjp_narrow_kernel: threads of a row group (a power of two <= 32)
 };
 
 // CTA size bound of kernel 1 by vectors per thread: one thread per vector up to 1024
@@ -630,6 +631,220 @@ __global__ void __launch_bounds__(256) vjp_generic_kernel(const VjpArgs a) {
             if constexpr (LAYER)
                 if (pdb) pdb[j] = first ? (float)gj : __fadd_rn(pdb[j], (float)gj);
         }
+    }
+}
+
+// ---- narrow rows: at most 64 vectors a row --------------------------------------------------
+// A row of the kernels above takes at least a warp and pays CTA-wide reductions; a row of
+// 128 bfloat16 features then leaves half of its warp idle.  Here a CTA of 256 threads holds
+// R = 256 / G row groups of G threads (a power of two up to 32, VPT vectors a thread); each
+// group walks its own rows (virtual part p = blockIdx.x R + group, rows p, p + gridDim.x R,
+// ...), reduces with shuffles over its own lanes only (no barrier), and keeps its column
+// partial sums in registers, with the next row's x and g loading into a second register set
+// meanwhile.  At the end the CTA adds its groups' partials in shared memory
+// in group order -- one partial row per CTA, as kernel 2 expects.  The arithmetic of a row
+// is that of RmsVjpRow / LayerVjpRow (the same roundings; the sums differ only in the order
+// of their additions).
+template <typename T, int VPT, bool LAYER>
+__global__ void __launch_bounds__(256) vjp_narrow_kernel(const VjpArgs a) {
+    pdl_wait();
+    pdl_release();
+    using E = Elem<T>;
+    constexpr int VEC = E::kVec;
+    constexpr int NP = VEC / 2;
+    constexpr int NSUM = LAYER ? 2 : 1;
+    constexpr bool kPacked = sizeof(T) == 2;
+    extern __shared__ float2 comb[];  // [R][nvec * NP]: the groups' partials of one sum
+    const int G = a.G;
+    const int R = blockDim.x / G;
+    const int grp = threadIdx.x / G;
+    const int t = threadIdx.x - grp * G;
+    const int64_t step = (int64_t)gridDim.x * R;
+    const float invD = 1.f / (float)a.D;
+
+    V16 wv[VPT];
+    float2 acc[NSUM][VPT * NP];
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+        const int v = t + k * G;
+        wv[k] = (a.w != nullptr && v < a.nvec)
+                    ? ld_param(static_cast<const char*>(a.w) + (size_t)v * 16)
+                    : ones_vec<T>();
+#pragma unroll
+        for (int i = 0; i < NP; ++i)
+#pragma unroll
+            for (int j = 0; j < NSUM; ++j) acc[j][k * NP + i] = splat2(0.f);
+    }
+
+    // the groups of one warp step together while the warp's first group has a row (the
+    // others then have one too, or take part as inactive rows): the shuffles are warp-wide
+    const int gpw = G < 32 ? 32 / G : 1;
+    const int first = grp / gpw * gpw;
+    // the next row's x and g load into a second register set before this row is reduced
+    auto load = [&](int64_t row, V16 (&xo)[VPT], V16 (&go)[VPT]) {
+        const size_t off = (size_t)row * (size_t)a.nvec * 16;
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            const int v = t + k * G;
+            const bool in = row < a.rows && v < a.nvec;
+            xo[k] = in ? ld_stream(static_cast<const char*>(a.x) + off + (size_t)v * 16)
+                       : zeros_vec<T>();
+            go[k] = in ? ld_stream(static_cast<const char*>(a.g) + off + (size_t)v * 16)
+                       : zeros_vec<T>();
+        }
+    };
+    V16 xn[VPT], gn[VPT];
+    load((int64_t)blockIdx.x * R + grp, xn, gn);
+    for (int64_t r0 = (int64_t)blockIdx.x * R + first; r0 < a.rows; r0 += step) {
+        const int64_t row = r0 + (grp - first);
+        const bool live = row < a.rows;
+        const size_t roff = (size_t)row * (size_t)a.nvec * 16;
+        V16 xv[VPT], gv[VPT];
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            xv[k] = xn[k];
+            gv[k] = gn[k];
+        }
+        load(row + step, xn, gn);
+        if constexpr (!LAYER) {
+            float2 s0 = splat2(0.f), s1 = splat2(0.f);
+#pragma unroll
+            for (int k = 0; k < VPT; ++k)
+#pragma unroll
+                for (int e = 0; e < VEC; e += 2) {
+                    const float2 w2 = E::get2(wv[k], e);
+                    if constexpr (kPacked) {
+                        s0 = bf16x2_mac(xv[k].u[e / 2], xv[k].u[e / 2], s0);
+                        s1 = fma2(bf16x2_mac(gv[k].u[e / 2], xv[k].u[e / 2], splat2(0.f)), w2,
+                                  s1);
+                    } else {
+                        const float2 x2 = E::get2(xv[k], e);
+                        const float2 u2 = mul2(E::get2(gv[k], e), w2);
+                        s0 = fma2(x2, x2, s0);
+                        s1 = fma2(u2, x2, s1);
+                    }
+                }
+            const float ss = group_sum(__fadd_rn(s0.x, s0.y), G);
+            const float sp = group_sum(__fadd_rn(s1.x, s1.y), G);
+            const float r = rsqrtf(__fmaf_rn(ss, invD, a.eps));
+            const float vr = __fmul_rn(__fmul_rn(r, r), __fmul_rn(sp, invD));
+            const float2 r2 = splat2(r), nv2 = splat2(-vr);
+#pragma unroll
+            for (int k = 0; k < VPT; ++k) {
+                const int v = t + k * G;
+                if (live && v < a.nvec) {
+                    V16 o;
+#pragma unroll
+                    for (int e = 0; e < VEC; e += 2) {
+                        const float2 x2 = E::get2(xv[k], e);
+                        const float2 g2 = E::get2(gv[k], e);
+                        const float2 u2 = mul2(g2, E::get2(wv[k], e));
+                        E::put2(o, e, mul2(r2, fma2(x2, nv2, u2)));  // r (g w - x v)
+                        acc[0][k * NP + e / 2] = fma2(mul2(g2, x2), r2, acc[0][k * NP + e / 2]);
+                    }
+                    st_stream(static_cast<char*>(a.dx) + roff + (size_t)v * 16, o);
+                }
+            }
+        } else {
+            // pass 1: sum x and sum a (a = w g), a first mean m1
+            float2 p0 = splat2(0.f), p1 = splat2(0.f);
+#pragma unroll
+            for (int k = 0; k < VPT; ++k)
+#pragma unroll
+                for (int e = 0; e < VEC; e += 2) {
+                    if constexpr (kPacked) {
+                        p0 = bf16x2_mac(xv[k].u[e / 2], kBf16x2One, p0);
+                        p1 = bf16x2_mac(wv[k].u[e / 2], gv[k].u[e / 2], p1);
+                    } else {
+                        p0 = add2(p0, E::get2(xv[k], e));
+                        p1 = add2(p1, mul2(E::get2(wv[k], e), E::get2(gv[k], e)));
+                    }
+                }
+            const float m1 = __fmul_rn(group_sum(__fadd_rn(p0.x, p0.y), G), invD);
+            const float sa = group_sum(__fadd_rn(p1.x, p1.y), G);
+            const float ma = __fmul_rn(sa, invD);
+            const float2 nm1 = splat2(-m1);
+            // pass 2: sum c', sum c'^2 and sum a c' around m1 (c' = x - m1)
+            float2 q0 = splat2(0.f), q1 = splat2(0.f), q2 = splat2(0.f);
+#pragma unroll
+            for (int k = 0; k < VPT; ++k) {
+                if (t + k * G < a.nvec)  // c' of a padding lane would be -m1
+#pragma unroll
+                    for (int e = 0; e < VEC; e += 2) {
+                        float2 cp, a2;
+                        if constexpr (kPacked) {
+                            cp = bf16x2_mac(xv[k].u[e / 2], kBf16x2One, nm1);
+                            a2 = bf16x2_mac(wv[k].u[e / 2], gv[k].u[e / 2], splat2(0.f));
+                        } else {
+                            cp = add2(E::get2(xv[k], e), nm1);
+                            a2 = mul2(E::get2(wv[k], e), E::get2(gv[k], e));
+                        }
+                        q0 = add2(q0, cp);
+                        q1 = fma2(cp, cp, q1);
+                        q2 = fma2(a2, cp, q2);
+                    }
+            }
+            const float c0 = group_sum(__fadd_rn(q0.x, q0.y), G);
+            const float c1 = group_sum(__fadd_rn(q1.x, q1.y), G);
+            const float c2 = group_sum(__fadd_rn(q2.x, q2.y), G);
+            const float dm = __fmul_rn(c0, invD);  // mean = m1 + dm
+            const float var = fmaxf(__fmaf_rn(c1, invD, -__fmul_rn(dm, dm)), 0.f);
+            const float r = rsqrtf(__fadd_rn(var, a.eps));
+            const float B = __fmul_rn(__fmul_rn(r, r), __fmul_rn(__fmaf_rn(-dm, sa, c2), invD));
+            const float rB = __fmul_rn(r, B);
+            const float2 r2 = splat2(r), nrB = splat2(-rB),
+                         k0 = splat2(__fmaf_rn(rB, dm, -__fmul_rn(r, ma))),
+                         ndmr = splat2(-__fmul_rn(dm, r));
+#pragma unroll
+            for (int k = 0; k < VPT; ++k) {
+                const int v = t + k * G;
+                if (live && v < a.nvec) {
+                    V16 o;
+#pragma unroll
+                    for (int e = 0; e < VEC; e += 2) {
+                        const float2 g2 = E::get2(gv[k], e);
+                        float2 a2, cp;
+                        if constexpr (kPacked) {
+                            a2 = bf16x2_mac(wv[k].u[e / 2], gv[k].u[e / 2], splat2(0.f));
+                            cp = bf16x2_mac(xv[k].u[e / 2], kBf16x2One, nm1);
+                        } else {
+                            a2 = mul2(E::get2(wv[k], e), g2);
+                            cp = add2(E::get2(xv[k], e), nm1);
+                        }
+                        E::put2(o, e, fma2(r2, a2, fma2(cp, nrB, k0)));
+                        float2& aw = acc[0][k * NP + e / 2];
+                        float2& ab = acc[NSUM - 1][k * NP + e / 2];
+                        aw = fma2(g2, fma2(cp, r2, ndmr), aw);
+                        ab = add2(ab, g2);
+                    }
+                    st_stream(static_cast<char*>(a.dx) + roff + (size_t)v * 16, o);
+                }
+            }
+        }
+    }
+
+    if (a.part == nullptr) return;
+    // the groups' partials, added per column in group order
+    const int ncol = a.nvec * NP;  // float pairs of a row
+#pragma unroll
+    for (int j = 0; j < NSUM; ++j) {
+        const bool want = j == 0 ? a.want_dw : a.want_db;
+        if (!want) continue;  // uniform over the CTA
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            const int v = t + k * G;
+            if (v < a.nvec)
+#pragma unroll
+                for (int i = 0; i < NP; ++i) comb[(size_t)grp * ncol + v * NP + i] = acc[j][k * NP + i];
+        }
+        __syncthreads();
+        float2* out = reinterpret_cast<float2*>(a.part + ((size_t)j * a.parts + blockIdx.x) * a.D);
+        for (int c = threadIdx.x; c < ncol; c += blockDim.x) {
+            float2 sum = comb[c];
+            for (int q = 1; q < R; ++q) sum = add2(sum, comb[(size_t)q * ncol + c]);
+            out[c] = sum;
+        }
+        __syncthreads();
     }
 }
 

@@ -1199,6 +1199,41 @@ def test_rms_norm_vjp(rows, D, weight, dt):
 
 
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,D", [(1, 8), (7, 16), (1237, 64), (2049, 128), (333, 256), (517, 512),
+                                    (64, 24), (4099, 128), (3, 200)])
+def test_vjp_rows_of_at_most_64_vectors(rows, D, dt):
+    """Rows of at most 64 vectors: row groups of G threads, several to a CTA, each walking its
+    own rows and reducing over its own lanes, their column partial sums added in shared
+    memory in group order.  Ragged row counts (groups of one warp running out of rows at
+    different times), with and without w, both gradients, against the oracle; dw and db
+    the same on a second call (the order of their sums is fixed)."""
+    for weight in (True, False):
+        inp = synth.layer_norm_inputs(rows, D, dt, seed=rows + 7 * D, weight=weight, bias=False)
+        g = synth.normal((rows, D), 0.0, 1.0, rows + 7 * D, 4, dt)
+        x, w, gd = dev(inp["x"]), dev(inp["w"]), dev(g)
+        dx, dw = nv.rms_norm_vjp(x, w, gd, eps=1e-5)
+        torch.cuda.synchronize()
+        ref_dx, ref_dw, mag_dx, mag_dw = oracle.rms_norm_vjp(host(inp["x"]), host(inp["w"]),
+                                                             host(g), 1e-5)
+        check_grad(dx, ref_dx, mag_dx, f"rms dx D={D} w={weight}")
+        if weight:
+            check_grad(dw, ref_dw, mag_dw, f"rms dw D={D}")
+            _, dw2 = nv.rms_norm_vjp(x, w, gd, eps=1e-5)
+            torch.cuda.synchronize()
+            assert torch.equal(dw, dw2), "rms dw not reproducible"
+        ldx, ldw, ldb = nv.layer_norm_vjp(x, w, gd, eps=1e-5)
+        torch.cuda.synchronize()
+        ref = oracle.layer_norm_vjp(host(inp["x"]), host(inp["w"]), host(g), 1e-5)
+        check_grad(ldx, ref[0], ref[3], f"layer dx D={D} w={weight}")
+        if weight:
+            check_grad(ldw, ref[1], ref[4], f"layer dw D={D}")
+        check_grad(ldb, ref[2], ref[5], f"layer db D={D}")
+        _, _, ldb2 = nv.layer_norm_vjp(x, w, gd, eps=1e-5)
+        torch.cuda.synchronize()
+        assert torch.equal(ldb, ldb2), "layer db not reproducible"
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
 @pytest.mark.parametrize("weight", [True, False])
 @pytest.mark.parametrize("rows,D", VJP_SHAPES)
 def test_layer_norm_vjp(rows, D, weight, dt):
