@@ -576,6 +576,11 @@ nv_status run_layer(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs
             const bool big = a.G * a.rows_per_cta > 768;
             auto pick = [&](auto vpt) {
                 constexpr int V = decltype(vpt)::value;
+                if (a.G < 32)  // several rows to a warp: the narrow form
+                    return big ? (pf ? layer_slots_kernel<V, true, 1024, true>
+                                     : layer_slots_kernel<V, false, 1024, true>)
+                               : (pf ? layer_slots_kernel<V, true, 768, true>
+                                     : layer_slots_kernel<V, false, 768, true>);
                 return big ? (pf ? layer_slots_kernel<V, true, 1024> : layer_slots_kernel<V, false, 1024>)
                            : (pf ? layer_slots_kernel<V, true, 768> : layer_slots_kernel<V, false, 768>);
             };
