@@ -1284,16 +1284,16 @@ nv_status run_vjp(Op op, VjpArgs a, int vpt, int cap, const DevInfo& di, cudaStr
                               : vpt == 2 ? layer_vjp_kernel<T, 2> : layer_vjp_kernel<T, 4>);
     nv_status st = NV_OK;
     // narrow rows: row groups of a power-of-two G <= 32 threads, several to a CTA of 256,
-    // each reducing with shuffles alone (vjp_narrow_kernel).  Taken where it measured
-    // faster than the kernels above (bf16, 2^26 elements, the same box):
-    //   rms_norm_vjp   D = 64 206.0 -> 86.2 us, 128 111.5 -> 87.1 (256: 75.3 against 88.3,
-    //                  512: 71.6 against 95.7 -- kept on the kernels above);
-    //   layer_norm_vjp D = 64 366.9 -> 94.5 us, 128 191.1 -> 100.4, 512 100.6 -> 83.8
-    //                  (256: 103.4 against 107.3 -- kept)
-    const bool narrow =
-        vpt != 0 && (a.nvec <= 16 || (op == OP_LAYER && a.nvec > 32 && a.nvec <= 64));
+    // each reducing with shuffles alone (vjp_narrow_kernel), one vector a thread up to 16
+    // vectors a row, two above.  Taken where it measured faster than the kernels above
+    // (bf16, 2^26 elements, the same box):
+    //   rms_norm_vjp   D = 64 206.0 -> 86.2 us, 128 111.5 -> 87.1 (256 and 512 stay: 75.9
+    //                  and 71.7 against 93.5 and 104.5 at two and four vectors a thread);
+    //   layer_norm_vjp D = 64 366.9 -> 94.5 us, 128 191.1 -> 100.4, 256 103.5 -> 79.5,
+    //                  512 100.6 -> 83.8
+    const bool narrow = vpt != 0 && (a.nvec <= 16 || (op == OP_LAYER && a.nvec <= 64));
     if (narrow && a.rows > 0) {
-        const int nvpt = a.nvec <= 32 ? 1 : 2;
+        const int nvpt = a.nvec <= 16 ? 1 : 2;
         a.G = pow2_ceil(std::max(1, (a.nvec + nvpt - 1) / nvpt));
         constexpr int kThreads = 256;
         constexpr int NP = Elem<T>::kVec / 2;
