@@ -653,6 +653,12 @@ WORKLOADS = {
     "norm_rope_yarn": lambda: Case("norm_rope", (8, 32, 2048, 128), "bf16", 0, eps=1e-6,
                                    dims=128, traditional=0, base=10000.0, scale=1.0,
                                    offset=16384, yarn=True),
+    # narrow rows: a per-head RMSNorm (128 features), a 256-feature LayerNorm and its
+    # gradient (rows narrower than a warp, several to a warp)
+    "rms_norm_per_head": lambda: Case("rms_norm", (524288, 128), "bf16", 0, eps=1e-6),
+    "layer_norm_narrow": lambda: Case("layer_norm", (262144, 256), "bf16", 0, eps=1e-5),
+    "layer_norm_vjp_narrow": lambda: Case("layer_norm_vjp", (262144, 256), "bf16", 0,
+                                          eps=1e-5),
     "rms_norm_vjp": lambda: Case("rms_norm_vjp", (8192, 4096), "bf16", 0, eps=1e-5),
     "layer_norm_vjp": lambda: Case("layer_norm_vjp", (16384, 8192), "bf16", 0, eps=1e-5),
     # a TP8 decoder's all-reduce + residual add + RMSNorm, the 8 partial outputs already
