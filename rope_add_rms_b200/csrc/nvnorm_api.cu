@@ -270,8 +270,8 @@ size_t staged_smem(Op op, int64_t D, nv_dtype dt, int stages) {
 constexpr int kStaticSmemReserve = 2048;  // static shared memory + per-CTA system use
 
 // Slots path shape (bfloat16 layer_norm): VPT vectors a thread (8, or 4 for narrow rows),
-// G threads a row (a multiple of 32, or 8 or 16), as many row slots as make 768 threads
-// (24 warps per SM, one CTA per SM),
+// G threads a row (a multiple of 32, or a power of two up to 16), as many row slots as make
+// 768 threads (24 warps per SM, one CTA per SM),
 // at most 15 when a row spans several warps (one named barrier each); the float32 w/b table
 // (64 bytes a vector) must fit the shared memory.
 bool slots_shape(int nvec, const nv_plan& req, const DevInfo* di, nv_plan* out) {
@@ -389,10 +389,10 @@ nv_status make_plan(Op op, int64_t rows, int64_t D, nv_dtype dt, bool aligned, c
         nv_plan sp{};
         // bfloat16 layer_norm: the slots kernel for rows of 8 vectors or more, whenever its
         // w/b table fits.  Measured against the register kernel on B200 (2^26 elements):
-        // D = 64 143.6 against 368.1 us and D = 128 80.8 against 188.6 (with 8 threads a
-        // row), D = 256 53.6 against 101.3, D = 512 54.2 against 71.8, D = 768 56.3
-        // against 77.6, D = 1024 48.1 against 64.6, D = 1536 54.1 against 67.0,
-        // D = 2048..16384 10-20 % faster
+        // D = 64 58.4 against 368.1 us (2 threads a row), D = 128 55.5 against 188.6 (4),
+        // D = 256 53.6 against 101.3, D = 512 54.2 against 71.8, D = 768 56.3 against
+        // 77.6, D = 1024 48.1 against 64.6, D = 1536 54.1 against 67.0, D = 2048..16384
+        // 10-20 % faster
         if (op == OP_LAYER && dt == NV_BF16 && vec_ok && nvec >= 8 && p.vec_per_thread == 0 &&
             p.threads_per_row == 0 && p.rows_per_cta == 0 && slots_shape(nvec, p, di, &sp))
             p.path = NV_PATH_SLOTS;
