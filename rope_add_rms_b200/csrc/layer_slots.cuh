@@ -85,8 +85,8 @@ constexpr int kSlotsMaxThreads = 1024;
 // when G > 32; G a multiple of 32 or a power of two up to 16),
 // dynamic shared memory = slots_table_bytes(a.nvec); persistent grid.
 // NARROW: G < 32, several rows to a warp (slot-width sums, a warp-wide vote for the
-// centred pass); the wide form keeps plain warp sums (the narrow form's code measured 3 %
-// slower on bf16 [16384, 8192]).
+// centred pass).  The wide form keeps plain warp sums: compiled into one kernel, the narrow
+// code cost the wide rows 3 % on bf16 [16384, 8192].
 template <int VPT, bool PREFETCH, int MAXT, bool NARROW = false>
 __global__ void __launch_bounds__(MAXT, 1) layer_slots_kernel(const RowArgs a) {
     pdl_wait();
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(MAXT, 1) layer_slots_kernel(const RowArgs a) {
             s1 = warp_sum((s1 + s1b) + (t1 + t1b));
             s2 = warp_sum((s2 + s2b) + (t2 + t2b));
         }
-        // the row is in registers: ask L2 for the slot's next row (see the header)
+        // the row's loads have landed: ask L2 for the slot's next row (see the header)
         if constexpr (PREFETCH) {
             if (t == 0 && row + row_step < a.rows)
                 prefetch_l2(static_cast<const char*>(a.x) + (size_t)(row + row_step) * row_bytes,
