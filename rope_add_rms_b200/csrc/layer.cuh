@@ -100,7 +100,9 @@ __device__ __forceinline__ V16 layer_vector_f64(V16 xv, V16 wv, V16 bv, double m
 // MAXT bounds the CTA: 128 (256) lets the compiler keep the 8-vector form under 85
 // registers, six (three) CTAs = 24 warps per SM -- measured 13 % faster on bf16
 // [16384, 8192] than four CTAs at 128 registers; wider rows use 512 threads.
-template <typename T, int VPT, int MAXT = layer_max_threads(VPT)>
+// NARROW: G < 32, several rows to a warp -- slot-width sums and a warp-wide vote for the
+// centred pass, in their own instantiation so the wide rows keep plain warp sums.
+template <typename T, int VPT, int MAXT = layer_max_threads(VPT), bool NARROW = false>
 __global__ void __launch_bounds__(MAXT, MAXT <= 256 ? 768 / MAXT : 1)
     layer_rows_kernel(const RowArgs a) {
     pdl_wait();
@@ -166,8 +168,13 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 256 ? 768 / MAXT : 1)
             }
         s1 += s1b;
         s2 += s2b;
-        s1 = warp_sum(s1);
-        s2 = warp_sum(s2);
+        if constexpr (NARROW) {
+            s1 = group_sum(s1, G);
+            s2 = group_sum(s2, G);
+        } else {
+            s1 = warp_sum(s1);
+            s2 = warp_sum(s2);
+        }
         // bfloat16: the row's loads have landed, so ask L2 for this slot's next row (one bulk
         // prefetch of the whole row from this GPU's own memory, nothing to wait on).
         // Measured: [65536, 1024] 70.3 -> 65.0 us, [131072, 512] 82.4 -> 72.1 us; float32
@@ -195,8 +202,13 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 256 ? 768 / MAXT : 1)
         }
         const double mean = s1 * invD;
         double var = s2 * invD - mean * mean;
-        if (!(var > ldexp(mean * mean, -20))) {
-            // centred second pass (uniform over the row's threads)
+        // centred second pass: uniform over a row's threads, and with several rows to a warp
+        // taken by the whole warp when any of its rows needs it (its shuffles are warp-wide),
+        // each row keeping its own result only if it asked for it
+        const bool centre = !(var > ldexp(mean * mean, -20));
+        bool centre_warp = centre;
+        if constexpr (NARROW) centre_warp = __any_sync(0xFFFFFFFFu, centre);
+        if (centre_warp) {
             double c2 = 0.0;
 #pragma unroll
             for (int k = 0; k < VPT; ++k)
@@ -206,7 +218,10 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 256 ? 768 / MAXT : 1)
                         const double dd = (double)E::get(xv[k], e) - mean;
                         c2 = fma(dd, dd, c2);
                     }
-            c2 = warp_sum(c2);
+            if constexpr (NARROW)
+                c2 = group_sum(c2, G);
+            else
+                c2 = warp_sum(c2);
             if (wpr > 1) {
                 __syncthreads();  // every thread has read red[it & 1] above
                 double* b1 = red[it & 1][0];
@@ -215,7 +230,7 @@ __global__ void __launch_bounds__(MAXT, MAXT <= 256 ? 768 / MAXT : 1)
                 c2 = 0.0;
                 for (int i = 0; i < wpr; ++i) c2 += b1[i];
             }
-            var = c2 * invD;
+            if (centre) var = c2 * invD;
         }
         const double rstd = rsqrt(var + eps);
         const float mu_hi = __double2float_rn(mean);

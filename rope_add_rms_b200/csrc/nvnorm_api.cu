@@ -230,11 +230,15 @@ bool rows_shape(Op op, int nvec, int vpt_req, int g_req, int* vpt, int* G,
         // layer_norm does more arithmetic per element and gains from longer rows per
         // thread (eight vectors); the rms kernels from more threads (four)
         const int pref = op == OP_LAYER ? 8 : 4;
-        if (narrow_rows && op == OP_RMS && nvec <= 128) {
-            // rms_norm rows of up to 128 vectors: four vectors a thread, rows narrower than
-            // a warp sharing warps (measured, bf16 2^26 elements, CTAs of 128 threads:
-            // D = 64 44.4 us, 128 41.4, 256 42.0, 512 42.1; one vector a thread 57-69 us)
-            v = std::min(4, pow2_ceil(nvec));
+        if (narrow_rows && (op == OP_RMS || op == OP_LAYER) && nvec <= 128) {
+            // rms_norm and layer_norm rows of up to 128 vectors: four (rms_norm) or eight
+            // (layer_norm, more arithmetic a row) vectors a thread, rows narrower than a
+            // warp sharing warps.  Measured at 2^25-2^26 elements, CTAs of 128 threads:
+            //   rms_norm bf16 D = 64 44.4 us, 128 41.4, 256 42.0, 512 42.1 (one vector a
+            //   thread 57-69 us);
+            //   layer_norm f32 D = 128 48.6 us, 256 48.6, 512 47.7 (four vectors 58.3,
+            //   58.7, 56.6; one or two vectors at 32 threads a row 73.0, 70.3)
+            v = std::min(op == OP_LAYER ? 8 : 4, pow2_ceil(nvec));
         } else if (nvec <= 32 * pref) {
             v = std::max(1, pow2_ceil((nvec + 31) / 32));
         } else {
@@ -246,10 +250,10 @@ bool rows_shape(Op op, int nvec, int vpt_req, int g_req, int* vpt, int* G,
     if (v != 1 && v != 2 && v != 4 && v != 8) return false;
     if (v > max_vpt(op)) return false;
     int g = g_req;
-    // register-path (narrow_rows) rms_norm / add_rms_norm rows of at most 16 x v vectors: a
-    // power of two of threads, several rows to a warp (their one reduction runs over the
-    // row's own lanes); every other row takes whole warps
-    const bool sub = narrow_rows && op != OP_LAYER;
+    // register-path (narrow_rows) rows of at most 16 x v vectors: a power of two of threads,
+    // several rows to a warp (their reductions run over the row's own lanes); every other
+    // row takes whole warps
+    const bool sub = narrow_rows;
     if (g == 0) {
         const int n = (nvec + v - 1) / v;
         g = (sub && n <= 16) ? pow2_ceil(std::max(n, 1)) : (n + 31) / 32 * 32;
@@ -630,11 +634,19 @@ nv_status run_layer(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs
         const int per_sm = p.ctas_per_sm > 0 ? p.ctas_per_sm : occupancy(kern, block, 0);
         return launch(kern, units, block, 0, std::max(per_sm, 1), di, s, a);
     };
+    const bool nar = a.G < 32;  // several rows to a warp: the narrow form
     switch (p.vec_per_thread) {
-        case 1: return go(layer_rows_kernel<T, 1>);
-        case 2: return go(layer_rows_kernel<T, 2>);
-        case 4: return go(layer_rows_kernel<T, 4>);
+        case 1: return nar ? go(layer_rows_kernel<T, 1, layer_max_threads(1), true>)
+                           : go(layer_rows_kernel<T, 1>);
+        case 2: return nar ? go(layer_rows_kernel<T, 2, layer_max_threads(2), true>)
+                           : go(layer_rows_kernel<T, 2>);
+        case 4: return nar ? go(layer_rows_kernel<T, 4, layer_max_threads(4), true>)
+                           : go(layer_rows_kernel<T, 4>);
         case 8:
+            if (nar)
+                return block <= 128 ? go(layer_rows_kernel<T, 8, 128, true>)
+                       : block <= 256 ? go(layer_rows_kernel<T, 8, 256, true>)
+                                      : go(layer_rows_kernel<T, 8, layer_max_threads(8), true>);
             return block <= 128   ? go(layer_rows_kernel<T, 8, 128>)
                    : block <= 256 ? go(layer_rows_kernel<T, 8, 256>)
                                   : go(layer_rows_kernel<T, 8>);

@@ -221,6 +221,8 @@ def test_plain_rope_ignores_eps():
     ("layer_norm", 8192, "bf16", dict(path=5, vec_per_thread=8, threads_per_row=128, rows_per_cta=6,
                                       stages=1)),
     ("layer_norm", 8192, "f32", dict(path=1, vec_per_thread=8, threads_per_row=256)),
+    ("layer_norm", 128, "f32", dict(path=1, vec_per_thread=8, threads_per_row=4, rows_per_cta=32)),
+    ("layer_norm", 512, "f32", dict(path=1, vec_per_thread=8, threads_per_row=16, rows_per_cta=8)),
     ("layer_norm", 32768, "bf16", dict(path=1)),
     ("norm_rope", 128, "bf16", dict(path=1, vec_per_thread=2, threads_per_row=8)),
     ("norm_rope", 1000, "bf16", dict(path=2)),

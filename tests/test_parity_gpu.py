@@ -94,6 +94,34 @@ def test_rms_rows_narrower_than_a_warp(D, dt):
 
 
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("D", [8, 16, 32, 64, 128, 256])
+def test_layer_rows_narrower_than_a_warp(D, dt):
+    """layer_norm rows of fewer than 32 lanes in the register kernel, several rows to a warp:
+    automatic and forced shapes, a ragged row count, rows whose mean dwarfs their spread
+    (the centred second pass, voted warp-wide and kept only by the rows that asked for it)
+    next to ordinary rows in the same warps, and guard bands."""
+    rows = 1237
+    x = synth.normal((rows, D), 0.5, 2.0, D, 0, dt)
+    far = synth.normal((rows, D), 3000.0, 0.25, D, 1, dt)
+    x[1::3] = far[1::3]   # every third row takes the centred pass
+    w = synth.uniform((D,), 0.5, 1.5, D, 2, dt)
+    b = synth.normal((D,), 0.0, 0.1, D, 3, dt)
+    ref = oracle.layer_norm(host(x), host(w), host(b), 1e-5)
+    xd, wd, bd = dev(x), dev(w), dev(b)
+    for p in NARROW_PLANS:
+        tag = f"D={D} {dt} {p}"
+        g = Guarded(xd.shape, xd.dtype)
+        try:
+            nv.nv_layer_norm(xd, wd, bd, g.t, 1e-5, plan=None if p is None else nv.Plan(**p))
+        except nv.NvError as e:
+            assert e.status == nv.NV_ERR_UNSUPPORTED, tag
+            continue
+        torch.cuda.synchronize()
+        assert g.bands_intact(), tag
+        check_out(g.t, ref, tag)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
 @pytest.mark.parametrize("rows,D", [(17, 7), (3, 127), (2, 129), (9, 1), (5, 33), (4, 1001)])
 def test_add_rms_norm_ragged_D_takes_generic_path(rows, D, dt):
     inp = synth.add_rms_inputs(rows, D, dt, seed=D)
