@@ -291,15 +291,18 @@ bool slots_shape(int nvec, const nv_plan& req, const DevInfo* di, nv_plan* out) 
     const auto lanes = [&](int vv) { return threads(vv) * vv; };
     // vectors a thread, measured on B200 (bf16, 2^26-2^27 elements, the prefetch after the
     // warp sums): 8 in CTAs of 768 threads from 256 vectors a row on (D = 4096: 51.9 us
-    // against 52.7 with 4 in CTAs of 1024 threads); below, 4 where they cover the row with
-    // no idle lane (D = 256, 512, 1024: 53.6, 54.2, 52.4 us; with 8, -, 57.8, 54.6), else
-    // whichever leaves fewer lanes idle, 8 on a tie (D = 768: 57.1 against 62.4 with 4;
-    // D = 1536: 54.1 against 61.4)
+    // against 52.7 with 4 in CTAs of 1024 threads); below, the first of 4, 8, 6 and 3 that
+    // covers the row with no idle lane (D = 256, 512, 1024 take 4: 53.6, 54.2, 48.3 us;
+    // D = 384, 768, 1536 take 6: 50.2, 50.1, 47.9 us, against 57.3, 57.1, 54.2 with 8 and
+    // 55.8, 52.3, 57.1 with 3), else whichever of 4 and 8 leaves fewer lanes idle, 8 on a tie
     int v = p.vec_per_thread ? p.vec_per_thread
                              : nvec >= 256 ? 8
                              : lanes(4) == nvec ? 4
-                             : lanes(8) == nvec || lanes(8) <= lanes(4) ? 8 : 4;
-    if (v != 4 && v != 8) return false;
+                             : lanes(8) == nvec ? 8
+                             : lanes(6) == nvec ? 6
+                             : lanes(3) == nvec ? 3
+                             : lanes(8) <= lanes(4) ? 8 : 4;
+    if (v != 3 && v != 4 && v != 6 && v != 8) return false;
     int g = p.threads_per_row ? p.threads_per_row : threads(v);
     if (g < 1 || (g % 32 && (g > 16 || (g & (g - 1)))) || (int64_t)g * v < nvec ||
         g > kSlotsMaxThreads)
@@ -588,8 +591,10 @@ nv_status run_layer(const nv_plan& p, const DevInfo& di, cudaStream_t s, RowArgs
                 return big ? (pf ? layer_slots_kernel<V, true, 1024> : layer_slots_kernel<V, false, 1024>)
                            : (pf ? layer_slots_kernel<V, true, 768> : layer_slots_kernel<V, false, 768>);
             };
-            auto kern = p.vec_per_thread == 8 ? pick(std::integral_constant<int, 8>{})
-                                              : pick(std::integral_constant<int, 4>{});
+            auto kern = p.vec_per_thread == 8   ? pick(std::integral_constant<int, 8>{})
+                        : p.vec_per_thread == 6 ? pick(std::integral_constant<int, 6>{})
+                        : p.vec_per_thread == 3 ? pick(std::integral_constant<int, 3>{})
+                                                : pick(std::integral_constant<int, 4>{});
             cudaError_t e =
                 cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");

@@ -208,11 +208,11 @@ def test_plain_rope_ignores_eps():
                                      stages=1)),
     ("layer_norm", 512, "bf16", dict(path=5, vec_per_thread=4, threads_per_row=16, rows_per_cta=48,
                                      stages=1)),
-    ("layer_norm", 768, "bf16", dict(path=5, vec_per_thread=8, threads_per_row=16, rows_per_cta=48,
+    ("layer_norm", 768, "bf16", dict(path=5, vec_per_thread=6, threads_per_row=16, rows_per_cta=48,
                                      stages=1)),
     ("layer_norm", 1024, "bf16", dict(path=5, vec_per_thread=4, threads_per_row=32, rows_per_cta=24,
                                       stages=1)),
-    ("layer_norm", 1536, "bf16", dict(path=5, vec_per_thread=8, threads_per_row=32, rows_per_cta=24,
+    ("layer_norm", 1536, "bf16", dict(path=5, vec_per_thread=6, threads_per_row=32, rows_per_cta=24,
                                       stages=1)),
     ("layer_norm", 2048, "bf16", dict(path=5, vec_per_thread=8, threads_per_row=32, rows_per_cta=24,
                                       stages=1)),

@@ -411,6 +411,7 @@ def test_layer_norm_in_place_and_large_mean():
 
 
 SLOTS = [dict(path=nv.PATH_SLOTS), dict(path=nv.PATH_SLOTS, vec_per_thread=4),
+         dict(path=nv.PATH_SLOTS, vec_per_thread=3), dict(path=nv.PATH_SLOTS, vec_per_thread=6),
          dict(path=nv.PATH_SLOTS, rows_per_cta=1), dict(path=nv.PATH_SLOTS, rows_per_cta=5),
          dict(path=nv.PATH_SLOTS, vec_per_thread=8, threads_per_row=64),
          dict(path=nv.PATH_SLOTS, stages=-1)]
@@ -422,6 +423,7 @@ SLOTS = [dict(path=nv.PATH_SLOTS), dict(path=nv.PATH_SLOTS, vec_per_thread=4),
                                         (1000, 2048, (1, 1)), (1, 8192, (1, 1)), (2, 8, (1, 1)),
                                         (77, 24576, (1, 1)), (500, 1024, (1, 1)),
                                         (129, 1536, (0, 1)), (311, 768, (1, 1)), (1001, 128, (1, 1)),
+                                        (513, 384, (1, 1)), (65, 3072, (1, 1)),
                                         (999, 64, (1, 0)), (77, 32, (1, 1))])
 def test_layer_norm_slots(rows, D, wb, plan):
     """The slots path (bfloat16): rows in registers, several per CTA sharing a float32 table
